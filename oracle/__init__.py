@@ -1,0 +1,193 @@
+"""CPU oracle for host-streamed paged quantized KV attention.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The product library
+(``host_streamed_paged_kvs_b200``) never imports it and shares no code with it.
+
+The arithmetic lives in ``kvs_oracle.c`` (plain C, single thread; quantization
+decisions in binary32, attention in binary64).  This module only builds that
+file with gcc and marshals numpy arrays through ctypes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kvs_oracle.c")
+_HDR = os.path.join(_HERE, "kvs_oracle.h")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+PAGE_ABSENT = -1
+PAGE_RESIDENT = 1
+PAGE_STREAMED = 2
+
+
+def build(force: bool = False) -> str:
+    """Compile kvs_oracle.c into liboracle.so (IEEE arithmetic, no contraction)."""
+    stale = (not os.path.exists(_LIB)) or any(
+        os.path.getmtime(p) > os.path.getmtime(_LIB) for p in (_SRC, _HDR))
+    if force or stale:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-ffp-contract=off",
+               "-fno-fast-math", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        u16p = ctypes.POINTER(ctypes.c_uint16)
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        f64p = ctypes.POINTER(ctypes.c_double)
+        L.oracle_half_to_double.restype = ctypes.c_double
+        L.oracle_half_to_double.argtypes = [ctypes.c_uint16]
+        L.oracle_float_to_half.restype = ctypes.c_uint16
+        L.oracle_float_to_half.argtypes = [ctypes.c_float]
+        L.oracle_q8_0_block.argtypes = [u16p, u8p]
+        L.oracle_q4_0_block.argtypes = [u16p, u8p]
+        L.oracle_dequant_q8_0.argtypes = [u8p, f64p]
+        L.oracle_dequant_q4_0.argtypes = [u8p, f64p]
+        L.oracle_quantize_rows.argtypes = [ctypes.c_int, ctypes.c_int, u16p, u16p, u8p, u8p]
+        L.oracle_attention.restype = ctypes.c_int
+        L.oracle_attention.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, u8p, u8p,
+                                       ctypes.c_int, ctypes.c_int, u16p, f64p, f64p]
+        L.oracle_pages_for.restype = ctypes.c_long
+        L.oracle_pages_for.argtypes = [ctypes.c_long, ctypes.c_int]
+        L.oracle_auto_resident_pages.restype = ctypes.c_long
+        L.oracle_auto_resident_pages.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_long,
+                                                 ctypes.c_int]
+        L.oracle_page_location.restype = ctypes.c_int
+        L.oracle_page_location.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_long,
+                                           ctypes.c_long, ctypes.POINTER(ctypes.c_int),
+                                           ctypes.POINTER(ctypes.c_long)]
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray, ctype):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _as_half_bits(x) -> np.ndarray:
+    a = np.asarray(x)
+    if a.dtype == np.float16:
+        a = a.view(np.uint16)
+    assert a.dtype == np.uint16
+    return np.ascontiguousarray(a)
+
+
+# --- binary16 conversions -------------------------------------------------
+
+def half_to_double(h) -> np.ndarray:
+    h = _as_half_bits(h)
+    L = lib()
+    return np.array([L.oracle_half_to_double(int(v)) for v in h.ravel()],
+                    dtype=np.float64).reshape(h.shape)
+
+
+def float_to_half(f) -> np.ndarray:
+    f = np.asarray(f, dtype=np.float32)
+    L = lib()
+    return np.array([L.oracle_float_to_half(float(v)) for v in f.ravel()],
+                    dtype=np.uint16).reshape(f.shape)
+
+
+# --- block quantization ---------------------------------------------------
+
+def q8_0_block(x) -> bytes:
+    x = _as_half_bits(x).reshape(32)
+    out = np.zeros(34, np.uint8)
+    lib().oracle_q8_0_block(_ptr(x, ctypes.c_uint16), _ptr(out, ctypes.c_uint8))
+    return out.tobytes()
+
+
+def q4_0_block(x) -> bytes:
+    x = _as_half_bits(x).reshape(32)
+    out = np.zeros(18, np.uint8)
+    lib().oracle_q4_0_block(_ptr(x, ctypes.c_uint16), _ptr(out, ctypes.c_uint8))
+    return out.tobytes()
+
+
+def dequant_q8_0(blk) -> np.ndarray:
+    b = np.frombuffer(bytes(blk), np.uint8).copy()
+    out = np.zeros(32, np.float64)
+    lib().oracle_dequant_q8_0(_ptr(b, ctypes.c_uint8), _ptr(out, ctypes.c_double))
+    return out
+
+
+def dequant_q4_0(blk) -> np.ndarray:
+    b = np.frombuffer(bytes(blk), np.uint8).copy()
+    out = np.zeros(32, np.float64)
+    lib().oracle_dequant_q4_0(_ptr(b, ctypes.c_uint8), _ptr(out, ctypes.c_double))
+    return out
+
+
+def quantize_rows(k, v):
+    """k, v: fp16 [..., dim] -> (Q8_0 blocks [..., dim/32, 34], Q4_0 blocks [..., dim/32, 18])."""
+    k = _as_half_bits(k)
+    v = _as_half_bits(v)
+    assert k.shape == v.shape
+    dim = k.shape[-1]
+    rows = int(np.prod(k.shape[:-1]))
+    kb = np.zeros(k.shape[:-1] + (dim // 32, 34), np.uint8)
+    vb = np.zeros(k.shape[:-1] + (dim // 32, 18), np.uint8)
+    lib().oracle_quantize_rows(rows, dim, _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16),
+                               _ptr(kb, ctypes.c_uint8), _ptr(vb, ctypes.c_uint8))
+    return kb, vb
+
+
+# --- attention ------------------------------------------------------------
+
+def attention(k_blocks: np.ndarray, v_blocks: np.ndarray, q, pos0: int):
+    """Exact attention over a quantized history.
+
+    k_blocks: uint8 [n_keys, n_kv, dim/32, 34]; v_blocks: uint8 [n_keys, n_kv, dim/32, 18]
+    q: fp16 [n_q, n_qh, dim]; query j sits at position pos0+j and sees keys 0..pos0+j.
+    Returns (out float64 [n_q, n_qh, dim], lse float64 [n_q, n_qh]).
+    """
+    q = _as_half_bits(q)
+    n_q, n_qh, dim = q.shape
+    n_kv = k_blocks.shape[1]
+    assert k_blocks.shape[0] >= pos0 + n_q
+    kb = np.ascontiguousarray(k_blocks, dtype=np.uint8)
+    vb = np.ascontiguousarray(v_blocks, dtype=np.uint8)
+    out = np.zeros((n_q, n_qh, dim), np.float64)
+    lse = np.zeros((n_q, n_qh), np.float64)
+    rc = lib().oracle_attention(n_kv, n_qh, dim, _ptr(kb, ctypes.c_uint8),
+                                _ptr(vb, ctypes.c_uint8), n_q, pos0,
+                                _ptr(q, ctypes.c_uint16), _ptr(out, ctypes.c_double),
+                                _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise ValueError(f"oracle_attention rejected its arguments (rc={rc})")
+    return out, lse
+
+
+# --- page policy ----------------------------------------------------------
+
+def pages_for(n_tokens: int, page_tokens: int = 256) -> int:
+    return int(lib().oracle_pages_for(n_tokens, page_tokens))
+
+
+def auto_resident_pages(max_ctx: int, page_bytes: int, n_layers: int,
+                        page_tokens: int = 256) -> int:
+    return int(lib().oracle_auto_resident_pages(max_ctx, page_tokens, page_bytes, n_layers))
+
+
+def page_location(n_tokens: int, n_resident: int, page: int, page_tokens: int = 256):
+    kind = ctypes.c_int()
+    idx = ctypes.c_long()
+    lib().oracle_page_location(n_tokens, page_tokens, n_resident, page,
+                               ctypes.byref(kind), ctypes.byref(idx))
+    return kind.value, idx.value

@@ -1,0 +1,32 @@
+/*
+ * kvs_oracle.h -- declarations of the CPU oracle (test infrastructure only;
+ * the product library never includes this header).
+ */
+#ifndef KVS_ORACLE_H
+#define KVS_ORACLE_H
+#include <stdint.h>
+
+#define ORACLE_PAGE_ABSENT   (-1)
+#define ORACLE_PAGE_RESIDENT 1
+#define ORACLE_PAGE_STREAMED 2
+
+double   oracle_half_to_double(uint16_t h);
+float    oracle_half_to_float(uint16_t h);
+uint16_t oracle_float_to_half(float f);
+
+void oracle_q8_0_block(const uint16_t x_h[32], uint8_t out[34]);
+void oracle_q4_0_block(const uint16_t x_h[32], uint8_t out[18]);
+void oracle_dequant_q8_0(const uint8_t blk[34], double out[32]);
+void oracle_dequant_q4_0(const uint8_t blk[18], double out[32]);
+void oracle_quantize_rows(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
+                          uint8_t* k_blocks, uint8_t* v_blocks);
+
+int oracle_attention(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
+                     const uint8_t* v_blocks, int n_q, int pos0, const uint16_t* q,
+                     double* out, double* lse);
+
+long oracle_pages_for(long n_tokens, int page_tokens);
+long oracle_auto_resident_pages(long max_ctx, int page_tokens, long page_bytes, int n_layers);
+int  oracle_page_location(long n_tokens, int page_tokens, long n_resident, long page,
+                          int* kind, long* index);
+#endif
