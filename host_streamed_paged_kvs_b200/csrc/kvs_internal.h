@@ -1,0 +1,95 @@
+// kvs_internal.h -- layout constants and kernel launcher declarations shared by
+// the host runtime (kvs_runtime.cpp) and the sm_100a kernels (kvs_kernels.cu,
+// kvs_chunk_mma.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kvs {
+
+// ---------------------------------------------------------------------------
+// Page layout in HBM and in pinned host memory (identical bytes on both sides).
+//
+// One page = 256 tokens of one layer, all kv heads: [n_kv][page_head].  One
+// page_head (53,248 B) is split by field so that every field is 16-byte
+// aligned and a 128-token half page of each field is contiguous:
+//   Kq  int8  [256 tok][128 dims]                 32,768 B  @ 0
+//   Kd  fp16  [256 tok][4 blocks]                   2,048 B  @ 32,768
+//   Vq  u8    [256 tok][4 blocks][16 B]            16,384 B  @ 34,816
+//         (byte j of a block holds code j in the low nibble, code j+16 high)
+//   Vd  fp16  [256 tok][4 blocks]                   2,048 B  @ 51,200
+// The canonical 34-byte Q8_0 / 18-byte Q4_0 blocks are a reshuffle of these
+// bytes (kvs_export_page does it on the host).
+// ---------------------------------------------------------------------------
+constexpr int kHeadDim = 128;
+constexpr int kPageTokens = 256;
+constexpr int kBlocks = kHeadDim / 32;                  // 4
+constexpr int kOffKq = 0;
+constexpr int kOffKd = kPageTokens * kHeadDim;          // 32768
+constexpr int kOffVq = kOffKd + kPageTokens * kBlocks * 2;  // 34816
+constexpr int kOffVd = kOffVq + kPageTokens * kHeadDim / 2;  // 51200
+constexpr int kPageHeadBytes = kOffVd + kPageTokens * kBlocks * 2;  // 53248
+constexpr int kPageHeadRows = kPageHeadBytes / 128;     // 416 rows of 128 B
+static_assert(kPageHeadBytes == 53248, "page-head layout");
+
+// split partials: per split and query row, (m, l) in the log2 domain + acc[128]
+struct PartialBuffers {
+    float2* ml;   // [n_splits][n_rows]
+    float* acc;   // [n_splits][n_rows][128]
+};
+
+struct AppendArgs {
+    const __half* k;         // [n_tok][n_kv][128]
+    const __half* v;
+    uint8_t* host_layer;     // device alias of the layer's host history (page 0)
+    uint8_t* res_layer;      // layer's resident region (slot 0)
+    int n_tok, pos0, n_kv;
+    int n_resident;          // R
+    int first_resident_page; // pages >= this are resident after the append
+    size_t page_bytes;
+};
+
+struct DecodeArgs {
+    const uint8_t* region;   // slot 0 of the region holding the pages (resident or ring)
+    int region_slot_base;    // global slot index of the region's first slot for the tensor map
+    int region_slots;        // slots in the region (R or N)
+    int slot0;               // region slot of unit 0
+    int page0;               // absolute page index of unit 0
+    int n_units;             // pages in this launch
+    int pages_per_split;
+    int split_base;          // first split index written by this launch
+    int len;                 // tokens in the history
+    int pos0, n_q;           // query positions pos0 .. pos0+n_q-1
+    const __half* q;         // [n_q][n_qh][128]
+    float q_scale;           // log2(e)/sqrt(128)
+    int n_qh, n_kv, group;   // group = n_qh / n_kv
+    int row_group_rows;      // rows handled per CTA (<= template ROWS)
+    PartialBuffers part;
+    int n_rows;              // n_q * n_qh
+    int* err;                // device error word (bounded waits)
+};
+
+struct MergeArgs {
+    PartialBuffers part;
+    int n_splits, n_rows;
+    float* out;              // [n_rows][128]
+    float* lse;              // [n_rows] or null
+};
+
+// launchers (return cudaGetLastError())
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
+                          cudaStream_t s);
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s);
+size_t decode_smem_bytes();
+
+// error bits written to the device error word
+enum : int {
+    kErrWaitTimeout = 1,
+};
+
+}  // namespace kvs

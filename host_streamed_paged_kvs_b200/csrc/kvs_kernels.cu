@@ -1,0 +1,513 @@
+// kvs_kernels.cu -- sm_100a kernels of the streamed quantized-KV attention path:
+//   K1 append_kernel  : fp16 K/V rows -> Q8_0 K / Q4_0 V blocks, written to the
+//                       pinned host history (mapped) and to the resident slot;
+//   K2 decode_kernel  : split-K flash-decode over resident pages or ring slots,
+//                       K/V dequantized in registers, per-split (m, l, acc);
+//   K3 merge_kernel   : log-sum-exp merge of the split partials.
+//
+// Method sources: "RaymondHuang210129/llama.cpp-adaptive-kv-streaming" (Summary:
+// pinned authoritative history, resident pages + one shared ring, Q8_0 K /
+// Q4_0 V) and "Feature/adaptive kv stream integration" (PR #326, section 1:
+// attention with streaming is the same computation as without it).
+#include <cuda_fp16.h>
+#include <math_constants.h>
+
+#include "kvs_internal.h"
+
+namespace kvs {
+
+// ----------------------------------------------------------------------------
+// small PTX helpers (TMA / bulk copies completing on an mbarrier)
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: gives up after ~2^24 polls (each poll suspends in hardware for
+// a short time), records the failure in the device error word and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err) {
+    for (uint32_t it = 0; it < (1u << 24); ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+    }
+    if (err) atomicOr(err, kErrWaitTimeout);
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// int8 byte i of w -> exact float, via 2^23 + (b + 128) - (2^23 + 128)
+__device__ __forceinline__ float s8_to_f(uint32_t w_biased, int i) {
+    return __uint_as_float(__byte_perm(w_biased, 0x4B00u, 0x5440u + i)) - 8388736.0f;
+}
+// 4-bit code c -> exact float (c - 8)
+__device__ __forceinline__ float q4_to_f(uint32_t c) {
+    return __uint_as_float(0x4B000000u | c) - 8388616.0f;
+}
+
+// ----------------------------------------------------------------------------
+// K1: quantize-on-append.  One warp per (token, kv head) row of 128 values;
+// lane l owns dims 4l..4l+3, so 8 lanes form one 32-value block.
+// Q8_0: d = amax/127 (binary32, correctly rounded), q = roundf(x/d).
+// Q4_0: m = value of largest |x| (first index on ties), d = m/-8,
+//       q = min(15, trunc(x/d + 8.5)), d == 0 -> q = 8.
+// The stored scales are the fp16 (round-to-nearest-even) values of d.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+    if (row >= a.n_tok * a.n_kv) return;
+    const int tok = row / a.n_kv;
+    const int h = row - tok * a.n_kv;
+    const int pos = a.pos0 + tok;
+    const int page = pos >> 8;
+    const int t = pos & 255;
+    const int b = lane >> 3;  // block of this lane
+    const int i = lane & 7;   // position of the lane in its block
+
+    const uint2 kraw = *reinterpret_cast<const uint2*>(a.k + (size_t)row * kHeadDim + 4 * lane);
+    const uint2 vraw = *reinterpret_cast<const uint2*>(a.v + (size_t)row * kHeadDim + 4 * lane);
+    float xk[4], xv[4];
+    {
+        const __half2 k01 = *reinterpret_cast<const __half2*>(&kraw.x);
+        const __half2 k23 = *reinterpret_cast<const __half2*>(&kraw.y);
+        const __half2 v01 = *reinterpret_cast<const __half2*>(&vraw.x);
+        const __half2 v23 = *reinterpret_cast<const __half2*>(&vraw.y);
+        xk[0] = __low2float(k01); xk[1] = __high2float(k01);
+        xk[2] = __low2float(k23); xk[3] = __high2float(k23);
+        xv[0] = __low2float(v01); xv[1] = __high2float(v01);
+        xv[2] = __low2float(v23); xv[3] = __high2float(v23);
+    }
+
+    // ---- Q8_0 (K) ----
+    float amax = fmaxf(fmaxf(fabsf(xk[0]), fabsf(xk[1])), fmaxf(fabsf(xk[2]), fabsf(xk[3])));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    const float dk = __fdiv_rn(amax, 127.0f);
+    uint32_t kq = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        int q = 0;
+        if (dk != 0.0f) q = static_cast<int>(roundf(__fdiv_rn(xk[u], dk)));
+        kq |= (static_cast<uint32_t>(q) & 0xffu) << (8 * u);
+    }
+    const __half dk_h = __float2half_rn(dk);
+
+    // ---- Q4_0 (V) ----
+    float va = 0.0f, vm = 0.0f;
+    int vi = 1 << 30;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const float ax = fabsf(xv[u]);
+        if (ax > va) { va = ax; vm = xv[u]; vi = 4 * i + u; }
+    }
+#pragma unroll
+    for (int off = 1; off <= 4; off <<= 1) {
+        const float pa = __shfl_xor_sync(0xffffffffu, va, off);
+        const float pm = __shfl_xor_sync(0xffffffffu, vm, off);
+        const int pi = __shfl_xor_sync(0xffffffffu, vi, off);
+        if (pa > va || (pa == va && pi < vi)) { va = pa; vm = pm; vi = pi; }
+    }
+    const float dv = __fdiv_rn(vm, -8.0f);
+    uint32_t codes = 0;  // 4 codes of this lane, one per byte
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        int q = 8;
+        if (dv != 0.0f) q = min(15, static_cast<int>(__fadd_rn(__fdiv_rn(xv[u], dv), 8.5f)));
+        codes |= static_cast<uint32_t>(q) << (8 * u);
+    }
+    const uint32_t partner = __shfl_xor_sync(0xffffffffu, codes, 4);  // codes j+16 for lanes i<4
+    const uint32_t vq = codes | (partner << 4);  // byte u: q_(4i+u) | q_(4i+u+16) << 4
+    const __half dv_h = __float2half_rn(dv);
+
+    // ---- stores: host history (always) and resident slot (if resident) ----
+    auto store = [&](uint8_t* ph) {
+        *reinterpret_cast<uint32_t*>(ph + kOffKq + t * kHeadDim + 4 * lane) = kq;
+        if (i == 0) {
+            *reinterpret_cast<__half*>(ph + kOffKd + t * 8 + 2 * b) = dk_h;
+            *reinterpret_cast<__half*>(ph + kOffVd + t * 8 + 2 * b) = dv_h;
+        }
+        if (i < 4) *reinterpret_cast<uint32_t*>(ph + kOffVq + t * 64 + b * 16 + 4 * i) = vq;
+    };
+    store(a.host_layer + (size_t)page * a.page_bytes + (size_t)h * kPageHeadBytes);
+    if (page >= a.first_resident_page) {
+        const int slot = page % a.n_resident;
+        store(a.res_layer + (size_t)slot * a.page_bytes + (size_t)h * kPageHeadBytes);
+    }
+}
+
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
+    const int rows = a.n_tok * a.n_kv;
+    append_kernel<<<(rows + 3) / 4, 128, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------------------
+// K2: split-K flash-decode.  CTA = (split, kv head, row group), 128 threads.
+// A split is a run of pages; each page is consumed as two 128-token stages.
+// Stage bytes land in shared memory through TMA: the K quants with the
+// 128-byte swizzle (so a thread per key reads its row without bank conflicts
+// while the query chunk is a broadcast), the K scales, V codes and V scales as
+// 1-D bulk copies.  QK^T: thread = key, all rows of the GQA group.  Softmax:
+// online, log2 domain, CTA-wide max per stage.  PV: warp = 32 keys, lane = 4
+// dims.  Output per split: (m, l) and acc[128] for every query row.
+// ----------------------------------------------------------------------------
+constexpr int kThreads = 128;
+constexpr int kStageKeys = 128;
+constexpr int kStageKq = 0;
+constexpr int kStageKd = kStageKeys * kHeadDim;            // 16384
+constexpr int kStageVq = kStageKd + kStageKeys * kBlocks * 2;  // 17408
+constexpr int kStageVd = kStageVq + kStageKeys * kHeadDim / 2;  // 25600
+constexpr int kStageBytes = kStageVd + kStageKeys * kBlocks * 2;  // 26624
+constexpr int kStages = 3;
+constexpr int kMaxRows = 8;
+constexpr size_t kDecodeSmem = 1024 /*align slack*/ + kStages * kStageBytes +
+                               kMaxRows * kHeadDim * 4 /*sQ*/ + kStageKeys * kMaxRows * 4 /*sP*/ +
+                               4 * kMaxRows * 4 /*sMax*/ + 4 * kMaxRows * 4 /*sL*/ + kStages * 8;
+static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-B swizzle alignment");
+static_assert(4 * kMaxRows * kHeadDim * 4 <= kStages * kStageBytes, "reduction scratch fits");
+
+size_t decode_smem_bytes() { return kDecodeSmem; }
+
+template <int ROWS>
+__global__ void __launch_bounds__(kThreads, 2)
+    decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* stage = smem;
+    float* sQ = reinterpret_cast<float*>(smem + kStages * kStageBytes);  // [ROWS][128]
+    float* sP = sQ + kMaxRows * kHeadDim;                              // [128 keys][8]
+    float* sMax = sP + kStageKeys * kMaxRows;                          // [4 warps][8]
+    float* sL = sMax + 4 * kMaxRows;                                   // [4 warps][8]
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sL + 4 * kMaxRows);    // [kStages]
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int h = blockIdx.y;
+    const int split = blockIdx.x;
+    const int row_begin = blockIdx.z * ROWS;
+    const int n_local_rows = a.n_q * a.group;
+    const int rows_here = min(ROWS, n_local_rows - row_begin);
+    const int u0 = split * a.pages_per_split;
+    const int u1 = min(a.n_units, u0 + a.pages_per_split);
+    const int n_st = 2 * (u1 - u0);
+
+    // queries of this CTA's rows, pre-scaled into the log2 domain
+    for (int idx = tid; idx < ROWS * kHeadDim; idx += kThreads) {
+        const int r = idx / kHeadDim, d = idx - r * kHeadDim;
+        float v = 0.0f;
+        if (r < rows_here) {
+            const int lr = row_begin + r;
+            const int j = lr / a.group, g = lr - j * a.group;
+            v = __half2float(a.q[((size_t)j * a.n_qh + h * a.group + g) * kHeadDim + d]) *
+                a.q_scale;
+        }
+        sQ[idx] = v;
+    }
+    int qpos[ROWS];
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r)
+        qpos[r] = (r < rows_here) ? a.pos0 + (row_begin + r) / a.group : -1;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&bar[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    auto issue = [&](int st) {
+        const int u = u0 + (st >> 1), half = st & 1;
+        const int slot = (a.slot0 + u) % a.region_slots;
+        const uint8_t* ph = a.region + ((size_t)slot * a.n_kv + h) * kPageHeadBytes;
+        uint8_t* dst = stage + (st % kStages) * kStageBytes;
+        uint64_t* b = &bar[st % kStages];
+        mbar_expect_tx(b, kStageBytes);
+        const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * kPageHeadRows + half * kStageKeys;
+        tma_load_2d(dst + kStageKq, &kmap, 0, krow, b);
+        bulk_load(dst + kStageKd, ph + kOffKd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
+        bulk_load(dst + kStageVq, ph + kOffVq + half * (kStageKeys * kHeadDim / 2), kStageKeys * kHeadDim / 2, b);
+        bulk_load(dst + kStageVd, ph + kOffVd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
+    };
+    if (tid == 0) {
+        for (int st = 0; st < kStages && st < n_st; ++st) issue(st);
+    }
+
+    float m_run[ROWS], l_run[ROWS], acc[ROWS][4];
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) {
+        m_run[r] = -CUDART_INF_F;
+        l_run[r] = 0.0f;
+        acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.0f;
+    }
+    const int vb = lane >> 3, vi = lane & 7;  // PV: block and byte pair of this lane
+    bool ok = true;
+
+    for (int st = 0; st < n_st; ++st) {
+        uint8_t* sb = stage + (st % kStages) * kStageBytes;
+        if (!mbar_wait_bounded(&bar[st % kStages], (st / kStages) & 1, a.err)) {
+            ok = false;
+        }
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+        const int u = u0 + (st >> 1), half = st & 1;
+        const int kpos0 = (a.page0 + u) * kPageTokens + half * kStageKeys;
+
+        // ---- QK^T: thread = key ----
+        const int key = tid;
+        const int kpos = kpos0 + key;
+        float s[ROWS];
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) s[r] = 0.0f;
+        const uint8_t* krow = sb + kStageKq + key * kHeadDim;
+#pragma unroll
+        for (int blk = 0; blk < kBlocks; ++blk) {
+            float part[ROWS];
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) part[r] = 0.0f;
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+                const int c = blk * 2 + c2;
+                const uint4 raw = *reinterpret_cast<const uint4*>(krow + ((c ^ (key & 7)) << 4));
+                const uint32_t w[4] = {raw.x ^ 0x80808080u, raw.y ^ 0x80808080u,
+                                       raw.z ^ 0x80808080u, raw.w ^ 0x80808080u};
+#pragma unroll
+                for (int uu = 0; uu < 4; ++uu) {
+                    const float k0 = s8_to_f(w[uu], 0), k1 = s8_to_f(w[uu], 1);
+                    const float k2 = s8_to_f(w[uu], 2), k3 = s8_to_f(w[uu], 3);
+#pragma unroll
+                    for (int r = 0; r < ROWS; ++r) {
+                        const float4 qv =
+                            *reinterpret_cast<const float4*>(sQ + r * kHeadDim + c * 16 + uu * 4);
+                        part[r] = fmaf(qv.x, k0, part[r]);
+                        part[r] = fmaf(qv.y, k1, part[r]);
+                        part[r] = fmaf(qv.z, k2, part[r]);
+                        part[r] = fmaf(qv.w, k3, part[r]);
+                    }
+                }
+            }
+            const float kd = __half2float(
+                *reinterpret_cast<const __half*>(sb + kStageKd + key * (kBlocks * 2) + blk * 2));
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) s[r] = fmaf(kd, part[r], s[r]);
+        }
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+            if (kpos >= a.len || kpos > qpos[r]) s[r] = -CUDART_INF_F;
+            float mx = s[r];
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1)
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            if (lane == 0) sMax[warp * kMaxRows + r] = mx;
+        }
+        __syncthreads();
+        // the previous stage's buffer is free once every thread has passed this barrier
+        if (tid == 0 && st >= 1 && st - 1 + kStages < n_st) issue(st - 1 + kStages);
+
+        float alpha[ROWS];
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+            const float mx = fmaxf(fmaxf(sMax[r], sMax[kMaxRows + r]),
+                                   fmaxf(sMax[2 * kMaxRows + r], sMax[3 * kMaxRows + r]));
+            const float mn = fmaxf(m_run[r], mx);
+            const float mu = (mn == -CUDART_INF_F) ? 0.0f : mn;
+            alpha[r] = exp2f(m_run[r] - mu);
+            m_run[r] = mn;
+            sP[key * kMaxRows + r] = exp2f(s[r] - mu);
+        }
+        __syncthreads();
+
+        // ---- PV: warp = 32 keys, lane = dims {32b+2i, +1, +16, +17} ----
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+            l_run[r] *= alpha[r];
+            acc[r][0] *= alpha[r]; acc[r][1] *= alpha[r];
+            acc[r][2] *= alpha[r]; acc[r][3] *= alpha[r];
+        }
+        const uint8_t* vq_base = sb + kStageVq + vb * 16 + 2 * vi;
+        const uint8_t* vd_base = sb + kStageVd + vb * 2;
+#pragma unroll 4
+        for (int kk = 0; kk < 32; ++kk) {
+            const int key2 = warp * 32 + kk;
+            const uint32_t code = *reinterpret_cast<const uint16_t*>(vq_base + key2 * 64);
+            const float dv = __half2float(*reinterpret_cast<const __half*>(vd_base + key2 * 8));
+            const float v0 = q4_to_f(code & 0xFu) * dv;          // dim 32b+2i
+            const float v2 = q4_to_f((code >> 4) & 0xFu) * dv;   // dim 32b+2i+16
+            const float v1 = q4_to_f((code >> 8) & 0xFu) * dv;   // dim 32b+2i+1
+            const float v3 = q4_to_f((code >> 12) & 0xFu) * dv;  // dim 32b+2i+17
+            const float* pr = sP + key2 * kMaxRows;
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) {
+                const float p = pr[r];
+                l_run[r] += p;
+                acc[r][0] = fmaf(p, v0, acc[r][0]);
+                acc[r][1] = fmaf(p, v1, acc[r][1]);
+                acc[r][2] = fmaf(p, v2, acc[r][2]);
+                acc[r][3] = fmaf(p, v3, acc[r][3]);
+            }
+        }
+    }
+    if (!ok) return;  // a bounded wait gave up; the error word is set
+
+    // ---- reduce the four warps' partials and write the split's result ----
+    __syncthreads();  // stage buffers are reused as scratch
+    float* red = reinterpret_cast<float*>(stage);  // [4 warps][ROWS][128]
+    const int d0 = vb * 32 + 2 * vi;
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) {
+        float* dst = red + (warp * ROWS + r) * kHeadDim;
+        dst[d0] = acc[r][0];
+        dst[d0 + 1] = acc[r][1];
+        dst[d0 + 16] = acc[r][2];
+        dst[d0 + 17] = acc[r][3];
+        if (lane == 0) sL[warp * kMaxRows + r] = l_run[r];
+    }
+    __syncthreads();
+    const int split_g = a.split_base + split;
+    for (int idx = tid; idx < rows_here * kHeadDim; idx += kThreads) {
+        const int r = idx / kHeadDim, d = idx - r * kHeadDim;
+        const float v = red[(0 * ROWS + r) * kHeadDim + d] + red[(1 * ROWS + r) * kHeadDim + d] +
+                        red[(2 * ROWS + r) * kHeadDim + d] + red[(3 * ROWS + r) * kHeadDim + d];
+        const int lr = row_begin + r;
+        const int j = lr / a.group, g = lr - j * a.group;
+        const int grow = j * a.n_qh + h * a.group + g;
+        a.part.acc[((size_t)split_g * a.n_rows + grow) * kHeadDim + d] = v;
+    }
+    if (tid < rows_here) {
+        const int r = tid;
+        const int lr = row_begin + r;
+        const int j = lr / a.group, g = lr - j * a.group;
+        const int grow = j * a.n_qh + h * a.group + g;
+        const float l = sL[r] + sL[kMaxRows + r] + sL[2 * kMaxRows + r] + sL[3 * kMaxRows + r];
+        float mr = -CUDART_INF_F;
+        // m_run is identical in every thread; pick row r's value without dynamic indexing
+#pragma unroll
+        for (int rr = 0; rr < ROWS; ++rr)
+            if (rr == r) mr = m_run[rr];
+        a.part.ml[(size_t)split_g * a.n_rows + grow] = make_float2(mr, l);
+    }
+}
+
+template <int ROWS>
+static cudaError_t launch_decode_t(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
+                                   int n_row_groups, cudaStream_t s) {
+    // the shared-memory opt-in is per device: remember which devices have it
+    static unsigned long long configured = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !(configured & (1ull << dev))) {
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<ROWS>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kDecodeSmem);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) configured |= 1ull << dev;
+    }
+    dim3 grid(n_splits, a.n_kv, n_row_groups);
+    decode_kernel<ROWS><<<grid, kThreads, kDecodeSmem, s>>>(a, *kmap);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
+                          cudaStream_t s) {
+    const int rows = a.n_q * a.group;
+    switch (rows) {
+        case 1: return launch_decode_t<1>(a, kmap, n_splits, 1, s);
+        case 2: return launch_decode_t<2>(a, kmap, n_splits, 1, s);
+        case 3: return launch_decode_t<3>(a, kmap, n_splits, 1, s);
+        case 4: return launch_decode_t<4>(a, kmap, n_splits, 1, s);
+        case 5: return launch_decode_t<5>(a, kmap, n_splits, 1, s);
+        case 6: return launch_decode_t<6>(a, kmap, n_splits, 1, s);
+        case 7: return launch_decode_t<7>(a, kmap, n_splits, 1, s);
+        default: return launch_decode_t<8>(a, kmap, n_splits, (rows + 7) / 8, s);
+    }
+}
+
+// ----------------------------------------------------------------------------
+// K3: log-sum-exp merge.  One CTA per query row: M = max_s m_s,
+// L = sum_s 2^(m_s-M) l_s, O = sum_s 2^(m_s-M) acc_s / L, lse = ln2 (M + log2 L).
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) merge_kernel(const MergeArgs a) {
+    __shared__ float sm[4];
+    __shared__ float sacc[4][kHeadDim];
+    __shared__ float sl[4];
+    const int row = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float m = -CUDART_INF_F;
+    for (int s = tid; s < a.n_splits; s += 128) m = fmaxf(m, a.part.ml[(size_t)s * a.n_rows + row].x);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) sm[warp] = m;
+    __syncthreads();
+    const float M = fmaxf(fmaxf(sm[0], sm[1]), fmaxf(sm[2], sm[3]));
+    float L = 0.0f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = warp; s < a.n_splits; s += 4) {
+        const float2 ml = a.part.ml[(size_t)s * a.n_rows + row];
+        if (ml.y > 0.0f) {
+            const float w = exp2f(ml.x - M);
+            L = fmaf(w, ml.y, L);
+            const float4 v = *reinterpret_cast<const float4*>(
+                a.part.acc + ((size_t)s * a.n_rows + row) * kHeadDim + 4 * lane);
+            o.x = fmaf(w, v.x, o.x); o.y = fmaf(w, v.y, o.y);
+            o.z = fmaf(w, v.z, o.z); o.w = fmaf(w, v.w, o.w);
+        }
+    }
+    sacc[warp][4 * lane + 0] = o.x; sacc[warp][4 * lane + 1] = o.y;
+    sacc[warp][4 * lane + 2] = o.z; sacc[warp][4 * lane + 3] = o.w;
+    if (lane == 0) sl[warp] = L;
+    __syncthreads();
+    const float Lt = sl[0] + sl[1] + sl[2] + sl[3];
+    const float inv = 1.0f / Lt;
+    const float v = sacc[0][tid] + sacc[1][tid] + sacc[2][tid] + sacc[3][tid];
+    a.out[(size_t)row * kHeadDim + tid] = v * inv;
+    if (tid == 0 && a.lse) a.lse[row] = (M + log2f(Lt)) * 0.69314718055994530942f;
+}
+
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s) {
+    merge_kernel<<<a.n_rows, 128, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace kvs

@@ -1,0 +1,846 @@
+// kvs_runtime.cpp -- host runtime behind the C ABI in include/kvs.h: config
+// validation and auto sizing, the pinned host history, the device arena
+// (resident pages, ring slots, split partials, staging), the page table, the
+// copy-engine ring with its events, and the call sequencing of append/attend.
+//
+// Method sources:
+//  * "RaymondHuang210129/llama.cpp-adaptive-kv-streaming", Summary: the full KV
+//    history stays in pinned system RAM, only resident pages plus one shared
+//    ring buffer occupy device memory, an auxiliary layer borrows the same pool.
+//  * "llama.cpp adaptive KV streaming - spec fork notes", Phase arena:
+//    speculative verify batches: a generation batch wider than the configured
+//    maximum fails ("decode batch too wide") -> KVS_E_WIDTH.
+//  * "Feature/adaptive kv stream integration" (PR #326): auto sizing (10 % of
+//    the context resident per layer, 2048-token floor, 8192 MiB ceiling), the
+//    configuration gates (supported K/V type pair, one page byte size for all
+//    streamed layers), the minimum stage of one page, and the review's
+//    observation that a real implementation needs a device staging pool, a
+//    page table and a cudaMemcpyAsync ring.
+#include <algorithm>
+#include <chrono>
+#include <climits>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <thread>
+#include <vector>
+
+#include "../../include/kvs.h"
+#include "kvs_internal.h"
+
+using namespace kvs;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+std::string fmt(const char* f, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, f);
+    vsnprintf(buf, sizeof buf, f, ap);
+    va_end(ap);
+    return buf;
+}
+
+long pages_for(long tokens) { return (tokens + kPageTokens - 1) / kPageTokens; }
+
+// Auto resident pages: 10 % of max_ctx per layer rounded up to whole pages,
+// 2048-token floor, 8192 MiB ceiling over all layers.
+long auto_resident(long max_ctx, size_t page_bytes, int n_layers) {
+    long pages = (max_ctx + 10L * kPageTokens - 1) / (10L * kPageTokens);
+    pages = std::max(pages, (2048L + kPageTokens - 1) / kPageTokens);
+    const long cap = (long)((8192ull << 20) / (page_bytes * (size_t)n_layers));
+    pages = std::min(pages, cap);
+    return std::max(pages, 1L);
+}
+
+// Split layout: pages per split on the resident set and inside one ring chunk.
+// Few query rows (decode) -> one page per split for parallelism; many rows ->
+// coarser splits keep the partial buffer and the merge small.
+struct SplitPolicy {
+    int res_pps, ring_pps;
+};
+SplitPolicy split_policy(const kvs_config& c, int n_rows_total) {
+    SplitPolicy p;
+    if (n_rows_total <= 64) {
+        p.res_pps = 1;
+        p.ring_pps = 1;
+    } else {
+        p.res_pps = std::max(1, c.n_resident_pages / 8);
+        p.ring_pps = std::max(1, c.chunk_pages);
+    }
+    return p;
+}
+
+size_t max_splits(const kvs_config& c) {
+    const long P = pages_for(c.max_ctx);
+    const long R = std::min<long>(c.n_resident_pages, P);
+    const long S = P - R;
+    size_t worst = 0;
+    // the split count grows as the rows shrink; bound it over both policies
+    for (int rows : {1, c.max_q_tokens * c.n_q_heads}) {
+        const SplitPolicy sp = split_policy(c, rows);
+        size_t n = (size_t)((R + sp.res_pps - 1) / sp.res_pps);
+        if (S > 0 && c.n_ring_slots > 0) {
+            const long chunks = (S + c.chunk_pages - 1) / c.chunk_pages;
+            n += (size_t)chunks * (size_t)((c.chunk_pages + sp.ring_pps - 1) / sp.ring_pps);
+        }
+        worst = std::max(worst, n);
+    }
+    return std::max<size_t>(worst, 1);
+}
+
+struct ArenaLayout {
+    size_t resident, ring, part_ml, part_acc, stage_q, stage_kv, stage_out, stage_lse, err, total;
+};
+
+ArenaLayout arena_layout(const kvs_config& c) {
+    const size_t pb = (size_t)c.n_kv_heads * kPageHeadBytes;
+    const size_t rows = (size_t)c.max_q_tokens * c.n_q_heads;
+    const size_t ns = max_splits(c);
+    ArenaLayout L{};
+    size_t off = 0;
+    L.resident = off; off = align_up(off + (size_t)c.n_layers * c.n_resident_pages * pb, 1024);
+    L.ring = off;     off = align_up(off + (size_t)c.n_ring_slots * pb, 1024);
+    L.part_ml = off;  off = align_up(off + ns * rows * sizeof(float2));
+    L.part_acc = off; off = align_up(off + ns * rows * kHeadDim * sizeof(float));
+    L.stage_q = off;  off = align_up(off + rows * kHeadDim * sizeof(__half));
+    L.stage_kv = off; off = align_up(off + 2 * (size_t)c.max_q_tokens * c.n_kv_heads * kHeadDim * sizeof(__half));
+    L.stage_out = off; off = align_up(off + rows * kHeadDim * sizeof(float));
+    L.stage_lse = off; off = align_up(off + rows * sizeof(float));
+    L.err = off;      off = align_up(off + 256);
+    L.total = off;
+    return L;
+}
+
+int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::string& why) {
+    if (!in || !out) { why = "null config"; return KVS_E_INVAL; }
+    kvs_config c = *in;
+    if (c.n_layers < 1) { why = "n_layers must be >= 1"; return KVS_E_INVAL; }
+    if (c.n_kv_heads < 1 || c.n_q_heads < 1 || c.n_q_heads % c.n_kv_heads != 0) {
+        why = fmt("n_q_heads (%d) must be a positive multiple of n_kv_heads (%d)", c.n_q_heads, c.n_kv_heads);
+        return KVS_E_INVAL;
+    }
+    if (c.head_dim != kHeadDim) { why = fmt("head_dim %d unsupported (only 128)", c.head_dim); return KVS_E_INVAL; }
+    if (c.page_tokens != kPageTokens) { why = fmt("page_tokens %d unsupported (only 256)", c.page_tokens); return KVS_E_INVAL; }
+    if (c.type_k != KVS_TYPE_Q8_0 || c.type_v != KVS_TYPE_Q4_0) {
+        why = "block KV streaming is not supported for this K/V cache type pair (only K=Q8_0, V=Q4_0)";
+        return KVS_E_INVAL;
+    }
+    if (c.max_ctx < 1) { why = "max_ctx must be >= 1"; return KVS_E_INVAL; }
+    if (c.max_q_tokens < 1 || c.max_q_tokens > 4096) { why = "max_q_tokens must be in [1, 4096]"; return KVS_E_INVAL; }
+    if (c.n_resident_pages < 0 || c.n_ring_slots < 0 || c.chunk_pages < 0) {
+        why = "negative page counts";
+        return KVS_E_INVAL;
+    }
+    const size_t pb = (size_t)c.n_kv_heads * kPageHeadBytes;
+    const long P = pages_for(c.max_ctx);
+    if (c.n_resident_pages == 0) c.n_resident_pages = (int)auto_resident(c.max_ctx, pb, c.n_layers);
+    if (c.n_resident_pages > P) c.n_resident_pages = (int)P;
+    if (c.n_ring_slots == 0) {
+        if (c.n_resident_pages < P) {
+            why = fmt("all-resident mode (n_ring_slots=0) needs n_resident_pages >= %ld", P);
+            return KVS_E_INVAL;
+        }
+        c.chunk_pages = 0;
+    } else {
+        if (c.chunk_pages == 0) c.chunk_pages = std::max(1, c.n_ring_slots / 2);
+        if (c.chunk_pages > c.n_ring_slots || c.n_ring_slots % c.chunk_pages != 0) {
+            why = fmt("chunk_pages (%d) must divide n_ring_slots (%d)", c.chunk_pages, c.n_ring_slots);
+            return KVS_E_INVAL;
+        }
+    }
+    const ArenaLayout L = arena_layout(c);
+    if (c.arena_bytes != 0) {
+        if (c.arena_bytes < pb) {
+            why = fmt("arena %zu B is below the minimum stage of one page (%zu B)", c.arena_bytes, pb);
+            return KVS_E_ARENA;
+        }
+        if (c.arena_bytes < L.total) {
+            why = fmt("arena %zu B cannot hold resident pages + ring + partials (%zu B)", c.arena_bytes, L.total);
+            return KVS_E_ARENA;
+        }
+    }
+    c.arena_bytes = L.total;
+    if (host_bytes) *host_bytes = (size_t)c.n_layers * (size_t)P * pb;
+    *out = c;
+    return KVS_OK;
+}
+
+int plan_page(const kvs_config& c, long n_tokens, long page, int* kind, int* index) {
+    const long P = pages_for(n_tokens);
+    if (page < 0 || page >= P) {
+        *kind = KVS_PAGE_ABSENT;
+        *index = -1;
+        return KVS_OK;
+    }
+    const long R = c.n_resident_pages;
+    if (page >= P - R) {
+        *kind = KVS_PAGE_RESIDENT;
+        *index = (int)(page % R);
+    } else {
+        *kind = KVS_PAGE_STREAMED;
+        *index = (int)page;
+    }
+    return KVS_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool is_host_ptr(const void* p) {
+    if (!p) return false;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return true;
+    }
+    return at.type == cudaMemoryTypeHost || at.type == cudaMemoryTypeUnregistered;
+}
+
+struct LayerState {
+    int len = 0;
+    int pending_min_page = INT_MAX;  // lowest page written to the host since the copy stream last waited
+    bool hist_recorded = false;
+};
+
+enum TimedKind { kTDecodeRes, kTDecodeRing, kTMerge, kTAppend, kTChunkMma };
+
+struct Timed {
+    cudaEvent_t a, b;
+    int kind;
+    uint64_t bytes;
+};
+
+}  // namespace
+
+struct kvs_s {
+    kvs_config cfg{};
+    int device = 0;
+    size_t page_bytes = 0;
+    long P_max = 0;
+    size_t host_bytes = 0;
+    uint8_t* host = nullptr;
+    uint8_t* host_dev = nullptr;
+    uint8_t* arena = nullptr;
+    ArenaLayout lay{};
+    uint8_t* resident = nullptr;
+    uint8_t* ring = nullptr;
+    PartialBuffers part{};
+    __half *stage_q = nullptr, *stage_k = nullptr, *stage_v = nullptr;
+    float *stage_out = nullptr, *stage_lse = nullptr;
+    int* err_word = nullptr;
+    CUtensorMap map_res{}, map_ring{};
+    cudaStream_t cs = nullptr;
+    int n_groups = 0;
+    std::vector<cudaEvent_t> ev_full, ev_free, ev_hist;
+    std::vector<char> free_valid;
+    uint64_t ring_ctr = 0;
+    std::vector<LayerState> layers;
+    kvs_stats stats{};
+    std::vector<Timed> timed;
+    std::vector<cudaEvent_t> ev_pool;
+    std::string err;
+};
+
+namespace {
+
+int fail(kvs_t* kv, int code, const std::string& why) {
+    if (kv) kv->err = why;
+    g_last_error = why;
+    return code;
+}
+
+#define KVS_CK(kv, call)                                                                    \
+    do {                                                                                    \
+        cudaError_t e_ = (call);                                                            \
+        if (e_ != cudaSuccess)                                                              \
+            return fail((kv), KVS_E_CUDA, fmt("%s failed: %s", #call, cudaGetErrorString(e_))); \
+    } while (0)
+
+struct DeviceGuard {
+    int prev = -1;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        if (prev != dev) cudaSetDevice(dev);
+    }
+    ~DeviceGuard() {
+        int cur;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+cudaEvent_t pool_event(kvs_t* kv) {
+    if (!kv->ev_pool.empty()) {
+        cudaEvent_t e = kv->ev_pool.back();
+        kv->ev_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+bool profiling(const kvs_t* kv, cudaStream_t s) {
+    if (!(kv->cfg.flags & KVS_FLAG_PROFILE)) return false;
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(s, &st);
+    return st == cudaStreamCaptureStatusNone;
+}
+
+struct TimedScope {
+    kvs_t* kv;
+    cudaStream_t s;
+    bool on;
+    Timed t{};
+    TimedScope(kvs_t* k, cudaStream_t st, int kind, uint64_t bytes) : kv(k), s(st) {
+        on = profiling(k, st);
+        if (on) {
+            t.a = pool_event(k);
+            t.b = pool_event(k);
+            t.kind = kind;
+            t.bytes = bytes;
+            cudaEventRecord(t.a, s);
+        }
+    }
+    ~TimedScope() {
+        if (on) {
+            cudaEventRecord(t.b, s);
+            kv->timed.push_back(t);
+        }
+    }
+};
+
+int encode_map(kvs_t* kv, EncodeTiledFn fn, CUtensorMap* map, void* base, uint64_t rows) {
+    if (rows == 0) return KVS_OK;
+    cuuint64_t dims[2] = {128, rows};
+    cuuint64_t strides[1] = {128};
+    cuuint32_t box[2] = {128, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(kv, KVS_E_CUDA, fmt("cuTensorMapEncodeTiled failed (%d)", (int)r));
+    return KVS_OK;
+}
+
+void release(kvs_t* kv) {
+    if (!kv) return;
+    DeviceGuard g(kv->device);
+    for (auto& t : kv->timed) { cudaEventDestroy(t.a); cudaEventDestroy(t.b); }
+    for (auto e : kv->ev_pool) cudaEventDestroy(e);
+    for (auto e : kv->ev_full) if (e) cudaEventDestroy(e);
+    for (auto e : kv->ev_free) if (e) cudaEventDestroy(e);
+    for (auto e : kv->ev_hist) if (e) cudaEventDestroy(e);
+    if (kv->cs) cudaStreamDestroy(kv->cs);
+    if (kv->arena) cudaFree(kv->arena);
+    if (kv->host) cudaFreeHost(kv->host);
+    delete kv;
+}
+
+// bounded host wait on an event
+int wait_event(kvs_t* kv, cudaEvent_t e, double timeout_s) {
+    const auto t0 = std::chrono::steady_clock::now();
+    for (;;) {
+        cudaError_t q = cudaEventQuery(e);
+        if (q == cudaSuccess) return KVS_OK;
+        if (q != cudaErrorNotReady) return fail(kv, KVS_E_CUDA, fmt("cudaEventQuery: %s", cudaGetErrorString(q)));
+        const double el = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
+        if (el > timeout_s) return fail(kv, KVS_E_TIMEOUT, "bounded wait for GPU work timed out");
+        std::this_thread::sleep_for(std::chrono::microseconds(50));
+    }
+}
+
+int sync_all(kvs_t* kv, cudaStream_t user, double timeout_s) {
+    cudaEvent_t e1 = pool_event(kv), e2 = pool_event(kv);
+    KVS_CK(kv, cudaEventRecord(e1, kv->cs));
+    KVS_CK(kv, cudaEventRecord(e2, user));
+    int rc = wait_event(kv, e1, timeout_s);
+    if (rc == KVS_OK) rc = wait_event(kv, e2, timeout_s);
+    kv->ev_pool.push_back(e1);
+    kv->ev_pool.push_back(e2);
+    if (rc != KVS_OK) return rc;
+    int err = 0;
+    KVS_CK(kv, cudaMemcpy(&err, kv->err_word, sizeof(int), cudaMemcpyDeviceToHost));
+    if (err) return fail(kv, KVS_E_TIMEOUT, fmt("a kernel's bounded wait gave up (error word %d)", err));
+    return KVS_OK;
+}
+
+void fold_timed(kvs_t* kv) {
+    for (auto& t : kv->timed) {
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, t.a, t.b) != cudaSuccess) { cudaGetLastError(); ms = 0.f; }
+        switch (t.kind) {
+            case kTDecodeRes: kv->stats.ms_decode_resident += ms; kv->stats.n_decode_resident++;
+                              kv->stats.bytes_decode_resident += t.bytes; break;
+            case kTDecodeRing: kv->stats.ms_decode_ring += ms; kv->stats.n_decode_ring++;
+                               kv->stats.bytes_decode_ring += t.bytes; break;
+            case kTMerge: kv->stats.ms_merge += ms; kv->stats.n_merge++; break;
+            case kTAppend: kv->stats.ms_append += ms; kv->stats.n_append++; break;
+            case kTChunkMma: kv->stats.ms_chunk_mma += ms; kv->stats.n_chunk_mma++; break;
+        }
+        kv->ev_pool.push_back(t.a);
+        kv->ev_pool.push_back(t.b);
+    }
+    kv->timed.clear();
+}
+
+}  // namespace
+
+// ============================================================================
+// C ABI
+// ============================================================================
+extern "C" {
+
+int kvs_resolve_config(const kvs_config* in, kvs_config* out, size_t* host_bytes) {
+    std::string why;
+    int rc = resolve(in, out, host_bytes, why);
+    if (rc != KVS_OK) g_last_error = why;
+    return rc;
+}
+
+size_t kvs_page_bytes(const kvs_config* cfg) {
+    return cfg ? (size_t)cfg->n_kv_heads * kPageHeadBytes : 0;
+}
+
+int kvs_plan_page(const kvs_config* c, int n_tokens, int page, int* kind, int* index) {
+    if (!c || !kind || !index || n_tokens < 0 || c->n_resident_pages < 1) {
+        g_last_error = "kvs_plan_page: bad arguments (config must be resolved)";
+        return KVS_E_INVAL;
+    }
+    return plan_page(*c, n_tokens, page, kind, index);
+}
+
+int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
+    if (!out) return fail(nullptr, KVS_E_INVAL, "kvs_create: null out");
+    *out = nullptr;
+    kvs_config c;
+    size_t host_bytes = 0;
+    std::string why;
+    int rc = resolve(cfg, &c, &host_bytes, why);
+    if (rc != KVS_OK) return fail(nullptr, rc, why);
+    int n_dev = 0;
+    if (cudaGetDeviceCount(&n_dev) != cudaSuccess || n_dev == 0) {
+        cudaGetLastError();
+        return fail(nullptr, KVS_E_CUDA, "no CUDA device: libkvs has no CPU fallback");
+    }
+    if (device < 0 || device >= n_dev) return fail(nullptr, KVS_E_INVAL, fmt("device %d out of range", device));
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, device) != cudaSuccess || prop.major < 10)
+        return fail(nullptr, KVS_E_INVAL, "libkvs is built for sm_100a (B200)");
+
+    kvs_t* kv = new kvs_t();
+    kv->cfg = c;
+    kv->device = device;
+    kv->page_bytes = (size_t)c.n_kv_heads * kPageHeadBytes;
+    kv->P_max = pages_for(c.max_ctx);
+    kv->host_bytes = host_bytes;
+    kv->lay = arena_layout(c);
+    DeviceGuard g(device);
+    auto bail = [&](int code, const std::string& w) {
+        g_last_error = w;
+        release(kv);
+        return code;
+    };
+    cudaError_t e = cudaHostAlloc(reinterpret_cast<void**>(&kv->host), host_bytes,
+                                  cudaHostAllocMapped | cudaHostAllocPortable);
+    if (e != cudaSuccess) {
+        kv->host = nullptr;
+        return bail(KVS_E_NOMEM, fmt("cudaHostAlloc(%zu B pinned history) failed: %s", host_bytes, cudaGetErrorString(e)));
+    }
+    std::memset(kv->host, 0, host_bytes);
+    e = cudaHostGetDevicePointer(reinterpret_cast<void**>(&kv->host_dev), kv->host, 0);
+    if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("cudaHostGetDevicePointer: %s", cudaGetErrorString(e)));
+    e = cudaMalloc(reinterpret_cast<void**>(&kv->arena), kv->lay.total);
+    if (e != cudaSuccess) {
+        kv->arena = nullptr;
+        return bail(KVS_E_ARENA, fmt("cudaMalloc(arena %zu B) failed: %s", kv->lay.total, cudaGetErrorString(e)));
+    }
+    e = cudaMemset(kv->arena, 0, kv->lay.total);
+    if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("cudaMemset: %s", cudaGetErrorString(e)));
+    kv->resident = kv->arena + kv->lay.resident;
+    kv->ring = kv->arena + kv->lay.ring;
+    kv->part.ml = reinterpret_cast<float2*>(kv->arena + kv->lay.part_ml);
+    kv->part.acc = reinterpret_cast<float*>(kv->arena + kv->lay.part_acc);
+    kv->stage_q = reinterpret_cast<__half*>(kv->arena + kv->lay.stage_q);
+    kv->stage_k = reinterpret_cast<__half*>(kv->arena + kv->lay.stage_kv);
+    kv->stage_v = kv->stage_k + (size_t)c.max_q_tokens * c.n_kv_heads * kHeadDim;
+    kv->stage_out = reinterpret_cast<float*>(kv->arena + kv->lay.stage_out);
+    kv->stage_lse = reinterpret_cast<float*>(kv->arena + kv->lay.stage_lse);
+    kv->err_word = reinterpret_cast<int*>(kv->arena + kv->lay.err);
+
+    e = cudaStreamCreateWithFlags(&kv->cs, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("cudaStreamCreate: %s", cudaGetErrorString(e)));
+    kv->n_groups = c.n_ring_slots > 0 ? c.n_ring_slots / c.chunk_pages : 0;
+    kv->ev_full.assign(kv->n_groups, nullptr);
+    kv->ev_free.assign(kv->n_groups, nullptr);
+    kv->free_valid.assign(kv->n_groups, 0);
+    for (int i = 0; i < kv->n_groups; ++i) {
+        if (cudaEventCreateWithFlags(&kv->ev_full[i], cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&kv->ev_free[i], cudaEventDisableTiming) != cudaSuccess)
+            return bail(KVS_E_CUDA, "cudaEventCreate failed");
+    }
+    kv->ev_hist.assign(c.n_layers, nullptr);
+    for (int i = 0; i < c.n_layers; ++i)
+        if (cudaEventCreateWithFlags(&kv->ev_hist[i], cudaEventDisableTiming) != cudaSuccess)
+            return bail(KVS_E_CUDA, "cudaEventCreate failed");
+    kv->layers.assign(c.n_layers, LayerState{});
+
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr);
+    if (e != cudaSuccess || qr != cudaDriverEntryPointSuccess || !fn)
+        return bail(KVS_E_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+    auto enc = reinterpret_cast<EncodeTiledFn>(fn);
+    const uint64_t res_rows = (uint64_t)c.n_layers * c.n_resident_pages * c.n_kv_heads * kPageHeadRows;
+    const uint64_t ring_rows = (uint64_t)c.n_ring_slots * c.n_kv_heads * kPageHeadRows;
+    if (encode_map(kv, enc, &kv->map_res, kv->resident, res_rows) != KVS_OK) return bail(KVS_E_CUDA, kv->err);
+    if (encode_map(kv, enc, &kv->map_ring, kv->ring, ring_rows) != KVS_OK) return bail(KVS_E_CUDA, kv->err);
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("create sync: %s", cudaGetErrorString(e)));
+    if (getenv("KVS_LOG")) {
+        fprintf(stderr,
+                "kvs: pool created: %d layer(s), %d resident pages/layer, %d ring slots (chunk %d), "
+                "page %zu B, arena %.2f MiB, pinned history %.2f MiB, device %d\n",
+                c.n_layers, c.n_resident_pages, c.n_ring_slots, c.chunk_pages, kv->page_bytes,
+                kv->lay.total / 1048576.0, host_bytes / 1048576.0, device);
+    }
+    *out = kv;
+    return KVS_OK;
+}
+
+void kvs_destroy(kvs_t* kv) {
+    if (!kv) return;
+    {
+        DeviceGuard g(kv->device);
+        cudaEvent_t e = pool_event(kv);
+        if (e && cudaEventRecord(e, kv->cs) == cudaSuccess) wait_event(kv, e, 60.0);
+        if (e) kv->ev_pool.push_back(e);
+        cudaDeviceSynchronize();
+    }
+    release(kv);
+}
+
+int kvs_append(kvs_t* kv, int layer, int pos0, int n_tok, const void* k_f16, const void* v_f16,
+               void* stream) {
+    if (!kv) return fail(nullptr, KVS_E_INVAL, "null handle");
+    const kvs_config& c = kv->cfg;
+    if (layer < 0 || layer >= c.n_layers) return fail(kv, KVS_E_INVAL, fmt("layer %d out of range", layer));
+    if (n_tok < 1) return fail(kv, KVS_E_INVAL, "n_tok must be >= 1");
+    if (!k_f16 || !v_f16) return fail(kv, KVS_E_INVAL, "null K/V");
+    const bool host_k = is_host_ptr(k_f16), host_v = is_host_ptr(v_f16);
+    // host K/V go through staging buffers sized for max_q_tokens; device K/V
+    // may be any width (history pre-fill)
+    if ((host_k || host_v) && n_tok > c.max_q_tokens)
+        return fail(kv, KVS_E_WIDTH, fmt("append batch too wide: %d > max_q_tokens %d", n_tok, c.max_q_tokens));
+    LayerState& ls = kv->layers[layer];
+    if (pos0 < 0 || pos0 > ls.len)
+        return fail(kv, KVS_E_ORDER, fmt("append at %d is not contiguous with length %d", pos0, ls.len));
+    if ((long)pos0 + n_tok > c.max_ctx)
+        return fail(kv, KVS_E_INVAL, fmt("append beyond max_ctx (%d)", c.max_ctx));
+    DeviceGuard g(kv->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t kv_elems = (size_t)n_tok * c.n_kv_heads * kHeadDim;
+    const __half* k = static_cast<const __half*>(k_f16);
+    const __half* v = static_cast<const __half*>(v_f16);
+    if (host_k) {
+        KVS_CK(kv, cudaMemcpyAsync(kv->stage_k, k_f16, kv_elems * 2, cudaMemcpyHostToDevice, s));
+        k = kv->stage_k;
+    }
+    if (host_v) {
+        KVS_CK(kv, cudaMemcpyAsync(kv->stage_v, v_f16, kv_elems * 2, cudaMemcpyHostToDevice, s));
+        v = kv->stage_v;
+    }
+    if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 7)
+        return fail(kv, KVS_E_INVAL, "K/V must be 8-byte aligned");
+
+    const long R = c.n_resident_pages;
+    const long P_old = pages_for(ls.len), P_new = pages_for((long)pos0 + n_tok);
+    const long f_old = std::max(0L, P_old - R), f_new = std::max(0L, P_new - R);
+    // pages that re-enter the resident set after a roll-back and keep tokens
+    // below pos0 are copied back from the authoritative host history
+    for (long p = f_new; p < P_new; ++p) {
+        const bool was_res = (p >= f_old && p < P_old);
+        if (!was_res && p * kPageTokens < pos0) {
+            const size_t src = ((size_t)layer * kv->P_max + p) * kv->page_bytes;
+            uint8_t* dst = kv->resident + ((size_t)layer * R + (size_t)(p % R)) * kv->page_bytes;
+            KVS_CK(kv, cudaMemcpyAsync(dst, kv->host + src, kv->page_bytes, cudaMemcpyHostToDevice, s));
+        }
+    }
+    AppendArgs a;
+    a.k = k;
+    a.v = v;
+    a.host_layer = kv->host_dev + (size_t)layer * kv->P_max * kv->page_bytes;
+    a.res_layer = kv->resident + (size_t)layer * R * kv->page_bytes;
+    a.n_tok = n_tok;
+    a.pos0 = pos0;
+    a.n_kv = c.n_kv_heads;
+    a.n_resident = (int)R;
+    a.first_resident_page = (int)f_new;
+    a.page_bytes = kv->page_bytes;
+    {
+        TimedScope ts(kv, s, kTAppend, 0);
+        KVS_CK(kv, launch_append(a, s));
+    }
+    kv->stats.kernel_launches++;
+    KVS_CK(kv, cudaEventRecord(kv->ev_hist[layer], s));
+    ls.hist_recorded = true;
+    ls.pending_min_page = std::min(ls.pending_min_page, pos0 / kPageTokens);
+    ls.len = pos0 + n_tok;
+    kv->stats.appends++;
+    kv->stats.tokens_appended += n_tok;
+    return KVS_OK;
+}
+
+int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float* out, float* lse,
+               void* stream) {
+    if (!kv) return fail(nullptr, KVS_E_INVAL, "null handle");
+    const kvs_config& c = kv->cfg;
+    if (layer < 0 || layer >= c.n_layers) return fail(kv, KVS_E_INVAL, fmt("layer %d out of range", layer));
+    if (n_q < 1) return fail(kv, KVS_E_INVAL, "n_q must be >= 1");
+    if (n_q > c.max_q_tokens)
+        return fail(kv, KVS_E_WIDTH, fmt("decode batch too wide: %d > max_q_tokens %d", n_q, c.max_q_tokens));
+    if (!q_f16 || !out) return fail(kv, KVS_E_INVAL, "null q/out");
+    LayerState& ls = kv->layers[layer];
+    if (pos0 < 0 || (long)pos0 + n_q > ls.len)
+        return fail(kv, KVS_E_ORDER, fmt("queries %d..%d beyond the history (length %d)", pos0, pos0 + n_q - 1, ls.len));
+    DeviceGuard g(kv->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int rows = n_q * c.n_q_heads;
+    const __half* q = static_cast<const __half*>(q_f16);
+    if (is_host_ptr(q_f16)) {
+        KVS_CK(kv, cudaMemcpyAsync(kv->stage_q, q_f16, (size_t)rows * kHeadDim * 2, cudaMemcpyHostToDevice, s));
+        q = kv->stage_q;
+    }
+    const bool host_out = is_host_ptr(out);
+    const bool host_lse = lse && is_host_ptr(lse);
+    float* dout = host_out ? kv->stage_out : out;
+    float* dlse = lse ? (host_lse ? kv->stage_lse : lse) : nullptr;
+
+    const long R = c.n_resident_pages;
+    const long P = pages_for(ls.len);
+    const long R_eff = std::min(R, P);
+    const long first_res = P - R_eff;
+    const long S = first_res;
+    const SplitPolicy sp = split_policy(c, rows);
+
+    DecodeArgs d{};
+    d.len = ls.len;
+    d.pos0 = pos0;
+    d.n_q = n_q;
+    d.q = q;
+    d.q_scale = (float)(1.4426950408889634 / std::sqrt((double)kHeadDim));
+    d.n_qh = c.n_q_heads;
+    d.n_kv = c.n_kv_heads;
+    d.group = c.n_q_heads / c.n_kv_heads;
+    d.part = kv->part;
+    d.n_rows = rows;
+    d.err = kv->err_word;
+
+    // 1) resident pages, attended in place
+    int split_base = 0;
+    {
+        d.region = kv->resident + (size_t)layer * R * kv->page_bytes;
+        d.region_slot_base = (int)(layer * R);
+        d.region_slots = (int)R;
+        d.slot0 = (int)(first_res % R);
+        d.page0 = (int)first_res;
+        d.n_units = (int)R_eff;
+        d.pages_per_split = sp.res_pps;
+        d.split_base = split_base;
+        const int ns = (int)((R_eff + sp.res_pps - 1) / sp.res_pps);
+        TimedScope ts(kv, s, kTDecodeRes, (uint64_t)R_eff * kv->page_bytes);
+        KVS_CK(kv, launch_decode(d, &kv->map_res, ns, s));
+        kv->stats.kernel_launches++;
+        split_base += ns;
+        kv->stats.bytes_resident_read += (uint64_t)R_eff * kv->page_bytes;
+    }
+    // 2) streamed pages through the ring, in ascending page order
+    if (S > 0) {
+        if (c.n_ring_slots == 0) return fail(kv, KVS_E_INVAL, "internal: streamed pages without a ring");
+        if (ls.hist_recorded && ls.pending_min_page < S) {
+            KVS_CK(kv, cudaStreamWaitEvent(kv->cs, kv->ev_hist[layer], 0));
+            ls.pending_min_page = INT_MAX;
+        }
+        const int chunk = c.chunk_pages;
+        for (long i0 = 0; i0 < S; i0 += chunk) {
+            const int cpages = (int)std::min<long>(chunk, S - i0);
+            const int gidx = (int)(kv->ring_ctr % kv->n_groups);
+            kv->ring_ctr++;
+            if (kv->free_valid[gidx]) KVS_CK(kv, cudaStreamWaitEvent(kv->cs, kv->ev_free[gidx], 0));
+            uint8_t* dst = kv->ring + (size_t)gidx * chunk * kv->page_bytes;
+            const uint8_t* src = kv->host + ((size_t)layer * kv->P_max + (size_t)i0) * kv->page_bytes;
+            KVS_CK(kv, cudaMemcpyAsync(dst, src, (size_t)cpages * kv->page_bytes, cudaMemcpyHostToDevice, kv->cs));
+            KVS_CK(kv, cudaEventRecord(kv->ev_full[gidx], kv->cs));
+            KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_full[gidx], 0));
+            d.region = kv->ring;
+            d.region_slot_base = 0;
+            d.region_slots = c.n_ring_slots;
+            d.slot0 = gidx * chunk;
+            d.page0 = (int)i0;
+            d.n_units = cpages;
+            d.pages_per_split = sp.ring_pps;
+            d.split_base = split_base;
+            const int ns = (cpages + sp.ring_pps - 1) / sp.ring_pps;
+            {
+                TimedScope ts(kv, s, kTDecodeRing, (uint64_t)cpages * kv->page_bytes);
+                KVS_CK(kv, launch_decode(d, &kv->map_ring, ns, s));
+            }
+            kv->stats.kernel_launches++;
+            KVS_CK(kv, cudaEventRecord(kv->ev_free[gidx], s));
+            kv->free_valid[gidx] = 1;
+            split_base += ns;
+            kv->stats.pages_streamed += cpages;
+            kv->stats.bytes_h2d += (uint64_t)cpages * kv->page_bytes;
+            kv->stats.h2d_copies++;
+        }
+    }
+    // 3) log-sum-exp merge of all splits
+    MergeArgs m;
+    m.part = kv->part;
+    m.n_splits = split_base;
+    m.n_rows = rows;
+    m.out = dout;
+    m.lse = dlse;
+    {
+        TimedScope ts(kv, s, kTMerge, 0);
+        KVS_CK(kv, launch_merge(m, s));
+    }
+    kv->stats.kernel_launches++;
+    if (host_out)
+        KVS_CK(kv, cudaMemcpyAsync(out, dout, (size_t)rows * kHeadDim * 4, cudaMemcpyDeviceToHost, s));
+    if (host_lse) KVS_CK(kv, cudaMemcpyAsync(lse, dlse, (size_t)rows * 4, cudaMemcpyDeviceToHost, s));
+    kv->stats.attends++;
+    return KVS_OK;
+}
+
+int kvs_export_page(kvs_t* kv, int layer, int page, int from_device, void* host_dst) {
+    if (!kv || !host_dst) return fail(kv, KVS_E_INVAL, "null argument");
+    const kvs_config& c = kv->cfg;
+    if (layer < 0 || layer >= c.n_layers || page < 0 || page >= kv->P_max)
+        return fail(kv, KVS_E_INVAL, "layer/page out of range");
+    std::vector<uint8_t> buf(kv->page_bytes);
+    if (from_device) {
+        int kind, idx;
+        plan_page(c, kv->layers[layer].len, page, &kind, &idx);
+        if (kind != KVS_PAGE_RESIDENT) return fail(kv, KVS_E_INVAL, "page is not resident");
+        DeviceGuard g(kv->device);
+        const uint8_t* src = kv->resident + ((size_t)layer * c.n_resident_pages + idx) * kv->page_bytes;
+        KVS_CK(kv, cudaMemcpy(buf.data(), src, kv->page_bytes, cudaMemcpyDeviceToHost));
+    } else {
+        std::memcpy(buf.data(), kv->host + ((size_t)layer * kv->P_max + page) * kv->page_bytes, kv->page_bytes);
+    }
+    uint8_t* out = static_cast<uint8_t*>(host_dst);
+    const int H = c.n_kv_heads;
+    uint8_t* kout = out;
+    uint8_t* vout = out + (size_t)kPageTokens * H * kBlocks * 34;
+    for (int t = 0; t < kPageTokens; ++t)
+        for (int h = 0; h < H; ++h) {
+            const uint8_t* ph = buf.data() + (size_t)h * kPageHeadBytes;
+            for (int b = 0; b < kBlocks; ++b) {
+                uint8_t* kb = kout + (((size_t)t * H + h) * kBlocks + b) * 34;
+                std::memcpy(kb, ph + kOffKd + t * 8 + b * 2, 2);
+                std::memcpy(kb + 2, ph + kOffKq + t * kHeadDim + b * 32, 32);
+                uint8_t* vb = vout + (((size_t)t * H + h) * kBlocks + b) * 18;
+                std::memcpy(vb, ph + kOffVd + t * 8 + b * 2, 2);
+                std::memcpy(vb + 2, ph + kOffVq + t * 64 + b * 16, 16);
+            }
+        }
+    return KVS_OK;
+}
+
+int kvs_page_location(kvs_t* kv, int layer, int page, int* kind, int* index) {
+    if (!kv || !kind || !index) return fail(kv, KVS_E_INVAL, "null argument");
+    if (layer < 0 || layer >= kv->cfg.n_layers) return fail(kv, KVS_E_INVAL, "layer out of range");
+    return plan_page(kv->cfg, kv->layers[layer].len, page, kind, index);
+}
+
+int kvs_layer_length(kvs_t* kv, int layer, int* n_tokens) {
+    if (!kv || !n_tokens || layer < 0 || layer >= kv->cfg.n_layers) return fail(kv, KVS_E_INVAL, "bad argument");
+    *n_tokens = kv->layers[layer].len;
+    return KVS_OK;
+}
+
+int kvs_get_config(kvs_t* kv, kvs_config* out) {
+    if (!kv || !out) return fail(kv, KVS_E_INVAL, "null argument");
+    *out = kv->cfg;
+    return KVS_OK;
+}
+
+int kvs_get_stats(kvs_t* kv, kvs_stats* out) {
+    if (!kv || !out) return fail(kv, KVS_E_INVAL, "null argument");
+    if (!kv->timed.empty()) {
+        DeviceGuard g(kv->device);
+        int rc = wait_event(kv, kv->timed.back().b, 120.0);
+        if (rc != KVS_OK) return rc;
+        fold_timed(kv);
+    }
+    *out = kv->stats;
+    return KVS_OK;
+}
+
+int kvs_reset_stats(kvs_t* kv) {
+    if (!kv) return fail(kv, KVS_E_INVAL, "null handle");
+    if (!kv->timed.empty()) {
+        DeviceGuard g(kv->device);
+        int rc = wait_event(kv, kv->timed.back().b, 120.0);
+        if (rc != KVS_OK) return rc;
+        fold_timed(kv);
+    }
+    kv->stats = kvs_stats{};
+    return KVS_OK;
+}
+
+int kvs_sync(kvs_t* kv, void* stream, double timeout_s) {
+    if (!kv) return fail(nullptr, KVS_E_INVAL, "null handle");
+    DeviceGuard g(kv->device);
+    return sync_all(kv, static_cast<cudaStream_t>(stream), timeout_s);
+}
+
+int kvs_measure_h2d(kvs_t* kv, size_t chunk_bytes, size_t total_bytes, int reps, double* gbs) {
+    if (!kv || !gbs || chunk_bytes == 0 || reps < 1) return fail(kv, KVS_E_INVAL, "bad argument");
+    uint8_t* dst = kv->cfg.n_ring_slots ? kv->ring : kv->resident;
+    const size_t dst_bytes = kv->cfg.n_ring_slots ? (size_t)kv->cfg.n_ring_slots * kv->page_bytes
+                                                  : (size_t)kv->cfg.n_layers * kv->cfg.n_resident_pages * kv->page_bytes;
+    if (chunk_bytes > dst_bytes) return fail(kv, KVS_E_INVAL, "chunk larger than the device region");
+    total_bytes = std::min(total_bytes, kv->host_bytes) / chunk_bytes * chunk_bytes;
+    if (total_bytes == 0) return fail(kv, KVS_E_INVAL, "total smaller than one chunk");
+    DeviceGuard g(kv->device);
+    KVS_CK(kv, cudaStreamSynchronize(kv->cs));
+    cudaEvent_t a, b;
+    KVS_CK(kv, cudaEventCreate(&a));
+    KVS_CK(kv, cudaEventCreate(&b));
+    double best = 0.0;
+    const size_t slots = dst_bytes / chunk_bytes;
+    for (int r = 0; r < reps; ++r) {
+        cudaEventRecord(a, kv->cs);
+        for (size_t off = 0, i = 0; off < total_bytes; off += chunk_bytes, ++i)
+            cudaMemcpyAsync(dst + (i % slots) * chunk_bytes, kv->host + off, chunk_bytes,
+                            cudaMemcpyHostToDevice, kv->cs);
+        cudaEventRecord(b, kv->cs);
+        int rc = wait_event(kv, b, 120.0);
+        if (rc != KVS_OK) { cudaEventDestroy(a); cudaEventDestroy(b); return rc; }
+        float ms = 0;
+        cudaEventElapsedTime(&ms, a, b);
+        best = std::max(best, total_bytes / (ms * 1e-3) / 1e9);
+    }
+    cudaEventDestroy(a);
+    cudaEventDestroy(b);
+    *gbs = best;
+    return KVS_OK;
+}
+
+const char* kvs_last_error(kvs_t* kv) {
+    if (kv) return kv->err.c_str();
+    return g_last_error.c_str();
+}
+
+}  // extern "C"

@@ -1,0 +1,273 @@
+"""Thin Python binding of libkvs (include/kvs.h).
+
+Argument marshalling only: every step of the path runs in the CUDA library.
+Tensors are passed by address (torch CUDA tensors, pinned or plain CPU tensors,
+numpy arrays); streams by their cudaStream_t handle.  There is no fallback:
+importing this module fails loudly if libkvs.so has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkvs.so")
+
+KVS_OK = 0
+KVS_E_INVAL = -1
+KVS_E_ARENA = -2
+KVS_E_WIDTH = -3
+KVS_E_ORDER = -4
+KVS_E_CUDA = -5
+KVS_E_TIMEOUT = -6
+KVS_E_NOMEM = -7
+KVS_TYPE_Q4_0 = 2
+KVS_TYPE_Q8_0 = 8
+KVS_PAGE_ABSENT = -1
+KVS_PAGE_RESIDENT = 1
+KVS_PAGE_STREAMED = 2
+KVS_FLAG_PROFILE = 1
+
+ERROR_NAMES = {0: "KVS_OK", -1: "KVS_E_INVAL", -2: "KVS_E_ARENA", -3: "KVS_E_WIDTH",
+               -4: "KVS_E_ORDER", -5: "KVS_E_CUDA", -6: "KVS_E_TIMEOUT", -7: "KVS_E_NOMEM"}
+
+# every symbol the header declares
+EXPORTS = ["kvs_resolve_config", "kvs_page_bytes", "kvs_plan_page", "kvs_create", "kvs_destroy",
+           "kvs_append", "kvs_attend", "kvs_export_page", "kvs_page_location", "kvs_layer_length",
+           "kvs_get_config", "kvs_get_stats", "kvs_reset_stats", "kvs_sync", "kvs_measure_h2d",
+           "kvs_last_error"]
+
+
+class kvs_config(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int), ("n_q_heads", ctypes.c_int),
+                ("n_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("page_tokens", ctypes.c_int), ("max_ctx", ctypes.c_int),
+                ("n_resident_pages", ctypes.c_int), ("n_ring_slots", ctypes.c_int),
+                ("max_q_tokens", ctypes.c_int), ("type_k", ctypes.c_int),
+                ("type_v", ctypes.c_int), ("chunk_pages", ctypes.c_int),
+                ("flags", ctypes.c_int), ("arena_bytes", ctypes.c_size_t)]
+
+    def as_dict(self):
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+class kvs_stats(ctypes.Structure):
+    _fields_ = ([(n, ctypes.c_uint64) for n in
+                 ("appends", "attends", "tokens_appended", "pages_streamed", "bytes_h2d",
+                  "bytes_resident_read", "h2d_copies", "kernel_launches")] +
+                [(n, ctypes.c_double) for n in
+                 ("ms_decode_resident", "ms_decode_ring", "ms_merge", "ms_append", "ms_chunk_mma")] +
+                [(n, ctypes.c_uint64) for n in
+                 ("n_decode_resident", "n_decode_ring", "n_merge", "n_append", "n_chunk_mma",
+                  "bytes_decode_resident", "bytes_decode_ring")])
+
+    def as_dict(self):
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libkvs.so not found at {LIB_PATH}: build it with "
+            "`python -m host_streamed_paged_kvs_b200.build` (there is no CPU fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, cp = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER
+    L.kvs_resolve_config.argtypes = [cp(kvs_config), cp(kvs_config), cp(ctypes.c_size_t)]
+    L.kvs_page_bytes.restype = ctypes.c_size_t
+    L.kvs_page_bytes.argtypes = [cp(kvs_config)]
+    L.kvs_plan_page.argtypes = [cp(kvs_config), i, i, cp(i), cp(i)]
+    L.kvs_create.argtypes = [cp(kvs_config), i, cp(vp)]
+    L.kvs_destroy.argtypes = [vp]
+    L.kvs_destroy.restype = None
+    L.kvs_append.argtypes = [vp, i, i, i, vp, vp, vp]
+    L.kvs_attend.argtypes = [vp, i, i, i, vp, vp, vp, vp]
+    L.kvs_export_page.argtypes = [vp, i, i, i, vp]
+    L.kvs_page_location.argtypes = [vp, i, i, cp(i), cp(i)]
+    L.kvs_layer_length.argtypes = [vp, i, cp(i)]
+    L.kvs_get_config.argtypes = [vp, cp(kvs_config)]
+    L.kvs_get_stats.argtypes = [vp, cp(kvs_stats)]
+    L.kvs_reset_stats.argtypes = [vp]
+    L.kvs_sync.argtypes = [vp, vp, ctypes.c_double]
+    L.kvs_measure_h2d.argtypes = [vp, ctypes.c_size_t, ctypes.c_size_t, i, cp(ctypes.c_double)]
+    L.kvs_last_error.restype = ctypes.c_char_p
+    L.kvs_last_error.argtypes = [vp]
+    return L
+
+
+lib = _load()
+
+
+class KvsError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{ERROR_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+def _addr(x) -> Optional[int]:
+    """Address of a tensor / array / raw int (None -> NULL)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    if hasattr(x, "ctypes"):
+        return x.ctypes.data
+    raise TypeError(f"cannot take the address of {type(x)}")
+
+
+def _stream(s) -> Optional[int]:
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream  # torch.cuda.Stream
+
+
+def _check(rc: int, handle=None):
+    if rc != KVS_OK:
+        raise KvsError(rc, lib.kvs_last_error(handle).decode())
+
+
+def make_config(n_layers, n_q_heads, n_kv_heads, max_ctx, n_resident_pages=0, n_ring_slots=0,
+                max_q_tokens=1, chunk_pages=0, flags=0, arena_bytes=0, head_dim=128,
+                page_tokens=256, type_k=KVS_TYPE_Q8_0, type_v=KVS_TYPE_Q4_0) -> kvs_config:
+    return kvs_config(n_layers, n_q_heads, n_kv_heads, head_dim, page_tokens, max_ctx,
+                      n_resident_pages, n_ring_slots, max_q_tokens, type_k, type_v, chunk_pages,
+                      flags, arena_bytes)
+
+
+# ---- functions with the C names ------------------------------------------
+
+def kvs_resolve_config(cfg: kvs_config):
+    out = kvs_config()
+    hb = ctypes.c_size_t()
+    _check(lib.kvs_resolve_config(ctypes.byref(cfg), ctypes.byref(out), ctypes.byref(hb)))
+    return out, hb.value
+
+
+def kvs_page_bytes(cfg: kvs_config) -> int:
+    return lib.kvs_page_bytes(ctypes.byref(cfg))
+
+
+def kvs_plan_page(cfg: kvs_config, n_tokens: int, page: int):
+    k, i = ctypes.c_int(), ctypes.c_int()
+    _check(lib.kvs_plan_page(ctypes.byref(cfg), n_tokens, page, ctypes.byref(k), ctypes.byref(i)))
+    return k.value, i.value
+
+
+def kvs_create(cfg: kvs_config, device: int = 0) -> int:
+    h = ctypes.c_void_p()
+    _check(lib.kvs_create(ctypes.byref(cfg), device, ctypes.byref(h)))
+    return h.value
+
+
+def kvs_destroy(h: int) -> None:
+    lib.kvs_destroy(h)
+
+
+def kvs_append(h, layer, pos0, n_tok, k, v, stream=None) -> None:
+    _check(lib.kvs_append(h, layer, pos0, n_tok, _addr(k), _addr(v), _stream(stream)), h)
+
+
+def kvs_attend(h, layer, pos0, n_q, q, out, lse=None, stream=None) -> None:
+    _check(lib.kvs_attend(h, layer, pos0, n_q, _addr(q), _addr(out), _addr(lse), _stream(stream)), h)
+
+
+def kvs_export_page(h, layer, page, from_device, dst) -> None:
+    _check(lib.kvs_export_page(h, layer, page, int(from_device), _addr(dst)), h)
+
+
+def kvs_page_location(h, layer, page):
+    k, i = ctypes.c_int(), ctypes.c_int()
+    _check(lib.kvs_page_location(h, layer, page, ctypes.byref(k), ctypes.byref(i)), h)
+    return k.value, i.value
+
+
+def kvs_layer_length(h, layer) -> int:
+    n = ctypes.c_int()
+    _check(lib.kvs_layer_length(h, layer, ctypes.byref(n)), h)
+    return n.value
+
+
+def kvs_get_config(h) -> kvs_config:
+    c = kvs_config()
+    _check(lib.kvs_get_config(h, ctypes.byref(c)), h)
+    return c
+
+
+def kvs_get_stats(h) -> dict:
+    s = kvs_stats()
+    _check(lib.kvs_get_stats(h, ctypes.byref(s)), h)
+    return s.as_dict()
+
+
+def kvs_reset_stats(h) -> None:
+    _check(lib.kvs_reset_stats(h), h)
+
+
+def kvs_sync(h, stream=None, timeout_s: float = 60.0) -> None:
+    _check(lib.kvs_sync(h, _stream(stream), timeout_s), h)
+
+
+def kvs_measure_h2d(h, chunk_bytes: int, total_bytes: int, reps: int = 10) -> float:
+    g = ctypes.c_double()
+    _check(lib.kvs_measure_h2d(h, chunk_bytes, total_bytes, reps, ctypes.byref(g)), h)
+    return g.value
+
+
+def kvs_last_error(h=None) -> str:
+    return lib.kvs_last_error(h).decode()
+
+
+class KVS:
+    """Owning handle with the same calls as methods."""
+
+    def __init__(self, cfg: kvs_config, device: int = 0):
+        self.h = kvs_create(cfg, device)
+        self.cfg = kvs_get_config(self.h)
+
+    def append(self, layer, pos0, n_tok, k, v, stream=None):
+        kvs_append(self.h, layer, pos0, n_tok, k, v, stream)
+
+    def attend(self, layer, pos0, n_q, q, out, lse=None, stream=None):
+        kvs_attend(self.h, layer, pos0, n_q, q, out, lse, stream)
+
+    def export_page(self, layer, page, from_device, dst):
+        kvs_export_page(self.h, layer, page, from_device, dst)
+
+    def page_location(self, layer, page):
+        return kvs_page_location(self.h, layer, page)
+
+    def layer_length(self, layer):
+        return kvs_layer_length(self.h, layer)
+
+    def stats(self):
+        return kvs_get_stats(self.h)
+
+    def reset_stats(self):
+        kvs_reset_stats(self.h)
+
+    def sync(self, stream=None, timeout_s=60.0):
+        kvs_sync(self.h, stream, timeout_s)
+
+    def measure_h2d(self, chunk_bytes, total_bytes, reps=10):
+        return kvs_measure_h2d(self.h, chunk_bytes, total_bytes, reps)
+
+    def close(self):
+        if self.h:
+            kvs_destroy(self.h)
+            self.h = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

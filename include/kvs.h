@@ -1,0 +1,195 @@
+/*
+ * kvs.h -- C ABI of libkvs: host-streamed paged quantized KV attention on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (sources: "RaymondHuang210129/llama.cpp-adaptive-kv-streaming",
+ * Summary; "llama.cpp adaptive KV streaming - spec fork notes", Phase arena and
+ * Configuration; "Feature/adaptive kv stream integration", PR #326):
+ *   - the full KV history of every layer lives in pinned host memory and is
+ *     authoritative; K is stored as Q8_0 and V as Q4_0 (blocks of 32 values,
+ *     fp16 scale), grouped in 256-token pages;
+ *   - per layer only the most recent R pages are resident in device memory;
+ *     older pages stream in order through one device ring of N page slots that
+ *     all layers share, on a copy stream, so the copy of page i+k overlaps
+ *     attention over page i;
+ *   - attention is exact over every page (streaming on == streaming off).
+ *
+ * Conventions for every call below:
+ *   - return 0 (KVS_OK) on success or a negative KVS_E_* code; on failure the
+ *     handle is unchanged and kvs_last_error() describes the cause;
+ *   - device pointers are plain CUDA device addresses (for example a torch
+ *     tensor's data_ptr()); kvs_append/kvs_attend also accept host pointers and
+ *     then stage them through library-owned device buffers on `stream`;
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     stream ordered and asynchronous: results are valid once `stream` has
+ *     completed.  Appends and attends of one handle must be issued on one
+ *     stream, or the caller orders its streams itself;
+ *   - the library owns the pinned host history, the device arena (resident
+ *     pages, ring slots, split partials, staging), its copy stream and events.
+ *     The caller owns Q/K/V/out/lse buffers and `stream`.
+ *   - there is no CPU fallback: without a usable CUDA device kvs_create fails.
+ */
+#ifndef KVS_H
+#define KVS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------- */
+#define KVS_OK         0
+#define KVS_E_INVAL   (-1) /* bad argument, shape or unsupported K/V type pair   */
+#define KVS_E_ARENA   (-2) /* arena smaller than one page or than its contents   */
+#define KVS_E_WIDTH   (-3) /* n_q > max_q_tokens ("decode batch too wide")        */
+#define KVS_E_ORDER   (-4) /* append not contiguous / attend beyond the history  */
+#define KVS_E_CUDA    (-5) /* a CUDA runtime call failed                          */
+#define KVS_E_TIMEOUT (-6) /* a bounded host wait gave up                         */
+#define KVS_E_NOMEM   (-7) /* host (pinned) allocation failed                     */
+
+/* ---- cache types (only the pair K=Q8_0, V=Q4_0 is qualified) ------------- */
+#define KVS_TYPE_Q4_0 2
+#define KVS_TYPE_Q8_0 8
+
+/* ---- page kinds reported by kvs_page_location --------------------------- */
+#define KVS_PAGE_ABSENT   (-1)
+#define KVS_PAGE_RESIDENT 1
+#define KVS_PAGE_STREAMED 2
+
+/* ---- flags --------------------------------------------------------------- */
+#define KVS_FLAG_PROFILE 1 /* record CUDA events around kernels (kvs_get_stats) */
+
+typedef struct kvs_config {
+    int n_layers;         /* attention layers sharing the pool, auxiliary layers included (e.g. 16+1) */
+    int n_q_heads;        /* query heads; a multiple of n_kv_heads */
+    int n_kv_heads;       /* KV heads; q head h reads kv head h / (n_q_heads/n_kv_heads) */
+    int head_dim;         /* must be 128 */
+    int page_tokens;      /* must be 256 */
+    int max_ctx;          /* host history capacity in tokens per layer */
+    int n_resident_pages; /* resident pages per layer; 0 = auto (10 % of max_ctx, 8-page floor,
+                             8192 MiB ceiling over all layers) */
+    int n_ring_slots;     /* device ring slots (pages); 0 = all-resident mode, which needs
+                             n_resident_pages >= pages(max_ctx) */
+    int max_q_tokens;     /* widest append / attend batch (1, 1+n_draft or a 256-token ubatch) */
+    int type_k;           /* must be KVS_TYPE_Q8_0 */
+    int type_v;           /* must be KVS_TYPE_Q4_0 */
+    int chunk_pages;      /* pages per H2D copy; 0 = auto (n_ring_slots/2); must divide n_ring_slots */
+    int flags;            /* KVS_FLAG_* */
+    size_t arena_bytes;   /* device arena budget; 0 = exact fit; else must hold one page and all
+                             resident pages + ring + partials + staging */
+} kvs_config;
+
+typedef struct kvs_stats {
+    uint64_t appends, attends;         /* calls */
+    uint64_t tokens_appended;
+    uint64_t pages_streamed;           /* pages copied host -> ring */
+    uint64_t bytes_h2d;                /* ring copy bytes */
+    uint64_t bytes_resident_read;      /* resident page bytes attended */
+    uint64_t h2d_copies;               /* cudaMemcpyAsync calls issued for the ring */
+    uint64_t kernel_launches;          /* kernels launched by the library */
+    /* filled when KVS_FLAG_PROFILE is set: summed CUDA-event durations, ms */
+    double ms_decode_resident, ms_decode_ring, ms_merge, ms_append, ms_chunk_mma;
+    uint64_t n_decode_resident, n_decode_ring, n_merge, n_append, n_chunk_mma;
+    uint64_t bytes_decode_resident, bytes_decode_ring; /* page bytes read by timed kernels */
+} kvs_stats;
+
+typedef struct kvs_s kvs_t;
+
+/* ---- pure host functions (no GPU needed) -------------------------------- */
+
+/* Validate `in` and fill `out` with every automatic field resolved
+ * (n_resident_pages, chunk_pages, arena_bytes = bytes actually needed).
+ * `host_bytes` (optional) receives the pinned history size.  The gates follow
+ * PR #326's configuration validation (type pair, single page byte size) and its
+ * minimum stage of one page ("Diagnostic log"). */
+int kvs_resolve_config(const kvs_config* in, kvs_config* out, size_t* host_bytes);
+
+/* Bytes of one page of one layer (all kv heads, K + V): 256 * n_kv * 1664/8. */
+size_t kvs_page_bytes(const kvs_config* cfg);
+
+/* Where page `page` of a layer holding n_tokens tokens lives: *kind is
+ * KVS_PAGE_RESIDENT (*index = resident slot = page mod R), KVS_PAGE_STREAMED
+ * (*index = streaming ordinal = page; pages 0..S-1 stream in ascending order)
+ * or KVS_PAGE_ABSENT.  The R most recent pages are resident. */
+int kvs_plan_page(const kvs_config* resolved, int n_tokens, int page, int* kind, int* index);
+
+/* ---- handle lifecycle ----------------------------------------------------- */
+
+/* Allocate the pinned host history (n_layers * pages(max_ctx) pages, mapped
+ * into the device address space) and the device arena on `device`, create the
+ * copy stream and ring events.  All-or-nothing: on failure nothing is leaked
+ * and *out is NULL. */
+int kvs_create(const kvs_config* cfg, int device, kvs_t** out);
+
+/* Wait (bounded by timeout_s, polling) for the library's copy stream and the
+ * given stream, then free everything.  NULL is a no-op. */
+void kvs_destroy(kvs_t* kv);
+
+/* ---- hot path ------------------------------------------------------------- */
+
+/* Quantize n_tok new K/V rows (fp16, layout [n_tok][n_kv_heads][head_dim]) of
+ * `layer` at positions pos0..pos0+n_tok-1: K -> Q8_0, V -> Q4_0.  The blocks
+ * are written to the host history and, for pages that are resident after the
+ * append, to their resident slot.  pos0 must be <= the layer's length (pos0 <
+ * length rolls the history back to pos0 first, as a rejected speculative draft
+ * does); pos0 + n_tok <= max_ctx; n_tok >= 1.  Device K/V may be of any width
+ * (history pre-fill); host K/V are staged and limited to max_q_tokens (else
+ * KVS_E_WIDTH).  Pages that re-enter the resident set on a roll-back are copied
+ * back from the host history on `stream`. */
+int kvs_append(kvs_t* kv, int layer, int pos0, int n_tok, const void* k_f16,
+               const void* v_f16, void* stream);
+
+/* Attention of n_q query tokens (fp16, [n_q][n_q_heads][head_dim]) at
+ * positions pos0..pos0+n_q-1 over the layer's quantized history: query j sees
+ * keys 0..pos0+j.  Needs pos0+n_q <= length and n_q <= max_q_tokens
+ * (KVS_E_WIDTH).  Writes out (fp32 [n_q][n_q_heads][head_dim]) and lse (fp32
+ * [n_q][n_q_heads], natural log of sum(exp(q.k/sqrt(head_dim)))); lse may be
+ * NULL.  Resident pages are attended in place; streamed pages are copied
+ * through the ring on the library's copy stream and attended as they land;
+ * per-split partials are merged by log-sum-exp. */
+int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float* out,
+               float* lse, void* stream);
+
+/* ---- diagnostics ---------------------------------------------------------- */
+
+/* Copy page `page` of `layer` to host_dst in canonical block layout:
+ * [256 tokens][n_kv_heads][head_dim/32] Q8_0 blocks of 34 bytes (fp16 d, 32 x
+ * int8), then [256][n_kv_heads][head_dim/32] Q4_0 blocks of 18 bytes (fp16 d,
+ * byte j = q_j | q_(j+16) << 4).  from_device = 0 reads the host history,
+ * 1 reads the resident slot (KVS_E_INVAL if the page is not resident).  The
+ * caller must have synchronized the streams that wrote the page. */
+int kvs_export_page(kvs_t* kv, int layer, int page, int from_device, void* host_dst);
+
+/* kvs_plan_page for the layer's current length. */
+int kvs_page_location(kvs_t* kv, int layer, int page, int* kind, int* index);
+
+/* Current length (tokens) of a layer's history. */
+int kvs_layer_length(kvs_t* kv, int layer, int* n_tokens);
+
+/* The resolved configuration of a handle. */
+int kvs_get_config(kvs_t* kv, kvs_config* out);
+
+/* Counters; with KVS_FLAG_PROFILE, first waits (bounded) for recorded events
+ * and folds their durations in.  kvs_reset_stats zeroes them. */
+int kvs_get_stats(kvs_t* kv, kvs_stats* out);
+int kvs_reset_stats(kvs_t* kv);
+
+/* Bounded host wait for all work the library enqueued (copy stream) and for
+ * `stream`: polls, returns KVS_E_TIMEOUT after timeout_s seconds. */
+int kvs_sync(kvs_t* kv, void* stream, double timeout_s);
+
+/* Measure pinned host->device copy bandwidth with `chunk_bytes` per
+ * cudaMemcpyAsync over `total_bytes` (best of `reps`), using the library's own
+ * copy stream and a scratch region of the device arena.  GB/s in *gbs. */
+int kvs_measure_h2d(kvs_t* kv, size_t chunk_bytes, size_t total_bytes, int reps, double* gbs);
+
+/* Last error text of the handle (or of the calling thread's last failed
+ * kvs_create / pure call when kv is NULL). */
+const char* kvs_last_error(kvs_t* kv);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVS_H */

@@ -1,0 +1,98 @@
+"""CPU checks of the C-ABI library: it loads, exports every symbol that
+include/kvs.h declares, and its pure host logic (config resolution, auto
+sizing, gates, page planning) agrees with the oracle and the pages."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from host_streamed_paged_kvs_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def kvs():
+    B.build()
+    from host_streamed_paged_kvs_b200 import kvs as K
+    return K
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "kvs.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvs_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(kvs):
+    names = declared_functions()
+    assert len(names) >= 15
+    lib = ctypes.CDLL(kvs.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), f"libkvs.so does not export {n}"
+    assert sorted(kvs.EXPORTS) == names
+
+
+def test_struct_sizes_match_header(kvs):
+    # 13 ints + size_t (padded) ; 8 u64 + 5 double + 7 u64
+    assert ctypes.sizeof(kvs.kvs_config) == 13 * 4 + 4 + 8
+    assert ctypes.sizeof(kvs.kvs_stats) == (8 + 5 + 7) * 8
+
+
+def test_auto_resident_matches_oracle_and_pages(kvs):
+    for ctx, L in [(262144, 16), (65536, 16), (4096, 1), (131072, 17), (1 << 24, 16), (20481, 1)]:
+        c = kvs.make_config(L, 40, 8, ctx, n_ring_slots=16)
+        r, host_bytes = kvs.kvs_resolve_config(c)
+        pb = kvs.kvs_page_bytes(r)
+        assert pb == 425984
+        want = min(oracle.auto_resident_pages(ctx, pb, L), oracle.pages_for(ctx))
+        assert r.n_resident_pages == want
+        assert host_bytes == L * oracle.pages_for(ctx) * pb
+    r, _ = kvs.kvs_resolve_config(kvs.make_config(16, 40, 8, 262144, n_ring_slots=16))
+    assert r.n_resident_pages == 103 and r.chunk_pages == 8
+
+
+def test_plan_page_matches_oracle(kvs):
+    for n_tokens, R in [(1, 4), (256, 4), (257, 4), (1025, 4), (32768, 64), (262144, 103), (5000, 1)]:
+        c = kvs.make_config(1, 8, 2, max(n_tokens, 1 << 20) if R < 1 << 12 else n_tokens,
+                            n_resident_pages=R, n_ring_slots=2)
+        r, _ = kvs.kvs_resolve_config(c)
+        P = oracle.pages_for(n_tokens)
+        for p in list(range(-1, min(P + 1, 300))) + [P - 1, P]:
+            assert kvs.kvs_plan_page(r, n_tokens, p) == oracle.page_location(n_tokens, R, p)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(type_k=2), -1), (dict(type_v=8), -1), (dict(head_dim=64), -1), (dict(page_tokens=128), -1),
+    (dict(n_q_heads=12, n_kv_heads=8), -1), (dict(n_ring_slots=0, n_resident_pages=4), -1),
+    (dict(n_ring_slots=6, chunk_pages=4), -1), (dict(arena_bytes=1000), -2),
+    (dict(arena_bytes=425984), -2), (dict(max_q_tokens=0), -1), (dict(n_layers=0), -1),
+])
+def test_gates(kvs, over, code):
+    args = dict(n_layers=2, n_q_heads=40, n_kv_heads=8, max_ctx=32768, n_resident_pages=8,
+                n_ring_slots=8, max_q_tokens=1)
+    args.update(over)
+    with pytest.raises(kvs.KvsError) as e:
+        kvs.kvs_resolve_config(kvs.make_config(**args))
+    assert e.value.code == code
+    assert kvs.kvs_last_error()
+
+
+def test_arena_fit_accepts_exact_size(kvs):
+    c = kvs.make_config(2, 40, 8, 32768, n_resident_pages=8, n_ring_slots=8)
+    r, _ = kvs.kvs_resolve_config(c)
+    c.arena_bytes = r.arena_bytes
+    r2, _ = kvs.kvs_resolve_config(c)
+    assert r2.arena_bytes == r.arena_bytes
+    assert r.arena_bytes >= (2 * 8 + 8) * 425984
+
+
+def test_create_without_gpu_fails_loudly(kvs):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(kvs.KvsError) as e:
+        kvs.kvs_create(kvs.make_config(1, 8, 2, 1024), 0)
+    assert e.value.code == kvs.KVS_E_CUDA

@@ -1,0 +1,68 @@
+"""Error paths of the C ABI on a GPU: every rejection is a status code, none
+faults the device, and the handle stays usable afterwards."""
+import numpy as np
+import pytest
+
+from host_streamed_paged_kvs_b200 import workload as W
+from kvs_testlib import oracle_step, assert_close, prefill, step, to_dev, torch
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kvs():
+    from host_streamed_paged_kvs_b200 import kvs as K
+    return K
+
+
+def test_width_order_and_recovery(kvs):
+    t = torch()
+    w = W.Workload("err", n_layers=1, n_q=1, n_q_heads=8, n_kv_heads=2, ctx=1000,
+                   n_resident_pages=2, n_ring_slots=2, seed=5)
+    cfg = kvs.make_config(1, 8, 2, 1000, n_resident_pages=2, n_ring_slots=2, max_q_tokens=4)
+    h = kvs.kvs_create(cfg, 0)
+    try:
+        prefill(h, w, 0, 999)
+        q = to_dev(W.queries(w, 0, 990, 8))
+        out = t.empty((8, 8, 128), dtype=t.float32, device="cuda")
+        with pytest.raises(kvs.KvsError) as e:
+            kvs.kvs_attend(h, 0, 990, 8, q, out)       # wider than max_q_tokens
+        assert e.value.code == kvs.KVS_E_WIDTH
+        with pytest.raises(kvs.KvsError) as e:
+            kvs.kvs_attend(h, 0, 998, 2, q, out)       # query 999 not appended yet
+        assert e.value.code == kvs.KVS_E_ORDER
+        k, v = W.kv_tokens(w, 0, 0, 1)
+        with pytest.raises(kvs.KvsError) as e:
+            kvs.kvs_append(h, 0, 1000, 1, to_dev(k), to_dev(v))  # gap after length 999
+        assert e.value.code == kvs.KVS_E_ORDER
+        with pytest.raises(kvs.KvsError) as e:
+            kvs.kvs_append(h, 0, 999, 2, to_dev(k), to_dev(v))   # beyond max_ctx
+        assert e.value.code == kvs.KVS_E_INVAL
+        with pytest.raises(kvs.KvsError) as e:
+            kvs.kvs_attend(h, 3, 0, 1, q, out)           # bad layer
+        assert e.value.code == kvs.KVS_E_INVAL
+        kh = t.from_numpy(np.zeros((8, 2, 128), np.float16)).pin_memory()
+        with pytest.raises(kvs.KvsError) as e:
+            kvs.kvs_append(h, 0, 999, 8, kh, kh)         # host K/V wider than the staging
+        assert e.value.code == kvs.KVS_E_WIDTH
+        # still usable
+        out1, lse1 = step(h, w, 0, 999, 1)
+        ref = oracle_step(w, 0, 999, 1)
+        assert_close(out1, lse1, *ref)
+        kvs.kvs_sync(h, None, 30.0)
+    finally:
+        kvs.kvs_destroy(h)
+
+
+def test_create_rejections(kvs):
+    bad_pair = kvs.make_config(1, 8, 2, 1000, n_ring_slots=2, type_v=kvs.KVS_TYPE_Q8_0)
+    with pytest.raises(kvs.KvsError) as e:
+        kvs.kvs_create(bad_pair, 0)
+    assert e.value.code == kvs.KVS_E_INVAL
+    tiny_arena = kvs.make_config(1, 8, 2, 1000, n_ring_slots=2, arena_bytes=4096)
+    with pytest.raises(kvs.KvsError) as e:
+        kvs.kvs_create(tiny_arena, 0)
+    assert e.value.code == kvs.KVS_E_ARENA
+    with pytest.raises(kvs.KvsError) as e:
+        kvs.kvs_create(kvs.make_config(1, 8, 2, 1000), 99)
+    assert e.value.code == kvs.KVS_E_INVAL
