@@ -1,0 +1,392 @@
+"""Benchmark: streamed decode-attention KV tokens/s/layer on B200, and its
+fraction of the max(resident bytes / HBM BW, streamed bytes / H2D BW) roofline.
+
+One step = one pass of the whole path over every layer of the workload:
+quantize-on-append of the step's tokens (rolled back to the same position each
+step, the steady state of a decode loop) and attention over the full history
+(resident pages in place, older pages streamed from pinned host memory through
+the copy-engine ring, split partials merged by log-sum-exp).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints one JSON line (rank 0).  With N > 1 (torchrun) every rank runs an
+independent replica on its own GPU ("replicas only": the path has no exchange
+step); value = all ranks' tokens / the slowest rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from host_streamed_paged_kvs_b200 import workload as W  # noqa: E402
+
+METRIC = "streamed decode-attn KV tokens/s/layer; % of max(HBM,H2D) roofline, 1xB200"
+UNIT = "KV tokens/s/layer"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.f = None
+
+    def start(self):
+        try:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        self.f.close()
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = max(mx, float(r[2]))
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (CPU baseline / reference arm)
+# ---------------------------------------------------------------------------
+def oracle_layer_step(w: W.Workload, layer: int = 0, prepared=None):
+    """Time the oracle on one layer's step of the workload: quantize the step's
+    tokens and attend over the whole history.  Returns (seconds, prepared)."""
+    import oracle
+    if prepared is None:
+        k, v = W.kv_tokens(w, layer, 0, w.pos0)
+        kb, vb = oracle.quantize_rows(k, v)
+        ks, vs = W.kv_tokens(w, layer, w.pos0, w.ctx)
+        q = W.queries(w, layer, w.pos0)
+        prepared = (kb, vb, ks, vs, q)
+    kb, vb, ks, vs, q = prepared
+    t0 = time.perf_counter()
+    kbs, vbs = oracle.quantize_rows(ks, vs)
+    kall = np.concatenate([kb, kbs])
+    vall = np.concatenate([vb, vbs])
+    oracle.attention(kall, vall, q, w.pos0)
+    return time.perf_counter() - t0, prepared
+
+
+def cpu_baseline(w: W.Workload, budget_s: float = 15.0):
+    secs, prep = oracle_layer_step(w)
+    times = [secs]
+    while sum(times) < budget_s and len(times) < 8:
+        t, _ = oracle_layer_step(w, prepared=prep)
+        times.append(t)
+    per_layer = statistics.median(times)
+    return {"value": w.ctx / per_layer, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{len(times)} x one layer's step of {w.name} (append {w.n_q} token(s), "
+                      f"binary64 attention of {w.n_q}x{w.n_q_heads} query rows over {w.ctx} keys), "
+                      f"single thread, median {per_layer:.2f} s"}
+
+
+def run_reference(args, w: W.Workload):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    times = []
+    _, prep = oracle_layer_step(w)
+    for i in range(args.warmup + args.steps):
+        t, _ = oracle_layer_step(w, prepared=prep)
+        if i >= args.warmup:
+            times.append(t)
+    per = statistics.median(times)
+    value = w.ctx / per
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "ctx": w.ctx, "n_layers_timed": 1,
+                       "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "n_q": w.n_q},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"each step = one layer's step of {w.name} on the CPU oracle "
+                                       f"(single thread)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+def run_gpu(args, w: W.Workload):
+    import torch
+    import torch.distributed as dist
+    from host_streamed_paged_kvs_b200 import kvs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600))
+    dev = torch.device("cuda", local)
+
+    L = w.n_layers
+    cfg = kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx, n_resident_pages=w.n_resident_pages,
+                          n_ring_slots=w.n_ring_slots, max_q_tokens=w.n_q,
+                          chunk_pages=args.chunk_pages)
+    h = kvs.kvs_create(cfg, local)
+    rc = kvs.kvs_get_config(h)
+    pb = kvs.kvs_page_bytes(rc)
+    stream = torch.cuda.Stream(device=dev)
+
+    # ---- history pre-fill (untimed) ----
+    t0 = time.time()
+    for layer in range(L):
+        pos = 0
+        while pos < w.pos0:
+            n = min(16384, w.pos0 - pos)
+            k, v = W.kv_tokens(w, layer, pos, pos + n)
+            kd = torch.from_numpy(k).to(dev)
+            vd = torch.from_numpy(v).to(dev)
+            with torch.cuda.stream(stream):
+                kvs.kvs_append(h, layer, pos, n, kd, vd, stream)
+            stream.synchronize()
+            pos += n
+    prefill_s = time.time() - t0
+
+    # ---- per-step inputs resident in HBM ----
+    ks, vs, qs = [], [], []
+    for layer in range(L):
+        k, v = W.kv_tokens(w, layer, w.pos0, w.ctx)
+        ks.append(torch.from_numpy(k).to(dev))
+        vs.append(torch.from_numpy(v).to(dev))
+        qs.append(torch.from_numpy(W.queries(w, layer, w.pos0)).to(dev))
+    out = torch.empty((L, w.n_q, w.n_q_heads, 128), dtype=torch.float32, device=dev)
+    lse = torch.empty((L, w.n_q, w.n_q_heads), dtype=torch.float32, device=dev)
+
+    def one_step(k_in, v_in, q_in, o, l):
+        for layer in range(L):
+            kvs.kvs_append(h, layer, w.pos0, w.n_q, k_in[layer], v_in[layer], stream)
+            kvs.kvs_attend(h, layer, w.pos0, w.n_q, q_in[layer], o[layer], l[layer], stream)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        one_step(ks, vs, qs, out, lse)
+    barrier()
+    kvs.kvs_reset_stats(h)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.25)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        one_step(ks, vs, qs, out, lse)
+    e1.record(stream)
+    barrier()
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    clk = clocks.stop()
+    st = kvs.kvs_get_stats(h)
+    ms_step = ms_total / args.steps
+    value = world * w.ctx * L / (ms_step * 1e-3)
+
+    # ---- end to end through the C ABI with pinned host buffers ----
+    kh = [x.cpu().pin_memory() for x in ks]
+    vh = [x.cpu().pin_memory() for x in vs]
+    qh = [x.cpu().pin_memory() for x in qs]
+    oh = torch.empty(tuple(out.shape), dtype=torch.float32).pin_memory()
+    lh = torch.empty(tuple(lse.shape), dtype=torch.float32).pin_memory()
+    for _ in range(max(1, args.warmup // 2)):
+        one_step(kh, vh, qh, oh, lh)
+    barrier()
+    e0.record(stream)
+    e2e_steps = max(1, args.steps // 2)
+    for _ in range(e2e_steps):
+        one_step(kh, vh, qh, oh, lh)
+    e1.record(stream)
+    barrier()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+    h2d_b = sum(x.numel() * x.element_size() for x in kh + vh + qh)
+    d2h_b = oh.numel() * 4 + lh.numel() * 4
+
+    # ---- kernel timing: the same steps again, with CUDA events around every
+    #      launch of the library's kernels (a separate timed pass, so the
+    #      events' host cost does not enter the step time above) ----
+    st_prof = None
+    if args.profile:
+        kvs.kvs_set_profiling(h, True)
+        one_step(ks, vs, qs, out, lse)
+        barrier()
+        kvs.kvs_reset_stats(h)
+        for _ in range(min(args.steps, 60)):
+            one_step(ks, vs, qs, out, lse)
+        barrier()
+        st_prof = kvs.kvs_get_stats(h)
+        kvs.kvs_set_profiling(h, False)
+
+    # ---- copy bandwidth of this machine (roofline denominator) ----
+    chunk_b = rc.chunk_pages * pb if rc.chunk_pages else pb
+    h2d_ring = kvs.kvs_measure_h2d(h, chunk_b, min(1 << 30, L * rc.n_resident_pages * pb), 10) \
+        if rc.n_ring_slots else None
+    big = torch.empty(1 << 30, dtype=torch.uint8).pin_memory()
+    dbig = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    best = 0.0
+    cs = torch.cuda.Stream(device=dev)
+    for _ in range(10):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(cs)
+        with torch.cuda.stream(cs):
+            for i in range(16):
+                dbig[i << 26:(i + 1) << 26].copy_(big[i << 26:(i + 1) << 26], non_blocking=True)
+        b.record(cs)
+        cs.synchronize()
+        best = max(best, (1 << 30) / (a.elapsed_time(b) * 1e-3) / 1e9)
+    h2d_peak = max(best, h2d_ring or 0.0)
+    del big, dbig
+
+    hbm_peak, peak_src = peaks()
+    P = w.n_pages
+    R = min(rc.n_resident_pages, P)
+    S = P - R
+    t_roof = L * max(R * pb / (hbm_peak * 1e9), S * pb / (h2d_peak * 1e9))
+    roof_frac = t_roof / (ms_step * 1e-3)
+
+    # dominant kernel: the split-K decode kernel (resident + ring launches)
+    kernel = None
+    if st_prof and st_prof["n_decode_resident"] + st_prof["n_decode_ring"] > 0:
+        st = dict(st, **{k: v for k, v in st_prof.items() if k.startswith(("ms_", "n_", "bytes_decode"))})
+        n_launch = st["n_decode_resident"] + st["n_decode_ring"]
+        ms_k = st["ms_decode_resident"] + st["ms_decode_ring"]
+        bytes_k = st["bytes_decode_resident"] + st["bytes_decode_ring"]
+        achieved = bytes_k / (ms_k * 1e-3) / 1e9
+        kernel = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                  "frac": achieved / hbm_peak, "traffic": None, "kernel": "decode_kernel",
+                  "launches": n_launch, "avg_launch_us": ms_k / n_launch * 1e3,
+                  "bytes_per_launch": bytes_k / n_launch, "peak_source": peak_src,
+                  "timing": "CUDA events around each launch on its stream, separate pass of the same steps",
+                  "other_kernels_avg_us": {
+                      "merge": st["ms_merge"] / max(1, st["n_merge"]) * 1e3,
+                      "append": st["ms_append"] / max(1, st["n_append"]) * 1e3},
+                  "resident_only": {
+                      "achieved": st["bytes_decode_resident"] / max(st["ms_decode_resident"], 1e-9) / 1e6,
+                      "launches": st["n_decode_resident"],
+                      "avg_launch_us": st["ms_decode_resident"] / max(1, st["n_decode_resident"]) * 1e3}}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "ctx": w.ctx, "n_layers": L, "n_q": w.n_q,
+                   "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": 128,
+                   "kv_types": "K q8_0 / V q4_0", "page_tokens": 256, "resident_pages": R,
+                   "streamed_pages": S, "ring_slots": rc.n_ring_slots, "chunk_pages": rc.chunk_pages,
+                   "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (resident "
+                   f"{L * R * pb / 1e6:.0f} MB + streamed {L * S * pb / 1e6:.0f} MB per step)",
+                   },
+        "roofline": kernel,
+        "step_roofline": {"bound": "h2d" if S * pb / h2d_peak > R * pb / hbm_peak else "hbm",
+                          "t_roof_ms": t_roof * 1e3, "t_step_ms": ms_step, "frac": roof_frac,
+                          "h2d_gbs_peak_measured": h2d_peak, "h2d_gbs_ring_chunk": h2d_ring,
+                          "h2d_gbs_achieved": L * S * pb / (ms_step * 1e-3) / 1e9,
+                          "hbm_gbs_peak": hbm_peak, "peak_source": peak_src},
+        "e2e": {"value": world * w.ctx * L / (ms_e2e * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b, "ms_per_step": ms_e2e},
+        "gpu_launches": int(st["kernel_launches"]),
+        "clocks": clk,
+        "prefill_s": prefill_s,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    kvs.kvs_destroy(h)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=0)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=W.DEFAULT_BENCH, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--chunk-pages", type=int, default=0)
+    ap.add_argument("--no-profile", dest="profile", action="store_false")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = W.WORKLOADS[args.workload]
+    if args.steps <= 0:
+        # a timed region of a few seconds
+        args.steps = {"tiny_decode_4k": 2000, "streamed_decode_32k": 300, "long_decode_256k": 30,
+                      "verify_128k": 60, "prefill_chunk_64k": 200}[w.name]
+        if args.impl == "reference":
+            args.steps = 5
+    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

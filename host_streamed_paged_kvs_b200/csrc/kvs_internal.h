@@ -59,8 +59,8 @@ struct DecodeArgs {
     int region_slots;        // slots in the region (R or N)
     int slot0;               // region slot of unit 0
     int page0;               // absolute page index of unit 0
-    int n_units;             // pages in this launch
-    int pages_per_split;
+    int n_units;             // pages in this launch (consumed as 2 half-page stages each)
+    int stages_per_split;    // half-page stages per split
     int split_base;          // first split index written by this launch
     int len;                 // tokens in the history
     int pos0, n_q;           // query positions pos0 .. pos0+n_q-1

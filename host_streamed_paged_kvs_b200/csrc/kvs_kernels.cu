@@ -186,54 +186,63 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
 }
 
 // ----------------------------------------------------------------------------
-// K2: split-K flash-decode.  CTA = (split, kv head, row group), 128 threads.
-// A split is a run of pages; each page is consumed as two 128-token stages.
-// Stage bytes land in shared memory through TMA: the K quants with the
-// 128-byte swizzle (so a thread per key reads its row without bank conflicts
-// while the query chunk is a broadcast), the K scales, V codes and V scales as
-// 1-D bulk copies.  QK^T: thread = key, all rows of the GQA group.  Softmax:
-// online, log2 domain, CTA-wide max per stage.  PV: warp = 32 keys, lane = 4
-// dims.  Output per split: (m, l) and acc[128] for every query row.
+// K2: split-K flash-decode.  CTA = (split, kv head, row group), 256 threads.
+// The pages of one launch are consumed as 128-token half-page stages; a split
+// is a run of `stages_per_split` consecutive stages.  Stage bytes land in
+// shared memory through TMA: the K quants with the 128-byte swizzle (a thread
+// reading its key's row then hits distinct banks while the query chunk it
+// multiplies is a broadcast), the K scales, V codes and V scales as 1-D bulk
+// copies; three stages are in flight.
+//   QK^T : two threads per key, 64 dims each; K dequantized in registers
+//          (exact int8 -> fp32), per-block scale applied to the block's partial.
+//   softmax: online, log2 domain, CTA-wide running max per row; the V scale of
+//          each (key, block) is folded into the probability, p' = p * d_v.
+//   PV   : warp = 16 keys, lane = 4 dims x all rows.
+// Output per split: (m, l) and acc[128] for every query row of the CTA.
 // ----------------------------------------------------------------------------
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
 constexpr int kStageKeys = 128;
 constexpr int kStageKq = 0;
-constexpr int kStageKd = kStageKeys * kHeadDim;            // 16384
-constexpr int kStageVq = kStageKd + kStageKeys * kBlocks * 2;  // 17408
-constexpr int kStageVd = kStageVq + kStageKeys * kHeadDim / 2;  // 25600
-constexpr int kStageBytes = kStageVd + kStageKeys * kBlocks * 2;  // 26624
+constexpr int kStageKd = kStageKeys * kHeadDim;                  // 16384
+constexpr int kStageVq = kStageKd + kStageKeys * kBlocks * 2;      // 17408
+constexpr int kStageVd = kStageVq + kStageKeys * kHeadDim / 2;     // 25600
+constexpr int kStageBytes = kStageVd + kStageKeys * kBlocks * 2;   // 26624
 constexpr int kStages = 3;
 constexpr int kMaxRows = 8;
-constexpr size_t kDecodeSmem = 1024 /*align slack*/ + kStages * kStageBytes +
-                               kMaxRows * kHeadDim * 4 /*sQ*/ + kStageKeys * kMaxRows * 4 /*sP*/ +
-                               4 * kMaxRows * 4 /*sMax*/ + 4 * kMaxRows * 4 /*sL*/ + kStages * 8;
-static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-B swizzle alignment");
-static_assert(4 * kMaxRows * kHeadDim * 4 <= kStages * kStageBytes, "reduction scratch fits");
+constexpr int kQHalf = 68;                  // floats per (row, half): 64 + 4 pad (bank offset)
+constexpr size_t kOffQ = kStages * kStageBytes;
+constexpr size_t kOffP = kOffQ + kMaxRows * 2 * kQHalf * 4;                 // sQ
+constexpr size_t kOffMax = kOffP + kStageKeys * kBlocks * kMaxRows * 4;     // sP
+constexpr size_t kOffL = kOffMax + kWarps * kMaxRows * 4;
+constexpr size_t kOffBar = kOffL + kWarps * kMaxRows * 4;
+constexpr size_t kDecodeSmem = 1024 /*align slack*/ + kOffBar + kStages * 8;
+static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-B swizzle alignment");
+static_assert(kWarps * kMaxRows * kHeadDim * 4 <= kStages * kStageBytes, "reduction scratch fits");
 
 size_t decode_smem_bytes() { return kDecodeSmem; }
 
 template <int ROWS>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap) {
+    constexpr int PR = ROWS <= 4 ? 4 : 8;  // padded rows of a p' record
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* stage = smem;
-    float* sQ = reinterpret_cast<float*>(smem + kStages * kStageBytes);  // [ROWS][128]
-    float* sP = sQ + kMaxRows * kHeadDim;                              // [128 keys][8]
-    float* sMax = sP + kStageKeys * kMaxRows;                          // [4 warps][8]
-    float* sL = sMax + 4 * kMaxRows;                                   // [4 warps][8]
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sL + 4 * kMaxRows);    // [kStages]
+    float* sQ = reinterpret_cast<float*>(smem + kOffQ);    // [ROWS][2][kQHalf]
+    float* sP = reinterpret_cast<float*>(smem + kOffP);    // [128 keys][4 blocks][PR]
+    float* sMax = reinterpret_cast<float*>(smem + kOffMax);  // [warps][8]
+    float* sL = reinterpret_cast<float*>(smem + kOffL);      // [warps][8]
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.y;
-    const int split = blockIdx.x;
     const int row_begin = blockIdx.z * ROWS;
-    const int n_local_rows = a.n_q * a.group;
-    const int rows_here = min(ROWS, n_local_rows - row_begin);
-    const int u0 = split * a.pages_per_split;
-    const int u1 = min(a.n_units, u0 + a.pages_per_split);
-    const int n_st = 2 * (u1 - u0);
+    const int rows_here = min(ROWS, a.n_q * a.group - row_begin);
+    const int n_stages_all = 2 * a.n_units;
+    const int st0 = blockIdx.x * a.stages_per_split;
+    const int n_st = min(a.stages_per_split, n_stages_all - st0);
 
     // queries of this CTA's rows, pre-scaled into the log2 domain
     for (int idx = tid; idx < ROWS * kHeadDim; idx += kThreads) {
@@ -242,15 +251,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (r < rows_here) {
             const int lr = row_begin + r;
             const int j = lr / a.group, g = lr - j * a.group;
-            v = __half2float(a.q[((size_t)j * a.n_qh + h * a.group + g) * kHeadDim + d]) *
-                a.q_scale;
+            v = __half2float(a.q[((size_t)j * a.n_qh + h * a.group + g) * kHeadDim + d]) * a.q_scale;
         }
-        sQ[idx] = v;
+        sQ[(r * 2 + (d >> 6)) * kQHalf + (d & 63)] = v;
     }
     int qpos[ROWS];
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r)
-        qpos[r] = (r < rows_here) ? a.pos0 + (row_begin + r) / a.group : -1;
+    for (int r = 0; r < ROWS; ++r) qpos[r] = (r < rows_here) ? a.pos0 + (row_begin + r) / a.group : -1;
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&bar[s], 1);
@@ -258,12 +265,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     __syncthreads();
 
-    auto issue = [&](int st) {
-        const int u = u0 + (st >> 1), half = st & 1;
+    auto issue = [&](int i) {  // i: stage index within this split
+        const int sg = st0 + i;
+        const int u = sg >> 1, half = sg & 1;
         const int slot = (a.slot0 + u) % a.region_slots;
         const uint8_t* ph = a.region + ((size_t)slot * a.n_kv + h) * kPageHeadBytes;
-        uint8_t* dst = stage + (st % kStages) * kStageBytes;
-        uint64_t* b = &bar[st % kStages];
+        uint8_t* dst = stage + (i % kStages) * kStageBytes;
+        uint64_t* b = &bar[i % kStages];
         mbar_expect_tx(b, kStageBytes);
         const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * kPageHeadRows + half * kStageKeys;
         tma_load_2d(dst + kStageKq, &kmap, 0, krow, b);
@@ -272,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         bulk_load(dst + kStageVd, ph + kOffVd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
     };
     if (tid == 0) {
-        for (int st = 0; st < kStages && st < n_st; ++st) issue(st);
+        for (int i = 0; i < kStages && i < n_st; ++i) issue(i);
     }
 
     float m_run[ROWS], l_run[ROWS], acc[ROWS][4];
@@ -282,34 +290,33 @@ __global__ void __launch_bounds__(kThreads, 2)
         l_run[r] = 0.0f;
         acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.0f;
     }
-    const int vb = lane >> 3, vi = lane & 7;  // PV: block and byte pair of this lane
+    const int key = tid >> 1, hf = tid & 1;   // QK / softmax role
+    const int vb = lane >> 3, vi = lane & 7;  // PV role: block and byte pair of this lane
     bool ok = true;
 
-    for (int st = 0; st < n_st; ++st) {
-        uint8_t* sb = stage + (st % kStages) * kStageBytes;
-        if (!mbar_wait_bounded(&bar[st % kStages], (st / kStages) & 1, a.err)) {
-            ok = false;
-        }
+    for (int i = 0; i < n_st; ++i) {
+        const uint8_t* sb = stage + (i % kStages) * kStageBytes;
+        if (!mbar_wait_bounded(&bar[i % kStages], (i / kStages) & 1, a.err)) ok = false;
         ok = __syncthreads_and(ok);
         if (!ok) break;
-        const int u = u0 + (st >> 1), half = st & 1;
-        const int kpos0 = (a.page0 + u) * kPageTokens + half * kStageKeys;
+        const int sg = st0 + i;
+        const int kpos = (a.page0 + (sg >> 1)) * kPageTokens + (sg & 1) * kStageKeys + key;
 
-        // ---- QK^T: thread = key ----
-        const int key = tid;
-        const int kpos = kpos0 + key;
+        // ---- QK^T: this thread's key, dims [64 hf, 64 hf + 64) ----
         float s[ROWS];
 #pragma unroll
         for (int r = 0; r < ROWS; ++r) s[r] = 0.0f;
         const uint8_t* krow = sb + kStageKq + key * kHeadDim;
+        const float* qh = sQ + hf * kQHalf;
 #pragma unroll
-        for (int blk = 0; blk < kBlocks; ++blk) {
+        for (int bb = 0; bb < 2; ++bb) {
+            const int blk = 2 * hf + bb;
             float part[ROWS];
 #pragma unroll
             for (int r = 0; r < ROWS; ++r) part[r] = 0.0f;
 #pragma unroll
             for (int c2 = 0; c2 < 2; ++c2) {
-                const int c = blk * 2 + c2;
+                const int c = 2 * blk + c2;  // logical 16-byte chunk of the row
                 const uint4 raw = *reinterpret_cast<const uint4*>(krow + ((c ^ (key & 7)) << 4));
                 const uint32_t w[4] = {raw.x ^ 0x80808080u, raw.y ^ 0x80808080u,
                                        raw.z ^ 0x80808080u, raw.w ^ 0x80808080u};
@@ -317,10 +324,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int uu = 0; uu < 4; ++uu) {
                     const float k0 = s8_to_f(w[uu], 0), k1 = s8_to_f(w[uu], 1);
                     const float k2 = s8_to_f(w[uu], 2), k3 = s8_to_f(w[uu], 3);
+                    const int qo = (c - 4 * hf) * 16 + uu * 4;
 #pragma unroll
                     for (int r = 0; r < ROWS; ++r) {
-                        const float4 qv =
-                            *reinterpret_cast<const float4*>(sQ + r * kHeadDim + c * 16 + uu * 4);
+                        const float4 qv = *reinterpret_cast<const float4*>(qh + r * 2 * kQHalf + qo);
                         part[r] = fmaf(qv.x, k0, part[r]);
                         part[r] = fmaf(qv.y, k1, part[r]);
                         part[r] = fmaf(qv.z, k2, part[r]);
@@ -335,98 +342,107 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
 #pragma unroll
         for (int r = 0; r < ROWS; ++r) {
+            s[r] += __shfl_xor_sync(0xffffffffu, s[r], 1);
             if (kpos >= a.len || kpos > qpos[r]) s[r] = -CUDART_INF_F;
             float mx = s[r];
 #pragma unroll
-            for (int off = 16; off >= 1; off >>= 1)
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            for (int off = 2; off <= 16; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
             if (lane == 0) sMax[warp * kMaxRows + r] = mx;
         }
         __syncthreads();
         // the previous stage's buffer is free once every thread has passed this barrier
-        if (tid == 0 && st >= 1 && st - 1 + kStages < n_st) issue(st - 1 + kStages);
+        if (tid == 0 && i >= 1 && i - 1 + kStages < n_st) issue(i - 1 + kStages);
 
+        // ---- online softmax; p' = p * d_v for this thread's two blocks ----
         float alpha[ROWS];
+        const __half2 dv2 = *reinterpret_cast<const __half2*>(sb + kStageVd + key * (kBlocks * 2) + hf * 4);
+        const float dva = __low2float(dv2), dvb = __high2float(dv2);
+        float* pdst = sP + (key * kBlocks + 2 * hf) * PR;
 #pragma unroll
         for (int r = 0; r < ROWS; ++r) {
-            const float mx = fmaxf(fmaxf(sMax[r], sMax[kMaxRows + r]),
-                                   fmaxf(sMax[2 * kMaxRows + r], sMax[3 * kMaxRows + r]));
+            float mx = sMax[r];
+#pragma unroll
+            for (int ww = 1; ww < kWarps; ++ww) mx = fmaxf(mx, sMax[ww * kMaxRows + r]);
             const float mn = fmaxf(m_run[r], mx);
             const float mu = (mn == -CUDART_INF_F) ? 0.0f : mn;
             alpha[r] = exp2f(m_run[r] - mu);
             m_run[r] = mn;
-            sP[key * kMaxRows + r] = exp2f(s[r] - mu);
+            const float p = exp2f(s[r] - mu);
+            pdst[r] = p * dva;
+            pdst[PR + r] = p * dvb;
+            float ps = hf ? 0.0f : p;
+#pragma unroll
+            for (int off = 2; off <= 16; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+            if (lane == 0) sL[warp * kMaxRows + r] = ps;
         }
         __syncthreads();
 
-        // ---- PV: warp = 32 keys, lane = dims {32b+2i, +1, +16, +17} ----
+        // ---- PV: warp = 16 keys, lane = dims {32b+2i, +1, +16, +17} ----
 #pragma unroll
         for (int r = 0; r < ROWS; ++r) {
-            l_run[r] *= alpha[r];
+            float ls = 0.0f;
+#pragma unroll
+            for (int ww = 0; ww < kWarps; ++ww) ls += sL[ww * kMaxRows + r];
+            l_run[r] = fmaf(l_run[r], alpha[r], ls);
             acc[r][0] *= alpha[r]; acc[r][1] *= alpha[r];
             acc[r][2] *= alpha[r]; acc[r][3] *= alpha[r];
         }
         const uint8_t* vq_base = sb + kStageVq + vb * 16 + 2 * vi;
-        const uint8_t* vd_base = sb + kStageVd + vb * 2;
+        const float* p_base = sP + vb * PR;
 #pragma unroll 4
-        for (int kk = 0; kk < 32; ++kk) {
-            const int key2 = warp * 32 + kk;
+        for (int kk = 0; kk < 16; ++kk) {
+            const int key2 = warp * 16 + kk;
             const uint32_t code = *reinterpret_cast<const uint16_t*>(vq_base + key2 * 64);
-            const float dv = __half2float(*reinterpret_cast<const __half*>(vd_base + key2 * 8));
-            const float v0 = q4_to_f(code & 0xFu) * dv;          // dim 32b+2i
-            const float v2 = q4_to_f((code >> 4) & 0xFu) * dv;   // dim 32b+2i+16
-            const float v1 = q4_to_f((code >> 8) & 0xFu) * dv;   // dim 32b+2i+1
-            const float v3 = q4_to_f((code >> 12) & 0xFu) * dv;  // dim 32b+2i+17
-            const float* pr = sP + key2 * kMaxRows;
+            const float v0 = q4_to_f(code & 0xFu);          // dim 32b+2i
+            const float v2 = q4_to_f((code >> 4) & 0xFu);   // dim 32b+2i+16
+            const float v1 = q4_to_f((code >> 8) & 0xFu);   // dim 32b+2i+1
+            const float v3 = q4_to_f((code >> 12) & 0xFu);  // dim 32b+2i+17
+            const float* pr = p_base + key2 * kBlocks * PR;
+            float pv[PR];
+            *reinterpret_cast<float4*>(pv) = *reinterpret_cast<const float4*>(pr);
+            if (PR == 8) *reinterpret_cast<float4*>(pv + 4) = *reinterpret_cast<const float4*>(pr + 4);
 #pragma unroll
             for (int r = 0; r < ROWS; ++r) {
-                const float p = pr[r];
-                l_run[r] += p;
-                acc[r][0] = fmaf(p, v0, acc[r][0]);
-                acc[r][1] = fmaf(p, v1, acc[r][1]);
-                acc[r][2] = fmaf(p, v2, acc[r][2]);
-                acc[r][3] = fmaf(p, v3, acc[r][3]);
+                acc[r][0] = fmaf(pv[r], v0, acc[r][0]);
+                acc[r][1] = fmaf(pv[r], v1, acc[r][1]);
+                acc[r][2] = fmaf(pv[r], v2, acc[r][2]);
+                acc[r][3] = fmaf(pv[r], v3, acc[r][3]);
             }
         }
     }
     if (!ok) return;  // a bounded wait gave up; the error word is set
 
-    // ---- reduce the four warps' partials and write the split's result ----
+    // ---- reduce the warps' partial sums and write the split's result ----
     __syncthreads();  // stage buffers are reused as scratch
-    float* red = reinterpret_cast<float*>(stage);  // [4 warps][ROWS][128]
+    float* red = reinterpret_cast<float*>(stage);  // [warps][ROWS][128]
     const int d0 = vb * 32 + 2 * vi;
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
         float* dst = red + (warp * ROWS + r) * kHeadDim;
-        dst[d0] = acc[r][0];
-        dst[d0 + 1] = acc[r][1];
-        dst[d0 + 16] = acc[r][2];
-        dst[d0 + 17] = acc[r][3];
-        if (lane == 0) sL[warp * kMaxRows + r] = l_run[r];
+        *reinterpret_cast<float2*>(dst + d0) = make_float2(acc[r][0], acc[r][1]);
+        *reinterpret_cast<float2*>(dst + d0 + 16) = make_float2(acc[r][2], acc[r][3]);
     }
     __syncthreads();
-    const int split_g = a.split_base + split;
+    const int split_g = a.split_base + blockIdx.x;
     for (int idx = tid; idx < rows_here * kHeadDim; idx += kThreads) {
         const int r = idx / kHeadDim, d = idx - r * kHeadDim;
-        const float v = red[(0 * ROWS + r) * kHeadDim + d] + red[(1 * ROWS + r) * kHeadDim + d] +
-                        red[(2 * ROWS + r) * kHeadDim + d] + red[(3 * ROWS + r) * kHeadDim + d];
+        float v = 0.0f;
+#pragma unroll
+        for (int ww = 0; ww < kWarps; ++ww) v += red[(ww * ROWS + r) * kHeadDim + d];
         const int lr = row_begin + r;
         const int j = lr / a.group, g = lr - j * a.group;
         const int grow = j * a.n_qh + h * a.group + g;
         a.part.acc[((size_t)split_g * a.n_rows + grow) * kHeadDim + d] = v;
     }
-    if (tid < rows_here) {
-        const int r = tid;
-        const int lr = row_begin + r;
-        const int j = lr / a.group, g = lr - j * a.group;
-        const int grow = j * a.n_qh + h * a.group + g;
-        const float l = sL[r] + sL[kMaxRows + r] + sL[2 * kMaxRows + r] + sL[3 * kMaxRows + r];
-        float mr = -CUDART_INF_F;
-        // m_run is identical in every thread; pick row r's value without dynamic indexing
+    if (tid < ROWS && tid < rows_here) {
+        float mr = 0.0f, lr_ = 0.0f;
 #pragma unroll
         for (int rr = 0; rr < ROWS; ++rr)
-            if (rr == r) mr = m_run[rr];
-        a.part.ml[(size_t)split_g * a.n_rows + grow] = make_float2(mr, l);
+            if (rr == tid) { mr = m_run[rr]; lr_ = l_run[rr]; }
+        const int lrow = row_begin + tid;
+        const int j = lrow / a.group, g = lrow - j * a.group;
+        const int grow = j * a.n_qh + h * a.group + g;
+        a.part.ml[(size_t)split_g * a.n_rows + grow] = make_float2(mr, lr_);
     }
 }
 
@@ -465,48 +481,74 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, int n_sp
 }
 
 // ----------------------------------------------------------------------------
-// K3: log-sum-exp merge.  One CTA per query row: M = max_s m_s,
+// K3: log-sum-exp merge.  CTA = (query row, 32-dim slice): M = max_s m_s,
 // L = sum_s 2^(m_s-M) l_s, O = sum_s 2^(m_s-M) acc_s / L, lse = ln2 (M + log2 L).
+// Warps stride over the splits with four independent loads in flight each.
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) merge_kernel(const MergeArgs a) {
-    __shared__ float sm[4];
-    __shared__ float sacc[4][kHeadDim];
-    __shared__ float sl[4];
+constexpr int kMergeThreads = 256;
+
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const MergeArgs a) {
+    __shared__ float sm[kMergeThreads / 32];
+    __shared__ float sacc[kMergeThreads / 32][32];
+    __shared__ float sl[kMergeThreads / 32];
     const int row = blockIdx.x;
+    const int slice = blockIdx.y;  // dims [32 slice, 32 slice + 32)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int W = kMergeThreads / 32;
+    const float2* ml = a.part.ml + row;
     float m = -CUDART_INF_F;
-    for (int s = tid; s < a.n_splits; s += 128) m = fmaxf(m, a.part.ml[(size_t)s * a.n_rows + row].x);
+    for (int s = tid; s < a.n_splits; s += kMergeThreads) m = fmaxf(m, ml[(size_t)s * a.n_rows].x);
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     if (lane == 0) sm[warp] = m;
     __syncthreads();
-    const float M = fmaxf(fmaxf(sm[0], sm[1]), fmaxf(sm[2], sm[3]));
-    float L = 0.0f;
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = warp; s < a.n_splits; s += 4) {
-        const float2 ml = a.part.ml[(size_t)s * a.n_rows + row];
-        if (ml.y > 0.0f) {
-            const float w = exp2f(ml.x - M);
-            L = fmaf(w, ml.y, L);
-            const float4 v = *reinterpret_cast<const float4*>(
-                a.part.acc + ((size_t)s * a.n_rows + row) * kHeadDim + 4 * lane);
-            o.x = fmaf(w, v.x, o.x); o.y = fmaf(w, v.y, o.y);
-            o.z = fmaf(w, v.z, o.z); o.w = fmaf(w, v.w, o.w);
+    float M = sm[0];
+#pragma unroll
+    for (int w = 1; w < W; ++w) M = fmaxf(M, sm[w]);
+    float L = 0.0f, o = 0.0f;
+    const float* accp = a.part.acc + (size_t)row * kHeadDim + slice * 32 + lane;
+    const size_t sstride = (size_t)a.n_rows * kHeadDim;
+    int s = warp;
+    for (; s + 3 * W < a.n_splits; s += 4 * W) {
+        float2 mls[4];
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            mls[u] = ml[(size_t)(s + u * W) * a.n_rows];
+            v[u] = accp[(size_t)(s + u * W) * sstride];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (mls[u].y > 0.0f) {
+                const float w = exp2f(mls[u].x - M);
+                L = fmaf(w, mls[u].y, L);
+                o = fmaf(w, v[u], o);
+            }
         }
     }
-    sacc[warp][4 * lane + 0] = o.x; sacc[warp][4 * lane + 1] = o.y;
-    sacc[warp][4 * lane + 2] = o.z; sacc[warp][4 * lane + 3] = o.w;
+    for (; s < a.n_splits; s += W) {
+        const float2 mlv = ml[(size_t)s * a.n_rows];
+        const float v = accp[(size_t)s * sstride];
+        if (mlv.y > 0.0f) {
+            const float w = exp2f(mlv.x - M);
+            L = fmaf(w, mlv.y, L);
+            o = fmaf(w, v, o);
+        }
+    }
+    sacc[warp][lane] = o;
     if (lane == 0) sl[warp] = L;
     __syncthreads();
-    const float Lt = sl[0] + sl[1] + sl[2] + sl[3];
-    const float inv = 1.0f / Lt;
-    const float v = sacc[0][tid] + sacc[1][tid] + sacc[2][tid] + sacc[3][tid];
-    a.out[(size_t)row * kHeadDim + tid] = v * inv;
-    if (tid == 0 && a.lse) a.lse[row] = (M + log2f(Lt)) * 0.69314718055994530942f;
+    if (warp == 0) {
+        float Lt = 0.0f, ot = 0.0f;
+#pragma unroll
+        for (int w = 0; w < W; ++w) { Lt += sl[w]; ot += sacc[w][lane]; }
+        a.out[(size_t)row * kHeadDim + slice * 32 + lane] = ot / Lt;
+        if (slice == 0 && lane == 0 && a.lse) a.lse[row] = (M + log2f(Lt)) * 0.69314718055994530942f;
+    }
 }
 
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s) {
-    merge_kernel<<<a.n_rows, 128, 0, s>>>(a);
+    merge_kernel<<<dim3(a.n_rows, kHeadDim / 32), kMergeThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 

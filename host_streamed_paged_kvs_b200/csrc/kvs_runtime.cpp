@@ -60,40 +60,36 @@ long auto_resident(long max_ctx, size_t page_bytes, int n_layers) {
     return std::max(pages, 1L);
 }
 
-// Split layout: pages per split on the resident set and inside one ring chunk.
-// Few query rows (decode) -> one page per split for parallelism; many rows ->
-// coarser splits keep the partial buffer and the merge small.
-struct SplitPolicy {
-    int res_pps, ring_pps;
-};
-SplitPolicy split_policy(const kvs_config& c, int n_rows_total) {
-    SplitPolicy p;
-    if (n_rows_total <= 64) {
-        p.res_pps = 1;
-        p.ring_pps = 1;
-    } else {
-        p.res_pps = std::max(1, c.n_resident_pages / 8);
-        p.ring_pps = std::max(1, c.chunk_pages);
-    }
-    return p;
+// Split layout, in half-page stages per split.  Decode (few query rows):
+// resident splits sized so the resident launch has about two CTAs per SM
+// (1..4 stages each), one stage per split inside a ring chunk so a chunk's
+// kernel spreads over many SMs.  Many rows (verify / prefill): at most 8
+// resident splits and one split per ring chunk, which keeps the partial buffer
+// and the merge small.
+constexpr int kSmallRows = 64;
+constexpr int kTargetCtas = 296;  // 148 SMs x 2 resident CTAs
+
+int res_stages_per_split(const kvs_config& c, long R_eff, int rows) {
+    if (rows > kSmallRows) return (int)std::max(1L, (2 * R_eff + 7) / 8);
+    const int per_head = rows / c.n_kv_heads;
+    const long groups = std::max(1, (per_head + 7) / 8);
+    const long sps = 2 * R_eff * c.n_kv_heads * groups / kTargetCtas;
+    return (int)std::min(4L, std::max(1L, sps));
 }
 
-size_t max_splits(const kvs_config& c) {
+int ring_stages_per_split(int rows, int chunk_pages) { return rows > kSmallRows ? 2 * chunk_pages : 1; }
+
+// capacity of the partial buffer in (split x row) records
+size_t partial_records(const kvs_config& c) {
     const long P = pages_for(c.max_ctx);
     const long R = std::min<long>(c.n_resident_pages, P);
     const long S = P - R;
-    size_t worst = 0;
-    // the split count grows as the rows shrink; bound it over both policies
-    for (int rows : {1, c.max_q_tokens * c.n_q_heads}) {
-        const SplitPolicy sp = split_policy(c, rows);
-        size_t n = (size_t)((R + sp.res_pps - 1) / sp.res_pps);
-        if (S > 0 && c.n_ring_slots > 0) {
-            const long chunks = (S + c.chunk_pages - 1) / c.chunk_pages;
-            n += (size_t)chunks * (size_t)((c.chunk_pages + sp.ring_pps - 1) / sp.ring_pps);
-        }
-        worst = std::max(worst, n);
-    }
-    return std::max<size_t>(worst, 1);
+    const long chunks = (S > 0 && c.chunk_pages > 0) ? (S + c.chunk_pages - 1) / c.chunk_pages : 0;
+    const size_t max_rows = (size_t)c.max_q_tokens * c.n_q_heads;
+    const size_t small_rows = std::min<size_t>(max_rows, kSmallRows);
+    size_t n = (size_t)(2 * P + 2) * small_rows;                          // decode regime
+    if (max_rows > kSmallRows) n = std::max(n, (size_t)(8 + chunks + 2) * max_rows);  // wide regime
+    return n;
 }
 
 struct ArenaLayout {
@@ -103,13 +99,13 @@ struct ArenaLayout {
 ArenaLayout arena_layout(const kvs_config& c) {
     const size_t pb = (size_t)c.n_kv_heads * kPageHeadBytes;
     const size_t rows = (size_t)c.max_q_tokens * c.n_q_heads;
-    const size_t ns = max_splits(c);
+    const size_t recs = partial_records(c);
     ArenaLayout L{};
     size_t off = 0;
     L.resident = off; off = align_up(off + (size_t)c.n_layers * c.n_resident_pages * pb, 1024);
     L.ring = off;     off = align_up(off + (size_t)c.n_ring_slots * pb, 1024);
-    L.part_ml = off;  off = align_up(off + ns * rows * sizeof(float2));
-    L.part_acc = off; off = align_up(off + ns * rows * kHeadDim * sizeof(float));
+    L.part_ml = off;  off = align_up(off + recs * sizeof(float2));
+    L.part_acc = off; off = align_up(off + recs * kHeadDim * sizeof(float));
     L.stage_q = off;  off = align_up(off + rows * kHeadDim * sizeof(__half));
     L.stage_kv = off; off = align_up(off + 2 * (size_t)c.max_q_tokens * c.n_kv_heads * kHeadDim * sizeof(__half));
     L.stage_out = off; off = align_up(off + rows * kHeadDim * sizeof(float));
@@ -239,7 +235,10 @@ struct kvs_s {
     float *stage_out = nullptr, *stage_lse = nullptr;
     int* err_word = nullptr;
     CUtensorMap map_res{}, map_ring{};
-    cudaStream_t cs = nullptr;
+    cudaStream_t cs = nullptr;       // copy stream (H2D ring)
+    cudaStream_t rs = nullptr;       // side stream: resident-page attention
+    cudaEvent_t ev_fork = nullptr, ev_res = nullptr;
+    size_t partial_capacity = 0;     // (split x row) records
     int n_groups = 0;
     std::vector<cudaEvent_t> ev_full, ev_free, ev_hist;
     std::vector<char> free_valid;
@@ -311,13 +310,26 @@ struct TimedScope {
             cudaEventRecord(t.a, s);
         }
     }
-    ~TimedScope() {
-        if (on) {
-            cudaEventRecord(t.b, s);
-            kv->timed.push_back(t);
-        }
-    }
+    ~TimedScope();
 };
+
+void fold_timed_upto(kvs_t* kv, size_t n);
+
+// fold the leading records whose end event has completed (non-blocking)
+void fold_completed(kvs_t* kv) {
+    size_t n = 0;
+    while (n < kv->timed.size() && cudaEventQuery(kv->timed[n].b) == cudaSuccess) ++n;
+    cudaGetLastError();
+    fold_timed_upto(kv, n);
+}
+
+TimedScope::~TimedScope() {
+    if (on) {
+        cudaEventRecord(t.b, s);
+        kv->timed.push_back(t);
+        if (kv->timed.size() >= 2048) fold_completed(kv);
+    }
+}
 
 int encode_map(kvs_t* kv, EncodeTiledFn fn, CUtensorMap* map, void* base, uint64_t rows) {
     if (rows == 0) return KVS_OK;
@@ -340,7 +352,10 @@ void release(kvs_t* kv) {
     for (auto e : kv->ev_full) if (e) cudaEventDestroy(e);
     for (auto e : kv->ev_free) if (e) cudaEventDestroy(e);
     for (auto e : kv->ev_hist) if (e) cudaEventDestroy(e);
+    if (kv->ev_fork) cudaEventDestroy(kv->ev_fork);
+    if (kv->ev_res) cudaEventDestroy(kv->ev_res);
     if (kv->cs) cudaStreamDestroy(kv->cs);
+    if (kv->rs) cudaStreamDestroy(kv->rs);
     if (kv->arena) cudaFree(kv->arena);
     if (kv->host) cudaFreeHost(kv->host);
     delete kv;
@@ -360,13 +375,16 @@ int wait_event(kvs_t* kv, cudaEvent_t e, double timeout_s) {
 }
 
 int sync_all(kvs_t* kv, cudaStream_t user, double timeout_s) {
-    cudaEvent_t e1 = pool_event(kv), e2 = pool_event(kv);
+    cudaEvent_t e1 = pool_event(kv), e2 = pool_event(kv), e3 = pool_event(kv);
     KVS_CK(kv, cudaEventRecord(e1, kv->cs));
     KVS_CK(kv, cudaEventRecord(e2, user));
+    KVS_CK(kv, cudaEventRecord(e3, kv->rs));
     int rc = wait_event(kv, e1, timeout_s);
     if (rc == KVS_OK) rc = wait_event(kv, e2, timeout_s);
+    if (rc == KVS_OK) rc = wait_event(kv, e3, timeout_s);
     kv->ev_pool.push_back(e1);
     kv->ev_pool.push_back(e2);
+    kv->ev_pool.push_back(e3);
     if (rc != KVS_OK) return rc;
     int err = 0;
     KVS_CK(kv, cudaMemcpy(&err, kv->err_word, sizeof(int), cudaMemcpyDeviceToHost));
@@ -374,8 +392,9 @@ int sync_all(kvs_t* kv, cudaStream_t user, double timeout_s) {
     return KVS_OK;
 }
 
-void fold_timed(kvs_t* kv) {
-    for (auto& t : kv->timed) {
+void fold_timed_upto(kvs_t* kv, size_t n) {
+    for (size_t i = 0; i < n; ++i) {
+        Timed& t = kv->timed[i];
         float ms = 0.f;
         if (cudaEventElapsedTime(&ms, t.a, t.b) != cudaSuccess) { cudaGetLastError(); ms = 0.f; }
         switch (t.kind) {
@@ -390,8 +409,10 @@ void fold_timed(kvs_t* kv) {
         kv->ev_pool.push_back(t.a);
         kv->ev_pool.push_back(t.b);
     }
-    kv->timed.clear();
+    kv->timed.erase(kv->timed.begin(), kv->timed.begin() + n);
 }
+
+void fold_timed(kvs_t* kv) { fold_timed_upto(kv, kv->timed.size()); }
 
 }  // namespace
 
@@ -479,6 +500,12 @@ int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
 
     e = cudaStreamCreateWithFlags(&kv->cs, cudaStreamNonBlocking);
     if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("cudaStreamCreate: %s", cudaGetErrorString(e)));
+    e = cudaStreamCreateWithFlags(&kv->rs, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("cudaStreamCreate: %s", cudaGetErrorString(e)));
+    if (cudaEventCreateWithFlags(&kv->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&kv->ev_res, cudaEventDisableTiming) != cudaSuccess)
+        return bail(KVS_E_CUDA, "cudaEventCreate failed");
+    kv->partial_capacity = partial_records(c);
     kv->n_groups = c.n_ring_slots > 0 ? c.n_ring_slots / c.chunk_pages : 0;
     kv->ev_full.assign(kv->n_groups, nullptr);
     kv->ev_free.assign(kv->n_groups, nullptr);
@@ -521,9 +548,11 @@ void kvs_destroy(kvs_t* kv) {
     if (!kv) return;
     {
         DeviceGuard g(kv->device);
-        cudaEvent_t e = pool_event(kv);
-        if (e && cudaEventRecord(e, kv->cs) == cudaSuccess) wait_event(kv, e, 60.0);
-        if (e) kv->ev_pool.push_back(e);
+        for (cudaStream_t st : {kv->cs, kv->rs}) {
+            cudaEvent_t e = pool_event(kv);
+            if (e && st && cudaEventRecord(e, st) == cudaSuccess) wait_event(kv, e, 60.0);
+            if (e) kv->ev_pool.push_back(e);
+        }
         cudaDeviceSynchronize();
     }
     release(kv);
@@ -630,7 +659,6 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     const long R_eff = std::min(R, P);
     const long first_res = P - R_eff;
     const long S = first_res;
-    const SplitPolicy sp = split_policy(c, rows);
 
     DecodeArgs d{};
     d.len = ls.len;
@@ -645,7 +673,8 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     d.n_rows = rows;
     d.err = kv->err_word;
 
-    // 1) resident pages, attended in place
+    // 1) resident pages, attended in place on the side stream so they overlap
+    //    the ring pipeline below
     int split_base = 0;
     {
         d.region = kv->resident + (size_t)layer * R * kv->page_bytes;
@@ -654,11 +683,16 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         d.slot0 = (int)(first_res % R);
         d.page0 = (int)first_res;
         d.n_units = (int)R_eff;
-        d.pages_per_split = sp.res_pps;
+        d.stages_per_split = res_stages_per_split(c, R_eff, rows);
         d.split_base = split_base;
-        const int ns = (int)((R_eff + sp.res_pps - 1) / sp.res_pps);
-        TimedScope ts(kv, s, kTDecodeRes, (uint64_t)R_eff * kv->page_bytes);
-        KVS_CK(kv, launch_decode(d, &kv->map_res, ns, s));
+        const int ns = (int)((2 * R_eff + d.stages_per_split - 1) / d.stages_per_split);
+        KVS_CK(kv, cudaEventRecord(kv->ev_fork, s));
+        KVS_CK(kv, cudaStreamWaitEvent(kv->rs, kv->ev_fork, 0));
+        {
+            TimedScope ts(kv, kv->rs, kTDecodeRes, (uint64_t)R_eff * kv->page_bytes);
+            KVS_CK(kv, launch_decode(d, &kv->map_res, ns, kv->rs));
+        }
+        KVS_CK(kv, cudaEventRecord(kv->ev_res, kv->rs));
         kv->stats.kernel_launches++;
         split_base += ns;
         kv->stats.bytes_resident_read += (uint64_t)R_eff * kv->page_bytes;
@@ -687,9 +721,9 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
             d.slot0 = gidx * chunk;
             d.page0 = (int)i0;
             d.n_units = cpages;
-            d.pages_per_split = sp.ring_pps;
+            d.stages_per_split = ring_stages_per_split(rows, chunk);
             d.split_base = split_base;
-            const int ns = (cpages + sp.ring_pps - 1) / sp.ring_pps;
+            const int ns = (2 * cpages + d.stages_per_split - 1) / d.stages_per_split;
             {
                 TimedScope ts(kv, s, kTDecodeRing, (uint64_t)cpages * kv->page_bytes);
                 KVS_CK(kv, launch_decode(d, &kv->map_ring, ns, s));
@@ -703,7 +737,10 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
             kv->stats.h2d_copies++;
         }
     }
-    // 3) log-sum-exp merge of all splits
+    // 3) log-sum-exp merge of all splits (after the side stream's resident splits)
+    KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_res, 0));
+    if ((size_t)split_base * rows > kv->partial_capacity)
+        return fail(kv, KVS_E_INVAL, "internal: partial buffer too small");
     MergeArgs m;
     m.part = kv->part;
     m.n_splits = split_base;
@@ -796,6 +833,13 @@ int kvs_reset_stats(kvs_t* kv) {
         fold_timed(kv);
     }
     kv->stats = kvs_stats{};
+    return KVS_OK;
+}
+
+int kvs_set_profiling(kvs_t* kv, int enable) {
+    if (!kv) return fail(nullptr, KVS_E_INVAL, "null handle");
+    if (enable) kv->cfg.flags |= KVS_FLAG_PROFILE;
+    else kv->cfg.flags &= ~KVS_FLAG_PROFILE;
     return KVS_OK;
 }
 

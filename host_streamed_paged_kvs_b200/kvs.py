@@ -35,8 +35,8 @@ ERROR_NAMES = {0: "KVS_OK", -1: "KVS_E_INVAL", -2: "KVS_E_ARENA", -3: "KVS_E_WID
 # every symbol the header declares
 EXPORTS = ["kvs_resolve_config", "kvs_page_bytes", "kvs_plan_page", "kvs_create", "kvs_destroy",
            "kvs_append", "kvs_attend", "kvs_export_page", "kvs_page_location", "kvs_layer_length",
-           "kvs_get_config", "kvs_get_stats", "kvs_reset_stats", "kvs_sync", "kvs_measure_h2d",
-           "kvs_last_error"]
+           "kvs_get_config", "kvs_get_stats", "kvs_reset_stats", "kvs_set_profiling", "kvs_sync",
+           "kvs_measure_h2d", "kvs_last_error"]
 
 
 class kvs_config(ctypes.Structure):
@@ -88,6 +88,7 @@ def _load():
     L.kvs_get_config.argtypes = [vp, cp(kvs_config)]
     L.kvs_get_stats.argtypes = [vp, cp(kvs_stats)]
     L.kvs_reset_stats.argtypes = [vp]
+    L.kvs_set_profiling.argtypes = [vp, i]
     L.kvs_sync.argtypes = [vp, vp, ctypes.c_double]
     L.kvs_measure_h2d.argtypes = [vp, ctypes.c_size_t, ctypes.c_size_t, i, cp(ctypes.c_double)]
     L.kvs_last_error.restype = ctypes.c_char_p
@@ -205,6 +206,10 @@ def kvs_get_stats(h) -> dict:
 
 def kvs_reset_stats(h) -> None:
     _check(lib.kvs_reset_stats(h), h)
+
+
+def kvs_set_profiling(h, enable: bool) -> None:
+    _check(lib.kvs_set_profiling(h, int(bool(enable))), h)
 
 
 def kvs_sync(h, stream=None, timeout_s: float = 60.0) -> None:

@@ -176,6 +176,9 @@ int kvs_get_config(kvs_t* kv, kvs_config* out);
 int kvs_get_stats(kvs_t* kv, kvs_stats* out);
 int kvs_reset_stats(kvs_t* kv);
 
+/* Turn KVS_FLAG_PROFILE on (1) or off (0) for later calls. */
+int kvs_set_profiling(kvs_t* kv, int enable);
+
 /* Bounded host wait for all work the library enqueued (copy stream) and for
  * `stream`: polls, returns KVS_E_TIMEOUT after timeout_s seconds. */
 int kvs_sync(kvs_t* kv, void* stream, double timeout_s);
