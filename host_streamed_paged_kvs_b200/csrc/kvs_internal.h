@@ -87,6 +87,9 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, int n_sp
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s);
 size_t decode_smem_bytes();
 
+// record the calling thread's last error text (returned by kvs_last_error(NULL))
+void set_last_error(const char* msg);
+
 // error bits written to the device error word
 enum : int {
     kErrWaitTimeout = 1,

@@ -218,6 +218,8 @@ struct Timed {
 
 }  // namespace
 
+void kvs::set_last_error(const char* msg) { g_last_error = msg ? msg : ""; }
+
 struct kvs_s {
     kvs_config cfg{};
     int device = 0;

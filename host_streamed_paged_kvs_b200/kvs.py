@@ -36,7 +36,7 @@ ERROR_NAMES = {0: "KVS_OK", -1: "KVS_E_INVAL", -2: "KVS_E_ARENA", -3: "KVS_E_WID
 EXPORTS = ["kvs_resolve_config", "kvs_page_bytes", "kvs_plan_page", "kvs_create", "kvs_destroy",
            "kvs_append", "kvs_attend", "kvs_export_page", "kvs_page_location", "kvs_layer_length",
            "kvs_get_config", "kvs_get_stats", "kvs_reset_stats", "kvs_set_profiling", "kvs_sync",
-           "kvs_measure_h2d", "kvs_last_error"]
+           "kvs_measure_h2d", "kvs_attend_pages_static", "kvs_last_error"]
 
 
 class kvs_config(ctypes.Structure):
@@ -91,6 +91,7 @@ def _load():
     L.kvs_set_profiling.argtypes = [vp, i]
     L.kvs_sync.argtypes = [vp, vp, ctypes.c_double]
     L.kvs_measure_h2d.argtypes = [vp, ctypes.c_size_t, ctypes.c_size_t, i, cp(ctypes.c_double)]
+    L.kvs_attend_pages_static.argtypes = [vp, i, i, i, i, i, i, vp, vp, vp, vp]
     L.kvs_last_error.restype = ctypes.c_char_p
     L.kvs_last_error.argtypes = [vp]
     return L
@@ -220,6 +221,13 @@ def kvs_measure_h2d(h, chunk_bytes: int, total_bytes: int, reps: int = 10) -> fl
     g = ctypes.c_double()
     _check(lib.kvs_measure_h2d(h, chunk_bytes, total_bytes, reps, ctypes.byref(g)), h)
     return g.value
+
+
+def kvs_attend_pages_static(pages, n_pages, n_tokens, n_q_heads, n_kv_heads, pos0, n_q, q, out,
+                            lse=None, stream=None) -> None:
+    """No-allocation attention over caller-owned device pages (see include/kvs.h)."""
+    _check(lib.kvs_attend_pages_static(_addr(pages), n_pages, n_tokens, n_q_heads, n_kv_heads, pos0,
+                                       n_q, _addr(q), _addr(out), _addr(lse), _stream(stream)))
 
 
 def kvs_last_error(h=None) -> str:

@@ -188,6 +188,32 @@ int kvs_sync(kvs_t* kv, void* stream, double timeout_s);
  * copy stream and a scratch region of the device arena.  GB/s in *gbs. */
 int kvs_measure_h2d(kvs_t* kv, size_t chunk_bytes, size_t total_bytes, int reps, double* gbs);
 
+/* Attention over caller-owned device pages that allocates nothing.
+ *
+ * The paper has no counterpart to this call.  It serves callers that cannot
+ * allocate device memory on their hot path: an engine whose own pool owns all
+ * device memory, a server whose allocations are frozen after start-up so no
+ * request can fail for memory, or a latency-critical loop that must avoid
+ * cudaMalloc's implicit device synchronization.  It needs no handle: the
+ * split partials live in one static device array inside libkvs (2 MiB + 32 KiB
+ * per GPU that loads the library, held until exit); nothing is allocated.
+ *
+ * pages: device, 16-byte aligned, n_pages pages in libkvs's page layout, page
+ *        p = tokens [256p, 256p+256): [n_kv_heads][53,248-byte page head] with
+ *        the page head = Kq int8 [256][128] | Kd fp16 [256][4] |
+ *        Vq u8 [256][4][16] (byte j: code j low nibble, code j+16 high) |
+ *        Vd fp16 [256][4];
+ * keys 0..n_tokens-1 are attended; query j sits at pos0+j and sees keys
+ * 0..pos0+j; q fp16 [n_q][n_q_heads][128]; out fp32 [n_q][n_q_heads][128];
+ * lse fp32 [n_q][n_q_heads] or NULL.  Limit: n_q * n_q_heads <= 64, else
+ * KVS_E_WIDTH.  The first call on a device looks up the static array's device
+ * address (with that device current); make that first call before any stream
+ * capture.  Every call shares the array, so calls whose kernels may overlap on
+ * the GPU race: order them on one stream.  Stream ordered and asynchronous. */
+int kvs_attend_pages_static(const void* pages, int n_pages, int n_tokens, int n_q_heads,
+                            int n_kv_heads, int pos0, int n_q, const void* q_f16, float* out,
+                            float* lse, void* stream);
+
 /* Last error text of the handle (or of the calling thread's last failed
  * kvs_create / pure call when kv is NULL). */
 const char* kvs_last_error(kvs_t* kv);
