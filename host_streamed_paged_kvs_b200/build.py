@@ -9,8 +9,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libkvs.so")
-SOURCES = ["kvs_kernels.cu", "kvs_runtime.cpp", "kvs_static.cu"]
-HEADERS = ["kvs_internal.h"]
+SOURCES = ["kvs_kernels.cu", "kvs_chunk_mma.cu", "kvs_runtime.cpp", "kvs_static.cu"]
+HEADERS = ["kvs_internal.h", "kvs_ptx.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 

@@ -85,6 +85,10 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                           cudaStream_t s);
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s);
+// multi-token (verify / prefill chunk) attention on tcgen05 tensor cores; same
+// arguments and partial format as launch_decode
+cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
+                             cudaStream_t s);
 size_t decode_smem_bytes();
 
 // record the calling thread's last error text (returned by kvs_last_error(NULL))

@@ -60,36 +60,71 @@ long auto_resident(long max_ctx, size_t page_bytes, int n_layers) {
     return std::max(pages, 1L);
 }
 
-// Split layout, in half-page stages per split.  Decode (few query rows):
-// resident splits sized so the resident launch has about two CTAs per SM
-// (1..4 stages each), one stage per split inside a ring chunk so a chunk's
-// kernel spreads over many SMs.  Many rows (verify / prefill): at most 8
-// resident splits and one split per ring chunk, which keeps the partial buffer
-// and the merge small.
+// Split layout, in half-page stages per split.
+//  * CUDA-core decode (<= 8 query rows per kv head): resident splits sized so
+//    the resident launch has about two CTAs per SM (1..4 stages each), one
+//    stage per split inside a ring chunk so a chunk's kernel spreads over many
+//    SMs.
+//  * tensor-core path (more rows per kv head: verify batches, prefill chunks)
+//    and very wide decode: at most 8 resident splits and one split per ring
+//    chunk, which keeps the partial buffer and the merge small.
 constexpr int kSmallRows = 64;
 constexpr int kTargetCtas = 296;  // 148 SMs x 2 resident CTAs
+constexpr int kMaxCudaCoreRows = 8;
 
-int res_stages_per_split(const kvs_config& c, long R_eff, int rows) {
-    if (rows > kSmallRows) return (int)std::max(1L, (2 * R_eff + 7) / 8);
-    const int per_head = rows / c.n_kv_heads;
-    const long groups = std::max(1, (per_head + 7) / 8);
-    const long sps = 2 * R_eff * c.n_kv_heads * groups / kTargetCtas;
+bool use_tensor_cores(const kvs_config& c, int n_q) { return n_q * (c.n_q_heads / c.n_kv_heads) > kMaxCudaCoreRows; }
+bool wide_regime(const kvs_config& c, int n_q) { return n_q * c.n_q_heads > kSmallRows; }
+int m_tiles(const kvs_config& c, int n_q) { return (n_q * (c.n_q_heads / c.n_kv_heads) + 127) / 128; }
+
+// Tensor-core path: splits sized for about one CTA per SM per ring chunk and
+// about two waves over the resident pages (the kernel holds one CTA per SM).
+constexpr int kSms = 148;
+
+int res_stages_per_split(const kvs_config& c, long R_eff, int n_q) {
+    const long stages = 2 * R_eff;
+    if (use_tensor_cores(c, n_q)) {
+        const long per_split = (long)c.n_kv_heads * m_tiles(c, n_q);
+        const long want = std::min(stages, std::max(1L, (2L * kSms + per_split - 1) / per_split));
+        return (int)std::max(1L, (stages + want - 1) / want);
+    }
+    if (wide_regime(c, n_q)) return (int)std::max(1L, (stages + 7) / 8);
+    const long sps = stages * c.n_kv_heads / kTargetCtas;
     return (int)std::min(4L, std::max(1L, sps));
 }
 
-int ring_stages_per_split(int rows, int chunk_pages) { return rows > kSmallRows ? 2 * chunk_pages : 1; }
+int ring_stages_per_split(const kvs_config& c, int n_q, int chunk_pages) {
+    const int stages = 2 * chunk_pages;
+    if (use_tensor_cores(c, n_q)) {
+        const int per_split = c.n_kv_heads * m_tiles(c, n_q);
+        const int want = std::min(stages, std::max(1, (kSms + per_split - 1) / per_split));
+        return std::max(1, (stages + want - 1) / want);
+    }
+    return wide_regime(c, n_q) ? stages : 1;
+}
 
-// capacity of the partial buffer in (split x row) records
+long count_splits(const kvs_config& c, int n_q, long R_eff, long S) {
+    const int sps_res = res_stages_per_split(c, R_eff, n_q);
+    long n = (2 * R_eff + sps_res - 1) / sps_res;
+    if (S > 0 && c.chunk_pages > 0) {
+        const int sps_ring = ring_stages_per_split(c, n_q, c.chunk_pages);
+        const long full = S / c.chunk_pages, tail = S % c.chunk_pages;
+        n += full * ((2 * c.chunk_pages + sps_ring - 1) / sps_ring);
+        if (tail) n += (2 * tail + sps_ring - 1) / sps_ring;
+    }
+    return n;
+}
+
+// capacity of the partial buffer in (split x row) records: the largest need
+// over every query width the handle accepts, at the longest history (split
+// counts only grow with the number of resident and streamed pages)
 size_t partial_records(const kvs_config& c) {
     const long P = pages_for(c.max_ctx);
-    const long R = std::min<long>(c.n_resident_pages, P);
-    const long S = P - R;
-    const long chunks = (S > 0 && c.chunk_pages > 0) ? (S + c.chunk_pages - 1) / c.chunk_pages : 0;
-    const size_t max_rows = (size_t)c.max_q_tokens * c.n_q_heads;
-    const size_t small_rows = std::min<size_t>(max_rows, kSmallRows);
-    size_t n = (size_t)(2 * P + 2) * small_rows;                          // decode regime
-    if (max_rows > kSmallRows) n = std::max(n, (size_t)(8 + chunks + 2) * max_rows);  // wide regime
-    return n;
+    const long R_eff = std::min<long>(c.n_resident_pages, P);
+    const long S = c.n_ring_slots > 0 ? P - R_eff : 0;
+    size_t best = 1;
+    for (int n_q = 1; n_q <= c.max_q_tokens; ++n_q)
+        best = std::max(best, (size_t)count_splits(c, n_q, R_eff, S) * (size_t)(n_q * c.n_q_heads));
+    return best;
 }
 
 struct ArenaLayout {
@@ -238,8 +273,9 @@ struct kvs_s {
     int* err_word = nullptr;
     CUtensorMap map_res{}, map_ring{};
     cudaStream_t cs = nullptr;       // copy stream (H2D ring)
-    cudaStream_t rs = nullptr;       // side stream: resident-page attention
-    cudaEvent_t ev_fork = nullptr, ev_res = nullptr;
+    cudaStream_t rs = nullptr;       // side stream: resident-page attention (lowest priority)
+    cudaStream_t xs = nullptr;       // ring attention stream (highest priority)
+    cudaEvent_t ev_fork = nullptr, ev_res = nullptr, ev_ring = nullptr;
     size_t partial_capacity = 0;     // (split x row) records
     int n_groups = 0;
     std::vector<cudaEvent_t> ev_full, ev_free, ev_hist;
@@ -356,6 +392,8 @@ void release(kvs_t* kv) {
     for (auto e : kv->ev_hist) if (e) cudaEventDestroy(e);
     if (kv->ev_fork) cudaEventDestroy(kv->ev_fork);
     if (kv->ev_res) cudaEventDestroy(kv->ev_res);
+    if (kv->ev_ring) cudaEventDestroy(kv->ev_ring);
+    if (kv->xs) cudaStreamDestroy(kv->xs);
     if (kv->cs) cudaStreamDestroy(kv->cs);
     if (kv->rs) cudaStreamDestroy(kv->rs);
     if (kv->arena) cudaFree(kv->arena);
@@ -377,16 +415,13 @@ int wait_event(kvs_t* kv, cudaEvent_t e, double timeout_s) {
 }
 
 int sync_all(kvs_t* kv, cudaStream_t user, double timeout_s) {
-    cudaEvent_t e1 = pool_event(kv), e2 = pool_event(kv), e3 = pool_event(kv);
-    KVS_CK(kv, cudaEventRecord(e1, kv->cs));
-    KVS_CK(kv, cudaEventRecord(e2, user));
-    KVS_CK(kv, cudaEventRecord(e3, kv->rs));
-    int rc = wait_event(kv, e1, timeout_s);
-    if (rc == KVS_OK) rc = wait_event(kv, e2, timeout_s);
-    if (rc == KVS_OK) rc = wait_event(kv, e3, timeout_s);
-    kv->ev_pool.push_back(e1);
-    kv->ev_pool.push_back(e2);
-    kv->ev_pool.push_back(e3);
+    int rc = KVS_OK;
+    for (cudaStream_t st : {kv->cs, user, kv->rs, kv->xs}) {
+        cudaEvent_t e = pool_event(kv);
+        KVS_CK(kv, cudaEventRecord(e, st));
+        if (rc == KVS_OK) rc = wait_event(kv, e, timeout_s);
+        kv->ev_pool.push_back(e);
+    }
     if (rc != KVS_OK) return rc;
     int err = 0;
     KVS_CK(kv, cudaMemcpy(&err, kv->err_word, sizeof(int), cudaMemcpyDeviceToHost));
@@ -502,10 +537,17 @@ int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
 
     e = cudaStreamCreateWithFlags(&kv->cs, cudaStreamNonBlocking);
     if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("cudaStreamCreate: %s", cudaGetErrorString(e)));
-    e = cudaStreamCreateWithFlags(&kv->rs, cudaStreamNonBlocking);
+    // the ring's attention kernels free ring slots for the copy engine, so they
+    // run at the highest priority; resident-page attention fills in behind them
+    int prio_low = 0, prio_high = 0;
+    cudaDeviceGetStreamPriorityRange(&prio_low, &prio_high);
+    e = cudaStreamCreateWithPriority(&kv->rs, cudaStreamNonBlocking, prio_low);
+    if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("cudaStreamCreate: %s", cudaGetErrorString(e)));
+    e = cudaStreamCreateWithPriority(&kv->xs, cudaStreamNonBlocking, prio_high);
     if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("cudaStreamCreate: %s", cudaGetErrorString(e)));
     if (cudaEventCreateWithFlags(&kv->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&kv->ev_res, cudaEventDisableTiming) != cudaSuccess)
+        cudaEventCreateWithFlags(&kv->ev_res, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&kv->ev_ring, cudaEventDisableTiming) != cudaSuccess)
         return bail(KVS_E_CUDA, "cudaEventCreate failed");
     kv->partial_capacity = partial_records(c);
     kv->n_groups = c.n_ring_slots > 0 ? c.n_ring_slots / c.chunk_pages : 0;
@@ -550,7 +592,7 @@ void kvs_destroy(kvs_t* kv) {
     if (!kv) return;
     {
         DeviceGuard g(kv->device);
-        for (cudaStream_t st : {kv->cs, kv->rs}) {
+        for (cudaStream_t st : {kv->cs, kv->rs, kv->xs}) {
             cudaEvent_t e = pool_event(kv);
             if (e && st && cudaEventRecord(e, st) == cudaSuccess) wait_event(kv, e, 60.0);
             if (e) kv->ev_pool.push_back(e);
@@ -656,6 +698,9 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     float* dout = host_out ? kv->stage_out : out;
     float* dlse = lse ? (host_lse ? kv->stage_lse : lse) : nullptr;
 
+    const bool tc = use_tensor_cores(c, n_q);
+    if (tc && (reinterpret_cast<uintptr_t>(q) & 15))
+        return fail(kv, KVS_E_INVAL, "q must be 16-byte aligned for multi-token attention");
     const long R = c.n_resident_pages;
     const long P = pages_for(ls.len);
     const long R_eff = std::min(R, P);
@@ -675,6 +720,9 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     d.n_rows = rows;
     d.err = kv->err_word;
 
+    // split counts first: the partial buffer must hold every (split, row) record
+    if ((size_t)count_splits(c, n_q, R_eff, S) * rows > kv->partial_capacity)
+        return fail(kv, KVS_E_INVAL, "internal: partial buffer too small for this call");
     // 1) resident pages, attended in place on the side stream so they overlap
     //    the ring pipeline below
     int split_base = 0;
@@ -685,14 +733,14 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         d.slot0 = (int)(first_res % R);
         d.page0 = (int)first_res;
         d.n_units = (int)R_eff;
-        d.stages_per_split = res_stages_per_split(c, R_eff, rows);
+        d.stages_per_split = res_stages_per_split(c, R_eff, n_q);
         d.split_base = split_base;
         const int ns = (int)((2 * R_eff + d.stages_per_split - 1) / d.stages_per_split);
         KVS_CK(kv, cudaEventRecord(kv->ev_fork, s));
         KVS_CK(kv, cudaStreamWaitEvent(kv->rs, kv->ev_fork, 0));
         {
-            TimedScope ts(kv, kv->rs, kTDecodeRes, (uint64_t)R_eff * kv->page_bytes);
-            KVS_CK(kv, launch_decode(d, &kv->map_res, ns, kv->rs));
+            TimedScope ts(kv, kv->rs, tc ? kTChunkMma : kTDecodeRes, (uint64_t)R_eff * kv->page_bytes);
+            KVS_CK(kv, tc ? launch_chunk_mma(d, &kv->map_res, ns, kv->rs) : launch_decode(d, &kv->map_res, ns, kv->rs));
         }
         KVS_CK(kv, cudaEventRecord(kv->ev_res, kv->rs));
         kv->stats.kernel_launches++;
@@ -707,6 +755,7 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
             ls.pending_min_page = INT_MAX;
         }
         const int chunk = c.chunk_pages;
+        KVS_CK(kv, cudaStreamWaitEvent(kv->xs, kv->ev_fork, 0));
         for (long i0 = 0; i0 < S; i0 += chunk) {
             const int cpages = (int)std::min<long>(chunk, S - i0);
             const int gidx = (int)(kv->ring_ctr % kv->n_groups);
@@ -716,33 +765,35 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
             const uint8_t* src = kv->host + ((size_t)layer * kv->P_max + (size_t)i0) * kv->page_bytes;
             KVS_CK(kv, cudaMemcpyAsync(dst, src, (size_t)cpages * kv->page_bytes, cudaMemcpyHostToDevice, kv->cs));
             KVS_CK(kv, cudaEventRecord(kv->ev_full[gidx], kv->cs));
-            KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_full[gidx], 0));
+            KVS_CK(kv, cudaStreamWaitEvent(kv->xs, kv->ev_full[gidx], 0));
             d.region = kv->ring;
             d.region_slot_base = 0;
             d.region_slots = c.n_ring_slots;
             d.slot0 = gidx * chunk;
             d.page0 = (int)i0;
             d.n_units = cpages;
-            d.stages_per_split = ring_stages_per_split(rows, chunk);
+            d.stages_per_split = ring_stages_per_split(c, n_q, chunk);
             d.split_base = split_base;
             const int ns = (2 * cpages + d.stages_per_split - 1) / d.stages_per_split;
             {
-                TimedScope ts(kv, s, kTDecodeRing, (uint64_t)cpages * kv->page_bytes);
-                KVS_CK(kv, launch_decode(d, &kv->map_ring, ns, s));
+                TimedScope ts(kv, kv->xs, tc ? kTChunkMma : kTDecodeRing, (uint64_t)cpages * kv->page_bytes);
+                KVS_CK(kv, tc ? launch_chunk_mma(d, &kv->map_ring, ns, kv->xs)
+                              : launch_decode(d, &kv->map_ring, ns, kv->xs));
             }
             kv->stats.kernel_launches++;
-            KVS_CK(kv, cudaEventRecord(kv->ev_free[gidx], s));
+            KVS_CK(kv, cudaEventRecord(kv->ev_free[gidx], kv->xs));
             kv->free_valid[gidx] = 1;
             split_base += ns;
             kv->stats.pages_streamed += cpages;
             kv->stats.bytes_h2d += (uint64_t)cpages * kv->page_bytes;
             kv->stats.h2d_copies++;
         }
+        KVS_CK(kv, cudaEventRecord(kv->ev_ring, kv->xs));
+        KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_ring, 0));
     }
+
     // 3) log-sum-exp merge of all splits (after the side stream's resident splits)
     KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_res, 0));
-    if ((size_t)split_base * rows > kv->partial_capacity)
-        return fail(kv, KVS_E_INVAL, "internal: partial buffer too small");
     MergeArgs m;
     m.part = kv->part;
     m.n_splits = split_base;
