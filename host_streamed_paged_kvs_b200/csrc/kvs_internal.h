@@ -91,6 +91,9 @@ cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n
                              cudaStream_t s);
 size_t decode_smem_bytes();
 
+// bounded-wait self-test kernel (one thread, an mbarrier nothing completes)
+cudaError_t launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t s);
+
 // record the calling thread's last error text (returned by kvs_last_error(NULL))
 void set_last_error(const char* msg);
 

@@ -491,4 +491,21 @@ cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// ----------------------------------------------------------------------------
+// Self-test of the bounded wait: one thread waits on an mbarrier phase that
+// nothing ever completes (no arrival, no transaction), through the same wait
+// routine the kernels use, and must give up after limit_ns.
+// ----------------------------------------------------------------------------
+__global__ void wait_selftest_kernel(int* err, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait_bounded(&bar, 0, err, limit_ns);  // phase 0 never completes
+}
+
+cudaError_t launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t s) {
+    wait_selftest_kernel<<<1, 1, 0, s>>>(err, limit_ns);
+    return cudaGetLastError();
+}
+
 }  // namespace kvs

@@ -41,14 +41,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait: gives up after ~2^24 polls (each poll suspends in hardware for
-// a short time), records the failure in the device error word and returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err) {
-    for (uint32_t it = 0; it < (1u << 24); ++it) {
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait on an mbarrier phase: gives up after limit_ns of wall time
+// (a healthy wait ends within microseconds), records the failure in the device
+// error word and returns false so the kernel can stop cleanly.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 31) == 31 && globaltimer_ns() - t0 > limit_ns) {
+            if (err) atomicOr(err, kErrWaitTimeout);
+            return false;
+        }
     }
-    if (err) atomicOr(err, kErrWaitTimeout);
-    return false;
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,

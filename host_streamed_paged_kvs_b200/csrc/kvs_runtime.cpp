@@ -280,6 +280,12 @@ struct kvs_s {
     int n_groups = 0;
     std::vector<cudaEvent_t> ev_full, ev_free, ev_hist;
     std::vector<char> free_valid;
+    // stream-capture bookkeeping: the capture id (0 = none) in which each
+    // ring-free / history event was last recorded, the capture the copy stream
+    // has joined, and whether a capture happened since the last plain call
+    std::vector<unsigned long long> free_cap, hist_cap;
+    unsigned long long cs_cap = 0;
+    bool capture_seen = false;
     uint64_t ring_ctr = 0;
     std::vector<LayerState> layers;
     kvs_stats stats{};
@@ -324,6 +330,17 @@ cudaEvent_t pool_event(kvs_t* kv) {
     cudaEvent_t e = nullptr;
     cudaEventCreate(&e);
     return e;
+}
+
+// id of the capture `s` is recording into, 0 when it is not capturing
+unsigned long long capture_id(cudaStream_t s) {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    unsigned long long id = 0;
+    if (cudaStreamGetCaptureInfo(s, &st, &id) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return st == cudaStreamCaptureStatusActive ? id : 0;
 }
 
 bool profiling(const kvs_t* kv, cudaStream_t s) {
@@ -554,6 +571,7 @@ int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
     kv->ev_full.assign(kv->n_groups, nullptr);
     kv->ev_free.assign(kv->n_groups, nullptr);
     kv->free_valid.assign(kv->n_groups, 0);
+    kv->free_cap.assign(kv->n_groups, 0);
     for (int i = 0; i < kv->n_groups; ++i) {
         if (cudaEventCreateWithFlags(&kv->ev_full[i], cudaEventDisableTiming) != cudaSuccess ||
             cudaEventCreateWithFlags(&kv->ev_free[i], cudaEventDisableTiming) != cudaSuccess)
@@ -564,6 +582,7 @@ int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
         if (cudaEventCreateWithFlags(&kv->ev_hist[i], cudaEventDisableTiming) != cudaSuccess)
             return bail(KVS_E_CUDA, "cudaEventCreate failed");
     kv->layers.assign(c.n_layers, LayerState{});
+    kv->hist_cap.assign(c.n_layers, 0);
 
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult qr;
@@ -665,6 +684,8 @@ int kvs_append(kvs_t* kv, int layer, int pos0, int n_tok, const void* k_f16, con
     }
     kv->stats.kernel_launches++;
     KVS_CK(kv, cudaEventRecord(kv->ev_hist[layer], s));
+    kv->hist_cap[layer] = capture_id(s);
+    if (kv->hist_cap[layer]) kv->capture_seen = true;
     ls.hist_recorded = true;
     ls.pending_min_page = std::min(ls.pending_min_page, pos0 / kPageTokens);
     ls.len = pos0 + n_tok;
@@ -723,6 +744,12 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     // split counts first: the partial buffer must hold every (split, row) record
     if ((size_t)count_splits(c, n_q, R_eff, S) * rows > kv->partial_capacity)
         return fail(kv, KVS_E_INVAL, "internal: partial buffer too small for this call");
+    // With profiling on, every kernel runs on the caller's stream so that the
+    // events around a launch time that launch alone.
+    const bool prof = profiling(kv, s);
+    const unsigned long long cap = capture_id(s);
+    cudaStream_t rstream = prof ? s : kv->rs;
+    cudaStream_t xstream = prof ? s : kv->xs;
     // 1) resident pages, attended in place on the side stream so they overlap
     //    the ring pipeline below
     int split_base = 0;
@@ -737,12 +764,34 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         d.split_base = split_base;
         const int ns = (int)((2 * R_eff + d.stages_per_split - 1) / d.stages_per_split);
         KVS_CK(kv, cudaEventRecord(kv->ev_fork, s));
-        KVS_CK(kv, cudaStreamWaitEvent(kv->rs, kv->ev_fork, 0));
-        {
-            TimedScope ts(kv, kv->rs, tc ? kTChunkMma : kTDecodeRes, (uint64_t)R_eff * kv->page_bytes);
-            KVS_CK(kv, tc ? launch_chunk_mma(d, &kv->map_res, ns, kv->rs) : launch_decode(d, &kv->map_res, ns, kv->rs));
+        KVS_CK(kv, cudaStreamWaitEvent(rstream, kv->ev_fork, 0));
+        // Stream capture: the copy stream joins a capture once, from the
+        // caller's stream; events recorded outside the current capture are not
+        // waited on (the graph runs after all earlier work on the caller's
+        // stream, and every earlier ring copy is consumed before its merge).
+        // After a capture, the first plain call orders the copy stream after
+        // the caller's stream once, since events recorded inside a capture
+        // carry no ordering outside it.
+        if (cap) {
+            if (kv->cs_cap != cap && S > 0) {
+                KVS_CK(kv, cudaStreamWaitEvent(kv->cs, kv->ev_fork, 0));
+                kv->cs_cap = cap;
+            }
+            kv->capture_seen = true;
+        } else if (kv->capture_seen) {
+            KVS_CK(kv, cudaStreamWaitEvent(kv->cs, kv->ev_fork, 0));
+            kv->capture_seen = false;
+            kv->cs_cap = 0;
+            for (int gi = 0; gi < kv->n_groups; ++gi)
+                if (kv->free_cap[gi]) kv->free_valid[gi] = 0;
+            for (int li = 0; li < c.n_layers; ++li)
+                if (kv->hist_cap[li]) kv->hist_cap[li] = 0;
         }
-        KVS_CK(kv, cudaEventRecord(kv->ev_res, kv->rs));
+        {
+            TimedScope ts(kv, rstream, tc ? kTChunkMma : kTDecodeRes, (uint64_t)R_eff * kv->page_bytes);
+            KVS_CK(kv, tc ? launch_chunk_mma(d, &kv->map_res, ns, rstream) : launch_decode(d, &kv->map_res, ns, rstream));
+        }
+        KVS_CK(kv, cudaEventRecord(kv->ev_res, rstream));
         kv->stats.kernel_launches++;
         split_base += ns;
         kv->stats.bytes_resident_read += (uint64_t)R_eff * kv->page_bytes;
@@ -751,21 +800,22 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     if (S > 0) {
         if (c.n_ring_slots == 0) return fail(kv, KVS_E_INVAL, "internal: streamed pages without a ring");
         if (ls.hist_recorded && ls.pending_min_page < S) {
-            KVS_CK(kv, cudaStreamWaitEvent(kv->cs, kv->ev_hist[layer], 0));
+            if (kv->hist_cap[layer] == cap) KVS_CK(kv, cudaStreamWaitEvent(kv->cs, kv->ev_hist[layer], 0));
             ls.pending_min_page = INT_MAX;
         }
         const int chunk = c.chunk_pages;
-        KVS_CK(kv, cudaStreamWaitEvent(kv->xs, kv->ev_fork, 0));
+        KVS_CK(kv, cudaStreamWaitEvent(xstream, kv->ev_fork, 0));
         for (long i0 = 0; i0 < S; i0 += chunk) {
             const int cpages = (int)std::min<long>(chunk, S - i0);
             const int gidx = (int)(kv->ring_ctr % kv->n_groups);
             kv->ring_ctr++;
-            if (kv->free_valid[gidx]) KVS_CK(kv, cudaStreamWaitEvent(kv->cs, kv->ev_free[gidx], 0));
+            if (kv->free_valid[gidx] && kv->free_cap[gidx] == cap)
+                KVS_CK(kv, cudaStreamWaitEvent(kv->cs, kv->ev_free[gidx], 0));
             uint8_t* dst = kv->ring + (size_t)gidx * chunk * kv->page_bytes;
             const uint8_t* src = kv->host + ((size_t)layer * kv->P_max + (size_t)i0) * kv->page_bytes;
             KVS_CK(kv, cudaMemcpyAsync(dst, src, (size_t)cpages * kv->page_bytes, cudaMemcpyHostToDevice, kv->cs));
             KVS_CK(kv, cudaEventRecord(kv->ev_full[gidx], kv->cs));
-            KVS_CK(kv, cudaStreamWaitEvent(kv->xs, kv->ev_full[gidx], 0));
+            KVS_CK(kv, cudaStreamWaitEvent(xstream, kv->ev_full[gidx], 0));
             d.region = kv->ring;
             d.region_slot_base = 0;
             d.region_slots = c.n_ring_slots;
@@ -776,19 +826,20 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
             d.split_base = split_base;
             const int ns = (2 * cpages + d.stages_per_split - 1) / d.stages_per_split;
             {
-                TimedScope ts(kv, kv->xs, tc ? kTChunkMma : kTDecodeRing, (uint64_t)cpages * kv->page_bytes);
-                KVS_CK(kv, tc ? launch_chunk_mma(d, &kv->map_ring, ns, kv->xs)
-                              : launch_decode(d, &kv->map_ring, ns, kv->xs));
+                TimedScope ts(kv, xstream, tc ? kTChunkMma : kTDecodeRing, (uint64_t)cpages * kv->page_bytes);
+                KVS_CK(kv, tc ? launch_chunk_mma(d, &kv->map_ring, ns, xstream)
+                              : launch_decode(d, &kv->map_ring, ns, xstream));
             }
             kv->stats.kernel_launches++;
-            KVS_CK(kv, cudaEventRecord(kv->ev_free[gidx], kv->xs));
+            KVS_CK(kv, cudaEventRecord(kv->ev_free[gidx], xstream));
             kv->free_valid[gidx] = 1;
+            kv->free_cap[gidx] = cap;
             split_base += ns;
             kv->stats.pages_streamed += cpages;
             kv->stats.bytes_h2d += (uint64_t)cpages * kv->page_bytes;
             kv->stats.h2d_copies++;
         }
-        KVS_CK(kv, cudaEventRecord(kv->ev_ring, kv->xs));
+        KVS_CK(kv, cudaEventRecord(kv->ev_ring, xstream));
         KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_ring, 0));
     }
 
@@ -933,6 +984,36 @@ int kvs_measure_h2d(kvs_t* kv, size_t chunk_bytes, size_t total_bytes, int reps,
     cudaEventDestroy(b);
     *gbs = best;
     return KVS_OK;
+}
+
+int kvs_selftest_bounded_wait(int device, double limit_s, int* err_bits) {
+    if (!err_bits || limit_s <= 0 || limit_s > 10) return fail(nullptr, KVS_E_INVAL, "bad argument");
+    int n_dev = 0;
+    if (cudaGetDeviceCount(&n_dev) != cudaSuccess || device < 0 || device >= n_dev) {
+        cudaGetLastError();
+        return fail(nullptr, KVS_E_INVAL, "no such CUDA device");
+    }
+    DeviceGuard g(device);
+    int* d_err = nullptr;
+    KVS_CK(nullptr, cudaMalloc(reinterpret_cast<void**>(&d_err), sizeof(int)));
+    cudaStream_t st = nullptr;
+    cudaEvent_t done = nullptr;
+    int rc = KVS_OK;
+    if (cudaMemset(d_err, 0, sizeof(int)) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&done, cudaEventDisableTiming) != cudaSuccess ||
+        launch_wait_selftest(d_err, (uint64_t)(limit_s * 1e9), st) != cudaSuccess ||
+        cudaEventRecord(done, st) != cudaSuccess) {
+        rc = fail(nullptr, KVS_E_CUDA, "self-test launch failed");
+    } else {
+        rc = wait_event(nullptr, done, limit_s + 30.0);
+        if (rc == KVS_OK && cudaMemcpy(err_bits, d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+            rc = fail(nullptr, KVS_E_CUDA, "self-test readback failed");
+    }
+    if (done) cudaEventDestroy(done);
+    if (st) cudaStreamDestroy(st);
+    cudaFree(d_err);
+    return rc;
 }
 
 const char* kvs_last_error(kvs_t* kv) {

@@ -36,7 +36,8 @@ ERROR_NAMES = {0: "KVS_OK", -1: "KVS_E_INVAL", -2: "KVS_E_ARENA", -3: "KVS_E_WID
 EXPORTS = ["kvs_resolve_config", "kvs_page_bytes", "kvs_plan_page", "kvs_create", "kvs_destroy",
            "kvs_append", "kvs_attend", "kvs_export_page", "kvs_page_location", "kvs_layer_length",
            "kvs_get_config", "kvs_get_stats", "kvs_reset_stats", "kvs_set_profiling", "kvs_sync",
-           "kvs_measure_h2d", "kvs_attend_pages_static", "kvs_last_error"]
+           "kvs_measure_h2d", "kvs_attend_pages_static", "kvs_selftest_bounded_wait",
+           "kvs_last_error"]
 
 
 class kvs_config(ctypes.Structure):
@@ -92,6 +93,7 @@ def _load():
     L.kvs_sync.argtypes = [vp, vp, ctypes.c_double]
     L.kvs_measure_h2d.argtypes = [vp, ctypes.c_size_t, ctypes.c_size_t, i, cp(ctypes.c_double)]
     L.kvs_attend_pages_static.argtypes = [vp, i, i, i, i, i, i, vp, vp, vp, vp]
+    L.kvs_selftest_bounded_wait.argtypes = [i, ctypes.c_double, cp(i)]
     L.kvs_last_error.restype = ctypes.c_char_p
     L.kvs_last_error.argtypes = [vp]
     return L
@@ -228,6 +230,15 @@ def kvs_attend_pages_static(pages, n_pages, n_tokens, n_q_heads, n_kv_heads, pos
     """No-allocation attention over caller-owned device pages (see include/kvs.h)."""
     _check(lib.kvs_attend_pages_static(_addr(pages), n_pages, n_tokens, n_q_heads, n_kv_heads, pos0,
                                        n_q, _addr(q), _addr(out), _addr(lse), _stream(stream)))
+
+
+KVS_ERR_WAIT_TIMEOUT = 1
+
+
+def kvs_selftest_bounded_wait(device: int = 0, limit_s: float = 0.2) -> int:
+    bits = ctypes.c_int()
+    _check(lib.kvs_selftest_bounded_wait(device, limit_s, ctypes.byref(bits)))
+    return bits.value
 
 
 def kvs_last_error(h=None) -> str:

@@ -214,6 +214,14 @@ int kvs_attend_pages_static(const void* pages, int n_pages, int n_tokens, int n_
                             int n_kv_heads, int pos0, int n_q, const void* q_f16, float* out,
                             float* lse, void* stream);
 
+/* Failure-detection self-test: launch one GPU thread that waits, through the
+ * same bounded mbarrier wait every libkvs kernel uses, on a barrier phase that
+ * nothing completes.  The wait gives up after limit_s seconds (0 < limit_s <=
+ * 10) and records KVS_ERR_WAIT_TIMEOUT in the error word, which is returned in
+ * *err_bits; the device stays usable.  Needs no handle. */
+#define KVS_ERR_WAIT_TIMEOUT 1
+int kvs_selftest_bounded_wait(int device, double limit_s, int* err_bits);
+
 /* Last error text of the handle (or of the calling thread's last failed
  * kvs_create / pure call when kv is NULL). */
 const char* kvs_last_error(kvs_t* kv);

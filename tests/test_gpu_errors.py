@@ -66,3 +66,31 @@ def test_create_rejections(kvs):
     with pytest.raises(kvs.KvsError) as e:
         kvs.kvs_create(kvs.make_config(1, 8, 2, 1000), 99)
     assert e.value.code == kvs.KVS_E_INVAL
+
+
+def test_device_bounded_wait_gives_up(kvs):
+    """A kernel wait that nothing completes ends after its limit with the
+    timeout bit set; the device stays usable."""
+    t = torch()
+    bits = kvs.kvs_selftest_bounded_wait(0, 0.2)
+    assert bits & kvs.KVS_ERR_WAIT_TIMEOUT
+    x = t.ones(1024, device="cuda")
+    assert float((x * 2).sum().item()) == 2048.0
+
+
+def test_host_sync_timeout_then_recovers(kvs):
+    """kvs_sync's host wait is bounded: a stream still busy returns KVS_E_TIMEOUT;
+    waiting longer succeeds."""
+    t = torch()
+    cfg = kvs.make_config(1, 8, 2, 1024, n_resident_pages=4, n_ring_slots=0)
+    h = kvs.kvs_create(cfg, 0)
+    try:
+        s = t.cuda.Stream()
+        with t.cuda.stream(s):
+            t.cuda._sleep(1 << 31)  # about a second of GPU clock cycles
+        with pytest.raises(kvs.KvsError) as e:
+            kvs.kvs_sync(h, s, 0.01)
+        assert e.value.code == kvs.KVS_E_TIMEOUT
+        kvs.kvs_sync(h, s, 60.0)
+    finally:
+        kvs.kvs_destroy(h)
