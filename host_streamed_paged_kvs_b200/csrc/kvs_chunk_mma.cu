@@ -111,8 +111,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5;
     const int h = blockIdx.y;
     const int rows_head = a.n_q * a.group;
-    const int st0 = blockIdx.x * a.stages_per_split;
-    const int n_st = min(a.stages_per_split, 2 * a.n_units - st0);
+    const int st0 = (int)(((long)blockIdx.x * 2 * a.n_units) / a.n_splits);
+    const int n_st = (int)(((long)(blockIdx.x + 1) * 2 * a.n_units) / a.n_splits) - st0;
 
     if (warp == 0) {
         tmem_alloc(tmem_slot, kTmemCols);

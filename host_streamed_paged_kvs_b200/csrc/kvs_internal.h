@@ -60,7 +60,8 @@ struct DecodeArgs {
     int slot0;               // region slot of unit 0
     int page0;               // absolute page index of unit 0
     int n_units;             // pages in this launch (consumed as 2 half-page stages each)
-    int stages_per_split;    // half-page stages per split
+    int n_splits;            // splits of this launch; split s covers half-page stages
+                             // [s*T/n_splits, (s+1)*T/n_splits) of the T = 2*n_units stages
     int split_base;          // first split index written by this launch
     int len;                 // tokens in the history
     int pos0, n_q;           // query positions pos0 .. pos0+n_q-1

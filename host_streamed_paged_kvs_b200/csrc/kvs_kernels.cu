@@ -127,21 +127,25 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
 // ----------------------------------------------------------------------------
 // K2: split-K flash-decode.  CTA = (split, kv head, row group), 256 threads.
 // The pages of one launch are consumed as 128-token half-page stages; a split
-// is a run of `stages_per_split` consecutive stages.  Stage bytes land in
-// shared memory through TMA: the K quants with the 128-byte swizzle (a thread
-// reading its key's row then hits distinct banks while the query chunk it
-// multiplies is a broadcast), the K scales, V codes and V scales as 1-D bulk
-// copies; three stages are in flight.
-//   QK^T : two threads per key, 64 dims each; K dequantized in registers
-//          (exact int8 -> fp32), per-block scale applied to the block's partial.
-//   softmax: online, log2 domain, CTA-wide running max per row; the V scale of
-//          each (key, block) is folded into the probability, p' = p * d_v.
-//   PV   : warp = 16 keys, lane = 4 dims x all rows.
-// Output per split: (m, l) and acc[128] for every query row of the CTA.
+// is an equal share of consecutive stages (the launch's n_splits splits).
+// Stage bytes land in shared memory through TMA: the K quants with the
+// 128-byte swizzle (a thread reading its key's row then hits distinct banks
+// while the query chunk it multiplies is a broadcast), the K scales, V codes
+// and V scales as 1-D bulk copies; three stages are in flight.  Every warp
+// owns 16 keys of each stage end to end, with its own online-softmax state:
+//   QK^T : two lanes per key, 64 dims each; K dequantized in registers (exact
+//          int8 -> fp32), the per-block scale applied to the block partial;
+//   softmax: warp-local running max per row (log2 domain); the V scale of each
+//          (key, block) folded into the probability, p' = p * d_v;
+//   PV   : lane = 4 dims x all rows over the warp's 16 keys.
+// A stage buffer is refilled once all eight warps have released it (an
+// mbarrier with eight arrivals); there is no CTA-wide barrier in the loop.  At
+// the end the eight warps' (m, l, acc) are merged into the split's partial.
 // ----------------------------------------------------------------------------
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kStageKeys = 128;
+constexpr int kWarpKeys = kStageKeys / kWarps;                    // 16
 constexpr int kStageKq = 0;
 constexpr int kStageKd = kStageKeys * kHeadDim;                  // 16384
 constexpr int kStageVq = kStageKd + kStageKeys * kBlocks * 2;      // 17408
@@ -150,38 +154,52 @@ constexpr int kStageBytes = kStageVd + kStageKeys * kBlocks * 2;   // 26624
 constexpr int kStages = 3;
 constexpr int kMaxRows = 8;
 constexpr int kQHalf = 68;                  // floats per (row, half): 64 + 4 pad (bank offset)
+// per-warp p' records [block][16 keys][PR], block stride padded so the two
+// lanes of a key and four consecutive keys store into distinct banks
+constexpr int kPWBlock = kWarpKeys * kMaxRows + 8;                 // 136 floats (PR = 8)
 constexpr size_t kOffQ = kStages * kStageBytes;
-constexpr size_t kOffP = kOffQ + kMaxRows * 2 * kQHalf * 4;                 // sQ
-constexpr size_t kOffMax = kOffP + kStageKeys * kBlocks * kMaxRows * 4;     // sP
-constexpr size_t kOffL = kOffMax + kWarps * kMaxRows * 4;
-constexpr size_t kOffBar = kOffL + kWarps * kMaxRows * 4;
-constexpr size_t kDecodeSmem = 1024 /*align slack*/ + kOffBar + kStages * 8;
+constexpr size_t kOffP = kOffQ + kMaxRows * 2 * kQHalf * 4;                    // sQ
+constexpr size_t kOffKend = kOffP + (size_t)kWarps * kBlocks * kPWBlock * 4;   // sP
+constexpr size_t kOffBar = kOffKend + kMaxRows * 4;                              // sKend
+constexpr size_t kDecodeSmem = 1024 /*align slack*/ + kOffBar + 2 * kStages * 8;
 static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-B swizzle alignment");
-static_assert(kWarps * kMaxRows * kHeadDim * 4 <= kStages * kStageBytes, "reduction scratch fits");
+static_assert(kWarps * kMaxRows * (kHeadDim + 2) * 4 <= kStages * kStageBytes, "merge scratch fits");
 
 size_t decode_smem_bytes() { return kDecodeSmem; }
+
+// 2^x with the hardware approximation (flush-to-zero; 2^-inf = 0)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 template <int ROWS>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap) {
-    constexpr int PR = ROWS <= 4 ? 4 : 8;  // padded rows of a p' record
+    constexpr int PR = ROWS <= 4 ? 4 : 8;          // padded rows of a p' record
+    constexpr int SB = kWarpKeys * PR + 8;           // block stride of a warp's p' area (floats)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* stage = smem;
     float* sQ = reinterpret_cast<float*>(smem + kOffQ);    // [ROWS][2][kQHalf]
-    float* sP = reinterpret_cast<float*>(smem + kOffP);    // [128 keys][4 blocks][PR]
-    float* sMax = reinterpret_cast<float*>(smem + kOffMax);  // [warps][8]
-    float* sL = reinterpret_cast<float*>(smem + kOffL);      // [warps][8]
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    int* sKend = reinterpret_cast<int*>(smem + kOffKend);           // last visible key per row
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);   // [kStages]
+    uint64_t* empty = full + kStages;                               // [kStages]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float* sPw = reinterpret_cast<float*>(smem + kOffP) + warp * kBlocks * kPWBlock;  // this warp's p'
     const int h = blockIdx.y;
     const int row_begin = blockIdx.z * ROWS;
     const int rows_here = min(ROWS, a.n_q * a.group - row_begin);
     const int n_stages_all = 2 * a.n_units;
-    const int st0 = blockIdx.x * a.stages_per_split;
-    const int n_st = min(a.stages_per_split, n_stages_all - st0);
+    const int st0 = (int)(((long)blockIdx.x * n_stages_all) / a.n_splits);
+    const int n_st = (int)(((long)(blockIdx.x + 1) * n_stages_all) / a.n_splits) - st0;
 
     // queries of this CTA's rows, pre-scaled into the log2 domain
     for (int idx = tid; idx < ROWS * kHeadDim; idx += kThreads) {
@@ -194,12 +212,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         sQ[(r * 2 + (d >> 6)) * kQHalf + (d & 63)] = v;
     }
-    int qpos[ROWS];
-#pragma unroll
-    for (int r = 0; r < ROWS; ++r) qpos[r] = (r < rows_here) ? a.pos0 + (row_begin + r) / a.group : -1;
+    if (tid < ROWS)  // row r sees keys 0 .. min(len-1, its query position); padding rows none
+        sKend[tid] = (tid < rows_here) ? min(a.len - 1, a.pos0 + (row_begin + tid) / a.group) : -1;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&bar[s], 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kWarps);
+        }
         fence_mbar_init();
     }
     __syncthreads();
@@ -210,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int slot = (a.slot0 + u) % a.region_slots;
         const uint8_t* ph = a.region + ((size_t)slot * a.n_kv + h) * kPageHeadBytes;
         uint8_t* dst = stage + (i % kStages) * kStageBytes;
-        uint64_t* b = &bar[i % kStages];
+        uint64_t* b = &full[i % kStages];
         mbar_expect_tx(b, kStageBytes);
         const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * kPageHeadRows + half * kStageKeys;
         tma_load_2d(dst + kStageKq, &kmap, 0, krow, b);
@@ -218,8 +238,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         bulk_load(dst + kStageVq, ph + kOffVq + half * (kStageKeys * kHeadDim / 2), kStageKeys * kHeadDim / 2, b);
         bulk_load(dst + kStageVd, ph + kOffVd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
     };
+    int next_issue = 0;
     if (tid == 0) {
-        for (int i = 0; i < kStages && i < n_st; ++i) issue(i);
+        for (; next_issue < kStages && next_issue < n_st; ++next_issue) issue(next_issue);
     }
 
     float m_run[ROWS], l_run[ROWS], acc[ROWS][4];
@@ -229,25 +250,37 @@ __global__ void __launch_bounds__(kThreads, 2)
         l_run[r] = 0.0f;
         acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.0f;
     }
-    const int key = tid >> 1, hf = tid & 1;   // QK / softmax role
+    const int kl = lane >> 1, hf = lane & 1;  // QK / softmax role: key kl of the warp, dim half hf
+    const int key = warp * kWarpKeys + kl;     // key within the stage
     const int vb = lane >> 3, vi = lane & 7;  // PV role: block and byte pair of this lane
     bool ok = true;
 
     for (int i = 0; i < n_st; ++i) {
+        // producer: keep the next two stages in flight (thread 0 waits for all
+        // warps to release the buffer it refills)
+        if (tid == 0) {
+            for (; next_issue < n_st && next_issue < i + kStages; ++next_issue) {
+                const int prev = next_issue - kStages;  // last stage that used this buffer
+                if (prev >= 0 && !mbar_wait_bounded(&empty[prev % kStages], (prev / kStages) & 1, a.err)) {
+                    ok = false;
+                    break;
+                }
+                issue(next_issue);
+            }
+        }
         const uint8_t* sb = stage + (i % kStages) * kStageBytes;
-        if (!mbar_wait_bounded(&bar[i % kStages], (i / kStages) & 1, a.err)) ok = false;
-        ok = __syncthreads_and(ok);
-        if (!ok) break;
+        if (!mbar_wait_bounded(&full[i % kStages], (i / kStages) & 1, a.err)) ok = false;
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         const int sg = st0 + i;
         const int kpos = (a.page0 + (sg >> 1)) * kPageTokens + (sg & 1) * kStageKeys + key;
 
-        // ---- QK^T: this thread's key, dims [64 hf, 64 hf + 64) ----
+        // ---- QK^T: this lane's key, dims [64 hf, 64 hf + 64) ----
         float s[ROWS];
 #pragma unroll
         for (int r = 0; r < ROWS; ++r) s[r] = 0.0f;
         const uint8_t* krow = sb + kStageKq + key * kHeadDim;
         const float* qh = sQ + hf * kQHalf;
-#pragma unroll
+#pragma unroll 1
         for (int bb = 0; bb < 2; ++bb) {
             const int blk = 2 * hf + bb;
             float part[ROWS];
@@ -279,64 +312,59 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int r = 0; r < ROWS; ++r) s[r] = fmaf(kd, part[r], s[r]);
         }
+
+        // ---- warp-local online softmax; p' = p * d_v for this lane's two blocks ----
+        // The reference max m_run only moves when some score of the warp
+        // exceeds it by more than 2^8 (one warp vote per row in the common
+        // case); probabilities are then at most 2^8, exact enough in fp32.
+        const __half2 dv2 = *reinterpret_cast<const __half2*>(sb + kStageVd + key * (kBlocks * 2) + hf * 4);
+        const float dva = __low2float(dv2), dvb = __high2float(dv2);
+        float pa[PR], pb[PR];
+#pragma unroll
+        for (int r = 0; r < PR; ++r) pa[r] = pb[r] = 0.0f;
 #pragma unroll
         for (int r = 0; r < ROWS; ++r) {
             s[r] += __shfl_xor_sync(0xffffffffu, s[r], 1);
-            if (kpos >= a.len || kpos > qpos[r]) s[r] = -CUDART_INF_F;
-            float mx = s[r];
+            if (kpos > sKend[r]) s[r] = -CUDART_INF_F;
+            if (__any_sync(0xffffffffu, s[r] > m_run[r] + 8.0f)) {
+                float mx = s[r];
 #pragma unroll
-            for (int off = 2; off <= 16; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            if (lane == 0) sMax[warp * kMaxRows + r] = mx;
+                for (int off = 2; off <= 16; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                const float mn = fmaxf(m_run[r], mx);
+                const float alpha = ex2_approx(m_run[r] - mn);  // 0 when m_run was -inf
+                m_run[r] = mn;
+                l_run[r] *= alpha;
+                acc[r][0] *= alpha; acc[r][1] *= alpha;
+                acc[r][2] *= alpha; acc[r][3] *= alpha;
+            }
+            const float mu = (m_run[r] == -CUDART_INF_F) ? 0.0f : m_run[r];
+            const float p = ex2_approx(s[r] - mu);
+            pa[r] = p * dva;
+            pb[r] = p * dvb;
+            if (!hf) l_run[r] += p;  // this lane's share of the row sum (reduced once at the end)
         }
-        __syncthreads();
-        // the previous stage's buffer is free once every thread has passed this barrier
-        if (tid == 0 && i >= 1 && i - 1 + kStages < n_st) issue(i - 1 + kStages);
+        {
+            float* pdst_a = sPw + (2 * hf) * SB + kl * PR;
+            float* pdst_b = sPw + (2 * hf + 1) * SB + kl * PR;
+#pragma unroll
+            for (int r4 = 0; r4 < PR; r4 += 4) {
+                *reinterpret_cast<float4*>(pdst_a + r4) = make_float4(pa[r4], pa[r4 + 1], pa[r4 + 2], pa[r4 + 3]);
+                *reinterpret_cast<float4*>(pdst_b + r4) = make_float4(pb[r4], pb[r4 + 1], pb[r4 + 2], pb[r4 + 3]);
+            }
+        }
+        __syncwarp();
 
-        // ---- online softmax; p' = p * d_v for this thread's two blocks ----
-        float alpha[ROWS];
-        const __half2 dv2 = *reinterpret_cast<const __half2*>(sb + kStageVd + key * (kBlocks * 2) + hf * 4);
-        const float dva = __low2float(dv2), dvb = __high2float(dv2);
-        float* pdst = sP + (key * kBlocks + 2 * hf) * PR;
-#pragma unroll
-        for (int r = 0; r < ROWS; ++r) {
-            float mx = sMax[r];
-#pragma unroll
-            for (int ww = 1; ww < kWarps; ++ww) mx = fmaxf(mx, sMax[ww * kMaxRows + r]);
-            const float mn = fmaxf(m_run[r], mx);
-            const float mu = (mn == -CUDART_INF_F) ? 0.0f : mn;
-            alpha[r] = exp2f(m_run[r] - mu);
-            m_run[r] = mn;
-            const float p = exp2f(s[r] - mu);
-            pdst[r] = p * dva;
-            pdst[PR + r] = p * dvb;
-            float ps = hf ? 0.0f : p;
-#pragma unroll
-            for (int off = 2; off <= 16; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-            if (lane == 0) sL[warp * kMaxRows + r] = ps;
-        }
-        __syncthreads();
-
-        // ---- PV: warp = 16 keys, lane = dims {32b+2i, +1, +16, +17} ----
-#pragma unroll
-        for (int r = 0; r < ROWS; ++r) {
-            float ls = 0.0f;
-#pragma unroll
-            for (int ww = 0; ww < kWarps; ++ww) ls += sL[ww * kMaxRows + r];
-            l_run[r] = fmaf(l_run[r], alpha[r], ls);
-            acc[r][0] *= alpha[r]; acc[r][1] *= alpha[r];
-            acc[r][2] *= alpha[r]; acc[r][3] *= alpha[r];
-        }
-        const uint8_t* vq_base = sb + kStageVq + vb * 16 + 2 * vi;
-        const float* p_base = sP + vb * PR;
+        // ---- PV over the warp's 16 keys: lane = dims {32b+2i, +1, +16, +17} ----
+        const uint8_t* vq_base = sb + kStageVq + (warp * kWarpKeys) * 64 + vb * 16 + 2 * vi;
+        const float* p_base = sPw + vb * SB;
 #pragma unroll 4
-        for (int kk = 0; kk < 16; ++kk) {
-            const int key2 = warp * 16 + kk;
-            const uint32_t code = *reinterpret_cast<const uint16_t*>(vq_base + key2 * 64);
+        for (int kk = 0; kk < kWarpKeys; ++kk) {
+            const uint32_t code = *reinterpret_cast<const uint16_t*>(vq_base + kk * 64);
             const float v0 = q4_to_f(code & 0xFu);          // dim 32b+2i
             const float v2 = q4_to_f((code >> 4) & 0xFu);   // dim 32b+2i+16
             const float v1 = q4_to_f((code >> 8) & 0xFu);   // dim 32b+2i+1
             const float v3 = q4_to_f((code >> 12) & 0xFu);  // dim 32b+2i+17
-            const float* pr = p_base + key2 * kBlocks * PR;
+            const float* pr = p_base + kk * PR;
             float pv[PR];
             *reinterpret_cast<float4*>(pv) = *reinterpret_cast<const float4*>(pr);
             if (PR == 8) *reinterpret_cast<float4*>(pv + 4) = *reinterpret_cast<const float4*>(pr + 4);
@@ -348,40 +376,50 @@ __global__ void __launch_bounds__(kThreads, 2)
                 acc[r][3] = fmaf(pv[r], v3, acc[r][3]);
             }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[i % kStages]);  // this warp is done with the stage
     }
+    ok = __syncthreads_and(ok);
     if (!ok) return;  // a bounded wait gave up; the error word is set
 
-    // ---- reduce the warps' partial sums and write the split's result ----
-    __syncthreads();  // stage buffers are reused as scratch
-    float* red = reinterpret_cast<float*>(stage);  // [warps][ROWS][128]
+    // ---- merge the eight warps' (m, l, acc) into the split's partial ----
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r)
+#pragma unroll
+        for (int off = 1; off <= 16; off <<= 1) l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], off);
+    float* red = reinterpret_cast<float*>(stage);          // [warps][ROWS][128]
+    float* sml = red + kWarps * ROWS * kHeadDim;           // [warps][ROWS][2]
     const int d0 = vb * 32 + 2 * vi;
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
         float* dst = red + (warp * ROWS + r) * kHeadDim;
         *reinterpret_cast<float2*>(dst + d0) = make_float2(acc[r][0], acc[r][1]);
         *reinterpret_cast<float2*>(dst + d0 + 16) = make_float2(acc[r][2], acc[r][3]);
+        if (lane == 0) {
+            sml[(warp * ROWS + r) * 2] = m_run[r];
+            sml[(warp * ROWS + r) * 2 + 1] = l_run[r];
+        }
     }
     __syncthreads();
     const int split_g = a.split_base + blockIdx.x;
     for (int idx = tid; idx < rows_here * kHeadDim; idx += kThreads) {
         const int r = idx / kHeadDim, d = idx - r * kHeadDim;
-        float v = 0.0f;
+        float M = -CUDART_INF_F;
 #pragma unroll
-        for (int ww = 0; ww < kWarps; ++ww) v += red[(ww * ROWS + r) * kHeadDim + d];
+        for (int ww = 0; ww < kWarps; ++ww) M = fmaxf(M, sml[(ww * ROWS + r) * 2]);
+        const float mu = (M == -CUDART_INF_F) ? 0.0f : M;
+        float v = 0.0f, L = 0.0f;
+#pragma unroll
+        for (int ww = 0; ww < kWarps; ++ww) {
+            const float wgt = ex2_approx(sml[(ww * ROWS + r) * 2] - mu);
+            v = fmaf(wgt, red[(ww * ROWS + r) * kHeadDim + d], v);
+            L = fmaf(wgt, sml[(ww * ROWS + r) * 2 + 1], L);
+        }
         const int lr = row_begin + r;
         const int j = lr / a.group, g = lr - j * a.group;
         const int grow = j * a.n_qh + h * a.group + g;
         a.part.acc[((size_t)split_g * a.n_rows + grow) * kHeadDim + d] = v;
-    }
-    if (tid < ROWS && tid < rows_here) {
-        float mr = 0.0f, lr_ = 0.0f;
-#pragma unroll
-        for (int rr = 0; rr < ROWS; ++rr)
-            if (rr == tid) { mr = m_run[rr]; lr_ = l_run[rr]; }
-        const int lrow = row_begin + tid;
-        const int j = lrow / a.group, g = lrow - j * a.group;
-        const int grow = j * a.n_qh + h * a.group + g;
-        a.part.ml[(size_t)split_g * a.n_rows + grow] = make_float2(mr, lr_);
+        if (d == 0) a.part.ml[(size_t)split_g * a.n_rows + grow] = make_float2(M, L);
     }
 }
 

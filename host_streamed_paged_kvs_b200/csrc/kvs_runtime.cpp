@@ -80,36 +80,35 @@ int m_tiles(const kvs_config& c, int n_q) { return (n_q * (c.n_q_heads / c.n_kv_
 // about two waves over the resident pages (the kernel holds one CTA per SM).
 constexpr int kSms = 148;
 
-int res_stages_per_split(const kvs_config& c, long R_eff, int n_q) {
+// Splits of the resident launch and of one ring-chunk launch (each split is an
+// equal share of the launch's half-page stages).
+int res_splits(const kvs_config& c, long R_eff, int n_q) {
     const long stages = 2 * R_eff;
     if (use_tensor_cores(c, n_q)) {
         const long per_split = (long)c.n_kv_heads * m_tiles(c, n_q);
-        const long want = std::min(stages, std::max(1L, (2L * kSms + per_split - 1) / per_split));
-        return (int)std::max(1L, (stages + want - 1) / want);
+        return (int)std::min(stages, std::max(1L, (2L * kSms + per_split - 1) / per_split));
     }
-    if (wide_regime(c, n_q)) return (int)std::max(1L, (stages + 7) / 8);
-    const long sps = stages * c.n_kv_heads / kTargetCtas;
-    return (int)std::min(4L, std::max(1L, sps));
+    if (wide_regime(c, n_q)) return (int)std::min(stages, 8L);
+    // CUDA-core decode: one wave of two CTAs per SM
+    const long per_split = (long)c.n_kv_heads * ((n_q * (c.n_q_heads / c.n_kv_heads) + 7) / 8);
+    return (int)std::min(stages, std::max(1L, (long)kTargetCtas / per_split));
 }
 
-int ring_stages_per_split(const kvs_config& c, int n_q, int chunk_pages) {
+int ring_splits(const kvs_config& c, int n_q, int chunk_pages) {
     const int stages = 2 * chunk_pages;
     if (use_tensor_cores(c, n_q)) {
         const int per_split = c.n_kv_heads * m_tiles(c, n_q);
-        const int want = std::min(stages, std::max(1, (kSms + per_split - 1) / per_split));
-        return std::max(1, (stages + want - 1) / want);
+        return std::min(stages, std::max(1, (kSms + per_split - 1) / per_split));
     }
-    return wide_regime(c, n_q) ? stages : 1;
+    return wide_regime(c, n_q) ? 1 : stages;
 }
 
 long count_splits(const kvs_config& c, int n_q, long R_eff, long S) {
-    const int sps_res = res_stages_per_split(c, R_eff, n_q);
-    long n = (2 * R_eff + sps_res - 1) / sps_res;
+    long n = res_splits(c, R_eff, n_q);
     if (S > 0 && c.chunk_pages > 0) {
-        const int sps_ring = ring_stages_per_split(c, n_q, c.chunk_pages);
         const long full = S / c.chunk_pages, tail = S % c.chunk_pages;
-        n += full * ((2 * c.chunk_pages + sps_ring - 1) / sps_ring);
-        if (tail) n += (2 * tail + sps_ring - 1) / sps_ring;
+        n += full * ring_splits(c, n_q, c.chunk_pages);
+        if (tail) n += ring_splits(c, n_q, (int)tail);
     }
     return n;
 }
@@ -760,9 +759,9 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         d.slot0 = (int)(first_res % R);
         d.page0 = (int)first_res;
         d.n_units = (int)R_eff;
-        d.stages_per_split = res_stages_per_split(c, R_eff, n_q);
+        const int ns = res_splits(c, R_eff, n_q);
+        d.n_splits = ns;
         d.split_base = split_base;
-        const int ns = (int)((2 * R_eff + d.stages_per_split - 1) / d.stages_per_split);
         KVS_CK(kv, cudaEventRecord(kv->ev_fork, s));
         KVS_CK(kv, cudaStreamWaitEvent(rstream, kv->ev_fork, 0));
         // Stream capture: the copy stream joins a capture once, from the
@@ -822,9 +821,9 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
             d.slot0 = gidx * chunk;
             d.page0 = (int)i0;
             d.n_units = cpages;
-            d.stages_per_split = ring_stages_per_split(c, n_q, chunk);
+            const int ns = ring_splits(c, n_q, cpages);
+            d.n_splits = ns;
             d.split_base = split_base;
-            const int ns = (2 * cpages + d.stages_per_split - 1) / d.stages_per_split;
             {
                 TimedScope ts(kv, xstream, tc ? kTChunkMma : kTDecodeRing, (uint64_t)cpages * kv->page_bytes);
                 KVS_CK(kv, tc ? launch_chunk_mma(d, &kv->map_ring, ns, xstream)

@@ -116,7 +116,7 @@ extern "C" int kvs_attend_pages_static(const void* pages, int n_pages, int n_tok
     d.slot0 = 0;
     d.page0 = 0;
     d.n_units = used_pages;
-    d.stages_per_split = sps;
+    d.n_splits = n_splits;
     d.split_base = 0;
     d.len = n_tokens;
     d.pos0 = pos0;
