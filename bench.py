@@ -35,6 +35,30 @@ METRIC = "streamed decode-attn KV tokens/s/layer; % of max(HBM,H2D) roofline, 1x
 UNIT = "KV tokens/s/layer"
 
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# the ncu captures summarized under profiles/.  A figure is used only for the
+# workload it was captured on and only while the kernel source is unchanged
+# (sha256 prefix of the .cu file); otherwise traffic is reported as null.
+NCU_TRAFFIC = {
+    "decode_kernel": {"src": "kvs_kernels.cu", "sha": "166b16890a75f30f",
+                      "workload": "streamed_decode_32k", "resident": 27297280, "ring": 1737984},
+    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "50c6d2c13826a107",
+                         "workload": "prefill_chunk_64k", "resident": 29949440, "ring": 6068992},
+}
+
+
+def ncu_traffic(kernel: str, workload: str, n_resident: int, n_ring: int):
+    import hashlib
+    t = NCU_TRAFFIC.get(kernel)
+    if not t or t["workload"] != workload or n_resident + n_ring == 0:
+        return None
+    path = os.path.join(ROOT, "host_streamed_paged_kvs_b200", "csrc", t["src"])
+    with open(path, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != t["sha"]:
+            return None
+    return (n_resident * t["resident"] + n_ring * t["ring"]) / (n_resident + n_ring)
+
+
 def reduce_max(x: float, dist=None, device=None) -> float:
     """Max of a per-rank time over all ranks (no-op for a single process)."""
     if dist is None:
@@ -348,7 +372,10 @@ def run_gpu(args, w: W.Workload):
             bytes_k = st_prof["bytes_decode_resident"] + st_prof["bytes_decode_ring"]
             achieved = bytes_k / (ms_dec * 1e-3) / 1e9
             kernel = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                      "frac": achieved / hbm_peak, "traffic": None, "kernel": "decode_kernel",
+                      "frac": achieved / hbm_peak,
+                      "traffic": ncu_traffic("decode_kernel", w.name, st_prof["n_decode_resident"],
+                                             st_prof["n_decode_ring"]),
+                      "kernel": "decode_kernel",
                       "launches": n_dec, "avg_launch_us": ms_dec / n_dec * 1e3,
                       "bytes_per_launch": bytes_k / n_dec,
                       "resident_only": {
@@ -361,8 +388,11 @@ def run_gpu(args, w: W.Workload):
             flops = prof_steps * L * 4.0 * w.n_q_heads * 128 * vis
             achieved = flops / (ms_tc * 1e-3) / 1e12
             tc_peak = peak_tflops()
+            n_res_l = prof_steps * L
             kernel = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                      "frac": achieved / tc_peak, "traffic": None, "kernel": "chunk_mma_kernel",
+                      "frac": achieved / tc_peak,
+                      "traffic": ncu_traffic("chunk_mma_kernel", w.name, n_res_l, n_tc - n_res_l),
+                      "kernel": "chunk_mma_kernel",
                       "launches": n_tc, "avg_launch_us": ms_tc / n_tc * 1e3,
                       "flops_per_launch": flops / n_tc,
                       "peak_note": "measured dense bf16 burst; fp16 has the same nominal rate"}

@@ -91,6 +91,27 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// 2^x on the FMA pipe, so that half of the softmax exponentials leave the
+// XU pipe (which the MUFU exponentials and fp16 packing saturate): x = n + f
+// with n the nearest integer (1.5 * 2^23 rounding trick) and f in [-0.5, 0.5];
+// 2^f from a degree-5 polynomial fitted by weighted least squares (Lawson
+// iterations) to 2^f on [-0.5, 0.5], max relative error 2.4e-7 in binary32;
+// 2^n added to the exponent field.  x <= -127 gives +0.
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -127.0f);
+    const float rn = x + 12582912.0f;
+    const float n = rn - 12582912.0f;
+    const float f = x - n;
+    float p = 0.001327646430581808f;
+    p = fmaf(p, f, 0.009675540961325169f);
+    p = fmaf(p, f, 0.05550713464617729f);
+    p = fmaf(p, f, 0.24022120237350464f);
+    p = fmaf(p, f, 0.6931469440460205f);
+    p = fmaf(p, f, 1.0000001192092896f);
+    const int e = __float_as_int(rn) - 0x4B400000;
+    return __int_as_float(__float_as_int(p) + (e << 23));
+}
+
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 
@@ -299,7 +320,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int e = 0; e < 64; e += 2) {
                 const float p0 = ex2_approx(fmaf(v[e], a.q_scale, -mu));      // 2^-inf = 0
-                const float p1 = ex2_approx(fmaf(v[e + 1], a.q_scale, -mu));
+                const float p1 = exp2_poly(fmaf(v[e + 1], a.q_scale, -mu));
                 l_part += p0 + p1;
                 pk[e >> 1] = h2u(__floats2half2_rn(p0, p1));
             }

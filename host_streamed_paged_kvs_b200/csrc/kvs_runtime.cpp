@@ -85,8 +85,15 @@ constexpr int kSms = 148;
 int res_splits(const kvs_config& c, long R_eff, int n_q) {
     const long stages = 2 * R_eff;
     if (use_tensor_cores(c, n_q)) {
-        const long per_split = (long)c.n_kv_heads * m_tiles(c, n_q);
-        return (int)std::min(stages, std::max(1L, (2L * kSms + per_split - 1) / per_split));
+        // one CTA per SM: pick the split count that minimizes waves x stages
+        // per split on a full machine (ties -> fewer splits, fewer partials)
+        const long units = (long)c.n_kv_heads * m_tiles(c, n_q);
+        long best = 1, best_cost = -1;
+        for (long sp = 1; sp <= std::min(stages, 32L); ++sp) {
+            const long cost = ((units * sp + kSms - 1) / kSms) * ((stages + sp - 1) / sp);
+            if (best_cost < 0 || cost < best_cost) { best = sp; best_cost = cost; }
+        }
+        return (int)best;
     }
     if (wide_regime(c, n_q)) return (int)std::min(stages, 8L);
     // CUDA-core decode: one wave of two CTAs per SM
@@ -97,8 +104,10 @@ int res_splits(const kvs_config& c, long R_eff, int n_q) {
 int ring_splits(const kvs_config& c, int n_q, int chunk_pages) {
     const int stages = 2 * chunk_pages;
     if (use_tensor_cores(c, n_q)) {
-        const int per_split = c.n_kv_heads * m_tiles(c, n_q);
-        return std::min(stages, std::max(1, (kSms + per_split - 1) / per_split));
+        // at most one wave, leaving SMs to the resident launch when a chunk's
+        // units cannot fill the machine twice
+        const int units = c.n_kv_heads * m_tiles(c, n_q);
+        return std::min(stages, std::max(1, kSms / units));
     }
     return wide_regime(c, n_q) ? 1 : stages;
 }
