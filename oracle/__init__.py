@@ -42,36 +42,40 @@ def build(force: bool = False) -> str:
 _lib = None
 
 
+def bind(L):
+    """Declare the C prototypes on a loaded oracle library and return it."""
+    u16p = ctypes.POINTER(ctypes.c_uint16)
+    u8p = ctypes.POINTER(ctypes.c_uint8)
+    f64p = ctypes.POINTER(ctypes.c_double)
+    L.oracle_half_to_double.restype = ctypes.c_double
+    L.oracle_half_to_double.argtypes = [ctypes.c_uint16]
+    L.oracle_float_to_half.restype = ctypes.c_uint16
+    L.oracle_float_to_half.argtypes = [ctypes.c_float]
+    L.oracle_q8_0_block.argtypes = [u16p, u8p]
+    L.oracle_q4_0_block.argtypes = [u16p, u8p]
+    L.oracle_dequant_q8_0.argtypes = [u8p, f64p]
+    L.oracle_dequant_q4_0.argtypes = [u8p, f64p]
+    L.oracle_quantize_rows.argtypes = [ctypes.c_int, ctypes.c_int, u16p, u16p, u8p, u8p]
+    L.oracle_attention.restype = ctypes.c_int
+    L.oracle_attention.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, u8p, u8p,
+                                   ctypes.c_int, ctypes.c_int, u16p, f64p, f64p]
+    L.oracle_pages_for.restype = ctypes.c_long
+    L.oracle_pages_for.argtypes = [ctypes.c_long, ctypes.c_int]
+    L.oracle_auto_resident_pages.restype = ctypes.c_long
+    L.oracle_auto_resident_pages.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_long,
+                                             ctypes.c_int]
+    L.oracle_page_location.restype = ctypes.c_int
+    L.oracle_page_location.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_long,
+                                       ctypes.c_long, ctypes.POINTER(ctypes.c_int),
+                                       ctypes.POINTER(ctypes.c_long)]
+    return L
+
+
 def lib():
     global _lib
     if _lib is None:
         build()
-        L = ctypes.CDLL(_LIB)
-        u16p = ctypes.POINTER(ctypes.c_uint16)
-        u8p = ctypes.POINTER(ctypes.c_uint8)
-        f64p = ctypes.POINTER(ctypes.c_double)
-        L.oracle_half_to_double.restype = ctypes.c_double
-        L.oracle_half_to_double.argtypes = [ctypes.c_uint16]
-        L.oracle_float_to_half.restype = ctypes.c_uint16
-        L.oracle_float_to_half.argtypes = [ctypes.c_float]
-        L.oracle_q8_0_block.argtypes = [u16p, u8p]
-        L.oracle_q4_0_block.argtypes = [u16p, u8p]
-        L.oracle_dequant_q8_0.argtypes = [u8p, f64p]
-        L.oracle_dequant_q4_0.argtypes = [u8p, f64p]
-        L.oracle_quantize_rows.argtypes = [ctypes.c_int, ctypes.c_int, u16p, u16p, u8p, u8p]
-        L.oracle_attention.restype = ctypes.c_int
-        L.oracle_attention.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, u8p, u8p,
-                                       ctypes.c_int, ctypes.c_int, u16p, f64p, f64p]
-        L.oracle_pages_for.restype = ctypes.c_long
-        L.oracle_pages_for.argtypes = [ctypes.c_long, ctypes.c_int]
-        L.oracle_auto_resident_pages.restype = ctypes.c_long
-        L.oracle_auto_resident_pages.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_long,
-                                                 ctypes.c_int]
-        L.oracle_page_location.restype = ctypes.c_int
-        L.oracle_page_location.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_long,
-                                           ctypes.c_long, ctypes.POINTER(ctypes.c_int),
-                                           ctypes.POINTER(ctypes.c_long)]
-        _lib = L
+        _lib = bind(ctypes.CDLL(_LIB))
     return _lib
 
 

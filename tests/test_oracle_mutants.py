@@ -1,0 +1,87 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a copy of oracle/kvs_oracle.c (on the CPU,
+never in the product), builds it, points the oracle binding at it, and runs
+the pin tests: at least one of them must fail.  The real oracle passes them.
+"""
+import ctypes
+import os
+import shutil
+import subprocess
+
+import pytest
+
+import oracle
+import test_oracle_attention as TA
+import test_oracle_fp16 as TF
+import test_oracle_pages as TP
+import test_oracle_quant as TQ
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "kvs_oracle.c")
+HDR = os.path.join(os.path.dirname(oracle.__file__), "kvs_oracle.h")
+
+MUTANTS = {
+    "q8 ties to even": ("q = (int)roundf(x[i] / d);", "q = (int)rintf(x[i] / d);"),
+    "q8 scale /128": ("float d = amax / 127.0f;", "float d = amax / 128.0f;"),
+    "q4 last index wins": ("if (a > amax) { /* strict", "if (a >= amax) { /* strict"),
+    "q4 offset 8.0": ("(int)(x[i] / d + 8.5f)", "(int)(x[i] / d + 8.0f)"),
+    "q4 nibble order": ("(uint8_t)(q[j] | (q[j + 16] << 4))", "(uint8_t)((q[j] << 4) | q[j + 16])"),
+    "q4 dequant offset": ("(int)(blk[2 + j] & 0x0f) - 8)", "(int)(blk[2 + j] & 0x0f) - 7)"),
+    "scale 1/d": ("double scale = 1.0 / sqrt((double)dim);", "double scale = 1.0 / (double)dim;"),
+    "causal off by one": ("int n_keys = pos0 + j + 1;", "int n_keys = pos0 + j;"),
+    "gqa interleaved": ("int g = h / group;", "int g = h % n_kv;"),
+    "lse base 2": ("lse[(size_t)j * n_qh + h] = m + log(sum);", "lse[(size_t)j * n_qh + h] = m + log2(sum);"),
+    "fp16 ties down": ("if (rem > 0x1000u || (rem == 0x1000u && (hm & 1u))) {", "if (rem > 0x1000u) {"),
+    "resident window": ("if (page >= P - n_resident) {", "if (page > P - n_resident) {"),
+    "auto floor": ("long floor_pages = (2048 + page_tokens - 1) / page_tokens;",
+                   "long floor_pages = (4096 + page_tokens - 1) / page_tokens;"),
+}
+
+
+def pins():
+    return [
+        TQ.test_q8_0_hand_worked, TQ.test_q4_0_hand_worked, TQ.test_zero_block,
+        lambda: TQ.test_constant_block(1.0), lambda: TQ.test_single_nonzero(7, -2.5),
+        TQ.test_q4_0_error_bound_and_range,
+        TA.test_two_key_closed_form_pins_scale, TA.test_gqa_grouping_is_contiguous,
+        TA.test_zero_query_is_uniform_mean_with_causal_lengths, TA.test_against_scipy_softmax_random,
+        TA.test_single_key_returns_its_value,
+        TP.test_auto_resident_matches_printed_numbers, TP.test_auto_resident_floor_and_ceiling,
+        lambda: TP.test_page_location_invariants(1025, 4),
+        TF.test_float_to_half_random,
+    ]
+
+
+def run_pins():
+    failures = 0
+    for pin in pins():
+        try:
+            pin()
+        except AssertionError:
+            failures += 1
+    return failures
+
+
+def test_real_oracle_passes_its_pins():
+    assert run_pins() == 0
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not found: {old}"
+    d = tmp_path / "m"
+    d.mkdir()
+    shutil.copy(HDR, d / "kvs_oracle.h")
+    (d / "kvs_oracle.c").write_text(src.replace(old, new))
+    so = str(d / "libmutant.so")
+    subprocess.run(["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+                    "-o", so, str(d / "kvs_oracle.c"), "-lm"], check=True)
+    real = oracle.lib()
+    try:
+        oracle._lib = oracle.bind(ctypes.CDLL(so))
+        caught = run_pins()
+    finally:
+        oracle._lib = real
+    assert caught >= 1, f"no pin caught the mutant '{name}'"
