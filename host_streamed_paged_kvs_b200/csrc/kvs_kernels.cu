@@ -524,8 +524,62 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const MergeArgs a)
     }
 }
 
+// Many query rows (verify / prefill chunks): one warp per row, lane = 4 dims,
+// four splits in flight per lane; M first, then the weighted sums.
+__global__ void __launch_bounds__(256) merge_rows_kernel(const MergeArgs a) {
+    const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= a.n_rows) return;
+    const float2* ml = a.part.ml + row;
+    float m = -CUDART_INF_F;
+    for (int s = lane; s < a.n_splits; s += 32) m = fmaxf(m, ml[(size_t)s * a.n_rows].x);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const float* accp = a.part.acc + (size_t)row * kHeadDim + 4 * lane;
+    const size_t sstride = (size_t)a.n_rows * kHeadDim;
+    float L = 0.0f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    int s = 0;
+    for (; s + 3 < a.n_splits; s += 4) {
+        float2 mls[4];
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            mls[u] = ml[(size_t)(s + u) * a.n_rows];
+            v[u] = *reinterpret_cast<const float4*>(accp + (size_t)(s + u) * sstride);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (mls[u].y > 0.0f) {
+                const float w = exp2f(mls[u].x - m);
+                L = fmaf(w, mls[u].y, L);
+                o.x = fmaf(w, v[u].x, o.x); o.y = fmaf(w, v[u].y, o.y);
+                o.z = fmaf(w, v[u].z, o.z); o.w = fmaf(w, v[u].w, o.w);
+            }
+        }
+    }
+    for (; s < a.n_splits; ++s) {
+        const float2 mlv = ml[(size_t)s * a.n_rows];
+        if (mlv.y > 0.0f) {
+            const float4 v = *reinterpret_cast<const float4*>(accp + (size_t)s * sstride);
+            const float w = exp2f(mlv.x - m);
+            L = fmaf(w, mlv.y, L);
+            o.x = fmaf(w, v.x, o.x); o.y = fmaf(w, v.y, o.y);
+            o.z = fmaf(w, v.z, o.z); o.w = fmaf(w, v.w, o.w);
+        }
+    }
+    const float inv = 1.0f / L;
+    *reinterpret_cast<float4*>(a.out + (size_t)row * kHeadDim + 4 * lane) =
+        make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+    if (lane == 0 && a.lse) a.lse[row] = (m + log2f(L)) * 0.69314718055994530942f;
+}
+
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s) {
-    merge_kernel<<<dim3(a.n_rows, kHeadDim / 32), kMergeThreads, 0, s>>>(a);
+    if (a.n_rows >= 1024) {
+        merge_rows_kernel<<<(a.n_rows + 7) / 8, 256, 0, s>>>(a);
+    } else {
+        merge_kernel<<<dim3(a.n_rows, kHeadDim / 32), kMergeThreads, 0, s>>>(a);
+    }
     return cudaGetLastError();
 }
 
