@@ -168,6 +168,26 @@ def oracle_layer_step(w: W.Workload, layer: int = 0, prepared=None):
     return time.perf_counter() - t0, prepared
 
 
+def oracle_step_threaded(w: W.Workload, prepared, threads: int) -> float:
+    """Wall time of the oracle over a whole step's attention, the (layer, kv
+    head) problems spread over `threads` threads (the C oracle runs without the
+    GIL).  Every layer reuses the prepared layer's data: the same work per layer."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    kb, vb, ks, vs, q = prepared
+    G = w.n_q_heads // w.n_kv_heads
+    t0 = time.perf_counter()
+    kbs, vbs = oracle.quantize_rows(ks, vs)
+    kall = np.concatenate([kb, kbs])
+    vall = np.concatenate([vb, vbs])
+    parts = [(np.ascontiguousarray(kall[:, g:g + 1]), np.ascontiguousarray(vall[:, g:g + 1]),
+              np.ascontiguousarray(q[:, g * G:(g + 1) * G])) for g in range(w.n_kv_heads)]
+    jobs = [parts[g] for _ in range(w.n_layers) for g in range(w.n_kv_heads)]
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(lambda p: oracle.attention(p[0], p[1], p[2], w.pos0), jobs))
+    return time.perf_counter() - t0
+
+
 def cpu_baseline(w: W.Workload, budget_s: float = 15.0):
     secs, prep = oracle_layer_step(w)
     times = [secs]
@@ -175,7 +195,16 @@ def cpu_baseline(w: W.Workload, budget_s: float = 15.0):
         t, _ = oracle_layer_step(w, prepared=prep)
         times.append(t)
     per_layer = statistics.median(times)
+    threads = min(os.cpu_count() or 1, w.n_layers * w.n_kv_heads)
+    threaded = None
+    # all cores, only when one threaded step stays within the budget
+    if per_layer * w.n_layers / threads < budget_s:
+        ts = oracle_step_threaded(w, prep, threads)
+        threaded = {"value": w.ctx * w.n_layers / ts, "unit": UNIT, "threads": threads,
+                    "sample": f"one whole step of {w.name}: {w.n_layers} layers x {w.n_kv_heads} kv heads "
+                              f"as independent oracle calls on a pool of {threads} threads"}
     return {"value": w.ctx / per_layer, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "all_cores": threaded,
             "sample": f"{len(times)} x one layer's step of {w.name} (append {w.n_q} token(s), "
                       f"binary64 attention of {w.n_q}x{w.n_q_heads} query rows over {w.ctx} keys), "
                       f"single thread, median {per_layer:.2f} s"}
@@ -275,22 +304,48 @@ def run_gpu(args, w: W.Workload):
         one_step(ks, vs, qs, out, lse)
     barrier()
     kvs.kvs_reset_stats(h)
+    one_step(ks, vs, qs, out, lse)
+    barrier()
+    launches_per_step = int(kvs.kvs_get_stats(h)["kernel_launches"])
+
+    # one step (append + attend of every layer) captured into a CUDA graph; the
+    # library's copy stream and side streams join the capture
+    graph = None
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            one_step(ks, vs, qs, out, lse)
+        for _ in range(args.warmup):
+            with torch.cuda.stream(stream):
+                graph.replay()
+        barrier()
+
+    def timed_step():
+        if graph is not None:
+            with torch.cuda.stream(stream):
+                graph.replay()
+        else:
+            one_step(ks, vs, qs, out, lse)
+
+    kvs.kvs_reset_stats(h)
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.25)
     barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        one_step(ks, vs, qs, out, lse)
-    e1.record(stream)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    ev[0].record(stream)
+    for i in range(args.steps):
+        timed_step()
+        ev[i + 1].record(stream)
     barrier()
-    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_total = max_over_ranks(ev[0].elapsed_time(ev[-1]))
+    ms_median = statistics.median(ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps))
     clk = clocks.stop()
     st = kvs.kvs_get_stats(h)
+    gpu_launches = launches_per_step * args.steps
     ms_step = ms_total / args.steps
     value = job_value(world, w.ctx, L, ms_step)
+    e0, e1 = ev[0], ev[-1]
 
     # ---- end to end through the C ABI with pinned host buffers ----
     kh = [x.cpu().pin_memory() for x in ks]
@@ -353,6 +408,13 @@ def run_gpu(args, w: W.Workload):
     S = P - R
     t_roof = L * max(R * pb / (hbm_peak * 1e9), S * pb / (h2d_peak * 1e9))
     roof_frac = t_roof / (ms_step * 1e-3)
+    # the same bound with the copy bandwidth of ring-sized chunks (the most a
+    # ring of this many slots can be fed at), and the HBM term that also counts
+    # the ring's own write and read of every streamed page
+    t_roof_chunk = L * max(R * pb / (hbm_peak * 1e9), S * pb / (h2d_ring * 1e9)) if h2d_ring else t_roof
+    t_hbm_ring = L * (R + 2 * S) * pb / (hbm_peak * 1e9)
+    vis_keys = sum(w.pos0 + j + 1 for j in range(w.n_q))
+    step_flops = L * 4.0 * w.n_q_heads * 128 * vis_keys
 
     # dominant kernel (largest summed launch time in the profiled pass): the
     # split-K decode kernel (HBM-bound) or the tensor-core chunk kernel
@@ -415,15 +477,23 @@ def run_gpu(args, w: W.Workload):
                           "t_roof_ms": t_roof * 1e3, "t_step_ms": ms_step, "frac": roof_frac,
                           "h2d_gbs_peak_measured": h2d_peak, "h2d_gbs_ring_chunk": h2d_ring,
                           "h2d_gbs_achieved": L * S * pb / (ms_step * 1e-3) / 1e9,
+                          "frac_at_ring_chunk_h2d": t_roof_chunk / (ms_step * 1e-3),
+                          "hbm_ms_incl_ring_write_read": t_hbm_ring * 1e3,
+                          "tensor_ms_at_peak": step_flops / (peak_tflops() * 1e12) * 1e3,
+                          "step_flops": step_flops,
                           "hbm_gbs_peak": hbm_peak, "peak_source": peak_src},
         "e2e": {"value": world * w.ctx * L / (ms_e2e * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b, "ms_per_step": ms_e2e},
-        "gpu_launches": int(st["kernel_launches"]),
+        "gpu_launches": gpu_launches,
+        "launch": "cuda graph (one step captured, replayed)" if graph is not None else "eager",
+        "ms_per_step_median": ms_median,
         "clocks": clk,
         "prefill_s": prefill_s,
     }
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
+    del graph, timed_step
+    torch.cuda.synchronize(dev)
     kvs.kvs_destroy(h)
     if world > 1:
         dist.barrier()
@@ -442,6 +512,8 @@ def main():
     ap.add_argument("--chunk-pages", type=int, default=0)
     ap.add_argument("--no-profile", dest="profile", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", dest="graph", action="store_false",
+                    help="time plain calls instead of replays of a captured step")
     args = ap.parse_args()
     w = W.WORKLOADS[args.workload]
     if args.steps <= 0:

@@ -59,7 +59,10 @@ extern "C" {
 #define KVS_PAGE_STREAMED 2
 
 /* ---- flags --------------------------------------------------------------- */
-#define KVS_FLAG_PROFILE 1 /* record CUDA events around kernels (kvs_get_stats) */
+/* Record CUDA events around every kernel (kvs_get_stats).  Profiling runs all
+ * kernels on the caller's stream, one after another, so that the events time
+ * one kernel each; steps are slower than without it. */
+#define KVS_FLAG_PROFILE 1
 
 typedef struct kvs_config {
     int n_layers;         /* attention layers sharing the pool, auxiliary layers included (e.g. 16+1) */
