@@ -158,6 +158,23 @@ ArenaLayout arena_layout(const kvs_config& c) {
     return L;
 }
 
+ArenaLayout arena_layout_with(kvs_config c, long resident_pages) {
+    c.n_resident_pages = (int)resident_pages;
+    return arena_layout(c);
+}
+
+// the most resident pages per layer (at most P) whose arena fits in `budget`
+// bytes, 0 if none does.  The arena is not monotone in the resident count:
+// fewer resident pages mean more streamed chunks and so more split partials,
+// so the counts are tried from P down.
+long resident_fit(const kvs_config& c, size_t budget, long P) {
+    const size_t per_page = (size_t)c.n_layers * c.n_kv_heads * kPageHeadBytes;
+    const long top = std::min<long>(std::max(1L, P), (long)(budget / per_page));  // resident bytes alone
+    for (long r = top; r >= 1; --r)
+        if (arena_layout_with(c, r).total <= budget) return r;
+    return 0;
+}
+
 int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::string& why) {
     if (!in || !out) { why = "null config"; return KVS_E_INVAL; }
     kvs_config c = *in;
@@ -180,13 +197,7 @@ int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::stri
     }
     const size_t pb = (size_t)c.n_kv_heads * kPageHeadBytes;
     const long P = pages_for(c.max_ctx);
-    if (c.n_resident_pages == 0) c.n_resident_pages = (int)auto_resident(c.max_ctx, pb, c.n_layers);
-    if (c.n_resident_pages > P) c.n_resident_pages = (int)P;
     if (c.n_ring_slots == 0) {
-        if (c.n_resident_pages < P) {
-            why = fmt("all-resident mode (n_ring_slots=0) needs n_resident_pages >= %ld", P);
-            return KVS_E_INVAL;
-        }
         c.chunk_pages = 0;
     } else {
         if (c.chunk_pages == 0) c.chunk_pages = std::max(1, c.n_ring_slots / 2);
@@ -195,12 +206,32 @@ int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::stri
             return KVS_E_INVAL;
         }
     }
+    if (c.arena_bytes != 0 && c.arena_bytes < pb) {
+        why = fmt("arena %zu B is below the minimum stage of one page (%zu B)", c.arena_bytes, pb);
+        return KVS_E_ARENA;
+    }
+    if (c.n_resident_pages == 0) {
+        if (c.arena_bytes == 0) {
+            c.n_resident_pages = (int)auto_resident(c.max_ctx, pb, c.n_layers);
+        } else {
+            // a fixed arena: the resident pages get what the ring, the split
+            // partials and the staging leave (the decode KV grant of the arena)
+            const long fit = resident_fit(c, c.arena_bytes, P);
+            if (fit < 1) {
+                why = fmt("arena %zu B cannot hold any resident set besides ring + partials (%zu B with one page)",
+                          c.arena_bytes, arena_layout_with(c, 1).total);
+                return KVS_E_ARENA;
+            }
+            c.n_resident_pages = (int)fit;
+        }
+    }
+    if (c.n_resident_pages > P) c.n_resident_pages = (int)P;
+    if (c.n_ring_slots == 0 && c.n_resident_pages < P) {
+        why = fmt("all-resident mode (n_ring_slots=0) needs n_resident_pages >= %ld", P);
+        return KVS_E_INVAL;
+    }
     const ArenaLayout L = arena_layout(c);
     if (c.arena_bytes != 0) {
-        if (c.arena_bytes < pb) {
-            why = fmt("arena %zu B is below the minimum stage of one page (%zu B)", c.arena_bytes, pb);
-            return KVS_E_ARENA;
-        }
         if (c.arena_bytes < L.total) {
             why = fmt("arena %zu B cannot hold resident pages + ring + partials (%zu B)", c.arena_bytes, L.total);
             return KVS_E_ARENA;

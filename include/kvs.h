@@ -71,8 +71,10 @@ typedef struct kvs_config {
     int head_dim;         /* must be 128 */
     int page_tokens;      /* must be 256 */
     int max_ctx;          /* host history capacity in tokens per layer */
-    int n_resident_pages; /* resident pages per layer; 0 = auto (10 % of max_ctx, 8-page floor,
-                             8192 MiB ceiling over all layers) */
+    int n_resident_pages; /* resident pages per layer; 0 = auto: with arena_bytes = 0, 10 % of
+                             max_ctx (8-page floor, 8192 MiB ceiling over all layers); with a
+                             fixed arena_bytes, the most pages that fit beside the ring, the
+                             split partials and the staging (at most pages(max_ctx)) */
     int n_ring_slots;     /* device ring slots (pages); 0 = all-resident mode, which needs
                              n_resident_pages >= pages(max_ctx) */
     int max_q_tokens;     /* widest append / attend batch (1, 1+n_draft or a 256-token ubatch) */
@@ -81,7 +83,7 @@ typedef struct kvs_config {
     int chunk_pages;      /* pages per H2D copy; 0 = auto (n_ring_slots/2); must divide n_ring_slots */
     int flags;            /* KVS_FLAG_* */
     size_t arena_bytes;   /* device arena budget; 0 = exact fit; else must hold one page and all
-                             resident pages + ring + partials + staging */
+                             resident pages + ring + partials + staging (KVS_E_ARENA if not) */
 } kvs_config;
 
 typedef struct kvs_stats {

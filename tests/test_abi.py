@@ -89,6 +89,42 @@ def test_arena_fit_accepts_exact_size(kvs):
     assert r.arena_bytes >= (2 * 8 + 8) * 425984
 
 
+@pytest.mark.parametrize("layers,qh,kvh,ctx,ring,mq,budget_mib", [
+    (16, 32, 8, 32768, 8, 1, 400), (17, 40, 8, 131072, 16, 4, 2240), (1, 40, 8, 65536, 16, 256, 320),
+    (2, 8, 2, 4096, 2, 1, 64), (16, 32, 8, 32768, 8, 1, 100000),
+])
+def test_arena_budget_sizes_the_resident_set(kvs, layers, qh, kvh, ctx, ring, mq, budget_mib):
+    """n_resident_pages = 0 with a fixed arena: the most resident pages that
+    fit (one more would not, unless every page already is resident)."""
+    budget = budget_mib << 20
+    c = kvs.make_config(layers, qh, kvh, ctx, n_ring_slots=ring, max_q_tokens=mq, arena_bytes=budget)
+    r, _ = kvs.kvs_resolve_config(c)
+    R = r.n_resident_pages
+    P = oracle.pages_for(ctx)
+    assert 1 <= R <= P and r.arena_bytes <= budget
+
+    def need(n):
+        e = kvs.make_config(layers, qh, kvh, ctx, n_resident_pages=n, n_ring_slots=ring, max_q_tokens=mq)
+        return kvs.kvs_resolve_config(e)[0].arena_bytes
+
+    assert need(R) == r.arena_bytes
+    if R < P:
+        assert need(R + 1) > budget
+    # the resident bytes dominate: the grant is the arena minus ring, partials and staging
+    assert r.arena_bytes >= layers * R * kvs.kvs_page_bytes(r)
+
+
+@pytest.mark.parametrize("layers,qh,kvh,ctx,ring,mq,budget", [
+    (16, 32, 8, 32768, 8, 1, 8 * 425984),             # below ring + one resident page per layer
+    (1, 40, 8, 65536, 16, 256, 100 << 20),            # the 256-row split partials alone need more
+])
+def test_arena_budget_without_room_is_rejected(kvs, layers, qh, kvh, ctx, ring, mq, budget):
+    c = kvs.make_config(layers, qh, kvh, ctx, n_ring_slots=ring, max_q_tokens=mq, arena_bytes=budget)
+    with pytest.raises(kvs.KvsError) as e:
+        kvs.kvs_resolve_config(c)
+    assert e.value.code == kvs.KVS_E_ARENA
+
+
 def test_create_without_gpu_fails_loudly(kvs):
     import torch
     if torch.cuda.is_available():
