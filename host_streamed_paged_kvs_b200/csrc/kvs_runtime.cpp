@@ -533,6 +533,59 @@ int kvs_plan_page(const kvs_config* c, int n_tokens, int page, int* kind, int* i
     return plan_page(*c, n_tokens, page, kind, index);
 }
 
+int kvs_eject_init(kvs_eject_params* p, kvs_eject_state* s) {
+    if (!p || !s || p->keep_pages < 0 || p->reenable_pages < 0 || p->stable_decodes < 0 ||
+        p->capacity_pages < 0) {
+        g_last_error = "kvs_eject_init: null pointer or negative field";
+        return KVS_E_INVAL;
+    }
+    if (p->reenable_pages == 0) p->reenable_pages = 8;
+    if (p->stable_decodes == 0) p->stable_decodes = 4;
+    if (p->keep_pages == 0 && p->capacity_pages == 0) {
+        g_last_error = "kvs_eject_init: the threshold (keep_pages, else capacity_pages) is zero";
+        return KVS_E_INVAL;
+    }
+    s->draft_active = 1;
+    s->streak = 0;
+    return KVS_OK;
+}
+
+int kvs_eject_step(const kvs_eject_params* p, kvs_eject_state* s, int working_pages) {
+    if (!p || !s || working_pages < 0 || p->stable_decodes < 1 || p->reenable_pages < 0) {
+        g_last_error = "kvs_eject_step: bad arguments (call kvs_eject_init first)";
+        return KVS_E_INVAL;
+    }
+    const long threshold = p->keep_pages > 0 ? p->keep_pages : p->capacity_pages;
+    const bool cond = s->draft_active ? (working_pages > threshold)
+                                      : ((long)working_pages <= threshold - p->reenable_pages);
+    s->streak = cond ? s->streak + 1 : 0;
+    if (s->streak < p->stable_decodes) return 0;
+    s->draft_active = !s->draft_active;
+    s->streak = 0;
+    return 1;
+}
+
+int kvs_draft_capacity_pages(const kvs_config* cfg, size_t pinned_bytes, int* pages) {
+    if (!cfg || !pages) { g_last_error = "kvs_draft_capacity_pages: null argument"; return KVS_E_INVAL; }
+    if (cfg->arena_bytes == 0) {
+        g_last_error = "kvs_draft_capacity_pages: needs a fixed arena_bytes";
+        return KVS_E_INVAL;
+    }
+    if (pinned_bytes >= cfg->arena_bytes) {
+        g_last_error = "kvs_draft_capacity_pages: the pinned reservation fills the arena";
+        return KVS_E_ARENA;
+    }
+    kvs_config c = *cfg;
+    c.n_resident_pages = 0;
+    c.arena_bytes -= pinned_bytes;
+    kvs_config r;
+    std::string why;
+    const int rc = resolve(&c, &r, nullptr, why);
+    if (rc != KVS_OK) { g_last_error = why; return rc; }
+    *pages = r.n_resident_pages;
+    return KVS_OK;
+}
+
 int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
     if (!out) return fail(nullptr, KVS_E_INVAL, "kvs_create: null out");
     *out = nullptr;

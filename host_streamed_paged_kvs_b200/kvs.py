@@ -37,7 +37,7 @@ EXPORTS = ["kvs_resolve_config", "kvs_page_bytes", "kvs_plan_page", "kvs_create"
            "kvs_append", "kvs_attend", "kvs_export_page", "kvs_page_location", "kvs_layer_length",
            "kvs_get_config", "kvs_get_stats", "kvs_reset_stats", "kvs_set_profiling", "kvs_sync",
            "kvs_measure_h2d", "kvs_attend_pages_static", "kvs_selftest_bounded_wait",
-           "kvs_last_error"]
+           "kvs_last_error", "kvs_eject_init", "kvs_eject_step", "kvs_draft_capacity_pages"]
 
 
 class kvs_config(ctypes.Structure):
@@ -65,6 +65,15 @@ class kvs_stats(ctypes.Structure):
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+class kvs_eject_params(ctypes.Structure):
+    _fields_ = [("keep_pages", ctypes.c_int), ("reenable_pages", ctypes.c_int),
+                ("stable_decodes", ctypes.c_int), ("capacity_pages", ctypes.c_int)]
+
+
+class kvs_eject_state(ctypes.Structure):
+    _fields_ = [("draft_active", ctypes.c_int), ("streak", ctypes.c_int)]
 
 
 def _load():
@@ -96,6 +105,9 @@ def _load():
     L.kvs_selftest_bounded_wait.argtypes = [i, ctypes.c_double, cp(i)]
     L.kvs_last_error.restype = ctypes.c_char_p
     L.kvs_last_error.argtypes = [vp]
+    L.kvs_eject_init.argtypes = [cp(kvs_eject_params), cp(kvs_eject_state)]
+    L.kvs_eject_step.argtypes = [cp(kvs_eject_params), cp(kvs_eject_state), i]
+    L.kvs_draft_capacity_pages.argtypes = [cp(kvs_config), ctypes.c_size_t, cp(i)]
     return L
 
 
@@ -243,6 +255,27 @@ def kvs_selftest_bounded_wait(device: int = 0, limit_s: float = 0.2) -> int:
 
 def kvs_last_error(h=None) -> str:
     return lib.kvs_last_error(h).decode()
+
+
+def kvs_eject_init(keep_pages=0, reenable_pages=0, stable_decodes=0, capacity_pages=0):
+    """Returns (params with defaults filled, state with the draft active)."""
+    p = kvs_eject_params(keep_pages, reenable_pages, stable_decodes, capacity_pages)
+    s = kvs_eject_state()
+    _check(lib.kvs_eject_init(ctypes.byref(p), ctypes.byref(s)))
+    return p, s
+
+
+def kvs_eject_step(params: kvs_eject_params, state: kvs_eject_state, working_pages: int) -> bool:
+    """One decode batch; True when the draft was ejected or re-enabled."""
+    rc = lib.kvs_eject_step(ctypes.byref(params), ctypes.byref(state), int(working_pages))
+    _check(rc if rc < 0 else 0)
+    return rc == 1
+
+
+def kvs_draft_capacity_pages(cfg: kvs_config, pinned_bytes: int) -> int:
+    n = ctypes.c_int()
+    _check(lib.kvs_draft_capacity_pages(ctypes.byref(cfg), int(pinned_bytes), ctypes.byref(n)))
+    return n.value
 
 
 class KVS:

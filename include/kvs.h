@@ -120,6 +120,48 @@ size_t kvs_page_bytes(const kvs_config* cfg);
  * or KVS_PAGE_ABSENT.  The R most recent pages are resident. */
 int kvs_plan_page(const kvs_config* resolved, int n_tokens, int page, int* kind, int* index);
 
+/* ---- draft eject controller (pure host) ------------------------------------
+ * The dynamic draft eject of "llama.cpp adaptive KV streaming - spec fork
+ * notes" (Dynamic draft eject; Results): a pinned draft (an MTP block and its
+ * KV, or a DFlash2 draft) borrows part of the arena; the controller ejects it
+ * when the target's decode working set outgrows the eject threshold and
+ * re-enables it when the working set fits again, with hysteresis and a
+ * stability count.  The library runs no draft model: a serving loop calls
+ * kvs_eject_step once per decode batch and acts on the transitions. */
+typedef struct kvs_eject_params {
+    int keep_pages;      /* eject threshold, in 256-token pages per layer of the target's decode
+                            working set; 0 = capacity_pages (eject at streaming onset) */
+    int reenable_pages;  /* re-enable once the working set is this many pages below the
+                            threshold; 0 = default 8 */
+    int stable_decodes;  /* consecutive decode batches a transition condition must hold;
+                            0 = default 4 */
+    int capacity_pages;  /* draft-active decode capacity: resident pages per layer the arena
+                            holds with the draft pinned (kvs_draft_capacity_pages) */
+} kvs_eject_params;
+
+typedef struct kvs_eject_state {
+    int draft_active;    /* 1 while the draft is active */
+    int streak;          /* consecutive batches for which the transition condition held */
+} kvs_eject_state;
+
+/* Fill the defaults of zero fields of *p and start with the draft active.
+ * KVS_E_INVAL for null pointers, negative fields or a zero threshold. */
+int kvs_eject_init(kvs_eject_params* p, kvs_eject_state* s);
+
+/* One decode batch whose target working set is `working_pages` pages per
+ * layer.  Active: the draft is ejected after stable_decodes consecutive
+ * batches above the threshold.  Ejected: it is re-enabled after
+ * stable_decodes consecutive batches at or below threshold - reenable_pages.
+ * A batch that breaks the condition resets the streak.  Returns 1 when the
+ * state changed (*s tells which way), 0 when not, KVS_E_INVAL on bad input. */
+int kvs_eject_step(const kvs_eject_params* p, kvs_eject_state* s, int working_pages);
+
+/* The draft-active decode capacity: the most resident pages per layer that
+ * fit in the config's arena (arena_bytes > 0) once `pinned_bytes` are
+ * reserved for the draft ("what remains of the arena after the pinned
+ * reservation and the phase compute slab").  KVS_E_ARENA if none fit. */
+int kvs_draft_capacity_pages(const kvs_config* cfg, size_t pinned_bytes, int* pages);
+
 /* ---- handle lifecycle ----------------------------------------------------- */
 
 /* Allocate the pinned host history (n_layers * pages(max_ctx) pages, mapped
