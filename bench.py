@@ -262,18 +262,21 @@ def run_gpu(args, w: W.Workload):
     stream = torch.cuda.Stream(device=dev)
 
     # ---- history pre-fill (untimed) ----
+    def prefill_history(hh):
+        for layer in range(L):
+            pos = 0
+            while pos < w.pos0:
+                n = min(16384, w.pos0 - pos)
+                k, v = W.kv_tokens(w, layer, pos, pos + n)
+                kd = torch.from_numpy(k).to(dev)
+                vd = torch.from_numpy(v).to(dev)
+                with torch.cuda.stream(stream):
+                    kvs.kvs_append(hh, layer, pos, n, kd, vd, stream)
+                stream.synchronize()
+                pos += n
+
     t0 = time.time()
-    for layer in range(L):
-        pos = 0
-        while pos < w.pos0:
-            n = min(16384, w.pos0 - pos)
-            k, v = W.kv_tokens(w, layer, pos, pos + n)
-            kd = torch.from_numpy(k).to(dev)
-            vd = torch.from_numpy(v).to(dev)
-            with torch.cuda.stream(stream):
-                kvs.kvs_append(h, layer, pos, n, kd, vd, stream)
-            stream.synchronize()
-            pos += n
+    prefill_history(h)
     prefill_s = time.time() - t0
 
     # ---- per-step inputs resident in HBM ----
@@ -286,10 +289,11 @@ def run_gpu(args, w: W.Workload):
     out = torch.empty((L, w.n_q, w.n_q_heads, 128), dtype=torch.float32, device=dev)
     lse = torch.empty((L, w.n_q, w.n_q_heads), dtype=torch.float32, device=dev)
 
-    def one_step(k_in, v_in, q_in, o, l):
+    def one_step(k_in, v_in, q_in, o, l, hh=None):
+        hh = h if hh is None else hh
         for layer in range(L):
-            kvs.kvs_append(h, layer, w.pos0, w.n_q, k_in[layer], v_in[layer], stream)
-            kvs.kvs_attend(h, layer, w.pos0, w.n_q, q_in[layer], o[layer], l[layer], stream)
+            kvs.kvs_append(hh, layer, w.pos0, w.n_q, k_in[layer], v_in[layer], stream)
+            kvs.kvs_attend(hh, layer, w.pos0, w.n_q, q_in[layer], o[layer], l[layer], stream)
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -358,6 +362,34 @@ def run_gpu(args, w: W.Workload):
         del graph
         barrier()
 
+    # ---- zero-copy comparison arm: the same steps on a second handle whose
+    #      decode kernel reads the streamed pages in place from the mapped
+    #      pinned history (no ring copies) ----
+    zc_line = None
+    zc_ok = (w.n_q * (w.n_q_heads // w.n_kv_heads) <= 8 and rc.n_resident_pages < w.n_pages
+             and L * w.n_pages * pb <= (4 << 30))
+    if args.zero_copy_arm and zc_ok:
+        cz = kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx, n_resident_pages=w.n_resident_pages,
+                             n_ring_slots=w.n_ring_slots, max_q_tokens=w.n_q,
+                             chunk_pages=args.chunk_pages, flags=kvs.KVS_FLAG_ZERO_COPY)
+        hz = kvs.kvs_create(cz, local)
+        prefill_history(hz)
+        for _ in range(args.warmup):
+            one_step(ks, vs, qs, out, lse, hz)
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            one_step(ks, vs, qs, out, lse, hz)
+        e1.record(stream)
+        barrier()
+        ms_zc = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+        S_z = w.n_pages - rc.n_resident_pages
+        zc_line = {"ms_per_step": ms_zc, "value": job_value(world, w.ctx, L, ms_zc), "unit": UNIT,
+                   "h2d_gbs_achieved": L * S_z * pb / (ms_zc * 1e-3) / 1e9,
+                   "what": "same steps, streamed pages read in place from mapped pinned host "
+                           "memory by the decode kernel (16-byte asynchronous copies), no ring"}
+        kvs.kvs_destroy(hz)
+
     # ---- end to end through the C ABI with pinned host buffers ----
     kh = [x.cpu().pin_memory() for x in ks]
     vh = [x.cpu().pin_memory() for x in vs]
@@ -424,6 +456,8 @@ def run_gpu(args, w: W.Workload):
     # the ring's own write and read of every streamed page
     t_roof_chunk = L * max(R * pb / (hbm_peak * 1e9), S * pb / (h2d_ring * 1e9)) if h2d_ring else t_roof
     t_hbm_ring = L * (R + 2 * S) * pb / (hbm_peak * 1e9)
+    if zc_line:
+        zc_line["frac"] = t_roof / (zc_line["ms_per_step"] * 1e-3)
     vis_keys = sum(w.pos0 + j + 1 for j in range(w.n_q))
     step_flops = L * 4.0 * w.n_q_heads * 128 * vis_keys
 
@@ -498,6 +532,7 @@ def run_gpu(args, w: W.Workload):
         "gpu_launches": gpu_launches,
         "launch": "library calls issued by the host without waiting between steps",
         "graph": graph_line,
+        "zero_copy": zc_line,
         "ms_per_step_median": ms_median,
         "clocks": clk,
         "prefill_s": prefill_s,
@@ -524,6 +559,8 @@ def main():
     ap.add_argument("--chunk-pages", type=int, default=0)
     ap.add_argument("--no-profile", dest="profile", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-zero-copy-arm", dest="zero_copy_arm", action="store_false",
+                    help="skip the zero-copy comparison arm")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="skip the extra pass that times replays of a captured step")
     args = ap.parse_args()

@@ -85,6 +85,10 @@ struct MergeArgs {
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                           cudaStream_t s);
+// the same kernel reading the pages in place from mapped pinned host memory
+// (a.region = the history's device alias) with 16-byte asynchronous copies
+cudaError_t launch_decode_zero_copy(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
+                                    cudaStream_t s);
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s);
 // multi-token (verify / prefill chunk) attention on tcgen05 tensor cores; same
 // arguments and partial format as launch_decode

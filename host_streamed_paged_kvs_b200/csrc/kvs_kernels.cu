@@ -178,7 +178,20 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-template <int ROWS>
+// 16-byte asynchronous copy global -> shared (plain loads, no TMA), and an
+// arrival on an mbarrier once all of this thread's earlier copies landed
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// ZC = true: the pages are read in place from mapped pinned host memory (the
+// history) by warp 0's 16-byte asynchronous copies instead of TMA, one stage
+// = 1664 copies, 52 per lane, the K quants placed in the same 128-byte
+// swizzle the tensor map produces
+template <int ROWS, bool ZC>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap) {
     constexpr int PR = ROWS <= 4 ? 4 : 8;          // padded rows of a p' record
@@ -217,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], ZC ? 32 : 1);
             mbar_init(&empty[s], kWarps);
         }
         fence_mbar_init();
@@ -231,15 +244,38 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint8_t* ph = a.region + ((size_t)slot * a.n_kv + h) * kPageHeadBytes;
         uint8_t* dst = stage + (i % kStages) * kStageBytes;
         uint64_t* b = &full[i % kStages];
-        mbar_expect_tx(b, kStageBytes);
-        const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * kPageHeadRows + half * kStageKeys;
-        tma_load_2d(dst + kStageKq, &kmap, 0, krow, b);
-        bulk_load(dst + kStageKd, ph + kOffKd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
-        bulk_load(dst + kStageVq, ph + kOffVq + half * (kStageKeys * kHeadDim / 2), kStageKeys * kHeadDim / 2, b);
-        bulk_load(dst + kStageVd, ph + kOffVd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
+        if constexpr (ZC) {
+            // K quants: row r of the half page, 16-byte chunk k -> swizzled
+            const uint8_t* kq = ph + kOffKq + half * (kStageKeys * kHeadDim);
+#pragma unroll 4
+            for (int c = lane; c < kStageKeys * 8; c += 32) {
+                const int r = c >> 3, k = c & 7;
+                cp_async16(dst + kStageKq + r * 128 + ((k ^ (r & 7)) << 4), kq + r * 128 + k * 16);
+            }
+            const uint8_t* kd = ph + kOffKd + half * (kStageKeys * kBlocks * 2);
+            const uint8_t* vq = ph + kOffVq + half * (kStageKeys * kHeadDim / 2);
+            const uint8_t* vd = ph + kOffVd + half * (kStageKeys * kBlocks * 2);
+            for (int c = lane; c < kStageKeys * kBlocks * 2 / 16; c += 32) {
+                cp_async16(dst + kStageKd + c * 16, kd + c * 16);
+                cp_async16(dst + kStageVd + c * 16, vd + c * 16);
+            }
+#pragma unroll 4
+            for (int c = lane; c < kStageKeys * kHeadDim / 2 / 16; c += 32)
+                cp_async16(dst + kStageVq + c * 16, vq + c * 16);
+            cp_async_arrive(b);
+        } else {
+            mbar_expect_tx(b, kStageBytes);
+            const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * kPageHeadRows + half * kStageKeys;
+            tma_load_2d(dst + kStageKq, &kmap, 0, krow, b);
+            bulk_load(dst + kStageKd, ph + kOffKd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
+            bulk_load(dst + kStageVq, ph + kOffVq + half * (kStageKeys * kHeadDim / 2), kStageKeys * kHeadDim / 2, b);
+            bulk_load(dst + kStageVd, ph + kOffVd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
+        }
     };
+    // the producer: thread 0 (TMA), or all of warp 0 (zero-copy)
+    const bool producer = ZC ? (warp == 0) : (tid == 0);
     int next_issue = 0;
-    if (tid == 0) {
+    if (producer) {
         for (; next_issue < kStages && next_issue < n_st; ++next_issue) issue(next_issue);
     }
 
@@ -256,9 +292,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     bool ok = true;
 
     for (int i = 0; i < n_st; ++i) {
-        // producer: keep the next two stages in flight (thread 0 waits for all
+        // producer: keep the next two stages in flight (it waits for all
         // warps to release the buffer it refills)
-        if (tid == 0) {
+        if (producer) {
             for (; next_issue < n_st && next_issue < i + kStages; ++next_issue) {
                 const int prev = next_issue - kStages;  // last stage that used this buffer
                 if (prev >= 0 && !mbar_wait_bounded(&empty[prev % kStages], (prev / kStages) & 1, a.err)) {
@@ -423,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-template <int ROWS>
+template <int ROWS, bool ZC>
 static cudaError_t launch_decode_t(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                                    int n_row_groups, cudaStream_t s) {
     // the shared-memory opt-in is per device: remember which devices have it
@@ -431,30 +467,41 @@ static cudaError_t launch_decode_t(const DecodeArgs& a, const CUtensorMap* kmap,
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !(configured & (1ull << dev))) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<ROWS>,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<ROWS, ZC>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kDecodeSmem);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured |= 1ull << dev;
     }
     dim3 grid(n_splits, a.n_kv, n_row_groups);
-    decode_kernel<ROWS><<<grid, kThreads, kDecodeSmem, s>>>(a, *kmap);
+    decode_kernel<ROWS, ZC><<<grid, kThreads, kDecodeSmem, s>>>(a, *kmap);
     return cudaGetLastError();
+}
+
+template <bool ZC>
+static cudaError_t launch_decode_rows(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
+                                      cudaStream_t s) {
+    const int rows = a.n_q * a.group;
+    switch (rows) {
+        case 1: return launch_decode_t<1, ZC>(a, kmap, n_splits, 1, s);
+        case 2: return launch_decode_t<2, ZC>(a, kmap, n_splits, 1, s);
+        case 3: return launch_decode_t<3, ZC>(a, kmap, n_splits, 1, s);
+        case 4: return launch_decode_t<4, ZC>(a, kmap, n_splits, 1, s);
+        case 5: return launch_decode_t<5, ZC>(a, kmap, n_splits, 1, s);
+        case 6: return launch_decode_t<6, ZC>(a, kmap, n_splits, 1, s);
+        case 7: return launch_decode_t<7, ZC>(a, kmap, n_splits, 1, s);
+        default: return launch_decode_t<8, ZC>(a, kmap, n_splits, (rows + 7) / 8, s);
+    }
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                           cudaStream_t s) {
-    const int rows = a.n_q * a.group;
-    switch (rows) {
-        case 1: return launch_decode_t<1>(a, kmap, n_splits, 1, s);
-        case 2: return launch_decode_t<2>(a, kmap, n_splits, 1, s);
-        case 3: return launch_decode_t<3>(a, kmap, n_splits, 1, s);
-        case 4: return launch_decode_t<4>(a, kmap, n_splits, 1, s);
-        case 5: return launch_decode_t<5>(a, kmap, n_splits, 1, s);
-        case 6: return launch_decode_t<6>(a, kmap, n_splits, 1, s);
-        case 7: return launch_decode_t<7>(a, kmap, n_splits, 1, s);
-        default: return launch_decode_t<8>(a, kmap, n_splits, (rows + 7) / 8, s);
-    }
+    return launch_decode_rows<false>(a, kmap, n_splits, s);
+}
+
+cudaError_t launch_decode_zero_copy(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
+                                    cudaStream_t s) {
+    return launch_decode_rows<true>(a, kmap, n_splits, s);
 }
 
 // ----------------------------------------------------------------------------

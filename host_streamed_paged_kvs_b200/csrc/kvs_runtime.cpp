@@ -112,9 +112,21 @@ int ring_splits(const kvs_config& c, int n_q, int chunk_pages) {
     return wide_regime(c, n_q) ? 1 : stages;
 }
 
+// Zero-copy decode: one launch over all streamed pages, about one CTA per SM
+// (the resident launch shares the SMs), each split a run of half-page stages.
+bool zero_copy_decode(const kvs_config& c, int n_q) {
+    return (c.flags & KVS_FLAG_ZERO_COPY) && !use_tensor_cores(c, n_q);
+}
+int zc_splits(const kvs_config& c, long S, int n_q) {
+    const long per_split = (long)c.n_kv_heads * ((n_q * (c.n_q_heads / c.n_kv_heads) + 7) / 8);
+    return (int)std::min(2 * S, std::max(1L, (long)kSms / per_split));
+}
+
 long count_splits(const kvs_config& c, int n_q, long R_eff, long S) {
     long n = res_splits(c, R_eff, n_q);
-    if (S > 0 && c.chunk_pages > 0) {
+    if (S > 0 && zero_copy_decode(c, n_q)) {
+        n += zc_splits(c, S, n_q);
+    } else if (S > 0 && c.chunk_pages > 0) {
         const long full = S / c.chunk_pages, tail = S % c.chunk_pages;
         n += full * ring_splits(c, n_q, c.chunk_pages);
         if (tail) n += ring_splits(c, n_q, (int)tail);
@@ -888,8 +900,32 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         split_base += ns;
         kv->stats.bytes_resident_read += (uint64_t)R_eff * kv->page_bytes;
     }
-    // 2) streamed pages through the ring, in ascending page order
-    if (S > 0) {
+    // 2a) zero-copy: the decode kernel reads the streamed pages in place from
+    //     the mapped pinned history (no ring, no copy engine)
+    if (S > 0 && zero_copy_decode(c, n_q)) {
+        KVS_CK(kv, cudaStreamWaitEvent(xstream, kv->ev_fork, 0));
+        d.region = kv->host_dev + (size_t)layer * kv->P_max * kv->page_bytes;
+        d.region_slot_base = 0;
+        d.region_slots = (int)kv->P_max;
+        d.slot0 = 0;
+        d.page0 = 0;
+        d.n_units = (int)S;
+        const int ns = zc_splits(c, S, n_q);
+        d.n_splits = ns;
+        d.split_base = split_base;
+        {
+            TimedScope ts(kv, xstream, kTDecodeRing, (uint64_t)S * kv->page_bytes);
+            KVS_CK(kv, launch_decode_zero_copy(d, &kv->map_res, ns, xstream));
+        }
+        kv->stats.kernel_launches++;
+        split_base += ns;
+        kv->stats.pages_streamed += S;
+        kv->stats.bytes_h2d += (uint64_t)S * kv->page_bytes;
+        KVS_CK(kv, cudaEventRecord(kv->ev_ring, xstream));
+        KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_ring, 0));
+    }
+    // 2b) streamed pages through the ring, in ascending page order
+    else if (S > 0) {
         if (c.n_ring_slots == 0) return fail(kv, KVS_E_INVAL, "internal: streamed pages without a ring");
         if (ls.hist_recorded && ls.pending_min_page < S) {
             if (kv->hist_cap[layer] == cap) KVS_CK(kv, cudaStreamWaitEvent(kv->cs, kv->ev_hist[layer], 0));

@@ -28,6 +28,7 @@ KVS_PAGE_ABSENT = -1
 KVS_PAGE_RESIDENT = 1
 KVS_PAGE_STREAMED = 2
 KVS_FLAG_PROFILE = 1
+KVS_FLAG_ZERO_COPY = 2
 
 ERROR_NAMES = {0: "KVS_OK", -1: "KVS_E_INVAL", -2: "KVS_E_ARENA", -3: "KVS_E_WIDTH",
                -4: "KVS_E_ORDER", -5: "KVS_E_CUDA", -6: "KVS_E_TIMEOUT", -7: "KVS_E_NOMEM"}

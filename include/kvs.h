@@ -63,6 +63,13 @@ extern "C" {
  * kernels on the caller's stream, one after another, so that the events time
  * one kernel each; steps are slower than without it. */
 #define KVS_FLAG_PROFILE 1
+/* Zero-copy decode: single-row-group decode calls (n_q * n_q_heads/n_kv_heads
+ * <= 8) attend the streamed pages in place in the mapped pinned history, read
+ * by the SMs over PCIe, instead of copying them through the ring (the design
+ * the "Feature/adaptive kv stream integration" pull request's review found in
+ * its kernels).  Wider calls still use the ring, so a ring is still required
+ * when pages stream. */
+#define KVS_FLAG_ZERO_COPY 2
 
 typedef struct kvs_config {
     int n_layers;         /* attention layers sharing the pool, auxiliary layers included (e.g. 16+1) */

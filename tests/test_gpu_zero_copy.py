@@ -1,0 +1,79 @@
+"""Zero-copy decode (KVS_FLAG_ZERO_COPY): the decode kernel reads the streamed
+pages in place from the mapped pinned history instead of through the ring.
+Parity against the oracle, agreement with the ring path on the same inputs,
+and the ring still serving the calls too wide for the CUDA-core kernel."""
+import numpy as np
+import pytest
+
+from host_streamed_paged_kvs_b200 import workload as W
+from kvs_testlib import assert_close, make_cfg, oracle_step, prefill, step, torch
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kvs():
+    from host_streamed_paged_kvs_b200 import kvs as K
+    return K
+
+
+@pytest.mark.parametrize("ctx,heads,n_q,R,N", [
+    (5000, (32, 8), 1, 3, 4),     # ragged last page, GQA 4
+    (4097, (8, 1), 1, 2, 2),      # GQA 8: 8 rows per kv head
+    (2600, (16, 8), 2, 1, 2),     # two query tokens x GQA 2
+    (700, (8, 2), 1, 1, 2),       # three pages, two streamed
+])
+def test_zero_copy_matches_oracle_and_ring(kvs, ctx, heads, n_q, R, N):
+    w = W.Workload("zc", n_layers=2, n_q=n_q, n_q_heads=heads[0], n_kv_heads=heads[1], ctx=ctx,
+                   n_resident_pages=R, n_ring_slots=N, seed=41)
+    hz = kvs.kvs_create(make_cfg(w, flags=kvs.KVS_FLAG_ZERO_COPY), 0)
+    hr = kvs.kvs_create(make_cfg(w), 0)
+    try:
+        for layer in range(w.n_layers):
+            for h in (hz, hr):
+                prefill(h, w, layer, w.pos0)
+            oz, lz = step(hz, w, layer, w.pos0, n_q)
+            orr, lr = step(hr, w, layer, w.pos0, n_q)
+            assert_close(oz, lz, *oracle_step(w, layer, w.pos0, n_q))
+            # same arithmetic, other split layout: fp32 rounding apart only
+            assert np.allclose(oz, orr, rtol=0, atol=2e-5) and np.allclose(lz, lr, rtol=0, atol=2e-5)
+        st = kvs.kvs_get_stats(hz)
+        assert st["pages_streamed"] > 0 and st["h2d_copies"] == 0
+    finally:
+        kvs.kvs_destroy(hz)
+        kvs.kvs_destroy(hr)
+
+
+def test_wide_calls_keep_the_ring(kvs):
+    """A verify batch (4 tokens x GQA 5 = 20 rows) goes to the tensor-core
+    kernel through the ring even with zero-copy set."""
+    w = W.Workload("zcw", n_layers=1, n_q=4, n_q_heads=40, n_kv_heads=8, ctx=3000,
+                   n_resident_pages=2, n_ring_slots=4, seed=43)
+    h = kvs.kvs_create(make_cfg(w, flags=kvs.KVS_FLAG_ZERO_COPY), 0)
+    p0 = w.ctx - 10
+    try:
+        prefill(h, w, 0, p0)
+        out, lse = step(h, w, 0, p0, 4)
+        assert_close(out, lse, *oracle_step(w, 0, p0, 4))
+        assert kvs.kvs_get_stats(h)["h2d_copies"] > 0
+        # and a single-token decode on the same handle reads in place
+        kvs.kvs_reset_stats(h)
+        out1, lse1 = step(h, w, 0, p0 + 4, 1)
+        assert_close(out1, lse1, *oracle_step(w, 0, p0 + 4, 1))
+        assert kvs.kvs_get_stats(h)["h2d_copies"] == 0
+    finally:
+        kvs.kvs_destroy(h)
+
+
+def test_zero_copy_full_size_32k_layer(kvs):
+    """The 32K decode workload's layer 0 in the bench configuration, zero-copy."""
+    w = W.WORKLOADS["streamed_decode_32k"]
+    h = kvs.kvs_create(make_cfg(w, flags=kvs.KVS_FLAG_ZERO_COPY), 0)
+    try:
+        prefill(h, w, 0, w.pos0)
+        out, lse = step(h, w, 0, w.pos0, 1)
+        assert_close(out, lse, *oracle_step(w, 0, w.pos0, 1))
+        assert kvs.kvs_get_stats(h)["pages_streamed"] == w.n_pages - w.n_resident_pages
+    finally:
+        torch().cuda.synchronize()
+        kvs.kvs_destroy(h)
