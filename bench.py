@@ -253,9 +253,13 @@ def run_gpu(args, w: W.Workload):
     dev = torch.device("cuda", local)
 
     L = w.n_layers
+    # decode-width steps with streamed pages can read a share of them in place
+    zc_able = (w.n_q * (w.n_q_heads // w.n_kv_heads) <= 8 and w.n_resident_pages < w.n_pages
+               and w.n_ring_slots > 0 and L * w.n_pages * w.n_kv_heads * 53248 <= (4 << 30))
+    zc_pct = (W.ZERO_COPY_PCT if args.zero_copy_pct < 0 else args.zero_copy_pct) if zc_able else 0
     cfg = kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx, n_resident_pages=w.n_resident_pages,
                           n_ring_slots=w.n_ring_slots, max_q_tokens=w.n_q,
-                          chunk_pages=args.chunk_pages)
+                          chunk_pages=args.chunk_pages, zero_copy_pct=zc_pct)
     h = kvs.kvs_create(cfg, local)
     rc = kvs.kvs_get_config(h)
     pb = kvs.kvs_page_bytes(rc)
@@ -362,33 +366,33 @@ def run_gpu(args, w: W.Workload):
         del graph
         barrier()
 
-    # ---- zero-copy comparison arm: the same steps on a second handle whose
-    #      decode kernel reads the streamed pages in place from the mapped
-    #      pinned history (no ring copies) ----
-    zc_line = None
-    zc_ok = (w.n_q * (w.n_q_heads // w.n_kv_heads) <= 8 and rc.n_resident_pages < w.n_pages
-             and L * w.n_pages * pb <= (4 << 30))
-    if args.zero_copy_arm and zc_ok:
-        cz = kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx, n_resident_pages=w.n_resident_pages,
-                             n_ring_slots=w.n_ring_slots, max_q_tokens=w.n_q,
-                             chunk_pages=args.chunk_pages, flags=kvs.KVS_FLAG_ZERO_COPY)
-        hz = kvs.kvs_create(cz, local)
-        prefill_history(hz)
-        for _ in range(args.warmup):
-            one_step(ks, vs, qs, out, lse, hz)
-        barrier()
-        e0.record(stream)
-        for _ in range(args.steps):
-            one_step(ks, vs, qs, out, lse, hz)
-        e1.record(stream)
-        barrier()
-        ms_zc = max_over_ranks(e0.elapsed_time(e1)) / args.steps
-        S_z = w.n_pages - rc.n_resident_pages
-        zc_line = {"ms_per_step": ms_zc, "value": job_value(world, w.ctx, L, ms_zc), "unit": UNIT,
-                   "h2d_gbs_achieved": L * S_z * pb / (ms_zc * 1e-3) / 1e9,
-                   "what": "same steps, streamed pages read in place from mapped pinned host "
-                           "memory by the decode kernel (16-byte asynchronous copies), no ring"}
-        kvs.kvs_destroy(hz)
+    # ---- comparison arms: the same steps on handles that split the streamed
+    #      pages differently between the copy-engine ring and in-place reads
+    #      of the mapped pinned history by the decode kernel ----
+    arms = {}
+    if args.arms and zc_able:
+        for name, pct in (("ring_only", 0), ("zero_copy_only", 100)):
+            if pct == zc_pct:
+                continue
+            cz = kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx, n_resident_pages=w.n_resident_pages,
+                                 n_ring_slots=w.n_ring_slots, max_q_tokens=w.n_q,
+                                 chunk_pages=args.chunk_pages, zero_copy_pct=pct)
+            hz = kvs.kvs_create(cz, local)
+            prefill_history(hz)
+            for _ in range(args.warmup):
+                one_step(ks, vs, qs, out, lse, hz)
+            barrier()
+            e0.record(stream)
+            for _ in range(args.steps):
+                one_step(ks, vs, qs, out, lse, hz)
+            e1.record(stream)
+            barrier()
+            ms_a = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+            S_a = w.n_pages - rc.n_resident_pages
+            arms[name] = {"zero_copy_pct": pct, "ms_per_step": ms_a,
+                          "value": job_value(world, w.ctx, L, ms_a), "unit": UNIT,
+                          "h2d_gbs_achieved": L * S_a * pb / (ms_a * 1e-3) / 1e9}
+            kvs.kvs_destroy(hz)
 
     # ---- end to end through the C ABI with pinned host buffers ----
     kh = [x.cpu().pin_memory() for x in ks]
@@ -456,8 +460,8 @@ def run_gpu(args, w: W.Workload):
     # the ring's own write and read of every streamed page
     t_roof_chunk = L * max(R * pb / (hbm_peak * 1e9), S * pb / (h2d_ring * 1e9)) if h2d_ring else t_roof
     t_hbm_ring = L * (R + 2 * S) * pb / (hbm_peak * 1e9)
-    if zc_line:
-        zc_line["frac"] = t_roof / (zc_line["ms_per_step"] * 1e-3)
+    for arm in arms.values():
+        arm["frac"] = t_roof / (arm["ms_per_step"] * 1e-3)
     vis_keys = sum(w.pos0 + j + 1 for j in range(w.n_q))
     step_flops = L * 4.0 * w.n_q_heads * 128 * vis_keys
 
@@ -514,6 +518,7 @@ def run_gpu(args, w: W.Workload):
                    "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": 128,
                    "kv_types": "K q8_0 / V q4_0", "page_tokens": 256, "resident_pages": R,
                    "streamed_pages": S, "ring_slots": rc.n_ring_slots, "chunk_pages": rc.chunk_pages,
+                   "zero_copy_pct": zc_pct,
                    "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (resident "
                    f"{L * R * pb / 1e6:.0f} MB + streamed {L * S * pb / 1e6:.0f} MB per step)",
                    },
@@ -532,7 +537,7 @@ def run_gpu(args, w: W.Workload):
         "gpu_launches": gpu_launches,
         "launch": "library calls issued by the host without waiting between steps",
         "graph": graph_line,
-        "zero_copy": zc_line,
+        "arms": arms or None,
         "ms_per_step_median": ms_median,
         "clocks": clk,
         "prefill_s": prefill_s,
@@ -559,8 +564,10 @@ def main():
     ap.add_argument("--chunk-pages", type=int, default=0)
     ap.add_argument("--no-profile", dest="profile", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-zero-copy-arm", dest="zero_copy_arm", action="store_false",
-                    help="skip the zero-copy comparison arm")
+    ap.add_argument("--no-arms", dest="arms", action="store_false",
+                    help="skip the ring-only / zero-copy-only comparison arms")
+    ap.add_argument("--zero-copy-pct", type=int, default=-1,
+                    help="share of streamed pages decode reads in place (default: the tuned share)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="skip the extra pass that times replays of a captured step")
     args = ap.parse_args()

@@ -112,22 +112,25 @@ int ring_splits(const kvs_config& c, int n_q, int chunk_pages) {
     return wide_regime(c, n_q) ? 1 : stages;
 }
 
-// Zero-copy decode: one launch over all streamed pages, about one CTA per SM
-// (the resident launch shares the SMs), each split a run of half-page stages.
-bool zero_copy_decode(const kvs_config& c, int n_q) {
-    return (c.flags & KVS_FLAG_ZERO_COPY) && !use_tensor_cores(c, n_q);
+// Zero-copy decode: the last zero_copy_pct % of a layer's streamed pages (the
+// ones nearest the resident window) are read in place by one launch, about one
+// CTA per SM (the resident and ring launches share the SMs); the ring brings
+// the older ones.
+long zero_copy_pages(const kvs_config& c, int n_q, long S) {
+    if (use_tensor_cores(c, n_q) || c.zero_copy_pct <= 0) return 0;
+    return std::min(S, (S * c.zero_copy_pct + 50) / 100);
 }
-int zc_splits(const kvs_config& c, long S, int n_q) {
+int zc_splits(const kvs_config& c, long S_zc, int n_q) {
     const long per_split = (long)c.n_kv_heads * ((n_q * (c.n_q_heads / c.n_kv_heads) + 7) / 8);
-    return (int)std::min(2 * S, std::max(1L, (long)kSms / per_split));
+    return (int)std::min(2 * S_zc, std::max(1L, (long)kSms / per_split));
 }
 
 long count_splits(const kvs_config& c, int n_q, long R_eff, long S) {
     long n = res_splits(c, R_eff, n_q);
-    if (S > 0 && zero_copy_decode(c, n_q)) {
-        n += zc_splits(c, S, n_q);
-    } else if (S > 0 && c.chunk_pages > 0) {
-        const long full = S / c.chunk_pages, tail = S % c.chunk_pages;
+    const long S_zc = zero_copy_pages(c, n_q, S), S_ring = S - S_zc;
+    if (S_zc > 0) n += zc_splits(c, S_zc, n_q);
+    if (S_ring > 0 && c.chunk_pages > 0) {
+        const long full = S_ring / c.chunk_pages, tail = S_ring % c.chunk_pages;
         n += full * ring_splits(c, n_q, c.chunk_pages);
         if (tail) n += ring_splits(c, n_q, (int)tail);
     }
@@ -205,6 +208,10 @@ int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::stri
     if (c.max_q_tokens < 1 || c.max_q_tokens > 4096) { why = "max_q_tokens must be in [1, 4096]"; return KVS_E_INVAL; }
     if (c.n_resident_pages < 0 || c.n_ring_slots < 0 || c.chunk_pages < 0) {
         why = "negative page counts";
+        return KVS_E_INVAL;
+    }
+    if (c.zero_copy_pct < 0 || c.zero_copy_pct > 100) {
+        why = fmt("zero_copy_pct %d outside 0..100", c.zero_copy_pct);
         return KVS_E_INVAL;
     }
     const size_t pb = (size_t)c.n_kv_heads * kPageHeadBytes;
@@ -326,7 +333,8 @@ struct kvs_s {
     cudaStream_t cs = nullptr;       // copy stream (H2D ring)
     cudaStream_t rs = nullptr;       // side stream: resident-page attention (lowest priority)
     cudaStream_t xs = nullptr;       // ring attention stream (highest priority)
-    cudaEvent_t ev_fork = nullptr, ev_res = nullptr, ev_ring = nullptr;
+    cudaStream_t zs = nullptr;       // in-place (zero-copy) attention of streamed pages (lowest)
+    cudaEvent_t ev_fork = nullptr, ev_res = nullptr, ev_ring = nullptr, ev_zc = nullptr;
     size_t partial_capacity = 0;     // (split x row) records
     int n_groups = 0;
     std::vector<cudaEvent_t> ev_full, ev_free, ev_hist;
@@ -461,6 +469,8 @@ void release(kvs_t* kv) {
     if (kv->ev_fork) cudaEventDestroy(kv->ev_fork);
     if (kv->ev_res) cudaEventDestroy(kv->ev_res);
     if (kv->ev_ring) cudaEventDestroy(kv->ev_ring);
+    if (kv->ev_zc) cudaEventDestroy(kv->ev_zc);
+    if (kv->zs) cudaStreamDestroy(kv->zs);
     if (kv->xs) cudaStreamDestroy(kv->xs);
     if (kv->cs) cudaStreamDestroy(kv->cs);
     if (kv->rs) cudaStreamDestroy(kv->rs);
@@ -484,7 +494,7 @@ int wait_event(kvs_t* kv, cudaEvent_t e, double timeout_s) {
 
 int sync_all(kvs_t* kv, cudaStream_t user, double timeout_s) {
     int rc = KVS_OK;
-    for (cudaStream_t st : {kv->cs, user, kv->rs, kv->xs}) {
+    for (cudaStream_t st : {kv->cs, user, kv->rs, kv->xs, kv->zs}) {
         cudaEvent_t e = pool_event(kv);
         KVS_CK(kv, cudaEventRecord(e, st));
         if (rc == KVS_OK) rc = wait_event(kv, e, timeout_s);
@@ -666,9 +676,12 @@ int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
     if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("cudaStreamCreate: %s", cudaGetErrorString(e)));
     e = cudaStreamCreateWithPriority(&kv->xs, cudaStreamNonBlocking, prio_high);
     if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("cudaStreamCreate: %s", cudaGetErrorString(e)));
+    e = cudaStreamCreateWithPriority(&kv->zs, cudaStreamNonBlocking, prio_low);
+    if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("cudaStreamCreate: %s", cudaGetErrorString(e)));
     if (cudaEventCreateWithFlags(&kv->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&kv->ev_res, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&kv->ev_ring, cudaEventDisableTiming) != cudaSuccess)
+        cudaEventCreateWithFlags(&kv->ev_ring, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&kv->ev_zc, cudaEventDisableTiming) != cudaSuccess)
         return bail(KVS_E_CUDA, "cudaEventCreate failed");
     kv->partial_capacity = partial_records(c);
     kv->n_groups = c.n_ring_slots > 0 ? c.n_ring_slots / c.chunk_pages : 0;
@@ -715,7 +728,7 @@ void kvs_destroy(kvs_t* kv) {
     if (!kv) return;
     {
         DeviceGuard g(kv->device);
-        for (cudaStream_t st : {kv->cs, kv->rs, kv->xs}) {
+        for (cudaStream_t st : {kv->cs, kv->rs, kv->xs, kv->zs}) {
             cudaEvent_t e = pool_event(kv);
             if (e && st && cudaEventRecord(e, st) == cudaSuccess) wait_event(kv, e, 60.0);
             if (e) kv->ev_pool.push_back(e);
@@ -831,6 +844,8 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     const long R_eff = std::min(R, P);
     const long first_res = P - R_eff;
     const long S = first_res;
+    const long S_zc = zero_copy_pages(c, n_q, S);  // streamed pages read in place
+    const long S_ring = S - S_zc;                  // streamed pages copied through the ring
 
     DecodeArgs d{};
     d.len = ls.len;
@@ -854,6 +869,7 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     const unsigned long long cap = capture_id(s);
     cudaStream_t rstream = prof ? s : kv->rs;
     cudaStream_t xstream = prof ? s : kv->xs;
+    cudaStream_t zstream = prof ? s : kv->zs;
     // 1) resident pages, attended in place on the side stream so they overlap
     //    the ring pipeline below
     int split_base = 0;
@@ -877,7 +893,7 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         // the caller's stream once, since events recorded inside a capture
         // carry no ordering outside it.
         if (cap) {
-            if (kv->cs_cap != cap && S > 0) {
+            if (kv->cs_cap != cap && S_ring > 0) {
                 KVS_CK(kv, cudaStreamWaitEvent(kv->cs, kv->ev_fork, 0));
                 kv->cs_cap = cap;
             }
@@ -895,46 +911,47 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
             TimedScope ts(kv, rstream, tc ? kTChunkMma : kTDecodeRes, (uint64_t)R_eff * kv->page_bytes);
             KVS_CK(kv, tc ? launch_chunk_mma(d, &kv->map_res, ns, rstream) : launch_decode(d, &kv->map_res, ns, rstream));
         }
-        KVS_CK(kv, cudaEventRecord(kv->ev_res, rstream));
         kv->stats.kernel_launches++;
         split_base += ns;
         kv->stats.bytes_resident_read += (uint64_t)R_eff * kv->page_bytes;
     }
-    // 2a) zero-copy: the decode kernel reads the streamed pages in place from
-    //     the mapped pinned history (no ring, no copy engine)
-    if (S > 0 && zero_copy_decode(c, n_q)) {
-        KVS_CK(kv, cudaStreamWaitEvent(xstream, kv->ev_fork, 0));
+    KVS_CK(kv, cudaEventRecord(kv->ev_res, rstream));
+    // 2a) zero-copy share: the decode kernel reads streamed pages [S_ring, S)
+    //     in place from the mapped pinned history over PCIe, on its own
+    //     stream, while the copy engine brings pages [0, S_ring) through the
+    //     ring below
+    if (S_zc > 0) {
+        KVS_CK(kv, cudaStreamWaitEvent(zstream, kv->ev_fork, 0));
         d.region = kv->host_dev + (size_t)layer * kv->P_max * kv->page_bytes;
         d.region_slot_base = 0;
         d.region_slots = (int)kv->P_max;
-        d.slot0 = 0;
-        d.page0 = 0;
-        d.n_units = (int)S;
-        const int ns = zc_splits(c, S, n_q);
+        d.slot0 = (int)S_ring;
+        d.page0 = (int)S_ring;
+        d.n_units = (int)S_zc;
+        const int ns = zc_splits(c, S_zc, n_q);
         d.n_splits = ns;
         d.split_base = split_base;
         {
-            TimedScope ts(kv, xstream, kTDecodeRing, (uint64_t)S * kv->page_bytes);
-            KVS_CK(kv, launch_decode_zero_copy(d, &kv->map_res, ns, xstream));
+            TimedScope ts(kv, zstream, kTDecodeRing, (uint64_t)S_zc * kv->page_bytes);
+            KVS_CK(kv, launch_decode_zero_copy(d, &kv->map_res, ns, zstream));
         }
+        KVS_CK(kv, cudaEventRecord(kv->ev_zc, zstream));
         kv->stats.kernel_launches++;
         split_base += ns;
-        kv->stats.pages_streamed += S;
-        kv->stats.bytes_h2d += (uint64_t)S * kv->page_bytes;
-        KVS_CK(kv, cudaEventRecord(kv->ev_ring, xstream));
-        KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_ring, 0));
+        kv->stats.pages_streamed += S_zc;
+        kv->stats.bytes_h2d += (uint64_t)S_zc * kv->page_bytes;
     }
-    // 2b) streamed pages through the ring, in ascending page order
-    else if (S > 0) {
+    // 2b) streamed pages [0, S_ring) through the ring, in ascending page order
+    if (S_ring > 0) {
         if (c.n_ring_slots == 0) return fail(kv, KVS_E_INVAL, "internal: streamed pages without a ring");
-        if (ls.hist_recorded && ls.pending_min_page < S) {
+        if (ls.hist_recorded && ls.pending_min_page < S_ring) {
             if (kv->hist_cap[layer] == cap) KVS_CK(kv, cudaStreamWaitEvent(kv->cs, kv->ev_hist[layer], 0));
             ls.pending_min_page = INT_MAX;
         }
         const int chunk = c.chunk_pages;
         KVS_CK(kv, cudaStreamWaitEvent(xstream, kv->ev_fork, 0));
-        for (long i0 = 0; i0 < S; i0 += chunk) {
-            const int cpages = (int)std::min<long>(chunk, S - i0);
+        for (long i0 = 0; i0 < S_ring; i0 += chunk) {
+            const int cpages = (int)std::min<long>(chunk, S_ring - i0);
             const int gidx = (int)(kv->ring_ctr % kv->n_groups);
             kv->ring_ctr++;
             if (kv->free_valid[gidx] && kv->free_cap[gidx] == cap)
@@ -973,6 +990,7 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
 
     // 3) log-sum-exp merge of all splits (after the side stream's resident splits)
     KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_res, 0));
+    if (S_zc > 0) KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_zc, 0));
     MergeArgs m;
     m.part = kv->part;
     m.n_splits = split_base;

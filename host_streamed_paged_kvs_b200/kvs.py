@@ -28,7 +28,6 @@ KVS_PAGE_ABSENT = -1
 KVS_PAGE_RESIDENT = 1
 KVS_PAGE_STREAMED = 2
 KVS_FLAG_PROFILE = 1
-KVS_FLAG_ZERO_COPY = 2
 
 ERROR_NAMES = {0: "KVS_OK", -1: "KVS_E_INVAL", -2: "KVS_E_ARENA", -3: "KVS_E_WIDTH",
                -4: "KVS_E_ORDER", -5: "KVS_E_CUDA", -6: "KVS_E_TIMEOUT", -7: "KVS_E_NOMEM"}
@@ -48,7 +47,8 @@ class kvs_config(ctypes.Structure):
                 ("n_resident_pages", ctypes.c_int), ("n_ring_slots", ctypes.c_int),
                 ("max_q_tokens", ctypes.c_int), ("type_k", ctypes.c_int),
                 ("type_v", ctypes.c_int), ("chunk_pages", ctypes.c_int),
-                ("flags", ctypes.c_int), ("arena_bytes", ctypes.c_size_t)]
+                ("flags", ctypes.c_int), ("zero_copy_pct", ctypes.c_int),
+                ("arena_bytes", ctypes.c_size_t)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -149,10 +149,11 @@ def _check(rc: int, handle=None):
 
 def make_config(n_layers, n_q_heads, n_kv_heads, max_ctx, n_resident_pages=0, n_ring_slots=0,
                 max_q_tokens=1, chunk_pages=0, flags=0, arena_bytes=0, head_dim=128,
-                page_tokens=256, type_k=KVS_TYPE_Q8_0, type_v=KVS_TYPE_Q4_0) -> kvs_config:
+                page_tokens=256, type_k=KVS_TYPE_Q8_0, type_v=KVS_TYPE_Q4_0,
+                zero_copy_pct=0) -> kvs_config:
     return kvs_config(n_layers, n_q_heads, n_kv_heads, head_dim, page_tokens, max_ctx,
                       n_resident_pages, n_ring_slots, max_q_tokens, type_k, type_v, chunk_pages,
-                      flags, arena_bytes)
+                      flags, zero_copy_pct, arena_bytes)
 
 
 # ---- functions with the C names ------------------------------------------

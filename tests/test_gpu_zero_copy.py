@@ -1,7 +1,8 @@
-"""Zero-copy decode (KVS_FLAG_ZERO_COPY): the decode kernel reads the streamed
-pages in place from the mapped pinned history instead of through the ring.
-Parity against the oracle, agreement with the ring path on the same inputs,
-and the ring still serving the calls too wide for the CUDA-core kernel."""
+"""Zero-copy decode (zero_copy_pct): the decode kernel reads a share of the
+streamed pages in place from the mapped pinned history while the ring brings
+the rest.  Parity against the oracle, agreement with the ring-only path on the
+same inputs, and the ring still serving the calls too wide for the CUDA-core
+kernel."""
 import numpy as np
 import pytest
 
@@ -17,16 +18,19 @@ def kvs():
     return K
 
 
-@pytest.mark.parametrize("ctx,heads,n_q,R,N", [
-    (5000, (32, 8), 1, 3, 4),     # ragged last page, GQA 4
-    (4097, (8, 1), 1, 2, 2),      # GQA 8: 8 rows per kv head
-    (2600, (16, 8), 2, 1, 2),     # two query tokens x GQA 2
-    (700, (8, 2), 1, 1, 2),       # three pages, two streamed
+@pytest.mark.parametrize("ctx,heads,n_q,R,N,pct", [
+    (5000, (32, 8), 1, 3, 4, 100),     # ragged last page, GQA 4, no ring copies
+    (5000, (32, 8), 1, 3, 4, 60),      # 10 of 17 streamed pages in place, 7 through the ring
+    (4097, (8, 1), 1, 2, 2, 100),      # GQA 8: 8 rows per kv head
+    (4097, (8, 1), 1, 2, 2, 33),
+    (2600, (16, 8), 2, 1, 2, 50),      # two query tokens x GQA 2
+    (700, (8, 2), 1, 1, 2, 100),       # three pages, two streamed
+    (700, (8, 2), 1, 1, 2, 10),        # rounds to zero pages in place
 ])
-def test_zero_copy_matches_oracle_and_ring(kvs, ctx, heads, n_q, R, N):
+def test_zero_copy_matches_oracle_and_ring(kvs, ctx, heads, n_q, R, N, pct):
     w = W.Workload("zc", n_layers=2, n_q=n_q, n_q_heads=heads[0], n_kv_heads=heads[1], ctx=ctx,
                    n_resident_pages=R, n_ring_slots=N, seed=41)
-    hz = kvs.kvs_create(make_cfg(w, flags=kvs.KVS_FLAG_ZERO_COPY), 0)
+    hz = kvs.kvs_create(make_cfg(w, zero_copy_pct=pct), 0)
     hr = kvs.kvs_create(make_cfg(w), 0)
     try:
         for layer in range(w.n_layers):
@@ -38,7 +42,10 @@ def test_zero_copy_matches_oracle_and_ring(kvs, ctx, heads, n_q, R, N):
             # same arithmetic, other split layout: fp32 rounding apart only
             assert np.allclose(oz, orr, rtol=0, atol=2e-5) and np.allclose(lz, lr, rtol=0, atol=2e-5)
         st = kvs.kvs_get_stats(hz)
-        assert st["pages_streamed"] > 0 and st["h2d_copies"] == 0
+        S = w.n_pages - R
+        zc = min(S, (S * pct + 50) // 100)
+        assert st["pages_streamed"] == w.n_layers * S
+        assert (st["h2d_copies"] == 0) == (zc == S)
     finally:
         kvs.kvs_destroy(hz)
         kvs.kvs_destroy(hr)
@@ -49,7 +56,7 @@ def test_wide_calls_keep_the_ring(kvs):
     kernel through the ring even with zero-copy set."""
     w = W.Workload("zcw", n_layers=1, n_q=4, n_q_heads=40, n_kv_heads=8, ctx=3000,
                    n_resident_pages=2, n_ring_slots=4, seed=43)
-    h = kvs.kvs_create(make_cfg(w, flags=kvs.KVS_FLAG_ZERO_COPY), 0)
+    h = kvs.kvs_create(make_cfg(w, zero_copy_pct=100), 0)
     p0 = w.ctx - 10
     try:
         prefill(h, w, 0, p0)
@@ -66,9 +73,10 @@ def test_wide_calls_keep_the_ring(kvs):
 
 
 def test_zero_copy_full_size_32k_layer(kvs):
-    """The 32K decode workload's layer 0 in the bench configuration, zero-copy."""
+    """The 32K decode workload's layer 0 in the bench configuration, a share of
+    the streamed pages in place."""
     w = W.WORKLOADS["streamed_decode_32k"]
-    h = kvs.kvs_create(make_cfg(w, flags=kvs.KVS_FLAG_ZERO_COPY), 0)
+    h = kvs.kvs_create(make_cfg(w, zero_copy_pct=W.ZERO_COPY_PCT), 0)
     try:
         prefill(h, w, 0, w.pos0)
         out, lse = step(h, w, 0, w.pos0, 1)
