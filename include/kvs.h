@@ -82,14 +82,15 @@ typedef struct kvs_config {
     int type_v;           /* must be KVS_TYPE_Q4_0 */
     int chunk_pages;      /* pages per H2D copy; 0 = auto (n_ring_slots/2); must divide n_ring_slots */
     int flags;            /* KVS_FLAG_* */
-    int zero_copy_pct;    /* 0..100: share of each layer's streamed pages that decode calls
-                             (n_q * n_q_heads/n_kv_heads <= 8) read in place from the mapped
-                             pinned history by the SMs, over PCIe, while the copy engine
-                             brings the rest through the ring; the two together move more
-                             bytes per second than either alone.  100 = no ring copies for
-                             decode (the design the "Feature/adaptive kv stream integration"
-                             pull request's review found in its kernels).  Wider calls always
-                             use the ring, so a ring is still required when pages stream. */
+    int zero_copy_pct;    /* 0..100: share of each layer's streamed pages (the newest ones) that
+                             decode calls (n_q * n_q_heads/n_kv_heads <= 8) read in place from
+                             the mapped pinned history by the SMs, over PCIe, while the copy
+                             engine brings the older ones through the ring.  In-place reads pay
+                             no per-copy cost; the ring can copy ahead into the next layer.
+                             100 = no ring copies for decode (the design the "Feature/adaptive
+                             kv stream integration" pull request's review found in its
+                             kernels).  Wider calls always use the ring, so a ring is still
+                             required when pages stream. */
     size_t arena_bytes;   /* device arena budget; 0 = exact fit; else must hold one page and all
                              resident pages + ring + partials + staging (KVS_E_ARENA if not) */
 } kvs_config;
