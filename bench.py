@@ -40,8 +40,10 @@ UNIT = "KV tokens/s/layer"
 # workload it was captured on and only while the kernel source is unchanged
 # (sha256 prefix of the .cu file); otherwise traffic is reported as null.
 NCU_TRAFFIC = {
-    "decode_kernel": {"src": "kvs_kernels.cu", "sha": "f335a27149fc7358",
-                      "workload": "streamed_decode_32k", "resident": 27297024, "ring": 1738240},
+    "decode_kernel": {"src": "kvs_kernels.cu", "sha": "42df8f9c58dd5950",
+                      "workload": "streamed_decode_32k", "resident": 27297280, "ring": 1738240,
+                      # in-place launches (51 pages): DRAM bytes, and host-memory bytes read over PCIe
+                      "in_place": 35584, "in_place_sysmem": 21725184},
     "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "d873ce2100c8ebeb",
                          "workload": "prefill_chunk_64k", "resident": 36893696, "ring": 6079232},
 }
@@ -57,6 +59,18 @@ def ncu_traffic(kernel: str, workload: str, n_resident: int, n_ring: int):
         if hashlib.sha256(f.read()).hexdigest()[:16] != t["sha"]:
             return None
     return (n_resident * t["resident"] + n_ring * t["ring"]) / (n_resident + n_ring)
+
+
+def ncu_in_place(workload: str, field: str):
+    """Per-launch traffic of the in-place decode launches, same guards as ncu_traffic."""
+    import hashlib
+    t = NCU_TRAFFIC["decode_kernel"]
+    if t["workload"] != workload:
+        return None
+    with open(os.path.join(ROOT, "host_streamed_paged_kvs_b200", "csrc", t["src"]), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != t["sha"]:
+            return None
+    return t[field]
 
 
 def reduce_max(x: float, dist=None, device=None) -> float:
@@ -254,8 +268,12 @@ def run_gpu(args, w: W.Workload):
 
     L = w.n_layers
     # decode-width steps with streamed pages can read a share of them in place
-    zc_able = (w.n_q * (w.n_q_heads // w.n_kv_heads) <= 8 and w.n_resident_pages < w.n_pages
-               and w.n_ring_slots > 0 and L * w.n_pages * w.n_kv_heads * 53248 <= (4 << 30))
+    R_res = kvs.kvs_resolve_config(kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx,
+                                                   n_resident_pages=w.n_resident_pages,
+                                                   n_ring_slots=w.n_ring_slots))[0].n_resident_pages
+    zc_able = (w.n_q * (w.n_q_heads // w.n_kv_heads) <= 8 and R_res < w.n_pages and w.n_ring_slots > 0)
+    # the comparison arms need a second pinned history: only when it is small
+    arms_able = zc_able and L * w.n_pages * w.n_kv_heads * 53248 <= (4 << 30)
     zc_pct = (W.ZERO_COPY_PCT if args.zero_copy_pct < 0 else args.zero_copy_pct) if zc_able else 0
     cfg = kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx, n_resident_pages=w.n_resident_pages,
                           n_ring_slots=w.n_ring_slots, max_q_tokens=w.n_q,
@@ -316,13 +334,27 @@ def run_gpu(args, w: W.Workload):
     barrier()
     launches_per_step = int(kvs.kvs_get_stats(h)["kernel_launches"])
 
-    # The timed steps are the library's calls as a decode loop issues them: the
-    # host enqueues each step without waiting, so the copy stream can start the
-    # next step's ring copies while the current step's last layers compute.
-    def timed_step():
-        one_step(ks, vs, qs, out, lse)
+    # The timed steps are replays of one step (append + attend of every layer)
+    # captured into a CUDA graph: the library's copy stream and side streams
+    # join the capture.  The same steps issued as plain library calls are
+    # timed afterwards and reported beside them ("eager").
+    graph = None
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            one_step(ks, vs, qs, out, lse)
+        for _ in range(args.warmup):
+            with torch.cuda.stream(stream):
+                graph.replay()
+        barrier()
 
-    kvs.kvs_reset_stats(h)
+    def timed_step():
+        if graph is not None:
+            with torch.cuda.stream(stream):
+                graph.replay()
+        else:
+            one_step(ks, vs, qs, out, lse)
+
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.25)
@@ -336,41 +368,34 @@ def run_gpu(args, w: W.Workload):
     ms_total = max_over_ranks(ev[0].elapsed_time(ev[-1]))
     ms_median = statistics.median(ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps))
     clk = clocks.stop()
-    st = kvs.kvs_get_stats(h)
-    gpu_launches = int(st["kernel_launches"])  # one eager step launched launches_per_step
+    # library kernels launched in the timed region: a replay launches what one
+    # plain step launched (counted above)
+    gpu_launches = launches_per_step * args.steps
     ms_step = ms_total / args.steps
     value = job_value(world, w.ctx, L, ms_step)
     e0, e1 = ev[0], ev[-1]
-
-    # the same step captured into a CUDA graph (the copy stream and the side
-    # streams join the capture) and replayed: replays run one after another, so
-    # a step's ring copies cannot start before the previous replay has ended
-    graph_line = None
-    if args.graph:
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            one_step(ks, vs, qs, out, lse)
-        for _ in range(args.warmup):
-            with torch.cuda.stream(stream):
-                graph.replay()
-        barrier()
-        e0.record(stream)
-        for _ in range(args.steps):
-            with torch.cuda.stream(stream):
-                graph.replay()
-        e1.record(stream)
-        barrier()
-        ms_graph = max_over_ranks(e0.elapsed_time(e1)) / args.steps
-        graph_line = {"ms_per_step": ms_graph, "value": job_value(world, w.ctx, L, ms_graph),
-                      "unit": UNIT}
+    if graph is not None:
         del graph
         barrier()
+
+    # the same steps as plain library calls issued by the host without waiting
+    eager_line = None
+    if args.graph:
+        kvs.kvs_reset_stats(h)
+        e0.record(stream)
+        for _ in range(args.steps):
+            one_step(ks, vs, qs, out, lse)
+        e1.record(stream)
+        barrier()
+        ms_eager = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+        eager_line = {"ms_per_step": ms_eager, "value": job_value(world, w.ctx, L, ms_eager),
+                      "unit": UNIT, "kernel_launches": int(kvs.kvs_get_stats(h)["kernel_launches"])}
 
     # ---- comparison arms: the same steps on handles that split the streamed
     #      pages differently between the copy-engine ring and in-place reads
     #      of the mapped pinned history by the decode kernel ----
     arms = {}
-    if args.arms and zc_able:
+    if args.arms and arms_able:
         for name, pct in (("ring_only", 0), ("zero_copy_only", 100)):
             if pct == zc_pct:
                 continue
@@ -465,50 +490,80 @@ def run_gpu(args, w: W.Workload):
     vis_keys = sum(w.pos0 + j + 1 for j in range(w.n_q))
     step_flops = L * 4.0 * w.n_q_heads * 128 * vis_keys
 
-    # dominant kernel (largest summed launch time in the profiled pass): the
-    # split-K decode kernel (HBM-bound) or the tensor-core chunk kernel
+    # Roofline of each kind of launch in the profiled pass, and of the dominant
+    # one (largest summed launch time):
+    #   decode_kernel (TMA): resident pages and ring slots, bound by HBM;
+    #   decode_kernel (in place): streamed pages read over PCIe from the mapped
+    #     pinned history, bound by the host-to-device link;
+    #   chunk_mma_kernel: tensor cores.
     kernel = None
+    kinds = {}
     if st_prof:
+        prof_steps = min(args.steps, 60)
         ms_dec = st_prof["ms_decode_resident"] + st_prof["ms_decode_ring"]
         n_dec = st_prof["n_decode_resident"] + st_prof["n_decode_ring"]
-        ms_tc, n_tc = st_prof["ms_chunk_mma"], st_prof["n_chunk_mma"]
-        prof_steps = min(args.steps, 60)
-        common = {"peak_source": peak_src,
-                  "timing": "CUDA events around each launch on its stream; separate pass of the same "
-                            "steps with the library's kernels serialized on one stream",
-                  "other_kernels_avg_us": {
-                      "merge": st_prof["ms_merge"] / max(1, st_prof["n_merge"]) * 1e3,
-                      "append": st_prof["ms_append"] / max(1, st_prof["n_append"]) * 1e3}}
-        if ms_dec >= ms_tc and n_dec > 0:
+        if n_dec > 0:
             bytes_k = st_prof["bytes_decode_resident"] + st_prof["bytes_decode_ring"]
             achieved = bytes_k / (ms_dec * 1e-3) / 1e9
-            kernel = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                      "frac": achieved / hbm_peak,
-                      "traffic": ncu_traffic("decode_kernel", w.name, st_prof["n_decode_resident"],
-                                             st_prof["n_decode_ring"]),
-                      "kernel": "decode_kernel",
-                      "launches": n_dec, "avg_launch_us": ms_dec / n_dec * 1e3,
-                      "bytes_per_launch": bytes_k / n_dec,
-                      "resident_only": {
-                          "achieved": st_prof["bytes_decode_resident"] / max(st_prof["ms_decode_resident"], 1e-9) / 1e6,
-                          "launches": st_prof["n_decode_resident"],
-                          "avg_launch_us": st_prof["ms_decode_resident"] / max(1, st_prof["n_decode_resident"]) * 1e3}}
-        elif n_tc > 0:
+            kinds["decode_kernel"] = (ms_dec, {
+                "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak,
+                "traffic": ncu_traffic("decode_kernel", w.name, st_prof["n_decode_resident"],
+                                       st_prof["n_decode_ring"]),
+                "kernel": "decode_kernel", "launches": n_dec, "avg_launch_us": ms_dec / n_dec * 1e3,
+                "bytes_per_launch": bytes_k / n_dec,
+                "resident_only": {
+                    "achieved": st_prof["bytes_decode_resident"] / max(st_prof["ms_decode_resident"], 1e-9) / 1e6,
+                    "launches": st_prof["n_decode_resident"],
+                    "avg_launch_us": st_prof["ms_decode_resident"] / max(1, st_prof["n_decode_resident"]) * 1e3}})
+        ms_zc, n_zc = st_prof["ms_decode_zc"], st_prof["n_decode_zc"]
+
+        def zc_traffic(kind):
+            # the capture's figures hold for this workload at the tuned share only
+            if zc_pct != W.ZERO_COPY_PCT:
+                return None
+            return ncu_in_place(w.name, "in_place" if kind == "dram" else "in_place_sysmem")
+
+        if n_zc > 0:
+            achieved = st_prof["bytes_decode_zc"] / (ms_zc * 1e-3) / 1e9
+            kinds["decode_kernel_in_place"] = (ms_zc, {
+                "bound": "h2d", "achieved": achieved, "peak": h2d_peak, "unit": "GB/s",
+                "frac": achieved / h2d_peak, "traffic": zc_traffic("dram"),
+                "sysmem_traffic": zc_traffic("sysmem"),
+                "traffic_note": "traffic: DRAM bytes of a launch (the split partials); sysmem_traffic: "
+                                "host-memory bytes it read over PCIe (ncu sysmem sectors x 32 B)",
+                "kernel": "decode_kernel (in-place reads of streamed pages)", "launches": n_zc,
+                "avg_launch_us": ms_zc / n_zc * 1e3, "bytes_per_launch": st_prof["bytes_decode_zc"] / n_zc,
+                "peak_note": "best pinned host-to-device copy rate measured in this run"})
+        ms_tc, n_tc = st_prof["ms_chunk_mma"], st_prof["n_chunk_mma"]
+        if n_tc > 0:
             # algorithmic flops: QK^T and PV over every visible key of every query row
             vis = sum(w.pos0 + j + 1 for j in range(w.n_q))
             flops = prof_steps * L * 4.0 * w.n_q_heads * 128 * vis
             achieved = flops / (ms_tc * 1e-3) / 1e12
             tc_peak = peak_tflops()
             n_res_l = prof_steps * L
-            kernel = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                      "frac": achieved / tc_peak,
-                      "traffic": ncu_traffic("chunk_mma_kernel", w.name, n_res_l, n_tc - n_res_l),
-                      "kernel": "chunk_mma_kernel",
-                      "launches": n_tc, "avg_launch_us": ms_tc / n_tc * 1e3,
-                      "flops_per_launch": flops / n_tc,
-                      "peak_note": "measured dense bf16 burst; fp16 has the same nominal rate"}
-        if kernel:
-            kernel.update(common)
+            kinds["chunk_mma_kernel"] = (ms_tc, {
+                "bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": achieved / tc_peak,
+                "traffic": ncu_traffic("chunk_mma_kernel", w.name, n_res_l, n_tc - n_res_l),
+                "kernel": "chunk_mma_kernel", "launches": n_tc, "avg_launch_us": ms_tc / n_tc * 1e3,
+                "flops_per_launch": flops / n_tc,
+                "peak_note": "measured dense bf16 burst; fp16 has the same nominal rate"})
+        if kinds:
+            total = sum(ms for ms, _ in kinds.values())
+            name = max(kinds, key=lambda k: kinds[k][0])
+            kernel = dict(kinds[name][1])
+            kernel.update({
+                "peak_source": peak_src, "time_share": kinds[name][0] / total,
+                "timing": "CUDA events around each launch on its stream; separate pass of the same "
+                          "steps with the library's kernels serialized on one stream",
+                "other_kinds": {k: {"frac": v[1]["frac"], "bound": v[1]["bound"], "time_share": v[0] / total,
+                                    "avg_launch_us": v[1]["avg_launch_us"]}
+                                for k, v in kinds.items() if k != name} or None,
+                "other_kernels_avg_us": {
+                    "merge": st_prof["ms_merge"] / max(1, st_prof["n_merge"]) * 1e3,
+                    "append": st_prof["ms_append"] / max(1, st_prof["n_append"]) * 1e3}})
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -535,8 +590,8 @@ def run_gpu(args, w: W.Workload):
         "e2e": {"value": world * w.ctx * L / (ms_e2e * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b, "ms_per_step": ms_e2e},
         "gpu_launches": gpu_launches,
-        "launch": "library calls issued by the host without waiting between steps",
-        "graph": graph_line,
+        "launch": "replays of one captured step (CUDA graph)" if args.graph else "plain library calls",
+        "eager": eager_line,
         "arms": arms or None,
         "ms_per_step_median": ms_median,
         "clocks": clk,
@@ -569,7 +624,7 @@ def main():
     ap.add_argument("--zero-copy-pct", type=int, default=-1,
                     help="share of streamed pages decode reads in place (default: the tuned share)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
-                    help="skip the extra pass that times replays of a captured step")
+                    help="time plain library calls instead of replays of a captured step")
     args = ap.parse_args()
     w = W.WORKLOADS[args.workload]
     if args.steps <= 0:
