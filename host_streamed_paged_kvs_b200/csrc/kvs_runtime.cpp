@@ -301,7 +301,7 @@ struct LayerState {
     bool hist_recorded = false;
 };
 
-enum TimedKind { kTDecodeRes, kTDecodeRing, kTMerge, kTAppend, kTChunkMma };
+enum TimedKind { kTDecodeRes, kTDecodeRing, kTMerge, kTAppend, kTChunkMma, kTDecodeZc };
 
 struct Timed {
     cudaEvent_t a, b;
@@ -520,6 +520,8 @@ void fold_timed_upto(kvs_t* kv, size_t n) {
             case kTMerge: kv->stats.ms_merge += ms; kv->stats.n_merge++; break;
             case kTAppend: kv->stats.ms_append += ms; kv->stats.n_append++; break;
             case kTChunkMma: kv->stats.ms_chunk_mma += ms; kv->stats.n_chunk_mma++; break;
+            case kTDecodeZc: kv->stats.ms_decode_zc += ms; kv->stats.n_decode_zc++;
+                             kv->stats.bytes_decode_zc += t.bytes; break;
         }
         kv->ev_pool.push_back(t.a);
         kv->ev_pool.push_back(t.b);
@@ -932,7 +934,7 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         d.n_splits = ns;
         d.split_base = split_base;
         {
-            TimedScope ts(kv, zstream, kTDecodeRing, (uint64_t)S_zc * kv->page_bytes);
+            TimedScope ts(kv, zstream, kTDecodeZc, (uint64_t)S_zc * kv->page_bytes);
             KVS_CK(kv, launch_decode_zero_copy(d, &kv->map_res, ns, zstream));
         }
         KVS_CK(kv, cudaEventRecord(kv->ev_zc, zstream));

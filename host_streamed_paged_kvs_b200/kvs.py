@@ -59,10 +59,11 @@ class kvs_stats(ctypes.Structure):
                  ("appends", "attends", "tokens_appended", "pages_streamed", "bytes_h2d",
                   "bytes_resident_read", "h2d_copies", "kernel_launches")] +
                 [(n, ctypes.c_double) for n in
-                 ("ms_decode_resident", "ms_decode_ring", "ms_merge", "ms_append", "ms_chunk_mma")] +
+                 ("ms_decode_resident", "ms_decode_ring", "ms_merge", "ms_append", "ms_chunk_mma",
+                  "ms_decode_zc")] +
                 [(n, ctypes.c_uint64) for n in
                  ("n_decode_resident", "n_decode_ring", "n_merge", "n_append", "n_chunk_mma",
-                  "bytes_decode_resident", "bytes_decode_ring")])
+                  "n_decode_zc", "bytes_decode_resident", "bytes_decode_ring", "bytes_decode_zc")])
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}

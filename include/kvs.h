@@ -103,10 +103,11 @@ typedef struct kvs_stats {
     uint64_t bytes_resident_read;      /* resident page bytes attended */
     uint64_t h2d_copies;               /* cudaMemcpyAsync calls issued for the ring */
     uint64_t kernel_launches;          /* kernels launched by the library */
-    /* filled when KVS_FLAG_PROFILE is set: summed CUDA-event durations, ms */
-    double ms_decode_resident, ms_decode_ring, ms_merge, ms_append, ms_chunk_mma;
-    uint64_t n_decode_resident, n_decode_ring, n_merge, n_append, n_chunk_mma;
-    uint64_t bytes_decode_resident, bytes_decode_ring; /* page bytes read by timed kernels */
+    /* filled when KVS_FLAG_PROFILE is set: summed CUDA-event durations, ms
+     * (decode_zc: the launches that read streamed pages in place over PCIe) */
+    double ms_decode_resident, ms_decode_ring, ms_merge, ms_append, ms_chunk_mma, ms_decode_zc;
+    uint64_t n_decode_resident, n_decode_ring, n_merge, n_append, n_chunk_mma, n_decode_zc;
+    uint64_t bytes_decode_resident, bytes_decode_ring, bytes_decode_zc; /* page bytes read */
 } kvs_stats;
 
 typedef struct kvs_s kvs_t;

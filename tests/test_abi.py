@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(kvs):
 def test_struct_sizes_match_header(kvs):
     # 13 ints + size_t (padded) ; 8 u64 + 5 double + 7 u64
     assert ctypes.sizeof(kvs.kvs_config) == 14 * 4 + 8
-    assert ctypes.sizeof(kvs.kvs_stats) == (8 + 5 + 7) * 8
+    assert ctypes.sizeof(kvs.kvs_stats) == (8 + 6 + 9) * 8
 
 
 def test_auto_resident_matches_oracle_and_pages(kvs):
