@@ -1,5 +1,6 @@
 """Parity at the workloads' full sizes, in the configuration bench.py times
-(same handle config: layers, resident pages, ring slots, chunking), on outputs
+(same handle config: layers, resident pages, ring slots, chunking, in-place
+share of the streamed pages), on outputs
 the oracle can compute one by one: whole layers of the decode and verify
 workloads, sampled query tokens of the 256-token prefill chunk."""
 import numpy as np
@@ -18,10 +19,17 @@ def kvs():
     return K
 
 
+def bench_pct(w):
+    """The in-place share bench.py gives this workload: the tuned share for
+    decode-width steps with streamed pages, else none."""
+    decode = w.n_q * (w.n_q_heads // w.n_kv_heads) <= 8
+    return W.ZERO_COPY_PCT if decode and w.n_ring_slots > 0 else 0
+
+
 def _full(kvs, name, layers, sample_q=None):
     t = torch()
     w = W.WORKLOADS[name]
-    h = kvs.kvs_create(make_cfg(w), 0)
+    h = kvs.kvs_create(make_cfg(w, zero_copy_pct=bench_pct(w)), 0)
     try:
         for layer in layers:
             prefill(h, w, layer, w.pos0)
