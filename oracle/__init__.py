@@ -59,6 +59,11 @@ def bind(L):
     L.oracle_attention.restype = ctypes.c_int
     L.oracle_attention.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, u8p, u8p,
                                    ctypes.c_int, ctypes.c_int, u16p, f64p, f64p]
+    L.oracle_quantize_rows_t.restype = ctypes.c_int
+    L.oracle_quantize_rows_t.argtypes = [ctypes.c_int, ctypes.c_int, u16p, u16p, u8p, u8p, ctypes.c_int]
+    L.oracle_attention_t.restype = ctypes.c_int
+    L.oracle_attention_t.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, u8p, u8p,
+                                     ctypes.c_int, ctypes.c_int, u16p, f64p, f64p, ctypes.c_int]
     L.oracle_pages_for.restype = ctypes.c_long
     L.oracle_pages_for.argtypes = [ctypes.c_long, ctypes.c_int]
     L.oracle_auto_resident_pages.restype = ctypes.c_long
@@ -138,26 +143,37 @@ def dequant_q4_0(blk) -> np.ndarray:
     return out
 
 
-def quantize_rows(k, v):
-    """k, v: fp16 [..., dim] -> (Q8_0 blocks [..., dim/32, 34], Q4_0 blocks [..., dim/32, 18])."""
+V_Q4_0 = 2
+V_Q8_0 = 8
+_V_BLOCK = {V_Q4_0: 18, V_Q8_0: 34}
+
+
+def quantize_rows(k, v, v_type: int = V_Q4_0):
+    """k, v: fp16 [..., dim] -> (Q8_0 blocks [..., dim/32, 34], V blocks [..., dim/32, 18 or 34])."""
     k = _as_half_bits(k)
     v = _as_half_bits(v)
     assert k.shape == v.shape
     dim = k.shape[-1]
     rows = int(np.prod(k.shape[:-1]))
     kb = np.zeros(k.shape[:-1] + (dim // 32, 34), np.uint8)
-    vb = np.zeros(k.shape[:-1] + (dim // 32, 18), np.uint8)
-    lib().oracle_quantize_rows(rows, dim, _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16),
-                               _ptr(kb, ctypes.c_uint8), _ptr(vb, ctypes.c_uint8))
+    vb = np.zeros(k.shape[:-1] + (dim // 32, _V_BLOCK[v_type]), np.uint8)
+    if v_type == V_Q4_0:
+        lib().oracle_quantize_rows(rows, dim, _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16),
+                                   _ptr(kb, ctypes.c_uint8), _ptr(vb, ctypes.c_uint8))
+    else:
+        rc = lib().oracle_quantize_rows_t(rows, dim, _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16),
+                                          _ptr(kb, ctypes.c_uint8), _ptr(vb, ctypes.c_uint8), v_type)
+        assert rc == 0
     return kb, vb
 
 
 # --- attention ------------------------------------------------------------
 
-def attention(k_blocks: np.ndarray, v_blocks: np.ndarray, q, pos0: int):
+def attention(k_blocks: np.ndarray, v_blocks: np.ndarray, q, pos0: int, v_type: int = V_Q4_0):
     """Exact attention over a quantized history.
 
     k_blocks: uint8 [n_keys, n_kv, dim/32, 34]; v_blocks: uint8 [n_keys, n_kv, dim/32, 18]
+    (Q4_0) or [..., 34] (Q8_0, v_type = V_Q8_0)
     q: fp16 [n_q, n_qh, dim]; query j sits at position pos0+j and sees keys 0..pos0+j.
     Returns (out float64 [n_q, n_qh, dim], lse float64 [n_q, n_qh]).
     """
@@ -169,10 +185,17 @@ def attention(k_blocks: np.ndarray, v_blocks: np.ndarray, q, pos0: int):
     vb = np.ascontiguousarray(v_blocks, dtype=np.uint8)
     out = np.zeros((n_q, n_qh, dim), np.float64)
     lse = np.zeros((n_q, n_qh), np.float64)
-    rc = lib().oracle_attention(n_kv, n_qh, dim, _ptr(kb, ctypes.c_uint8),
-                                _ptr(vb, ctypes.c_uint8), n_q, pos0,
-                                _ptr(q, ctypes.c_uint16), _ptr(out, ctypes.c_double),
-                                _ptr(lse, ctypes.c_double))
+    assert vb.shape[-1] == _V_BLOCK[v_type]
+    if v_type == V_Q4_0:
+        rc = lib().oracle_attention(n_kv, n_qh, dim, _ptr(kb, ctypes.c_uint8),
+                                    _ptr(vb, ctypes.c_uint8), n_q, pos0,
+                                    _ptr(q, ctypes.c_uint16), _ptr(out, ctypes.c_double),
+                                    _ptr(lse, ctypes.c_double))
+    else:
+        rc = lib().oracle_attention_t(n_kv, n_qh, dim, _ptr(kb, ctypes.c_uint8),
+                                      _ptr(vb, ctypes.c_uint8), n_q, pos0,
+                                      _ptr(q, ctypes.c_uint16), _ptr(out, ctypes.c_double),
+                                      _ptr(lse, ctypes.c_double), v_type)
     if rc != 0:
         raise ValueError(f"oracle_attention rejected its arguments (rc={rc})")
     return out, lse

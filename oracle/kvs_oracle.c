@@ -166,24 +166,37 @@ void oracle_dequant_q4_0(const uint8_t blk[18], double out[32]) {
     }
 }
 
-void oracle_quantize_rows(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
-                          uint8_t* k_blocks, uint8_t* v_blocks) {
+/* bytes of one 32-value block of a V type (2 = Q4_0, 8 = Q8_0), 0 if unknown */
+static int v_block_bytes(int v_type) { return v_type == 2 ? 18 : (v_type == 8 ? 34 : 0); }
+
+/* K rows -> Q8_0 blocks; V rows -> Q4_0 (v_type 2) or Q8_0 (v_type 8) blocks */
+int oracle_quantize_rows_t(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
+                           uint8_t* k_blocks, uint8_t* v_blocks, int v_type) {
     int nb = dim / 32;
+    int vbb = v_block_bytes(v_type);
+    if (!vbb) return -1;
     for (int r = 0; r < n_rows; ++r) {
         for (int b = 0; b < nb; ++b) {
             const uint16_t* kx = k + (size_t)r * dim + (size_t)b * 32;
             const uint16_t* vx = v + (size_t)r * dim + (size_t)b * 32;
             oracle_q8_0_block(kx, k_blocks + ((size_t)r * nb + b) * 34);
-            oracle_q4_0_block(vx, v_blocks + ((size_t)r * nb + b) * 18);
+            if (v_type == 2) oracle_q4_0_block(vx, v_blocks + ((size_t)r * nb + b) * 18);
+            else oracle_q8_0_block(vx, v_blocks + ((size_t)r * nb + b) * vbb);
         }
     }
+    return 0;
+}
+
+void oracle_quantize_rows(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
+                          uint8_t* k_blocks, uint8_t* v_blocks) {
+    oracle_quantize_rows_t(n_rows, dim, k, v, k_blocks, v_blocks, 2);
 }
 
 /* ------------------------------------------------------------------------ */
 /* Attention over the quantized history, binary64.                            */
 /*                                                                            */
 /* k_blocks: [n_keys][n_kv][dim/32] Q8_0 blocks (token-major history)         */
-/* v_blocks: [n_keys][n_kv][dim/32] Q4_0 blocks                               */
+/* v_blocks: [n_keys][n_kv][dim/32] Q4_0 blocks (v_type 2) or Q8_0 (8)       */
 /* q:        [n_q][n_qh][dim] fp16; query j sits at absolute position pos0+j  */
 /*           and sees keys 0..pos0+j (causal).                                */
 /* q head h reads kv head h / (n_qh/n_kv) (contiguous grouping).              */
@@ -191,10 +204,11 @@ void oracle_quantize_rows(int n_rows, int dim, const uint16_t* k, const uint16_t
 /*           exp(scaled logits).                                              */
 /* ------------------------------------------------------------------------ */
 
-int oracle_attention(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
-                     const uint8_t* v_blocks, int n_q, int pos0, const uint16_t* q,
-                     double* out, double* lse) {
-    if (n_kv <= 0 || n_qh % n_kv != 0 || dim % 32 != 0 || n_q <= 0 || pos0 < 0) return -1;
+int oracle_attention_t(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
+                       const uint8_t* v_blocks, int n_q, int pos0, const uint16_t* q,
+                       double* out, double* lse, int v_type) {
+    int vbb = v_block_bytes(v_type);
+    if (n_kv <= 0 || n_qh % n_kv != 0 || dim % 32 != 0 || n_q <= 0 || pos0 < 0 || !vbb) return -1;
     int group = n_qh / n_kv;
     int nb = dim / 32;
     int max_keys = pos0 + n_q;
@@ -232,7 +246,9 @@ int oracle_attention(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
                 double p = exp(s[i] - m);
                 sum += p;
                 for (int b = 0; b < nb; ++b) {
-                    oracle_dequant_q4_0(v_blocks + (((size_t)i * n_kv + g) * nb + b) * 18, vd);
+                    const uint8_t* vblk = v_blocks + (((size_t)i * n_kv + g) * nb + b) * vbb;
+                    if (v_type == 2) oracle_dequant_q4_0(vblk, vd);
+                    else oracle_dequant_q8_0(vblk, vd);
                     for (int t = 0; t < 32; ++t) o[b * 32 + t] += p * vd[t];
                 }
             }
@@ -242,6 +258,12 @@ int oracle_attention(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
     }
     free(s); free(qd); free(kd); free(vd);
     return 0;
+}
+
+int oracle_attention(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
+                     const uint8_t* v_blocks, int n_q, int pos0, const uint16_t* q,
+                     double* out, double* lse) {
+    return oracle_attention_t(n_kv, n_qh, dim, k_blocks, v_blocks, n_q, pos0, q, out, lse, 2);
 }
 
 /* ------------------------------------------------------------------------ */
