@@ -57,27 +57,38 @@ constexpr int kRawKeys = 128;  // keys per raw (TMA) stage
 constexpr int kSubKeys = 64;   // keys per dequant / MMA sub-stage
 constexpr int kRawKq = 0;
 constexpr int kRawKd = kRawKeys * kHeadDim;                 // 16384
-constexpr int kRawVq = kRawKd + kRawKeys * kBlocks * 2;     // 17408
-constexpr int kRawVd = kRawVq + kRawKeys * kHeadDim / 2;    // 25600
-constexpr int kRawBytes = kRawVd + kRawKeys * kBlocks * 2;  // 26624
 constexpr int kRawStages = 2;
 constexpr int kKBufs = 2;
 constexpr int kVBufs = 3;
 constexpr int kKVBytes = kSubKeys * kHeadDim * 2;     // 16384: K^hi, K^lo or V^ [64][128] fp16
-constexpr size_t kOffK = (size_t)kRawStages * kRawBytes;      // 53248: [2] x (K^hi | K^lo)
-constexpr size_t kOffV = kOffK + kKBufs * 2 * kKVBytes;       // 118784: [3] x V^
-constexpr size_t kOffBar = kOffV + kVBufs * kKVBytes;         // 167936
 // barriers: raw_full[2] raw_free[2] k_full[2] k_free[2] v_full[3] v_free[3]
 //           s_full[2] s_free[2] p_full[2] p_free[2]
 constexpr int kNumBars = 22;
-constexpr size_t kOffTmem = kOffBar + kNumBars * 8;
-constexpr size_t kOffAbort = kOffTmem + 4;
-constexpr size_t kTcSmem = 1024 + kOffTmem + 16;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 128, kColP = 256, kColQ = 320;
-static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0, "swizzled tiles need 1024-B alignment");
-static_assert(kRawBytes % 1024 == 0 && kKVBytes % 1024 == 0, "swizzled tiles need 1024-B alignment");
-static_assert(kTcSmem <= 232448, "shared memory budget");
+static_assert(kKVBytes % 1024 == 0, "swizzled tiles need 1024-B alignment");
+
+// Raw-stage and shared-memory layout by V type.  Raw stage (128 keys, as the
+// pages hold them): Kq [128][128] @ 0, Kd @ 16384, Vq @ 17408 (64 B per key
+// for Q4_0 V, 128 B for Q8_0 V), Vd after it.  Shared memory: two raw
+// stages, then [2] x (K^hi | K^lo), [3] x V^, the barriers, the TMEM slot and
+// the abort flag (Q4_0 V: K^ @ 53248, V^ @ 118784, barriers @ 167936).
+template <int VT>
+struct TcGeom {
+    static constexpr int kRawVq = kRawKd + kRawKeys * kBlocks * 2;                    // 17408
+    static constexpr int kRawVd = kRawVq + kRawKeys * PageGeom<VT>::kVqRow;
+    static constexpr int kRawBytes = kRawVd + kRawKeys * kBlocks * 2;
+    static constexpr size_t kOffK = (size_t)kRawStages * kRawBytes;
+    static constexpr size_t kOffV = kOffK + kKBufs * 2 * kKVBytes;
+    static constexpr size_t kOffBar = kOffV + kVBufs * kKVBytes;
+    static constexpr size_t kOffTmem = kOffBar + kNumBars * 8;
+    static constexpr size_t kOffAbort = kOffTmem + 4;
+    static constexpr size_t kSmem = 1024 + kOffTmem + 16;
+    static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kRawBytes % 1024 == 0,
+                  "swizzled tiles need 1024-B alignment");
+    static_assert(kSmem <= 232448, "shared memory budget");
+};
+static_assert(TcGeom<kVQ4_0>::kOffBar == 167936, "Q4_0 geometry");
 
 // instruction descriptors: f16 x f16 -> f32, M = 128; A K-major;
 // S: N = 64, B K-major; PV: N = 128, B MN-major
@@ -153,8 +164,14 @@ __device__ __forceinline__ void mbar_arrive_cta(uint64_t* bar) {
 }
 
 
+template <int VT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     chunk_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap) {
+    using TG = TcGeom<VT>;
+    using PG = PageGeom<VT>;
+    constexpr int kRawVq = TG::kRawVq, kRawVd = TG::kRawVd, kRawBytes = TG::kRawBytes;
+    constexpr size_t kOffK = TG::kOffK, kOffV = TG::kOffV, kOffBar = TG::kOffBar;
+    constexpr size_t kOffTmem = TG::kOffTmem, kOffAbort = TG::kOffAbort;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -249,15 +266,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int sg = raw0 + r;
                 const int u = sg >> 1, half = sg & 1;
                 const int slot = (a.slot0 + u) % a.region_slots;
-                const uint8_t* ph = a.region + ((size_t)slot * a.n_kv + h) * kPageHeadBytes;
+                const uint8_t* ph = a.region + ((size_t)slot * a.n_kv + h) * PG::kHeadBytes;
                 uint8_t* dst = raw + (r & 1) * kRawBytes;
                 uint64_t* b = &raw_full[r & 1];
                 mbar_expect_tx(b, kRawBytes);
-                const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * kPageHeadRows + half * kRawKeys;
+                const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * PG::kRows + half * kRawKeys;
                 tma_load_2d(dst + kRawKq, &kmap, 0, krow, b);
                 bulk_load(dst + kRawKd, ph + kOffKd + half * (kRawKeys * kBlocks * 2), kRawKeys * kBlocks * 2, b);
-                bulk_load(dst + kRawVq, ph + kOffVq + half * (kRawKeys * kHeadDim / 2), kRawKeys * kHeadDim / 2, b);
-                bulk_load(dst + kRawVd, ph + kOffVd + half * (kRawKeys * kBlocks * 2), kRawKeys * kBlocks * 2, b);
+                bulk_load(dst + kRawVq, ph + PG::kOffVq + half * (kRawKeys * PG::kVqRow), kRawKeys * PG::kVqRow, b);
+                bulk_load(dst + kRawVd, ph + PG::kOffVd + half * (kRawKeys * kBlocks * 2), kRawKeys * kBlocks * 2, b);
             };
             int ir = 0;        // next raw stage to load
             for (; ir < kRawStages && ir < n_raw; ++ir) issue_raw(ir);
@@ -360,6 +377,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             //      the buffer; block b of a key: byte j = dims 32b+j (low), 32b+16+j (high) ----
             if (i >= kVBufs && fail_wait(&v_free[i % kVBufs], ((i - kVBufs) / kVBufs) & 1)) break;
             uint8_t* sVb = sV + (i % kVBufs) * kKVBytes;
+            if constexpr (VT == kVQ8_0) {
+                // Q8_0 V: V^ = fp16(d * q), the 32 codes of block blk of a key in
+                // dims 32 blk .. 32 blk + 31 (exact int8 -> fp16, one rounding)
+                for (int un = ptid; un < kSubKeys * kBlocks; un += kProdThreads) {
+                    const int blk = un & 3, kloc = un >> 2;
+                    const int key = sub * kSubKeys + kloc;
+                    const uint4* src = reinterpret_cast<const uint4*>(rb + kRawVq + key * 128 + blk * 32);
+                    const __half dh = *reinterpret_cast<const __half*>(rb + kRawVd + key * 8 + blk * 2);
+                    const __half2 d2 = __halves2half2(dh, dh);
+                    const __half2 bias = __float2half2_rn(1152.0f);
+#pragma unroll
+                    for (int hq = 0; hq < 2; ++hq) {
+                        const uint4 q = src[hq];
+                        const uint32_t w[4] = {q.x ^ 0x80808080u, q.y ^ 0x80808080u, q.z ^ 0x80808080u,
+                                               q.w ^ 0x80808080u};
+                        uint32_t o[8];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            o[2 * u] = h2u(__hmul2(__hsub2(u2h(__byte_perm(w[u], 0x6464u, 0x5140u)), bias), d2));
+                            o[2 * u + 1] = h2u(__hmul2(__hsub2(u2h(__byte_perm(w[u], 0x6464u, 0x5342u)), bias), d2));
+                        }
+                        *reinterpret_cast<uint4*>(sVb + tile_off(kSubKeys, kloc, 32 * blk + 16 * hq)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
+                        *reinterpret_cast<uint4*>(sVb + tile_off(kSubKeys, kloc, 32 * blk + 16 * hq + 8)) =
+                            make_uint4(o[4], o[5], o[6], o[7]);
+                    }
+                }
+            } else
             for (int un = ptid; un < kSubKeys * kBlocks; un += kProdThreads) {
                 const int blk = un & 3, kloc = un >> 2;
                 const int key = sub * kSubKeys + kloc;
@@ -518,14 +563,20 @@ cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !(configured & (1ull << dev))) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kTcSmem);
+        cudaError_t e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ4_0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)TcGeom<kVQ4_0>::kSmem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ8_0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)TcGeom<kVQ8_0>::kSmem);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured |= 1ull << dev;
     }
     const int m_tiles = (a.n_q * a.group + kMTile - 1) / kMTile;
     dim3 grid(n_splits, a.n_kv, m_tiles);
-    chunk_mma_kernel<<<grid, kTcThreads, kTcSmem, s>>>(a, *kmap);
+    if (a.v_type == kVQ8_0)
+        chunk_mma_kernel<kVQ8_0><<<grid, kTcThreads, TcGeom<kVQ8_0>::kSmem, s>>>(a, *kmap);
+    else
+        chunk_mma_kernel<kVQ4_0><<<grid, kTcThreads, TcGeom<kVQ4_0>::kSmem, s>>>(a, *kmap);
     return cudaGetLastError();
 }
 

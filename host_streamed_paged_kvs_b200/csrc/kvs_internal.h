@@ -36,6 +36,30 @@ constexpr int kPageHeadBytes = kOffVd + kPageTokens * kBlocks * 2;  // 53248
 constexpr int kPageHeadRows = kPageHeadBytes / 128;     // 416 rows of 128 B
 static_assert(kPageHeadBytes == 53248, "page-head layout");
 
+// V type codes (the public KVS_TYPE_* values)
+constexpr int kVQ4_0 = 2;
+constexpr int kVQ8_0 = 8;
+
+// Page-head geometry by V type.  Q4_0 V is the layout above; Q8_0 V stores
+// its codes like K (int8 [256 tok][128 dims], block b = dims 32b..32b+31):
+//   Kq @ 0, Kd @ 32,768, Vq int8 [256][128] @ 34,816, Vd @ 67,584; 69,632 B.
+template <int VT>
+struct PageGeom {
+    static_assert(VT == kVQ4_0 || VT == kVQ8_0, "V type");
+    static constexpr int kVqRow = VT == kVQ8_0 ? kHeadDim : kHeadDim / 2;  // V code bytes per token
+    static constexpr int kOffVq = kOffKd + kPageTokens * kBlocks * 2;       // 34816
+    static constexpr int kOffVd = kOffVq + kPageTokens * kVqRow;
+    static constexpr int kHeadBytes = kOffVd + kPageTokens * kBlocks * 2;
+    static constexpr int kRows = kHeadBytes / 128;
+};
+static_assert(PageGeom<kVQ4_0>::kHeadBytes == kPageHeadBytes && PageGeom<kVQ4_0>::kOffVd == kOffVd,
+              "Q4_0 geometry");
+static_assert(PageGeom<kVQ8_0>::kHeadBytes == 69632 && PageGeom<kVQ8_0>::kHeadBytes % 128 == 0,
+              "Q8_0 geometry");
+inline int page_head_bytes(int v_type) {
+    return v_type == kVQ8_0 ? PageGeom<kVQ8_0>::kHeadBytes : PageGeom<kVQ4_0>::kHeadBytes;
+}
+
 // split partials: per split and query row, (m, l) in the log2 domain + acc[128]
 struct PartialBuffers {
     float2* ml;   // [n_splits][n_rows]
@@ -51,6 +75,7 @@ struct AppendArgs {
     int n_resident;          // R
     int first_resident_page; // pages >= this are resident after the append
     size_t page_bytes;
+    int v_type;              // kVQ4_0 or kVQ8_0
 };
 
 struct DecodeArgs {
@@ -72,6 +97,7 @@ struct DecodeArgs {
     PartialBuffers part;
     int n_rows;              // n_q * n_qh
     int* err;                // device error word (bounded waits)
+    int v_type;              // kVQ4_0 or kVQ8_0: the page-head geometry
 };
 
 struct MergeArgs {

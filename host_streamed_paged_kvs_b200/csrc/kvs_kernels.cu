@@ -33,8 +33,29 @@ __device__ __forceinline__ float q4_to_f(uint32_t c) {
 // Q4_0: m = value of largest |x| (first index on ties), d = m/-8,
 //       q = min(15, trunc(x/d + 8.5)), d == 0 -> q = 8.
 // The stored scales are the fp16 (round-to-nearest-even) values of d.
+// K is always Q8_0; V is Q4_0 (VT = 2) or Q8_0 (VT = 8).
 // ----------------------------------------------------------------------------
+// Q8_0 of the 32-value block spread over 8 lanes (4 values each): the lane's
+// 4 codes packed in one word (byte u = code of value u), and the block scale
+__device__ __forceinline__ uint32_t q8_0_lane(const float (&x)[4], float& d) {
+    float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    d = __fdiv_rn(amax, 127.0f);
+    uint32_t w = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        int q = 0;
+        if (d != 0.0f) q = static_cast<int>(roundf(__fdiv_rn(x[u], d)));
+        w |= (static_cast<uint32_t>(q) & 0xffu) << (8 * u);
+    }
+    return w;
+}
+
+template <int VT>
 __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
+    using G = PageGeom<VT>;
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
     if (row >= a.n_tok * a.n_kv) return;
@@ -61,19 +82,30 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
     }
 
     // ---- Q8_0 (K) ----
-    float amax = fmaxf(fmaxf(fabsf(xk[0]), fabsf(xk[1])), fmaxf(fabsf(xk[2]), fabsf(xk[3])));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-    const float dk = __fdiv_rn(amax, 127.0f);
-    uint32_t kq = 0;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        int q = 0;
-        if (dk != 0.0f) q = static_cast<int>(roundf(__fdiv_rn(xk[u], dk)));
-        kq |= (static_cast<uint32_t>(q) & 0xffu) << (8 * u);
-    }
+    float dk;
+    const uint32_t kq = q8_0_lane(xk, dk);
     const __half dk_h = __float2half_rn(dk);
+
+    if constexpr (VT == kVQ8_0) {
+        // ---- Q8_0 (V) ----
+        float dv;
+        const uint32_t vq = q8_0_lane(xv, dv);
+        const __half dv_h = __float2half_rn(dv);
+        auto store = [&](uint8_t* ph) {
+            *reinterpret_cast<uint32_t*>(ph + kOffKq + t * kHeadDim + 4 * lane) = kq;
+            *reinterpret_cast<uint32_t*>(ph + G::kOffVq + t * kHeadDim + 4 * lane) = vq;
+            if (i == 0) {
+                *reinterpret_cast<__half*>(ph + kOffKd + t * 8 + 2 * b) = dk_h;
+                *reinterpret_cast<__half*>(ph + G::kOffVd + t * 8 + 2 * b) = dv_h;
+            }
+        };
+        store(a.host_layer + (size_t)page * a.page_bytes + (size_t)h * G::kHeadBytes);
+        if (page >= a.first_resident_page) {
+            const int slot = page % a.n_resident;
+            store(a.res_layer + (size_t)slot * a.page_bytes + (size_t)h * G::kHeadBytes);
+        }
+        return;
+    }
 
     // ---- Q4_0 (V) ----
     float va = 0.0f, vm = 0.0f;
@@ -120,7 +152,10 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
     const int rows = a.n_tok * a.n_kv;
-    append_kernel<<<(rows + 3) / 4, 128, 0, s>>>(a);
+    if (a.v_type == kVQ8_0)
+        append_kernel<kVQ8_0><<<(rows + 3) / 4, 128, 0, s>>>(a);
+    else
+        append_kernel<kVQ4_0><<<(rows + 3) / 4, 128, 0, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -165,6 +200,28 @@ constexpr size_t kDecodeSmem = 1024 /*align slack*/ + kOffBar + 2 * kStages * 8;
 static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-B swizzle alignment");
 static_assert(kWarps * kMaxRows * (kHeadDim + 2) * 4 <= kStages * kStageBytes, "merge scratch fits");
 
+// Stage and shared-memory geometry by V type: a Q8_0-V stage carries 128 B of
+// V codes per key (34,816 B per stage), so it keeps two stages in flight to
+// stay at two CTAs per SM.
+template <int VT>
+struct DecGeom {
+    static constexpr int kVqRow = PageGeom<VT>::kVqRow;
+    static constexpr int kStageVq = kStageKd + kStageKeys * kBlocks * 2;   // 17408
+    static constexpr int kStageVd = kStageVq + kStageKeys * kVqRow;
+    static constexpr int kStageBytes = kStageVd + kStageKeys * kBlocks * 2;
+    static constexpr int kStages = VT == kVQ8_0 ? 2 : 3;
+    static constexpr size_t kOffQ = (size_t)kStages * kStageBytes;
+    static constexpr size_t kOffP = kOffQ + kMaxRows * 2 * kQHalf * 4;
+    static constexpr size_t kOffKend = kOffP + (size_t)kWarps * kBlocks * kPWBlock * 4;
+    static constexpr size_t kOffBar = kOffKend + kMaxRows * 4;
+    static constexpr size_t kSmem = 1024 + kOffBar + 2 * kStages * 8;
+    static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-B swizzle alignment");
+    static_assert(kWarps * kMaxRows * (kHeadDim + 2) * 4 <= kStages * kStageBytes, "merge scratch fits");
+};
+static_assert(DecGeom<kVQ4_0>::kStageBytes == kStageBytes && DecGeom<kVQ4_0>::kSmem == kDecodeSmem,
+              "Q4_0 decode geometry");
+static_assert(2 * DecGeom<kVQ8_0>::kSmem <= 232448, "two Q8_0-V CTAs per SM");
+
 size_t decode_smem_bytes() { return kDecodeSmem; }
 
 // 2^x with the hardware approximation (flush-to-zero; 2^-inf = 0)
@@ -191,22 +248,28 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 // history) by warp 0's 16-byte asynchronous copies instead of TMA, one stage
 // = 1664 copies, 52 per lane, the K quants placed in the same 128-byte
 // swizzle the tensor map produces
-template <int ROWS, bool ZC>
+template <int ROWS, bool ZC, int VT>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap) {
+    using G = DecGeom<VT>;
+    using PG = PageGeom<VT>;
+    constexpr int kStages = G::kStages;
+    constexpr int kStageBytes = G::kStageBytes;
+    constexpr int kStageVq = G::kStageVq;
+    constexpr int kStageVd = G::kStageVd;
     constexpr int PR = ROWS <= 4 ? 4 : 8;          // padded rows of a p' record
     constexpr int SB = kWarpKeys * PR + 8;           // block stride of a warp's p' area (floats)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* stage = smem;
-    float* sQ = reinterpret_cast<float*>(smem + kOffQ);    // [ROWS][2][kQHalf]
-    int* sKend = reinterpret_cast<int*>(smem + kOffKend);           // last visible key per row
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);   // [kStages]
+    float* sQ = reinterpret_cast<float*>(smem + G::kOffQ);    // [ROWS][2][kQHalf]
+    int* sKend = reinterpret_cast<int*>(smem + G::kOffKend);           // last visible key per row
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + G::kOffBar);   // [kStages]
     uint64_t* empty = full + kStages;                               // [kStages]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    float* sPw = reinterpret_cast<float*>(smem + kOffP) + warp * kBlocks * kPWBlock;  // this warp's p'
+    float* sPw = reinterpret_cast<float*>(smem + G::kOffP) + warp * kBlocks * kPWBlock;  // this warp's p'
     const int h = blockIdx.y;
     const int row_begin = blockIdx.z * ROWS;
     const int rows_here = min(ROWS, a.n_q * a.group - row_begin);
@@ -241,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int sg = st0 + i;
         const int u = sg >> 1, half = sg & 1;
         const int slot = (a.slot0 + u) % a.region_slots;
-        const uint8_t* ph = a.region + ((size_t)slot * a.n_kv + h) * kPageHeadBytes;
+        const uint8_t* ph = a.region + ((size_t)slot * a.n_kv + h) * PG::kHeadBytes;
         uint8_t* dst = stage + (i % kStages) * kStageBytes;
         uint64_t* b = &full[i % kStages];
         if constexpr (ZC) {
@@ -253,23 +316,23 @@ __global__ void __launch_bounds__(kThreads, 2)
                 cp_async16(dst + kStageKq + r * 128 + ((k ^ (r & 7)) << 4), kq + r * 128 + k * 16);
             }
             const uint8_t* kd = ph + kOffKd + half * (kStageKeys * kBlocks * 2);
-            const uint8_t* vq = ph + kOffVq + half * (kStageKeys * kHeadDim / 2);
-            const uint8_t* vd = ph + kOffVd + half * (kStageKeys * kBlocks * 2);
+            const uint8_t* vq = ph + PG::kOffVq + half * (kStageKeys * PG::kVqRow);
+            const uint8_t* vd = ph + PG::kOffVd + half * (kStageKeys * kBlocks * 2);
             for (int c = lane; c < kStageKeys * kBlocks * 2 / 16; c += 32) {
                 cp_async16(dst + kStageKd + c * 16, kd + c * 16);
                 cp_async16(dst + kStageVd + c * 16, vd + c * 16);
             }
 #pragma unroll 4
-            for (int c = lane; c < kStageKeys * kHeadDim / 2 / 16; c += 32)
+            for (int c = lane; c < kStageKeys * PG::kVqRow / 16; c += 32)
                 cp_async16(dst + kStageVq + c * 16, vq + c * 16);
             cp_async_arrive(b);
         } else {
             mbar_expect_tx(b, kStageBytes);
-            const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * kPageHeadRows + half * kStageKeys;
+            const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * PG::kRows + half * kStageKeys;
             tma_load_2d(dst + kStageKq, &kmap, 0, krow, b);
             bulk_load(dst + kStageKd, ph + kOffKd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
-            bulk_load(dst + kStageVq, ph + kOffVq + half * (kStageKeys * kHeadDim / 2), kStageKeys * kHeadDim / 2, b);
-            bulk_load(dst + kStageVd, ph + kOffVd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
+            bulk_load(dst + kStageVq, ph + PG::kOffVq + half * (kStageKeys * PG::kVqRow), kStageKeys * PG::kVqRow, b);
+            bulk_load(dst + kStageVd, ph + PG::kOffVd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
         }
     };
     // the producer: thread 0 (TMA), or all of warp 0 (zero-copy)
@@ -391,15 +454,29 @@ __global__ void __launch_bounds__(kThreads, 2)
         __syncwarp();
 
         // ---- PV over the warp's 16 keys: lane = dims {32b+2i, +1, +16, +17} ----
-        const uint8_t* vq_base = sb + kStageVq + (warp * kWarpKeys) * 64 + vb * 16 + 2 * vi;
+        const uint8_t* vq_base = VT == kVQ8_0
+            ? sb + kStageVq + (warp * kWarpKeys) * kHeadDim + vb * 32 + 2 * vi
+            : sb + kStageVq + (warp * kWarpKeys) * 64 + vb * 16 + 2 * vi;
         const float* p_base = sPw + vb * SB;
 #pragma unroll 4
         for (int kk = 0; kk < kWarpKeys; ++kk) {
-            const uint32_t code = *reinterpret_cast<const uint16_t*>(vq_base + kk * 64);
-            const float v0 = q4_to_f(code & 0xFu);          // dim 32b+2i
-            const float v2 = q4_to_f((code >> 4) & 0xFu);   // dim 32b+2i+16
-            const float v1 = q4_to_f((code >> 8) & 0xFu);   // dim 32b+2i+1
-            const float v3 = q4_to_f((code >> 12) & 0xFu);  // dim 32b+2i+17
+            float v0, v1, v2, v3;
+            if constexpr (VT == kVQ8_0) {
+                // int8 codes of dims 32b+2i, +1 and 32b+2i+16, +17
+                const uint32_t lo = *reinterpret_cast<const uint16_t*>(vq_base + kk * kHeadDim);
+                const uint32_t hi = *reinterpret_cast<const uint16_t*>(vq_base + kk * kHeadDim + 16);
+                const uint32_t w = (lo | (hi << 16)) ^ 0x80808080u;
+                v0 = s8_to_f(w, 0);
+                v1 = s8_to_f(w, 1);
+                v2 = s8_to_f(w, 2);
+                v3 = s8_to_f(w, 3);
+            } else {
+                const uint32_t code = *reinterpret_cast<const uint16_t*>(vq_base + kk * 64);
+                v0 = q4_to_f(code & 0xFu);          // dim 32b+2i
+                v2 = q4_to_f((code >> 4) & 0xFu);   // dim 32b+2i+16
+                v1 = q4_to_f((code >> 8) & 0xFu);   // dim 32b+2i+1
+                v3 = q4_to_f((code >> 12) & 0xFu);  // dim 32b+2i+17
+            }
             const float* pr = p_base + kk * PR;
             float pv[PR];
             *reinterpret_cast<float4*>(pv) = *reinterpret_cast<const float4*>(pr);
@@ -459,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-template <int ROWS, bool ZC>
+template <int ROWS, bool ZC, int VT>
 static cudaError_t launch_decode_t(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                                    int n_row_groups, cudaStream_t s) {
     // the shared-memory opt-in is per device: remember which devices have it
@@ -467,41 +544,43 @@ static cudaError_t launch_decode_t(const DecodeArgs& a, const CUtensorMap* kmap,
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !(configured & (1ull << dev))) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<ROWS, ZC>,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<ROWS, ZC, VT>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kDecodeSmem);
+                                             (int)DecGeom<VT>::kSmem);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured |= 1ull << dev;
     }
     dim3 grid(n_splits, a.n_kv, n_row_groups);
-    decode_kernel<ROWS, ZC><<<grid, kThreads, kDecodeSmem, s>>>(a, *kmap);
+    decode_kernel<ROWS, ZC, VT><<<grid, kThreads, DecGeom<VT>::kSmem, s>>>(a, *kmap);
     return cudaGetLastError();
 }
 
-template <bool ZC>
+template <bool ZC, int VT>
 static cudaError_t launch_decode_rows(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                                       cudaStream_t s) {
     const int rows = a.n_q * a.group;
     switch (rows) {
-        case 1: return launch_decode_t<1, ZC>(a, kmap, n_splits, 1, s);
-        case 2: return launch_decode_t<2, ZC>(a, kmap, n_splits, 1, s);
-        case 3: return launch_decode_t<3, ZC>(a, kmap, n_splits, 1, s);
-        case 4: return launch_decode_t<4, ZC>(a, kmap, n_splits, 1, s);
-        case 5: return launch_decode_t<5, ZC>(a, kmap, n_splits, 1, s);
-        case 6: return launch_decode_t<6, ZC>(a, kmap, n_splits, 1, s);
-        case 7: return launch_decode_t<7, ZC>(a, kmap, n_splits, 1, s);
-        default: return launch_decode_t<8, ZC>(a, kmap, n_splits, (rows + 7) / 8, s);
+        case 1: return launch_decode_t<1, ZC, VT>(a, kmap, n_splits, 1, s);
+        case 2: return launch_decode_t<2, ZC, VT>(a, kmap, n_splits, 1, s);
+        case 3: return launch_decode_t<3, ZC, VT>(a, kmap, n_splits, 1, s);
+        case 4: return launch_decode_t<4, ZC, VT>(a, kmap, n_splits, 1, s);
+        case 5: return launch_decode_t<5, ZC, VT>(a, kmap, n_splits, 1, s);
+        case 6: return launch_decode_t<6, ZC, VT>(a, kmap, n_splits, 1, s);
+        case 7: return launch_decode_t<7, ZC, VT>(a, kmap, n_splits, 1, s);
+        default: return launch_decode_t<8, ZC, VT>(a, kmap, n_splits, (rows + 7) / 8, s);
     }
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                           cudaStream_t s) {
-    return launch_decode_rows<false>(a, kmap, n_splits, s);
+    return a.v_type == kVQ8_0 ? launch_decode_rows<false, kVQ8_0>(a, kmap, n_splits, s)
+                              : launch_decode_rows<false, kVQ4_0>(a, kmap, n_splits, s);
 }
 
 cudaError_t launch_decode_zero_copy(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                                     cudaStream_t s) {
-    return launch_decode_rows<true>(a, kmap, n_splits, s);
+    return a.v_type == kVQ8_0 ? launch_decode_rows<true, kVQ8_0>(a, kmap, n_splits, s)
+                              : launch_decode_rows<true, kVQ4_0>(a, kmap, n_splits, s);
 }
 
 // ----------------------------------------------------------------------------

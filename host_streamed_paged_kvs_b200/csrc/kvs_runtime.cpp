@@ -155,7 +155,7 @@ struct ArenaLayout {
 };
 
 ArenaLayout arena_layout(const kvs_config& c) {
-    const size_t pb = (size_t)c.n_kv_heads * kPageHeadBytes;
+    const size_t pb = (size_t)c.n_kv_heads * page_head_bytes(c.type_v);
     const size_t rows = (size_t)c.max_q_tokens * c.n_q_heads;
     const size_t recs = partial_records(c);
     ArenaLayout L{};
@@ -183,7 +183,7 @@ ArenaLayout arena_layout_with(kvs_config c, long resident_pages) {
 // fewer resident pages mean more streamed chunks and so more split partials,
 // so the counts are tried from P down.
 long resident_fit(const kvs_config& c, size_t budget, long P) {
-    const size_t per_page = (size_t)c.n_layers * c.n_kv_heads * kPageHeadBytes;
+    const size_t per_page = (size_t)c.n_layers * c.n_kv_heads * page_head_bytes(c.type_v);
     const long top = std::min<long>(std::max(1L, P), (long)(budget / per_page));  // resident bytes alone
     for (long r = top; r >= 1; --r)
         if (arena_layout_with(c, r).total <= budget) return r;
@@ -200,8 +200,9 @@ int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::stri
     }
     if (c.head_dim != kHeadDim) { why = fmt("head_dim %d unsupported (only 128)", c.head_dim); return KVS_E_INVAL; }
     if (c.page_tokens != kPageTokens) { why = fmt("page_tokens %d unsupported (only 256)", c.page_tokens); return KVS_E_INVAL; }
-    if (c.type_k != KVS_TYPE_Q8_0 || c.type_v != KVS_TYPE_Q4_0) {
-        why = "block KV streaming is not supported for this K/V cache type pair (only K=Q8_0, V=Q4_0)";
+    if (c.type_k != KVS_TYPE_Q8_0 || (c.type_v != KVS_TYPE_Q4_0 && c.type_v != KVS_TYPE_Q8_0)) {
+        why = "block KV streaming is not supported for this K/V cache type pair "
+              "(K=Q8_0 with V=Q4_0 or V=Q8_0)";
         return KVS_E_INVAL;
     }
     if (c.max_ctx < 1) { why = "max_ctx must be >= 1"; return KVS_E_INVAL; }
@@ -214,7 +215,7 @@ int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::stri
         why = fmt("zero_copy_pct %d outside 0..100", c.zero_copy_pct);
         return KVS_E_INVAL;
     }
-    const size_t pb = (size_t)c.n_kv_heads * kPageHeadBytes;
+    const size_t pb = (size_t)c.n_kv_heads * page_head_bytes(c.type_v);
     const long P = pages_for(c.max_ctx);
     if (c.n_ring_slots == 0) {
         c.chunk_pages = 0;
@@ -546,7 +547,7 @@ int kvs_resolve_config(const kvs_config* in, kvs_config* out, size_t* host_bytes
 }
 
 size_t kvs_page_bytes(const kvs_config* cfg) {
-    return cfg ? (size_t)cfg->n_kv_heads * kPageHeadBytes : 0;
+    return cfg ? (size_t)cfg->n_kv_heads * page_head_bytes(cfg->type_v) : 0;
 }
 
 int kvs_plan_page(const kvs_config* c, int n_tokens, int page, int* kind, int* index) {
@@ -631,7 +632,7 @@ int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
     kvs_t* kv = new kvs_t();
     kv->cfg = c;
     kv->device = device;
-    kv->page_bytes = (size_t)c.n_kv_heads * kPageHeadBytes;
+    kv->page_bytes = (size_t)c.n_kv_heads * page_head_bytes(c.type_v);
     kv->P_max = pages_for(c.max_ctx);
     kv->host_bytes = host_bytes;
     kv->lay = arena_layout(c);
@@ -709,8 +710,9 @@ int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
     if (e != cudaSuccess || qr != cudaDriverEntryPointSuccess || !fn)
         return bail(KVS_E_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
     auto enc = reinterpret_cast<EncodeTiledFn>(fn);
-    const uint64_t res_rows = (uint64_t)c.n_layers * c.n_resident_pages * c.n_kv_heads * kPageHeadRows;
-    const uint64_t ring_rows = (uint64_t)c.n_ring_slots * c.n_kv_heads * kPageHeadRows;
+    const uint64_t head_rows = (uint64_t)page_head_bytes(c.type_v) / 128;
+    const uint64_t res_rows = (uint64_t)c.n_layers * c.n_resident_pages * c.n_kv_heads * head_rows;
+    const uint64_t ring_rows = (uint64_t)c.n_ring_slots * c.n_kv_heads * head_rows;
     if (encode_map(kv, enc, &kv->map_res, kv->resident, res_rows) != KVS_OK) return bail(KVS_E_CUDA, kv->err);
     if (encode_map(kv, enc, &kv->map_ring, kv->ring, ring_rows) != KVS_OK) return bail(KVS_E_CUDA, kv->err);
     e = cudaDeviceSynchronize();
@@ -797,6 +799,7 @@ int kvs_append(kvs_t* kv, int layer, int pos0, int n_tok, const void* k_f16, con
     a.n_resident = (int)R;
     a.first_resident_page = (int)f_new;
     a.page_bytes = kv->page_bytes;
+    a.v_type = c.type_v;
     {
         TimedScope ts(kv, s, kTAppend, 0);
         KVS_CK(kv, launch_append(a, s));
@@ -850,6 +853,7 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     const long S_ring = S - S_zc;                  // streamed pages copied through the ring
 
     DecodeArgs d{};
+    d.v_type = c.type_v;
     d.len = ls.len;
     d.pos0 = pos0;
     d.n_q = n_q;
@@ -1029,18 +1033,24 @@ int kvs_export_page(kvs_t* kv, int layer, int page, int from_device, void* host_
     }
     uint8_t* out = static_cast<uint8_t*>(host_dst);
     const int H = c.n_kv_heads;
+    const bool v8 = c.type_v == KVS_TYPE_Q8_0;
+    const int vblk = v8 ? 34 : 18;
+    const int off_vq = v8 ? PageGeom<kVQ8_0>::kOffVq : PageGeom<kVQ4_0>::kOffVq;
+    const int off_vd = v8 ? PageGeom<kVQ8_0>::kOffVd : PageGeom<kVQ4_0>::kOffVd;
+    const int phb = page_head_bytes(c.type_v);
     uint8_t* kout = out;
     uint8_t* vout = out + (size_t)kPageTokens * H * kBlocks * 34;
     for (int t = 0; t < kPageTokens; ++t)
         for (int h = 0; h < H; ++h) {
-            const uint8_t* ph = buf.data() + (size_t)h * kPageHeadBytes;
+            const uint8_t* ph = buf.data() + (size_t)h * phb;
             for (int b = 0; b < kBlocks; ++b) {
                 uint8_t* kb = kout + (((size_t)t * H + h) * kBlocks + b) * 34;
                 std::memcpy(kb, ph + kOffKd + t * 8 + b * 2, 2);
                 std::memcpy(kb + 2, ph + kOffKq + t * kHeadDim + b * 32, 32);
-                uint8_t* vb = vout + (((size_t)t * H + h) * kBlocks + b) * 18;
-                std::memcpy(vb, ph + kOffVd + t * 8 + b * 2, 2);
-                std::memcpy(vb + 2, ph + kOffVq + t * 64 + b * 16, 16);
+                uint8_t* vb = vout + (((size_t)t * H + h) * kBlocks + b) * vblk;
+                std::memcpy(vb, ph + off_vd + t * 8 + b * 2, 2);
+                if (v8) std::memcpy(vb + 2, ph + off_vq + t * kHeadDim + b * 32, 32);
+                else std::memcpy(vb + 2, ph + off_vq + t * 64 + b * 16, 16);
             }
         }
     return KVS_OK;

@@ -110,6 +110,7 @@ extern "C" int kvs_attend_pages_static(const void* pages, int n_pages, int n_tok
     const int n_splits = (stages + sps - 1) / sps;
 
     DecodeArgs d{};
+    d.v_type = kVQ4_0;  // caller pages use the K Q8_0 / V Q4_0 page layout
     d.region = static_cast<const uint8_t*>(pages);
     d.region_slot_base = 0;
     d.region_slots = used_pages;

@@ -59,16 +59,16 @@ def step(h, w: W.Workload, layer: int, pos0: int, n_q: int, stream=None):
     return out.cpu().numpy(), lse.cpu().numpy()
 
 
-def oracle_blocks(w: W.Workload, layer: int, upto: int):
+def oracle_blocks(w: W.Workload, layer: int, upto: int, v_type: int = oracle.V_Q4_0):
     k, v = W.kv_tokens(w, layer, 0, upto)
-    return oracle.quantize_rows(k, v)
+    return oracle.quantize_rows(k, v, v_type)
 
 
-def oracle_step(w: W.Workload, layer: int, pos0: int, n_q: int, rows=None):
+def oracle_step(w: W.Workload, layer: int, pos0: int, n_q: int, rows=None, v_type: int = oracle.V_Q4_0):
     """Oracle out/lse for the step's queries over the layer's history [0, pos0+n_q)."""
-    kb, vb = oracle_blocks(w, layer, pos0 + n_q)
+    kb, vb = oracle_blocks(w, layer, pos0 + n_q, v_type)
     q = W.queries(w, layer, pos0, n_q)
-    return oracle.attention(kb, vb, q, pos0)
+    return oracle.attention(kb, vb, q, pos0, v_type)
 
 
 def assert_close(out, lse, ref_out, ref_lse):
@@ -84,10 +84,11 @@ def assert_close(out, lse, ref_out, ref_lse):
 def export_page(h, cfg, layer, page, from_device):
     from host_streamed_paged_kvs_b200 import kvs
     H = cfg.n_kv_heads
+    vbytes = 34 if cfg.type_v == kvs.KVS_TYPE_Q8_0 else 18
     nk = T * H * 4 * 34
-    nv = T * H * 4 * 18
+    nv = T * H * 4 * vbytes
     buf = np.zeros(nk + nv, np.uint8)
     kvs.kvs_export_page(h, layer, page, from_device, buf)
     kb = buf[:nk].reshape(T, H, 4, 34)
-    vb = buf[nk:].reshape(T, H, 4, 18)
+    vb = buf[nk:].reshape(T, H, 4, vbytes)
     return kb, vb

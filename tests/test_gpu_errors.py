@@ -55,7 +55,7 @@ def test_width_order_and_recovery(kvs):
 
 
 def test_create_rejections(kvs):
-    bad_pair = kvs.make_config(1, 8, 2, 1000, n_ring_slots=2, type_v=kvs.KVS_TYPE_Q8_0)
+    bad_pair = kvs.make_config(1, 8, 2, 1000, n_ring_slots=2, type_k=kvs.KVS_TYPE_Q4_0)
     with pytest.raises(kvs.KvsError) as e:
         kvs.kvs_create(bad_pair, 0)
     assert e.value.code == kvs.KVS_E_INVAL
