@@ -169,16 +169,16 @@ def oracle_layer_step(w: W.Workload, layer: int = 0, prepared=None):
     import oracle
     if prepared is None:
         k, v = W.kv_tokens(w, layer, 0, w.pos0)
-        kb, vb = oracle.quantize_rows(k, v)
+        kb, vb = oracle.quantize_rows(k, v, w.type_v)
         ks, vs = W.kv_tokens(w, layer, w.pos0, w.ctx)
         q = W.queries(w, layer, w.pos0)
         prepared = (kb, vb, ks, vs, q)
     kb, vb, ks, vs, q = prepared
     t0 = time.perf_counter()
-    kbs, vbs = oracle.quantize_rows(ks, vs)
+    kbs, vbs = oracle.quantize_rows(ks, vs, w.type_v)
     kall = np.concatenate([kb, kbs])
     vall = np.concatenate([vb, vbs])
-    oracle.attention(kall, vall, q, w.pos0)
+    oracle.attention(kall, vall, q, w.pos0, w.type_v)
     return time.perf_counter() - t0, prepared
 
 
@@ -191,14 +191,14 @@ def oracle_step_threaded(w: W.Workload, prepared, threads: int) -> float:
     kb, vb, ks, vs, q = prepared
     G = w.n_q_heads // w.n_kv_heads
     t0 = time.perf_counter()
-    kbs, vbs = oracle.quantize_rows(ks, vs)
+    kbs, vbs = oracle.quantize_rows(ks, vs, w.type_v)
     kall = np.concatenate([kb, kbs])
     vall = np.concatenate([vb, vbs])
     parts = [(np.ascontiguousarray(kall[:, g:g + 1]), np.ascontiguousarray(vall[:, g:g + 1]),
               np.ascontiguousarray(q[:, g * G:(g + 1) * G])) for g in range(w.n_kv_heads)]
     jobs = [parts[g] for _ in range(w.n_layers) for g in range(w.n_kv_heads)]
     with ThreadPoolExecutor(max_workers=threads) as ex:
-        list(ex.map(lambda p: oracle.attention(p[0], p[1], p[2], w.pos0), jobs))
+        list(ex.map(lambda p: oracle.attention(p[0], p[1], p[2], w.pos0, w.type_v), jobs))
     return time.perf_counter() - t0
 
 
@@ -268,16 +268,17 @@ def run_gpu(args, w: W.Workload):
 
     L = w.n_layers
     # decode-width steps with streamed pages can read a share of them in place
-    R_res = kvs.kvs_resolve_config(kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx,
-                                                   n_resident_pages=w.n_resident_pages,
-                                                   n_ring_slots=w.n_ring_slots))[0].n_resident_pages
-    zc_able = (w.n_q * (w.n_q_heads // w.n_kv_heads) <= 8 and R_res < w.n_pages and w.n_ring_slots > 0)
+    r0 = kvs.kvs_resolve_config(kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx,
+                                                n_resident_pages=w.n_resident_pages,
+                                                n_ring_slots=w.n_ring_slots, type_v=w.type_v))[0]
+    zc_able = (w.n_q * (w.n_q_heads // w.n_kv_heads) <= 8 and r0.n_resident_pages < w.n_pages
+               and w.n_ring_slots > 0)
     # the comparison arms need a second pinned history: only when it is small
-    arms_able = zc_able and L * w.n_pages * w.n_kv_heads * 53248 <= (4 << 30)
+    arms_able = zc_able and L * w.n_pages * kvs.kvs_page_bytes(r0) <= (4 << 30)
     zc_pct = (W.ZERO_COPY_PCT if args.zero_copy_pct < 0 else args.zero_copy_pct) if zc_able else 0
     cfg = kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx, n_resident_pages=w.n_resident_pages,
                           n_ring_slots=w.n_ring_slots, max_q_tokens=w.n_q,
-                          chunk_pages=args.chunk_pages, zero_copy_pct=zc_pct)
+                          chunk_pages=args.chunk_pages, zero_copy_pct=zc_pct, type_v=w.type_v)
     h = kvs.kvs_create(cfg, local)
     rc = kvs.kvs_get_config(h)
     pb = kvs.kvs_page_bytes(rc)
@@ -401,7 +402,7 @@ def run_gpu(args, w: W.Workload):
                 continue
             cz = kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx, n_resident_pages=w.n_resident_pages,
                                  n_ring_slots=w.n_ring_slots, max_q_tokens=w.n_q,
-                                 chunk_pages=args.chunk_pages, zero_copy_pct=pct)
+                                 chunk_pages=args.chunk_pages, zero_copy_pct=pct, type_v=w.type_v)
             hz = kvs.kvs_create(cz, local)
             prefill_history(hz)
             for _ in range(args.warmup):
@@ -571,7 +572,8 @@ def run_gpu(args, w: W.Workload):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name, "ctx": w.ctx, "n_layers": L, "n_q": w.n_q,
                    "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": 128,
-                   "kv_types": "K q8_0 / V q4_0", "page_tokens": 256, "resident_pages": R,
+                   "kv_types": "K q8_0 / V " + ("q8_0" if w.type_v == 8 else "q4_0"),
+                   "page_tokens": 256, "resident_pages": R,
                    "streamed_pages": S, "ring_slots": rc.n_ring_slots, "chunk_pages": rc.chunk_pages,
                    "zero_copy_pct": zc_pct,
                    "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (resident "
@@ -629,7 +631,8 @@ def main():
     w = W.WORKLOADS[args.workload]
     if args.steps <= 0:
         # a timed region of a few seconds
-        args.steps = {"tiny_decode_4k": 2000, "streamed_decode_32k": 300, "long_decode_256k": 30,
+        args.steps = {"tiny_decode_4k": 2000, "streamed_decode_32k": 300, "streamed_decode_32k_q8v": 240,
+                      "long_decode_256k": 30,
                       "verify_128k": 60, "prefill_chunk_64k": 200}[w.name]
         if args.impl == "reference":
             args.steps = 5

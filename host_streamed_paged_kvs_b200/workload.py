@@ -40,6 +40,7 @@ class Workload:
     outlier_scale: float = 1.0
     head_dim: int = HEAD_DIM
     page_tokens: int = PAGE_TOKENS
+    type_v: int = 2       # V block type: 2 = Q4_0, 8 = Q8_0 (the q8_0/q8_0 pair)
 
     @property
     def n_pages(self) -> int:
@@ -77,6 +78,10 @@ WORKLOADS = {
     "prefill_chunk_64k": Workload("prefill_chunk_64k", n_layers=1, n_q=256, n_q_heads=40,
                                   n_kv_heads=8, ctx=65536, n_resident_pages=64, n_ring_slots=16,
                                   seed=4),
+    # the 32K streamed decode with the q8_0/q8_0 pair (V as Q8_0: 2176 B per token per layer)
+    "streamed_decode_32k_q8v": Workload("streamed_decode_32k_q8v", n_layers=16, n_q=1, n_q_heads=32,
+                                        n_kv_heads=8, ctx=32768, n_resident_pages=64, n_ring_slots=8,
+                                        seed=5, outlier_frac=0.01, outlier_scale=8.0, type_v=8),
 }
 DEFAULT_BENCH = "streamed_decode_32k"
 # Share (%) of a decode step's streamed pages that the decode kernel reads in

@@ -29,17 +29,17 @@ def bench_pct(w):
 def _full(kvs, name, layers, sample_q=None):
     t = torch()
     w = W.WORKLOADS[name]
-    h = kvs.kvs_create(make_cfg(w, zero_copy_pct=bench_pct(w)), 0)
+    h = kvs.kvs_create(make_cfg(w, zero_copy_pct=bench_pct(w), type_v=w.type_v), 0)
     try:
         for layer in layers:
             prefill(h, w, layer, w.pos0)
             out, lse = step(h, w, layer, w.pos0, w.n_q)
             k, v = W.kv_tokens(w, layer, 0, w.ctx)
-            kb, vb = oracle.quantize_rows(k, v)
+            kb, vb = oracle.quantize_rows(k, v, w.type_v)
             q = W.queries(w, layer, w.pos0)
             js = range(w.n_q) if sample_q is None else sample_q
             for j in js:
-                ro, rl = oracle.attention(kb, vb, q[j:j + 1].copy(), w.pos0 + j)
+                ro, rl = oracle.attention(kb, vb, q[j:j + 1].copy(), w.pos0 + j, w.type_v)
                 assert_close(out[j:j + 1], lse[j:j + 1], ro, rl)
             st = kvs.kvs_get_stats(h)
             assert st["pages_streamed"] > 0
@@ -49,6 +49,10 @@ def _full(kvs, name, layers, sample_q=None):
 
 def test_streamed_decode_32k_full(kvs):
     _full(kvs, "streamed_decode_32k", layers=[0, 15])
+
+
+def test_streamed_decode_32k_q8v_full(kvs):
+    _full(kvs, "streamed_decode_32k_q8v", layers=[3])
 
 
 def test_long_decode_256k_full(kvs):
