@@ -124,6 +124,9 @@ size_t decode_smem_bytes();
 
 // bounded-wait self-test kernel (one thread, an mbarrier nothing completes)
 cudaError_t launch_wait_selftest(int* err, uint64_t limit_ns, cudaStream_t s);
+// copy `bytes` (a multiple of 16; both pointers 16-byte aligned) with plain
+// 16-byte loads and stores, e.g. from a pinned host buffer's device alias
+cudaError_t launch_copy16(void* dst, const void* src, size_t bytes, cudaStream_t s);
 
 // record the calling thread's last error text (returned by kvs_last_error(NULL))
 void set_last_error(const char* msg);

@@ -12,6 +12,8 @@
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
+#include <algorithm>
+
 #include "kvs_internal.h"
 #include "kvs_ptx.cuh"
 
@@ -714,6 +716,22 @@ cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s) {
 // nothing ever completes (no arrival, no transaction), through the same wait
 // routine the kernels use, and must give up after limit_ns.
 // ----------------------------------------------------------------------------
+// small copies between pinned host memory and the device without the copy
+// engines (whose queues the ring's chunk copies keep busy)
+__global__ void __launch_bounds__(256) copy16_kernel(uint4* __restrict__ dst, const uint4* __restrict__ src,
+                                                     size_t n) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        dst[i] = src[i];
+}
+
+cudaError_t launch_copy16(void* dst, const void* src, size_t bytes, cudaStream_t s) {
+    const size_t n = bytes / 16;
+    if (n == 0) return cudaSuccess;
+    const int blocks = (int)std::min<size_t>(64, (n + 255) / 256);
+    copy16_kernel<<<blocks, 256, 0, s>>>(static_cast<uint4*>(dst), static_cast<const uint4*>(src), n);
+    return cudaGetLastError();
+}
+
 __global__ void wait_selftest_kernel(int* err, uint64_t limit_ns) {
     __shared__ __align__(8) uint64_t bar;
     mbar_init(&bar, 1);

@@ -286,6 +286,20 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// device alias of a pinned (page-locked) host buffer when it is 16-byte
+// aligned; nullptr for pageable host memory, device memory or misalignment.
+// Small inputs and outputs in pinned memory then cross PCIe inside the
+// library's kernels instead of queueing on the copy engines behind the ring.
+const void* pinned_alias16(const void* p) {
+    cudaPointerAttributes at;
+    if (!p || cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (at.type != cudaMemoryTypeHost || !at.devicePointer) return nullptr;
+    return (reinterpret_cast<uintptr_t>(at.devicePointer) & 15) ? nullptr : at.devicePointer;
+}
+
 bool is_host_ptr(const void* p) {
     if (!p) return false;
     cudaPointerAttributes at;
@@ -764,13 +778,25 @@ int kvs_append(kvs_t* kv, int layer, int pos0, int n_tok, const void* k_f16, con
     const size_t kv_elems = (size_t)n_tok * c.n_kv_heads * kHeadDim;
     const __half* k = static_cast<const __half*>(k_f16);
     const __half* v = static_cast<const __half*>(v_f16);
+    // pinned host K/V: the append kernel reads them in place over PCIe;
+    // pageable ones are staged by the copy engine
     if (host_k) {
-        KVS_CK(kv, cudaMemcpyAsync(kv->stage_k, k_f16, kv_elems * 2, cudaMemcpyHostToDevice, s));
-        k = kv->stage_k;
+        const void* a = pinned_alias16(k_f16);
+        if (a) {
+            k = static_cast<const __half*>(a);
+        } else {
+            KVS_CK(kv, cudaMemcpyAsync(kv->stage_k, k_f16, kv_elems * 2, cudaMemcpyHostToDevice, s));
+            k = kv->stage_k;
+        }
     }
     if (host_v) {
-        KVS_CK(kv, cudaMemcpyAsync(kv->stage_v, v_f16, kv_elems * 2, cudaMemcpyHostToDevice, s));
-        v = kv->stage_v;
+        const void* a = pinned_alias16(v_f16);
+        if (a) {
+            v = static_cast<const __half*>(a);
+        } else {
+            KVS_CK(kv, cudaMemcpyAsync(kv->stage_v, v_f16, kv_elems * 2, cudaMemcpyHostToDevice, s));
+            v = kv->stage_v;
+        }
     }
     if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 7)
         return fail(kv, KVS_E_INVAL, "K/V must be 8-byte aligned");
@@ -833,13 +859,19 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     const int rows = n_q * c.n_q_heads;
     const __half* q = static_cast<const __half*>(q_f16);
     if (is_host_ptr(q_f16)) {
-        KVS_CK(kv, cudaMemcpyAsync(kv->stage_q, q_f16, (size_t)rows * kHeadDim * 2, cudaMemcpyHostToDevice, s));
+        // pinned: one small copy kernel pulls Q over PCIe; pageable: copy engine
+        const void* a = pinned_alias16(q_f16);
+        if (a) KVS_CK(kv, launch_copy16(kv->stage_q, a, (size_t)rows * kHeadDim * 2, s));
+        else KVS_CK(kv, cudaMemcpyAsync(kv->stage_q, q_f16, (size_t)rows * kHeadDim * 2, cudaMemcpyHostToDevice, s));
         q = kv->stage_q;
     }
-    const bool host_out = is_host_ptr(out);
-    const bool host_lse = lse && is_host_ptr(lse);
-    float* dout = host_out ? kv->stage_out : out;
-    float* dlse = lse ? (host_lse ? kv->stage_lse : lse) : nullptr;
+    // pinned host out/lse: the merge kernel writes them in place over PCIe
+    float* out_alias = is_host_ptr(out) ? static_cast<float*>(const_cast<void*>(pinned_alias16(out))) : nullptr;
+    float* lse_alias = (lse && is_host_ptr(lse)) ? static_cast<float*>(const_cast<void*>(pinned_alias16(lse))) : nullptr;
+    const bool host_out = is_host_ptr(out) && !out_alias;
+    const bool host_lse = lse && is_host_ptr(lse) && !lse_alias;
+    float* dout = out_alias ? out_alias : (host_out ? kv->stage_out : out);
+    float* dlse = lse ? (lse_alias ? lse_alias : (host_lse ? kv->stage_lse : lse)) : nullptr;
 
     const bool tc = use_tensor_cores(c, n_q);
     if (tc && (reinterpret_cast<uintptr_t>(q) & 15))

@@ -216,28 +216,40 @@ def test_rollback_and_reappend(kvs):
         kvs.kvs_destroy(h)
 
 
-def test_host_pointer_io(kvs):
-    """Q/K/V/out/lse in pinned host memory go through the library's staging buffers."""
+@pytest.mark.parametrize("mem", ["pinned", "pageable"])
+@pytest.mark.parametrize("n_q,heads", [(1, (8, 2)), (4, (40, 8))])
+def test_host_pointer_io(kvs, mem, n_q, heads):
+    """Q/K/V/out/lse in host memory: pinned buffers cross PCIe inside the
+    library's kernels, pageable ones through its staging buffers.  Either way
+    the results are the bits the device-pointer calls give."""
     t = torch()
-    w = small("hostio", ctx=1500, n_layers=1)
-    cfg = make_cfg(w)
-    h = kvs.kvs_create(cfg, 0)
+    w = small("hostio", ctx=1500, n_layers=1, n_q=n_q, n_q_heads=heads[0], n_kv_heads=heads[1])
+    hd = kvs.kvs_create(make_cfg(w), 0)
+    hh = kvs.kvs_create(make_cfg(w), 0)
     try:
-        prefill(h, w, 0, w.pos0)
         k, v = W.kv_tokens(w, 0, w.pos0, w.ctx)
-        q = W.queries(w, 0, w.pos0, 1)
-        kh = t.from_numpy(k).pin_memory()
-        vh = t.from_numpy(v).pin_memory()
-        qh = t.from_numpy(q).pin_memory()
-        out = t.empty((1, w.n_q_heads, 128), dtype=t.float32).pin_memory()
-        lse = t.empty((1, w.n_q_heads), dtype=t.float32).pin_memory()
-        kvs.kvs_append(h, 0, w.pos0, 1, kh, vh)
-        kvs.kvs_attend(h, 0, w.pos0, 1, qh, out, lse)
-        kvs.kvs_sync(h, None, 30.0)
-        ref_out, ref_lse = oracle_step(w, 0, w.pos0, 1)
-        assert_close(out.numpy(), lse.numpy(), ref_out, ref_lse)
+        q = W.queries(w, 0, w.pos0, n_q)
+        # device pointers
+        prefill(hd, w, 0, w.pos0)
+        out_d, lse_d = step(hd, w, 0, w.pos0, n_q)
+        # host pointers
+        prefill(hh, w, 0, w.pos0)
+        if mem == "pinned":
+            kh, vh, qh = (t.from_numpy(x).pin_memory() for x in (k, v, q))
+            out = t.empty((n_q, w.n_q_heads, 128), dtype=t.float32).pin_memory()
+            lse = t.empty((n_q, w.n_q_heads), dtype=t.float32).pin_memory()
+        else:
+            kh, vh, qh = (np.ascontiguousarray(x) for x in (k, v, q))
+            out = t.from_numpy(np.zeros((n_q, w.n_q_heads, 128), np.float32))
+            lse = t.from_numpy(np.zeros((n_q, w.n_q_heads), np.float32))
+        kvs.kvs_append(hh, 0, w.pos0, n_q, kh, vh)
+        kvs.kvs_attend(hh, 0, w.pos0, n_q, qh, out, lse)
+        kvs.kvs_sync(hh, None, 30.0)
+        assert np.array_equal(out.numpy(), out_d) and np.array_equal(lse.numpy(), lse_d)
+        assert_close(out.numpy(), lse.numpy(), *oracle_step(w, 0, w.pos0, n_q))
     finally:
-        kvs.kvs_destroy(h)
+        kvs.kvs_destroy(hd)
+        kvs.kvs_destroy(hh)
 
 
 def test_repeated_steps_are_stable(kvs):
