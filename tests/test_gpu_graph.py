@@ -1,7 +1,7 @@
 """A whole decode step (append + attend for every layer) captured into a CUDA
-graph and replayed: the ring's copy stream and the two attention side streams
-join the capture, and replays give the same bits as plain calls before and
-after."""
+graph and replayed: the ring's copy stream and the attention side streams
+(resident, ring, in-place share) join the capture, and replays give the same
+bits as plain calls before and after."""
 import numpy as np
 import pytest
 
@@ -11,13 +11,14 @@ from kvs_testlib import assert_close, make_cfg, oracle_step, prefill, to_dev, to
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("n_q,heads", [(1, (32, 8)), (4, (40, 8))])
-def test_graph_captured_step_matches_plain_calls(n_q, heads):
+@pytest.mark.parametrize("n_q,heads,pct", [(1, (32, 8), 0), (1, (32, 8), 80), (1, (32, 8), 100),
+                                            (4, (40, 8), 0)])
+def test_graph_captured_step_matches_plain_calls(n_q, heads, pct):
     t = torch()
     from host_streamed_paged_kvs_b200 import kvs
     w = W.Workload("graph", n_layers=3, n_q=n_q, n_q_heads=heads[0], n_kv_heads=heads[1], ctx=3000,
                    n_resident_pages=3, n_ring_slots=4, seed=31)
-    h = kvs.kvs_create(make_cfg(w), 0)
+    h = kvs.kvs_create(make_cfg(w, zero_copy_pct=pct), 0)
     s = t.cuda.Stream()
     try:
         for layer in range(w.n_layers):
