@@ -1,7 +1,10 @@
 // kvs_runtime.cpp -- host runtime behind the C ABI in include/kvs.h: config
-// validation and auto sizing, the pinned host history, the device arena
-// (resident pages, ring slots, split partials, staging), the page table, the
-// copy-engine ring with its events, and the call sequencing of append/attend.
+// validation and auto sizing (10 % rule, or the resident fit of a fixed
+// arena), the pinned host history, the device arena (resident pages, ring
+// slots, split partials, staging), the page table, the copy-engine ring with
+// its events, the share of streamed pages decode reads in place from the
+// mapped history, the call sequencing of append/attend over the caller's
+// stream and four library streams, and the draft eject controller.
 //
 // Method sources:
 //  * "RaymondHuang210129/llama.cpp-adaptive-kv-streaming", Summary: the full KV
@@ -15,7 +18,10 @@
 //    configuration gates (supported K/V type pair, one page byte size for all
 //    streamed layers), the minimum stage of one page, and the review's
 //    observation that a real implementation needs a device staging pool, a
-//    page table and a cudaMemcpyAsync ring.
+//    page table and a cudaMemcpyAsync ring (its own kernels read mapped host
+//    memory directly: the in-place share keeps that design as an option).
+//  * "llama.cpp adaptive KV streaming - spec fork notes", Dynamic draft eject:
+//    the eject threshold, re-enable band and stability count.
 #include <algorithm>
 #include <chrono>
 #include <climits>
