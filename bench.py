@@ -40,12 +40,12 @@ UNIT = "KV tokens/s/layer"
 # workload it was captured on and only while the kernel source is unchanged
 # (sha256 prefix of the .cu file); otherwise traffic is reported as null.
 NCU_TRAFFIC = {
-    "decode_kernel": {"src": "kvs_kernels.cu", "sha": "42df8f9c58dd5950",
-                      "workload": "streamed_decode_32k", "resident": 27297280, "ring": 1738240,
+    "decode_kernel": {"src": "kvs_kernels.cu", "sha": "e9caa7f0678a97d5",
+                      "workload": "streamed_decode_32k", "resident": 27297024, "ring": 1737984,
                       # in-place launches (51 pages): DRAM bytes, and host-memory bytes read over PCIe
                       "in_place": 35584, "in_place_sysmem": 21725184},
-    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "d873ce2100c8ebeb",
-                         "workload": "prefill_chunk_64k", "resident": 36893696, "ring": 6079232},
+    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "26ac8cef13592c1b",
+                         "workload": "prefill_chunk_64k", "resident": 37882880, "ring": 6078976},
 }
 
 
