@@ -169,15 +169,19 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
 // 128-byte swizzle (a thread reading its key's row then hits distinct banks
 // while the query chunk it multiplies is a broadcast), the K scales, V codes
 // and V scales as 1-D bulk copies; three stages are in flight.  Every warp
-// owns 16 keys of each stage end to end, with its own online-softmax state:
-//   QK^T : two lanes per key, 64 dims each; K dequantized in registers (exact
-//          int8 -> fp32), the per-block scale applied to the block partial;
-//   softmax: warp-local running max per row (log2 domain); the V scale of each
-//          (key, block) folded into the probability, p' = p * d_v;
-//   PV   : lane = 4 dims x all rows over the warp's 16 keys.
+// owns 16 keys of each stage end to end, with its own online-softmax state,
+// and does its math on the tensor cores with warp-level mma.sync m16n8k16
+// (fp16 operands, fp32 accumulate; the <= 8 query rows of a row group fill
+// rows 0..7 of the 16-row tile):
+//   QK^T : int8 K codes are exact in fp16; per 32-dim block the MMA gives the
+//          block's partial score in fp32 and the block's K scale multiplies it;
+//   softmax: warp-local lazy running max per row (log2 domain);
+//   PV   : the probability times the V scale of each (key, block) is the A
+//          operand (one fp16 rounding), the V codes (q - 8 for Q4_0, q for
+//          Q8_0) exact in fp16 are the B operand.
 // A stage buffer is refilled once all eight warps have released it (an
 // mbarrier with eight arrivals); there is no CTA-wide barrier in the loop.  At
-// the end the eight warps' (m, l, acc) are merged into the split's partial.
+// the end the eight warps' (m, l, O) are merged into the split's partial.
 // ----------------------------------------------------------------------------
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
@@ -190,13 +194,9 @@ constexpr int kStageVd = kStageVq + kStageKeys * kHeadDim / 2;     // 25600
 constexpr int kStageBytes = kStageVd + kStageKeys * kBlocks * 2;   // 26624
 constexpr int kStages = 3;
 constexpr int kMaxRows = 8;
-constexpr int kQHalf = 68;                  // floats per (row, half): 64 + 4 pad (bank offset)
-// per-warp p' records [block][16 keys][PR], block stride padded so the two
-// lanes of a key and four consecutive keys store into distinct banks
-constexpr int kPWBlock = kWarpKeys * kMaxRows + 8;                 // 136 floats (PR = 8)
+constexpr int kQFragBytes = 32 * 16 * 4;    // Q operand fragments: 16 words per lane
 constexpr size_t kOffQ = kStages * kStageBytes;
-constexpr size_t kOffP = kOffQ + kMaxRows * 2 * kQHalf * 4;                    // sQ
-constexpr size_t kOffKend = kOffP + (size_t)kWarps * kBlocks * kPWBlock * 4;   // sP
+constexpr size_t kOffKend = kOffQ + kQFragBytes;                                 // sQf
 constexpr size_t kOffBar = kOffKend + kMaxRows * 4;                              // sKend
 constexpr size_t kDecodeSmem = 1024 /*align slack*/ + kOffBar + 2 * kStages * 8;
 static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-B swizzle alignment");
@@ -213,8 +213,7 @@ struct DecGeom {
     static constexpr int kStageBytes = kStageVd + kStageKeys * kBlocks * 2;
     static constexpr int kStages = VT == kVQ8_0 ? 2 : 3;
     static constexpr size_t kOffQ = (size_t)kStages * kStageBytes;
-    static constexpr size_t kOffP = kOffQ + kMaxRows * 2 * kQHalf * 4;
-    static constexpr size_t kOffKend = kOffP + (size_t)kWarps * kBlocks * kPWBlock * 4;
+    static constexpr size_t kOffKend = kOffQ + kQFragBytes;
     static constexpr size_t kOffBar = kOffKend + kMaxRows * 4;
     static constexpr size_t kSmem = 1024 + kOffBar + 2 * kStages * 8;
     static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-B swizzle alignment");
@@ -232,6 +231,19 @@ __device__ __forceinline__ float ex2_approx(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+
+// D += A B, m16n8k16, fp16 operands, fp32 accumulate; the A rows 8..15 are
+// zero (a1 = a3 = 0): a0 = {row g, k 2q..2q+1}, a2 = {row g, k 2q+8..2q+9}
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+__device__ __forceinline__ uint32_t h2u(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -259,19 +271,16 @@ __global__ void __launch_bounds__(kThreads, 2)
     constexpr int kStageBytes = G::kStageBytes;
     constexpr int kStageVq = G::kStageVq;
     constexpr int kStageVd = G::kStageVd;
-    constexpr int PR = ROWS <= 4 ? 4 : 8;          // padded rows of a p' record
-    constexpr int SB = kWarpKeys * PR + 8;           // block stride of a warp's p' area (floats)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* stage = smem;
-    float* sQ = reinterpret_cast<float*>(smem + G::kOffQ);    // [ROWS][2][kQHalf]
+    uint32_t* sQf = reinterpret_cast<uint32_t*>(smem + G::kOffQ);  // [32 lanes][16] Q fragments
     int* sKend = reinterpret_cast<int*>(smem + G::kOffKend);           // last visible key per row
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + G::kOffBar);   // [kStages]
     uint64_t* empty = full + kStages;                               // [kStages]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    float* sPw = reinterpret_cast<float*>(smem + G::kOffP) + warp * kBlocks * kPWBlock;  // this warp's p'
     const int h = blockIdx.y;
     const int row_begin = blockIdx.z * ROWS;
     const int rows_here = min(ROWS, a.n_q * a.group - row_begin);
@@ -279,16 +288,23 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int st0 = (int)(((long)blockIdx.x * n_stages_all) / a.n_splits);
     const int n_st = (int)(((long)(blockIdx.x + 1) * n_stages_all) / a.n_splits) - st0;
 
-    // queries of this CTA's rows, pre-scaled into the log2 domain
-    for (int idx = tid; idx < ROWS * kHeadDim; idx += kThreads) {
-        const int r = idx / kHeadDim, d = idx - r * kHeadDim;
-        float v = 0.0f;
-        if (r < rows_here) {
-            const int lr = row_begin + r;
-            const int j = lr / a.group, g = lr - j * a.group;
-            v = __half2float(a.q[((size_t)j * a.n_qh + h * a.group + g) * kHeadDim + d]) * a.q_scale;
+    // Q as the tensor-core A operand, one 16-word fragment set per lane
+    // (the same for every warp): lane (g, q) holds, for k-step kk = 2b + s,
+    // row g's fp16 dims {d0, d0+1} and {d0+2, d0+3}, d0 = 32b + 8q + 4s
+    // (zero for rows past the CTA's rows)
+    if (tid < 32) {
+        const int g = tid >> 2, q = tid & 3;
+        const bool vr = g < rows_here;
+        const int lr = row_begin + g;
+        const __half* qrow = a.q + ((size_t)(lr / a.group) * a.n_qh + h * a.group + (lr % a.group)) * kHeadDim;
+        uint32_t* qf = sQf + tid * 16;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const int d0 = 32 * (kk >> 1) + 8 * q + 4 * (kk & 1);
+            const uint2 v = vr ? *reinterpret_cast<const uint2*>(qrow + d0) : make_uint2(0u, 0u);
+            qf[2 * kk] = v.x;
+            qf[2 * kk + 1] = v.y;
         }
-        sQ[(r * 2 + (d >> 6)) * kQHalf + (d & 63)] = v;
     }
     if (tid < ROWS)  // row r sees keys 0 .. min(len-1, its query position); padding rows none
         sKend[tid] = (tid < rows_here) ? min(a.len - 1, a.pos0 + (row_begin + tid) / a.group) : -1;
@@ -344,17 +360,27 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (; next_issue < kStages && next_issue < n_st; ++next_issue) issue(next_issue);
     }
 
-    float m_run[ROWS], l_run[ROWS], acc[ROWS][4];
+    // ---- tensor-core math (mma.sync m16n8k16: fp16 operands, fp32 accumulate) ----
+    // Row g = lane / 4 of the MMA tile is query row g of this CTA (rows past
+    // rows_here, and the tile's rows 8..15, are zero); q = lane % 4.
+    // QK^T, per 32-dim block b: two k-steps s; MMA k-index 2q+{0,1} and
+    //   2q+8+{0,1} of k-step s stand for dims 32b+8q+4s+{0,1} and {2,3}, so a
+    //   lane's K operand is 4 consecutive int8 of its key's row (exact in fp16)
+    //   and the block's scale multiplies the block's fp32 partial score.
+    // PV: n-tile nt = 4b + m holds dims 32b + 4n + m (column n); the MMA
+    //   k-index runs over the warp's 16 keys in the order of the score tile's
+    //   columns, and the probabilities carry the V scale of block b (one fp16
+    //   rounding of p * d_v; the codes q - 8 are exact in fp16).
+    const int g = lane >> 2, q = lane & 3;
+    const uint4* qfrag = reinterpret_cast<const uint4*>(sQf + lane * 16);  // block b: qfrag[b]
+    const int kend = g < ROWS ? sKend[g] : -1;  // last visible key of this lane's row
+    float o[16][2];                              // O (row g; dims of n-tile nt, columns 2q, 2q+1)
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r) {
-        m_run[r] = -CUDART_INF_F;
-        l_run[r] = 0.0f;
-        acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.0f;
-    }
-    const int kl = lane >> 1, hf = lane & 1;  // QK / softmax role: key kl of the warp, dim half hf
-    const int key = warp * kWarpKeys + kl;     // key within the stage
-    const int vb = lane >> 3, vi = lane & 7;  // PV role: block and byte pair of this lane
+    for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = 0.0f;
+    float zr0 = 0.0f, zr1 = 0.0f;  // the tile's rows 8..15: zero operands keep them zero
+    float m_run = -CUDART_INF_F, l_run = 0.0f;
     bool ok = true;
+    const __half2 b1152 = __float2half2_rn(1152.0f), b1032 = __float2half2_rn(1032.0f);
 
     for (int i = 0; i < n_st; ++i) {
         // producer: keep the next two stages in flight (it waits for all
@@ -373,122 +399,118 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!mbar_wait_bounded(&full[i % kStages], (i / kStages) & 1, a.err)) ok = false;
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         const int sg = st0 + i;
-        const int kpos = (a.page0 + (sg >> 1)) * kPageTokens + (sg & 1) * kStageKeys + key;
+        const int kbase = (a.page0 + (sg >> 1)) * kPageTokens + (sg & 1) * kStageKeys + warp * kWarpKeys;
+        const int wkey = warp * kWarpKeys;  // first key of this warp within the stage
 
-        // ---- QK^T: this lane's key, dims [64 hf, 64 hf + 64) ----
-        float s[ROWS];
-#pragma unroll
-        for (int r = 0; r < ROWS; ++r) s[r] = 0.0f;
-        const uint8_t* krow = sb + kStageKq + key * kHeadDim;
-        const float* qh = sQ + hf * kQHalf;
+        // K / V scale of block blk of this lane's key wkey + 8t + 2q + j
+        const __half2* kd2 = reinterpret_cast<const __half2*>(sb + kStageKd + (wkey + 2 * q) * (kBlocks * 2));
+        const __half2* vd2 = reinterpret_cast<const __half2*>(sb + kStageVd + (wkey + 2 * q) * (kBlocks * 2));
+        // keys 2q, 2q+1 (t = 0) and 8+2q, 8+2q+1 (t = 1): scale of block blk as a pair (j = 0, 1)
+        auto scales = [&](const __half2* base, int t, int blk) {
+            const __half* hb = reinterpret_cast<const __half*>(base + t * 8 * (kBlocks / 2));
+            return make_float2(__half2float(hb[blk]), __half2float(hb[kBlocks + blk]));
+        };
+
+        // ---- QK^T ----
+        float sc[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
+        const uint8_t* kst = sb + kStageKq;
 #pragma unroll 1
-        for (int bb = 0; bb < 2; ++bb) {
-            const int blk = 2 * hf + bb;
-            float part[ROWS];
+        for (int blk = 0; blk < kBlocks; ++blk) {
+            const uint4 qb = qfrag[blk];  // k-steps 2 blk (x, y) and 2 blk + 1 (z, w)
 #pragma unroll
-            for (int r = 0; r < ROWS; ++r) part[r] = 0.0f;
+            for (int t = 0; t < 2; ++t) {
+                const int key = wkey + 8 * t + g;  // this lane's column of the K operand
+                const int chunk = 2 * blk + (q >> 1);
+                const uint2 w = *reinterpret_cast<const uint2*>(kst + key * kHeadDim + ((chunk ^ (key & 7)) << 4) +
+                                                                8 * (q & 1));
+                const uint32_t x0 = w.x ^ 0x80808080u, x1 = w.y ^ 0x80808080u;
+                float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                mma16816(c, qb.x, qb.y,
+                         h2u(__hsub2(u2h(__byte_perm(x0, 0x6464u, 0x5140u)), b1152)),
+                         h2u(__hsub2(u2h(__byte_perm(x0, 0x6464u, 0x5342u)), b1152)));
+                mma16816(c, qb.z, qb.w,
+                         h2u(__hsub2(u2h(__byte_perm(x1, 0x6464u, 0x5140u)), b1152)),
+                         h2u(__hsub2(u2h(__byte_perm(x1, 0x6464u, 0x5342u)), b1152)));
+                const float2 kd = scales(kd2, t, blk);
+                sc[t][0] = fmaf(kd.x, c[0], sc[t][0]);
+                sc[t][1] = fmaf(kd.y, c[1], sc[t][1]);
+            }
+        }
+
+        // ---- warp-local online softmax (log2 domain) for row g over the warp's 16 keys ----
+        float sv[2][2];
+        float mx = -CUDART_INF_F;
 #pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                const int c = 2 * blk + c2;  // logical 16-byte chunk of the row
-                const uint4 raw = *reinterpret_cast<const uint4*>(krow + ((c ^ (key & 7)) << 4));
-                const uint32_t w[4] = {raw.x ^ 0x80808080u, raw.y ^ 0x80808080u,
-                                       raw.z ^ 0x80808080u, raw.w ^ 0x80808080u};
+        for (int t = 0; t < 2; ++t)
 #pragma unroll
-                for (int uu = 0; uu < 4; ++uu) {
-                    const float k0 = s8_to_f(w[uu], 0), k1 = s8_to_f(w[uu], 1);
-                    const float k2 = s8_to_f(w[uu], 2), k3 = s8_to_f(w[uu], 3);
-                    const int qo = (c - 4 * hf) * 16 + uu * 4;
+            for (int j = 0; j < 2; ++j) {
+                const float v = (kbase + 8 * t + 2 * q + j <= kend) ? sc[t][j] * a.q_scale : -CUDART_INF_F;
+                sv[t][j] = v;
+                mx = fmaxf(mx, v);
+            }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        // the reference max moves only when the row's max exceeds it by more than 2^8
+        const bool need = mx > m_run + 8.0f;
+        if (__any_sync(0xffffffffu, need)) {
+            const float mn = need ? fmaxf(m_run, mx) : m_run;
+            const float alpha = (mn == m_run) ? 1.0f : ex2_approx(m_run - mn);  // 0 when m_run was -inf
+            m_run = mn;
+            l_run *= alpha;
 #pragma unroll
-                    for (int r = 0; r < ROWS; ++r) {
-                        const float4 qv = *reinterpret_cast<const float4*>(qh + r * 2 * kQHalf + qo);
-                        part[r] = fmaf(qv.x, k0, part[r]);
-                        part[r] = fmaf(qv.y, k1, part[r]);
-                        part[r] = fmaf(qv.z, k2, part[r]);
-                        part[r] = fmaf(qv.w, k3, part[r]);
-                    }
+            for (int nt = 0; nt < 16; ++nt) {
+                o[nt][0] *= alpha;
+                o[nt][1] *= alpha;
+            }
+        }
+        const float mu = (m_run == -CUDART_INF_F) ? 0.0f : m_run;
+        float p[2][2];
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                p[t][j] = ex2_approx(sv[t][j] - mu);  // 2^-inf = 0
+                l_run += p[t][j];                       // this lane's share of the row sum
+            }
+
+        // ---- PV ----
+        const uint8_t* vst = sb + kStageVq;
+#pragma unroll
+        for (int blk = 0; blk < kBlocks; ++blk) {
+            // probabilities x the V scale of block blk, as the A operand
+            const float2 dv0 = scales(vd2, 0, blk), dv1 = scales(vd2, 1, blk);
+            const uint32_t pa0 = h2u(__floats2half2_rn(p[0][0] * dv0.x, p[0][1] * dv0.y));
+            const uint32_t pa1 = h2u(__floats2half2_rn(p[1][0] * dv1.x, p[1][1] * dv1.y));
+            // V code words of the lane's keys 2q+j (t = 0) and 8+2q+j (t = 1):
+            // the four codes of dims 32 blk + 4g + {0..3}
+            uint32_t wv[2][2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int key = wkey + 8 * t + 2 * q + j;
+                    if constexpr (VT == kVQ8_0)
+                        wv[t][j] = *reinterpret_cast<const uint32_t*>(vst + key * kHeadDim + 32 * blk + 4 * g) ^
+                                   0x80808080u;
+                    else
+                        wv[t][j] = *reinterpret_cast<const uint32_t*>(vst + key * 64 + 16 * blk + 4 * (g & 3));
                 }
-            }
-            const float kd = __half2float(
-                *reinterpret_cast<const __half*>(sb + kStageKd + key * (kBlocks * 2) + blk * 2));
 #pragma unroll
-            for (int r = 0; r < ROWS; ++r) s[r] = fmaf(kd, part[r], s[r]);
-        }
-
-        // ---- warp-local online softmax; p' = p * d_v for this lane's two blocks ----
-        // The reference max m_run only moves when some score of the warp
-        // exceeds it by more than 2^8 (one warp vote per row in the common
-        // case); probabilities are then at most 2^8, exact enough in fp32.
-        const __half2 dv2 = *reinterpret_cast<const __half2*>(sb + kStageVd + key * (kBlocks * 2) + hf * 4);
-        const float dva = __low2float(dv2), dvb = __high2float(dv2);
-        float pa[PR], pb[PR];
+            for (int m = 0; m < 4; ++m) {
+                const uint32_t sel = (uint32_t)m | ((uint32_t)(4 + m) << 8);  // byte m of both words -> bytes 0, 2
+                uint32_t bv[2];
 #pragma unroll
-        for (int r = 0; r < PR; ++r) pa[r] = pb[r] = 0.0f;
-#pragma unroll
-        for (int r = 0; r < ROWS; ++r) {
-            s[r] += __shfl_xor_sync(0xffffffffu, s[r], 1);
-            if (kpos > sKend[r]) s[r] = -CUDART_INF_F;
-            if (__any_sync(0xffffffffu, s[r] > m_run[r] + 8.0f)) {
-                float mx = s[r];
-#pragma unroll
-                for (int off = 2; off <= 16; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-                const float mn = fmaxf(m_run[r], mx);
-                const float alpha = ex2_approx(m_run[r] - mn);  // 0 when m_run was -inf
-                m_run[r] = mn;
-                l_run[r] *= alpha;
-                acc[r][0] *= alpha; acc[r][1] *= alpha;
-                acc[r][2] *= alpha; acc[r][3] *= alpha;
-            }
-            const float mu = (m_run[r] == -CUDART_INF_F) ? 0.0f : m_run[r];
-            const float p = ex2_approx(s[r] - mu);
-            pa[r] = p * dva;
-            pb[r] = p * dvb;
-            if (!hf) l_run[r] += p;  // this lane's share of the row sum (reduced once at the end)
-        }
-        {
-            float* pdst_a = sPw + (2 * hf) * SB + kl * PR;
-            float* pdst_b = sPw + (2 * hf + 1) * SB + kl * PR;
-#pragma unroll
-            for (int r4 = 0; r4 < PR; r4 += 4) {
-                *reinterpret_cast<float4*>(pdst_a + r4) = make_float4(pa[r4], pa[r4 + 1], pa[r4 + 2], pa[r4 + 3]);
-                *reinterpret_cast<float4*>(pdst_b + r4) = make_float4(pb[r4], pb[r4 + 1], pb[r4 + 2], pb[r4 + 3]);
-            }
-        }
-        __syncwarp();
-
-        // ---- PV over the warp's 16 keys: lane = dims {32b+2i, +1, +16, +17} ----
-        const uint8_t* vq_base = VT == kVQ8_0
-            ? sb + kStageVq + (warp * kWarpKeys) * kHeadDim + vb * 32 + 2 * vi
-            : sb + kStageVq + (warp * kWarpKeys) * 64 + vb * 16 + 2 * vi;
-        const float* p_base = sPw + vb * SB;
-#pragma unroll 4
-        for (int kk = 0; kk < kWarpKeys; ++kk) {
-            float v0, v1, v2, v3;
-            if constexpr (VT == kVQ8_0) {
-                // int8 codes of dims 32b+2i, +1 and 32b+2i+16, +17
-                const uint32_t lo = *reinterpret_cast<const uint16_t*>(vq_base + kk * kHeadDim);
-                const uint32_t hi = *reinterpret_cast<const uint16_t*>(vq_base + kk * kHeadDim + 16);
-                const uint32_t w = (lo | (hi << 16)) ^ 0x80808080u;
-                v0 = s8_to_f(w, 0);
-                v1 = s8_to_f(w, 1);
-                v2 = s8_to_f(w, 2);
-                v3 = s8_to_f(w, 3);
-            } else {
-                const uint32_t code = *reinterpret_cast<const uint16_t*>(vq_base + kk * 64);
-                v0 = q4_to_f(code & 0xFu);          // dim 32b+2i
-                v2 = q4_to_f((code >> 4) & 0xFu);   // dim 32b+2i+16
-                v1 = q4_to_f((code >> 8) & 0xFu);   // dim 32b+2i+1
-                v3 = q4_to_f((code >> 12) & 0xFu);  // dim 32b+2i+17
-            }
-            const float* pr = p_base + kk * PR;
-            float pv[PR];
-            *reinterpret_cast<float4*>(pv) = *reinterpret_cast<const float4*>(pr);
-            if (PR == 8) *reinterpret_cast<float4*>(pv + 4) = *reinterpret_cast<const float4*>(pr + 4);
-#pragma unroll
-            for (int r = 0; r < ROWS; ++r) {
-                acc[r][0] = fmaf(pv[r], v0, acc[r][0]);
-                acc[r][1] = fmaf(pv[r], v1, acc[r][1]);
-                acc[r][2] = fmaf(pv[r], v2, acc[r][2]);
-                acc[r][3] = fmaf(pv[r], v3, acc[r][3]);
+                for (int t = 0; t < 2; ++t) {
+                    const uint32_t pr = __byte_perm(wv[t][0], wv[t][1], sel);
+                    if constexpr (VT == kVQ8_0)
+                        bv[t] = h2u(__hsub2(u2h((pr & 0x00ff00ffu) | 0x64006400u), b1152));
+                    else
+                        bv[t] = h2u(__hsub2(u2h(((pr >> (4 * (g >> 2))) & 0x000f000fu) | 0x64006400u), b1032));
+                }
+                float c[4] = {o[4 * blk + m][0], o[4 * blk + m][1], zr0, zr1};
+                mma16816(c, pa0, pa1, bv[0], bv[1]);
+                o[4 * blk + m][0] = c[0];
+                o[4 * blk + m][1] = c[1];
             }
         }
         __syncwarp();
@@ -497,22 +519,22 @@ __global__ void __launch_bounds__(kThreads, 2)
     ok = __syncthreads_and(ok);
     if (!ok) return;  // a bounded wait gave up; the error word is set
 
-    // ---- merge the eight warps' (m, l, acc) into the split's partial ----
-#pragma unroll
-    for (int r = 0; r < ROWS; ++r)
-#pragma unroll
-        for (int off = 1; off <= 16; off <<= 1) l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], off);
+    // ---- merge the eight warps' (m, l, O) into the split's partial ----
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
     float* red = reinterpret_cast<float*>(stage);          // [warps][ROWS][128]
     float* sml = red + kWarps * ROWS * kHeadDim;           // [warps][ROWS][2]
-    const int d0 = vb * 32 + 2 * vi;
+    if (g < ROWS) {
+        float* dst = red + (warp * ROWS + g) * kHeadDim;
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r) {
-        float* dst = red + (warp * ROWS + r) * kHeadDim;
-        *reinterpret_cast<float2*>(dst + d0) = make_float2(acc[r][0], acc[r][1]);
-        *reinterpret_cast<float2*>(dst + d0 + 16) = make_float2(acc[r][2], acc[r][3]);
-        if (lane == 0) {
-            sml[(warp * ROWS + r) * 2] = m_run[r];
-            sml[(warp * ROWS + r) * 2 + 1] = l_run[r];
+        for (int nt = 0; nt < 16; ++nt) {
+            const int d = 32 * (nt >> 2) + 8 * q + (nt & 3);  // columns 2q, 2q+1 -> dims d, d + 4
+            dst[d] = o[nt][0];
+            dst[d + 4] = o[nt][1];
+        }
+        if (q == 0) {
+            sml[(warp * ROWS + g) * 2] = m_run;
+            sml[(warp * ROWS + g) * 2 + 1] = l_run;
         }
     }
     __syncthreads();
