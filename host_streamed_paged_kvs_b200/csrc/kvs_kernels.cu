@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* stage = smem;
-    uint32_t* sQf = reinterpret_cast<uint32_t*>(smem + G::kOffQ);  // [32 lanes][16] Q fragments
+    uint32_t* sQf = reinterpret_cast<uint32_t*>(smem + G::kOffQ);  // [4 blocks][32 lanes][4] Q fragments
     int* sKend = reinterpret_cast<int*>(smem + G::kOffKend);           // last visible key per row
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + G::kOffBar);   // [kStages]
     uint64_t* empty = full + kStages;                               // [kStages]
@@ -297,13 +297,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         const bool vr = g < rows_here;
         const int lr = row_begin + g;
         const __half* qrow = a.q + ((size_t)(lr / a.group) * a.n_qh + h * a.group + (lr % a.group)) * kHeadDim;
-        uint32_t* qf = sQf + tid * 16;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             const int d0 = 32 * (kk >> 1) + 8 * q + 4 * (kk & 1);
             const uint2 v = vr ? *reinterpret_cast<const uint2*>(qrow + d0) : make_uint2(0u, 0u);
-            qf[2 * kk] = v.x;
-            qf[2 * kk + 1] = v.y;
+            uint32_t* qf = sQf + ((kk >> 1) * 32 + tid) * 4 + 2 * (kk & 1);  // lane-contiguous per block
+            qf[0] = v.x;
+            qf[1] = v.y;
         }
     }
     if (tid < ROWS)  // row r sees keys 0 .. min(len-1, its query position); padding rows none
@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     //   columns, and the probabilities carry the V scale of block b (one fp16
     //   rounding of p * d_v; the codes q - 8 are exact in fp16).
     const int g = lane >> 2, q = lane & 3;
-    const uint4* qfrag = reinterpret_cast<const uint4*>(sQf + lane * 16);  // block b: qfrag[b]
+    const uint4* qfrag = reinterpret_cast<const uint4*>(sQf) + lane;  // block b: qfrag[32 b]
     const int kend = g < ROWS ? sKend[g] : -1;  // last visible key of this lane's row
     float o[16][2];                              // O (row g; dims of n-tile nt, columns 2q, 2q+1)
 #pragma unroll
@@ -402,13 +402,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int kbase = (a.page0 + (sg >> 1)) * kPageTokens + (sg & 1) * kStageKeys + warp * kWarpKeys;
         const int wkey = warp * kWarpKeys;  // first key of this warp within the stage
 
-        // K / V scale of block blk of this lane's key wkey + 8t + 2q + j
-        const __half2* kd2 = reinterpret_cast<const __half2*>(sb + kStageKd + (wkey + 2 * q) * (kBlocks * 2));
-        const __half2* vd2 = reinterpret_cast<const __half2*>(sb + kStageVd + (wkey + 2 * q) * (kBlocks * 2));
-        // keys 2q, 2q+1 (t = 0) and 8+2q, 8+2q+1 (t = 1): scale of block blk as a pair (j = 0, 1)
-        auto scales = [&](const __half2* base, int t, int blk) {
-            const __half* hb = reinterpret_cast<const __half*>(base + t * 8 * (kBlocks / 2));
-            return make_float2(__half2float(hb[blk]), __half2float(hb[kBlocks + blk]));
+        // The score tile's column n of n-tile t is key wkey + 8t + kperm(n): the
+        // eight keys of a column half-range sit at even / odd rows, so the K
+        // operand loads of a half warp hit distinct banks of the swizzled rows.
+        // This lane's keys (columns 2q + j) are wkey + 8t + k0 / k1.
+        const int k0 = 2 * ((2 * q) & 3) + ((2 * q) >> 2), k1 = 2 * ((2 * q + 1) & 3) + ((2 * q + 1) >> 2);
+        // K / V scale of block blk of this lane's keys of n-tile t, as a pair (j = 0, 1)
+        auto scales = [&](int off, int t, int blk) {
+            const __half* h0 = reinterpret_cast<const __half*>(sb + off + (wkey + 8 * t + k0) * (kBlocks * 2));
+            const __half* h1 = reinterpret_cast<const __half*>(sb + off + (wkey + 8 * t + k1) * (kBlocks * 2));
+            return make_float2(__half2float(h0[blk]), __half2float(h1[blk]));
         };
 
         // ---- QK^T ----
@@ -416,10 +419,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint8_t* kst = sb + kStageKq;
 #pragma unroll 1
         for (int blk = 0; blk < kBlocks; ++blk) {
-            const uint4 qb = qfrag[blk];  // k-steps 2 blk (x, y) and 2 blk + 1 (z, w)
+            const uint4 qb = qfrag[32 * blk];  // k-steps 2 blk (x, y) and 2 blk + 1 (z, w)
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
-                const int key = wkey + 8 * t + g;  // this lane's column of the K operand
+                const int key = wkey + 8 * t + 2 * (g & 3) + (g >> 2);  // this lane's column of the K operand
                 const int chunk = 2 * blk + (q >> 1);
                 const uint2 w = *reinterpret_cast<const uint2*>(kst + key * kHeadDim + ((chunk ^ (key & 7)) << 4) +
                                                                 8 * (q & 1));
@@ -431,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mma16816(c, qb.z, qb.w,
                          h2u(__hsub2(u2h(__byte_perm(x1, 0x6464u, 0x5140u)), b1152)),
                          h2u(__hsub2(u2h(__byte_perm(x1, 0x6464u, 0x5342u)), b1152)));
-                const float2 kd = scales(kd2, t, blk);
+                const float2 kd = scales(kStageKd, t, blk);
                 sc[t][0] = fmaf(kd.x, c[0], sc[t][0]);
                 sc[t][1] = fmaf(kd.y, c[1], sc[t][1]);
             }
@@ -444,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int t = 0; t < 2; ++t)
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const float v = (kbase + 8 * t + 2 * q + j <= kend) ? sc[t][j] * a.q_scale : -CUDART_INF_F;
+                const float v = (kbase + 8 * t + (j ? k1 : k0) <= kend) ? sc[t][j] * a.q_scale : -CUDART_INF_F;
                 sv[t][j] = v;
                 mx = fmaxf(mx, v);
             }
@@ -478,17 +481,17 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int blk = 0; blk < kBlocks; ++blk) {
             // probabilities x the V scale of block blk, as the A operand
-            const float2 dv0 = scales(vd2, 0, blk), dv1 = scales(vd2, 1, blk);
+            const float2 dv0 = scales(kStageVd, 0, blk), dv1 = scales(kStageVd, 1, blk);
             const uint32_t pa0 = h2u(__floats2half2_rn(p[0][0] * dv0.x, p[0][1] * dv0.y));
             const uint32_t pa1 = h2u(__floats2half2_rn(p[1][0] * dv1.x, p[1][1] * dv1.y));
-            // V code words of the lane's keys 2q+j (t = 0) and 8+2q+j (t = 1):
-            // the four codes of dims 32 blk + 4g + {0..3}
+            // V code words of this lane's keys (k0, k1 of n-tiles 0 and 1): the
+            // four codes of dims 32 blk + 4g + {0..3}
             uint32_t wv[2][2];
 #pragma unroll
             for (int t = 0; t < 2; ++t)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const int key = wkey + 8 * t + 2 * q + j;
+                    const int key = wkey + 8 * t + (j ? k1 : k0);
                     if constexpr (VT == kVQ8_0)
                         wv[t][j] = *reinterpret_cast<const uint32_t*>(vst + key * kHeadDim + 32 * blk + 4 * g) ^
                                    0x80808080u;
