@@ -528,7 +528,8 @@ def run_gpu(args, w: W.Workload):
         if n_zc > 0:
             achieved = st_prof["bytes_decode_zc"] / (ms_zc * 1e-3) / 1e9
             kinds["decode_kernel_in_place"] = (ms_zc, {
-                "bound": "h2d", "achieved": achieved, "peak": h2d_peak, "unit": "GB/s",
+                "bound": "h2d", "bound_note": "the host-to-device PCIe link: the launch reads host memory",
+                "achieved": achieved, "peak": h2d_peak, "unit": "GB/s",
                 "frac": achieved / h2d_peak, "traffic": zc_traffic("dram"),
                 "sysmem_traffic": zc_traffic("sysmem"),
                 "traffic_note": "traffic: DRAM bytes of a launch (the split partials); sysmem_traffic: "
@@ -569,7 +570,8 @@ def run_gpu(args, w: W.Workload):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f16*f16->f32",  # tensor-core operands (exact codes), fp32 accumulate/softmax
+        "data": "synthetic",
         "config": {"workload": w.name, "ctx": w.ctx, "n_layers": L, "n_q": w.n_q,
                    "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": 128,
                    "kv_types": "K q8_0 / V " + ("q8_0" if w.type_v == 8 else "q4_0"),
