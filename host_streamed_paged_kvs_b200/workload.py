@@ -88,7 +88,7 @@ DEFAULT_BENCH = "streamed_decode_32k"
 # place from the mapped pinned history while the copy engine brings the rest
 # through the ring: in-place reads pay no per-copy cost, and the ring keeps
 # copying ahead into the next layer.  Tuned on the 32K streamed decode
-# workload (75-85 % within noise of each other, ring-only 4 % slower).
+# workload (70-90 % within noise of each other, ring-only 4 % slower).
 ZERO_COPY_PCT = 80
 
 
