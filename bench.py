@@ -44,8 +44,8 @@ NCU_TRAFFIC = {
                       "workload": "streamed_decode_32k", "resident": 27296256, "ring": 1737472,
                       # in-place launches (51 pages): DRAM bytes, and host-memory bytes read over PCIe
                       "in_place": 35328, "in_place_sysmem": 21725184},
-    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "c51cd9a85718b053",
-                         "workload": "prefill_chunk_64k", "resident": 37882880, "ring": 6078976},
+    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "44a34bfc87d20120",
+                         "workload": "prefill_chunk_64k", "resident": 35606272, "ring": 6079232},
 }
 
 

@@ -457,15 +457,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int sg = raw0 + (i >> 1);
             const int kbase = (a.page0 + (sg >> 1)) * kPageTokens + (sg & 1) * kRawKeys + (i & 1) * kSubKeys;
             float v[64];
-            if (warp_active) {
-                float t[32];
-                tmem_ld32(taddr + kColS + b * kSubKeys + lane_off, t);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = t[e];
-                tmem_ld32(taddr + kColS + b * kSubKeys + lane_off + 32, t);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[32 + e] = t[e];
-            }
+            if (warp_active) tmem_ld64(taddr + kColS + b * kSubKeys + lane_off, v);
             // S buffer b may be overwritten from here on
             tc_fence_before();
             __syncwarp();
@@ -519,8 +511,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         tmem_st32(taddr + kColO + lane_off + c * 32, o);
                     }
                 }
-                tmem_st32u(taddr + kColP + b * (kSubKeys / 2) + lane_off, pk);
-                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                tmem_st32u(taddr + kColP + b * (kSubKeys / 2) + lane_off, pk);  // waits for the store
             }
             tc_fence_before();
             __syncwarp();

@@ -12,7 +12,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("n_q,heads,pct", [(1, (32, 8), 0), (1, (32, 8), 80), (1, (32, 8), 100),
-                                            (4, (40, 8), 0)])
+                                            (4, (40, 8), 0), (64, (40, 8), 0)])
 def test_graph_captured_step_matches_plain_calls(n_q, heads, pct):
     t = torch()
     from host_streamed_paged_kvs_b200 import kvs
