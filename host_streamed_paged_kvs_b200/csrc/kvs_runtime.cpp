@@ -67,22 +67,23 @@ long auto_resident(long max_ctx, size_t page_bytes, int n_layers) {
 }
 
 // Split layout, in half-page stages per split.
-//  * CUDA-core decode (<= 8 query rows per kv head): resident splits sized so
-//    the resident launch has about two CTAs per SM (1..4 stages each), one
-//    stage per split inside a ring chunk so a chunk's kernel spreads over many
-//    SMs.
-//  * tensor-core path (more rows per kv head: verify batches, prefill chunks)
-//    and very wide decode: at most 8 resident splits and one split per ring
-//    chunk, which keeps the partial buffer and the merge small.
+//  * decode kernel (<= 8 query rows per kv head, warp-level mma.sync): resident
+//    splits sized so the resident launch has about two CTAs per SM, one stage
+//    per split inside a ring chunk so a chunk's kernel spreads over many SMs;
+//    decode batches wider than 64 rows in all: at most 8 resident splits and
+//    one split per ring chunk, which keeps the partial buffer and merge small.
+//  * tcgen05 kernel (more rows per kv head: verify batches, prefill chunks):
+//    one CTA per SM; resident splits chosen for the fewest waves x stages, and
+//    per ring chunk as many splits as fit one wave beside the other units.
 constexpr int kSmallRows = 64;
 constexpr int kTargetCtas = 296;  // 148 SMs x 2 resident CTAs
-constexpr int kMaxCudaCoreRows = 8;
+constexpr int kMaxDecodeRows = 8;
 
-bool use_tensor_cores(const kvs_config& c, int n_q) { return n_q * (c.n_q_heads / c.n_kv_heads) > kMaxCudaCoreRows; }
+bool use_tcgen05(const kvs_config& c, int n_q) { return n_q * (c.n_q_heads / c.n_kv_heads) > kMaxDecodeRows; }
 bool wide_regime(const kvs_config& c, int n_q) { return n_q * c.n_q_heads > kSmallRows; }
 int m_tiles(const kvs_config& c, int n_q) { return (n_q * (c.n_q_heads / c.n_kv_heads) + 127) / 128; }
 
-// Tensor-core path: splits sized for about one CTA per SM per ring chunk and
+// tcgen05 path: splits sized for about one CTA per SM per ring chunk and
 // about two waves over the resident pages (the kernel holds one CTA per SM).
 constexpr int kSms = 148;
 
@@ -90,7 +91,7 @@ constexpr int kSms = 148;
 // equal share of the launch's half-page stages).
 int res_splits(const kvs_config& c, long R_eff, int n_q) {
     const long stages = 2 * R_eff;
-    if (use_tensor_cores(c, n_q)) {
+    if (use_tcgen05(c, n_q)) {
         // one CTA per SM: pick the split count that minimizes waves x stages
         // per split on a full machine (ties -> fewer splits, fewer partials)
         const long units = (long)c.n_kv_heads * m_tiles(c, n_q);
@@ -102,14 +103,14 @@ int res_splits(const kvs_config& c, long R_eff, int n_q) {
         return (int)best;
     }
     if (wide_regime(c, n_q)) return (int)std::min(stages, 8L);
-    // CUDA-core decode: one wave of two CTAs per SM
+    // decode kernel: one wave of two CTAs per SM
     const long per_split = (long)c.n_kv_heads * ((n_q * (c.n_q_heads / c.n_kv_heads) + 7) / 8);
     return (int)std::min(stages, std::max(1L, (long)kTargetCtas / per_split));
 }
 
 int ring_splits(const kvs_config& c, int n_q, int chunk_pages) {
     const int stages = 2 * chunk_pages;
-    if (use_tensor_cores(c, n_q)) {
+    if (use_tcgen05(c, n_q)) {
         // at most one wave, leaving SMs to the resident launch when a chunk's
         // units cannot fill the machine twice
         const int units = c.n_kv_heads * m_tiles(c, n_q);
@@ -123,7 +124,7 @@ int ring_splits(const kvs_config& c, int n_q, int chunk_pages) {
 // CTA per SM (the resident and ring launches share the SMs); the ring brings
 // the older ones.
 long zero_copy_pages(const kvs_config& c, int n_q, long S) {
-    if (use_tensor_cores(c, n_q) || c.zero_copy_pct <= 0) return 0;
+    if (use_tcgen05(c, n_q) || c.zero_copy_pct <= 0) return 0;
     return std::min(S, (S * c.zero_copy_pct + 50) / 100);
 }
 int zc_splits(const kvs_config& c, long S_zc, int n_q) {
@@ -879,7 +880,7 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     float* dout = out_alias ? out_alias : (host_out ? kv->stage_out : out);
     float* dlse = lse ? (lse_alias ? lse_alias : (host_lse ? kv->stage_lse : lse)) : nullptr;
 
-    const bool tc = use_tensor_cores(c, n_q);
+    const bool tc = use_tcgen05(c, n_q);
     if (tc && (reinterpret_cast<uintptr_t>(q) & 15))
         return fail(kv, KVS_E_INVAL, "q must be 16-byte aligned for multi-token attention");
     const long R = c.n_resident_pages;
