@@ -105,6 +105,9 @@ uint16_t oracle_float_to_half(float f) {
 /*   Q8_0: 2-byte fp16 scale d, then 32 signed bytes q      (34 bytes)        */
 /*   Q4_0: 2-byte fp16 scale d, then 16 bytes, byte j holding q_j in its low  */
 /*         nibble and q_{j+16} in its high nibble             (18 bytes)      */
+/*   Q5_0: 2-byte fp16 scale d, a 4-byte word whose bit j is bit 4 of q_j,    */
+/*         then 16 bytes holding the low 4 bits of q_j / q_{j+16} as Q4_0    */
+/*         does                                               (22 bytes)      */
 /* ------------------------------------------------------------------------ */
 
 void oracle_q8_0_block(const uint16_t x_h[32], uint8_t out[34]) {
@@ -153,6 +156,41 @@ void oracle_q4_0_block(const uint16_t x_h[32], uint8_t out[18]) {
     for (int j = 0; j < 16; ++j) out[2 + j] = (uint8_t)(q[j] | (q[j + 16] << 4));
 }
 
+/* Q5_0: the 5-bit member of the same family, one of the cache types the
+ * flash-attention build lists as legal ("RaymondHuang210129/llama.cpp-
+ * adaptive-kv-streaming", build section: -DGGML_CUDA_FA_QUANTS).  The pages
+ * give no rule; it is read as Q4_0's with 32 levels: d = (signed max)/-16,
+ * q = min(31, trunc(x/d + 16.5)), so x ~ d (q - 16). */
+void oracle_q5_0_block(const uint16_t x_h[32], uint8_t out[22]) {
+    float x[32];
+    float amax = 0.0f, m = 0.0f;
+    for (int i = 0; i < 32; ++i) {
+        x[i] = oracle_half_to_float(x_h[i]);
+        float a = fabsf(x[i]);
+        if (a > amax) { /* the first index of the largest |x| wins (strict) */
+            amax = a;
+            m = x[i];
+        }
+    }
+    float d = m / -16.0f; /* signed max over -16 */
+    uint16_t dh = oracle_float_to_half(d);
+    out[0] = (uint8_t)(dh & 0xff);
+    out[1] = (uint8_t)(dh >> 8);
+    int q[32];
+    for (int i = 0; i < 32; ++i) {
+        if (d == 0.0f) {
+            q[i] = 16;
+        } else {
+            int t = (int)(x[i] / d + 16.5f); /* argument >= 0.5: truncation */
+            q[i] = t < 31 ? t : 31;
+        }
+    }
+    uint32_t high = 0;
+    for (int i = 0; i < 32; ++i) high |= (uint32_t)(q[i] >> 4) << i;
+    for (int b = 0; b < 4; ++b) out[2 + b] = (uint8_t)(high >> (8 * b));
+    for (int j = 0; j < 16; ++j) out[6 + j] = (uint8_t)((q[j] & 15) | ((q[j + 16] & 15) << 4));
+}
+
 void oracle_dequant_q8_0(const uint8_t blk[34], double out[32]) {
     double d = oracle_half_to_double((uint16_t)(blk[0] | (blk[1] << 8)));
     for (int i = 0; i < 32; ++i) out[i] = d * (double)(int8_t)blk[2 + i];
@@ -166,10 +204,36 @@ void oracle_dequant_q4_0(const uint8_t blk[18], double out[32]) {
     }
 }
 
-/* bytes of one 32-value block of a V type (2 = Q4_0, 8 = Q8_0), 0 if unknown */
-static int v_block_bytes(int v_type) { return v_type == 2 ? 18 : (v_type == 8 ? 34 : 0); }
+void oracle_dequant_q5_0(const uint8_t blk[22], double out[32]) {
+    double d = oracle_half_to_double((uint16_t)(blk[0] | (blk[1] << 8)));
+    uint32_t high = (uint32_t)blk[2] | ((uint32_t)blk[3] << 8) | ((uint32_t)blk[4] << 16) | ((uint32_t)blk[5] << 24);
+    for (int j = 0; j < 16; ++j) {
+        int lo = (int)(blk[6 + j] & 0x0f) | (int)(((high >> j) & 1u) << 4);
+        int hi = (int)(blk[6 + j] >> 4) | (int)(((high >> (j + 16)) & 1u) << 4);
+        out[j] = d * (double)(lo - 16);
+        out[j + 16] = d * (double)(hi - 16);
+    }
+}
 
-/* K rows -> Q8_0 blocks; V rows -> Q4_0 (v_type 2) or Q8_0 (v_type 8) blocks */
+/* bytes of one 32-value block of a V type (2 = Q4_0, 6 = Q5_0, 8 = Q8_0),
+ * 0 if unknown */
+static int v_block_bytes(int v_type) {
+    return v_type == 2 ? 18 : (v_type == 6 ? 22 : (v_type == 8 ? 34 : 0));
+}
+
+static void v_block(int v_type, const uint16_t* x, uint8_t* out) {
+    if (v_type == 2) oracle_q4_0_block(x, out);
+    else if (v_type == 6) oracle_q5_0_block(x, out);
+    else oracle_q8_0_block(x, out);
+}
+
+static void v_dequant(int v_type, const uint8_t* blk, double* out) {
+    if (v_type == 2) oracle_dequant_q4_0(blk, out);
+    else if (v_type == 6) oracle_dequant_q5_0(blk, out);
+    else oracle_dequant_q8_0(blk, out);
+}
+
+/* K rows -> Q8_0 blocks; V rows -> Q4_0 (v_type 2), Q5_0 (6) or Q8_0 (8) blocks */
 int oracle_quantize_rows_t(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
                            uint8_t* k_blocks, uint8_t* v_blocks, int v_type) {
     int nb = dim / 32;
@@ -180,8 +244,7 @@ int oracle_quantize_rows_t(int n_rows, int dim, const uint16_t* k, const uint16_
             const uint16_t* kx = k + (size_t)r * dim + (size_t)b * 32;
             const uint16_t* vx = v + (size_t)r * dim + (size_t)b * 32;
             oracle_q8_0_block(kx, k_blocks + ((size_t)r * nb + b) * 34);
-            if (v_type == 2) oracle_q4_0_block(vx, v_blocks + ((size_t)r * nb + b) * 18);
-            else oracle_q8_0_block(vx, v_blocks + ((size_t)r * nb + b) * vbb);
+            v_block(v_type, vx, v_blocks + ((size_t)r * nb + b) * vbb);
         }
     }
     return 0;
@@ -196,7 +259,7 @@ void oracle_quantize_rows(int n_rows, int dim, const uint16_t* k, const uint16_t
 /* Attention over the quantized history, binary64.                            */
 /*                                                                            */
 /* k_blocks: [n_keys][n_kv][dim/32] Q8_0 blocks (token-major history)         */
-/* v_blocks: [n_keys][n_kv][dim/32] Q4_0 blocks (v_type 2) or Q8_0 (8)       */
+/* v_blocks: [n_keys][n_kv][dim/32] Q4_0 (v_type 2), Q5_0 (6) or Q8_0 (8)    */
 /* q:        [n_q][n_qh][dim] fp16; query j sits at absolute position pos0+j  */
 /*           and sees keys 0..pos0+j (causal).                                */
 /* q head h reads kv head h / (n_qh/n_kv) (contiguous grouping).              */
@@ -247,8 +310,7 @@ int oracle_attention_t(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
                 sum += p;
                 for (int b = 0; b < nb; ++b) {
                     const uint8_t* vblk = v_blocks + (((size_t)i * n_kv + g) * nb + b) * vbb;
-                    if (v_type == 2) oracle_dequant_q4_0(vblk, vd);
-                    else oracle_dequant_q8_0(vblk, vd);
+                    v_dequant(v_type, vblk, vd);
                     for (int t = 0; t < 32; ++t) o[b * 32 + t] += p * vd[t];
                 }
             }

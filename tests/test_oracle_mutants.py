@@ -15,6 +15,7 @@ import oracle
 import test_oracle_attention as TA
 import test_oracle_fp16 as TF
 import test_oracle_pages as TP
+import test_oracle_q5_0 as T5
 import test_oracle_quant as TQ
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "kvs_oracle.c")
@@ -32,6 +33,14 @@ MUTANTS = {
     "gqa interleaved": ("int g = h / group;", "int g = h % n_kv;"),
     "lse base 2": ("lse[(size_t)j * n_qh + h] = m + log(sum);", "lse[(size_t)j * n_qh + h] = m + log2(sum);"),
     "fp16 ties down": ("if (rem > 0x1000u || (rem == 0x1000u && (hm & 1u))) {", "if (rem > 0x1000u) {"),
+    "q5 last index wins": ("if (a > amax) { /* the first index", "if (a >= amax) { /* the first index"),
+    "q5 offset 16.0": ("(int)(x[i] / d + 16.5f)", "(int)(x[i] / d + 16.0f)"),
+    "q5 scale /-15": ("float d = m / -16.0f;", "float d = m / -15.0f;"),
+    "q5 no clamp": ("q[i] = t < 31 ? t : 31;", "q[i] = t;"),
+    "q5 high bits reversed": ("high |= (uint32_t)(q[i] >> 4) << i;", "high |= (uint32_t)(q[i] >> 4) << (31 - i);"),
+    "q5 dequant offset": ("out[j] = d * (double)(lo - 16);", "out[j] = d * (double)(lo - 15);"),
+    "v type dispatch": ("else if (v_type == 6) oracle_dequant_q5_0(blk, out);",
+                        "else if (v_type == 6) oracle_dequant_q4_0(blk, out);"),
     "resident window": ("if (page >= P - n_resident) {", "if (page > P - n_resident) {"),
     "auto floor": ("long floor_pages = (2048 + page_tokens - 1) / page_tokens;",
                    "long floor_pages = (4096 + page_tokens - 1) / page_tokens;"),
@@ -49,6 +58,8 @@ def pins():
         TP.test_auto_resident_matches_printed_numbers, TP.test_auto_resident_floor_and_ceiling,
         lambda: TP.test_page_location_invariants(1025, 4),
         TF.test_float_to_half_random,
+        T5.test_q5_0_hand_worked, T5.test_q5_0_dequant_of_hand_block, T5.test_q5_0_error_bound_and_range,
+        T5.test_q5_0_zero_query_is_uniform_mean, T5.test_q5_0_against_scipy_softmax_random,
     ]
 
 
