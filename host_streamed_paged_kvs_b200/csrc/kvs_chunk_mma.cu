@@ -72,13 +72,15 @@ static_assert(kKVBytes % 1024 == 0, "swizzled tiles need 1024-B alignment");
 
 // Raw-stage and shared-memory layout by V type.  Raw stage (128 keys, as the
 // pages hold them): Kq [128][128] @ 0, Kd @ 16384, Vq @ 17408 (64 B per key
-// for Q4_0 V, 128 B for Q8_0 V), Vd after it.  Shared memory: two raw
+// for Q4_0 and Q5_0 V, 128 B for Q8_0 V), the Q5_0 fifth bits (16 B per key),
+// Vd after them.  Shared memory: two raw
 // stages, then [2] x (K^hi | K^lo), [3] x V^, the barriers, the TMEM slot and
 // the abort flag (Q4_0 V: K^ @ 53248, V^ @ 118784, barriers @ 167936).
 template <int VT>
 struct TcGeom {
     static constexpr int kRawVq = kRawKd + kRawKeys * kBlocks * 2;                    // 17408
-    static constexpr int kRawVd = kRawVq + kRawKeys * PageGeom<VT>::kVqRow;
+    static constexpr int kRawVh = kRawVq + kRawKeys * PageGeom<VT>::kVqRow;           // Q5_0 fifth bits
+    static constexpr int kRawVd = kRawVh + kRawKeys * PageGeom<VT>::kVhRow;
     static constexpr int kRawBytes = kRawVd + kRawKeys * kBlocks * 2;
     static constexpr size_t kOffK = (size_t)kRawStages * kRawBytes;
     static constexpr size_t kOffV = kOffK + kKBufs * 2 * kKVBytes;
@@ -91,6 +93,7 @@ struct TcGeom {
     static_assert(kSmem <= 232448, "shared memory budget");
 };
 static_assert(TcGeom<kVQ4_0>::kOffBar == 167936, "Q4_0 geometry");
+static_assert(TcGeom<kVQ5_0>::kRawBytes == 28672, "Q5_0 raw stage");
 
 // instruction descriptors: f16 x f16 -> f32, M = 128; A K-major;
 // S: N = 64, B K-major; PV: N = 128, B MN-major
@@ -165,13 +168,19 @@ __device__ __forceinline__ void mbar_arrive_cta(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Q5_0 V: bit 4 of the codes of dims j and j + 1 of a block (bits j, j + 1 of
+// its fifth-bit word hw), placed at bit 4 of the low and high fp16 halves
+__device__ __forceinline__ uint32_t fifth_bits(uint32_t hw, int j) {
+    return (((hw >> j) & 1u) << 4) | (((hw >> (j + 1)) & 1u) << 20);
+}
+
 
 template <int VT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     chunk_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap) {
     using TG = TcGeom<VT>;
     using PG = PageGeom<VT>;
-    constexpr int kRawVq = TG::kRawVq, kRawVd = TG::kRawVd, kRawBytes = TG::kRawBytes;
+    constexpr int kRawVq = TG::kRawVq, kRawVh = TG::kRawVh, kRawVd = TG::kRawVd, kRawBytes = TG::kRawBytes;
     constexpr size_t kOffK = TG::kOffK, kOffV = TG::kOffV, kOffBar = TG::kOffBar;
     constexpr size_t kOffTmem = TG::kOffTmem, kOffAbort = TG::kOffAbort;
     extern __shared__ uint8_t smem_raw[];
@@ -276,6 +285,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tma_load_2d(dst + kRawKq, &kmap, 0, krow, b);
                 bulk_load(dst + kRawKd, ph + kOffKd + half * (kRawKeys * kBlocks * 2), kRawKeys * kBlocks * 2, b);
                 bulk_load(dst + kRawVq, ph + PG::kOffVq + half * (kRawKeys * PG::kVqRow), kRawKeys * PG::kVqRow, b);
+                if constexpr (PG::kVhRow > 0)
+                    bulk_load(dst + kRawVh, ph + PG::kOffVh + half * (kRawKeys * PG::kVhRow), kRawKeys * PG::kVhRow, b);
                 bulk_load(dst + kRawVd, ph + PG::kOffVd + half * (kRawKeys * kBlocks * 2), kRawKeys * kBlocks * 2, b);
             };
             int ir = 0;        // next raw stage to load
@@ -408,22 +419,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
             } else
             for (int un = ptid; un < kSubKeys * kBlocks; un += kProdThreads) {
+                // Q4_0 V: V^ = fp16(d * (q - 8)); Q5_0 V: the same nibbles with
+                // the fifth bits added, V^ = fp16(d * (q - 16))
                 const int blk = un & 3, kloc = un >> 2;
                 const int key = sub * kSubKeys + kloc;
                 const uint4 q = *reinterpret_cast<const uint4*>(rb + kRawVq + key * 64 + blk * 16);
                 const __half dh = *reinterpret_cast<const __half*>(rb + kRawVd + key * 8 + blk * 2);
+                uint32_t hw = 0;
+                if constexpr (VT == kVQ5_0) hw = *reinterpret_cast<const uint32_t*>(rb + kRawVh + key * 16 + blk * 4);
                 const __half2 d2 = __halves2half2(dh, dh);
-                const __half2 bias = __float2half2_rn(1032.0f);
+                const __half2 bias = __float2half2_rn(VT == kVQ5_0 ? 1040.0f : 1032.0f);
                 const uint32_t w[4] = {q.x, q.y, q.z, q.w};
                 uint32_t lo[8], hi[8];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const uint32_t p01 = __byte_perm(w[u], 0u, 0x4140u);  // bytes 4u, 4u+1 at positions 0, 2
                     const uint32_t p23 = __byte_perm(w[u], 0u, 0x4342u);
-                    lo[2 * u] = h2u(__hmul2(__hsub2(u2h((p01 & 0x000F000Fu) | 0x64006400u), bias), d2));
-                    lo[2 * u + 1] = h2u(__hmul2(__hsub2(u2h((p23 & 0x000F000Fu) | 0x64006400u), bias), d2));
-                    hi[2 * u] = h2u(__hmul2(__hsub2(u2h(((p01 >> 4) & 0x000F000Fu) | 0x64006400u), bias), d2));
-                    hi[2 * u + 1] = h2u(__hmul2(__hsub2(u2h(((p23 >> 4) & 0x000F000Fu) | 0x64006400u), bias), d2));
+                    lo[2 * u] = h2u(__hmul2(
+                        __hsub2(u2h((p01 & 0x000F000Fu) | fifth_bits(hw, 4 * u) | 0x64006400u), bias), d2));
+                    lo[2 * u + 1] = h2u(__hmul2(
+                        __hsub2(u2h((p23 & 0x000F000Fu) | fifth_bits(hw, 4 * u + 2) | 0x64006400u), bias), d2));
+                    hi[2 * u] = h2u(__hmul2(
+                        __hsub2(u2h(((p01 >> 4) & 0x000F000Fu) | fifth_bits(hw, 16 + 4 * u) | 0x64006400u), bias), d2));
+                    hi[2 * u + 1] = h2u(__hmul2(
+                        __hsub2(u2h(((p23 >> 4) & 0x000F000Fu) | fifth_bits(hw, 18 + 4 * u) | 0x64006400u), bias), d2));
                 }
                 *reinterpret_cast<uint4*>(sVb + tile_off(kSubKeys, kloc, 32 * blk)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
                 *reinterpret_cast<uint4*>(sVb + tile_off(kSubKeys, kloc, 32 * blk + 8)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
@@ -563,6 +582,9 @@ cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ8_0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)TcGeom<kVQ8_0>::kSmem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ5_0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)TcGeom<kVQ5_0>::kSmem);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_acq_rel);
     }
@@ -570,6 +592,8 @@ cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n
     dim3 grid(n_splits, a.n_kv, m_tiles);
     if (a.v_type == kVQ8_0)
         chunk_mma_kernel<kVQ8_0><<<grid, kTcThreads, TcGeom<kVQ8_0>::kSmem, s>>>(a, *kmap);
+    else if (a.v_type == kVQ5_0)
+        chunk_mma_kernel<kVQ5_0><<<grid, kTcThreads, TcGeom<kVQ5_0>::kSmem, s>>>(a, *kmap);
     else
         chunk_mma_kernel<kVQ4_0><<<grid, kTcThreads, TcGeom<kVQ4_0>::kSmem, s>>>(a, *kmap);
     return cudaGetLastError();

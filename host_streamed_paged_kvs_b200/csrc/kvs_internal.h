@@ -38,27 +38,39 @@ static_assert(kPageHeadBytes == 53248, "page-head layout");
 
 // V type codes (the public KVS_TYPE_* values)
 constexpr int kVQ4_0 = 2;
+constexpr int kVQ5_0 = 6;
 constexpr int kVQ8_0 = 8;
 
-// Page-head geometry by V type.  Q4_0 V is the layout above; Q8_0 V stores
+// Page-head geometry by V type.  Q4_0 V is the layout above.  Q8_0 V stores
 // its codes like K (int8 [256 tok][128 dims], block b = dims 32b..32b+31):
 //   Kq @ 0, Kd @ 32,768, Vq int8 [256][128] @ 34,816, Vd @ 67,584; 69,632 B.
+// Q5_0 V keeps the low 4 bits of its codes as Q4_0 keeps its codes, and adds
+// the fifth bits, one 32-bit word per block (bit j = code j's bit 4):
+//   Vq u8 [256][4][16] @ 34,816, Vh u32 [256][4] @ 51,200, Vd @ 55,296; 57,344 B.
 template <int VT>
 struct PageGeom {
-    static_assert(VT == kVQ4_0 || VT == kVQ8_0, "V type");
+    static_assert(VT == kVQ4_0 || VT == kVQ5_0 || VT == kVQ8_0, "V type");
     static constexpr int kVqRow = VT == kVQ8_0 ? kHeadDim : kHeadDim / 2;  // V code bytes per token
+    static constexpr int kVhRow = VT == kVQ5_0 ? kBlocks * 4 : 0;         // V fifth-bit bytes per token
     static constexpr int kOffVq = kOffKd + kPageTokens * kBlocks * 2;       // 34816
-    static constexpr int kOffVd = kOffVq + kPageTokens * kVqRow;
+    static constexpr int kOffVh = kOffVq + kPageTokens * kVqRow;
+    static constexpr int kOffVd = kOffVh + kPageTokens * kVhRow;
     static constexpr int kHeadBytes = kOffVd + kPageTokens * kBlocks * 2;
     static constexpr int kRows = kHeadBytes / 128;
+    static constexpr int kVBlockBytes = VT == kVQ8_0 ? 34 : (VT == kVQ5_0 ? 22 : 18);  // canonical block
 };
 static_assert(PageGeom<kVQ4_0>::kHeadBytes == kPageHeadBytes && PageGeom<kVQ4_0>::kOffVd == kOffVd,
               "Q4_0 geometry");
 static_assert(PageGeom<kVQ8_0>::kHeadBytes == 69632 && PageGeom<kVQ8_0>::kHeadBytes % 128 == 0,
               "Q8_0 geometry");
+static_assert(PageGeom<kVQ5_0>::kHeadBytes == 57344 && PageGeom<kVQ5_0>::kOffVh == 51200 &&
+                  PageGeom<kVQ5_0>::kOffVd == 55296 && PageGeom<kVQ5_0>::kHeadBytes % 128 == 0,
+              "Q5_0 geometry");
 inline int page_head_bytes(int v_type) {
-    return v_type == kVQ8_0 ? PageGeom<kVQ8_0>::kHeadBytes : PageGeom<kVQ4_0>::kHeadBytes;
+    return v_type == kVQ8_0 ? PageGeom<kVQ8_0>::kHeadBytes
+                            : (v_type == kVQ5_0 ? PageGeom<kVQ5_0>::kHeadBytes : PageGeom<kVQ4_0>::kHeadBytes);
 }
+inline bool v_type_supported(int v_type) { return v_type == kVQ4_0 || v_type == kVQ5_0 || v_type == kVQ8_0; }
 
 // split partials: per split and query row, (m, l) in the log2 domain + acc[128]
 struct PartialBuffers {

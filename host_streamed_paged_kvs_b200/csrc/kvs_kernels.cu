@@ -36,8 +36,11 @@ __device__ __forceinline__ float q4_to_f(uint32_t c) {
 // Q8_0: d = amax/127 (binary32, correctly rounded), q = roundf(x/d).
 // Q4_0: m = value of largest |x| (first index on ties), d = m/-8,
 //       q = min(15, trunc(x/d + 8.5)), d == 0 -> q = 8.
+// Q5_0: the same with 32 levels: d = m/-16, q = min(31, trunc(x/d + 16.5)),
+//       d == 0 -> q = 16; the low 4 bits are packed as Q4_0's codes, the
+//       fifth bits in one 32-bit word per block (bit j = code j).
 // The stored scales are the fp16 (round-to-nearest-even) values of d.
-// K is always Q8_0; V is Q4_0 (VT = 2) or Q8_0 (VT = 8).
+// K is always Q8_0; V is Q4_0 (VT = 2), Q5_0 (VT = 6) or Q8_0 (VT = 8).
 // ----------------------------------------------------------------------------
 // Q8_0 of the 32-value block spread over 8 lanes (4 values each): the lane's
 // 4 codes packed in one word (byte u = code of value u), and the block scale
@@ -111,7 +114,11 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
         return;
     }
 
-    // ---- Q4_0 (V) ----
+    // ---- Q4_0 / Q5_0 (V) ----
+    constexpr bool kQ5 = VT == kVQ5_0;
+    constexpr float kNegLevels = kQ5 ? -16.0f : -8.0f;
+    constexpr float kRoundOff = kQ5 ? 16.5f : 8.5f;
+    constexpr int kTop = kQ5 ? 31 : 15, kMid = kQ5 ? 16 : 8;
     float va = 0.0f, vm = 0.0f;
     int vi = 1 << 30;
 #pragma unroll
@@ -126,16 +133,23 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
         const int pi = __shfl_xor_sync(0xffffffffu, vi, off);
         if (pa > va || (pa == va && pi < vi)) { va = pa; vm = pm; vi = pi; }
     }
-    const float dv = __fdiv_rn(vm, -8.0f);
+    const float dv = __fdiv_rn(vm, kNegLevels);
     uint32_t codes = 0;  // 4 codes of this lane, one per byte
+    uint32_t high = 0;   // Q5_0: bit 4 of code 4i+u at bit 4i+u
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-        int q = 8;
-        if (dv != 0.0f) q = min(15, static_cast<int>(__fadd_rn(__fdiv_rn(xv[u], dv), 8.5f)));
-        codes |= static_cast<uint32_t>(q) << (8 * u);
+        int q = kMid;
+        if (dv != 0.0f) q = min(kTop, static_cast<int>(__fadd_rn(__fdiv_rn(xv[u], dv), kRoundOff)));
+        codes |= static_cast<uint32_t>(q & 15) << (8 * u);
+        high |= static_cast<uint32_t>(q >> 4) << (4 * i + u);
     }
     const uint32_t partner = __shfl_xor_sync(0xffffffffu, codes, 4);  // codes j+16 for lanes i<4
-    const uint32_t vq = codes | (partner << 4);  // byte u: q_(4i+u) | q_(4i+u+16) << 4
+    const uint32_t vq = codes | (partner << 4);  // byte u: q_(4i+u) | q_(4i+u+16) << 4 (low 4 bits)
+    if constexpr (kQ5) {
+        high |= __shfl_xor_sync(0xffffffffu, high, 1);
+        high |= __shfl_xor_sync(0xffffffffu, high, 2);
+        high |= __shfl_xor_sync(0xffffffffu, high, 4);
+    }
     const __half dv_h = __float2half_rn(dv);
 
     // ---- stores: host history (always) and resident slot (if resident) ----
@@ -143,14 +157,15 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
         *reinterpret_cast<uint32_t*>(ph + kOffKq + t * kHeadDim + 4 * lane) = kq;
         if (i == 0) {
             *reinterpret_cast<__half*>(ph + kOffKd + t * 8 + 2 * b) = dk_h;
-            *reinterpret_cast<__half*>(ph + kOffVd + t * 8 + 2 * b) = dv_h;
+            *reinterpret_cast<__half*>(ph + G::kOffVd + t * 8 + 2 * b) = dv_h;
+            if constexpr (kQ5) *reinterpret_cast<uint32_t*>(ph + G::kOffVh + t * 16 + 4 * b) = high;
         }
-        if (i < 4) *reinterpret_cast<uint32_t*>(ph + kOffVq + t * 64 + b * 16 + 4 * i) = vq;
+        if (i < 4) *reinterpret_cast<uint32_t*>(ph + G::kOffVq + t * 64 + b * 16 + 4 * i) = vq;
     };
-    store(a.host_layer + (size_t)page * a.page_bytes + (size_t)h * kPageHeadBytes);
+    store(a.host_layer + (size_t)page * a.page_bytes + (size_t)h * G::kHeadBytes);
     if (page >= a.first_resident_page) {
         const int slot = page % a.n_resident;
-        store(a.res_layer + (size_t)slot * a.page_bytes + (size_t)h * kPageHeadBytes);
+        store(a.res_layer + (size_t)slot * a.page_bytes + (size_t)h * G::kHeadBytes);
     }
 }
 
@@ -158,6 +173,8 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
     const int rows = a.n_tok * a.n_kv;
     if (a.v_type == kVQ8_0)
         append_kernel<kVQ8_0><<<(rows + 3) / 4, 128, 0, s>>>(a);
+    else if (a.v_type == kVQ5_0)
+        append_kernel<kVQ5_0><<<(rows + 3) / 4, 128, 0, s>>>(a);
     else
         append_kernel<kVQ4_0><<<(rows + 3) / 4, 128, 0, s>>>(a);
     return cudaGetLastError();
@@ -179,8 +196,8 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
 //          block's partial score in fp32 and the block's K scale multiplies it;
 //   softmax: warp-local lazy running max per row (log2 domain);
 //   PV   : the probability times the V scale of each (key, block) is the A
-//          operand (one fp16 rounding), the V codes (q - 8 for Q4_0, q for
-//          Q8_0) exact in fp16 are the B operand.
+//          operand (one fp16 rounding), the V codes (q - 8 for Q4_0, q - 16
+//          for Q5_0, q for Q8_0) exact in fp16 are the B operand.
 // A stage buffer is refilled once all eight warps have released it (an
 // mbarrier with eight arrivals); there is no CTA-wide barrier in the loop.  At
 // the end the eight warps' (m, l, O) are merged into the split's partial.
@@ -206,12 +223,15 @@ static_assert(kWarps * kMaxRows * (kHeadDim + 2) * 4 <= kStages * kStageBytes, "
 
 // Stage and shared-memory geometry by V type: a Q8_0-V stage carries 128 B of
 // V codes per key (34,816 B per stage), so it keeps two stages in flight to
-// stay at two CTAs per SM.
+// stay at two CTAs per SM; a Q5_0-V stage adds 16 B of fifth bits per key
+// (28,672 B) and keeps three.
 template <int VT>
 struct DecGeom {
     static constexpr int kVqRow = PageGeom<VT>::kVqRow;
+    static constexpr int kVhRow = PageGeom<VT>::kVhRow;
     static constexpr int kStageVq = kStageKd + kStageKeys * kBlocks * 2;   // 17408
-    static constexpr int kStageVd = kStageVq + kStageKeys * kVqRow;
+    static constexpr int kStageVh = kStageVq + kStageKeys * kVqRow;
+    static constexpr int kStageVd = kStageVh + kStageKeys * kVhRow;
     static constexpr int kStageBytes = kStageVd + kStageKeys * kBlocks * 2;
     static constexpr int kStages = VT == kVQ8_0 ? 2 : 3;
     static constexpr size_t kOffQ = (size_t)kStages * kStageBytes;
@@ -224,6 +244,8 @@ struct DecGeom {
 static_assert(DecGeom<kVQ4_0>::kStageBytes == kStageBytes && DecGeom<kVQ4_0>::kSmem == kDecodeSmem,
               "Q4_0 decode geometry");
 static_assert(2 * DecGeom<kVQ8_0>::kSmem <= 232448, "two Q8_0-V CTAs per SM");
+static_assert(2 * DecGeom<kVQ5_0>::kSmem <= 232448 && DecGeom<kVQ5_0>::kStageBytes == 28672,
+              "two Q5_0-V CTAs per SM");
 
 size_t decode_smem_bytes() { return kDecodeSmem; }
 
@@ -272,6 +294,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     constexpr int kStages = G::kStages;
     constexpr int kStageBytes = G::kStageBytes;
     constexpr int kStageVq = G::kStageVq;
+    constexpr int kStageVh = G::kStageVh;
     constexpr int kStageVd = G::kStageVd;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -345,6 +368,11 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll 4
             for (int c = lane; c < kStageKeys * PG::kVqRow / 16; c += 32)
                 cp_async16(dst + kStageVq + c * 16, vq + c * 16);
+            if constexpr (PG::kVhRow > 0) {
+                const uint8_t* vh = ph + PG::kOffVh + half * (kStageKeys * PG::kVhRow);
+                for (int c = lane; c < kStageKeys * PG::kVhRow / 16; c += 32)
+                    cp_async16(dst + kStageVh + c * 16, vh + c * 16);
+            }
             cp_async_arrive(b);
         } else {
             mbar_expect_tx(b, kStageBytes);
@@ -352,6 +380,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             tma_load_2d(dst + kStageKq, &kmap, 0, krow, b);
             bulk_load(dst + kStageKd, ph + kOffKd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
             bulk_load(dst + kStageVq, ph + PG::kOffVq + half * (kStageKeys * PG::kVqRow), kStageKeys * PG::kVqRow, b);
+            if constexpr (PG::kVhRow > 0)
+                bulk_load(dst + kStageVh, ph + PG::kOffVh + half * (kStageKeys * PG::kVhRow), kStageKeys * PG::kVhRow, b);
             bulk_load(dst + kStageVd, ph + PG::kOffVd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
         }
     };
@@ -383,6 +413,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     float m_run = -CUDART_INF_F, l_run = 0.0f;
     bool ok = true;
     const __half2 b1152 = __float2half2_rn(1152.0f), b1032 = __float2half2_rn(1032.0f);
+    const __half2 b1040 = __float2half2_rn(1040.0f);
 
     for (int i = 0; i < n_st; ++i) {
         // producer: keep the next two stages in flight (it waits for all
@@ -489,6 +520,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             // V code words of this lane's keys (k0, k1 of n-tiles 0 and 1): the
             // four codes of dims 32 blk + 4g + {0..3}
             uint32_t wv[2][2];
+            // Q5_0: fifth bits of dims 32 blk + 4g + {0..3} of both keys of
+            // n-tile t, in bits 0..3 (first key) and 16..19 (second key)
+            uint32_t hv[2] = {0u, 0u};
 #pragma unroll
             for (int t = 0; t < 2; ++t)
 #pragma unroll
@@ -499,6 +533,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                                    0x80808080u;
                     else
                         wv[t][j] = *reinterpret_cast<const uint32_t*>(vst + key * 64 + 16 * blk + 4 * (g & 3));
+                    if constexpr (VT == kVQ5_0)
+                        hv[t] |= ((*reinterpret_cast<const uint32_t*>(sb + kStageVh + key * 16 + 4 * blk) >> (4 * g)) &
+                                  0xfu) << (16 * j);
                 }
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
@@ -509,6 +546,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                     const uint32_t pr = __byte_perm(wv[t][0], wv[t][1], sel);
                     if constexpr (VT == kVQ8_0)
                         bv[t] = h2u(__hsub2(u2h((pr & 0x00ff00ffu) | 0x64006400u), b1152));
+                    else if constexpr (VT == kVQ5_0)  // 1024 + (nibble | fifth bit << 4) - 1040
+                        bv[t] = h2u(__hsub2(u2h(((pr >> (4 * (g >> 2))) & 0x000f000fu) |
+                                                (((hv[t] >> m) & 0x00010001u) << 4) | 0x64006400u),
+                                            b1040));
                     else
                         bv[t] = h2u(__hsub2(u2h(((pr >> (4 * (g >> 2))) & 0x000f000fu) | 0x64006400u), b1032));
                 }
@@ -604,14 +645,16 @@ static cudaError_t launch_decode_rows(const DecodeArgs& a, const CUtensorMap* km
 
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                           cudaStream_t s) {
-    return a.v_type == kVQ8_0 ? launch_decode_rows<false, kVQ8_0>(a, kmap, n_splits, s)
-                              : launch_decode_rows<false, kVQ4_0>(a, kmap, n_splits, s);
+    if (a.v_type == kVQ8_0) return launch_decode_rows<false, kVQ8_0>(a, kmap, n_splits, s);
+    if (a.v_type == kVQ5_0) return launch_decode_rows<false, kVQ5_0>(a, kmap, n_splits, s);
+    return launch_decode_rows<false, kVQ4_0>(a, kmap, n_splits, s);
 }
 
 cudaError_t launch_decode_zero_copy(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                                     cudaStream_t s) {
-    return a.v_type == kVQ8_0 ? launch_decode_rows<true, kVQ8_0>(a, kmap, n_splits, s)
-                              : launch_decode_rows<true, kVQ4_0>(a, kmap, n_splits, s);
+    if (a.v_type == kVQ8_0) return launch_decode_rows<true, kVQ8_0>(a, kmap, n_splits, s);
+    if (a.v_type == kVQ5_0) return launch_decode_rows<true, kVQ5_0>(a, kmap, n_splits, s);
+    return launch_decode_rows<true, kVQ4_0>(a, kmap, n_splits, s);
 }
 
 // ----------------------------------------------------------------------------

@@ -40,7 +40,7 @@ class Workload:
     outlier_scale: float = 1.0
     head_dim: int = HEAD_DIM
     page_tokens: int = PAGE_TOKENS
-    type_v: int = 2       # V block type: 2 = Q4_0, 8 = Q8_0 (the q8_0/q8_0 pair)
+    type_v: int = 2       # V block type: 2 = Q4_0, 6 = Q5_0, 8 = Q8_0 (the q8_0/q8_0 pair)
 
     @property
     def n_pages(self) -> int:
@@ -82,6 +82,10 @@ WORKLOADS = {
     "streamed_decode_32k_q8v": Workload("streamed_decode_32k_q8v", n_layers=16, n_q=1, n_q_heads=32,
                                         n_kv_heads=8, ctx=32768, n_resident_pages=64, n_ring_slots=8,
                                         seed=5, outlier_frac=0.01, outlier_scale=8.0, type_v=8),
+    # the same with V as Q5_0 (1728 B per token per layer)
+    "streamed_decode_32k_q5v": Workload("streamed_decode_32k_q5v", n_layers=16, n_q=1, n_q_heads=32,
+                                        n_kv_heads=8, ctx=32768, n_resident_pages=64, n_ring_slots=8,
+                                        seed=6, outlier_frac=0.01, outlier_scale=8.0, type_v=6),
 }
 DEFAULT_BENCH = "streamed_decode_32k"
 # Share (%) of a decode step's streamed pages that the decode kernel reads in

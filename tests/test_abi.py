@@ -65,7 +65,8 @@ def test_plan_page_matches_oracle(kvs):
 
 
 @pytest.mark.parametrize("over,code", [
-    (dict(type_k=2), -1), (dict(type_v=1), -1), (dict(type_k=8, type_v=3), -1), (dict(head_dim=64), -1), (dict(page_tokens=128), -1),
+    (dict(type_k=2), -1), (dict(type_v=1), -1), (dict(type_k=8, type_v=3), -1), (dict(type_v=7), -1),
+    (dict(type_k=6, type_v=6), -1), (dict(head_dim=64), -1), (dict(page_tokens=128), -1),
     (dict(n_q_heads=12, n_kv_heads=8), -1), (dict(n_ring_slots=0, n_resident_pages=4), -1),
     (dict(n_ring_slots=6, chunk_pages=4), -1), (dict(arena_bytes=1000), -2),
     (dict(arena_bytes=425984), -2), (dict(max_q_tokens=0), -1), (dict(n_layers=0), -1),
@@ -91,6 +92,20 @@ def test_q8_0_v_pair_geometry(kvs):
     r4, _ = kvs.kvs_resolve_config(c4)
     assert kvs.kvs_page_bytes(r4) == 8 * 53248
     assert r.arena_bytes - r4.arena_bytes == (2 * 8 + 8) * 8 * (69632 - 53248)
+
+
+def test_q5_0_v_pair_geometry(kvs):
+    """The q8_0/q5_0 pair: Q4_0's V nibbles plus 16 B of fifth bits per token
+    and kv head, 57,344 B per page head."""
+    c = kvs.make_config(2, 32, 8, 32768, n_resident_pages=8, n_ring_slots=8,
+                        type_v=kvs.KVS_TYPE_Q5_0)
+    r, host = kvs.kvs_resolve_config(c)
+    assert r.type_v == kvs.KVS_TYPE_Q5_0
+    assert kvs.kvs_page_bytes(r) == 8 * 57344
+    assert host == 2 * 128 * 8 * 57344
+    c4 = kvs.make_config(2, 32, 8, 32768, n_resident_pages=8, n_ring_slots=8)
+    r4, _ = kvs.kvs_resolve_config(c4)
+    assert r.arena_bytes - r4.arena_bytes == (2 * 8 + 8) * 8 * (57344 - 53248)
 
 
 def test_arena_fit_accepts_exact_size(kvs):

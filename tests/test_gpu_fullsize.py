@@ -55,6 +55,10 @@ def test_streamed_decode_32k_q8v_full(kvs):
     _full(kvs, "streamed_decode_32k_q8v", layers=[3])
 
 
+def test_streamed_decode_32k_q5v_full(kvs):
+    _full(kvs, "streamed_decode_32k_q5v", layers=[9])
+
+
 def test_long_decode_256k_full(kvs):
     _full(kvs, "long_decode_256k", layers=[7])
 
