@@ -22,8 +22,8 @@ namespace kvs {
 //   Vq  u8    [256 tok][4 blocks][16 B]            16,384 B  @ 34,816
 //         (byte j of a block holds code j in the low nibble, code j+16 high)
 //   Vd  fp16  [256 tok][4 blocks]                   2,048 B  @ 51,200
-// The canonical 34-byte Q8_0 / 18-byte Q4_0 blocks are a reshuffle of these
-// bytes (kvs_export_page does it on the host).
+// The canonical 34-byte Q8_0 / 18-byte Q4_0 (22-byte Q5_0) blocks are a
+// reshuffle of these bytes (kvs_export_page does it on the host).
 // ---------------------------------------------------------------------------
 constexpr int kHeadDim = 128;
 constexpr int kPageTokens = 256;

@@ -57,6 +57,10 @@ def bind(L):
     L.oracle_dequant_q4_0.argtypes = [u8p, f64p]
     L.oracle_q5_0_block.argtypes = [u16p, u8p]
     L.oracle_dequant_q5_0.argtypes = [u8p, f64p]
+    L.oracle_q4_1_block.argtypes = [u16p, u8p]
+    L.oracle_dequant_q4_1.argtypes = [u8p, f64p]
+    L.oracle_q5_1_block.argtypes = [u16p, u8p]
+    L.oracle_dequant_q5_1.argtypes = [u8p, f64p]
     L.oracle_quantize_rows.argtypes = [ctypes.c_int, ctypes.c_int, u16p, u16p, u8p, u8p]
     L.oracle_attention.restype = ctypes.c_int
     L.oracle_attention.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, u8p, u8p,
@@ -159,14 +163,44 @@ def dequant_q5_0(blk) -> np.ndarray:
     return out
 
 
+def q4_1_block(x) -> bytes:
+    x = _as_half_bits(x).reshape(32)
+    out = np.zeros(20, np.uint8)
+    lib().oracle_q4_1_block(_ptr(x, ctypes.c_uint16), _ptr(out, ctypes.c_uint8))
+    return out.tobytes()
+
+
+def q5_1_block(x) -> bytes:
+    x = _as_half_bits(x).reshape(32)
+    out = np.zeros(24, np.uint8)
+    lib().oracle_q5_1_block(_ptr(x, ctypes.c_uint16), _ptr(out, ctypes.c_uint8))
+    return out.tobytes()
+
+
+def dequant_q4_1(blk) -> np.ndarray:
+    b = np.frombuffer(bytes(blk), np.uint8).copy()
+    out = np.zeros(32, np.float64)
+    lib().oracle_dequant_q4_1(_ptr(b, ctypes.c_uint8), _ptr(out, ctypes.c_double))
+    return out
+
+
+def dequant_q5_1(blk) -> np.ndarray:
+    b = np.frombuffer(bytes(blk), np.uint8).copy()
+    out = np.zeros(32, np.float64)
+    lib().oracle_dequant_q5_1(_ptr(b, ctypes.c_uint8), _ptr(out, ctypes.c_double))
+    return out
+
+
 V_Q4_0 = 2
+V_Q4_1 = 3
 V_Q5_0 = 6
+V_Q5_1 = 7
 V_Q8_0 = 8
-_V_BLOCK = {V_Q4_0: 18, V_Q5_0: 22, V_Q8_0: 34}
+_V_BLOCK = {V_Q4_0: 18, V_Q4_1: 20, V_Q5_0: 22, V_Q5_1: 24, V_Q8_0: 34}
 
 
 def quantize_rows(k, v, v_type: int = V_Q4_0):
-    """k, v: fp16 [..., dim] -> (Q8_0 blocks [..., dim/32, 34], V blocks [..., dim/32, 18, 22 or 34])."""
+    """k, v: fp16 [..., dim] -> (Q8_0 blocks [..., dim/32, 34], V blocks [..., dim/32, block bytes of v_type])."""
     k = _as_half_bits(k)
     v = _as_half_bits(v)
     assert k.shape == v.shape
@@ -190,7 +224,7 @@ def attention(k_blocks: np.ndarray, v_blocks: np.ndarray, q, pos0: int, v_type: 
     """Exact attention over a quantized history.
 
     k_blocks: uint8 [n_keys, n_kv, dim/32, 34]; v_blocks: uint8 [n_keys, n_kv, dim/32, 18]
-    (Q4_0), [..., 22] (Q5_0, v_type = V_Q5_0) or [..., 34] (Q8_0, v_type = V_Q8_0)
+    (Q4_0), or [..., 20 / 22 / 24 / 34] for v_type = V_Q4_1 / V_Q5_0 / V_Q5_1 / V_Q8_0
     q: fp16 [n_q, n_qh, dim]; query j sits at position pos0+j and sees keys 0..pos0+j.
     Returns (out float64 [n_q, n_qh, dim], lse float64 [n_q, n_qh]).
     """

@@ -11,6 +11,9 @@
  *  - the K cache is Q8_0 and the V cache is Q4_0, blocks of 32 values with an
  *    fp16 scale ("RaymondHuang210129/llama.cpp-adaptive-kv-streaming",
  *    Summary; "llama.cpp adaptive KV streaming - spec fork notes", Results);
+ *    V may also be Q8_0 (the q8_0/q8_0 runs of PR #326) or another of the
+ *    legal cache types of the flash-attention build (the first page's build
+ *    section), each with its own block rule below;
  *  - the KV history is quantized once, when a token is appended, and attention
  *    is exact over every token of the history; streaming only changes where
  *    the bytes live ("Feature/adaptive kv stream integration", PR #326,
@@ -108,6 +111,10 @@ uint16_t oracle_float_to_half(float f) {
 /*   Q5_0: 2-byte fp16 scale d, a 4-byte word whose bit j is bit 4 of q_j,    */
 /*         then 16 bytes holding the low 4 bits of q_j / q_{j+16} as Q4_0    */
 /*         does                                               (22 bytes)      */
+/*   Q4_1: fp16 d, fp16 m (the block minimum), then the 16 code bytes of      */
+/*         Q4_0                                               (20 bytes)      */
+/*   Q5_1: fp16 d, fp16 m, the fifth-bit word, then the 16 bytes of Q5_0      */
+/*                                                            (24 bytes)      */
 /* ------------------------------------------------------------------------ */
 
 void oracle_q8_0_block(const uint16_t x_h[32], uint8_t out[34]) {
@@ -191,6 +198,57 @@ void oracle_q5_0_block(const uint16_t x_h[32], uint8_t out[22]) {
     for (int j = 0; j < 16; ++j) out[6 + j] = (uint8_t)((q[j] & 15) | ((q[j + 16] & 15) << 4));
 }
 
+/* Q4_1 / Q5_1: the asymmetric members of the family, also among the legal
+ * cache types of the flash-attention build (same page and section as Q5_0).
+ * The pages give no rule; it is read as the block's range split into 15 (31)
+ * steps from its minimum: d = (max - min)/levels, q = min(levels,
+ * trunc((x - min)/d + 0.5)), q = 0 when d = 0, so x ~ d q + min. */
+static void min_block(const uint16_t x_h[32], int levels, uint16_t* dh, uint16_t* mh, int q[32]) {
+    float x[32];
+    float lo = 0.0f, hi = 0.0f;
+    for (int i = 0; i < 32; ++i) {
+        x[i] = oracle_half_to_float(x_h[i]);
+        if (i == 0 || x[i] < lo) lo = x[i];
+        if (i == 0 || x[i] > hi) hi = x[i];
+    }
+    float d = (hi - lo) / (float)levels; /* binary32 difference, then division */
+    *dh = oracle_float_to_half(d);
+    *mh = oracle_float_to_half(lo);
+    for (int i = 0; i < 32; ++i) {
+        if (d == 0.0f) {
+            q[i] = 0;
+        } else {
+            int t = (int)((x[i] - lo) / d + 0.5f); /* argument >= 0.5: truncation */
+            q[i] = t < levels ? t : levels;
+        }
+    }
+}
+
+void oracle_q4_1_block(const uint16_t x_h[32], uint8_t out[20]) {
+    uint16_t dh, mh;
+    int q[32];
+    min_block(x_h, 15, &dh, &mh, q);
+    out[0] = (uint8_t)(dh & 0xff);
+    out[1] = (uint8_t)(dh >> 8);
+    out[2] = (uint8_t)(mh & 0xff);
+    out[3] = (uint8_t)(mh >> 8);
+    for (int j = 0; j < 16; ++j) out[4 + j] = (uint8_t)(q[j] | (q[j + 16] << 4));
+}
+
+void oracle_q5_1_block(const uint16_t x_h[32], uint8_t out[24]) {
+    uint16_t dh, mh;
+    int q[32];
+    min_block(x_h, 31, &dh, &mh, q);
+    out[0] = (uint8_t)(dh & 0xff);
+    out[1] = (uint8_t)(dh >> 8);
+    out[2] = (uint8_t)(mh & 0xff);
+    out[3] = (uint8_t)(mh >> 8);
+    uint32_t top = 0;
+    for (int i = 0; i < 32; ++i) top |= (uint32_t)(q[i] >> 4) << i;
+    for (int b = 0; b < 4; ++b) out[4 + b] = (uint8_t)(top >> (8 * b));
+    for (int j = 0; j < 16; ++j) out[8 + j] = (uint8_t)((q[j] & 15) | ((q[j + 16] & 15) << 4));
+}
+
 void oracle_dequant_q8_0(const uint8_t blk[34], double out[32]) {
     double d = oracle_half_to_double((uint16_t)(blk[0] | (blk[1] << 8)));
     for (int i = 0; i < 32; ++i) out[i] = d * (double)(int8_t)blk[2 + i];
@@ -215,25 +273,58 @@ void oracle_dequant_q5_0(const uint8_t blk[22], double out[32]) {
     }
 }
 
-/* bytes of one 32-value block of a V type (2 = Q4_0, 6 = Q5_0, 8 = Q8_0),
- * 0 if unknown */
+void oracle_dequant_q4_1(const uint8_t blk[20], double out[32]) {
+    double d = oracle_half_to_double((uint16_t)(blk[0] | (blk[1] << 8)));
+    double m = oracle_half_to_double((uint16_t)(blk[2] | (blk[3] << 8)));
+    for (int j = 0; j < 16; ++j) {
+        out[j] = d * (double)(blk[4 + j] & 0x0f) + m;
+        out[j + 16] = d * (double)(blk[4 + j] >> 4) + m;
+    }
+}
+
+void oracle_dequant_q5_1(const uint8_t blk[24], double out[32]) {
+    double d = oracle_half_to_double((uint16_t)(blk[0] | (blk[1] << 8)));
+    double m = oracle_half_to_double((uint16_t)(blk[2] | (blk[3] << 8)));
+    uint32_t top = (uint32_t)blk[4] | ((uint32_t)blk[5] << 8) | ((uint32_t)blk[6] << 16) | ((uint32_t)blk[7] << 24);
+    for (int j = 0; j < 16; ++j) {
+        int a = (int)(blk[8 + j] & 0x0f) | (int)(((top >> j) & 1u) << 4);
+        int b = (int)(blk[8 + j] >> 4) | (int)(((top >> (j + 16)) & 1u) << 4);
+        out[j] = d * (double)a + m;
+        out[j + 16] = d * (double)b + m;
+    }
+}
+
+/* bytes of one 32-value block of a V type (2 = Q4_0, 3 = Q4_1, 6 = Q5_0,
+ * 7 = Q5_1, 8 = Q8_0), 0 if unknown */
 static int v_block_bytes(int v_type) {
-    return v_type == 2 ? 18 : (v_type == 6 ? 22 : (v_type == 8 ? 34 : 0));
+    switch (v_type) {
+        case 2: return 18;
+        case 3: return 20;
+        case 6: return 22;
+        case 7: return 24;
+        case 8: return 34;
+        default: return 0;
+    }
 }
 
 static void v_block(int v_type, const uint16_t* x, uint8_t* out) {
     if (v_type == 2) oracle_q4_0_block(x, out);
+    else if (v_type == 3) oracle_q4_1_block(x, out);
     else if (v_type == 6) oracle_q5_0_block(x, out);
+    else if (v_type == 7) oracle_q5_1_block(x, out);
     else oracle_q8_0_block(x, out);
 }
 
 static void v_dequant(int v_type, const uint8_t* blk, double* out) {
     if (v_type == 2) oracle_dequant_q4_0(blk, out);
+    else if (v_type == 3) oracle_dequant_q4_1(blk, out);
     else if (v_type == 6) oracle_dequant_q5_0(blk, out);
+    else if (v_type == 7) oracle_dequant_q5_1(blk, out);
     else oracle_dequant_q8_0(blk, out);
 }
 
-/* K rows -> Q8_0 blocks; V rows -> Q4_0 (v_type 2), Q5_0 (6) or Q8_0 (8) blocks */
+/* K rows -> Q8_0 blocks; V rows -> blocks of the V type (2 Q4_0, 3 Q4_1,
+ * 6 Q5_0, 7 Q5_1, 8 Q8_0) */
 int oracle_quantize_rows_t(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
                            uint8_t* k_blocks, uint8_t* v_blocks, int v_type) {
     int nb = dim / 32;
@@ -259,7 +350,7 @@ void oracle_quantize_rows(int n_rows, int dim, const uint16_t* k, const uint16_t
 /* Attention over the quantized history, binary64.                            */
 /*                                                                            */
 /* k_blocks: [n_keys][n_kv][dim/32] Q8_0 blocks (token-major history)         */
-/* v_blocks: [n_keys][n_kv][dim/32] Q4_0 (v_type 2), Q5_0 (6) or Q8_0 (8)    */
+/* v_blocks: [n_keys][n_kv][dim/32] blocks of the V type (v_block_bytes)     */
 /* q:        [n_q][n_qh][dim] fp16; query j sits at absolute position pos0+j  */
 /*           and sees keys 0..pos0+j (causal).                                */
 /* q head h reads kv head h / (n_qh/n_kv) (contiguous grouping).              */

@@ -20,6 +20,10 @@ void oracle_dequant_q8_0(const uint8_t blk[34], double out[32]);
 void oracle_dequant_q4_0(const uint8_t blk[18], double out[32]);
 void oracle_q5_0_block(const uint16_t x_h[32], uint8_t out[22]);
 void oracle_dequant_q5_0(const uint8_t blk[22], double out[32]);
+void oracle_q4_1_block(const uint16_t x_h[32], uint8_t out[20]);
+void oracle_dequant_q4_1(const uint8_t blk[20], double out[32]);
+void oracle_q5_1_block(const uint16_t x_h[32], uint8_t out[24]);
+void oracle_dequant_q5_1(const uint8_t blk[24], double out[32]);
 void oracle_quantize_rows(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
                           uint8_t* k_blocks, uint8_t* v_blocks);
 
@@ -28,7 +32,7 @@ int oracle_attention(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
                      double* out, double* lse);
 
 /* the same with the V block type explicit: 2 = Q4_0 (18-byte blocks),
- * 6 = Q5_0 (22-byte blocks), 8 = Q8_0 (34-byte blocks); -1 for any other */
+ * 3 = Q4_1 (20), 6 = Q5_0 (22), 7 = Q5_1 (24), 8 = Q8_0 (34); -1 for any other */
 int oracle_quantize_rows_t(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
                            uint8_t* k_blocks, uint8_t* v_blocks, int v_type);
 int oracle_attention_t(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,

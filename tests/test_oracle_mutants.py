@@ -16,6 +16,7 @@ import test_oracle_attention as TA
 import test_oracle_fp16 as TF
 import test_oracle_pages as TP
 import test_oracle_q5_0 as T5
+import test_oracle_q_min as TM
 import test_oracle_quant as TQ
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "kvs_oracle.c")
@@ -26,7 +27,10 @@ MUTANTS = {
     "q8 scale /128": ("float d = amax / 127.0f;", "float d = amax / 128.0f;"),
     "q4 last index wins": ("if (a > amax) { /* strict", "if (a >= amax) { /* strict"),
     "q4 offset 8.0": ("(int)(x[i] / d + 8.5f)", "(int)(x[i] / d + 8.0f)"),
-    "q4 nibble order": ("(uint8_t)(q[j] | (q[j + 16] << 4))", "(uint8_t)((q[j] << 4) | q[j + 16])"),
+    "q4 nibble order": ("out[2 + j] = (uint8_t)(q[j] | (q[j + 16] << 4))",
+                        "out[2 + j] = (uint8_t)((q[j] << 4) | q[j + 16])"),
+    "q4_1 nibble order": ("out[4 + j] = (uint8_t)(q[j] | (q[j + 16] << 4))",
+                          "out[4 + j] = (uint8_t)((q[j] << 4) | q[j + 16])"),
     "q4 dequant offset": ("(int)(blk[2 + j] & 0x0f) - 8)", "(int)(blk[2 + j] & 0x0f) - 7)"),
     "scale 1/d": ("double scale = 1.0 / sqrt((double)dim);", "double scale = 1.0 / (double)dim;"),
     "causal off by one": ("int n_keys = pos0 + j + 1;", "int n_keys = pos0 + j;"),
@@ -41,6 +45,12 @@ MUTANTS = {
     "q5 dequant offset": ("out[j] = d * (double)(lo - 16);", "out[j] = d * (double)(lo - 15);"),
     "v type dispatch": ("else if (v_type == 6) oracle_dequant_q5_0(blk, out);",
                         "else if (v_type == 6) oracle_dequant_q4_0(blk, out);"),
+    "q1 no rounding offset": ("int t = (int)((x[i] - lo) / d + 0.5f);", "int t = (int)((x[i] - lo) / d);"),
+    "q1 stores the max": ("*mh = oracle_float_to_half(lo);", "*mh = oracle_float_to_half(hi);"),
+    "q1 one step too many": ("float d = (hi - lo) / (float)levels;", "float d = (hi - lo) / (float)(levels + 1);"),
+    "q4_1 dequant drops m": ("out[j] = d * (double)(blk[4 + j] & 0x0f) + m;", "out[j] = d * (double)(blk[4 + j] & 0x0f);"),
+    "q5_1 fifth bit shifted": ("int a = (int)(blk[8 + j] & 0x0f) | (int)(((top >> j) & 1u) << 4);",
+                               "int a = (int)(blk[8 + j] & 0x0f) | (int)(((top >> (j + 1)) & 1u) << 4);"),
     "resident window": ("if (page >= P - n_resident) {", "if (page > P - n_resident) {"),
     "auto floor": ("long floor_pages = (2048 + page_tokens - 1) / page_tokens;",
                    "long floor_pages = (4096 + page_tokens - 1) / page_tokens;"),
@@ -60,6 +70,9 @@ def pins():
         TF.test_float_to_half_random,
         T5.test_q5_0_hand_worked, T5.test_q5_0_dequant_of_hand_block, T5.test_q5_0_error_bound_and_range,
         T5.test_q5_0_zero_query_is_uniform_mean, T5.test_q5_0_against_scipy_softmax_random,
+        lambda: TM.test_hand_worked("q4_1"), lambda: TM.test_hand_worked("q5_1"),
+        lambda: TM.test_error_bound_and_range("q4_1"), lambda: TM.test_error_bound_and_range("q5_1"),
+        lambda: TM.test_against_scipy_softmax_random("q5_1"),
     ]
 
 
