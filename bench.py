@@ -574,7 +574,7 @@ def run_gpu(args, w: W.Workload):
         "data": "synthetic",
         "config": {"workload": w.name, "ctx": w.ctx, "n_layers": L, "n_q": w.n_q,
                    "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": 128,
-                   "kv_types": "K q8_0 / V " + {8: "q8_0", 6: "q5_0"}.get(w.type_v, "q4_0"),
+                   "kv_types": "K q8_0 / V " + {8: "q8_0", 6: "q5_0", 3: "q4_1", 7: "q5_1"}.get(w.type_v, "q4_0"),
                    "page_tokens": 256, "resident_pages": R,
                    "streamed_pages": S, "ring_slots": rc.n_ring_slots, "chunk_pages": rc.chunk_pages,
                    "zero_copy_pct": zc_pct,
@@ -634,7 +634,8 @@ def main():
     if args.steps <= 0:
         # a timed region of a few seconds
         args.steps = {"tiny_decode_4k": 2000, "streamed_decode_32k": 300, "streamed_decode_32k_q8v": 240,
-                      "streamed_decode_32k_q5v": 280,
+                      "streamed_decode_32k_q5v": 280, "streamed_decode_32k_q41v": 280,
+                      "streamed_decode_32k_q51v": 260,
                       "long_decode_256k": 30,
                       "verify_128k": 60, "prefill_chunk_64k": 200}[w.name]
         if args.impl == "reference":

@@ -72,16 +72,17 @@ static_assert(kKVBytes % 1024 == 0, "swizzled tiles need 1024-B alignment");
 
 // Raw-stage and shared-memory layout by V type.  Raw stage (128 keys, as the
 // pages hold them): Kq [128][128] @ 0, Kd @ 16384, Vq @ 17408 (64 B per key
-// for Q4_0 and Q5_0 V, 128 B for Q8_0 V), the Q5_0 fifth bits (16 B per key),
-// Vd after them.  Shared memory: two raw
+// for Q4_0 and Q5_0 V, 128 B for Q8_0 V), the Q5_x fifth bits (16 B per key),
+// Vd, then the Q4_1 / Q5_1 minima (8 B per key).  Shared memory: two raw
 // stages, then [2] x (K^hi | K^lo), [3] x V^, the barriers, the TMEM slot and
 // the abort flag (Q4_0 V: K^ @ 53248, V^ @ 118784, barriers @ 167936).
 template <int VT>
 struct TcGeom {
     static constexpr int kRawVq = kRawKd + kRawKeys * kBlocks * 2;                    // 17408
-    static constexpr int kRawVh = kRawVq + kRawKeys * PageGeom<VT>::kVqRow;           // Q5_0 fifth bits
+    static constexpr int kRawVh = kRawVq + kRawKeys * PageGeom<VT>::kVqRow;           // Q5_x fifth bits
     static constexpr int kRawVd = kRawVh + kRawKeys * PageGeom<VT>::kVhRow;
-    static constexpr int kRawBytes = kRawVd + kRawKeys * kBlocks * 2;
+    static constexpr int kRawVm = kRawVd + kRawKeys * kBlocks * 2;                    // Q4_1 / Q5_1 minima
+    static constexpr int kRawBytes = kRawVm + kRawKeys * PageGeom<VT>::kVmRow;
     static constexpr size_t kOffK = (size_t)kRawStages * kRawBytes;
     static constexpr size_t kOffV = kOffK + kKBufs * 2 * kKVBytes;
     static constexpr size_t kOffBar = kOffV + kVBufs * kKVBytes;
@@ -94,6 +95,7 @@ struct TcGeom {
 };
 static_assert(TcGeom<kVQ4_0>::kOffBar == 167936, "Q4_0 geometry");
 static_assert(TcGeom<kVQ5_0>::kRawBytes == 28672, "Q5_0 raw stage");
+static_assert(TcGeom<kVQ4_1>::kRawBytes == 27648 && TcGeom<kVQ5_1>::kRawBytes == 29696, "Q4_1 / Q5_1 raw stages");
 
 // instruction descriptors: f16 x f16 -> f32, M = 128; A K-major;
 // S: N = 64, B K-major; PV: N = 128, B MN-major
@@ -181,6 +183,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     using TG = TcGeom<VT>;
     using PG = PageGeom<VT>;
     constexpr int kRawVq = TG::kRawVq, kRawVh = TG::kRawVh, kRawVd = TG::kRawVd, kRawBytes = TG::kRawBytes;
+    constexpr int kRawVm = TG::kRawVm;
     constexpr size_t kOffK = TG::kOffK, kOffV = TG::kOffV, kOffBar = TG::kOffBar;
     constexpr size_t kOffTmem = TG::kOffTmem, kOffAbort = TG::kOffAbort;
     extern __shared__ uint8_t smem_raw[];
@@ -288,6 +291,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if constexpr (PG::kVhRow > 0)
                     bulk_load(dst + kRawVh, ph + PG::kOffVh + half * (kRawKeys * PG::kVhRow), kRawKeys * PG::kVhRow, b);
                 bulk_load(dst + kRawVd, ph + PG::kOffVd + half * (kRawKeys * kBlocks * 2), kRawKeys * kBlocks * 2, b);
+                if constexpr (PG::kVmRow > 0)
+                    bulk_load(dst + kRawVm, ph + PG::kOffVm + half * (kRawKeys * PG::kVmRow), kRawKeys * PG::kVmRow, b);
             };
             int ir = 0;        // next raw stage to load
             for (; ir < kRawStages && ir < n_raw; ++ir) issue_raw(ir);
@@ -420,29 +425,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             } else
             for (int un = ptid; un < kSubKeys * kBlocks; un += kProdThreads) {
                 // Q4_0 V: V^ = fp16(d * (q - 8)); Q5_0 V: the same nibbles with
-                // the fifth bits added, V^ = fp16(d * (q - 16))
+                // the fifth bits added, V^ = fp16(d * (q - 16)); Q4_1 / Q5_1 V:
+                // V^ = fp16(d * q + m) (one rounding)
                 const int blk = un & 3, kloc = un >> 2;
                 const int key = sub * kSubKeys + kloc;
                 const uint4 q = *reinterpret_cast<const uint4*>(rb + kRawVq + key * 64 + blk * 16);
                 const __half dh = *reinterpret_cast<const __half*>(rb + kRawVd + key * 8 + blk * 2);
                 uint32_t hw = 0;
-                if constexpr (VT == kVQ5_0) hw = *reinterpret_cast<const uint32_t*>(rb + kRawVh + key * 16 + blk * 4);
+                if constexpr (v_has_fifth(VT)) hw = *reinterpret_cast<const uint32_t*>(rb + kRawVh + key * 16 + blk * 4);
                 const __half2 d2 = __halves2half2(dh, dh);
-                const __half2 bias = __float2half2_rn(VT == kVQ5_0 ? 1040.0f : 1032.0f);
+                __half2 m2 = __float2half2_rn(0.0f);
+                if constexpr (v_has_min(VT)) {
+                    const __half mh = *reinterpret_cast<const __half*>(rb + kRawVm + key * 8 + blk * 2);
+                    m2 = __halves2half2(mh, mh);
+                }
+                const __half2 bias = __float2half2_rn(v_has_min(VT) ? 1024.0f : (VT == kVQ5_0 ? 1040.0f : 1032.0f));
+                // code pair (exact in fp16) -> V^ pair
+                auto val = [&](uint32_t bits) {
+                    const __half2 x = __hsub2(u2h(bits | 0x64006400u), bias);
+                    if constexpr (v_has_min(VT)) return h2u(__hfma2(x, d2, m2));
+                    else return h2u(__hmul2(x, d2));
+                };
                 const uint32_t w[4] = {q.x, q.y, q.z, q.w};
                 uint32_t lo[8], hi[8];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const uint32_t p01 = __byte_perm(w[u], 0u, 0x4140u);  // bytes 4u, 4u+1 at positions 0, 2
                     const uint32_t p23 = __byte_perm(w[u], 0u, 0x4342u);
-                    lo[2 * u] = h2u(__hmul2(
-                        __hsub2(u2h((p01 & 0x000F000Fu) | fifth_bits(hw, 4 * u) | 0x64006400u), bias), d2));
-                    lo[2 * u + 1] = h2u(__hmul2(
-                        __hsub2(u2h((p23 & 0x000F000Fu) | fifth_bits(hw, 4 * u + 2) | 0x64006400u), bias), d2));
-                    hi[2 * u] = h2u(__hmul2(
-                        __hsub2(u2h(((p01 >> 4) & 0x000F000Fu) | fifth_bits(hw, 16 + 4 * u) | 0x64006400u), bias), d2));
-                    hi[2 * u + 1] = h2u(__hmul2(
-                        __hsub2(u2h(((p23 >> 4) & 0x000F000Fu) | fifth_bits(hw, 18 + 4 * u) | 0x64006400u), bias), d2));
+                    lo[2 * u] = val((p01 & 0x000F000Fu) | fifth_bits(hw, 4 * u));
+                    lo[2 * u + 1] = val((p23 & 0x000F000Fu) | fifth_bits(hw, 4 * u + 2));
+                    hi[2 * u] = val(((p01 >> 4) & 0x000F000Fu) | fifth_bits(hw, 16 + 4 * u));
+                    hi[2 * u + 1] = val(((p23 >> 4) & 0x000F000Fu) | fifth_bits(hw, 18 + 4 * u));
                 }
                 *reinterpret_cast<uint4*>(sVb + tile_off(kSubKeys, kloc, 32 * blk)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
                 *reinterpret_cast<uint4*>(sVb + tile_off(kSubKeys, kloc, 32 * blk + 8)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
@@ -585,6 +598,12 @@ cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ5_0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)TcGeom<kVQ5_0>::kSmem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ4_1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)TcGeom<kVQ4_1>::kSmem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ5_1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)TcGeom<kVQ5_1>::kSmem);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_acq_rel);
     }
@@ -594,6 +613,10 @@ cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n
         chunk_mma_kernel<kVQ8_0><<<grid, kTcThreads, TcGeom<kVQ8_0>::kSmem, s>>>(a, *kmap);
     else if (a.v_type == kVQ5_0)
         chunk_mma_kernel<kVQ5_0><<<grid, kTcThreads, TcGeom<kVQ5_0>::kSmem, s>>>(a, *kmap);
+    else if (a.v_type == kVQ4_1)
+        chunk_mma_kernel<kVQ4_1><<<grid, kTcThreads, TcGeom<kVQ4_1>::kSmem, s>>>(a, *kmap);
+    else if (a.v_type == kVQ5_1)
+        chunk_mma_kernel<kVQ5_1><<<grid, kTcThreads, TcGeom<kVQ5_1>::kSmem, s>>>(a, *kmap);
     else
         chunk_mma_kernel<kVQ4_0><<<grid, kTcThreads, TcGeom<kVQ4_0>::kSmem, s>>>(a, *kmap);
     return cudaGetLastError();

@@ -22,8 +22,8 @@ namespace kvs {
 //   Vq  u8    [256 tok][4 blocks][16 B]            16,384 B  @ 34,816
 //         (byte j of a block holds code j in the low nibble, code j+16 high)
 //   Vd  fp16  [256 tok][4 blocks]                   2,048 B  @ 51,200
-// The canonical 34-byte Q8_0 / 18-byte Q4_0 (22-byte Q5_0) blocks are a
-// reshuffle of these bytes (kvs_export_page does it on the host).
+// The canonical blocks (34-byte Q8_0, 18-byte Q4_0 and the V types below)
+// are a reshuffle of these bytes (kvs_export_page does it on the host).
 // ---------------------------------------------------------------------------
 constexpr int kHeadDim = 128;
 constexpr int kPageTokens = 256;
@@ -38,26 +38,39 @@ static_assert(kPageHeadBytes == 53248, "page-head layout");
 
 // V type codes (the public KVS_TYPE_* values)
 constexpr int kVQ4_0 = 2;
+constexpr int kVQ4_1 = 3;
 constexpr int kVQ5_0 = 6;
+constexpr int kVQ5_1 = 7;
 constexpr int kVQ8_0 = 8;
+
+// V type traits: fifth code bit (Q5_x), block minimum (Q4_1, Q5_1), levels
+__host__ __device__ constexpr bool v_has_fifth(int vt) { return vt == kVQ5_0 || vt == kVQ5_1; }
+__host__ __device__ constexpr bool v_has_min(int vt) { return vt == kVQ4_1 || vt == kVQ5_1; }
 
 // Page-head geometry by V type.  Q4_0 V is the layout above.  Q8_0 V stores
 // its codes like K (int8 [256 tok][128 dims], block b = dims 32b..32b+31):
 //   Kq @ 0, Kd @ 32,768, Vq int8 [256][128] @ 34,816, Vd @ 67,584; 69,632 B.
-// Q5_0 V keeps the low 4 bits of its codes as Q4_0 keeps its codes, and adds
-// the fifth bits, one 32-bit word per block (bit j = code j's bit 4):
-//   Vq u8 [256][4][16] @ 34,816, Vh u32 [256][4] @ 51,200, Vd @ 55,296; 57,344 B.
+// The other types keep the low 4 bits of their codes as Q4_0 keeps its codes;
+// Q5_x add the fifth bits, one 32-bit word per block (bit j = code j's bit 4),
+// and Q4_1 / Q5_1 the block minimum m (fp16) after the scales:
+//   Q5_0: Vq @ 34,816, Vh u32 [256][4] @ 51,200, Vd @ 55,296; 57,344 B.
+//   Q4_1: Vq @ 34,816, Vd @ 51,200, Vm fp16 [256][4] @ 53,248; 55,296 B.
+//   Q5_1: Vq @ 34,816, Vh @ 51,200, Vd @ 55,296, Vm @ 57,344; 59,392 B.
 template <int VT>
 struct PageGeom {
-    static_assert(VT == kVQ4_0 || VT == kVQ5_0 || VT == kVQ8_0, "V type");
+    static_assert(VT == kVQ4_0 || VT == kVQ4_1 || VT == kVQ5_0 || VT == kVQ5_1 || VT == kVQ8_0, "V type");
     static constexpr int kVqRow = VT == kVQ8_0 ? kHeadDim : kHeadDim / 2;  // V code bytes per token
-    static constexpr int kVhRow = VT == kVQ5_0 ? kBlocks * 4 : 0;         // V fifth-bit bytes per token
+    static constexpr int kVhRow = v_has_fifth(VT) ? kBlocks * 4 : 0;      // V fifth-bit bytes per token
+    static constexpr int kVmRow = v_has_min(VT) ? kBlocks * 2 : 0;        // V minimum bytes per token
     static constexpr int kOffVq = kOffKd + kPageTokens * kBlocks * 2;       // 34816
     static constexpr int kOffVh = kOffVq + kPageTokens * kVqRow;
     static constexpr int kOffVd = kOffVh + kPageTokens * kVhRow;
-    static constexpr int kHeadBytes = kOffVd + kPageTokens * kBlocks * 2;
+    static constexpr int kOffVm = kOffVd + kPageTokens * kBlocks * 2;
+    static constexpr int kHeadBytes = kOffVm + kPageTokens * kVmRow;
     static constexpr int kRows = kHeadBytes / 128;
-    static constexpr int kVBlockBytes = VT == kVQ8_0 ? 34 : (VT == kVQ5_0 ? 22 : 18);  // canonical block
+    static constexpr int kLevels = VT == kVQ4_1 ? 15 : 31;                // Q4_1 / Q5_1 steps
+    static constexpr int kVBlockBytes =                                    // canonical block
+        VT == kVQ8_0 ? 34 : (VT == kVQ5_0 ? 22 : (VT == kVQ4_1 ? 20 : (VT == kVQ5_1 ? 24 : 18)));
 };
 static_assert(PageGeom<kVQ4_0>::kHeadBytes == kPageHeadBytes && PageGeom<kVQ4_0>::kOffVd == kOffVd,
               "Q4_0 geometry");
@@ -66,11 +79,25 @@ static_assert(PageGeom<kVQ8_0>::kHeadBytes == 69632 && PageGeom<kVQ8_0>::kHeadBy
 static_assert(PageGeom<kVQ5_0>::kHeadBytes == 57344 && PageGeom<kVQ5_0>::kOffVh == 51200 &&
                   PageGeom<kVQ5_0>::kOffVd == 55296 && PageGeom<kVQ5_0>::kHeadBytes % 128 == 0,
               "Q5_0 geometry");
+static_assert(PageGeom<kVQ4_1>::kHeadBytes == 55296 && PageGeom<kVQ4_1>::kOffVd == 51200 &&
+                  PageGeom<kVQ4_1>::kOffVm == 53248 && PageGeom<kVQ4_1>::kHeadBytes % 128 == 0,
+              "Q4_1 geometry");
+static_assert(PageGeom<kVQ5_1>::kHeadBytes == 59392 && PageGeom<kVQ5_1>::kOffVh == 51200 &&
+                  PageGeom<kVQ5_1>::kOffVd == 55296 && PageGeom<kVQ5_1>::kOffVm == 57344 &&
+                  PageGeom<kVQ5_1>::kHeadBytes % 128 == 0,
+              "Q5_1 geometry");
 inline int page_head_bytes(int v_type) {
-    return v_type == kVQ8_0 ? PageGeom<kVQ8_0>::kHeadBytes
-                            : (v_type == kVQ5_0 ? PageGeom<kVQ5_0>::kHeadBytes : PageGeom<kVQ4_0>::kHeadBytes);
+    switch (v_type) {
+        case kVQ8_0: return PageGeom<kVQ8_0>::kHeadBytes;
+        case kVQ5_0: return PageGeom<kVQ5_0>::kHeadBytes;
+        case kVQ4_1: return PageGeom<kVQ4_1>::kHeadBytes;
+        case kVQ5_1: return PageGeom<kVQ5_1>::kHeadBytes;
+        default: return PageGeom<kVQ4_0>::kHeadBytes;
+    }
 }
-inline bool v_type_supported(int v_type) { return v_type == kVQ4_0 || v_type == kVQ5_0 || v_type == kVQ8_0; }
+inline bool v_type_supported(int v_type) {
+    return v_type == kVQ4_0 || v_type == kVQ4_1 || v_type == kVQ5_0 || v_type == kVQ5_1 || v_type == kVQ8_0;
+}
 
 // split partials: per split and query row, (m, l) in the log2 domain + acc[128]
 struct PartialBuffers {

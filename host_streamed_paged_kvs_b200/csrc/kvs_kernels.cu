@@ -39,8 +39,11 @@ __device__ __forceinline__ float q4_to_f(uint32_t c) {
 // Q5_0: the same with 32 levels: d = m/-16, q = min(31, trunc(x/d + 16.5)),
 //       d == 0 -> q = 16; the low 4 bits are packed as Q4_0's codes, the
 //       fifth bits in one 32-bit word per block (bit j = code j).
+// Q4_1 / Q5_1: lo, hi = block minimum and maximum (first index on ties),
+//       d = (hi - lo)/L with L = 15 / 31, q = min(L, trunc((x - lo)/d + 0.5)),
+//       d == 0 -> q = 0; the block minimum is stored as an fp16 m.
 // The stored scales are the fp16 (round-to-nearest-even) values of d.
-// K is always Q8_0; V is Q4_0 (VT = 2), Q5_0 (VT = 6) or Q8_0 (VT = 8).
+// K is always Q8_0; V is Q4_0 (VT = 2), Q4_1 (3), Q5_0 (6), Q5_1 (7) or Q8_0 (8).
 // ----------------------------------------------------------------------------
 // Q8_0 of the 32-value block spread over 8 lanes (4 values each): the lane's
 // 4 codes packed in one word (byte u = code of value u), and the block scale
@@ -114,6 +117,60 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
         return;
     }
 
+    if constexpr (v_has_min(VT)) {
+        // ---- Q4_1 / Q5_1 (V): block minimum and maximum, first index on ties ----
+        float lo = xv[0], hi = xv[0];
+        int ilo = 4 * i, ihi = 4 * i;
+#pragma unroll
+        for (int u = 1; u < 4; ++u) {
+            if (xv[u] < lo) { lo = xv[u]; ilo = 4 * i + u; }
+            if (xv[u] > hi) { hi = xv[u]; ihi = 4 * i + u; }
+        }
+#pragma unroll
+        for (int off = 1; off <= 4; off <<= 1) {
+            const float plo = __shfl_xor_sync(0xffffffffu, lo, off);
+            const int pilo = __shfl_xor_sync(0xffffffffu, ilo, off);
+            const float phi = __shfl_xor_sync(0xffffffffu, hi, off);
+            const int pihi = __shfl_xor_sync(0xffffffffu, ihi, off);
+            if (plo < lo || (plo == lo && pilo < ilo)) { lo = plo; ilo = pilo; }
+            if (phi > hi || (phi == hi && pihi < ihi)) { hi = phi; ihi = pihi; }
+        }
+        constexpr int kL = G::kLevels;
+        const float dv = __fdiv_rn(__fsub_rn(hi, lo), static_cast<float>(kL));
+        uint32_t codes = 0, high = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            int q = 0;
+            if (dv != 0.0f) q = min(kL, static_cast<int>(__fadd_rn(__fdiv_rn(__fsub_rn(xv[u], lo), dv), 0.5f)));
+            codes |= static_cast<uint32_t>(q & 15) << (8 * u);
+            high |= static_cast<uint32_t>(q >> 4) << (4 * i + u);
+        }
+        const uint32_t partner = __shfl_xor_sync(0xffffffffu, codes, 4);
+        const uint32_t vq = codes | (partner << 4);
+        if constexpr (v_has_fifth(VT)) {
+            high |= __shfl_xor_sync(0xffffffffu, high, 1);
+            high |= __shfl_xor_sync(0xffffffffu, high, 2);
+            high |= __shfl_xor_sync(0xffffffffu, high, 4);
+        }
+        const __half dv_h = __float2half_rn(dv), mv_h = __float2half_rn(lo);
+        auto store = [&](uint8_t* ph) {
+            *reinterpret_cast<uint32_t*>(ph + kOffKq + t * kHeadDim + 4 * lane) = kq;
+            if (i == 0) {
+                *reinterpret_cast<__half*>(ph + kOffKd + t * 8 + 2 * b) = dk_h;
+                *reinterpret_cast<__half*>(ph + G::kOffVd + t * 8 + 2 * b) = dv_h;
+                *reinterpret_cast<__half*>(ph + G::kOffVm + t * 8 + 2 * b) = mv_h;
+                if constexpr (v_has_fifth(VT)) *reinterpret_cast<uint32_t*>(ph + G::kOffVh + t * 16 + 4 * b) = high;
+            }
+            if (i < 4) *reinterpret_cast<uint32_t*>(ph + G::kOffVq + t * 64 + b * 16 + 4 * i) = vq;
+        };
+        store(a.host_layer + (size_t)page * a.page_bytes + (size_t)h * G::kHeadBytes);
+        if (page >= a.first_resident_page) {
+            const int slot = page % a.n_resident;
+            store(a.res_layer + (size_t)slot * a.page_bytes + (size_t)h * G::kHeadBytes);
+        }
+        return;
+    }
+
     // ---- Q4_0 / Q5_0 (V) ----
     constexpr bool kQ5 = VT == kVQ5_0;
     constexpr float kNegLevels = kQ5 ? -16.0f : -8.0f;
@@ -175,6 +232,10 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
         append_kernel<kVQ8_0><<<(rows + 3) / 4, 128, 0, s>>>(a);
     else if (a.v_type == kVQ5_0)
         append_kernel<kVQ5_0><<<(rows + 3) / 4, 128, 0, s>>>(a);
+    else if (a.v_type == kVQ4_1)
+        append_kernel<kVQ4_1><<<(rows + 3) / 4, 128, 0, s>>>(a);
+    else if (a.v_type == kVQ5_1)
+        append_kernel<kVQ5_1><<<(rows + 3) / 4, 128, 0, s>>>(a);
     else
         append_kernel<kVQ4_0><<<(rows + 3) / 4, 128, 0, s>>>(a);
     return cudaGetLastError();
@@ -197,7 +258,8 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
 //   softmax: warp-local lazy running max per row (log2 domain);
 //   PV   : the probability times the V scale of each (key, block) is the A
 //          operand (one fp16 rounding), the V codes (q - 8 for Q4_0, q - 16
-//          for Q5_0, q for Q8_0) exact in fp16 are the B operand.
+//          for Q5_0, q for Q8_0) exact in fp16 are the B operand; for Q4_1 /
+//          Q5_1 the A operand is p and B the value fp16(q d + m).
 // A stage buffer is refilled once all eight warps have released it (an
 // mbarrier with eight arrivals); there is no CTA-wide barrier in the loop.  At
 // the end the eight warps' (m, l, O) are merged into the split's partial.
@@ -229,10 +291,12 @@ template <int VT>
 struct DecGeom {
     static constexpr int kVqRow = PageGeom<VT>::kVqRow;
     static constexpr int kVhRow = PageGeom<VT>::kVhRow;
+    static constexpr int kVmRow = PageGeom<VT>::kVmRow;
     static constexpr int kStageVq = kStageKd + kStageKeys * kBlocks * 2;   // 17408
     static constexpr int kStageVh = kStageVq + kStageKeys * kVqRow;
     static constexpr int kStageVd = kStageVh + kStageKeys * kVhRow;
-    static constexpr int kStageBytes = kStageVd + kStageKeys * kBlocks * 2;
+    static constexpr int kStageVm = kStageVd + kStageKeys * kBlocks * 2;
+    static constexpr int kStageBytes = kStageVm + kStageKeys * kVmRow;
     static constexpr int kStages = VT == kVQ8_0 ? 2 : 3;
     static constexpr size_t kOffQ = (size_t)kStages * kStageBytes;
     static constexpr size_t kOffKend = kOffQ + kQFragBytes;
@@ -246,6 +310,10 @@ static_assert(DecGeom<kVQ4_0>::kStageBytes == kStageBytes && DecGeom<kVQ4_0>::kS
 static_assert(2 * DecGeom<kVQ8_0>::kSmem <= 232448, "two Q8_0-V CTAs per SM");
 static_assert(2 * DecGeom<kVQ5_0>::kSmem <= 232448 && DecGeom<kVQ5_0>::kStageBytes == 28672,
               "two Q5_0-V CTAs per SM");
+static_assert(2 * DecGeom<kVQ4_1>::kSmem <= 232448 && DecGeom<kVQ4_1>::kStageBytes == 27648,
+              "two Q4_1-V CTAs per SM");
+static_assert(2 * DecGeom<kVQ5_1>::kSmem <= 232448 && DecGeom<kVQ5_1>::kStageBytes == 29696,
+              "two Q5_1-V CTAs per SM");
 
 size_t decode_smem_bytes() { return kDecodeSmem; }
 
@@ -296,6 +364,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     constexpr int kStageVq = G::kStageVq;
     constexpr int kStageVh = G::kStageVh;
     constexpr int kStageVd = G::kStageVd;
+    constexpr int kStageVm = G::kStageVm;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -373,6 +442,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int c = lane; c < kStageKeys * PG::kVhRow / 16; c += 32)
                     cp_async16(dst + kStageVh + c * 16, vh + c * 16);
             }
+            if constexpr (PG::kVmRow > 0) {
+                const uint8_t* vm = ph + PG::kOffVm + half * (kStageKeys * PG::kVmRow);
+                for (int c = lane; c < kStageKeys * PG::kVmRow / 16; c += 32)
+                    cp_async16(dst + kStageVm + c * 16, vm + c * 16);
+            }
             cp_async_arrive(b);
         } else {
             mbar_expect_tx(b, kStageBytes);
@@ -383,6 +457,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             if constexpr (PG::kVhRow > 0)
                 bulk_load(dst + kStageVh, ph + PG::kOffVh + half * (kStageKeys * PG::kVhRow), kStageKeys * PG::kVhRow, b);
             bulk_load(dst + kStageVd, ph + PG::kOffVd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
+            if constexpr (PG::kVmRow > 0)
+                bulk_load(dst + kStageVm, ph + PG::kOffVm + half * (kStageKeys * PG::kVmRow), kStageKeys * PG::kVmRow, b);
         }
     };
     // the producer: thread 0 (TMA), or all of warp 0 (zero-copy)
@@ -413,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     float m_run = -CUDART_INF_F, l_run = 0.0f;
     bool ok = true;
     const __half2 b1152 = __float2half2_rn(1152.0f), b1032 = __float2half2_rn(1032.0f);
-    const __half2 b1040 = __float2half2_rn(1040.0f);
+    const __half2 b1040 = __float2half2_rn(1040.0f), b1024 = __float2half2_rn(1024.0f);
 
     for (int i = 0; i < n_st; ++i) {
         // producer: keep the next two stages in flight (it waits for all
@@ -511,12 +587,32 @@ __global__ void __launch_bounds__(kThreads, 2)
 
         // ---- PV ----
         const uint8_t* vst = sb + kStageVq;
+        // Q4_1 / Q5_1: A = p and B = the dequantized value fp16(q d + m), each
+        // rounded once relative to itself (a separate fp32 sum of p m would
+        // cancel against q d when the block minimum is large)
+        uint32_t pp0 = 0u, pp1 = 0u;
+        if constexpr (v_has_min(VT)) {
+            pp0 = h2u(__floats2half2_rn(p[0][0], p[0][1]));
+            pp1 = h2u(__floats2half2_rn(p[1][0], p[1][1]));
+        }
+        // the two keys' fp16 values of a per-(key, block) field, as a pair
+        auto pair = [&](int off, int t, int blk) {
+            const __half* h0 = reinterpret_cast<const __half*>(sb + off + (wkey + 8 * t + k0) * (kBlocks * 2));
+            const __half* h1 = reinterpret_cast<const __half*>(sb + off + (wkey + 8 * t + k1) * (kBlocks * 2));
+            return __halves2half2(h0[blk], h1[blk]);
+        };
 #pragma unroll
         for (int blk = 0; blk < kBlocks; ++blk) {
             // probabilities x the V scale of block blk, as the A operand
-            const float2 dv0 = scales(kStageVd, 0, blk), dv1 = scales(kStageVd, 1, blk);
-            const uint32_t pa0 = h2u(__floats2half2_rn(p[0][0] * dv0.x, p[0][1] * dv0.y));
-            const uint32_t pa1 = h2u(__floats2half2_rn(p[1][0] * dv1.x, p[1][1] * dv1.y));
+            uint32_t pa0, pa1;
+            if constexpr (v_has_min(VT)) {
+                pa0 = pp0;
+                pa1 = pp1;
+            } else {
+                const float2 dv0 = scales(kStageVd, 0, blk), dv1 = scales(kStageVd, 1, blk);
+                pa0 = h2u(__floats2half2_rn(p[0][0] * dv0.x, p[0][1] * dv0.y));
+                pa1 = h2u(__floats2half2_rn(p[1][0] * dv1.x, p[1][1] * dv1.y));
+            }
             // V code words of this lane's keys (k0, k1 of n-tiles 0 and 1): the
             // four codes of dims 32 blk + 4g + {0..3}
             uint32_t wv[2][2];
@@ -533,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                                    0x80808080u;
                     else
                         wv[t][j] = *reinterpret_cast<const uint32_t*>(vst + key * 64 + 16 * blk + 4 * (g & 3));
-                    if constexpr (VT == kVQ5_0)
+                    if constexpr (v_has_fifth(VT))
                         hv[t] |= ((*reinterpret_cast<const uint32_t*>(sb + kStageVh + key * 16 + 4 * blk) >> (4 * g)) &
                                   0xfu) << (16 * j);
                 }
@@ -550,6 +646,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                         bv[t] = h2u(__hsub2(u2h(((pr >> (4 * (g >> 2))) & 0x000f000fu) |
                                                 (((hv[t] >> m) & 0x00010001u) << 4) | 0x64006400u),
                                             b1040));
+                    else if constexpr (v_has_min(VT))  // fp16(q d + m), q = nibble (| fifth bit << 4)
+                        bv[t] = h2u(__hfma2(__hsub2(u2h(((pr >> (4 * (g >> 2))) & 0x000f000fu) |
+                                                        (((hv[t] >> m) & 0x00010001u) << 4) | 0x64006400u),
+                                                    b1024),
+                                            pair(kStageVd, t, blk), pair(kStageVm, t, blk)));
                     else
                         bv[t] = h2u(__hsub2(u2h(((pr >> (4 * (g >> 2))) & 0x000f000fu) | 0x64006400u), b1032));
                 }
@@ -647,6 +748,8 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, int n_sp
                           cudaStream_t s) {
     if (a.v_type == kVQ8_0) return launch_decode_rows<false, kVQ8_0>(a, kmap, n_splits, s);
     if (a.v_type == kVQ5_0) return launch_decode_rows<false, kVQ5_0>(a, kmap, n_splits, s);
+    if (a.v_type == kVQ4_1) return launch_decode_rows<false, kVQ4_1>(a, kmap, n_splits, s);
+    if (a.v_type == kVQ5_1) return launch_decode_rows<false, kVQ5_1>(a, kmap, n_splits, s);
     return launch_decode_rows<false, kVQ4_0>(a, kmap, n_splits, s);
 }
 
@@ -654,6 +757,8 @@ cudaError_t launch_decode_zero_copy(const DecodeArgs& a, const CUtensorMap* kmap
                                     cudaStream_t s) {
     if (a.v_type == kVQ8_0) return launch_decode_rows<true, kVQ8_0>(a, kmap, n_splits, s);
     if (a.v_type == kVQ5_0) return launch_decode_rows<true, kVQ5_0>(a, kmap, n_splits, s);
+    if (a.v_type == kVQ4_1) return launch_decode_rows<true, kVQ4_1>(a, kmap, n_splits, s);
+    if (a.v_type == kVQ5_1) return launch_decode_rows<true, kVQ5_1>(a, kmap, n_splits, s);
     return launch_decode_rows<true, kVQ4_0>(a, kmap, n_splits, s);
 }
 

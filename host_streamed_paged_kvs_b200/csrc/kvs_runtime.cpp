@@ -209,7 +209,7 @@ int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::stri
     if (c.page_tokens != kPageTokens) { why = fmt("page_tokens %d unsupported (only 256)", c.page_tokens); return KVS_E_INVAL; }
     if (c.type_k != KVS_TYPE_Q8_0 || !v_type_supported(c.type_v)) {
         why = "block KV streaming is not supported for this K/V cache type pair "
-              "(K=Q8_0 with V=Q4_0, Q5_0 or Q8_0)";
+              "(K=Q8_0 with V=Q4_0, Q4_1, Q5_0, Q5_1 or Q8_0)";
         return KVS_E_INVAL;
     }
     if (c.max_ctx < 1) { why = "max_ctx must be >= 1"; return KVS_E_INVAL; }
@@ -1072,12 +1072,23 @@ int kvs_export_page(kvs_t* kv, int layer, int page, int from_device, void* host_
     }
     uint8_t* out = static_cast<uint8_t*>(host_dst);
     const int H = c.n_kv_heads;
-    const bool v8 = c.type_v == KVS_TYPE_Q8_0, v5 = c.type_v == KVS_TYPE_Q5_0;
-    const int vblk = v8 ? PageGeom<kVQ8_0>::kVBlockBytes
-                        : (v5 ? PageGeom<kVQ5_0>::kVBlockBytes : PageGeom<kVQ4_0>::kVBlockBytes);
+    // canonical V block: fp16 d, [fp16 m], [fifth-bit word], codes
+    int vblk = 0, off_vh = 0, off_vd = 0, off_vm = 0;
+    bool has_h = false, has_m = false;
+    switch (c.type_v) {
+#define KVS_V_FIELDS(T)                                                               \
+    vblk = PageGeom<T>::kVBlockBytes; off_vh = PageGeom<T>::kOffVh;                   \
+    off_vd = PageGeom<T>::kOffVd; off_vm = PageGeom<T>::kOffVm;                      \
+    has_h = PageGeom<T>::kVhRow > 0; has_m = PageGeom<T>::kVmRow > 0;
+        case KVS_TYPE_Q8_0: KVS_V_FIELDS(kVQ8_0) break;
+        case KVS_TYPE_Q5_0: KVS_V_FIELDS(kVQ5_0) break;
+        case KVS_TYPE_Q4_1: KVS_V_FIELDS(kVQ4_1) break;
+        case KVS_TYPE_Q5_1: KVS_V_FIELDS(kVQ5_1) break;
+        default: KVS_V_FIELDS(kVQ4_0) break;
+#undef KVS_V_FIELDS
+    }
+    const bool v8 = c.type_v == KVS_TYPE_Q8_0;
     const int off_vq = PageGeom<kVQ4_0>::kOffVq;  // the same for every V type
-    const int off_vh = PageGeom<kVQ5_0>::kOffVh;  // Q5_0 only
-    const int off_vd = v8 ? PageGeom<kVQ8_0>::kOffVd : (v5 ? PageGeom<kVQ5_0>::kOffVd : PageGeom<kVQ4_0>::kOffVd);
     const int phb = page_head_bytes(c.type_v);
     uint8_t* kout = out;
     uint8_t* vout = out + (size_t)kPageTokens * H * kBlocks * 34;
@@ -1090,14 +1101,11 @@ int kvs_export_page(kvs_t* kv, int layer, int page, int from_device, void* host_
                 std::memcpy(kb + 2, ph + kOffKq + t * kHeadDim + b * 32, 32);
                 uint8_t* vb = vout + (((size_t)t * H + h) * kBlocks + b) * vblk;
                 std::memcpy(vb, ph + off_vd + t * 8 + b * 2, 2);
-                if (v8) {
-                    std::memcpy(vb + 2, ph + off_vq + t * kHeadDim + b * 32, 32);
-                } else if (v5) {  // fifth-bit word, then the low nibbles
-                    std::memcpy(vb + 2, ph + off_vh + t * 16 + b * 4, 4);
-                    std::memcpy(vb + 6, ph + off_vq + t * 64 + b * 16, 16);
-                } else {
-                    std::memcpy(vb + 2, ph + off_vq + t * 64 + b * 16, 16);
-                }
+                int at = 2;
+                if (has_m) { std::memcpy(vb + at, ph + off_vm + t * 8 + b * 2, 2); at += 2; }
+                if (has_h) { std::memcpy(vb + at, ph + off_vh + t * 16 + b * 4, 4); at += 4; }
+                if (v8) std::memcpy(vb + at, ph + off_vq + t * kHeadDim + b * 32, 32);
+                else std::memcpy(vb + at, ph + off_vq + t * 64 + b * 16, 16);
             }
         }
     return KVS_OK;

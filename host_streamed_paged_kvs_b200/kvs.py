@@ -23,7 +23,9 @@ KVS_E_CUDA = -5
 KVS_E_TIMEOUT = -6
 KVS_E_NOMEM = -7
 KVS_TYPE_Q4_0 = 2
+KVS_TYPE_Q4_1 = 3
 KVS_TYPE_Q5_0 = 6
+KVS_TYPE_Q5_1 = 7
 KVS_TYPE_Q8_0 = 8
 KVS_PAGE_ABSENT = -1
 KVS_PAGE_RESIDENT = 1

@@ -40,7 +40,7 @@ class Workload:
     outlier_scale: float = 1.0
     head_dim: int = HEAD_DIM
     page_tokens: int = PAGE_TOKENS
-    type_v: int = 2       # V block type: 2 = Q4_0, 6 = Q5_0, 8 = Q8_0 (the q8_0/q8_0 pair)
+    type_v: int = 2       # V block type: 2 Q4_0, 3 Q4_1, 6 Q5_0, 7 Q5_1, 8 Q8_0 (the q8_0/q8_0 pair)
 
     @property
     def n_pages(self) -> int:
@@ -86,6 +86,13 @@ WORKLOADS = {
     "streamed_decode_32k_q5v": Workload("streamed_decode_32k_q5v", n_layers=16, n_q=1, n_q_heads=32,
                                         n_kv_heads=8, ctx=32768, n_resident_pages=64, n_ring_slots=8,
                                         seed=6, outlier_frac=0.01, outlier_scale=8.0, type_v=6),
+    # V as Q4_1 / Q5_1 (1728 / 1856 B per token per layer)
+    "streamed_decode_32k_q41v": Workload("streamed_decode_32k_q41v", n_layers=16, n_q=1, n_q_heads=32,
+                                         n_kv_heads=8, ctx=32768, n_resident_pages=64, n_ring_slots=8,
+                                         seed=7, outlier_frac=0.01, outlier_scale=8.0, type_v=3),
+    "streamed_decode_32k_q51v": Workload("streamed_decode_32k_q51v", n_layers=16, n_q=1, n_q_heads=32,
+                                         n_kv_heads=8, ctx=32768, n_resident_pages=64, n_ring_slots=8,
+                                         seed=8, outlier_frac=0.01, outlier_scale=8.0, type_v=7),
 }
 DEFAULT_BENCH = "streamed_decode_32k"
 # Share (%) of a decode step's streamed pages that the decode kernel reads in

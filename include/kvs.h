@@ -49,9 +49,11 @@ extern "C" {
 #define KVS_E_TIMEOUT (-6) /* a bounded host wait gave up                         */
 #define KVS_E_NOMEM   (-7) /* host (pinned) allocation failed                     */
 
-/* ---- cache types: K is Q8_0; V is Q4_0, Q5_0 or Q8_0 ---------------------- */
+/* ---- cache types: K is Q8_0; V is Q4_0, Q4_1, Q5_0, Q5_1 or Q8_0 ----------- */
 #define KVS_TYPE_Q4_0 2
+#define KVS_TYPE_Q4_1 3
 #define KVS_TYPE_Q5_0 6
+#define KVS_TYPE_Q5_1 7
 #define KVS_TYPE_Q8_0 8
 
 /* ---- page kinds reported by kvs_page_location --------------------------- */
@@ -82,10 +84,13 @@ typedef struct kvs_config {
     int type_k;           /* must be KVS_TYPE_Q8_0 */
     int type_v;           /* KVS_TYPE_Q4_0 (page head 53,248 B), KVS_TYPE_Q8_0 (69,632 B: V codes
                              stored like K's; the q8_0/q8_0 pair of the "Feature/adaptive kv
-                             stream integration" pull request's runs) or KVS_TYPE_Q5_0
-                             (57,344 B: Q4_0's nibbles plus a word of fifth bits per block;
-                             one of the legal cache types of the flash-attention build on
-                             "RaymondHuang210129/llama.cpp-adaptive-kv-streaming") */
+                             stream integration" pull request's runs), or one of the other
+                             legal cache types of the flash-attention build on
+                             "RaymondHuang210129/llama.cpp-adaptive-kv-streaming":
+                             KVS_TYPE_Q5_0 (57,344 B: Q4_0's nibbles plus a word of fifth
+                             bits per block), KVS_TYPE_Q4_1 (55,296 B: Q4_0's layout plus an
+                             fp16 block minimum m, x = d q + m), KVS_TYPE_Q5_1 (59,392 B:
+                             Q5_0's layout plus m) */
     int chunk_pages;      /* pages per H2D copy; 0 = auto (n_ring_slots/2); must divide n_ring_slots */
     int flags;            /* KVS_FLAG_* */
     int zero_copy_pct;    /* 0..100: share of each layer's streamed pages (the newest ones) that
@@ -223,7 +228,8 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
  * bytes (fp16 d, byte j = q_j | q_(j+16) << 4), Q8_0 blocks of 34 bytes when
  * type_v is KVS_TYPE_Q8_0, or Q5_0 blocks of 22 bytes when it is KVS_TYPE_Q5_0
  * (fp16 d, a little-endian word whose bit j is bit 4 of q_j, then 16 bytes
- * holding the low 4 bits as Q4_0 does).  from_device = 0 reads the host history,
+ * holding the low 4 bits as Q4_0 does); Q4_1 (20 bytes) and Q5_1 (24 bytes)
+ * blocks put the fp16 block minimum m right after d.  from_device = 0 reads the host history,
  * 1 reads the resident slot (KVS_E_INVAL if the page is not resident).  The
  * caller must have synchronized the streams that wrote the page. */
 int kvs_export_page(kvs_t* kv, int layer, int page, int from_device, void* host_dst);
