@@ -191,12 +191,13 @@ def dequant_q5_1(blk) -> np.ndarray:
     return out
 
 
+V_F16 = 1
 V_Q4_0 = 2
 V_Q4_1 = 3
 V_Q5_0 = 6
 V_Q5_1 = 7
 V_Q8_0 = 8
-_V_BLOCK = {V_Q4_0: 18, V_Q4_1: 20, V_Q5_0: 22, V_Q5_1: 24, V_Q8_0: 34}
+_V_BLOCK = {V_F16: 64, V_Q4_0: 18, V_Q4_1: 20, V_Q5_0: 22, V_Q5_1: 24, V_Q8_0: 34}
 
 
 def quantize_rows(k, v, v_type: int = V_Q4_0):
@@ -224,7 +225,7 @@ def attention(k_blocks: np.ndarray, v_blocks: np.ndarray, q, pos0: int, v_type: 
     """Exact attention over a quantized history.
 
     k_blocks: uint8 [n_keys, n_kv, dim/32, 34]; v_blocks: uint8 [n_keys, n_kv, dim/32, 18]
-    (Q4_0), or [..., 20 / 22 / 24 / 34] for v_type = V_Q4_1 / V_Q5_0 / V_Q5_1 / V_Q8_0
+    (Q4_0), or [..., 20 / 22 / 24 / 34 / 64] for v_type = V_Q4_1 / V_Q5_0 / V_Q5_1 / V_Q8_0 / V_F16
     q: fp16 [n_q, n_qh, dim]; query j sits at position pos0+j and sees keys 0..pos0+j.
     Returns (out float64 [n_q, n_qh, dim], lse float64 [n_q, n_qh]).
     """

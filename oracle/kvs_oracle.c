@@ -294,10 +294,24 @@ void oracle_dequant_q5_1(const uint8_t blk[24], double out[32]) {
     }
 }
 
-/* bytes of one 32-value block of a V type (2 = Q4_0, 3 = Q4_1, 6 = Q5_0,
- * 7 = Q5_1, 8 = Q8_0), 0 if unknown */
+/* F16 V: the values themselves, 32 fp16 per block (64 bytes, little endian);
+ * f16 is a legal cache type of the same build list.  Nothing is rounded. */
+static void f16_block(const uint16_t x_h[32], uint8_t out[64]) {
+    for (int i = 0; i < 32; ++i) {
+        out[2 * i] = (uint8_t)(x_h[i] & 0xff);
+        out[2 * i + 1] = (uint8_t)(x_h[i] >> 8);
+    }
+}
+
+static void f16_dequant(const uint8_t blk[64], double out[32]) {
+    for (int i = 0; i < 32; ++i) out[i] = oracle_half_to_double((uint16_t)(blk[2 * i] | (blk[2 * i + 1] << 8)));
+}
+
+/* bytes of one 32-value block of a V type (1 = F16, 2 = Q4_0, 3 = Q4_1,
+ * 6 = Q5_0, 7 = Q5_1, 8 = Q8_0), 0 if unknown */
 static int v_block_bytes(int v_type) {
     switch (v_type) {
+        case 1: return 64;
         case 2: return 18;
         case 3: return 20;
         case 6: return 22;
@@ -308,7 +322,8 @@ static int v_block_bytes(int v_type) {
 }
 
 static void v_block(int v_type, const uint16_t* x, uint8_t* out) {
-    if (v_type == 2) oracle_q4_0_block(x, out);
+    if (v_type == 1) f16_block(x, out);
+    else if (v_type == 2) oracle_q4_0_block(x, out);
     else if (v_type == 3) oracle_q4_1_block(x, out);
     else if (v_type == 6) oracle_q5_0_block(x, out);
     else if (v_type == 7) oracle_q5_1_block(x, out);
@@ -316,15 +331,16 @@ static void v_block(int v_type, const uint16_t* x, uint8_t* out) {
 }
 
 static void v_dequant(int v_type, const uint8_t* blk, double* out) {
-    if (v_type == 2) oracle_dequant_q4_0(blk, out);
+    if (v_type == 1) f16_dequant(blk, out);
+    else if (v_type == 2) oracle_dequant_q4_0(blk, out);
     else if (v_type == 3) oracle_dequant_q4_1(blk, out);
     else if (v_type == 6) oracle_dequant_q5_0(blk, out);
     else if (v_type == 7) oracle_dequant_q5_1(blk, out);
     else oracle_dequant_q8_0(blk, out);
 }
 
-/* K rows -> Q8_0 blocks; V rows -> blocks of the V type (2 Q4_0, 3 Q4_1,
- * 6 Q5_0, 7 Q5_1, 8 Q8_0) */
+/* K rows -> Q8_0 blocks; V rows -> blocks of the V type (1 F16, 2 Q4_0,
+ * 3 Q4_1, 6 Q5_0, 7 Q5_1, 8 Q8_0) */
 int oracle_quantize_rows_t(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
                            uint8_t* k_blocks, uint8_t* v_blocks, int v_type) {
     int nb = dim / 32;

@@ -31,8 +31,9 @@ int oracle_attention(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
                      const uint8_t* v_blocks, int n_q, int pos0, const uint16_t* q,
                      double* out, double* lse);
 
-/* the same with the V block type explicit: 2 = Q4_0 (18-byte blocks),
- * 3 = Q4_1 (20), 6 = Q5_0 (22), 7 = Q5_1 (24), 8 = Q8_0 (34); -1 for any other */
+/* the same with the V block type explicit: 1 = F16 (64-byte blocks of the
+ * values), 2 = Q4_0 (18), 3 = Q4_1 (20), 6 = Q5_0 (22), 7 = Q5_1 (24),
+ * 8 = Q8_0 (34); -1 for any other */
 int oracle_quantize_rows_t(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
                            uint8_t* k_blocks, uint8_t* v_blocks, int v_type);
 int oracle_attention_t(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,

@@ -17,6 +17,7 @@ import test_oracle_fp16 as TF
 import test_oracle_pages as TP
 import test_oracle_q5_0 as T5
 import test_oracle_q_min as TM
+import test_oracle_v_f16 as TV16
 import test_oracle_quant as TQ
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "kvs_oracle.c")
@@ -51,6 +52,7 @@ MUTANTS = {
     "q4_1 dequant drops m": ("out[j] = d * (double)(blk[4 + j] & 0x0f) + m;", "out[j] = d * (double)(blk[4 + j] & 0x0f);"),
     "q5_1 fifth bit shifted": ("int a = (int)(blk[8 + j] & 0x0f) | (int)(((top >> j) & 1u) << 4);",
                                "int a = (int)(blk[8 + j] & 0x0f) | (int)(((top >> (j + 1)) & 1u) << 4);"),
+    "f16 V byte order": ("out[2 * i] = (uint8_t)(x_h[i] & 0xff);", "out[2 * i] = (uint8_t)(x_h[i] >> 8);"),
     "resident window": ("if (page >= P - n_resident) {", "if (page > P - n_resident) {"),
     "auto floor": ("long floor_pages = (2048 + page_tokens - 1) / page_tokens;",
                    "long floor_pages = (4096 + page_tokens - 1) / page_tokens;"),
@@ -73,6 +75,7 @@ def pins():
         lambda: TM.test_hand_worked("q4_1"), lambda: TM.test_hand_worked("q5_1"),
         lambda: TM.test_error_bound_and_range("q4_1"), lambda: TM.test_error_bound_and_range("q5_1"),
         lambda: TM.test_against_scipy_softmax_random("q5_1"),
+        TV16.test_v_blocks_are_the_input_bits, TV16.test_against_scipy_over_exact_values,
     ]
 
 
