@@ -72,8 +72,9 @@ static_assert(kKVBytes % 1024 == 0, "swizzled tiles need 1024-B alignment");
 
 // Raw-stage and shared-memory layout by V type.  Raw stage (128 keys, as the
 // pages hold them): Kq [128][128] @ 0, Kd @ 16384, Vq @ 17408 (64 B per key
-// for Q4_0 and Q5_0 V, 128 B for Q8_0 V), the Q5_x fifth bits (16 B per key),
-// Vd, then the Q4_1 / Q5_1 minima (8 B per key).  Shared memory: two raw
+// for Q4_0 and Q5_0 V, 128 B for Q8_0 V, 256 B of values for F16 V), the Q5_x
+// fifth bits (16 B per key), Vd (none for F16), then the Q4_1 / Q5_1 minima
+// (8 B per key).  Shared memory: two raw
 // stages, then [2] x (K^hi | K^lo), [3] x V^, the barriers, the TMEM slot and
 // the abort flag (Q4_0 V: K^ @ 53248, V^ @ 118784, barriers @ 167936).
 template <int VT>
@@ -81,7 +82,7 @@ struct TcGeom {
     static constexpr int kRawVq = kRawKd + kRawKeys * kBlocks * 2;                    // 17408
     static constexpr int kRawVh = kRawVq + kRawKeys * PageGeom<VT>::kVqRow;           // Q5_x fifth bits
     static constexpr int kRawVd = kRawVh + kRawKeys * PageGeom<VT>::kVhRow;
-    static constexpr int kRawVm = kRawVd + kRawKeys * kBlocks * 2;                    // Q4_1 / Q5_1 minima
+    static constexpr int kRawVm = kRawVd + kRawKeys * PageGeom<VT>::kVdRow;           // Q4_1 / Q5_1 minima
     static constexpr int kRawBytes = kRawVm + kRawKeys * PageGeom<VT>::kVmRow;
     static constexpr size_t kOffK = (size_t)kRawStages * kRawBytes;
     static constexpr size_t kOffV = kOffK + kKBufs * 2 * kKVBytes;
@@ -96,6 +97,7 @@ struct TcGeom {
 static_assert(TcGeom<kVQ4_0>::kOffBar == 167936, "Q4_0 geometry");
 static_assert(TcGeom<kVQ5_0>::kRawBytes == 28672, "Q5_0 raw stage");
 static_assert(TcGeom<kVQ4_1>::kRawBytes == 27648 && TcGeom<kVQ5_1>::kRawBytes == 29696, "Q4_1 / Q5_1 raw stages");
+static_assert(TcGeom<kVF16>::kRawBytes == 50176, "F16 raw stage");
 
 // instruction descriptors: f16 x f16 -> f32, M = 128; A K-major;
 // S: N = 64, B K-major; PV: N = 128, B MN-major
@@ -290,7 +292,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 bulk_load(dst + kRawVq, ph + PG::kOffVq + half * (kRawKeys * PG::kVqRow), kRawKeys * PG::kVqRow, b);
                 if constexpr (PG::kVhRow > 0)
                     bulk_load(dst + kRawVh, ph + PG::kOffVh + half * (kRawKeys * PG::kVhRow), kRawKeys * PG::kVhRow, b);
-                bulk_load(dst + kRawVd, ph + PG::kOffVd + half * (kRawKeys * kBlocks * 2), kRawKeys * kBlocks * 2, b);
+                if constexpr (PG::kVdRow > 0)
+                    bulk_load(dst + kRawVd, ph + PG::kOffVd + half * (kRawKeys * kBlocks * 2), kRawKeys * kBlocks * 2, b);
                 if constexpr (PG::kVmRow > 0)
                     bulk_load(dst + kRawVm, ph + PG::kOffVm + half * (kRawKeys * PG::kVmRow), kRawKeys * PG::kVmRow, b);
             };
@@ -421,6 +424,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         *reinterpret_cast<uint4*>(sVb + tile_off(kSubKeys, kloc, 32 * blk + 16 * hq + 8)) =
                             make_uint4(o[4], o[5], o[6], o[7]);
                     }
+                }
+            } else if constexpr (VT == kVF16) {
+                // F16 V: V^ is the stored values, copied 16 B (8 dims) at a time
+                for (int un = ptid; un < kSubKeys * 16; un += kProdThreads) {
+                    const int kloc = un >> 4, c = un & 15;
+                    const int key = sub * kSubKeys + kloc;
+                    *reinterpret_cast<uint4*>(sVb + tile_off(kSubKeys, kloc, 8 * c)) =
+                        *reinterpret_cast<const uint4*>(rb + kRawVq + key * (kHeadDim * 2) + 16 * c);
                 }
             } else
             for (int un = ptid; un < kSubKeys * kBlocks; un += kProdThreads) {
@@ -604,6 +615,9 @@ cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ5_1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)TcGeom<kVQ5_1>::kSmem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(chunk_mma_kernel<kVF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)TcGeom<kVF16>::kSmem);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_acq_rel);
     }
@@ -617,6 +631,8 @@ cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n
         chunk_mma_kernel<kVQ4_1><<<grid, kTcThreads, TcGeom<kVQ4_1>::kSmem, s>>>(a, *kmap);
     else if (a.v_type == kVQ5_1)
         chunk_mma_kernel<kVQ5_1><<<grid, kTcThreads, TcGeom<kVQ5_1>::kSmem, s>>>(a, *kmap);
+    else if (a.v_type == kVF16)
+        chunk_mma_kernel<kVF16><<<grid, kTcThreads, TcGeom<kVF16>::kSmem, s>>>(a, *kmap);
     else
         chunk_mma_kernel<kVQ4_0><<<grid, kTcThreads, TcGeom<kVQ4_0>::kSmem, s>>>(a, *kmap);
     return cudaGetLastError();

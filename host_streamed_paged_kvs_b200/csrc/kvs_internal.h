@@ -37,6 +37,7 @@ constexpr int kPageHeadRows = kPageHeadBytes / 128;     // 416 rows of 128 B
 static_assert(kPageHeadBytes == 53248, "page-head layout");
 
 // V type codes (the public KVS_TYPE_* values)
+constexpr int kVF16 = 1;
 constexpr int kVQ4_0 = 2;
 constexpr int kVQ4_1 = 3;
 constexpr int kVQ5_0 = 6;
@@ -46,6 +47,8 @@ constexpr int kVQ8_0 = 8;
 // V type traits: fifth code bit (Q5_x), block minimum (Q4_1, Q5_1), levels
 __host__ __device__ constexpr bool v_has_fifth(int vt) { return vt == kVQ5_0 || vt == kVQ5_1; }
 __host__ __device__ constexpr bool v_has_min(int vt) { return vt == kVQ4_1 || vt == kVQ5_1; }
+// decode feeds the tensor cores p and the V value itself (no per-block scale in A)
+__host__ __device__ constexpr bool v_a_is_p(int vt) { return v_has_min(vt) || vt == kVF16; }
 
 // Page-head geometry by V type.  Q4_0 V is the layout above.  Q8_0 V stores
 // its codes like K (int8 [256 tok][128 dims], block b = dims 32b..32b+31):
@@ -56,21 +59,27 @@ __host__ __device__ constexpr bool v_has_min(int vt) { return vt == kVQ4_1 || vt
 //   Q5_0: Vq @ 34,816, Vh u32 [256][4] @ 51,200, Vd @ 55,296; 57,344 B.
 //   Q4_1: Vq @ 34,816, Vd @ 51,200, Vm fp16 [256][4] @ 53,248; 55,296 B.
 //   Q5_1: Vq @ 34,816, Vh @ 51,200, Vd @ 55,296, Vm @ 57,344; 59,392 B.
+// F16 V stores the values, fp16 [256 tok][128 dims] @ 34,816, and no scales;
+// 100,352 B.
 template <int VT>
 struct PageGeom {
-    static_assert(VT == kVQ4_0 || VT == kVQ4_1 || VT == kVQ5_0 || VT == kVQ5_1 || VT == kVQ8_0, "V type");
-    static constexpr int kVqRow = VT == kVQ8_0 ? kHeadDim : kHeadDim / 2;  // V code bytes per token
+    static_assert(VT == kVF16 || VT == kVQ4_0 || VT == kVQ4_1 || VT == kVQ5_0 || VT == kVQ5_1 || VT == kVQ8_0,
+                  "V type");
+    static constexpr int kVqRow =                                           // V code bytes per token
+        VT == kVQ8_0 ? kHeadDim : (VT == kVF16 ? kHeadDim * 2 : kHeadDim / 2);
     static constexpr int kVhRow = v_has_fifth(VT) ? kBlocks * 4 : 0;      // V fifth-bit bytes per token
+    static constexpr int kVdRow = VT == kVF16 ? 0 : kBlocks * 2;          // V scale bytes per token
     static constexpr int kVmRow = v_has_min(VT) ? kBlocks * 2 : 0;        // V minimum bytes per token
     static constexpr int kOffVq = kOffKd + kPageTokens * kBlocks * 2;       // 34816
     static constexpr int kOffVh = kOffVq + kPageTokens * kVqRow;
     static constexpr int kOffVd = kOffVh + kPageTokens * kVhRow;
-    static constexpr int kOffVm = kOffVd + kPageTokens * kBlocks * 2;
+    static constexpr int kOffVm = kOffVd + kPageTokens * kVdRow;
     static constexpr int kHeadBytes = kOffVm + kPageTokens * kVmRow;
     static constexpr int kRows = kHeadBytes / 128;
     static constexpr int kLevels = VT == kVQ4_1 ? 15 : 31;                // Q4_1 / Q5_1 steps
     static constexpr int kVBlockBytes =                                    // canonical block
-        VT == kVQ8_0 ? 34 : (VT == kVQ5_0 ? 22 : (VT == kVQ4_1 ? 20 : (VT == kVQ5_1 ? 24 : 18)));
+        VT == kVQ8_0 ? 34
+                     : (VT == kVQ5_0 ? 22 : (VT == kVQ4_1 ? 20 : (VT == kVQ5_1 ? 24 : (VT == kVF16 ? 64 : 18))));
 };
 static_assert(PageGeom<kVQ4_0>::kHeadBytes == kPageHeadBytes && PageGeom<kVQ4_0>::kOffVd == kOffVd,
               "Q4_0 geometry");
@@ -82,6 +91,7 @@ static_assert(PageGeom<kVQ5_0>::kHeadBytes == 57344 && PageGeom<kVQ5_0>::kOffVh 
 static_assert(PageGeom<kVQ4_1>::kHeadBytes == 55296 && PageGeom<kVQ4_1>::kOffVd == 51200 &&
                   PageGeom<kVQ4_1>::kOffVm == 53248 && PageGeom<kVQ4_1>::kHeadBytes % 128 == 0,
               "Q4_1 geometry");
+static_assert(PageGeom<kVF16>::kHeadBytes == 100352 && PageGeom<kVF16>::kHeadBytes % 128 == 0, "F16 geometry");
 static_assert(PageGeom<kVQ5_1>::kHeadBytes == 59392 && PageGeom<kVQ5_1>::kOffVh == 51200 &&
                   PageGeom<kVQ5_1>::kOffVd == 55296 && PageGeom<kVQ5_1>::kOffVm == 57344 &&
                   PageGeom<kVQ5_1>::kHeadBytes % 128 == 0,
@@ -92,11 +102,13 @@ inline int page_head_bytes(int v_type) {
         case kVQ5_0: return PageGeom<kVQ5_0>::kHeadBytes;
         case kVQ4_1: return PageGeom<kVQ4_1>::kHeadBytes;
         case kVQ5_1: return PageGeom<kVQ5_1>::kHeadBytes;
+        case kVF16: return PageGeom<kVF16>::kHeadBytes;
         default: return PageGeom<kVQ4_0>::kHeadBytes;
     }
 }
 inline bool v_type_supported(int v_type) {
-    return v_type == kVQ4_0 || v_type == kVQ4_1 || v_type == kVQ5_0 || v_type == kVQ5_1 || v_type == kVQ8_0;
+    return v_type == kVF16 || v_type == kVQ4_0 || v_type == kVQ4_1 || v_type == kVQ5_0 || v_type == kVQ5_1 ||
+           v_type == kVQ8_0;
 }
 
 // split partials: per split and query row, (m, l) in the log2 domain + acc[128]

@@ -43,7 +43,8 @@ __device__ __forceinline__ float q4_to_f(uint32_t c) {
 //       d = (hi - lo)/L with L = 15 / 31, q = min(L, trunc((x - lo)/d + 0.5)),
 //       d == 0 -> q = 0; the block minimum is stored as an fp16 m.
 // The stored scales are the fp16 (round-to-nearest-even) values of d.
-// K is always Q8_0; V is Q4_0 (VT = 2), Q4_1 (3), Q5_0 (6), Q5_1 (7) or Q8_0 (8).
+// K is always Q8_0; V is F16 (VT = 1, the values as they are), Q4_0 (2),
+// Q4_1 (3), Q5_0 (6), Q5_1 (7) or Q8_0 (8).
 // ----------------------------------------------------------------------------
 // Q8_0 of the 32-value block spread over 8 lanes (4 values each): the lane's
 // 4 codes packed in one word (byte u = code of value u), and the block scale
@@ -108,6 +109,21 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
                 *reinterpret_cast<__half*>(ph + kOffKd + t * 8 + 2 * b) = dk_h;
                 *reinterpret_cast<__half*>(ph + G::kOffVd + t * 8 + 2 * b) = dv_h;
             }
+        };
+        store(a.host_layer + (size_t)page * a.page_bytes + (size_t)h * G::kHeadBytes);
+        if (page >= a.first_resident_page) {
+            const int slot = page % a.n_resident;
+            store(a.res_layer + (size_t)slot * a.page_bytes + (size_t)h * G::kHeadBytes);
+        }
+        return;
+    }
+
+    if constexpr (VT == kVF16) {
+        // ---- F16 (V): the values as they are ----
+        auto store = [&](uint8_t* ph) {
+            *reinterpret_cast<uint32_t*>(ph + kOffKq + t * kHeadDim + 4 * lane) = kq;
+            if (i == 0) *reinterpret_cast<__half*>(ph + kOffKd + t * 8 + 2 * b) = dk_h;
+            *reinterpret_cast<uint2*>(ph + G::kOffVq + t * G::kVqRow + 8 * lane) = vraw;
         };
         store(a.host_layer + (size_t)page * a.page_bytes + (size_t)h * G::kHeadBytes);
         if (page >= a.first_resident_page) {
@@ -236,6 +252,8 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
         append_kernel<kVQ4_1><<<(rows + 3) / 4, 128, 0, s>>>(a);
     else if (a.v_type == kVQ5_1)
         append_kernel<kVQ5_1><<<(rows + 3) / 4, 128, 0, s>>>(a);
+    else if (a.v_type == kVF16)
+        append_kernel<kVF16><<<(rows + 3) / 4, 128, 0, s>>>(a);
     else
         append_kernel<kVQ4_0><<<(rows + 3) / 4, 128, 0, s>>>(a);
     return cudaGetLastError();
@@ -259,7 +277,8 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
 //   PV   : the probability times the V scale of each (key, block) is the A
 //          operand (one fp16 rounding), the V codes (q - 8 for Q4_0, q - 16
 //          for Q5_0, q for Q8_0) exact in fp16 are the B operand; for Q4_1 /
-//          Q5_1 the A operand is p and B the value fp16(q d + m).
+//          Q5_1 the A operand is p and B the value fp16(q d + m), for F16 V
+//          p and the stored value.
 // A stage buffer is refilled once all eight warps have released it (an
 // mbarrier with eight arrivals); there is no CTA-wide barrier in the loop.  At
 // the end the eight warps' (m, l, O) are merged into the split's partial.
@@ -284,9 +303,9 @@ static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-B swizzle alignment
 static_assert(kWarps * kMaxRows * (kHeadDim + 2) * 4 <= kStages * kStageBytes, "merge scratch fits");
 
 // Stage and shared-memory geometry by V type: a Q8_0-V stage carries 128 B of
-// V codes per key (34,816 B per stage), so it keeps two stages in flight to
-// stay at two CTAs per SM; a Q5_0-V stage adds 16 B of fifth bits per key
-// (28,672 B) and keeps three.
+// V codes per key (34,816 B per stage) and an F16-V stage 256 B of values
+// (50,176 B), so they keep two stages in flight to stay at two CTAs per SM;
+// a Q5_0-V stage adds 16 B of fifth bits per key (28,672 B) and keeps three.
 template <int VT>
 struct DecGeom {
     static constexpr int kVqRow = PageGeom<VT>::kVqRow;
@@ -295,9 +314,9 @@ struct DecGeom {
     static constexpr int kStageVq = kStageKd + kStageKeys * kBlocks * 2;   // 17408
     static constexpr int kStageVh = kStageVq + kStageKeys * kVqRow;
     static constexpr int kStageVd = kStageVh + kStageKeys * kVhRow;
-    static constexpr int kStageVm = kStageVd + kStageKeys * kBlocks * 2;
+    static constexpr int kStageVm = kStageVd + kStageKeys * PageGeom<VT>::kVdRow;
     static constexpr int kStageBytes = kStageVm + kStageKeys * kVmRow;
-    static constexpr int kStages = VT == kVQ8_0 ? 2 : 3;
+    static constexpr int kStages = (VT == kVQ8_0 || VT == kVF16) ? 2 : 3;
     static constexpr size_t kOffQ = (size_t)kStages * kStageBytes;
     static constexpr size_t kOffKend = kOffQ + kQFragBytes;
     static constexpr size_t kOffBar = kOffKend + kMaxRows * 4;
@@ -314,6 +333,8 @@ static_assert(2 * DecGeom<kVQ4_1>::kSmem <= 232448 && DecGeom<kVQ4_1>::kStageByt
               "two Q4_1-V CTAs per SM");
 static_assert(2 * DecGeom<kVQ5_1>::kSmem <= 232448 && DecGeom<kVQ5_1>::kStageBytes == 29696,
               "two Q5_1-V CTAs per SM");
+static_assert(2 * DecGeom<kVF16>::kSmem <= 232448 && DecGeom<kVF16>::kStageBytes == 50176,
+              "two F16-V CTAs per SM");
 
 size_t decode_smem_bytes() { return kDecodeSmem; }
 
@@ -432,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const uint8_t* vd = ph + PG::kOffVd + half * (kStageKeys * kBlocks * 2);
             for (int c = lane; c < kStageKeys * kBlocks * 2 / 16; c += 32) {
                 cp_async16(dst + kStageKd + c * 16, kd + c * 16);
-                cp_async16(dst + kStageVd + c * 16, vd + c * 16);
+                if constexpr (PG::kVdRow > 0) cp_async16(dst + kStageVd + c * 16, vd + c * 16);
             }
 #pragma unroll 4
             for (int c = lane; c < kStageKeys * PG::kVqRow / 16; c += 32)
@@ -456,7 +477,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             bulk_load(dst + kStageVq, ph + PG::kOffVq + half * (kStageKeys * PG::kVqRow), kStageKeys * PG::kVqRow, b);
             if constexpr (PG::kVhRow > 0)
                 bulk_load(dst + kStageVh, ph + PG::kOffVh + half * (kStageKeys * PG::kVhRow), kStageKeys * PG::kVhRow, b);
-            bulk_load(dst + kStageVd, ph + PG::kOffVd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
+            if constexpr (PG::kVdRow > 0)
+                bulk_load(dst + kStageVd, ph + PG::kOffVd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
             if constexpr (PG::kVmRow > 0)
                 bulk_load(dst + kStageVm, ph + PG::kOffVm + half * (kStageKeys * PG::kVmRow), kStageKeys * PG::kVmRow, b);
         }
@@ -591,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         // rounded once relative to itself (a separate fp32 sum of p m would
         // cancel against q d when the block minimum is large)
         uint32_t pp0 = 0u, pp1 = 0u;
-        if constexpr (v_has_min(VT)) {
+        if constexpr (v_a_is_p(VT)) {
             pp0 = h2u(__floats2half2_rn(p[0][0], p[0][1]));
             pp1 = h2u(__floats2half2_rn(p[1][0], p[1][1]));
         }
@@ -605,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int blk = 0; blk < kBlocks; ++blk) {
             // probabilities x the V scale of block blk, as the A operand
             uint32_t pa0, pa1;
-            if constexpr (v_has_min(VT)) {
+            if constexpr (v_a_is_p(VT)) {
                 pa0 = pp0;
                 pa1 = pp1;
             } else {
@@ -619,12 +641,16 @@ __global__ void __launch_bounds__(kThreads, 2)
             // Q5_0: fifth bits of dims 32 blk + 4g + {0..3} of both keys of
             // n-tile t, in bits 0..3 (first key) and 16..19 (second key)
             uint32_t hv[2] = {0u, 0u};
+            // F16: the four fp16 values of dims 32 blk + 4g + {0..3} of each key
+            uint2 wf[2][2];
 #pragma unroll
             for (int t = 0; t < 2; ++t)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int key = wkey + 8 * t + (j ? k1 : k0);
-                    if constexpr (VT == kVQ8_0)
+                    if constexpr (VT == kVF16)
+                        wf[t][j] = *reinterpret_cast<const uint2*>(vst + key * (kHeadDim * 2) + (32 * blk + 4 * g) * 2);
+                    else if constexpr (VT == kVQ8_0)
                         wv[t][j] = *reinterpret_cast<const uint32_t*>(vst + key * kHeadDim + 32 * blk + 4 * g) ^
                                    0x80808080u;
                     else
@@ -639,6 +665,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                 uint32_t bv[2];
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
+                    if constexpr (VT == kVF16) {  // the two keys' values of dim 32 blk + 4g + m
+                        const uint32_t a0 = (m < 2) ? wf[t][0].x : wf[t][0].y;
+                        const uint32_t a1 = (m < 2) ? wf[t][1].x : wf[t][1].y;
+                        bv[t] = __byte_perm(a0, a1, (m & 1) ? 0x7632u : 0x5410u);
+                        continue;
+                    }
                     const uint32_t pr = __byte_perm(wv[t][0], wv[t][1], sel);
                     if constexpr (VT == kVQ8_0)
                         bv[t] = h2u(__hsub2(u2h((pr & 0x00ff00ffu) | 0x64006400u), b1152));
@@ -750,6 +782,7 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, int n_sp
     if (a.v_type == kVQ5_0) return launch_decode_rows<false, kVQ5_0>(a, kmap, n_splits, s);
     if (a.v_type == kVQ4_1) return launch_decode_rows<false, kVQ4_1>(a, kmap, n_splits, s);
     if (a.v_type == kVQ5_1) return launch_decode_rows<false, kVQ5_1>(a, kmap, n_splits, s);
+    if (a.v_type == kVF16) return launch_decode_rows<false, kVF16>(a, kmap, n_splits, s);
     return launch_decode_rows<false, kVQ4_0>(a, kmap, n_splits, s);
 }
 
@@ -759,6 +792,7 @@ cudaError_t launch_decode_zero_copy(const DecodeArgs& a, const CUtensorMap* kmap
     if (a.v_type == kVQ5_0) return launch_decode_rows<true, kVQ5_0>(a, kmap, n_splits, s);
     if (a.v_type == kVQ4_1) return launch_decode_rows<true, kVQ4_1>(a, kmap, n_splits, s);
     if (a.v_type == kVQ5_1) return launch_decode_rows<true, kVQ5_1>(a, kmap, n_splits, s);
+    if (a.v_type == kVF16) return launch_decode_rows<true, kVF16>(a, kmap, n_splits, s);
     return launch_decode_rows<true, kVQ4_0>(a, kmap, n_splits, s);
 }
 

@@ -209,7 +209,7 @@ int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::stri
     if (c.page_tokens != kPageTokens) { why = fmt("page_tokens %d unsupported (only 256)", c.page_tokens); return KVS_E_INVAL; }
     if (c.type_k != KVS_TYPE_Q8_0 || !v_type_supported(c.type_v)) {
         why = "block KV streaming is not supported for this K/V cache type pair "
-              "(K=Q8_0 with V=Q4_0, Q4_1, Q5_0, Q5_1 or Q8_0)";
+              "(K=Q8_0 with V=F16, Q4_0, Q4_1, Q5_0, Q5_1 or Q8_0)";
         return KVS_E_INVAL;
     }
     if (c.max_ctx < 1) { why = "max_ctx must be >= 1"; return KVS_E_INVAL; }
@@ -1084,6 +1084,7 @@ int kvs_export_page(kvs_t* kv, int layer, int page, int from_device, void* host_
         case KVS_TYPE_Q5_0: KVS_V_FIELDS(kVQ5_0) break;
         case KVS_TYPE_Q4_1: KVS_V_FIELDS(kVQ4_1) break;
         case KVS_TYPE_Q5_1: KVS_V_FIELDS(kVQ5_1) break;
+        case KVS_TYPE_F16: KVS_V_FIELDS(kVF16) break;
         default: KVS_V_FIELDS(kVQ4_0) break;
 #undef KVS_V_FIELDS
     }
@@ -1100,6 +1101,10 @@ int kvs_export_page(kvs_t* kv, int layer, int page, int from_device, void* host_
                 std::memcpy(kb, ph + kOffKd + t * 8 + b * 2, 2);
                 std::memcpy(kb + 2, ph + kOffKq + t * kHeadDim + b * 32, 32);
                 uint8_t* vb = vout + (((size_t)t * H + h) * kBlocks + b) * vblk;
+                if (c.type_v == KVS_TYPE_F16) {  // the 32 values of the block
+                    std::memcpy(vb, ph + off_vq + t * (kHeadDim * 2) + b * 64, 64);
+                    continue;
+                }
                 std::memcpy(vb, ph + off_vd + t * 8 + b * 2, 2);
                 int at = 2;
                 if (has_m) { std::memcpy(vb + at, ph + off_vm + t * 8 + b * 2, 2); at += 2; }

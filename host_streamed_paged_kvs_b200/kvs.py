@@ -22,6 +22,7 @@ KVS_E_ORDER = -4
 KVS_E_CUDA = -5
 KVS_E_TIMEOUT = -6
 KVS_E_NOMEM = -7
+KVS_TYPE_F16 = 1
 KVS_TYPE_Q4_0 = 2
 KVS_TYPE_Q4_1 = 3
 KVS_TYPE_Q5_0 = 6

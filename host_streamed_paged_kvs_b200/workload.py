@@ -40,7 +40,7 @@ class Workload:
     outlier_scale: float = 1.0
     head_dim: int = HEAD_DIM
     page_tokens: int = PAGE_TOKENS
-    type_v: int = 2       # V block type: 2 Q4_0, 3 Q4_1, 6 Q5_0, 7 Q5_1, 8 Q8_0 (the q8_0/q8_0 pair)
+    type_v: int = 2       # V type: 1 F16, 2 Q4_0, 3 Q4_1, 6 Q5_0, 7 Q5_1, 8 Q8_0 (the q8_0/q8_0 pair)
 
     @property
     def n_pages(self) -> int:

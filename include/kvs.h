@@ -49,7 +49,8 @@ extern "C" {
 #define KVS_E_TIMEOUT (-6) /* a bounded host wait gave up                         */
 #define KVS_E_NOMEM   (-7) /* host (pinned) allocation failed                     */
 
-/* ---- cache types: K is Q8_0; V is Q4_0, Q4_1, Q5_0, Q5_1 or Q8_0 ----------- */
+/* ---- cache types: K is Q8_0; V is F16, Q4_0, Q4_1, Q5_0, Q5_1 or Q8_0 ------ */
+#define KVS_TYPE_F16  1
 #define KVS_TYPE_Q4_0 2
 #define KVS_TYPE_Q4_1 3
 #define KVS_TYPE_Q5_0 6
@@ -90,7 +91,8 @@ typedef struct kvs_config {
                              KVS_TYPE_Q5_0 (57,344 B: Q4_0's nibbles plus a word of fifth
                              bits per block), KVS_TYPE_Q4_1 (55,296 B: Q4_0's layout plus an
                              fp16 block minimum m, x = d q + m), KVS_TYPE_Q5_1 (59,392 B:
-                             Q5_0's layout plus m) */
+                             Q5_0's layout plus m), KVS_TYPE_F16 (100,352 B: the V values
+                             as fp16 [256 tok][128 dims], no scales) */
     int chunk_pages;      /* pages per H2D copy; 0 = auto (n_ring_slots/2); must divide n_ring_slots */
     int flags;            /* KVS_FLAG_* */
     int zero_copy_pct;    /* 0..100: share of each layer's streamed pages (the newest ones) that
@@ -229,7 +231,8 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
  * type_v is KVS_TYPE_Q8_0, or Q5_0 blocks of 22 bytes when it is KVS_TYPE_Q5_0
  * (fp16 d, a little-endian word whose bit j is bit 4 of q_j, then 16 bytes
  * holding the low 4 bits as Q4_0 does); Q4_1 (20 bytes) and Q5_1 (24 bytes)
- * blocks put the fp16 block minimum m right after d.  from_device = 0 reads the host history,
+ * blocks put the fp16 block minimum m right after d; F16 blocks are the 32
+ * fp16 values (64 bytes).  from_device = 0 reads the host history,
  * 1 reads the resident slot (KVS_E_INVAL if the page is not resident).  The
  * caller must have synchronized the streams that wrote the page. */
 int kvs_export_page(kvs_t* kv, int layer, int page, int from_device, void* host_dst);

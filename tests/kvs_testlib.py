@@ -85,7 +85,7 @@ def export_page(h, cfg, layer, page, from_device):
     from host_streamed_paged_kvs_b200 import kvs
     H = cfg.n_kv_heads
     vbytes = {kvs.KVS_TYPE_Q8_0: 34, kvs.KVS_TYPE_Q5_0: 22, kvs.KVS_TYPE_Q4_1: 20,
-              kvs.KVS_TYPE_Q5_1: 24}.get(cfg.type_v, 18)
+              kvs.KVS_TYPE_Q5_1: 24, kvs.KVS_TYPE_F16: 64}.get(cfg.type_v, 18)
     nk = T * H * 4 * 34
     nv = T * H * 4 * vbytes
     buf = np.zeros(nk + nv, np.uint8)

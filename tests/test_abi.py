@@ -65,7 +65,8 @@ def test_plan_page_matches_oracle(kvs):
 
 
 @pytest.mark.parametrize("over,code", [
-    (dict(type_k=2), -1), (dict(type_v=1), -1), (dict(type_k=8, type_v=4), -1), (dict(type_v=5), -1),
+    (dict(type_k=2), -1), (dict(type_v=0), -1), (dict(type_k=8, type_v=4), -1), (dict(type_v=5), -1),
+    (dict(type_k=1, type_v=1), -1),
     (dict(type_v=9), -1),
     (dict(type_k=6, type_v=6), -1), (dict(head_dim=64), -1), (dict(page_tokens=128), -1),
     (dict(n_q_heads=12, n_kv_heads=8), -1), (dict(n_ring_slots=0, n_resident_pages=4), -1),
@@ -109,10 +110,10 @@ def test_q5_0_v_pair_geometry(kvs):
     assert r.arena_bytes - r4.arena_bytes == (2 * 8 + 8) * 8 * (57344 - 53248)
 
 
-@pytest.mark.parametrize("tv,head", [(3, 55296), (7, 59392)])
+@pytest.mark.parametrize("tv,head", [(3, 55296), (7, 59392), (1, 100352)])
 def test_min_type_v_pair_geometry(kvs, tv, head):
     """The q8_0/q4_1 and q8_0/q5_1 pairs: Q4_0's (Q5_0's) V fields plus an fp16
-    block minimum per token, kv head and block."""
+    block minimum per token, kv head and block; q8_0/f16: the V values as fp16."""
     c = kvs.make_config(2, 32, 8, 32768, n_resident_pages=8, n_ring_slots=8, type_v=tv)
     r, host = kvs.kvs_resolve_config(c)
     assert r.type_v == tv

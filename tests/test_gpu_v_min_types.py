@@ -1,8 +1,10 @@
 """The q8_0 / q4_1 and q8_0 / q5_1 K/V pairs (V blocks with a minimum m,
-x = d q + m): bit-exact pages against the oracle's blocks, and attention parity
-on every path (resident, ring, in-place share, tensor-core verify and prefill
-widths).  The values carry 1-2 % outliers x8 of both signs, so blocks with a
-large-magnitude minimum (where q d and m nearly cancel) occur."""
+x = d q + m) and q8_0 / f16 (V stored as its fp16 values): the V types whose
+decode path feeds the tensor cores p and the V value itself.  Bit-exact pages
+against the oracle's blocks, and attention parity on every path (resident,
+ring, in-place share, tensor-core verify and prefill widths).  The values carry
+1-2 % outliers x8 of both signs, so blocks with a large-magnitude minimum
+(where q d and m nearly cancel) occur."""
 import numpy as np
 import pytest
 
@@ -11,7 +13,7 @@ from host_streamed_paged_kvs_b200 import workload as W
 from kvs_testlib import assert_close, export_page, make_cfg, oracle_blocks, oracle_step, prefill, step, to_dev, torch
 
 pytestmark = pytest.mark.gpu
-TYPES = [oracle.V_Q4_1, oracle.V_Q5_1]
+TYPES = [oracle.V_F16, oracle.V_Q4_1, oracle.V_Q5_1]
 
 
 @pytest.fixture(scope="module")
