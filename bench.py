@@ -40,11 +40,11 @@ UNIT = "KV tokens/s/layer"
 # workload it was captured on and only while the kernel source is unchanged
 # (sha256 prefix of the .cu file); otherwise traffic is reported as null.
 NCU_TRAFFIC = {
-    "decode_kernel": {"src": "kvs_kernels.cu", "sha": "000b5e26d6982e24",
+    "decode_kernel": {"src": "kvs_kernels.cu", "sha": "afede6bf62475eb3",
                       "workload": "streamed_decode_32k", "resident": 27296256, "ring": 1737472,
                       # in-place launches (51 pages): DRAM bytes, and host-memory bytes read over PCIe
                       "in_place": 35328, "in_place_sysmem": 21725184},
-    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "721e05dd0b415542",
+    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "d15b6e259e840f49",
                          "workload": "prefill_chunk_64k", "resident": 35606272, "ring": 6079232},
 }
 
