@@ -35,8 +35,31 @@ def test_exports_every_declared_symbol(kvs):
     assert sorted(kvs.EXPORTS) == names
 
 
+def header_defines(prefix):
+    src = open(os.path.join(ROOT, "include", "kvs.h")).read()
+    return {m.group(1): int(m.group(2), 0)
+            for m in re.finditer(r"#define\s+(" + prefix + r"[A-Z0-9_]+)\s+\(?(-?\w+)\)?", src)}
+
+
+def test_header_constants_match_binding_and_oracle(kvs):
+    """The cache-type, page-kind, flag and error codes of include/kvs.h are the
+    binding's, and the V type codes are the oracle's block-type ids."""
+    types = header_defines("KVS_TYPE_")
+    assert types == {"KVS_TYPE_F16": 1, "KVS_TYPE_Q4_0": 2, "KVS_TYPE_Q4_1": 3, "KVS_TYPE_Q5_0": 6,
+                     "KVS_TYPE_Q5_1": 7, "KVS_TYPE_Q8_0": 8}
+    for name, val in types.items():
+        assert getattr(kvs, name) == val
+        assert getattr(oracle, "V_" + name[len("KVS_TYPE_"):]) == val
+    for prefix in ("KVS_PAGE_", "KVS_FLAG_"):
+        for name, val in header_defines(prefix).items():
+            assert getattr(kvs, name) == val, name
+    errors = header_defines("KVS_E_")
+    assert errors and all(kvs.ERROR_NAMES[v] == k for k, v in errors.items())
+    assert kvs.ERROR_NAMES[0] == "KVS_OK"
+
+
 def test_struct_sizes_match_header(kvs):
-    # 13 ints + size_t (padded) ; 8 u64 + 5 double + 7 u64
+    # 14 ints + size_t ; 8 u64, 6 double, 9 u64
     assert ctypes.sizeof(kvs.kvs_config) == 14 * 4 + 8
     assert ctypes.sizeof(kvs.kvs_stats) == (8 + 6 + 9) * 8
 
