@@ -7,7 +7,8 @@
  * Configuration; "Feature/adaptive kv stream integration", PR #326):
  *   - the full KV history of every layer lives in pinned host memory and is
  *     authoritative; K is stored as Q8_0 and V as Q4_0 (blocks of 32 values,
- *     fp16 scale), grouped in 256-token pages;
+ *     fp16 scale; the other V types are listed at kvs_config.type_v), grouped
+ *     in 256-token pages;
  *   - per layer only the most recent R pages are resident in device memory;
  *     older pages stream in order through one device ring of N page slots that
  *     all layers share, on a copy stream, so the copy of page i+k overlaps
