@@ -87,8 +87,8 @@ typedef struct kvs_config {
     int type_v;           /* KVS_TYPE_Q4_0 (page head 53,248 B), KVS_TYPE_Q8_0 (69,632 B: V codes
                              stored like K's; the q8_0/q8_0 pair of the "Feature/adaptive kv
                              stream integration" pull request's runs), or one of the other
-                             legal cache types of the flash-attention build on
-                             "RaymondHuang210129/llama.cpp-adaptive-kv-streaming":
+                             legal cache types of the flash-attention build ("llama.cpp
+                             adaptive KV streaming - spec fork notes", TLDR):
                              KVS_TYPE_Q5_0 (57,344 B: Q4_0's nibbles plus a word of fifth
                              bits per block), KVS_TYPE_Q4_1 (55,296 B: Q4_0's layout plus an
                              fp16 block minimum m, x = d q + m), KVS_TYPE_Q5_1 (59,392 B:

@@ -12,8 +12,9 @@
  *    fp16 scale ("RaymondHuang210129/llama.cpp-adaptive-kv-streaming",
  *    Summary; "llama.cpp adaptive KV streaming - spec fork notes", Results);
  *    V may also be Q8_0 (the q8_0/q8_0 runs of PR #326) or another of the
- *    legal cache types of the flash-attention build (the first page's build
- *    section), each with its own block rule below;
+ *    legal cache types of the flash-attention build ("llama.cpp adaptive KV
+ *    streaming - spec fork notes", TLDR: -DGGML_CUDA_FA_QUANTS), each with its
+ *    own block rule below;
  *  - the KV history is quantized once, when a token is appended, and attention
  *    is exact over every token of the history; streaming only changes where
  *    the bytes live ("Feature/adaptive kv stream integration", PR #326,
@@ -164,8 +165,8 @@ void oracle_q4_0_block(const uint16_t x_h[32], uint8_t out[18]) {
 }
 
 /* Q5_0: the 5-bit member of the same family, one of the cache types the
- * flash-attention build lists as legal ("RaymondHuang210129/llama.cpp-
- * adaptive-kv-streaming", build section: -DGGML_CUDA_FA_QUANTS).  The pages
+ * flash-attention build lists as legal ("llama.cpp adaptive KV streaming -
+ * spec fork notes", TLDR: -DGGML_CUDA_FA_QUANTS).  The pages
  * give no rule; it is read as Q4_0's with 32 levels: d = (signed max)/-16,
  * q = min(31, trunc(x/d + 16.5)), so x ~ d (q - 16). */
 void oracle_q5_0_block(const uint16_t x_h[32], uint8_t out[22]) {

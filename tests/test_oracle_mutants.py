@@ -53,6 +53,19 @@ MUTANTS = {
     "q5_1 fifth bit shifted": ("int a = (int)(blk[8 + j] & 0x0f) | (int)(((top >> j) & 1u) << 4);",
                                "int a = (int)(blk[8 + j] & 0x0f) | (int)(((top >> (j + 1)) & 1u) << 4);"),
     "f16 V byte order": ("out[2 * i] = (uint8_t)(x_h[i] & 0xff);", "out[2 * i] = (uint8_t)(x_h[i] >> 8);"),
+    "q8 reciprocal": ("if (d != 0.0f) q = (int)roundf(x[i] / d);",
+                      "if (d != 0.0f) q = (int)roundf(x[i] * (1.0f / d));"),
+    "q8 fp16 divisor": ("if (d != 0.0f) q = (int)roundf(x[i] / d);",
+                        "if (d != 0.0f) q = (int)roundf(x[i] / oracle_half_to_float(dh));"),
+    "q4 reciprocal": ("int t = (int)(x[i] / d + 8.5f);", "int t = (int)(x[i] * (1.0f / d) + 8.5f);"),
+    "q4 fp16 divisor": ("int t = (int)(x[i] / d + 8.5f);",
+                        "int t = (int)(x[i] / oracle_half_to_float(dh) + 8.5f);"),
+    "q5 reciprocal": ("int t = (int)(x[i] / d + 16.5f);", "int t = (int)(x[i] * (1.0f / d) + 16.5f);"),
+    "q5 fp16 divisor": ("int t = (int)(x[i] / d + 16.5f);",
+                        "int t = (int)(x[i] / oracle_half_to_float(dh) + 16.5f);"),
+    "q1 reciprocal": ("int t = (int)((x[i] - lo) / d + 0.5f);", "int t = (int)((x[i] - lo) * (1.0f / d) + 0.5f);"),
+    "q1 fp16 divisor": ("int t = (int)((x[i] - lo) / d + 0.5f);",
+                        "int t = (int)((x[i] - lo) / oracle_half_to_float(*dh) + 0.5f);"),
     "resident window": ("if (page >= P - n_resident) {", "if (page > P - n_resident) {"),
     "auto floor": ("long floor_pages = (2048 + page_tokens - 1) / page_tokens;",
                    "long floor_pages = (4096 + page_tokens - 1) / page_tokens;"),

@@ -38,7 +38,8 @@ def split_q5(blk: bytes):
 
 def test_q5_0_hand_worked():
     f, _ = read_fixture("q5_0_hand.txt")
-    for tag in ("A", "B", "C"):
+    # D: division, not a rounded reciprocal; E: the binary32 d, not the stored fp16 d
+    for tag in ("A", "B", "C", "D", "E"):
         xs = [float(v) for v in f[f"{tag}_x"]]
         x = h(xs)
         assert np.array_equal(x.astype(np.float64), np.array(xs))  # the inputs are exact in fp16

@@ -49,7 +49,8 @@ def bits_to_float(bits: int) -> float:
 def test_hand_worked(name):
     vt, levels, nbytes, blockfn, deqfn, fixture = TYPES[name]
     f, _ = read_fixture(fixture)
-    for tag in ("A", "B"):
+    # C: division, not a rounded reciprocal; D: the binary32 d, not the stored fp16 d
+    for tag in ("A", "B", "C", "D"):
         xs = [float(v) for v in f[f"{tag}_x"]]
         x = h(xs)
         assert np.array_equal(x.astype(np.float64), np.array(xs))  # exact in fp16

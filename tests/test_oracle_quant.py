@@ -37,12 +37,24 @@ def test_q8_0_hand_worked():
     d, q = split_q8(oracle.q8_0_block(x))
     assert d == int(f["d_bits"][0], 16)
     assert q.tolist() == [int(v) for v in f["q"]]
+    # C: the code of a correctly rounded x / d (a rounded 1/d would flip it);
+    # D: the code with the binary32 d as divisor (the stored fp16 d would flip it)
+    for tag in ("C", "D"):
+        xs = [float(v) for v in f[f"{tag}_x"]]
+        x = h(xs)
+        assert np.array_equal(x.astype(np.float64), np.array(xs))
+        d, q = split_q8(oracle.q8_0_block(x))
+        assert d == int(f[f"{tag}_d_bits"][0], 16), tag
+        assert q.tolist() == [int(v) for v in f[f"{tag}_q"]], tag
 
 
 def test_q4_0_hand_worked():
     f, _ = read_fixture("q4_0_hand.txt")
-    for tag in ("A", "B"):
-        x = h([float(v) for v in f[f"{tag}_x"]])
+    # C: division, not a rounded reciprocal; D: the binary32 d, not the stored fp16 d
+    for tag in ("A", "B", "C", "D"):
+        xs = [float(v) for v in f[f"{tag}_x"]]
+        x = h(xs)
+        assert np.array_equal(x.astype(np.float64), np.array(xs))  # exact in fp16
         blk = oracle.q4_0_block(x)
         d, q = split_q4(blk)
         assert d == int(f[f"{tag}_d_bits"][0], 16)
