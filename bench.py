@@ -250,6 +250,110 @@ def run_reference(args, w: W.Workload):
 
 
 # ---------------------------------------------------------------------------
+# copy / compute timeline (CUPTI activity records through torch.profiler)
+# ---------------------------------------------------------------------------
+def _union(iv):
+    """Merged [start, end) intervals of a list of (start, end)."""
+    out = []
+    for a, b in sorted(iv):
+        if out and a <= out[-1][1]:
+            out[-1][1] = max(out[-1][1], b)
+        else:
+            out.append([a, b])
+    return out
+
+
+def _length(iv):
+    return sum(b - a for a, b in iv)
+
+
+def _intersect(x, y):
+    """Total length of the intersection of two merged interval lists."""
+    i = j = 0
+    tot = 0.0
+    while i < len(x) and j < len(y):
+        a, b = max(x[i][0], y[j][0]), min(x[i][1], y[j][1])
+        if b > a:
+            tot += b - a
+        if x[i][1] < y[j][1]:
+            i += 1
+        else:
+            j += 1
+    return tot
+
+
+def timeline_summary(trace_path: str, n_steps: int, h2d_peak: float):
+    """Summary of one profiled run of n_steps steps from its trace: the
+    host-to-device copy rows (the ring's copy engine), the library's kernels
+    per kind, how much of the copy time overlaps kernels, and how busy the
+    host-to-device link is (ring copies together with the in-place decode
+    launches, which read host memory over the same link)."""
+    with open(trace_path) as f:
+        ev = json.load(f)["traceEvents"]
+    kern, copies = [], []
+    for e in ev:
+        if e.get("ph") != "X":
+            continue
+        cat = e.get("cat", "")
+        if cat == "kernel":
+            kern.append(e)
+        elif cat == "gpu_memcpy" and "HtoD" in e.get("name", ""):
+            copies.append(e)
+    if not kern:
+        return None
+
+    def kind(name):
+        if "decode_kernel" in name:
+            return "decode_in_place" if ", true," in name else "decode_tma"
+        for k in ("chunk_mma_kernel", "merge_rows_kernel", "merge_kernel", "append_kernel", "copy16_kernel"):
+            if k in name:
+                return k
+        return "other"
+
+    t0 = min(e["ts"] for e in kern + copies)
+    t1 = max(e["ts"] + e["dur"] for e in kern + copies)
+    win = t1 - t0
+    cp = _union([(e["ts"], e["ts"] + e["dur"]) for e in copies])
+    kinds = {}
+    for e in kern:
+        kinds.setdefault(kind(e["name"]), []).append((e["ts"], e["ts"] + e["dur"]))
+    all_k = _union([iv for v in kinds.values() for iv in v])
+    zc = _union(kinds.get("decode_in_place", []))
+    link = _union(cp + zc)
+    gaps = sorted((b[0] - a[1] for a, b in zip(link, link[1:])), reverse=True)
+    cbytes = sum(float(e.get("args", {}).get("bytes", 0)) for e in copies)
+    streams = sorted({(e.get("args", {}).get("stream"), kind(e["name"])) for e in kern}, key=str)
+    return {
+        "steps": n_steps, "window_us": win, "us_per_step": win / n_steps,
+        "h2d_copies": len(copies), "h2d_copy_bytes": cbytes,
+        "copy_engine_busy_us": _length(cp), "copy_engine_busy_frac": _length(cp) / win,
+        "copy_gbs_while_busy": cbytes / (_length(cp) * 1e-6) / 1e9 if cp else None,
+        "copy_time_overlapping_kernels_frac": _intersect(cp, all_k) / _length(cp) if cp else None,
+        "link_busy_frac": _length(link) / win,
+        "link_busy_note": "union of ring copies and in-place decode launches (both read host memory over PCIe)",
+        "largest_link_gaps_us": gaps[:5],
+        "kernel_busy_us": {k: _length(_union(v)) for k, v in kinds.items()},
+        "kernel_launches": {k: len(v) for k, v in kinds.items()},
+        "streams_by_kind": [f"{st}:{k}" for st, k in streams],
+        "h2d_gbs_peak_measured": h2d_peak,
+    }
+
+
+def capture_timeline(step_fn, n_steps: int, path: str, sync):
+    """Record n_steps calls of step_fn under torch.profiler (CUPTI activity
+    records of every kernel and copy, the library's included) and write the
+    Chrome trace to path."""
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+    sync()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        for _ in range(n_steps):
+            step_fn()
+        sync()
+    prof.export_chrome_trace(path)
+
+
+# ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
 def run_gpu(args, w: W.Workload):
@@ -273,8 +377,6 @@ def run_gpu(args, w: W.Workload):
                                                 n_ring_slots=w.n_ring_slots, type_v=w.type_v))[0]
     zc_able = (w.n_q * (w.n_q_heads // w.n_kv_heads) <= 8 and r0.n_resident_pages < w.n_pages
                and w.n_ring_slots > 0)
-    # the comparison arms need a second pinned history: only when it is small
-    arms_able = zc_able and L * w.n_pages * kvs.kvs_page_bytes(r0) <= (4 << 30)
     zc_pct = (W.ZERO_COPY_PCT if args.zero_copy_pct < 0 else args.zero_copy_pct) if zc_able else 0
     cfg = kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx, n_resident_pages=w.n_resident_pages,
                           n_ring_slots=w.n_ring_slots, max_q_tokens=w.n_q,
@@ -392,33 +494,31 @@ def run_gpu(args, w: W.Workload):
         eager_line = {"ms_per_step": ms_eager, "value": job_value(world, w.ctx, L, ms_eager),
                       "unit": UNIT, "kernel_launches": int(kvs.kvs_get_stats(h)["kernel_launches"])}
 
-    # ---- comparison arms: the same steps on handles that split the streamed
-    #      pages differently between the copy-engine ring and in-place reads
-    #      of the mapped pinned history by the decode kernel ----
+    # ---- comparison arms: the same steps with the streamed pages split
+    #      differently between the copy-engine ring and in-place reads of the
+    #      mapped pinned history by the decode kernel (the share is switched
+    #      on the same handle: its partial buffer is sized for every share) ----
     arms = {}
-    if args.arms and arms_able:
+    if args.arms and zc_able:
         for name, pct in (("ring_only", 0), ("zero_copy_only", 100)):
             if pct == zc_pct:
                 continue
-            cz = kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx, n_resident_pages=w.n_resident_pages,
-                                 n_ring_slots=w.n_ring_slots, max_q_tokens=w.n_q,
-                                 chunk_pages=args.chunk_pages, zero_copy_pct=pct, type_v=w.type_v)
-            hz = kvs.kvs_create(cz, local)
-            prefill_history(hz)
+            kvs.kvs_set_zero_copy_pct(h, pct)
             for _ in range(args.warmup):
-                one_step(ks, vs, qs, out, lse, hz)
+                one_step(ks, vs, qs, out, lse)
             barrier()
             e0.record(stream)
             for _ in range(args.steps):
-                one_step(ks, vs, qs, out, lse, hz)
+                one_step(ks, vs, qs, out, lse)
             e1.record(stream)
             barrier()
             ms_a = max_over_ranks(e0.elapsed_time(e1)) / args.steps
             S_a = w.n_pages - rc.n_resident_pages
             arms[name] = {"zero_copy_pct": pct, "ms_per_step": ms_a,
                           "value": job_value(world, w.ctx, L, ms_a), "unit": UNIT,
-                          "h2d_gbs_achieved": L * S_a * pb / (ms_a * 1e-3) / 1e9}
-            kvs.kvs_destroy(hz)
+                          "h2d_gbs_achieved": L * S_a * pb / (ms_a * 1e-3) / 1e9,
+                          "launch": "plain library calls"}
+        kvs.kvs_set_zero_copy_pct(h, zc_pct)
 
     # ---- end to end through the C ABI with pinned host buffers ----
     kh = [x.cpu().pin_memory() for x in ks]
@@ -474,6 +574,25 @@ def run_gpu(args, w: W.Workload):
         best = max(best, (1 << 30) / (a.elapsed_time(b) * 1e-3) / 1e9)
     h2d_peak = max(best, h2d_ring or 0.0)
     del big, dbig
+
+    # ---- copy / compute timeline of a few plain steps, at the tuned share and
+    #      ring-only (optional: --timeline DIR) ----
+    timeline = None
+    if args.timeline and rank == 0:
+        os.makedirs(args.timeline, exist_ok=True)
+        timeline = {}
+        shares = [("tuned", zc_pct)] + ([("ring_only", 0)] if zc_able and zc_pct != 0 else [])
+        for tag, pct in shares:
+            kvs.kvs_set_zero_copy_pct(h, pct)
+            for _ in range(2):
+                one_step(ks, vs, qs, out, lse)
+            path = os.path.join(args.timeline, f"timeline_{w.name}_{tag}.json")
+            n_tl = 3
+            capture_timeline(lambda: one_step(ks, vs, qs, out, lse), n_tl, path, barrier)
+            timeline[tag] = timeline_summary(path, n_tl, h2d_peak)
+            if timeline[tag] is not None:
+                timeline[tag]["zero_copy_pct"] = pct
+        kvs.kvs_set_zero_copy_pct(h, zc_pct)
 
     hbm_peak, peak_src = peaks()
     P = w.n_pages
@@ -601,6 +720,8 @@ def run_gpu(args, w: W.Workload):
         "clocks": clk,
         "prefill_s": prefill_s,
     }
+    if timeline is not None:
+        line["timeline"] = timeline
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     del timed_step
@@ -629,6 +750,9 @@ def main():
                     help="share of streamed pages decode reads in place (default: the tuned share)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time plain library calls instead of replays of a captured step")
+    ap.add_argument("--timeline", default="",
+                    help="directory: after timing, record a few plain steps' copy/compute timeline "
+                         "(Chrome trace) and add its summary to the line")
     args = ap.parse_args()
     w = W.WORKLOADS[args.workload]
     if args.steps <= 0:

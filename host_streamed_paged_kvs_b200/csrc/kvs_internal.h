@@ -151,11 +151,16 @@ struct DecodeArgs {
     int v_type;              // kVQ4_0 or kVQ8_0: the page-head geometry
 };
 
+// query rows from which the merge writes out with 16-byte stores
+constexpr int kMergeRowsMin = 1024;
+
 struct MergeArgs {
     PartialBuffers part;
     int n_splits, n_rows;
     float* out;              // [n_rows][128]
     float* lse;              // [n_rows] or null
+    const int* err;          // optional error word: when it is non-zero the
+                             // merge writes NaN (a split's partial is missing)
 };
 
 // launchers (return cudaGetLastError())

@@ -811,6 +811,13 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const MergeArgs a)
     const int slice = blockIdx.y;  // dims [32 slice, 32 slice + 32)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int W = kMergeThreads / 32;
+    if (a.err && *reinterpret_cast<const volatile int*>(a.err)) {  // a split's partial is missing
+        if (warp == 0) {
+            a.out[(size_t)row * kHeadDim + slice * 32 + lane] = CUDART_NAN_F;
+            if (slice == 0 && lane == 0 && a.lse) a.lse[row] = CUDART_NAN_F;
+        }
+        return;
+    }
     const float2* ml = a.part.ml + row;
     float m = -CUDART_INF_F;
     for (int s = tid; s < a.n_splits; s += kMergeThreads) m = fmaxf(m, ml[(size_t)s * a.n_rows].x);
@@ -869,6 +876,12 @@ __global__ void __launch_bounds__(256) merge_rows_kernel(const MergeArgs a) {
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= a.n_rows) return;
+    if (a.err && *reinterpret_cast<const volatile int*>(a.err)) {  // a split's partial is missing
+        *reinterpret_cast<float4*>(a.out + (size_t)row * kHeadDim + 4 * lane) =
+            make_float4(CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F);
+        if (lane == 0 && a.lse) a.lse[row] = CUDART_NAN_F;
+        return;
+    }
     const float2* ml = a.part.ml + row;
     float m = -CUDART_INF_F;
     for (int s = lane; s < a.n_splits; s += 32) m = fmaxf(m, ml[(size_t)s * a.n_rows].x);
@@ -914,7 +927,7 @@ __global__ void __launch_bounds__(256) merge_rows_kernel(const MergeArgs a) {
 }
 
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s) {
-    if (a.n_rows >= 1024) {
+    if (a.n_rows >= kMergeRowsMin) {
         merge_rows_kernel<<<(a.n_rows + 7) / 8, 256, 0, s>>>(a);
     } else {
         merge_kernel<<<dim3(a.n_rows, kHeadDim / 32), kMergeThreads, 0, s>>>(a);

@@ -146,14 +146,22 @@ long count_splits(const kvs_config& c, int n_q, long R_eff, long S) {
 
 // capacity of the partial buffer in (split x row) records: the largest need
 // over every query width the handle accepts, at the longest history (split
-// counts only grow with the number of resident and streamed pages)
+// counts only grow with the number of resident and streamed pages), and over
+// every in-place share, so that kvs_set_zero_copy_pct can change it later
 size_t partial_records(const kvs_config& c) {
     const long P = pages_for(c.max_ctx);
     const long R_eff = std::min<long>(c.n_resident_pages, P);
     const long S = c.n_ring_slots > 0 ? P - R_eff : 0;
     size_t best = 1;
-    for (int n_q = 1; n_q <= c.max_q_tokens; ++n_q)
-        best = std::max(best, (size_t)count_splits(c, n_q, R_eff, S) * (size_t)(n_q * c.n_q_heads));
+    for (int n_q = 1; n_q <= c.max_q_tokens; ++n_q) {
+        kvs_config cz = c;
+        // the share only matters for decode widths
+        const int shares = use_tcgen05(c, n_q) ? 1 : 101;
+        for (int pct = 0; pct < shares; ++pct) {
+            if (shares > 1) cz.zero_copy_pct = pct;
+            best = std::max(best, (size_t)count_splits(cz, n_q, R_eff, S) * (size_t)(n_q * c.n_q_heads));
+        }
+    }
     return best;
 }
 
@@ -864,6 +872,23 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     DeviceGuard g(kv->device);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int rows = n_q * c.n_q_heads;
+    const bool tc = use_tcgen05(c, n_q);
+    // Device buffers go to the kernels as they are, so their addresses must
+    // suit the kernels' vector accesses: Q is read in 8-byte words by the
+    // decode kernel and 16-byte words by the tensor-core kernel; out is
+    // written in 16-byte words when the many-row merge runs (>= 1024 rows).
+    // Host buffers are staged or aliased only when 16-byte aligned.
+    {
+        const uintptr_t qa = reinterpret_cast<uintptr_t>(q_f16), oa = reinterpret_cast<uintptr_t>(out);
+        if (!is_host_ptr(q_f16) && (qa & (tc ? 15 : 7)))
+            return fail(kv, KVS_E_INVAL, tc ? "q must be 16-byte aligned for multi-token attention"
+                                            : "q must be 8-byte aligned");
+        if (!is_host_ptr(out) && (oa & (rows >= kMergeRowsMin ? 15 : 3)))
+            return fail(kv, KVS_E_INVAL, rows >= kMergeRowsMin ? "out must be 16-byte aligned for >= 1024 query rows"
+                                                               : "out must be 4-byte aligned");
+        if (lse && !is_host_ptr(lse) && (reinterpret_cast<uintptr_t>(lse) & 3))
+            return fail(kv, KVS_E_INVAL, "lse must be 4-byte aligned");
+    }
     const __half* q = static_cast<const __half*>(q_f16);
     if (is_host_ptr(q_f16)) {
         // pinned: one small copy kernel pulls Q over PCIe; pageable: copy engine
@@ -880,9 +905,6 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     float* dout = out_alias ? out_alias : (host_out ? kv->stage_out : out);
     float* dlse = lse ? (lse_alias ? lse_alias : (host_lse ? kv->stage_lse : lse)) : nullptr;
 
-    const bool tc = use_tcgen05(c, n_q);
-    if (tc && (reinterpret_cast<uintptr_t>(q) & 15))
-        return fail(kv, KVS_E_INVAL, "q must be 16-byte aligned for multi-token attention");
     const long R = c.n_resident_pages;
     const long P = pages_for(ls.len);
     const long R_eff = std::min(R, P);
@@ -1042,6 +1064,7 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     m.n_rows = rows;
     m.out = dout;
     m.lse = dlse;
+    m.err = nullptr;  // a timed-out wait is reported by kvs_sync / kvs_get_stats
     {
         TimedScope ts(kv, s, kTMerge, 0);
         KVS_CK(kv, launch_merge(m, s));
@@ -1155,6 +1178,13 @@ int kvs_reset_stats(kvs_t* kv) {
         fold_timed(kv);
     }
     kv->stats = kvs_stats{};
+    return KVS_OK;
+}
+
+int kvs_set_zero_copy_pct(kvs_t* kv, int pct) {
+    if (!kv) return fail(nullptr, KVS_E_INVAL, "null handle");
+    if (pct < 0 || pct > 100) return fail(kv, KVS_E_INVAL, fmt("zero_copy_pct %d outside 0..100", pct));
+    kv->cfg.zero_copy_pct = pct;  // the partial buffer is sized for every share
     return KVS_OK;
 }
 

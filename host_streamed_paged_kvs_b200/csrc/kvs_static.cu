@@ -12,10 +12,13 @@
 // array of this library, so no handle and no allocation are needed at all.
 //
 // The array is shared by every call on a device and keeps the previous call's
-// contents.  Nothing in it has to start at zero: the split kernel writes every
-// (split, row) record that the merge kernel then reads.  Two calls whose
-// kernels overlap on the GPU (different streams without ordering between them)
-// race on the array; callers must order such calls.
+// contents.  The partials need no clearing: the split kernel writes every
+// (split, row) record that the merge kernel then reads.  One record can be
+// missing only if a split kernel's bounded wait gives up; that sets a static
+// error word, which each call clears first (a 4-byte cudaMemsetAsync, no
+// allocation), and the merge then writes NaN instead of reading stale records.
+// Two calls whose kernels overlap on the GPU (different streams without
+// ordering between them) race on the array; callers must order such calls.
 #include <mutex>
 
 #include "../../include/kvs.h"
@@ -32,6 +35,8 @@ constexpr size_t kStaticFloats = kStaticAccFloats + (size_t)kStaticMaxSplits * k
 
 // 2 MiB + 32 KiB per device, held by every GPU that loads the library until exit
 static __device__ __align__(256) float g_static_scratch[kStaticFloats];
+// set by a split kernel whose bounded wait gave up; cleared at the start of each call
+static __device__ int g_static_err;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -40,6 +45,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 std::mutex g_mu;
 float* g_scratch_addr[64] = {};  // device address of g_static_scratch, per device
+int* g_err_addr[64] = {};        // device address of g_static_err, per device
 EncodeTiledFn g_encode = nullptr;
 
 int fail(int code, const char* msg) {
@@ -49,13 +55,17 @@ int fail(int code, const char* msg) {
 
 // Once per device, with that device current: look up the array's device address
 // (the host-side symbol is only a stand-in and must never reach a kernel).
-int setup(int dev, float** scratch) {
+int setup(int dev, float** scratch, int** err) {
     std::lock_guard<std::mutex> lock(g_mu);
     if (dev < 0 || dev >= 64) return fail(KVS_E_INVAL, "device index out of range");
     if (!g_scratch_addr[dev]) {
         void* p = nullptr;
+        void* pe = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
         if (e != cudaSuccess || !p) return fail(KVS_E_CUDA, "cudaGetSymbolAddress(scratch) failed");
+        e = cudaGetSymbolAddress(&pe, g_static_err);
+        if (e != cudaSuccess || !pe) return fail(KVS_E_CUDA, "cudaGetSymbolAddress(error word) failed");
+        g_err_addr[dev] = static_cast<int*>(pe);
         g_scratch_addr[dev] = static_cast<float*>(p);
     }
     if (!g_encode) {
@@ -67,6 +77,7 @@ int setup(int dev, float** scratch) {
         g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     }
     *scratch = g_scratch_addr[dev];
+    *err = g_err_addr[dev];
     return KVS_OK;
 }
 
@@ -84,12 +95,17 @@ extern "C" int kvs_attend_pages_static(const void* pages, int n_pages, int n_tok
         return fail(KVS_E_ORDER, "queries must lie inside the n_tokens history");
     if ((long)n_q * n_q_heads > kStaticMaxRows)
         return fail(KVS_E_WIDTH, "n_q * n_q_heads exceeds the static scratch maximum of 64 rows");
-    if ((reinterpret_cast<uintptr_t>(pages) & 15) || (reinterpret_cast<uintptr_t>(q_f16) & 1))
-        return fail(KVS_E_INVAL, "pages must be 16-byte aligned");
+    // the kernels' vector accesses: pages by TMA and 16-byte copies, Q in
+    // 8-byte words, out and lse as single floats
+    if (reinterpret_cast<uintptr_t>(pages) & 15) return fail(KVS_E_INVAL, "pages must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(q_f16) & 7) return fail(KVS_E_INVAL, "q must be 8-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(out) & 3) || (reinterpret_cast<uintptr_t>(lse) & 3))
+        return fail(KVS_E_INVAL, "out and lse must be 4-byte aligned");
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(KVS_E_CUDA, "cudaGetDevice failed");
     float* scratch = nullptr;
-    int rc = setup(dev, &scratch);
+    int* err = nullptr;
+    int rc = setup(dev, &scratch, &err);
     if (rc != KVS_OK) return rc;
 
     const int used_pages = (n_tokens + kPageTokens - 1) / kPageTokens;
@@ -130,9 +146,11 @@ extern "C" int kvs_attend_pages_static(const void* pages, int n_pages, int n_tok
     d.part.acc = scratch;
     d.part.ml = reinterpret_cast<float2*>(scratch + kStaticAccFloats);
     d.n_rows = rows;
-    d.err = nullptr;
+    d.err = err;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_decode(d, &kmap, n_splits, s);
+    cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), s);
+    if (e != cudaSuccess) return fail(KVS_E_CUDA, cudaGetErrorString(e));
+    e = launch_decode(d, &kmap, n_splits, s);
     if (e != cudaSuccess) return fail(KVS_E_CUDA, cudaGetErrorString(e));
     MergeArgs m;
     m.part = d.part;
@@ -140,6 +158,7 @@ extern "C" int kvs_attend_pages_static(const void* pages, int n_pages, int n_tok
     m.n_rows = rows;
     m.out = out;
     m.lse = lse;
+    m.err = err;
     e = launch_merge(m, s);
     if (e != cudaSuccess) return fail(KVS_E_CUDA, cudaGetErrorString(e));
     return KVS_OK;

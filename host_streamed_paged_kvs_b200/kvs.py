@@ -39,7 +39,8 @@ ERROR_NAMES = {0: "KVS_OK", -1: "KVS_E_INVAL", -2: "KVS_E_ARENA", -3: "KVS_E_WID
 # every symbol the header declares
 EXPORTS = ["kvs_resolve_config", "kvs_page_bytes", "kvs_plan_page", "kvs_create", "kvs_destroy",
            "kvs_append", "kvs_attend", "kvs_export_page", "kvs_page_location", "kvs_layer_length",
-           "kvs_get_config", "kvs_get_stats", "kvs_reset_stats", "kvs_set_profiling", "kvs_sync",
+           "kvs_get_config", "kvs_get_stats", "kvs_reset_stats", "kvs_set_profiling",
+           "kvs_set_zero_copy_pct", "kvs_sync",
            "kvs_measure_h2d", "kvs_attend_pages_static", "kvs_selftest_bounded_wait",
            "kvs_last_error", "kvs_eject_init", "kvs_eject_step", "kvs_draft_capacity_pages"]
 
@@ -105,6 +106,7 @@ def _load():
     L.kvs_get_stats.argtypes = [vp, cp(kvs_stats)]
     L.kvs_reset_stats.argtypes = [vp]
     L.kvs_set_profiling.argtypes = [vp, i]
+    L.kvs_set_zero_copy_pct.argtypes = [vp, i]
     L.kvs_sync.argtypes = [vp, vp, ctypes.c_double]
     L.kvs_measure_h2d.argtypes = [vp, ctypes.c_size_t, ctypes.c_size_t, i, cp(ctypes.c_double)]
     L.kvs_attend_pages_static.argtypes = [vp, i, i, i, i, i, i, vp, vp, vp, vp]
@@ -232,6 +234,10 @@ def kvs_reset_stats(h) -> None:
 
 def kvs_set_profiling(h, enable: bool) -> None:
     _check(lib.kvs_set_profiling(h, int(bool(enable))), h)
+
+
+def kvs_set_zero_copy_pct(h, pct: int) -> None:
+    _check(lib.kvs_set_zero_copy_pct(h, int(pct)), h)
 
 
 def kvs_sync(h, stream=None, timeout_s: float = 60.0) -> None:

@@ -94,7 +94,9 @@ WORKLOADS = {
                                          n_kv_heads=8, ctx=32768, n_resident_pages=64, n_ring_slots=8,
                                          seed=8, outlier_frac=0.01, outlier_scale=8.0, type_v=7),
 }
-DEFAULT_BENCH = "streamed_decode_32k"
+# The bench's default is the largest single-GPU decode configuration: 256K
+# context, where most of every step streams from host memory.
+DEFAULT_BENCH = "long_decode_256k"
 # Share (%) of a decode step's streamed pages that the decode kernel reads in
 # place from the mapped pinned history while the copy engine brings the rest
 # through the ring: in-place reads pay no per-copy cost, and the ring keeps

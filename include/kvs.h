@@ -219,7 +219,11 @@ int kvs_append(kvs_t* kv, int layer, int pos0, int n_tok, const void* k_f16,
  * [n_q][n_q_heads], natural log of sum(exp(q.k/sqrt(head_dim)))); lse may be
  * NULL.  Resident pages are attended in place; streamed pages are copied
  * through the ring on the library's copy stream and attended as they land;
- * per-split partials are merged by log-sum-exp. */
+ * per-split partials are merged by log-sum-exp.  Device buffers must suit the
+ * kernels' vector accesses (KVS_E_INVAL otherwise): q 8-byte aligned for
+ * decode widths (n_q * n_q_heads/n_kv_heads <= 8) and 16-byte aligned for
+ * wider calls; out 16-byte aligned when n_q * n_q_heads >= 1024, else 4-byte;
+ * lse 4-byte.  Host buffers have no alignment requirement. */
 int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float* out,
                float* lse, void* stream);
 
@@ -252,6 +256,13 @@ int kvs_get_config(kvs_t* kv, kvs_config* out);
 int kvs_get_stats(kvs_t* kv, kvs_stats* out);
 int kvs_reset_stats(kvs_t* kv);
 
+/* Change the in-place share of decode calls' streamed pages (kvs_config
+ * zero_copy_pct, 0..100) for later calls, e.g. to compare the copy-engine ring
+ * alone (0) with in-place reads alone (100) on one handle.  The split
+ * partials are sized for every share at kvs_create.  KVS_E_INVAL outside
+ * 0..100.  A CUDA graph captured earlier keeps the share it was captured with. */
+int kvs_set_zero_copy_pct(kvs_t* kv, int pct);
+
 /* Turn KVS_FLAG_PROFILE on (1) or off (0) for later calls. */
 int kvs_set_profiling(kvs_t* kv, int enable);
 
@@ -282,7 +293,9 @@ int kvs_measure_h2d(kvs_t* kv, size_t chunk_bytes, size_t total_bytes, int reps,
  * keys 0..n_tokens-1 are attended; query j sits at pos0+j and sees keys
  * 0..pos0+j; q fp16 [n_q][n_q_heads][128]; out fp32 [n_q][n_q_heads][128];
  * lse fp32 [n_q][n_q_heads] or NULL.  Limit: n_q * n_q_heads <= 64, else
- * KVS_E_WIDTH.  The first call on a device looks up the static array's device
+ * KVS_E_WIDTH.  Alignment (KVS_E_INVAL otherwise): pages 16 bytes, q 8 bytes,
+ * out and lse 4 bytes.  If a bounded wait inside the kernels gives up (the
+ * GPU stalled for over a second), out and lse come back as NaN.  The first call on a device looks up the static array's device
  * address (with that device current); make that first call before any stream
  * capture.  Every call shares the array, so calls whose kernels may overlap on
  * the GPU race: order them on one stream.  Stream ordered and asynchronous. */

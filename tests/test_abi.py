@@ -196,3 +196,24 @@ def test_create_without_gpu_fails_loudly(kvs):
     with pytest.raises(kvs.KvsError) as e:
         kvs.kvs_create(kvs.make_config(1, 8, 2, 1024), 0)
     assert e.value.code == kvs.KVS_E_CUDA
+
+
+def test_static_entry_rejects_misaligned_pointers_on_the_host(kvs):
+    """kvs_attend_pages_static checks its pointers before any CUDA call, so
+    these rejections need no GPU (the addresses are never dereferenced)."""
+    base = 1 << 20
+    cases = [
+        (base + 8, base, base, 0, "pages"),      # pages: TMA and 16-byte copies
+        (base, base + 4, base, 0, "8-byte"),     # q: 8-byte words
+        (base, base + 2, base, 0, "8-byte"),
+        (base, base, base + 2, 0, "4-byte"),     # out: floats
+        (base, base, base, base + 1, "4-byte"),  # lse: floats
+    ]
+    for pages, q, out, lse, what in cases:
+        rc = kvs.lib.kvs_attend_pages_static(pages, 4, 1000, 8, 2, 999, 1, q, out, lse or None, None)
+        assert rc == kvs.KVS_E_INVAL
+        assert what in kvs.kvs_last_error()
+
+
+def test_zero_copy_share_setter_range(kvs):
+    assert kvs.lib.kvs_set_zero_copy_pct(None, 10) == kvs.KVS_E_INVAL

@@ -94,3 +94,47 @@ def test_host_sync_timeout_then_recovers(kvs):
         kvs.kvs_sync(h, s, 60.0)
     finally:
         kvs.kvs_destroy(h)
+
+
+def test_misaligned_device_buffers_are_rejected_before_any_launch(kvs):
+    """Device Q/out/lse whose addresses the kernels' vector accesses cannot
+    take are refused on the host with KVS_E_INVAL; the handle stays usable."""
+    t = torch()
+    w = W.Workload("align", n_layers=1, n_q=1, n_q_heads=8, n_kv_heads=2, ctx=1000,
+                   n_resident_pages=2, n_ring_slots=2, seed=6)
+    # 160 q heads: a 7-token batch has 1120 rows, where the merge stores 16-byte words
+    cfg = kvs.make_config(1, 8, 2, 1000, n_resident_pages=2, n_ring_slots=2, max_q_tokens=8)
+    h = kvs.kvs_create(cfg, 0)
+    cfg2 = kvs.make_config(1, 160, 2, 1000, n_resident_pages=2, n_ring_slots=2, max_q_tokens=8)
+    h2 = kvs.kvs_create(cfg2, 0)
+    try:
+        prefill(h, w, 0, 999)
+        qbuf = t.zeros(8 * 8 * 128 + 64, dtype=t.float16, device="cuda")
+        obuf = t.zeros(8 * 8 * 128 + 64, dtype=t.float32, device="cuda")
+        q_ok, out_ok = qbuf.data_ptr(), obuf.data_ptr()
+
+        def rejected(pos0, n_q, q, out, lse=None, handle=h):
+            with pytest.raises(kvs.KvsError) as e:
+                kvs.kvs_attend(handle, 0, pos0, n_q, q, out, lse)
+            assert e.value.code == kvs.KVS_E_INVAL
+            return kvs.kvs_last_error(handle)
+
+        assert "8-byte" in rejected(998, 1, q_ok + 4, out_ok)     # decode reads Q in 8-byte words
+        assert "16-byte" in rejected(995, 4, q_ok + 8, out_ok)    # 16 rows: tensor-core path
+        assert "4-byte" in rejected(998, 1, q_ok, out_ok + 2)
+        assert "lse" in rejected(998, 1, q_ok, out_ok, obuf.data_ptr() + 2)
+        # the many-row merge writes out in 16-byte words
+        w2 = W.Workload("align2", n_layers=1, n_q=7, n_q_heads=160, n_kv_heads=2, ctx=1000,
+                        n_resident_pages=2, n_ring_slots=2, seed=6)
+        prefill(h2, w2, 0, 999)
+        q2 = t.zeros(7 * 160 * 128, dtype=t.float16, device="cuda")
+        o2 = t.zeros(7 * 160 * 128 + 16, dtype=t.float32, device="cuda")
+        assert "16-byte" in rejected(992, 7, q2, o2.data_ptr() + 4, handle=h2)
+        assert kvs.kvs_get_stats(h)["attends"] == 0 and kvs.kvs_get_stats(h2)["attends"] == 0
+        # still usable
+        out1, lse1 = step(h, w, 0, 999, 1)
+        assert_close(out1, lse1, *oracle_step(w, 0, 999, 1))
+        kvs.kvs_sync(h, None, 30.0)
+    finally:
+        kvs.kvs_destroy(h)
+        kvs.kvs_destroy(h2)
