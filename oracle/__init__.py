@@ -70,6 +70,13 @@ def bind(L):
     L.oracle_attention_t.restype = ctypes.c_int
     L.oracle_attention_t.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, u8p, u8p,
                                      ctypes.c_int, ctypes.c_int, u16p, f64p, f64p, ctypes.c_int]
+    L.oracle_quantize_rows_kv.restype = ctypes.c_int
+    L.oracle_quantize_rows_kv.argtypes = [ctypes.c_int, ctypes.c_int, u16p, u16p, u8p, u8p, ctypes.c_int,
+                                          ctypes.c_int]
+    L.oracle_attention_kv.restype = ctypes.c_int
+    L.oracle_attention_kv.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, u8p, u8p,
+                                      ctypes.c_int, ctypes.c_int, u16p, f64p, f64p, ctypes.c_int,
+                                      ctypes.c_int]
     L.oracle_pages_for.restype = ctypes.c_long
     L.oracle_pages_for.argtypes = [ctypes.c_long, ctypes.c_int]
     L.oracle_auto_resident_pages.restype = ctypes.c_long
@@ -198,18 +205,26 @@ V_Q5_0 = 6
 V_Q5_1 = 7
 V_Q8_0 = 8
 _V_BLOCK = {V_F16: 64, V_Q4_0: 18, V_Q4_1: 20, V_Q5_0: 22, V_Q5_1: 24, V_Q8_0: 34}
+K_F16 = 1
+K_Q8_0 = 8
+_K_BLOCK = {K_F16: 64, K_Q8_0: 34}
 
 
-def quantize_rows(k, v, v_type: int = V_Q4_0):
-    """k, v: fp16 [..., dim] -> (Q8_0 blocks [..., dim/32, 34], V blocks [..., dim/32, block bytes of v_type])."""
+def quantize_rows(k, v, v_type: int = V_Q4_0, k_type: int = K_Q8_0):
+    """k, v: fp16 [..., dim] -> (K blocks [..., dim/32, 34 (Q8_0) or 64 (F16)],
+    V blocks [..., dim/32, block bytes of v_type])."""
     k = _as_half_bits(k)
     v = _as_half_bits(v)
     assert k.shape == v.shape
     dim = k.shape[-1]
     rows = int(np.prod(k.shape[:-1]))
-    kb = np.zeros(k.shape[:-1] + (dim // 32, 34), np.uint8)
+    kb = np.zeros(k.shape[:-1] + (dim // 32, _K_BLOCK[k_type]), np.uint8)
     vb = np.zeros(k.shape[:-1] + (dim // 32, _V_BLOCK[v_type]), np.uint8)
-    if v_type == V_Q4_0:
+    if k_type != K_Q8_0:
+        rc = lib().oracle_quantize_rows_kv(rows, dim, _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16),
+                                           _ptr(kb, ctypes.c_uint8), _ptr(vb, ctypes.c_uint8), k_type, v_type)
+        assert rc == 0
+    elif v_type == V_Q4_0:
         lib().oracle_quantize_rows(rows, dim, _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16),
                                    _ptr(kb, ctypes.c_uint8), _ptr(vb, ctypes.c_uint8))
     else:
@@ -221,10 +236,12 @@ def quantize_rows(k, v, v_type: int = V_Q4_0):
 
 # --- attention ------------------------------------------------------------
 
-def attention(k_blocks: np.ndarray, v_blocks: np.ndarray, q, pos0: int, v_type: int = V_Q4_0):
+def attention(k_blocks: np.ndarray, v_blocks: np.ndarray, q, pos0: int, v_type: int = V_Q4_0,
+              k_type: int = K_Q8_0):
     """Exact attention over a quantized history.
 
-    k_blocks: uint8 [n_keys, n_kv, dim/32, 34]; v_blocks: uint8 [n_keys, n_kv, dim/32, 18]
+    k_blocks: uint8 [n_keys, n_kv, dim/32, 34] (Q8_0) or [..., 64] (k_type = K_F16);
+    v_blocks: uint8 [n_keys, n_kv, dim/32, 18]
     (Q4_0), or [..., 20 / 22 / 24 / 34 / 64] for v_type = V_Q4_1 / V_Q5_0 / V_Q5_1 / V_Q8_0 / V_F16
     q: fp16 [n_q, n_qh, dim]; query j sits at position pos0+j and sees keys 0..pos0+j.
     Returns (out float64 [n_q, n_qh, dim], lse float64 [n_q, n_qh]).
@@ -237,8 +254,13 @@ def attention(k_blocks: np.ndarray, v_blocks: np.ndarray, q, pos0: int, v_type: 
     vb = np.ascontiguousarray(v_blocks, dtype=np.uint8)
     out = np.zeros((n_q, n_qh, dim), np.float64)
     lse = np.zeros((n_q, n_qh), np.float64)
-    assert vb.shape[-1] == _V_BLOCK[v_type]
-    if v_type == V_Q4_0:
+    assert vb.shape[-1] == _V_BLOCK[v_type] and kb.shape[-1] == _K_BLOCK[k_type]
+    if k_type != K_Q8_0:
+        rc = lib().oracle_attention_kv(n_kv, n_qh, dim, _ptr(kb, ctypes.c_uint8),
+                                       _ptr(vb, ctypes.c_uint8), n_q, pos0,
+                                       _ptr(q, ctypes.c_uint16), _ptr(out, ctypes.c_double),
+                                       _ptr(lse, ctypes.c_double), k_type, v_type)
+    elif v_type == V_Q4_0:
         rc = lib().oracle_attention(n_kv, n_qh, dim, _ptr(kb, ctypes.c_uint8),
                                     _ptr(vb, ctypes.c_uint8), n_q, pos0,
                                     _ptr(q, ctypes.c_uint16), _ptr(out, ctypes.c_double),

@@ -340,22 +340,36 @@ static void v_dequant(int v_type, const uint8_t* blk, double* out) {
     else oracle_dequant_q8_0(blk, out);
 }
 
-/* K rows -> Q8_0 blocks; V rows -> blocks of the V type (1 F16, 2 Q4_0,
- * 3 Q4_1, 6 Q5_0, 7 Q5_1, 8 Q8_0) */
-int oracle_quantize_rows_t(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
-                           uint8_t* k_blocks, uint8_t* v_blocks, int v_type) {
+/* K types: Q8_0 (8, 34-byte blocks) or F16 (1, the 64-byte blocks of the
+ * values; "f16-f16 is always compiled" in the flash-attention build of "llama.cpp
+ * adaptive KV streaming - spec fork notes", TLDR) */
+static int k_block_bytes(int k_type) {
+    return k_type == 8 ? 34 : (k_type == 1 ? 64 : 0);
+}
+
+/* K rows -> blocks of the K type; V rows -> blocks of the V type (1 F16,
+ * 2 Q4_0, 3 Q4_1, 6 Q5_0, 7 Q5_1, 8 Q8_0) */
+int oracle_quantize_rows_kv(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
+                            uint8_t* k_blocks, uint8_t* v_blocks, int k_type, int v_type) {
     int nb = dim / 32;
+    int kbb = k_block_bytes(k_type);
     int vbb = v_block_bytes(v_type);
-    if (!vbb) return -1;
+    if (!vbb || !kbb) return -1;
     for (int r = 0; r < n_rows; ++r) {
         for (int b = 0; b < nb; ++b) {
             const uint16_t* kx = k + (size_t)r * dim + (size_t)b * 32;
             const uint16_t* vx = v + (size_t)r * dim + (size_t)b * 32;
-            oracle_q8_0_block(kx, k_blocks + ((size_t)r * nb + b) * 34);
+            if (k_type == 8) oracle_q8_0_block(kx, k_blocks + ((size_t)r * nb + b) * kbb);
+            else f16_block(kx, k_blocks + ((size_t)r * nb + b) * kbb);
             v_block(v_type, vx, v_blocks + ((size_t)r * nb + b) * vbb);
         }
     }
     return 0;
+}
+
+int oracle_quantize_rows_t(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
+                           uint8_t* k_blocks, uint8_t* v_blocks, int v_type) {
+    return oracle_quantize_rows_kv(n_rows, dim, k, v, k_blocks, v_blocks, 8, v_type);
 }
 
 void oracle_quantize_rows(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
@@ -375,11 +389,12 @@ void oracle_quantize_rows(int n_rows, int dim, const uint16_t* k, const uint16_t
 /*           exp(scaled logits).                                              */
 /* ------------------------------------------------------------------------ */
 
-int oracle_attention_t(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
-                       const uint8_t* v_blocks, int n_q, int pos0, const uint16_t* q,
-                       double* out, double* lse, int v_type) {
+int oracle_attention_kv(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
+                        const uint8_t* v_blocks, int n_q, int pos0, const uint16_t* q,
+                        double* out, double* lse, int k_type, int v_type) {
     int vbb = v_block_bytes(v_type);
-    if (n_kv <= 0 || n_qh % n_kv != 0 || dim % 32 != 0 || n_q <= 0 || pos0 < 0 || !vbb) return -1;
+    int kbb = k_block_bytes(k_type);
+    if (n_kv <= 0 || n_qh % n_kv != 0 || dim % 32 != 0 || n_q <= 0 || pos0 < 0 || !vbb || !kbb) return -1;
     int group = n_qh / n_kv;
     int nb = dim / 32;
     int max_keys = pos0 + n_q;
@@ -403,7 +418,9 @@ int oracle_attention_t(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
             for (int i = 0; i < n_keys; ++i) {
                 double acc = 0.0;
                 for (int b = 0; b < nb; ++b) {
-                    oracle_dequant_q8_0(k_blocks + (((size_t)i * n_kv + g) * nb + b) * 34, kd);
+                    const uint8_t* kblk = k_blocks + (((size_t)i * n_kv + g) * nb + b) * kbb;
+                    if (k_type == 8) oracle_dequant_q8_0(kblk, kd);
+                    else f16_dequant(kblk, kd);
                     for (int t = 0; t < 32; ++t) acc += qd[b * 32 + t] * kd[t];
                 }
                 s[i] = acc * scale;
@@ -428,6 +445,12 @@ int oracle_attention_t(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
     }
     free(s); free(qd); free(kd); free(vd);
     return 0;
+}
+
+int oracle_attention_t(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
+                       const uint8_t* v_blocks, int n_q, int pos0, const uint16_t* q,
+                       double* out, double* lse, int v_type) {
+    return oracle_attention_kv(n_kv, n_qh, dim, k_blocks, v_blocks, n_q, pos0, q, out, lse, 8, v_type);
 }
 
 int oracle_attention(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,

@@ -40,6 +40,14 @@ int oracle_attention_t(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
                        const uint8_t* v_blocks, int n_q, int pos0, const uint16_t* q,
                        double* out, double* lse, int v_type);
 
+/* the same with the K block type explicit as well: 8 = Q8_0 (34-byte blocks)
+ * or 1 = F16 (64-byte blocks of the values); -1 for any other */
+int oracle_quantize_rows_kv(int n_rows, int dim, const uint16_t* k, const uint16_t* v,
+                            uint8_t* k_blocks, uint8_t* v_blocks, int k_type, int v_type);
+int oracle_attention_kv(int n_kv, int n_qh, int dim, const uint8_t* k_blocks,
+                        const uint8_t* v_blocks, int n_q, int pos0, const uint16_t* q,
+                        double* out, double* lse, int k_type, int v_type);
+
 long oracle_pages_for(long n_tokens, int page_tokens);
 long oracle_auto_resident_pages(long max_ctx, int page_tokens, long page_bytes, int n_layers);
 int  oracle_page_location(long n_tokens, int page_tokens, long n_resident, long page,

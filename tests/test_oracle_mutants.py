@@ -17,6 +17,7 @@ import test_oracle_fp16 as TF
 import test_oracle_pages as TP
 import test_oracle_q5_0 as T5
 import test_oracle_q_min as TM
+import test_oracle_k_f16 as TK16
 import test_oracle_v_f16 as TV16
 import test_oracle_quant as TQ
 
@@ -66,6 +67,10 @@ MUTANTS = {
     "q1 reciprocal": ("int t = (int)((x[i] - lo) / d + 0.5f);", "int t = (int)((x[i] - lo) * (1.0f / d) + 0.5f);"),
     "q1 fp16 divisor": ("int t = (int)((x[i] - lo) / d + 0.5f);",
                         "int t = (int)((x[i] - lo) / oracle_half_to_float(*dh) + 0.5f);"),
+    "f16 K read as Q8_0": ("if (k_type == 8) oracle_dequant_q8_0(kblk, kd);\n                    else f16_dequant(kblk, kd);",
+                           "oracle_dequant_q8_0(kblk, kd);"),
+    "f16 K stored as Q8_0": ("else f16_block(kx, k_blocks + ((size_t)r * nb + b) * kbb);",
+                             "else oracle_q8_0_block(kx, k_blocks + ((size_t)r * nb + b) * kbb);"),
     "resident window": ("if (page >= P - n_resident) {", "if (page > P - n_resident) {"),
     "auto floor": ("long floor_pages = (2048 + page_tokens - 1) / page_tokens;",
                    "long floor_pages = (4096 + page_tokens - 1) / page_tokens;"),
@@ -89,6 +94,7 @@ def pins():
         lambda: TM.test_error_bound_and_range("q4_1"), lambda: TM.test_error_bound_and_range("q5_1"),
         lambda: TM.test_against_scipy_softmax_random("q5_1"),
         TV16.test_v_blocks_are_the_input_bits, TV16.test_against_scipy_over_exact_values,
+        TK16.test_k_blocks_are_the_input_bits, TK16.test_f16_f16_against_scipy_over_exact_values,
     ]
 
 
