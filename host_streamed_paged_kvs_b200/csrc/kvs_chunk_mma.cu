@@ -4,38 +4,42 @@
 // arena: speculative verify batches of 1 + n_draft tokens; 256-token ubatches
 // on "RaymondHuang210129/llama.cpp-adaptive-kv-streaming", Summary).
 //
-// CTA = (split, kv head, 128-row M tile of the head's n_q x G query rows),
-// 384 threads in three warp-specialized roles working on 64-key sub-stages,
-// handing work to each other only through mbarriers:
+// CTA = (split, kv head, pair of 128-row M tiles of the head's n_q x G query
+// rows): both tiles share every dequantized K/V sub-stage, so the producers'
+// work and the shared-memory operand traffic they cause are paid once per two
+// tiles, and the tensor cores alternate between the tiles' products while
+// each tile's softmax runs.  512 threads in three warp-specialized roles on
+// 64-key sub-stages, handing work to each other only through mbarriers:
 //
-//   softmax warps 0..3 (thread = query row = TMEM lane, whole 64-key rows)
-//     put the Q tile into tensor memory once, then per sub-stage read S,
-//     apply the causal mask and the 1/sqrt(128) scale in the log2 domain,
-//     keep a per-row reference max that only moves when the row max exceeds
-//     it by more than 2^8 (then rescale the row of O in TMEM), and write P in
-//     fp16 into one of two P buffers in tensor memory;
-//   producer warps 4..10
+//   softmax warps 0..3 (tile 0) and 4..7 (tile 1), thread = query row = TMEM
+//     lane, whole 64-key rows: put the tile's Q into tensor memory once, then
+//     per sub-stage read S, apply the causal mask and the 1/sqrt(128) scale in
+//     the log2 domain, keep a per-row reference max that only moves when the
+//     row max exceeds it by more than 2^8 (then rescale the row of O in TMEM),
+//     and write P in fp16 over the S columns just read;
+//   producer warps 8..14
 //     dequantize each 64-key half of a raw Q8_0/Q4_0 stage (128 keys, landed
 //     by TMA, two raw stages in flight) into fp16 UMMA operand tiles with the
 //     128-byte swizzle:
 //       K^ = d*q8 as [keys][dims] (K-major), split into hi = fp16(d*q8) and
 //       lo = fp16(d*q8 - hi) so the scores carry no fp16 rounding of K
-//       (two buffers, free again once the S MMAs that read them complete);
+//       (two buffers, free again once both tiles' S MMAs that read them
+//       complete);
 //       V^ = fp16(d*(q4-8)) as [keys][dims] (read as an MN-major B operand;
-//       three buffers, free again once the PV MMA that read them completes);
-//   MMA warp 11 (one elected lane)
+//       three buffers, free again once both tiles' PV MMAs complete);
+//   MMA warp 15 (one elected lane)
 //     polls the barriers without blocking and issues, whichever is ready
 //     first: the next raw TMA stage into a buffer the producers released;
-//     S = Q K^_hi^T + Q K^_lo^T (tcgen05.mma M=128 N=64 K=16, A = Q from
-//     tensor memory, fp32 accumulate into one of two TMEM S buffers) once a
-//     K^ buffer is full; and O += P V^ (M=128 N=128 K=16, A = P from tensor
-//     memory) once P and the V^ buffer are written.  Only the B operands
-//     (K^, V^) are read from shared memory.  Dequantization runs up to two
-//     sub-stages ahead of the softmax, the softmax one sub-stage ahead of the
-//     PV product, and the tensor-core work overlaps both.
+//     S_t = Q_t K^_hi^T + Q_t K^_lo^T (tcgen05.mma M=128 N=64 K=16, A = Q_t
+//     from tensor memory, fp32 accumulate) of tile t once the K^ buffer is
+//     full and the tile's previous PV product has completed (P_t lives in the
+//     S_t columns); and O_t += P_t V^ (M=128 N=128 K=16, A = P_t from tensor
+//     memory) once the softmax wrote P_t and V^ is written.  Only the B
+//     operands (K^, V^) are read from shared memory.
 //
-// Tensor memory (512 columns, one CTA per SM): S[2] at 0 and 64, O at 128,
-// P[2] (fp16 pairs) at 256 and 288, Q (fp16 pairs) at 320.
+// Tensor memory (512 columns, one CTA per SM), per tile t at 256 t: O_t (128
+// fp32 columns) at +0, S_t (64) at +128 with P_t (fp16 pairs, 32) over its
+// first half, Q_t (fp16 pairs, 64) at +192.
 // At the end O, m, l of every valid row are written as the split's partials
 // for the LSE merge.  No cluster, no multicast.
 #include <cuda_fp16.h>
@@ -49,10 +53,12 @@
 namespace kvs {
 namespace {
 
-constexpr int kSoftWarps = 4;
+constexpr int kTiles = 2;                                   // M tiles per CTA
+constexpr int kTileWarps = 4;                               // softmax warps per tile
+constexpr int kSoftWarps = kTiles * kTileWarps;             // 8
 constexpr int kProdWarps = 7;
-constexpr int kMmaWarp = kSoftWarps + kProdWarps;           // 11
-constexpr int kTcThreads = (kMmaWarp + 1) * 32;             // 384
+constexpr int kMmaWarp = kSoftWarps + kProdWarps;           // 15
+constexpr int kTcThreads = (kMmaWarp + 1) * 32;             // 512
 constexpr int kProdThreads = kProdWarps * 32;
 constexpr int kMTile = 128;
 constexpr int kRawKeys = 128;  // keys per raw (TMA) stage
@@ -64,10 +70,11 @@ constexpr int kKBufs = 2;
 constexpr int kVBufs = 3;
 constexpr int kKVBytes = kSubKeys * kHeadDim * 2;     // 16384: K^hi, K^lo or V^ [64][128] fp16
 // barriers: raw_full[2] raw_free[2] k_full[2] k_free[2] v_full[3] v_free[3]
-//           s_full[2] s_free[2] p_full[2] p_free[2]
-constexpr int kNumBars = 22;
+//           s_full[tile] p_full[tile] o_free[tile]
+constexpr int kNumBars = 14 + 3 * kTiles;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 128, kColP = 256, kColQ = 320;
+// columns within a tile's 256: O, S (P over its first 32 columns), Q
+constexpr uint32_t kTileCols = 256, kColO = 0, kColS = 128, kColQ = 192;
 static_assert(kKVBytes % 1024 == 0, "swizzled tiles need 1024-B alignment");
 
 // Raw-stage and shared-memory layout by V type.  Raw stage (128 keys, as the
@@ -77,15 +84,21 @@ static_assert(kKVBytes % 1024 == 0, "swizzled tiles need 1024-B alignment");
 // (8 B per key).  Shared memory: two raw
 // stages, then [2] x (K^hi | K^lo), [3] x V^, the barriers, the TMEM slot and
 // the abort flag (Q4_0 V: K^ @ 53248, V^ @ 118784, barriers @ 167936).
-template <int VT>
+// f16 K (the f16-f16 pair): the raw stage holds each key's values as two
+// 128-byte rows (dims 0..63, 64..127) and K^ needs no lo tile.
+template <int VT, int KT = kKQ8_0>
 struct TcGeom {
-    static constexpr int kRawVq = kRawKd + kRawKeys * kBlocks * 2;                    // 17408
-    static constexpr int kRawVh = kRawVq + kRawKeys * PageGeom<VT>::kVqRow;           // Q5_x fifth bits
-    static constexpr int kRawVd = kRawVh + kRawKeys * PageGeom<VT>::kVhRow;
-    static constexpr int kRawVm = kRawVd + kRawKeys * PageGeom<VT>::kVdRow;           // Q4_1 / Q5_1 minima
-    static constexpr int kRawBytes = kRawVm + kRawKeys * PageGeom<VT>::kVmRow;
+    using PG = PageGeom<VT, KT>;
+    static constexpr int kKRows = kRawKeys * PG::kKqRow / 128;                  // 128-byte K rows per raw stage
+    static constexpr int kRawKd = kRawKeys * PG::kKqRow;                         // 16384 for Q8_0 K
+    static constexpr int kRawVq = kRawKd + kRawKeys * PG::kKdRow;                // 17408 for Q8_0 K
+    static constexpr int kRawVh = kRawVq + kRawKeys * PG::kVqRow;                // Q5_x fifth bits
+    static constexpr int kRawVd = kRawVh + kRawKeys * PG::kVhRow;
+    static constexpr int kRawVm = kRawVd + kRawKeys * PG::kVdRow;                // Q4_1 / Q5_1 minima
+    static constexpr int kRawBytes = kRawVm + kRawKeys * PG::kVmRow;
+    static constexpr int kKHalves = KT == kKF16 ? 1 : 2;                         // K^ tiles per buffer
     static constexpr size_t kOffK = (size_t)kRawStages * kRawBytes;
-    static constexpr size_t kOffV = kOffK + kKBufs * 2 * kKVBytes;
+    static constexpr size_t kOffV = kOffK + kKBufs * kKHalves * kKVBytes;
     static constexpr size_t kOffBar = kOffV + kVBufs * kKVBytes;
     static constexpr size_t kOffTmem = kOffBar + kNumBars * 8;
     static constexpr size_t kOffAbort = kOffTmem + 4;
@@ -98,6 +111,7 @@ static_assert(TcGeom<kVQ4_0>::kOffBar == 167936, "Q4_0 geometry");
 static_assert(TcGeom<kVQ5_0>::kRawBytes == 28672, "Q5_0 raw stage");
 static_assert(TcGeom<kVQ4_1>::kRawBytes == 27648 && TcGeom<kVQ5_1>::kRawBytes == 29696, "Q4_1 / Q5_1 raw stages");
 static_assert(TcGeom<kVF16>::kRawBytes == 50176, "F16 raw stage");
+static_assert(TcGeom<kVF16, kKF16>::kRawBytes == 65536, "f16-f16 raw stage");
 
 // instruction descriptors: f16 x f16 -> f32, M = 128; A K-major;
 // S: N = 64, B K-major; PV: N = 128, B MN-major
@@ -179,11 +193,12 @@ __device__ __forceinline__ uint32_t fifth_bits(uint32_t hw, int j) {
 }
 
 
-template <int VT>
+template <int VT, int KT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     chunk_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap) {
-    using TG = TcGeom<VT>;
-    using PG = PageGeom<VT>;
+    using TG = TcGeom<VT, KT>;
+    using PG = PageGeom<VT, KT>;
+    constexpr int kRawKd = TG::kRawKd, kKHalves = TG::kKHalves;
     constexpr int kRawVq = TG::kRawVq, kRawVh = TG::kRawVh, kRawVd = TG::kRawVd, kRawBytes = TG::kRawBytes;
     constexpr int kRawVm = TG::kRawVm;
     constexpr size_t kOffK = TG::kOffK, kOffV = TG::kOffV, kOffBar = TG::kOffBar;
@@ -198,13 +213,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t* raw_full = bars + 0;   // [2] TMA bytes landed
     uint64_t* raw_free = bars + 2;   // [2] producers done reading a raw stage (7 warp arrivals)
     uint64_t* k_full = bars + 4;     // [2] producers wrote K^hi/K^lo (7 warp arrivals)
-    uint64_t* k_free = bars + 6;     // [2] S MMAs reading a K^ buffer complete
+    uint64_t* k_free = bars + 6;     // [2] both tiles' S MMAs reading a K^ buffer complete
     uint64_t* v_full = bars + 8;     // [3] producers wrote V^ (7 warp arrivals)
-    uint64_t* v_free = bars + 11;    // [3] PV MMA reading a V^ buffer complete
-    uint64_t* s_full = bars + 14;    // [2] S MMA complete
-    uint64_t* s_free = bars + 16;    // [2] softmax done reading S (4 warp arrivals)
-    uint64_t* p_full = bars + 18;    // [2] softmax wrote P into a TMEM P buffer (4 warp arrivals)
-    uint64_t* p_free = bars + 20;    // [2] PV MMA reading a P buffer complete
+    uint64_t* v_free = bars + 11;    // [3] both tiles' PV MMAs reading a V^ buffer complete
+    uint64_t* s_full = bars + 14;    // [tile] S_t MMA complete
+    uint64_t* p_full = bars + 14 + kTiles;      // [tile] softmax wrote P_t (4 warp arrivals)
+    uint64_t* o_free = bars + 14 + 2 * kTiles;  // [tile] PV_t MMA complete (P_t / S_t columns free)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmem);
     // set by a thread whose bounded wait gave up; everyone then skips the
     // remaining waits and work (there are no named barriers to leave behind)
@@ -213,6 +227,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.y;
     const int rows_head = a.n_q * a.group;
+    // tiles of this CTA: 2 z and 2 z + 1 (the second one only if it has rows)
+    const int n_tiles = ((2 * blockIdx.z + 1) * kMTile < rows_head) ? 2 : 1;
     const int raw0 = (int)(((long)blockIdx.x * 2 * a.n_units) / a.n_splits);  // first raw stage
     const int n_raw = (int)(((long)(blockIdx.x + 1) * 2 * a.n_units) / a.n_splits) - raw0;
     const int n_sub = 2 * n_raw;  // 64-key sub-stages
@@ -228,26 +244,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(&raw_free[k], kProdWarps);
             mbar_init(&k_full[k], kProdWarps);
             mbar_init(&k_free[k], 1);
-            mbar_init(&s_full[k], 1);
-            mbar_init(&s_free[k], kSoftWarps);
-            mbar_init(&p_full[k], kSoftWarps);
-            mbar_init(&p_free[k], 1);
         }
         for (int k = 0; k < kVBufs; ++k) {
             mbar_init(&v_full[k], kProdWarps);
             mbar_init(&v_free[k], 1);
+        }
+        for (int t = 0; t < kTiles; ++t) {
+            mbar_init(&s_full[t], 1);
+            mbar_init(&p_full[t], kTileWarps);
+            mbar_init(&o_free[t], 1);
         }
         fence_mbar_init();
     }
     __syncthreads();
     tc_fence_after();
     const uint32_t taddr = *tmem_slot;
-    if (warp < kSoftWarps) {
-        // Q tile into tensor memory: lane r = local query row mt*128 + r (rows
-        // past the head's rows are zero), dims 2c, 2c+1 in column kColQ + c
-        const int r = warp * 32 + lane;
-        const int lr = blockIdx.z * kMTile + r;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // softmax warps: tile of this warp, its first TMEM column, the warp's lanes
+    const int my_tile = warp / kTileWarps;
+    const uint32_t tcol = (uint32_t)my_tile * kTileCols;
+    const uint32_t lane_off = (uint32_t)((warp % kTileWarps) * 32) << 16;
+    if (warp < kSoftWarps && my_tile < n_tiles) {
+        // Q tile into tensor memory: lane r = local query row (2 z + t) 128 + r
+        // (rows past the head's rows are zero), dims 2c, 2c+1 in column Q + c
+        const int r = (warp % kTileWarps) * 32 + lane;
+        const int lr = (2 * blockIdx.z + my_tile) * kMTile + r;
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
             uint32_t qv[32];
@@ -261,7 +281,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 qv[4 * c] = v.x; qv[4 * c + 1] = v.y; qv[4 * c + 2] = v.z; qv[4 * c + 3] = v.w;
             }
-            tmem_st32u(taddr + lane_off + kColQ + half * 32, qv);
+            tmem_st32u(taddr + lane_off + tcol + kColQ + half * 32, qv);
         }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     }
@@ -286,9 +306,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 uint8_t* dst = raw + (r & 1) * kRawBytes;
                 uint64_t* b = &raw_full[r & 1];
                 mbar_expect_tx(b, kRawBytes);
-                const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * PG::kRows + half * kRawKeys;
-                tma_load_2d(dst + kRawKq, &kmap, 0, krow, b);
-                bulk_load(dst + kRawKd, ph + kOffKd + half * (kRawKeys * kBlocks * 2), kRawKeys * kBlocks * 2, b);
+                const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * PG::kRows + half * TG::kKRows;
+#pragma unroll
+                for (int kr = 0; kr < TG::kKRows; kr += 128)  // boxes of 128 rows of 128 B
+                    tma_load_2d(dst + kRawKq + kr * 128, &kmap, 0, krow + kr, b);
+                if constexpr (PG::kKdRow > 0)
+                    bulk_load(dst + kRawKd, ph + PG::kOffKd + half * (kRawKeys * PG::kKdRow), kRawKeys * PG::kKdRow, b);
                 bulk_load(dst + kRawVq, ph + PG::kOffVq + half * (kRawKeys * PG::kVqRow), kRawKeys * PG::kVqRow, b);
                 if constexpr (PG::kVhRow > 0)
                     bulk_load(dst + kRawVh, ph + PG::kOffVh + half * (kRawKeys * PG::kVhRow), kRawKeys * PG::kVhRow, b);
@@ -299,47 +322,66 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             };
             int ir = 0;        // next raw stage to load
             for (; ir < kRawStages && ir < n_raw; ++ir) issue_raw(ir);
-            int is = 0, ip = 0;  // next S and PV sub-stage to issue
+            // next S and PV sub-stage of tile 0 and tile 1 (an absent tile is always done)
+            int is0 = 0, ip0 = 0, is1 = 0, ip1 = 0;
+            if (n_tiles < kTiles) is1 = ip1 = n_sub;
+            // S_t(i) once K^(i) is written and PV_t(i - 1), which reads P_t
+            // from the S_t columns, has completed
+            auto try_s = [&](const int t, int& is_t, const int ip_t, const int is_other) {
+                const int i = is_t;
+                if (!(i < n_sub && ip_t == i && mbar_test(&k_full[i & 1], (i >> 1) & 1) &&
+                      (i == 0 || mbar_test(&o_free[t], (i - 1) & 1))))
+                    return false;
+                tc_fence_after();
+                const uint32_t aKh = smem_u32(sK + (i & 1) * kKHalves * kKVBytes), aKl = aKh + kKVBytes;
+                const uint32_t t_s = taddr + t * kTileCols + kColS;
+                const uint32_t t_q = taddr + t * kTileCols + kColQ;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc_mma_f16_ts(t_s, t_q + 8 * kk, desc_k(aKh, kSubKeys, kk), kIdescS, kk > 0);
+                if constexpr (KT == kKQ8_0) {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc_mma_f16_ts(t_s, t_q + 8 * kk, desc_k(aKl, kSubKeys, kk), kIdescS, 1u);
+                }
+                tc_commit(&s_full[t]);
+                is_t = i + 1;
+                // the K^ buffer is free once every tile's S(i) has completed
+                if (is_other > i) tc_commit(&k_free[i & 1]);
+                return true;
+            };
+            // O_t += P_t(i) V^(i) once the softmax wrote P_t(i) and V^(i) is written
+            auto try_pv = [&](const int t, int& ip_t, const int is_t, const int ip_other) {
+                const int i = ip_t;
+                if (!(i < is_t && mbar_test(&p_full[t], i & 1) && mbar_test(&v_full[i % kVBufs], (i / kVBufs) & 1)))
+                    return false;
+                tc_fence_after();
+                const uint32_t aV = smem_u32(sV + (i % kVBufs) * kKVBytes);
+                const uint32_t t_p = taddr + t * kTileCols + kColS;
+                const uint32_t t_o = taddr + t * kTileCols + kColO;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc_mma_f16_ts(t_o, t_p + 8 * kk, desc_mn(aV, kk), kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(&o_free[t]);
+                ip_t = i + 1;
+                // the V^ buffer is free once every tile's PV(i) has completed
+                if (ip_other > i) tc_commit(&v_free[i % kVBufs]);
+                return true;
+            };
             const uint64_t t0 = globaltimer_ns();
-            for (uint32_t spin = 0; ip < n_sub; ++spin) {
+            for (uint32_t spin = 0; ip0 < n_sub || ip1 < n_sub; ++spin) {
                 // raw stage ir reuses buffer ir & 1 once stage ir - 2 is dequantized
                 if (ir < n_raw && mbar_test(&raw_free[ir & 1], ((ir - 2) >> 1) & 1)) {
                     issue_raw(ir);
                     ++ir;
                 }
-                // S(is) into TMEM S buffer is & 1 once K^(is) is written and the
-                // softmax has read S(is - 2) out of that buffer
-                if (is < n_sub && mbar_test(&k_full[is & 1], (is >> 1) & 1) &&
-                    (is < 2 || mbar_test(&s_free[is & 1], ((is - 2) >> 1) & 1))) {
-                    tc_fence_after();
-                    const uint32_t aKh = smem_u32(sK + (is & 1) * 2 * kKVBytes), aKl = aKh + kKVBytes;
-                    const uint32_t t_s = taddr + kColS + (is & 1) * kSubKeys;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc_mma_f16_ts(t_s, taddr + kColQ + 8 * kk, desc_k(aKh, kSubKeys, kk), kIdescS, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc_mma_f16_ts(t_s, taddr + kColQ + 8 * kk, desc_k(aKl, kSubKeys, kk), kIdescS, 1u);
-                    tc_commit(&s_full[is & 1]);
-                    tc_commit(&k_free[is & 1]);
-                    ++is;
-                    continue;  // re-check the PV side with fresh state
+                // S products first, the tile that is behind first; then PV products
+                if (is1 < is0) {
+                    if (try_s(1, is1, ip1, is0) || try_s(0, is0, ip0, is1)) continue;
+                } else {
+                    if (try_s(0, is0, ip0, is1) || try_s(1, is1, ip1, is0)) continue;
                 }
-                // O += P(ip) V^(ip) once the softmax wrote P(ip) and V^(ip) is written
-                if (ip < is && mbar_test(&p_full[ip & 1], (ip >> 1) & 1) &&
-                    mbar_test(&v_full[ip % kVBufs], (ip / kVBufs) & 1)) {
-                    tc_fence_after();
-                    const uint32_t aV = smem_u32(sV + (ip % kVBufs) * kKVBytes);
-                    const uint32_t t_p = taddr + kColP + (ip & 1) * (kSubKeys / 2);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc_mma_f16_ts(taddr + kColO, t_p + 8 * kk, desc_mn(aV, kk), kIdescPV,
-                                      (ip > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(&p_free[ip & 1]);
-                    tc_commit(&v_free[ip % kVBufs]);
-                    ++ip;
-                    continue;
-                }
+                if (try_pv(0, ip0, is0, ip1) || try_pv(1, ip1, is1, ip0)) continue;
                 if ((spin & 255) == 255) {
                     if (*sAbort) { ok = false; break; }
                     if (globaltimer_ns() - t0 > kWaitLimitNs * 4) {
@@ -362,8 +404,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // ---- K^ hi / lo for keys [64 sub, 64 sub + 64) of the raw stage,
             //      once the S MMAs of sub-stage i - 2 released the buffer ----
             if (i >= 2 && fail_wait(&k_free[i & 1], ((i - 2) >> 1) & 1)) break;
-            uint8_t* sKh = sK + (i & 1) * 2 * kKVBytes;
+            uint8_t* sKh = sK + (i & 1) * kKHalves * kKVBytes;
             uint8_t* sKl = sKh + kKVBytes;
+            if constexpr (KT == kKF16) {
+                // f16 K: K^ is the stored values; 16 B of raw row 2 key + dims/64
+                // (swizzled by the TMA) to the operand tile's swizzled chunk
+                for (int un = ptid; un < kSubKeys * 16; un += kProdThreads) {
+                    const int kloc = un & 63, cc = un >> 6, hf = cc >> 3, c8 = cc & 7;
+                    const int row = 2 * (sub * kSubKeys + kloc) + hf;
+                    *reinterpret_cast<uint4*>(sKh + tile_off(kSubKeys, kloc, hf * 64 + 8 * c8)) =
+                        *reinterpret_cast<const uint4*>(rb + kRawKq + row * 128 + ((c8 ^ (row & 7)) << 4));
+                }
+            } else
             for (int un = ptid; un < kSubKeys * 8; un += kProdThreads) {
                 const int kloc = un & 63, g = un >> 6;  // key in the sub-stage, 16-dim chunk
                 const int key = sub * kSubKeys + kloc;   // key in the raw stage
@@ -482,41 +534,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (sub == 1) mbar_arrive_cta(&raw_free[r & 1]);
             }
         }
-    } else {
+    } else if (my_tile < n_tiles) {
         // ============================ softmax warps ============================
-        const int srow = warp * 32 + lane;  // TMEM lane = query row of the tile
-        const int lrow = blockIdx.z * kMTile + srow;
+        const int srow = (warp % kTileWarps) * 32 + lane;  // TMEM lane = query row of the tile
+        const int lrow = (2 * blockIdx.z + my_tile) * kMTile + srow;
         const bool row_valid = lrow < rows_head;
         const bool warp_active = __any_sync(0xffffffffu, row_valid);
         const int qpos = row_valid ? a.pos0 + lrow / a.group : -1;
         const int kend = min(a.len - 1, qpos);  // last visible key position of this row
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t t_s = taddr + tcol + kColS + lane_off, t_o = taddr + tcol + kColO + lane_off;
         float m_ref = -CUDART_INF_F, l_run = 0.0f;
         for (int i = 0; i < n_sub; ++i) {
-            const int b = i & 1;
-            const bool bad = fail_wait(&s_full[b], (i >> 1) & 1);
+            // S_t(i) is issued only after PV_t(i - 1) completed, so once it has
+            // landed O_t is stable and the S_t columns may take P_t(i)
+            const bool bad = fail_wait(&s_full[my_tile], i & 1);
             if (!__all_sync(0xffffffffu, !bad)) break;
             tc_fence_after();
             const int sg = raw0 + (i >> 1);
             const int kbase = (a.page0 + (sg >> 1)) * kPageTokens + (sg & 1) * kRawKeys + (i & 1) * kSubKeys;
             float v[64];
-            if (warp_active) tmem_ld64(taddr + kColS + b * kSubKeys + lane_off, v);
-            // S buffer b may be overwritten from here on
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cta(&s_free[b]);
+            if (warp_active) tmem_ld64(t_s, v);
+            // row max over the 64 keys as eight independent chains
             float mx = -CUDART_INF_F;
             if (warp_active) {
-                if (kbase + 63 <= kend) {
+                if (kbase + 63 > kend) {
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) mx = fmaxf(mx, v[e]);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 64; ++e) {
+                    for (int e = 0; e < 64; ++e)
                         if (kbase + e > kend) v[e] = -CUDART_INF_F;
-                        mx = fmaxf(mx, v[e]);
-                    }
                 }
+                float m8[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) m8[j] = v[j];
+#pragma unroll
+                for (int e = 8; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], v[e]);
+                mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                           fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
             }
             // keep the reference max unless the row's max grew by more than 2^8
             const float m_stage = mx * a.q_scale;
@@ -526,42 +578,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const float alpha = (m_use == m_ref) ? 1.0f : ex2_approx(m_ref - mu);
             m_ref = m_use;
             l_run *= alpha;
-            uint32_t pk[32];
             if (warp_active) {
+                uint32_t pk[32];
+                float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four independent partial sums
 #pragma unroll
                 for (int e = 0; e < 64; e += 2) {
                     const float p0 = ex2_approx(fmaf(v[e], a.q_scale, -mu));      // 2^-inf = 0
                     const float p1 = ex2_approx(fmaf(v[e + 1], a.q_scale, -mu));
-                    l_run += p0 + p1;
+                    l4[(e >> 1) & 3] += p0 + p1;
                     pk[e >> 1] = h2u(__floats2half2_rn(p0, p1));
                 }
-            }
-            // P buffer b is free once the PV MMA of sub-stage i-2 completed; a
-            // rescale of O also needs the PV of sub-stage i-1 complete
-            const bool resc = i > 0 && __any_sync(0xffffffffu, alpha != 1.0f);
-            bool bad2 = (i >= 2) && fail_wait(&p_free[b], ((i - 2) >> 1) & 1);
-            if (resc && !bad2) bad2 = fail_wait(&p_free[(i - 1) & 1], ((i - 1) >> 1) & 1);
-            if (!__all_sync(0xffffffffu, !bad2)) break;
-            tc_fence_after();
-            if (warp_active) {
-                if (resc) {
+                l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                tmem_st32u(t_s, pk);  // P_t over the first 32 S_t columns (waits for the store)
+                // rescale the row of O_t (stable: PV_t(i - 1) completed before S_t(i) was issued)
+                if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
                     float o[32];
 #pragma unroll 1
                     for (int c = 0; c < 4; ++c) {
-                        tmem_ld32(taddr + kColO + lane_off + c * 32, o);
+                        tmem_ld32(t_o + c * 32, o);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) o[e] *= alpha;
-                        tmem_st32(taddr + kColO + lane_off + c * 32, o);
+                        tmem_st32(t_o + c * 32, o);
                     }
                 }
-                tmem_st32u(taddr + kColP + b * (kSubKeys / 2) + lane_off, pk);  // waits for the store
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cta(&p_full[b]);
+            if (lane == 0) mbar_arrive_cta(&p_full[my_tile]);
         }
-        // ---- epilogue: wait for the last PV, write the split's partials ----
-        const bool bad3 = (n_sub > 0) && fail_wait(&p_free[(n_sub - 1) & 1], ((n_sub - 1) >> 1) & 1);
+        // ---- epilogue: wait for the tile's last PV, write the split's partials ----
+        const bool bad3 = (n_sub > 0) && fail_wait(&o_free[my_tile], (n_sub - 1) & 1);
         tc_fence_after();
         if (__all_sync(0xffffffffu, !bad3 && ok) && warp_active) {
             const int split_g = a.split_base + blockIdx.x;
@@ -570,7 +616,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 float o[32];
-                tmem_ld32(taddr + kColO + lane_off + c * 32, o);
+                tmem_ld32(t_o + c * 32, o);
                 if (n_sub == 0) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = 0.0f;
@@ -592,50 +638,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 }
 
-}  // namespace
-
-cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits, cudaStream_t s) {
+template <int VT, int KT = kKQ8_0>
+static cudaError_t launch_chunk_t(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits, cudaStream_t s) {
     // devices whose shared-memory opt-in is done (calls from several host
     // threads may race to set a bit; the attribute call is idempotent)
     static std::atomic<unsigned long long> configured{0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !(configured.load(std::memory_order_acquire) & (1ull << dev))) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ4_0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)TcGeom<kVQ4_0>::kSmem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ8_0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)TcGeom<kVQ8_0>::kSmem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ5_0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)TcGeom<kVQ5_0>::kSmem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ4_1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)TcGeom<kVQ4_1>::kSmem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(chunk_mma_kernel<kVQ5_1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)TcGeom<kVQ5_1>::kSmem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(chunk_mma_kernel<kVF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)TcGeom<kVF16>::kSmem);
+        const cudaError_t e = cudaFuncSetAttribute(chunk_mma_kernel<VT, KT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)TcGeom<VT, KT>::kSmem);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_acq_rel);
     }
     const int m_tiles = (a.n_q * a.group + kMTile - 1) / kMTile;
-    dim3 grid(n_splits, a.n_kv, m_tiles);
-    if (a.v_type == kVQ8_0)
-        chunk_mma_kernel<kVQ8_0><<<grid, kTcThreads, TcGeom<kVQ8_0>::kSmem, s>>>(a, *kmap);
-    else if (a.v_type == kVQ5_0)
-        chunk_mma_kernel<kVQ5_0><<<grid, kTcThreads, TcGeom<kVQ5_0>::kSmem, s>>>(a, *kmap);
-    else if (a.v_type == kVQ4_1)
-        chunk_mma_kernel<kVQ4_1><<<grid, kTcThreads, TcGeom<kVQ4_1>::kSmem, s>>>(a, *kmap);
-    else if (a.v_type == kVQ5_1)
-        chunk_mma_kernel<kVQ5_1><<<grid, kTcThreads, TcGeom<kVQ5_1>::kSmem, s>>>(a, *kmap);
-    else if (a.v_type == kVF16)
-        chunk_mma_kernel<kVF16><<<grid, kTcThreads, TcGeom<kVF16>::kSmem, s>>>(a, *kmap);
-    else
-        chunk_mma_kernel<kVQ4_0><<<grid, kTcThreads, TcGeom<kVQ4_0>::kSmem, s>>>(a, *kmap);
+    dim3 grid(n_splits, a.n_kv, (m_tiles + kTiles - 1) / kTiles);
+    chunk_mma_kernel<VT, KT><<<grid, kTcThreads, TcGeom<VT, KT>::kSmem, s>>>(a, *kmap);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits, cudaStream_t s) {
+    if (a.k_type == kKF16) return launch_chunk_t<kVF16, kKF16>(a, kmap, n_splits, s);
+    switch (a.v_type) {
+        case kVQ8_0: return launch_chunk_t<kVQ8_0>(a, kmap, n_splits, s);
+        case kVQ5_0: return launch_chunk_t<kVQ5_0>(a, kmap, n_splits, s);
+        case kVQ4_1: return launch_chunk_t<kVQ4_1>(a, kmap, n_splits, s);
+        case kVQ5_1: return launch_chunk_t<kVQ5_1>(a, kmap, n_splits, s);
+        case kVF16: return launch_chunk_t<kVF16>(a, kmap, n_splits, s);
+        default: return launch_chunk_t<kVQ4_0>(a, kmap, n_splits, s);
+    }
 }
 
 }  // namespace kvs

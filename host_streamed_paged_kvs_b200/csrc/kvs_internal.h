@@ -36,6 +36,10 @@ constexpr int kPageHeadBytes = kOffVd + kPageTokens * kBlocks * 2;  // 53248
 constexpr int kPageHeadRows = kPageHeadBytes / 128;     // 416 rows of 128 B
 static_assert(kPageHeadBytes == 53248, "page-head layout");
 
+// K type codes (the public KVS_TYPE_* values): Q8_0, or F16 (the f16-f16 pair)
+constexpr int kKF16 = 1;
+constexpr int kKQ8_0 = 8;
+
 // V type codes (the public KVS_TYPE_* values)
 constexpr int kVF16 = 1;
 constexpr int kVQ4_0 = 2;
@@ -61,16 +65,24 @@ __host__ __device__ constexpr bool v_a_is_p(int vt) { return v_has_min(vt) || vt
 //   Q5_1: Vq @ 34,816, Vh @ 51,200, Vd @ 55,296, Vm @ 57,344; 59,392 B.
 // F16 V stores the values, fp16 [256 tok][128 dims] @ 34,816, and no scales;
 // 100,352 B.
-template <int VT>
+// F16 K (only with F16 V: the f16-f16 pair) stores the K values the same way,
+// fp16 [256 tok][128 dims] @ 0, and no K scales; V then starts at 65,536 and
+// the page head is 131,072 B.
+template <int VT, int KT = kKQ8_0>
 struct PageGeom {
     static_assert(VT == kVF16 || VT == kVQ4_0 || VT == kVQ4_1 || VT == kVQ5_0 || VT == kVQ5_1 || VT == kVQ8_0,
                   "V type");
+    static_assert(KT == kKQ8_0 || (KT == kKF16 && VT == kVF16), "K/V type pair");
+    static constexpr int kKqRow = KT == kKF16 ? kHeadDim * 2 : kHeadDim;  // K bytes per token
+    static constexpr int kKdRow = KT == kKF16 ? 0 : kBlocks * 2;          // K scale bytes per token
+    static constexpr int kOffKq = 0;
+    static constexpr int kOffKd = kPageTokens * kKqRow;                    // 32768 for Q8_0 K
     static constexpr int kVqRow =                                           // V code bytes per token
         VT == kVQ8_0 ? kHeadDim : (VT == kVF16 ? kHeadDim * 2 : kHeadDim / 2);
     static constexpr int kVhRow = v_has_fifth(VT) ? kBlocks * 4 : 0;      // V fifth-bit bytes per token
     static constexpr int kVdRow = VT == kVF16 ? 0 : kBlocks * 2;          // V scale bytes per token
     static constexpr int kVmRow = v_has_min(VT) ? kBlocks * 2 : 0;        // V minimum bytes per token
-    static constexpr int kOffVq = kOffKd + kPageTokens * kBlocks * 2;       // 34816
+    static constexpr int kOffVq = kOffKd + kPageTokens * kKdRow;           // 34816 for Q8_0 K
     static constexpr int kOffVh = kOffVq + kPageTokens * kVqRow;
     static constexpr int kOffVd = kOffVh + kPageTokens * kVhRow;
     static constexpr int kOffVm = kOffVd + kPageTokens * kVdRow;
@@ -92,11 +104,14 @@ static_assert(PageGeom<kVQ4_1>::kHeadBytes == 55296 && PageGeom<kVQ4_1>::kOffVd 
                   PageGeom<kVQ4_1>::kOffVm == 53248 && PageGeom<kVQ4_1>::kHeadBytes % 128 == 0,
               "Q4_1 geometry");
 static_assert(PageGeom<kVF16>::kHeadBytes == 100352 && PageGeom<kVF16>::kHeadBytes % 128 == 0, "F16 geometry");
+static_assert(PageGeom<kVF16, kKF16>::kHeadBytes == 131072 && PageGeom<kVF16, kKF16>::kOffVq == 65536,
+              "F16-F16 geometry");
 static_assert(PageGeom<kVQ5_1>::kHeadBytes == 59392 && PageGeom<kVQ5_1>::kOffVh == 51200 &&
                   PageGeom<kVQ5_1>::kOffVd == 55296 && PageGeom<kVQ5_1>::kOffVm == 57344 &&
                   PageGeom<kVQ5_1>::kHeadBytes % 128 == 0,
               "Q5_1 geometry");
-inline int page_head_bytes(int v_type) {
+inline int page_head_bytes(int v_type, int k_type = kKQ8_0) {
+    if (k_type == kKF16) return PageGeom<kVF16, kKF16>::kHeadBytes;
     switch (v_type) {
         case kVQ8_0: return PageGeom<kVQ8_0>::kHeadBytes;
         case kVQ5_0: return PageGeom<kVQ5_0>::kHeadBytes;
@@ -109,6 +124,10 @@ inline int page_head_bytes(int v_type) {
 inline bool v_type_supported(int v_type) {
     return v_type == kVF16 || v_type == kVQ4_0 || v_type == kVQ4_1 || v_type == kVQ5_0 || v_type == kVQ5_1 ||
            v_type == kVQ8_0;
+}
+// the K/V pairs the kernels are built for: K Q8_0 with every V type, and f16-f16
+inline bool kv_pair_supported(int k_type, int v_type) {
+    return (k_type == kKQ8_0 && v_type_supported(v_type)) || (k_type == kKF16 && v_type == kVF16);
 }
 
 // split partials: per split and query row, (m, l) in the log2 domain + acc[128]
@@ -126,7 +145,8 @@ struct AppendArgs {
     int n_resident;          // R
     int first_resident_page; // pages >= this are resident after the append
     size_t page_bytes;
-    int v_type;              // kVQ4_0 or kVQ8_0
+    int v_type;              // V type (kV*)
+    int k_type;              // K type (kKQ8_0 or kKF16)
 };
 
 struct DecodeArgs {
@@ -148,7 +168,8 @@ struct DecodeArgs {
     PartialBuffers part;
     int n_rows;              // n_q * n_qh
     int* err;                // device error word (bounded waits)
-    int v_type;              // kVQ4_0 or kVQ8_0: the page-head geometry
+    int v_type;              // V type (kV*): with k_type, the page-head geometry
+    int k_type;              // K type (kKQ8_0 or kKF16)
 };
 
 // query rows from which the merge writes out with 16-byte stores

@@ -64,9 +64,9 @@ __device__ __forceinline__ uint32_t q8_0_lane(const float (&x)[4], float& d) {
     return w;
 }
 
-template <int VT>
+template <int VT, int KT = kKQ8_0>
 __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
-    using G = PageGeom<VT>;
+    using G = PageGeom<VT, KT>;
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
     if (row >= a.n_tok * a.n_kv) return;
@@ -119,10 +119,14 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
     }
 
     if constexpr (VT == kVF16) {
-        // ---- F16 (V): the values as they are ----
+        // ---- F16 (V): the values as they are; F16 K (the f16-f16 pair) likewise ----
         auto store = [&](uint8_t* ph) {
-            *reinterpret_cast<uint32_t*>(ph + kOffKq + t * kHeadDim + 4 * lane) = kq;
-            if (i == 0) *reinterpret_cast<__half*>(ph + kOffKd + t * 8 + 2 * b) = dk_h;
+            if constexpr (KT == kKF16) {
+                *reinterpret_cast<uint2*>(ph + G::kOffKq + t * G::kKqRow + 8 * lane) = kraw;
+            } else {
+                *reinterpret_cast<uint32_t*>(ph + kOffKq + t * kHeadDim + 4 * lane) = kq;
+                if (i == 0) *reinterpret_cast<__half*>(ph + kOffKd + t * 8 + 2 * b) = dk_h;
+            }
             *reinterpret_cast<uint2*>(ph + G::kOffVq + t * G::kVqRow + 8 * lane) = vraw;
         };
         store(a.host_layer + (size_t)page * a.page_bytes + (size_t)h * G::kHeadBytes);
@@ -244,7 +248,9 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
     const int rows = a.n_tok * a.n_kv;
-    if (a.v_type == kVQ8_0)
+    if (a.k_type == kKF16)
+        append_kernel<kVF16, kKF16><<<(rows + 3) / 4, 128, 0, s>>>(a);
+    else if (a.v_type == kVQ8_0)
         append_kernel<kVQ8_0><<<(rows + 3) / 4, 128, 0, s>>>(a);
     else if (a.v_type == kVQ5_0)
         append_kernel<kVQ5_0><<<(rows + 3) / 4, 128, 0, s>>>(a);
@@ -306,15 +312,20 @@ static_assert(kWarps * kMaxRows * (kHeadDim + 2) * 4 <= kStages * kStageBytes, "
 // V codes per key (34,816 B per stage) and an F16-V stage 256 B of values
 // (50,176 B), so they keep two stages in flight to stay at two CTAs per SM;
 // a Q5_0-V stage adds 16 B of fifth bits per key (28,672 B) and keeps three.
-template <int VT>
+// An f16-f16 stage carries 256 B of K values and 256 B of V values per key
+// (65,536 B): two stages, one CTA per SM.
+template <int VT, int KT = kKQ8_0>
 struct DecGeom {
-    static constexpr int kVqRow = PageGeom<VT>::kVqRow;
-    static constexpr int kVhRow = PageGeom<VT>::kVhRow;
-    static constexpr int kVmRow = PageGeom<VT>::kVmRow;
-    static constexpr int kStageVq = kStageKd + kStageKeys * kBlocks * 2;   // 17408
+    using PG = PageGeom<VT, KT>;
+    static constexpr int kVqRow = PG::kVqRow;
+    static constexpr int kVhRow = PG::kVhRow;
+    static constexpr int kVmRow = PG::kVmRow;
+    static constexpr int kKRows = kStageKeys * PG::kKqRow / 128;          // 128-byte K rows per stage
+    static constexpr int kStageKd = kStageKeys * PG::kKqRow;               // 16384 for Q8_0 K
+    static constexpr int kStageVq = kStageKd + kStageKeys * PG::kKdRow;   // 17408 for Q8_0 K
     static constexpr int kStageVh = kStageVq + kStageKeys * kVqRow;
     static constexpr int kStageVd = kStageVh + kStageKeys * kVhRow;
-    static constexpr int kStageVm = kStageVd + kStageKeys * PageGeom<VT>::kVdRow;
+    static constexpr int kStageVm = kStageVd + kStageKeys * PG::kVdRow;
     static constexpr int kStageBytes = kStageVm + kStageKeys * kVmRow;
     static constexpr int kStages = (VT == kVQ8_0 || VT == kVF16) ? 2 : 3;
     static constexpr size_t kOffQ = (size_t)kStages * kStageBytes;
@@ -335,6 +346,8 @@ static_assert(2 * DecGeom<kVQ5_1>::kSmem <= 232448 && DecGeom<kVQ5_1>::kStageByt
               "two Q5_1-V CTAs per SM");
 static_assert(2 * DecGeom<kVF16>::kSmem <= 232448 && DecGeom<kVF16>::kStageBytes == 50176,
               "two F16-V CTAs per SM");
+static_assert(DecGeom<kVF16, kKF16>::kSmem <= 232448 && DecGeom<kVF16, kKF16>::kStageBytes == 65536,
+              "one f16-f16 CTA per SM");
 
 size_t decode_smem_bytes() { return kDecodeSmem; }
 
@@ -375,13 +388,14 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 // history) by warp 0's 16-byte asynchronous copies instead of TMA, one stage
 // = 1664 copies, 52 per lane, the K quants placed in the same 128-byte
 // swizzle the tensor map produces
-template <int ROWS, bool ZC, int VT>
+template <int ROWS, bool ZC, int VT, int KT>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap) {
-    using G = DecGeom<VT>;
-    using PG = PageGeom<VT>;
+    using G = DecGeom<VT, KT>;
+    using PG = PageGeom<VT, KT>;
     constexpr int kStages = G::kStages;
     constexpr int kStageBytes = G::kStageBytes;
+    constexpr int kStageKd = G::kStageKd;
     constexpr int kStageVq = G::kStageVq;
     constexpr int kStageVh = G::kStageVh;
     constexpr int kStageVd = G::kStageVd;
@@ -441,18 +455,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         uint8_t* dst = stage + (i % kStages) * kStageBytes;
         uint64_t* b = &full[i % kStages];
         if constexpr (ZC) {
-            // K quants: row r of the half page, 16-byte chunk k -> swizzled
-            const uint8_t* kq = ph + kOffKq + half * (kStageKeys * kHeadDim);
+            // K quants (or f16 K values): 128-byte row r of the half page,
+            // 16-byte chunk k -> swizzled
+            const uint8_t* kq = ph + PG::kOffKq + half * (kStageKeys * PG::kKqRow);
 #pragma unroll 4
-            for (int c = lane; c < kStageKeys * 8; c += 32) {
+            for (int c = lane; c < G::kKRows * 8; c += 32) {
                 const int r = c >> 3, k = c & 7;
                 cp_async16(dst + kStageKq + r * 128 + ((k ^ (r & 7)) << 4), kq + r * 128 + k * 16);
             }
-            const uint8_t* kd = ph + kOffKd + half * (kStageKeys * kBlocks * 2);
+            const uint8_t* kd = ph + PG::kOffKd + half * (kStageKeys * PG::kKdRow);
             const uint8_t* vq = ph + PG::kOffVq + half * (kStageKeys * PG::kVqRow);
             const uint8_t* vd = ph + PG::kOffVd + half * (kStageKeys * kBlocks * 2);
             for (int c = lane; c < kStageKeys * kBlocks * 2 / 16; c += 32) {
-                cp_async16(dst + kStageKd + c * 16, kd + c * 16);
+                if constexpr (PG::kKdRow > 0) cp_async16(dst + kStageKd + c * 16, kd + c * 16);
                 if constexpr (PG::kVdRow > 0) cp_async16(dst + kStageVd + c * 16, vd + c * 16);
             }
 #pragma unroll 4
@@ -471,9 +486,12 @@ __global__ void __launch_bounds__(kThreads, 2)
             cp_async_arrive(b);
         } else {
             mbar_expect_tx(b, kStageBytes);
-            const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * PG::kRows + half * kStageKeys;
-            tma_load_2d(dst + kStageKq, &kmap, 0, krow, b);
-            bulk_load(dst + kStageKd, ph + kOffKd + half * (kStageKeys * kBlocks * 2), kStageKeys * kBlocks * 2, b);
+            const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * PG::kRows + half * G::kKRows;
+#pragma unroll
+            for (int kr = 0; kr < G::kKRows; kr += 128)  // boxes of 128 rows of 128 B
+                tma_load_2d(dst + kStageKq + kr * 128, &kmap, 0, krow + kr, b);
+            if constexpr (PG::kKdRow > 0)
+                bulk_load(dst + kStageKd, ph + PG::kOffKd + half * (kStageKeys * PG::kKdRow), kStageKeys * PG::kKdRow, b);
             bulk_load(dst + kStageVq, ph + PG::kOffVq + half * (kStageKeys * PG::kVqRow), kStageKeys * PG::kVqRow, b);
             if constexpr (PG::kVhRow > 0)
                 bulk_load(dst + kStageVh, ph + PG::kOffVh + half * (kStageKeys * PG::kVhRow), kStageKeys * PG::kVhRow, b);
@@ -548,6 +566,26 @@ __global__ void __launch_bounds__(kThreads, 2)
         // ---- QK^T ----
         float sc[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
         const uint8_t* kst = sb + kStageKq;
+        if constexpr (KT == kKF16) {
+            // f16 K: the stage holds each key as two 128-byte rows (dims 0..63,
+            // 64..127), row 2 key + dims/64, swizzled like the int8 rows; the
+            // lane's operand is the 8 values of dims 32 blk + 8q .. + 7, exact
+#pragma unroll 1
+            for (int blk = 0; blk < kBlocks; ++blk) {
+                const uint4 qb = qfrag[32 * blk];
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const int key = wkey + 8 * t + 2 * (g & 3) + (g >> 2);
+                    const int row = 2 * key + (blk >> 1), chunk = 4 * (blk & 1) + q;
+                    const uint4 w = *reinterpret_cast<const uint4*>(kst + row * 128 + ((chunk ^ (row & 7)) << 4));
+                    float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                    mma16816(c, qb.x, qb.y, w.x, w.y);
+                    mma16816(c, qb.z, qb.w, w.z, w.w);
+                    sc[t][0] += c[0];
+                    sc[t][1] += c[1];
+                }
+            }
+        } else
 #pragma unroll 1
         for (int blk = 0; blk < kBlocks; ++blk) {
             const uint4 qb = qfrag[32 * blk];  // k-steps 2 blk (x, y) and 2 blk + 1 (z, w)
@@ -739,7 +777,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-template <int ROWS, bool ZC, int VT>
+template <int ROWS, bool ZC, int VT, int KT>
 static cudaError_t launch_decode_t(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                                    int n_row_groups, cudaStream_t s) {
     // the shared-memory opt-in is per device: remember which devices have it
@@ -749,35 +787,36 @@ static cudaError_t launch_decode_t(const DecodeArgs& a, const CUtensorMap* kmap,
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !(configured.load(std::memory_order_acquire) & (1ull << dev))) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<ROWS, ZC, VT>,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<ROWS, ZC, VT, KT>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)DecGeom<VT>::kSmem);
+                                             (int)DecGeom<VT, KT>::kSmem);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_acq_rel);
     }
     dim3 grid(n_splits, a.n_kv, n_row_groups);
-    decode_kernel<ROWS, ZC, VT><<<grid, kThreads, DecGeom<VT>::kSmem, s>>>(a, *kmap);
+    decode_kernel<ROWS, ZC, VT, KT><<<grid, kThreads, DecGeom<VT, KT>::kSmem, s>>>(a, *kmap);
     return cudaGetLastError();
 }
 
-template <bool ZC, int VT>
+template <bool ZC, int VT, int KT = kKQ8_0>
 static cudaError_t launch_decode_rows(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                                       cudaStream_t s) {
     const int rows = a.n_q * a.group;
     switch (rows) {
-        case 1: return launch_decode_t<1, ZC, VT>(a, kmap, n_splits, 1, s);
-        case 2: return launch_decode_t<2, ZC, VT>(a, kmap, n_splits, 1, s);
-        case 3: return launch_decode_t<3, ZC, VT>(a, kmap, n_splits, 1, s);
-        case 4: return launch_decode_t<4, ZC, VT>(a, kmap, n_splits, 1, s);
-        case 5: return launch_decode_t<5, ZC, VT>(a, kmap, n_splits, 1, s);
-        case 6: return launch_decode_t<6, ZC, VT>(a, kmap, n_splits, 1, s);
-        case 7: return launch_decode_t<7, ZC, VT>(a, kmap, n_splits, 1, s);
-        default: return launch_decode_t<8, ZC, VT>(a, kmap, n_splits, (rows + 7) / 8, s);
+        case 1: return launch_decode_t<1, ZC, VT, KT>(a, kmap, n_splits, 1, s);
+        case 2: return launch_decode_t<2, ZC, VT, KT>(a, kmap, n_splits, 1, s);
+        case 3: return launch_decode_t<3, ZC, VT, KT>(a, kmap, n_splits, 1, s);
+        case 4: return launch_decode_t<4, ZC, VT, KT>(a, kmap, n_splits, 1, s);
+        case 5: return launch_decode_t<5, ZC, VT, KT>(a, kmap, n_splits, 1, s);
+        case 6: return launch_decode_t<6, ZC, VT, KT>(a, kmap, n_splits, 1, s);
+        case 7: return launch_decode_t<7, ZC, VT, KT>(a, kmap, n_splits, 1, s);
+        default: return launch_decode_t<8, ZC, VT, KT>(a, kmap, n_splits, (rows + 7) / 8, s);
     }
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                           cudaStream_t s) {
+    if (a.k_type == kKF16) return launch_decode_rows<false, kVF16, kKF16>(a, kmap, n_splits, s);
     if (a.v_type == kVQ8_0) return launch_decode_rows<false, kVQ8_0>(a, kmap, n_splits, s);
     if (a.v_type == kVQ5_0) return launch_decode_rows<false, kVQ5_0>(a, kmap, n_splits, s);
     if (a.v_type == kVQ4_1) return launch_decode_rows<false, kVQ4_1>(a, kmap, n_splits, s);
@@ -788,6 +827,7 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, int n_sp
 
 cudaError_t launch_decode_zero_copy(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                                     cudaStream_t s) {
+    if (a.k_type == kKF16) return launch_decode_rows<true, kVF16, kKF16>(a, kmap, n_splits, s);
     if (a.v_type == kVQ8_0) return launch_decode_rows<true, kVQ8_0>(a, kmap, n_splits, s);
     if (a.v_type == kVQ5_0) return launch_decode_rows<true, kVQ5_0>(a, kmap, n_splits, s);
     if (a.v_type == kVQ4_1) return launch_decode_rows<true, kVQ4_1>(a, kmap, n_splits, s);

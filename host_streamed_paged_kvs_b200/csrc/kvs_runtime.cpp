@@ -82,6 +82,8 @@ constexpr int kMaxDecodeRows = 8;
 bool use_tcgen05(const kvs_config& c, int n_q) { return n_q * (c.n_q_heads / c.n_kv_heads) > kMaxDecodeRows; }
 bool wide_regime(const kvs_config& c, int n_q) { return n_q * c.n_q_heads > kSmallRows; }
 int m_tiles(const kvs_config& c, int n_q) { return (n_q * (c.n_q_heads / c.n_kv_heads) + 127) / 128; }
+// CTAs per kv head and split of the tcgen05 kernel: one per pair of M tiles
+int tile_pairs(const kvs_config& c, int n_q) { return (m_tiles(c, n_q) + 1) / 2; }
 
 // tcgen05 path: splits sized for about one CTA per SM per ring chunk and
 // about two waves over the resident pages (the kernel holds one CTA per SM).
@@ -94,7 +96,7 @@ int res_splits(const kvs_config& c, long R_eff, int n_q) {
     if (use_tcgen05(c, n_q)) {
         // one CTA per SM: pick the split count that minimizes waves x stages
         // per split on a full machine (ties -> fewer splits, fewer partials)
-        const long units = (long)c.n_kv_heads * m_tiles(c, n_q);
+        const long units = (long)c.n_kv_heads * tile_pairs(c, n_q);
         long best = 1, best_cost = -1;
         for (long sp = 1; sp <= std::min(stages, 32L); ++sp) {
             const long cost = ((units * sp + kSms - 1) / kSms) * ((stages + sp - 1) / sp);
@@ -113,7 +115,7 @@ int ring_splits(const kvs_config& c, int n_q, int chunk_pages) {
     if (use_tcgen05(c, n_q)) {
         // at most one wave, leaving SMs to the resident launch when a chunk's
         // units cannot fill the machine twice
-        const int units = c.n_kv_heads * m_tiles(c, n_q);
+        const int units = c.n_kv_heads * tile_pairs(c, n_q);
         return std::min(stages, std::max(1, kSms / units));
     }
     return wide_regime(c, n_q) ? 1 : stages;
@@ -170,7 +172,7 @@ struct ArenaLayout {
 };
 
 ArenaLayout arena_layout(const kvs_config& c) {
-    const size_t pb = (size_t)c.n_kv_heads * page_head_bytes(c.type_v);
+    const size_t pb = (size_t)c.n_kv_heads * page_head_bytes(c.type_v, c.type_k);
     const size_t rows = (size_t)c.max_q_tokens * c.n_q_heads;
     const size_t recs = partial_records(c);
     ArenaLayout L{};
@@ -198,7 +200,7 @@ ArenaLayout arena_layout_with(kvs_config c, long resident_pages) {
 // fewer resident pages mean more streamed chunks and so more split partials,
 // so the counts are tried from P down.
 long resident_fit(const kvs_config& c, size_t budget, long P) {
-    const size_t per_page = (size_t)c.n_layers * c.n_kv_heads * page_head_bytes(c.type_v);
+    const size_t per_page = (size_t)c.n_layers * c.n_kv_heads * page_head_bytes(c.type_v, c.type_k);
     const long top = std::min<long>(std::max(1L, P), (long)(budget / per_page));  // resident bytes alone
     for (long r = top; r >= 1; --r)
         if (arena_layout_with(c, r).total <= budget) return r;
@@ -215,9 +217,9 @@ int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::stri
     }
     if (c.head_dim != kHeadDim) { why = fmt("head_dim %d unsupported (only 128)", c.head_dim); return KVS_E_INVAL; }
     if (c.page_tokens != kPageTokens) { why = fmt("page_tokens %d unsupported (only 256)", c.page_tokens); return KVS_E_INVAL; }
-    if (c.type_k != KVS_TYPE_Q8_0 || !v_type_supported(c.type_v)) {
+    if (!kv_pair_supported(c.type_k, c.type_v)) {
         why = "block KV streaming is not supported for this K/V cache type pair "
-              "(K=Q8_0 with V=F16, Q4_0, Q4_1, Q5_0, Q5_1 or Q8_0)";
+              "(K=Q8_0 with V=F16, Q4_0, Q4_1, Q5_0, Q5_1 or Q8_0; or K=F16 with V=F16)";
         return KVS_E_INVAL;
     }
     if (c.max_ctx < 1) { why = "max_ctx must be >= 1"; return KVS_E_INVAL; }
@@ -230,7 +232,7 @@ int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::stri
         why = fmt("zero_copy_pct %d outside 0..100", c.zero_copy_pct);
         return KVS_E_INVAL;
     }
-    const size_t pb = (size_t)c.n_kv_heads * page_head_bytes(c.type_v);
+    const size_t pb = (size_t)c.n_kv_heads * page_head_bytes(c.type_v, c.type_k);
     const long P = pages_for(c.max_ctx);
     if (c.n_ring_slots == 0) {
         c.chunk_pages = 0;
@@ -576,7 +578,7 @@ int kvs_resolve_config(const kvs_config* in, kvs_config* out, size_t* host_bytes
 }
 
 size_t kvs_page_bytes(const kvs_config* cfg) {
-    return cfg ? (size_t)cfg->n_kv_heads * page_head_bytes(cfg->type_v) : 0;
+    return cfg ? (size_t)cfg->n_kv_heads * page_head_bytes(cfg->type_v, cfg->type_k) : 0;
 }
 
 int kvs_plan_page(const kvs_config* c, int n_tokens, int page, int* kind, int* index) {
@@ -661,7 +663,7 @@ int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
     kvs_t* kv = new kvs_t();
     kv->cfg = c;
     kv->device = device;
-    kv->page_bytes = (size_t)c.n_kv_heads * page_head_bytes(c.type_v);
+    kv->page_bytes = (size_t)c.n_kv_heads * page_head_bytes(c.type_v, c.type_k);
     kv->P_max = pages_for(c.max_ctx);
     kv->host_bytes = host_bytes;
     kv->lay = arena_layout(c);
@@ -739,7 +741,7 @@ int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
     if (e != cudaSuccess || qr != cudaDriverEntryPointSuccess || !fn)
         return bail(KVS_E_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
     auto enc = reinterpret_cast<EncodeTiledFn>(fn);
-    const uint64_t head_rows = (uint64_t)page_head_bytes(c.type_v) / 128;
+    const uint64_t head_rows = (uint64_t)page_head_bytes(c.type_v, c.type_k) / 128;
     const uint64_t res_rows = (uint64_t)c.n_layers * c.n_resident_pages * c.n_kv_heads * head_rows;
     const uint64_t ring_rows = (uint64_t)c.n_ring_slots * c.n_kv_heads * head_rows;
     if (encode_map(kv, enc, &kv->map_res, kv->resident, res_rows) != KVS_OK) return bail(KVS_E_CUDA, kv->err);
@@ -841,6 +843,7 @@ int kvs_append(kvs_t* kv, int layer, int pos0, int n_tok, const void* k_f16, con
     a.first_resident_page = (int)f_new;
     a.page_bytes = kv->page_bytes;
     a.v_type = c.type_v;
+    a.k_type = c.type_k;
     {
         TimedScope ts(kv, s, kTAppend, 0);
         KVS_CK(kv, launch_append(a, s));
@@ -915,6 +918,7 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
 
     DecodeArgs d{};
     d.v_type = c.type_v;
+    d.k_type = c.type_k;
     d.len = ls.len;
     d.pos0 = pos0;
     d.n_q = n_q;
@@ -1112,17 +1116,24 @@ int kvs_export_page(kvs_t* kv, int layer, int page, int from_device, void* host_
 #undef KVS_V_FIELDS
     }
     const bool v8 = c.type_v == KVS_TYPE_Q8_0;
-    const int off_vq = PageGeom<kVQ4_0>::kOffVq;  // the same for every V type
-    const int phb = page_head_bytes(c.type_v);
+    const bool k16 = c.type_k == KVS_TYPE_F16;
+    // V fields follow K: 34,816 B in for Q8_0 K, 65,536 B for f16 K
+    const int off_vq = k16 ? PageGeom<kVF16, kKF16>::kOffVq : PageGeom<kVQ4_0>::kOffVq;
+    const int phb = page_head_bytes(c.type_v, c.type_k);
+    const int kblk = k16 ? 64 : 34;  // canonical K block: Q8_0, or the 32 fp16 values
     uint8_t* kout = out;
-    uint8_t* vout = out + (size_t)kPageTokens * H * kBlocks * 34;
+    uint8_t* vout = out + (size_t)kPageTokens * H * kBlocks * kblk;
     for (int t = 0; t < kPageTokens; ++t)
         for (int h = 0; h < H; ++h) {
             const uint8_t* ph = buf.data() + (size_t)h * phb;
             for (int b = 0; b < kBlocks; ++b) {
-                uint8_t* kb = kout + (((size_t)t * H + h) * kBlocks + b) * 34;
-                std::memcpy(kb, ph + kOffKd + t * 8 + b * 2, 2);
-                std::memcpy(kb + 2, ph + kOffKq + t * kHeadDim + b * 32, 32);
+                uint8_t* kb = kout + (((size_t)t * H + h) * kBlocks + b) * kblk;
+                if (k16) {
+                    std::memcpy(kb, ph + t * (kHeadDim * 2) + b * 64, 64);
+                } else {
+                    std::memcpy(kb, ph + kOffKd + t * 8 + b * 2, 2);
+                    std::memcpy(kb + 2, ph + kOffKq + t * kHeadDim + b * 32, 32);
+                }
                 uint8_t* vb = vout + (((size_t)t * H + h) * kBlocks + b) * vblk;
                 if (c.type_v == KVS_TYPE_F16) {  // the 32 values of the block
                     std::memcpy(vb, ph + off_vq + t * (kHeadDim * 2) + b * 64, 64);

@@ -50,7 +50,8 @@ extern "C" {
 #define KVS_E_TIMEOUT (-6) /* a bounded host wait gave up                         */
 #define KVS_E_NOMEM   (-7) /* host (pinned) allocation failed                     */
 
-/* ---- cache types: K is Q8_0; V is F16, Q4_0, Q4_1, Q5_0, Q5_1 or Q8_0 ------ */
+/* ---- cache types: K Q8_0 with V F16, Q4_0, Q4_1, Q5_0, Q5_1 or Q8_0; or the
+ *      f16-f16 pair (K and V both F16) ------------------------------------- */
 #define KVS_TYPE_F16  1
 #define KVS_TYPE_Q4_0 2
 #define KVS_TYPE_Q4_1 3
@@ -83,7 +84,11 @@ typedef struct kvs_config {
     int n_ring_slots;     /* device ring slots (pages); 0 = all-resident mode, which needs
                              n_resident_pages >= pages(max_ctx) */
     int max_q_tokens;     /* widest append / attend batch (1, 1+n_draft or a 256-token ubatch) */
-    int type_k;           /* must be KVS_TYPE_Q8_0 */
+    int type_k;           /* KVS_TYPE_Q8_0, or KVS_TYPE_F16 together with type_v = KVS_TYPE_F16:
+                             the f16-f16 pair, which the flash-attention build always compiles
+                             ("llama.cpp adaptive KV streaming - spec fork notes", TLDR); its
+                             page head is 131,072 B (K values fp16 [256 tok][128 dims], then V
+                             values the same way, no scales) */
     int type_v;           /* KVS_TYPE_Q4_0 (page head 53,248 B), KVS_TYPE_Q8_0 (69,632 B: V codes
                              stored like K's; the q8_0/q8_0 pair of the "Feature/adaptive kv
                              stream integration" pull request's runs), or one of the other
@@ -237,7 +242,8 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
  * (fp16 d, a little-endian word whose bit j is bit 4 of q_j, then 16 bytes
  * holding the low 4 bits as Q4_0 does); Q4_1 (20 bytes) and Q5_1 (24 bytes)
  * blocks put the fp16 block minimum m right after d; F16 blocks are the 32
- * fp16 values (64 bytes).  from_device = 0 reads the host history,
+ * fp16 values (64 bytes); with type_k = KVS_TYPE_F16 the K blocks are the 32
+ * fp16 values too (64 bytes).  from_device = 0 reads the host history,
  * 1 reads the resident slot (KVS_E_INVAL if the page is not resident).  The
  * caller must have synchronized the streams that wrote the page. */
 int kvs_export_page(kvs_t* kv, int layer, int page, int from_device, void* host_dst);

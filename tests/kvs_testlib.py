@@ -59,16 +59,18 @@ def step(h, w: W.Workload, layer: int, pos0: int, n_q: int, stream=None):
     return out.cpu().numpy(), lse.cpu().numpy()
 
 
-def oracle_blocks(w: W.Workload, layer: int, upto: int, v_type: int = oracle.V_Q4_0):
+def oracle_blocks(w: W.Workload, layer: int, upto: int, v_type: int = oracle.V_Q4_0,
+                  k_type: int = oracle.K_Q8_0):
     k, v = W.kv_tokens(w, layer, 0, upto)
-    return oracle.quantize_rows(k, v, v_type)
+    return oracle.quantize_rows(k, v, v_type, k_type)
 
 
-def oracle_step(w: W.Workload, layer: int, pos0: int, n_q: int, rows=None, v_type: int = oracle.V_Q4_0):
+def oracle_step(w: W.Workload, layer: int, pos0: int, n_q: int, rows=None, v_type: int = oracle.V_Q4_0,
+                k_type: int = oracle.K_Q8_0):
     """Oracle out/lse for the step's queries over the layer's history [0, pos0+n_q)."""
-    kb, vb = oracle_blocks(w, layer, pos0 + n_q, v_type)
+    kb, vb = oracle_blocks(w, layer, pos0 + n_q, v_type, k_type)
     q = W.queries(w, layer, pos0, n_q)
-    return oracle.attention(kb, vb, q, pos0, v_type)
+    return oracle.attention(kb, vb, q, pos0, v_type, k_type)
 
 
 def assert_close(out, lse, ref_out, ref_lse):
@@ -86,10 +88,11 @@ def export_page(h, cfg, layer, page, from_device):
     H = cfg.n_kv_heads
     vbytes = {kvs.KVS_TYPE_Q8_0: 34, kvs.KVS_TYPE_Q5_0: 22, kvs.KVS_TYPE_Q4_1: 20,
               kvs.KVS_TYPE_Q5_1: 24, kvs.KVS_TYPE_F16: 64}.get(cfg.type_v, 18)
-    nk = T * H * 4 * 34
+    kbytes = 64 if cfg.type_k == kvs.KVS_TYPE_F16 else 34
+    nk = T * H * 4 * kbytes
     nv = T * H * 4 * vbytes
     buf = np.zeros(nk + nv, np.uint8)
     kvs.kvs_export_page(h, layer, page, from_device, buf)
-    kb = buf[:nk].reshape(T, H, 4, 34)
+    kb = buf[:nk].reshape(T, H, 4, kbytes)
     vb = buf[nk:].reshape(T, H, 4, vbytes)
     return kb, vb

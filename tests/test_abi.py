@@ -89,7 +89,7 @@ def test_plan_page_matches_oracle(kvs):
 
 @pytest.mark.parametrize("over,code", [
     (dict(type_k=2), -1), (dict(type_v=0), -1), (dict(type_k=8, type_v=4), -1), (dict(type_v=5), -1),
-    (dict(type_k=1, type_v=1), -1),
+    (dict(type_k=1, type_v=2), -1), (dict(type_k=1, type_v=8), -1),
     (dict(type_v=9), -1),
     (dict(type_k=6, type_v=6), -1), (dict(head_dim=64), -1), (dict(page_tokens=128), -1),
     (dict(n_q_heads=12, n_kv_heads=8), -1), (dict(n_ring_slots=0, n_resident_pages=4), -1),
@@ -217,3 +217,21 @@ def test_static_entry_rejects_misaligned_pointers_on_the_host(kvs):
 
 def test_zero_copy_share_setter_range(kvs):
     assert kvs.lib.kvs_set_zero_copy_pct(None, 10) == kvs.KVS_E_INVAL
+
+
+def test_f16_f16_pair_geometry_and_gates(kvs):
+    """The f16-f16 pair: K and V both stored as fp16 values, 131,072 B per page
+    head; F16 K with any other V type is rejected."""
+    c = kvs.make_config(2, 32, 8, 32768, n_resident_pages=8, n_ring_slots=8,
+                        type_k=kvs.KVS_TYPE_F16, type_v=kvs.KVS_TYPE_F16)
+    r, host = kvs.kvs_resolve_config(c)
+    assert (r.type_k, r.type_v) == (kvs.KVS_TYPE_F16, kvs.KVS_TYPE_F16)
+    assert kvs.kvs_page_bytes(r) == 8 * 131072
+    assert host == 2 * 128 * 8 * 131072
+    for tv in (kvs.KVS_TYPE_Q4_0, kvs.KVS_TYPE_Q8_0, kvs.KVS_TYPE_Q5_1):
+        bad = kvs.make_config(2, 32, 8, 32768, n_resident_pages=8, n_ring_slots=8,
+                              type_k=kvs.KVS_TYPE_F16, type_v=tv)
+        with pytest.raises(kvs.KvsError) as e:
+            kvs.kvs_resolve_config(bad)
+        assert e.value.code == kvs.KVS_E_INVAL
+        assert "pair" in kvs.kvs_last_error()

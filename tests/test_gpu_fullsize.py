@@ -69,4 +69,7 @@ def test_verify_128k_full_aux_layer(kvs):
 
 
 def test_prefill_chunk_64k_sampled(kvs):
-    _full(kvs, "prefill_chunk_64k", layers=[0], sample_q=[0, 1, 100, 255])
+    # one query token in each of the ten 128-row M tiles (5 rows per token):
+    # token j owns rows 5j..5j+4, so these tokens fall in tiles 0, 1, ..., 9
+    _full(kvs, "prefill_chunk_64k", layers=[0],
+          sample_q=[0, 26, 52, 77, 103, 128, 154, 180, 205, 231, 255])
