@@ -613,6 +613,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int split_g = a.split_base + blockIdx.x;
             const int j = lrow / a.group, g = lrow - j * a.group;
             const int grow = j * a.n_qh + h * a.group + g;
+            // accumulate: fold in the record the previous launch left for this
+            // (split, row): with M = max of the two reference maxima, O and l
+            // are the 2^(m - M)-weighted sums (a record with l = 0 counts as empty)
+            float w_new = 1.0f, w_old = 0.0f, m_out = m_ref, l_out = l_run;
+            float2 prev = make_float2(-CUDART_INF_F, 0.0f);
+            if (a.accumulate && row_valid) prev = a.part.ml[(size_t)split_g * a.n_rows + grow];
+            if (prev.y > 0.0f) {
+                if (l_run > 0.0f) {
+                    m_out = fmaxf(prev.x, m_ref);
+                    w_old = ex2_approx(prev.x - m_out);
+                    w_new = ex2_approx(m_ref - m_out);
+                } else {
+                    m_out = prev.x;
+                    w_old = 1.0f;
+                    w_new = 0.0f;
+                }
+                l_out = w_old * prev.y + w_new * l_run;
+            }
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 float o[32];
@@ -624,10 +642,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (row_valid) {
                     float* dst = a.part.acc + ((size_t)split_g * a.n_rows + grow) * kHeadDim + c * 32;
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+                    for (int e = 0; e < 32; e += 4) {
+                        float4 v = make_float4(o[e] * w_new, o[e + 1] * w_new, o[e + 2] * w_new, o[e + 3] * w_new);
+                        if (w_old != 0.0f) {
+                            const float4 pv = *reinterpret_cast<const float4*>(dst + e);
+                            v.x = fmaf(w_old, pv.x, v.x); v.y = fmaf(w_old, pv.y, v.y);
+                            v.z = fmaf(w_old, pv.z, v.z); v.w = fmaf(w_old, pv.w, v.w);
+                        }
+                        *reinterpret_cast<float4*>(dst + e) = v;
+                    }
                 }
             }
-            if (row_valid) a.part.ml[(size_t)split_g * a.n_rows + grow] = make_float2(m_ref, l_run);
+            if (row_valid) a.part.ml[(size_t)split_g * a.n_rows + grow] = make_float2(m_out, l_out);
         }
     }
     tc_fence_before();

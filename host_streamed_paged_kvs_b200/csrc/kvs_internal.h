@@ -159,6 +159,9 @@ struct DecodeArgs {
     int n_splits;            // splits of this launch; split s covers half-page stages
                              // [s*T/n_splits, (s+1)*T/n_splits) of the T = 2*n_units stages
     int split_base;          // first split index written by this launch
+    int accumulate;          // tensor-core kernel: 1 = merge this launch's partials into the
+                             // records already at split_base.. (the same stream's previous
+                             // launch wrote them) instead of overwriting them
     int len;                 // tokens in the history
     int pos0, n_q;           // query positions pos0 .. pos0+n_q-1
     const __half* q;         // [n_q][n_qh][128]

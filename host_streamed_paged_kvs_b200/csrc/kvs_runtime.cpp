@@ -140,8 +140,14 @@ long count_splits(const kvs_config& c, int n_q, long R_eff, long S) {
     if (S_zc > 0) n += zc_splits(c, S_zc, n_q);
     if (S_ring > 0 && c.chunk_pages > 0) {
         const long full = S_ring / c.chunk_pages, tail = S_ring % c.chunk_pages;
-        n += full * ring_splits(c, n_q, c.chunk_pages);
-        if (tail) n += ring_splits(c, n_q, (int)tail);
+        if (use_tcgen05(c, n_q)) {
+            // the tensor-core ring launches merge into one set of records (the
+            // first chunk, the widest, writes them; later chunks accumulate)
+            n += ring_splits(c, n_q, full > 0 ? c.chunk_pages : (int)tail);
+        } else {
+            n += full * ring_splits(c, n_q, c.chunk_pages);
+            if (tail) n += ring_splits(c, n_q, (int)tail);
+        }
     }
     return n;
 }
@@ -150,9 +156,9 @@ long count_splits(const kvs_config& c, int n_q, long R_eff, long S) {
 // over every query width the handle accepts, at the longest history (split
 // counts only grow with the number of resident and streamed pages), and over
 // every in-place share, so that kvs_set_zero_copy_pct can change it later
-size_t partial_records(const kvs_config& c) {
+size_t partial_records_r(const kvs_config& c, long R) {
     const long P = pages_for(c.max_ctx);
-    const long R_eff = std::min<long>(c.n_resident_pages, P);
+    const long R_eff = std::min<long>(R, P);
     const long S = c.n_ring_slots > 0 ? P - R_eff : 0;
     size_t best = 1;
     for (int n_q = 1; n_q <= c.max_q_tokens; ++n_q) {
@@ -166,7 +172,24 @@ size_t partial_records(const kvs_config& c) {
     }
     return best;
 }
+// over the target layers' and the auxiliary layers' resident counts
+size_t partial_records(const kvs_config& c) {
+    size_t n = partial_records_r(c, c.n_resident_pages);
+    if (c.n_aux_layers > 0) n = std::max(n, partial_records_r(c, std::max(1, c.aux_resident_pages)));
+    return n;
+}
 
+// the layers whose resident pages sit in the main resident region
+int target_layers(const kvs_config& c) { return c.n_layers - c.n_aux_layers; }
+
+// bytes of the auxiliary layers' resident pages (pinned at the arena top)
+size_t aux_region_bytes(const kvs_config& c) {
+    const size_t pb = (size_t)c.n_kv_heads * page_head_bytes(c.type_v, c.type_k);
+    return align_up((size_t)c.n_aux_layers * c.aux_resident_pages * pb, 1024);
+}
+
+// Layout of the arena's lower part: resident pages of the target layers, ring,
+// split partials and staging for the widest batch (max_q_tokens), error word.
 struct ArenaLayout {
     size_t resident, ring, part_ml, part_acc, stage_q, stage_kv, stage_out, stage_lse, err, total;
 };
@@ -177,7 +200,7 @@ ArenaLayout arena_layout(const kvs_config& c) {
     const size_t recs = partial_records(c);
     ArenaLayout L{};
     size_t off = 0;
-    L.resident = off; off = align_up(off + (size_t)c.n_layers * c.n_resident_pages * pb, 1024);
+    L.resident = off; off = align_up(off + (size_t)target_layers(c) * c.n_resident_pages * pb, 1024);
     L.ring = off;     off = align_up(off + (size_t)c.n_ring_slots * pb, 1024);
     L.part_ml = off;  off = align_up(off + recs * sizeof(float2));
     L.part_acc = off; off = align_up(off + recs * kHeadDim * sizeof(float));
@@ -200,7 +223,7 @@ ArenaLayout arena_layout_with(kvs_config c, long resident_pages) {
 // fewer resident pages mean more streamed chunks and so more split partials,
 // so the counts are tried from P down.
 long resident_fit(const kvs_config& c, size_t budget, long P) {
-    const size_t per_page = (size_t)c.n_layers * c.n_kv_heads * page_head_bytes(c.type_v, c.type_k);
+    const size_t per_page = (size_t)target_layers(c) * c.n_kv_heads * page_head_bytes(c.type_v, c.type_k);
     const long top = std::min<long>(std::max(1L, P), (long)(budget / per_page));  // resident bytes alone
     for (long r = top; r >= 1; --r)
         if (arena_layout_with(c, r).total <= budget) return r;
@@ -232,6 +255,18 @@ int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::stri
         why = fmt("zero_copy_pct %d outside 0..100", c.zero_copy_pct);
         return KVS_E_INVAL;
     }
+    // a phase arena: a fixed budget with the resident set fitted to it (a
+    // resolved phase-arena config carries the flag and is re-fitted)
+    const bool phase = c.arena_bytes != 0 && (c.n_resident_pages == 0 || (c.flags & KVS_FLAG_PHASE_ARENA));
+    if (phase) c.n_resident_pages = 0;
+    if (c.n_aux_layers < 0 || c.n_aux_layers >= c.n_layers || c.aux_resident_pages < 0) {
+        why = fmt("n_aux_layers (%d) must be in [0, n_layers) and aux_resident_pages >= 0", c.n_aux_layers);
+        return KVS_E_INVAL;
+    }
+    if ((c.n_aux_layers > 0 || c.aux_resident_pages > 0) && !phase) {
+        why = "auxiliary layers need a phase arena (arena_bytes with n_resident_pages = 0)";
+        return KVS_E_INVAL;
+    }
     const size_t pb = (size_t)c.n_kv_heads * page_head_bytes(c.type_v, c.type_k);
     const long P = pages_for(c.max_ctx);
     if (c.n_ring_slots == 0) {
@@ -247,16 +282,24 @@ int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::stri
         why = fmt("arena %zu B is below the minimum stage of one page (%zu B)", c.arena_bytes, pb);
         return KVS_E_ARENA;
     }
+    size_t aux_bytes = 0;
     if (c.n_resident_pages == 0) {
         if (c.arena_bytes == 0) {
             c.n_resident_pages = (int)auto_resident(c.max_ctx, pb, c.n_layers);
         } else {
-            // a fixed arena: the resident pages get what the ring, the split
+            // a fixed arena: the auxiliary layers' pages are pinned at its top;
+            // the target's resident pages get what the pin, the ring, the split
             // partials and the staging leave (the decode KV grant of the arena)
-            const long fit = resident_fit(c, c.arena_bytes, P);
+            if (c.n_aux_layers > 0) {
+                c.aux_resident_pages = (int)std::min<long>(
+                    P, c.aux_resident_pages > 0 ? c.aux_resident_pages : auto_resident(c.max_ctx, pb, c.n_aux_layers));
+                aux_bytes = aux_region_bytes(c);
+            }
+            const long fit = aux_bytes < c.arena_bytes ? resident_fit(c, c.arena_bytes - aux_bytes, P) : 0;
             if (fit < 1) {
-                why = fmt("arena %zu B cannot hold any resident set besides ring + partials (%zu B with one page)",
-                          c.arena_bytes, arena_layout_with(c, 1).total);
+                why = fmt("arena %zu B cannot hold any resident set besides ring + partials (%zu B with one page)"
+                          " and the auxiliary layers' %zu B",
+                          c.arena_bytes, arena_layout_with(c, 1).total, aux_bytes);
                 return KVS_E_ARENA;
             }
             c.n_resident_pages = (int)fit;
@@ -269,25 +312,27 @@ int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::stri
     }
     const ArenaLayout L = arena_layout(c);
     if (c.arena_bytes != 0) {
-        if (c.arena_bytes < L.total) {
-            why = fmt("arena %zu B cannot hold resident pages + ring + partials (%zu B)", c.arena_bytes, L.total);
+        if (c.arena_bytes < L.total + aux_bytes) {
+            why = fmt("arena %zu B cannot hold resident pages + ring + partials (%zu B)", c.arena_bytes,
+                      L.total + aux_bytes);
             return KVS_E_ARENA;
         }
     }
-    c.arena_bytes = L.total;
+    // a phase arena keeps its budget: the whole allocation, re-lent by phase
+    if (phase) c.flags |= KVS_FLAG_PHASE_ARENA;
+    else c.arena_bytes = L.total;
     if (host_bytes) *host_bytes = (size_t)c.n_layers * (size_t)P * pb;
     *out = c;
     return KVS_OK;
 }
 
-int plan_page(const kvs_config& c, long n_tokens, long page, int* kind, int* index) {
+int plan_page_r(long R, long n_tokens, long page, int* kind, int* index) {
     const long P = pages_for(n_tokens);
     if (page < 0 || page >= P) {
         *kind = KVS_PAGE_ABSENT;
         *index = -1;
         return KVS_OK;
     }
-    const long R = c.n_resident_pages;
     if (page >= P - R) {
         *kind = KVS_PAGE_RESIDENT;
         *index = (int)(page % R);
@@ -296,6 +341,9 @@ int plan_page(const kvs_config& c, long n_tokens, long page, int* kind, int* ind
         *index = (int)page;
     }
     return KVS_OK;
+}
+int plan_page(const kvs_config& c, long n_tokens, long page, int* kind, int* index) {
+    return plan_page_r(c.n_resident_pages, n_tokens, page, kind, index);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -361,7 +409,18 @@ struct kvs_s {
     __half *stage_q = nullptr, *stage_k = nullptr, *stage_v = nullptr;
     float *stage_out = nullptr, *stage_lse = nullptr;
     int* err_word = nullptr;
-    CUtensorMap map_res{}, map_ring{};
+    CUtensorMap map_res{}, map_ring{}, map_aux{};
+    // phase arena: the phase, its width (widest batch), the allocation, the
+    // auxiliary layers' pinned pages (at the top) and the kvs_pin bytes below
+    bool phase_arena = false;
+    int phase = KVS_PHASE_PREFILL;
+    int width = 1;
+    int aux_R = 0;                   // auxiliary layers' resident pages (configured)
+    bool draft_active = true;
+    size_t alloc_bytes = 0;
+    size_t pin_bytes = 0;
+    uint8_t* aux = nullptr;          // auxiliary layers' resident region
+    void* encode_fn = nullptr;       // cuTensorMapEncodeTiled
     cudaStream_t cs = nullptr;       // copy stream (H2D ring)
     cudaStream_t rs = nullptr;       // side stream: resident-page attention (lowest priority)
     cudaStream_t xs = nullptr;       // ring attention stream (highest priority)
@@ -490,6 +549,106 @@ int encode_map(kvs_t* kv, EncodeTiledFn fn, CUtensorMap* map, void* base, uint64
     return KVS_OK;
 }
 
+// The arena laid out for resident count R and the phase width: pointers into
+// the allocation, tensor maps, partial capacity.  The auxiliary layers' pages
+// sit at the top of the allocation while the draft is active.
+int apply_layout(kvs_t* kv, long R, int width) {
+    kvs_config c = kv->cfg;
+    c.n_resident_pages = (int)R;
+    c.max_q_tokens = width;
+    const ArenaLayout L = arena_layout(c);
+    kv->lay = L;
+    kv->cfg.n_resident_pages = (int)R;
+    kv->width = width;
+    kv->resident = kv->arena + L.resident;
+    kv->ring = kv->arena + L.ring;
+    kv->part.ml = reinterpret_cast<float2*>(kv->arena + L.part_ml);
+    kv->part.acc = reinterpret_cast<float*>(kv->arena + L.part_acc);
+    kv->stage_q = reinterpret_cast<__half*>(kv->arena + L.stage_q);
+    kv->stage_k = reinterpret_cast<__half*>(kv->arena + L.stage_kv);
+    kv->stage_v = kv->stage_k + (size_t)width * c.n_kv_heads * kHeadDim;
+    kv->stage_out = reinterpret_cast<float*>(kv->arena + L.stage_out);
+    kv->stage_lse = reinterpret_cast<float*>(kv->arena + L.stage_lse);
+    kv->err_word = reinterpret_cast<int*>(kv->arena + L.err);
+    kv->partial_capacity = partial_records(c);
+    auto enc = reinterpret_cast<EncodeTiledFn>(kv->encode_fn);
+    const uint64_t head_rows = (uint64_t)page_head_bytes(c.type_v, c.type_k) / 128;
+    const uint64_t res_rows = (uint64_t)target_layers(c) * R * c.n_kv_heads * head_rows;
+    const uint64_t ring_rows = (uint64_t)c.n_ring_slots * c.n_kv_heads * head_rows;
+    if (encode_map(kv, enc, &kv->map_res, kv->resident, res_rows) != KVS_OK) return KVS_E_CUDA;
+    if (encode_map(kv, enc, &kv->map_ring, kv->ring, ring_rows) != KVS_OK) return KVS_E_CUDA;
+    kv->aux = nullptr;
+    if (c.n_aux_layers > 0 && kv->draft_active) {
+        kv->aux = kv->arena + kv->alloc_bytes - aux_region_bytes(c);
+        const uint64_t aux_rows = (uint64_t)c.n_aux_layers * c.aux_resident_pages * c.n_kv_heads * head_rows;
+        if (encode_map(kv, enc, &kv->map_aux, kv->aux, aux_rows) != KVS_OK) return KVS_E_CUDA;
+    }
+    return KVS_OK;
+}
+
+// where a layer's resident pages live: region base, slots per layer, global
+// slot index of the layer's slot 0 in the region's tensor map, the map
+struct LayerRes {
+    uint8_t* base;
+    long R;
+    long slot_base;
+    const CUtensorMap* map;
+};
+LayerRes layer_res(kvs_t* kv, int layer) {
+    const int LT = target_layers(kv->cfg);
+    if (layer < LT) {
+        const long R = kv->cfg.n_resident_pages;
+        return {kv->resident + (size_t)layer * R * kv->page_bytes, R, (long)layer * R, &kv->map_res};
+    }
+    const long R = kv->cfg.aux_resident_pages;
+    const int a = layer - LT;
+    return {kv->aux + (size_t)a * R * kv->page_bytes, R, (long)a * R, &kv->map_aux};
+}
+bool aux_layer(const kvs_t* kv, int layer) { return layer >= target_layers(kv->cfg); }
+
+// copy a layer's resident pages (the newest R of its history) from the
+// authoritative host history into their slots (page p -> slot p mod R), one
+// copy per run of consecutive slots
+int recopy_layer(kvs_t* kv, int layer, cudaStream_t s) {
+    const LayerRes r = layer_res(kv, layer);
+    const long P = pages_for(kv->layers[layer].len);
+    long p = std::max(0L, P - r.R);
+    while (p < P) {
+        long q = p + 1;
+        while (q < P && (q % r.R) != 0) ++q;  // slots p mod R .. stay consecutive until the wrap
+        const size_t src = ((size_t)layer * kv->P_max + (size_t)p) * kv->page_bytes;
+        const cudaError_t e = cudaMemcpyAsync(r.base + (size_t)(p % r.R) * kv->page_bytes, kv->host + src,
+                                              (size_t)(q - p) * kv->page_bytes, cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return fail(kv, KVS_E_CUDA, fmt("cudaMemcpyAsync: %s", cudaGetErrorString(e)));
+        p = q;
+    }
+    return KVS_OK;
+}
+
+// status of a phase arena laid out for resident count R and `width`
+void fill_status(const kvs_config& c, long R, int width, size_t alloc, size_t pin, bool draft, int phase,
+                 kvs_arena_status* st) {
+    kvs_config cw = c;
+    cw.n_resident_pages = (int)R;
+    cw.max_q_tokens = width;
+    const ArenaLayout L = arena_layout(cw);
+    std::memset(st, 0, sizeof(*st));
+    st->phase = phase;
+    st->width = width;
+    st->n_resident_pages = (int)R;
+    st->draft_active = draft ? 1 : 0;
+    st->aux_resident_pages = draft ? c.aux_resident_pages : 0;
+    st->phase_arena = (c.flags & KVS_FLAG_PHASE_ARENA) ? 1 : 0;
+    st->arena_bytes = alloc;
+    st->resident_bytes = L.ring - L.resident;
+    st->ring_bytes = L.part_ml - L.ring;
+    st->compute_bytes = L.total - L.part_ml;
+    st->aux_bytes = draft ? aux_region_bytes(c) : 0;
+    st->pinned_bytes = pin;
+    const size_t used = L.total + st->aux_bytes + pin;
+    st->free_bytes = alloc > used ? alloc - used : 0;
+}
+
 void release(kvs_t* kv) {
     if (!kv) return;
     DeviceGuard g(kv->device);
@@ -562,6 +721,43 @@ void fold_timed_upto(kvs_t* kv, size_t n) {
 }
 
 void fold_timed(kvs_t* kv) { fold_timed_upto(kv, kv->timed.size()); }
+
+// Re-lend a phase arena: the phase width, the kvs_pin bytes and the draft's
+// state decide the layout.  Fits the target's resident count first (the state
+// is untouched if nothing fits), waits for the handle's work, lays the arena
+// out and copies from the host history every page that is resident in the new
+// layout but was not (all target pages when R changes; the auxiliary layers'
+// pages when the draft comes back).
+int relayout(kvs_t* kv, int width, size_t pin_bytes, bool draft_active, cudaStream_t s) {
+    if (capture_id(s)) return fail(kv, KVS_E_INVAL, "the arena cannot be re-lent during stream capture");
+    kvs_config c = kv->cfg;
+    c.max_q_tokens = width;
+    const size_t aux_bytes = (draft_active && c.n_aux_layers > 0) ? aux_region_bytes(c) : 0;
+    if (aux_bytes + pin_bytes >= kv->alloc_bytes)
+        return fail(kv, KVS_E_ARENA, "the pinned region would fill the arena");
+    const long R = resident_fit(c, kv->alloc_bytes - aux_bytes - pin_bytes, kv->P_max);
+    if (R < 1)
+        return fail(kv, KVS_E_ARENA, fmt("no resident page fits a width-%d phase beside %zu pinned bytes", width,
+                                         aux_bytes + pin_bytes));
+    int rc = sync_all(kv, s, 60.0);
+    if (rc != KVS_OK) return rc;
+    const bool r_changed = R != kv->cfg.n_resident_pages;
+    const bool aux_back = draft_active && !kv->draft_active;
+    kv->pin_bytes = pin_bytes;
+    kv->draft_active = draft_active;
+    if (r_changed || width != kv->width || aux_back || !draft_active) {
+        if (apply_layout(kv, R, width) != KVS_OK) return KVS_E_CUDA;
+        KVS_CK(kv, cudaMemsetAsync(kv->err_word, 0, sizeof(int), s));
+    }
+    const int LT = target_layers(kv->cfg);
+    if (r_changed)
+        for (int l = 0; l < LT; ++l)
+            if ((rc = recopy_layer(kv, l, s)) != KVS_OK) return rc;
+    if (aux_back)
+        for (int l = LT; l < kv->cfg.n_layers; ++l)
+            if ((rc = recopy_layer(kv, l, s)) != KVS_OK) return rc;
+    return KVS_OK;
+}
 
 }  // namespace
 
@@ -667,6 +863,12 @@ int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
     kv->P_max = pages_for(c.max_ctx);
     kv->host_bytes = host_bytes;
     kv->lay = arena_layout(c);
+    // a phase arena allocates its whole budget and starts in the prefill phase
+    // (the widest batch); otherwise the arena is the exact fit
+    kv->phase_arena = (c.flags & KVS_FLAG_PHASE_ARENA) != 0;
+    kv->alloc_bytes = kv->phase_arena ? c.arena_bytes : kv->lay.total;
+    kv->phase = KVS_PHASE_PREFILL;
+    kv->width = c.max_q_tokens;
     DeviceGuard g(device);
     auto bail = [&](int code, const std::string& w) {
         g_last_error = w;
@@ -682,23 +884,13 @@ int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
     std::memset(kv->host, 0, host_bytes);
     e = cudaHostGetDevicePointer(reinterpret_cast<void**>(&kv->host_dev), kv->host, 0);
     if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("cudaHostGetDevicePointer: %s", cudaGetErrorString(e)));
-    e = cudaMalloc(reinterpret_cast<void**>(&kv->arena), kv->lay.total);
+    e = cudaMalloc(reinterpret_cast<void**>(&kv->arena), kv->alloc_bytes);
     if (e != cudaSuccess) {
         kv->arena = nullptr;
-        return bail(KVS_E_ARENA, fmt("cudaMalloc(arena %zu B) failed: %s", kv->lay.total, cudaGetErrorString(e)));
+        return bail(KVS_E_ARENA, fmt("cudaMalloc(arena %zu B) failed: %s", kv->alloc_bytes, cudaGetErrorString(e)));
     }
-    e = cudaMemset(kv->arena, 0, kv->lay.total);
+    e = cudaMemset(kv->arena, 0, kv->alloc_bytes);
     if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("cudaMemset: %s", cudaGetErrorString(e)));
-    kv->resident = kv->arena + kv->lay.resident;
-    kv->ring = kv->arena + kv->lay.ring;
-    kv->part.ml = reinterpret_cast<float2*>(kv->arena + kv->lay.part_ml);
-    kv->part.acc = reinterpret_cast<float*>(kv->arena + kv->lay.part_acc);
-    kv->stage_q = reinterpret_cast<__half*>(kv->arena + kv->lay.stage_q);
-    kv->stage_k = reinterpret_cast<__half*>(kv->arena + kv->lay.stage_kv);
-    kv->stage_v = kv->stage_k + (size_t)c.max_q_tokens * c.n_kv_heads * kHeadDim;
-    kv->stage_out = reinterpret_cast<float*>(kv->arena + kv->lay.stage_out);
-    kv->stage_lse = reinterpret_cast<float*>(kv->arena + kv->lay.stage_lse);
-    kv->err_word = reinterpret_cast<int*>(kv->arena + kv->lay.err);
 
     e = cudaStreamCreateWithFlags(&kv->cs, cudaStreamNonBlocking);
     if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("cudaStreamCreate: %s", cudaGetErrorString(e)));
@@ -717,7 +909,6 @@ int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
         cudaEventCreateWithFlags(&kv->ev_ring, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&kv->ev_zc, cudaEventDisableTiming) != cudaSuccess)
         return bail(KVS_E_CUDA, "cudaEventCreate failed");
-    kv->partial_capacity = partial_records(c);
     kv->n_groups = c.n_ring_slots > 0 ? c.n_ring_slots / c.chunk_pages : 0;
     kv->ev_full.assign(kv->n_groups, nullptr);
     kv->ev_free.assign(kv->n_groups, nullptr);
@@ -740,20 +931,17 @@ int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
     e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr);
     if (e != cudaSuccess || qr != cudaDriverEntryPointSuccess || !fn)
         return bail(KVS_E_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
-    auto enc = reinterpret_cast<EncodeTiledFn>(fn);
-    const uint64_t head_rows = (uint64_t)page_head_bytes(c.type_v, c.type_k) / 128;
-    const uint64_t res_rows = (uint64_t)c.n_layers * c.n_resident_pages * c.n_kv_heads * head_rows;
-    const uint64_t ring_rows = (uint64_t)c.n_ring_slots * c.n_kv_heads * head_rows;
-    if (encode_map(kv, enc, &kv->map_res, kv->resident, res_rows) != KVS_OK) return bail(KVS_E_CUDA, kv->err);
-    if (encode_map(kv, enc, &kv->map_ring, kv->ring, ring_rows) != KVS_OK) return bail(KVS_E_CUDA, kv->err);
+    kv->encode_fn = fn;
+    if (apply_layout(kv, c.n_resident_pages, c.max_q_tokens) != KVS_OK) return bail(KVS_E_CUDA, kv->err);
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return bail(KVS_E_CUDA, fmt("create sync: %s", cudaGetErrorString(e)));
     if (getenv("KVS_LOG")) {
         fprintf(stderr,
                 "kvs: pool created: %d layer(s), %d resident pages/layer, %d ring slots (chunk %d), "
-                "page %zu B, arena %.2f MiB, pinned history %.2f MiB, device %d\n",
+                "page %zu B, arena %.2f MiB%s, pinned history %.2f MiB, device %d\n",
                 c.n_layers, c.n_resident_pages, c.n_ring_slots, c.chunk_pages, kv->page_bytes,
-                kv->lay.total / 1048576.0, host_bytes / 1048576.0, device);
+                kv->alloc_bytes / 1048576.0, kv->phase_arena ? " (phase arena)" : "", host_bytes / 1048576.0,
+                device);
     }
     *out = kv;
     return KVS_OK;
@@ -780,11 +968,13 @@ int kvs_append(kvs_t* kv, int layer, int pos0, int n_tok, const void* k_f16, con
     if (layer < 0 || layer >= c.n_layers) return fail(kv, KVS_E_INVAL, fmt("layer %d out of range", layer));
     if (n_tok < 1) return fail(kv, KVS_E_INVAL, "n_tok must be >= 1");
     if (!k_f16 || !v_f16) return fail(kv, KVS_E_INVAL, "null K/V");
+    if (aux_layer(kv, layer) && !kv->draft_active)
+        return fail(kv, KVS_E_INVAL, "auxiliary layers are ejected (kvs_draft_restore brings them back)");
     const bool host_k = is_host_ptr(k_f16), host_v = is_host_ptr(v_f16);
-    // host K/V go through staging buffers sized for max_q_tokens; device K/V
-    // may be any width (history pre-fill)
-    if ((host_k || host_v) && n_tok > c.max_q_tokens)
-        return fail(kv, KVS_E_WIDTH, fmt("append batch too wide: %d > max_q_tokens %d", n_tok, c.max_q_tokens));
+    // host K/V go through staging buffers sized for the phase's width; device
+    // K/V may be any width (history pre-fill)
+    if ((host_k || host_v) && n_tok > kv->width)
+        return fail(kv, KVS_E_WIDTH, fmt("append batch too wide: %d > width %d", n_tok, kv->width));
     LayerState& ls = kv->layers[layer];
     if (pos0 < 0 || pos0 > ls.len)
         return fail(kv, KVS_E_ORDER, fmt("append at %d is not contiguous with length %d", pos0, ls.len));
@@ -818,7 +1008,8 @@ int kvs_append(kvs_t* kv, int layer, int pos0, int n_tok, const void* k_f16, con
     if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 7)
         return fail(kv, KVS_E_INVAL, "K/V must be 8-byte aligned");
 
-    const long R = c.n_resident_pages;
+    const LayerRes lr = layer_res(kv, layer);
+    const long R = lr.R;
     const long P_old = pages_for(ls.len), P_new = pages_for((long)pos0 + n_tok);
     const long f_old = std::max(0L, P_old - R), f_new = std::max(0L, P_new - R);
     // pages that re-enter the resident set after a roll-back and keep tokens
@@ -827,7 +1018,7 @@ int kvs_append(kvs_t* kv, int layer, int pos0, int n_tok, const void* k_f16, con
         const bool was_res = (p >= f_old && p < P_old);
         if (!was_res && p * kPageTokens < pos0) {
             const size_t src = ((size_t)layer * kv->P_max + p) * kv->page_bytes;
-            uint8_t* dst = kv->resident + ((size_t)layer * R + (size_t)(p % R)) * kv->page_bytes;
+            uint8_t* dst = lr.base + (size_t)(p % R) * kv->page_bytes;
             KVS_CK(kv, cudaMemcpyAsync(dst, kv->host + src, kv->page_bytes, cudaMemcpyHostToDevice, s));
         }
     }
@@ -835,7 +1026,7 @@ int kvs_append(kvs_t* kv, int layer, int pos0, int n_tok, const void* k_f16, con
     a.k = k;
     a.v = v;
     a.host_layer = kv->host_dev + (size_t)layer * kv->P_max * kv->page_bytes;
-    a.res_layer = kv->resident + (size_t)layer * R * kv->page_bytes;
+    a.res_layer = lr.base;
     a.n_tok = n_tok;
     a.pos0 = pos0;
     a.n_kv = c.n_kv_heads;
@@ -866,9 +1057,13 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     const kvs_config& c = kv->cfg;
     if (layer < 0 || layer >= c.n_layers) return fail(kv, KVS_E_INVAL, fmt("layer %d out of range", layer));
     if (n_q < 1) return fail(kv, KVS_E_INVAL, "n_q must be >= 1");
-    if (n_q > c.max_q_tokens)
-        return fail(kv, KVS_E_WIDTH, fmt("decode batch too wide: %d > max_q_tokens %d", n_q, c.max_q_tokens));
+    if (n_q > kv->width)
+        return fail(kv, KVS_E_WIDTH, kv->phase_arena && kv->phase == KVS_PHASE_DECODE
+                                         ? fmt("phase arena decode batch too wide: %d > width %d", n_q, kv->width)
+                                         : fmt("decode batch too wide: %d > max_q_tokens %d", n_q, kv->width));
     if (!q_f16 || !out) return fail(kv, KVS_E_INVAL, "null q/out");
+    if (aux_layer(kv, layer) && !kv->draft_active)
+        return fail(kv, KVS_E_INVAL, "auxiliary layers are ejected (kvs_draft_restore brings them back)");
     LayerState& ls = kv->layers[layer];
     if (pos0 < 0 || (long)pos0 + n_q > ls.len)
         return fail(kv, KVS_E_ORDER, fmt("queries %d..%d beyond the history (length %d)", pos0, pos0 + n_q - 1, ls.len));
@@ -908,7 +1103,8 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     float* dout = out_alias ? out_alias : (host_out ? kv->stage_out : out);
     float* dlse = lse ? (lse_alias ? lse_alias : (host_lse ? kv->stage_lse : lse)) : nullptr;
 
-    const long R = c.n_resident_pages;
+    const LayerRes lres = layer_res(kv, layer);
+    const long R = lres.R;
     const long P = pages_for(ls.len);
     const long R_eff = std::min(R, P);
     const long first_res = P - R_eff;
@@ -932,7 +1128,8 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     d.err = kv->err_word;
 
     // split counts first: the partial buffer must hold every (split, row) record
-    if ((size_t)count_splits(c, n_q, R_eff, S) * rows > kv->partial_capacity)
+    if ((size_t)count_splits(c, n_q, R_eff, S) * rows > kv->partial_capacity ||
+        (size_t)rows > (size_t)kv->width * c.n_q_heads)
         return fail(kv, KVS_E_INVAL, "internal: partial buffer too small for this call");
     // With profiling on, every kernel runs on the caller's stream so that the
     // events around a launch time that launch alone.
@@ -945,8 +1142,8 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     //    the ring pipeline below
     int split_base = 0;
     {
-        d.region = kv->resident + (size_t)layer * R * kv->page_bytes;
-        d.region_slot_base = (int)(layer * R);
+        d.region = lres.base;
+        d.region_slot_base = (int)lres.slot_base;
         d.region_slots = (int)R;
         d.slot0 = (int)(first_res % R);
         d.page0 = (int)first_res;
@@ -980,7 +1177,7 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         }
         {
             TimedScope ts(kv, rstream, tc ? kTChunkMma : kTDecodeRes, (uint64_t)R_eff * kv->page_bytes);
-            KVS_CK(kv, tc ? launch_chunk_mma(d, &kv->map_res, ns, rstream) : launch_decode(d, &kv->map_res, ns, rstream));
+            KVS_CK(kv, tc ? launch_chunk_mma(d, lres.map, ns, rstream) : launch_decode(d, lres.map, ns, rstream));
         }
         kv->stats.kernel_launches++;
         split_base += ns;
@@ -1021,6 +1218,10 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         }
         const int chunk = c.chunk_pages;
         KVS_CK(kv, cudaStreamWaitEvent(xstream, kv->ev_fork, 0));
+        // tensor-core ring launches run in order on one stream and fold their
+        // partials into the records of the first one
+        const int ring_base = split_base;
+        int ring_width = 0;
         for (long i0 = 0; i0 < S_ring; i0 += chunk) {
             const int cpages = (int)std::min<long>(chunk, S_ring - i0);
             const int gidx = (int)(kv->ring_ctr % kv->n_groups);
@@ -1040,21 +1241,25 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
             d.n_units = cpages;
             const int ns = ring_splits(c, n_q, cpages);
             d.n_splits = ns;
-            d.split_base = split_base;
+            d.split_base = tc ? ring_base : split_base;
+            d.accumulate = (tc && i0 > 0) ? 1 : 0;
             {
                 TimedScope ts(kv, xstream, tc ? kTChunkMma : kTDecodeRing, (uint64_t)cpages * kv->page_bytes);
                 KVS_CK(kv, tc ? launch_chunk_mma(d, &kv->map_ring, ns, xstream)
                               : launch_decode(d, &kv->map_ring, ns, xstream));
             }
+            d.accumulate = 0;
             kv->stats.kernel_launches++;
             KVS_CK(kv, cudaEventRecord(kv->ev_free[gidx], xstream));
             kv->free_valid[gidx] = 1;
             kv->free_cap[gidx] = cap;
-            split_base += ns;
+            if (tc) ring_width = std::max(ring_width, ns);
+            else split_base += ns;
             kv->stats.pages_streamed += cpages;
             kv->stats.bytes_h2d += (uint64_t)cpages * kv->page_bytes;
             kv->stats.h2d_copies++;
         }
+        split_base += ring_width;
         KVS_CK(kv, cudaEventRecord(kv->ev_ring, xstream));
         KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_ring, 0));
     }
@@ -1088,11 +1293,13 @@ int kvs_export_page(kvs_t* kv, int layer, int page, int from_device, void* host_
         return fail(kv, KVS_E_INVAL, "layer/page out of range");
     std::vector<uint8_t> buf(kv->page_bytes);
     if (from_device) {
+        if (aux_layer(kv, layer) && !kv->draft_active)
+            return fail(kv, KVS_E_INVAL, "auxiliary layers are ejected: no resident pages");
         int kind, idx;
-        plan_page(c, kv->layers[layer].len, page, &kind, &idx);
+        plan_page_r(layer_res(kv, layer).R, kv->layers[layer].len, page, &kind, &idx);
         if (kind != KVS_PAGE_RESIDENT) return fail(kv, KVS_E_INVAL, "page is not resident");
         DeviceGuard g(kv->device);
-        const uint8_t* src = kv->resident + ((size_t)layer * c.n_resident_pages + idx) * kv->page_bytes;
+        const uint8_t* src = layer_res(kv, layer).base + (size_t)idx * kv->page_bytes;
         KVS_CK(kv, cudaMemcpy(buf.data(), src, kv->page_bytes, cudaMemcpyDeviceToHost));
     } else {
         std::memcpy(buf.data(), kv->host + ((size_t)layer * kv->P_max + page) * kv->page_bytes, kv->page_bytes);
@@ -1153,7 +1360,9 @@ int kvs_export_page(kvs_t* kv, int layer, int page, int from_device, void* host_
 int kvs_page_location(kvs_t* kv, int layer, int page, int* kind, int* index) {
     if (!kv || !kind || !index) return fail(kv, KVS_E_INVAL, "null argument");
     if (layer < 0 || layer >= kv->cfg.n_layers) return fail(kv, KVS_E_INVAL, "layer out of range");
-    return plan_page(kv->cfg, kv->layers[layer].len, page, kind, index);
+    if (aux_layer(kv, layer) && !kv->draft_active)
+        return fail(kv, KVS_E_INVAL, "auxiliary layers are ejected: no resident pages");
+    return plan_page_r(layer_res(kv, layer).R, kv->layers[layer].len, page, kind, index);
 }
 
 int kvs_layer_length(kvs_t* kv, int layer, int* n_tokens) {
@@ -1199,6 +1408,87 @@ int kvs_set_zero_copy_pct(kvs_t* kv, int pct) {
     return KVS_OK;
 }
 
+int kvs_phase_layout(const kvs_config* resolved, int width, size_t pinned_bytes, int draft_active,
+                     kvs_arena_status* out) {
+    if (!resolved || !out) { g_last_error = "kvs_phase_layout: null argument"; return KVS_E_INVAL; }
+    const kvs_config& c = *resolved;
+    if (!(c.flags & KVS_FLAG_PHASE_ARENA) || c.arena_bytes == 0) {
+        g_last_error = "kvs_phase_layout: the config is not a resolved phase arena";
+        return KVS_E_INVAL;
+    }
+    if (width < 1 || width > c.max_q_tokens) {
+        g_last_error = fmt("kvs_phase_layout: width %d outside 1..max_q_tokens (%d)", width, c.max_q_tokens);
+        return KVS_E_INVAL;
+    }
+    kvs_config cw = c;
+    cw.max_q_tokens = width;
+    const size_t aux_bytes = (draft_active && c.n_aux_layers > 0) ? aux_region_bytes(c) : 0;
+    const long R = aux_bytes + pinned_bytes < c.arena_bytes
+                       ? resident_fit(cw, c.arena_bytes - aux_bytes - pinned_bytes, pages_for(c.max_ctx))
+                       : 0;
+    if (R < 1) {
+        g_last_error = "kvs_phase_layout: no resident page fits";
+        return KVS_E_ARENA;
+    }
+    fill_status(c, R, width, c.arena_bytes, pinned_bytes, draft_active != 0,
+                width == c.max_q_tokens ? KVS_PHASE_PREFILL : KVS_PHASE_DECODE, out);
+    return KVS_OK;
+}
+
+int kvs_set_phase(kvs_t* kv, int phase, int width, void* stream) {
+    if (!kv) return fail(nullptr, KVS_E_INVAL, "null handle");
+    if (!kv->phase_arena) return fail(kv, KVS_E_INVAL, "no phase arena (arena_bytes with n_resident_pages = 0)");
+    if (phase == KVS_PHASE_PREFILL) {
+        if (width == 0) width = kv->cfg.max_q_tokens;
+    } else if (phase == KVS_PHASE_DECODE) {
+        if (width == 0) width = 1;
+    } else {
+        return fail(kv, KVS_E_INVAL, fmt("unknown phase %d", phase));
+    }
+    if (width < 1 || width > kv->cfg.max_q_tokens)
+        return fail(kv, KVS_E_INVAL, fmt("phase width %d outside 1..max_q_tokens (%d)", width, kv->cfg.max_q_tokens));
+    DeviceGuard g(kv->device);
+    const int rc = relayout(kv, width, kv->pin_bytes, kv->draft_active, static_cast<cudaStream_t>(stream));
+    if (rc == KVS_OK) kv->phase = phase;
+    return rc;
+}
+
+int kvs_pin(kvs_t* kv, size_t bytes, void** dev_ptr, void* stream) {
+    if (!kv || !dev_ptr || bytes == 0) return fail(kv, KVS_E_INVAL, "kvs_pin: bad argument");
+    if (!kv->phase_arena) return fail(kv, KVS_E_INVAL, "no phase arena (arena_bytes with n_resident_pages = 0)");
+    if (!kv->draft_active) return fail(kv, KVS_E_INVAL, "the draft is ejected: nothing can be pinned");
+    const size_t total = kv->pin_bytes + align_up(bytes);
+    DeviceGuard g(kv->device);
+    const int rc = relayout(kv, kv->width, total, true, static_cast<cudaStream_t>(stream));
+    if (rc != KVS_OK) return rc;
+    const size_t aux_bytes = kv->cfg.n_aux_layers > 0 ? aux_region_bytes(kv->cfg) : 0;
+    *dev_ptr = kv->arena + kv->alloc_bytes - aux_bytes - total;
+    return KVS_OK;
+}
+
+int kvs_draft_eject(kvs_t* kv, void* stream) {
+    if (!kv) return fail(nullptr, KVS_E_INVAL, "null handle");
+    if (!kv->phase_arena) return fail(kv, KVS_E_INVAL, "no phase arena (arena_bytes with n_resident_pages = 0)");
+    if (!kv->draft_active) return KVS_OK;
+    DeviceGuard g(kv->device);
+    return relayout(kv, kv->width, 0, false, static_cast<cudaStream_t>(stream));
+}
+
+int kvs_draft_restore(kvs_t* kv, void* stream) {
+    if (!kv) return fail(nullptr, KVS_E_INVAL, "null handle");
+    if (!kv->phase_arena) return fail(kv, KVS_E_INVAL, "no phase arena (arena_bytes with n_resident_pages = 0)");
+    if (kv->draft_active) return KVS_OK;
+    DeviceGuard g(kv->device);
+    return relayout(kv, kv->width, 0, true, static_cast<cudaStream_t>(stream));
+}
+
+int kvs_get_arena(kvs_t* kv, kvs_arena_status* out) {
+    if (!kv || !out) return fail(kv, KVS_E_INVAL, "null argument");
+    fill_status(kv->cfg, kv->cfg.n_resident_pages, kv->width, kv->alloc_bytes, kv->pin_bytes, kv->draft_active,
+                kv->phase, out);
+    return KVS_OK;
+}
+
 int kvs_set_profiling(kvs_t* kv, int enable) {
     if (!kv) return fail(nullptr, KVS_E_INVAL, "null handle");
     if (enable) kv->cfg.flags |= KVS_FLAG_PROFILE;
@@ -1216,7 +1506,7 @@ int kvs_measure_h2d(kvs_t* kv, size_t chunk_bytes, size_t total_bytes, int reps,
     if (!kv || !gbs || chunk_bytes == 0 || reps < 1) return fail(kv, KVS_E_INVAL, "bad argument");
     uint8_t* dst = kv->cfg.n_ring_slots ? kv->ring : kv->resident;
     const size_t dst_bytes = kv->cfg.n_ring_slots ? (size_t)kv->cfg.n_ring_slots * kv->page_bytes
-                                                  : (size_t)kv->cfg.n_layers * kv->cfg.n_resident_pages * kv->page_bytes;
+                                                  : (size_t)target_layers(kv->cfg) * kv->cfg.n_resident_pages * kv->page_bytes;
     if (chunk_bytes > dst_bytes) return fail(kv, KVS_E_INVAL, "chunk larger than the device region");
     total_bytes = std::min(total_bytes, kv->host_bytes) / chunk_bytes * chunk_bytes;
     if (total_bytes == 0) return fail(kv, KVS_E_INVAL, "total smaller than one chunk");

@@ -32,6 +32,9 @@ KVS_PAGE_ABSENT = -1
 KVS_PAGE_RESIDENT = 1
 KVS_PAGE_STREAMED = 2
 KVS_FLAG_PROFILE = 1
+KVS_FLAG_PHASE_ARENA = 2
+KVS_PHASE_PREFILL = 0
+KVS_PHASE_DECODE = 1
 
 ERROR_NAMES = {0: "KVS_OK", -1: "KVS_E_INVAL", -2: "KVS_E_ARENA", -3: "KVS_E_WIDTH",
                -4: "KVS_E_ORDER", -5: "KVS_E_CUDA", -6: "KVS_E_TIMEOUT", -7: "KVS_E_NOMEM"}
@@ -42,7 +45,9 @@ EXPORTS = ["kvs_resolve_config", "kvs_page_bytes", "kvs_plan_page", "kvs_create"
            "kvs_get_config", "kvs_get_stats", "kvs_reset_stats", "kvs_set_profiling",
            "kvs_set_zero_copy_pct", "kvs_sync",
            "kvs_measure_h2d", "kvs_attend_pages_static", "kvs_selftest_bounded_wait",
-           "kvs_last_error", "kvs_eject_init", "kvs_eject_step", "kvs_draft_capacity_pages"]
+           "kvs_last_error", "kvs_eject_init", "kvs_eject_step", "kvs_draft_capacity_pages",
+           "kvs_phase_layout", "kvs_set_phase", "kvs_pin", "kvs_draft_eject", "kvs_draft_restore",
+           "kvs_get_arena"]
 
 
 class kvs_config(ctypes.Structure):
@@ -53,7 +58,18 @@ class kvs_config(ctypes.Structure):
                 ("max_q_tokens", ctypes.c_int), ("type_k", ctypes.c_int),
                 ("type_v", ctypes.c_int), ("chunk_pages", ctypes.c_int),
                 ("flags", ctypes.c_int), ("zero_copy_pct", ctypes.c_int),
-                ("arena_bytes", ctypes.c_size_t)]
+                ("arena_bytes", ctypes.c_size_t), ("n_aux_layers", ctypes.c_int),
+                ("aux_resident_pages", ctypes.c_int)]
+
+    def as_dict(self):
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+class kvs_arena_status(ctypes.Structure):
+    _fields_ = ([(n, ctypes.c_int) for n in ("phase", "width", "n_resident_pages", "aux_resident_pages",
+                                             "draft_active", "phase_arena")] +
+                [(n, ctypes.c_size_t) for n in ("arena_bytes", "compute_bytes", "resident_bytes", "ring_bytes",
+                                                "aux_bytes", "pinned_bytes", "free_bytes")])
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -116,6 +132,12 @@ def _load():
     L.kvs_eject_init.argtypes = [cp(kvs_eject_params), cp(kvs_eject_state)]
     L.kvs_eject_step.argtypes = [cp(kvs_eject_params), cp(kvs_eject_state), i]
     L.kvs_draft_capacity_pages.argtypes = [cp(kvs_config), ctypes.c_size_t, cp(i)]
+    L.kvs_phase_layout.argtypes = [cp(kvs_config), i, ctypes.c_size_t, i, cp(kvs_arena_status)]
+    L.kvs_set_phase.argtypes = [vp, i, i, vp]
+    L.kvs_pin.argtypes = [vp, ctypes.c_size_t, cp(vp), vp]
+    L.kvs_draft_eject.argtypes = [vp, vp]
+    L.kvs_draft_restore.argtypes = [vp, vp]
+    L.kvs_get_arena.argtypes = [vp, cp(kvs_arena_status)]
     return L
 
 
@@ -157,10 +179,10 @@ def _check(rc: int, handle=None):
 def make_config(n_layers, n_q_heads, n_kv_heads, max_ctx, n_resident_pages=0, n_ring_slots=0,
                 max_q_tokens=1, chunk_pages=0, flags=0, arena_bytes=0, head_dim=128,
                 page_tokens=256, type_k=KVS_TYPE_Q8_0, type_v=KVS_TYPE_Q4_0,
-                zero_copy_pct=0) -> kvs_config:
+                zero_copy_pct=0, n_aux_layers=0, aux_resident_pages=0) -> kvs_config:
     return kvs_config(n_layers, n_q_heads, n_kv_heads, head_dim, page_tokens, max_ctx,
                       n_resident_pages, n_ring_slots, max_q_tokens, type_k, type_v, chunk_pages,
-                      flags, zero_copy_pct, arena_bytes)
+                      flags, zero_copy_pct, arena_bytes, n_aux_layers, aux_resident_pages)
 
 
 # ---- functions with the C names ------------------------------------------
@@ -238,6 +260,37 @@ def kvs_set_profiling(h, enable: bool) -> None:
 
 def kvs_set_zero_copy_pct(h, pct: int) -> None:
     _check(lib.kvs_set_zero_copy_pct(h, int(pct)), h)
+
+
+def kvs_phase_layout(cfg: kvs_config, width: int, pinned_bytes: int = 0, draft_active: bool = True) -> dict:
+    st = kvs_arena_status()
+    _check(lib.kvs_phase_layout(ctypes.byref(cfg), int(width), int(pinned_bytes), int(bool(draft_active)),
+                                ctypes.byref(st)))
+    return st.as_dict()
+
+
+def kvs_set_phase(h, phase: int, width: int = 0, stream=None) -> None:
+    _check(lib.kvs_set_phase(h, int(phase), int(width), _stream(stream)), h)
+
+
+def kvs_pin(h, nbytes: int, stream=None) -> int:
+    p = ctypes.c_void_p()
+    _check(lib.kvs_pin(h, int(nbytes), ctypes.byref(p), _stream(stream)), h)
+    return p.value
+
+
+def kvs_draft_eject(h, stream=None) -> None:
+    _check(lib.kvs_draft_eject(h, _stream(stream)), h)
+
+
+def kvs_draft_restore(h, stream=None) -> None:
+    _check(lib.kvs_draft_restore(h, _stream(stream)), h)
+
+
+def kvs_get_arena(h) -> dict:
+    st = kvs_arena_status()
+    _check(lib.kvs_get_arena(h, ctypes.byref(st)), h)
+    return st.as_dict()
 
 
 def kvs_sync(h, stream=None, timeout_s: float = 60.0) -> None:

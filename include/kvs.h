@@ -69,6 +69,9 @@ extern "C" {
  * kernels on the caller's stream, one after another, so that the events time
  * one kernel each; steps are slower than without it. */
 #define KVS_FLAG_PROFILE 1
+/* Set by config resolution when the handle runs a phase arena (arena_bytes
+ * with n_resident_pages = 0); a resolved config passed back keeps it. */
+#define KVS_FLAG_PHASE_ARENA 2
 
 typedef struct kvs_config {
     int n_layers;         /* attention layers sharing the pool, auxiliary layers included (e.g. 16+1) */
@@ -111,8 +114,49 @@ typedef struct kvs_config {
                              kernels).  Wider calls always use the ring, so a ring is still
                              required when pages stream. */
     size_t arena_bytes;   /* device arena budget; 0 = exact fit; else must hold one page and all
-                             resident pages + ring + partials + staging (KVS_E_ARENA if not) */
+                             resident pages + ring + partials + staging (KVS_E_ARENA if not).
+                             With n_resident_pages = 0 the handle runs a phase arena: it
+                             allocates exactly arena_bytes and lends it to the current phase
+                             (kvs_set_phase), with a pinned region at its top (below) */
+    int n_aux_layers;     /* phase arena only: the last n_aux_layers layers are auxiliary (a
+                             speculative draft's attention layer, e.g. MTP): their resident pages
+                             live in the pinned region at the arena top, they stream the rest
+                             through the shared ring, and kvs_draft_eject returns their bytes to
+                             the pool; 0 = none */
+    int aux_resident_pages; /* resident pages per auxiliary layer (in the pinned region); 0 = the
+                             10 % rule of the target layers */
 } kvs_config;
+
+/* ---- phase arena ------------------------------------------------------------
+ * "RaymondHuang210129/llama.cpp-adaptive-kv-streaming", Summary: one bounded
+ * device allocation is lent to either prefill or decode, never both; "llama.cpp
+ * adaptive KV streaming - spec fork notes", Phase arena and New arena and
+ * context API: the decode layout is re-reserved at the verify width, a pinned
+ * region is bump-allocated from the arena top (the draft's KV and weights) with
+ * the compute region below it, and the draft-active decode pool is what
+ * remains after the pin and the phase compute slab.
+ * Layout from the bottom: error word, resident pages of the target layers
+ * (R per layer), ring, compute slab (split partials and staging for the
+ * phase's width), free bytes; from the top: the auxiliary layers' resident
+ * pages, then kvs_pin reservations. */
+#define KVS_PHASE_PREFILL 0
+#define KVS_PHASE_DECODE  1
+
+typedef struct kvs_arena_status {
+    int phase;               /* KVS_PHASE_PREFILL or KVS_PHASE_DECODE */
+    int width;               /* widest append / attend batch of the phase */
+    int n_resident_pages;    /* resident pages per target layer */
+    int aux_resident_pages;  /* resident pages per auxiliary layer; 0 while the draft is ejected */
+    int draft_active;        /* 1 unless kvs_draft_eject released the pinned region */
+    int phase_arena;         /* 1 when the handle runs a phase arena */
+    size_t arena_bytes;      /* the allocation */
+    size_t compute_bytes;    /* split partials + staging + error word of the phase */
+    size_t resident_bytes;   /* target layers' resident pages */
+    size_t ring_bytes;
+    size_t aux_bytes;        /* auxiliary layers' resident pages (pinned, at the top) */
+    size_t pinned_bytes;     /* kvs_pin reservations (below the auxiliary pages) */
+    size_t free_bytes;       /* arena_bytes minus everything above */
+} kvs_arena_status;
 
 typedef struct kvs_stats {
     uint64_t appends, attends;         /* calls */
@@ -268,6 +312,44 @@ int kvs_reset_stats(kvs_t* kv);
  * partials are sized for every share at kvs_create.  KVS_E_INVAL outside
  * 0..100.  A CUDA graph captured earlier keeps the share it was captured with. */
 int kvs_set_zero_copy_pct(kvs_t* kv, int pct);
+
+/* Pure host: the layout a phase arena (resolved config with a budget and
+ * auto resident pages) takes for a phase of the given width (1..max_q_tokens)
+ * with `pinned_bytes` of kvs_pin reservations and the draft active or
+ * ejected.  KVS_E_ARENA if no resident page fits; KVS_E_INVAL if the config
+ * is not a phase arena. */
+int kvs_phase_layout(const kvs_config* resolved, int width, size_t pinned_bytes, int draft_active,
+                     kvs_arena_status* out);
+
+/* Re-lend the arena to a phase: KVS_PHASE_PREFILL takes width max_q_tokens,
+ * KVS_PHASE_DECODE takes `width` (1 + n_draft; 0 = 1).  Waits (bounded) for
+ * the handle's work, lays the arena out for the phase (a narrower compute slab
+ * leaves room for more resident pages) and copies the pages that are resident
+ * in the new layout from the authoritative host history on `stream`.  Later
+ * calls wider than the phase's width fail with KVS_E_WIDTH ("phase arena decode
+ * batch too wide").  CUDA graphs captured before the switch are invalid after
+ * it.  KVS_E_INVAL if the handle has no phase arena. */
+int kvs_set_phase(kvs_t* kv, int phase, int width, void* stream);
+
+/* Bump-allocate `bytes` (rounded up to 256) from the top of the arena, below
+ * the auxiliary layers' pages and earlier reservations, for a draft's weights
+ * or state; the target's resident set shrinks if it must (pages copied as in
+ * kvs_set_phase, on `stream`).  *dev_ptr = the reservation's device address.
+ * KVS_E_ARENA if the current phase would keep no resident page; KVS_E_INVAL
+ * while the draft is ejected or without a phase arena. */
+int kvs_pin(kvs_t* kv, size_t bytes, void** dev_ptr, void* stream);
+
+/* Draft eject: release the whole pinned region (the auxiliary layers' pages
+ * and every kvs_pin reservation) to the target's resident pages; appends and
+ * attends on auxiliary layers fail with KVS_E_INVAL until kvs_draft_restore.
+ * Restore re-reserves the auxiliary pages at the top (the target shrinks back)
+ * and copies them from the host history, which stayed authoritative.  Both
+ * are no-ops when already in that state. */
+int kvs_draft_eject(kvs_t* kv, void* stream);
+int kvs_draft_restore(kvs_t* kv, void* stream);
+
+/* The arena layout in use. */
+int kvs_get_arena(kvs_t* kv, kvs_arena_status* out);
 
 /* Turn KVS_FLAG_PROFILE on (1) or off (0) for later calls. */
 int kvs_set_profiling(kvs_t* kv, int enable);

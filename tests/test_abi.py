@@ -59,8 +59,9 @@ def test_header_constants_match_binding_and_oracle(kvs):
 
 
 def test_struct_sizes_match_header(kvs):
-    # 14 ints + size_t ; 8 u64, 6 double, 9 u64
-    assert ctypes.sizeof(kvs.kvs_config) == 14 * 4 + 8
+    # 14 ints + size_t + 2 ints (padded to 8) ; 8 u64, 6 double, 9 u64
+    assert ctypes.sizeof(kvs.kvs_config) == 14 * 4 + 8 + 2 * 4
+    assert ctypes.sizeof(kvs.kvs_arena_status) == 6 * 4 + 7 * 8
     assert ctypes.sizeof(kvs.kvs_stats) == (8 + 6 + 9) * 8
 
 
@@ -165,22 +166,23 @@ def test_arena_budget_sizes_the_resident_set(kvs, layers, qh, kvh, ctx, ring, mq
     r, _ = kvs.kvs_resolve_config(c)
     R = r.n_resident_pages
     P = oracle.pages_for(ctx)
-    assert 1 <= R <= P and r.arena_bytes <= budget
+    # a phase arena keeps the whole budget as its allocation
+    assert 1 <= R <= P and r.arena_bytes == budget and r.flags & kvs.KVS_FLAG_PHASE_ARENA
 
     def need(n):
         e = kvs.make_config(layers, qh, kvh, ctx, n_resident_pages=n, n_ring_slots=ring, max_q_tokens=mq)
         return kvs.kvs_resolve_config(e)[0].arena_bytes
 
-    assert need(R) == r.arena_bytes
+    assert need(R) <= budget
     if R < P:
         assert need(R + 1) > budget
     # the resident bytes dominate: the grant is the arena minus ring, partials and staging
-    assert r.arena_bytes >= layers * R * kvs.kvs_page_bytes(r)
+    assert need(R) >= layers * R * kvs.kvs_page_bytes(r)
 
 
 @pytest.mark.parametrize("layers,qh,kvh,ctx,ring,mq,budget", [
     (16, 32, 8, 32768, 8, 1, 8 * 425984),             # below ring + one resident page per layer
-    (1, 40, 8, 65536, 16, 256, 100 << 20),            # the 256-row split partials alone need more
+    (1, 40, 8, 65536, 16, 256, 40 << 20),             # the 256-row split partials alone need more
 ])
 def test_arena_budget_without_room_is_rejected(kvs, layers, qh, kvh, ctx, ring, mq, budget):
     c = kvs.make_config(layers, qh, kvh, ctx, n_ring_slots=ring, max_q_tokens=mq, arena_bytes=budget)
