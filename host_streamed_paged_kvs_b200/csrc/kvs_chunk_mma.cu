@@ -415,12 +415,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     *reinterpret_cast<uint4*>(sKh + tile_off(kSubKeys, kloc, hf * 64 + 8 * c8)) =
                         *reinterpret_cast<const uint4*>(rb + kRawKq + row * 128 + ((c8 ^ (row & 7)) << 4));
                 }
-            } else
-            for (int un = ptid; un < kSubKeys * 8; un += kProdThreads) {
+            } else {
+            // each thread's (up to three) units: all shared-memory loads first,
+            // so they are in flight together, then the conversions and stores
+            constexpr int kKUnits = kSubKeys * 8, kKIters = (kKUnits + kProdThreads - 1) / kProdThreads;
+            uint4 qk[kKIters];
+            __half dk[kKIters];
+#pragma unroll
+            for (int it = 0; it < kKIters; ++it) {
+                const int un = ptid + it * kProdThreads;
+                if (un < kKUnits) {
+                    const int kloc = un & 63, g = un >> 6, key = sub * kSubKeys + kloc;
+                    qk[it] = *reinterpret_cast<const uint4*>(rb + kRawKq + key * 128 + ((g ^ (key & 7)) << 4));
+                    dk[it] = *reinterpret_cast<const __half*>(rb + kRawKd + key * 8 + (g >> 1) * 2);
+                }
+            }
+#pragma unroll
+            for (int it = 0; it < kKIters; ++it) {
+                const int un = ptid + it * kProdThreads;
+                if (un >= kKUnits) break;
                 const int kloc = un & 63, g = un >> 6;  // key in the sub-stage, 16-dim chunk
-                const int key = sub * kSubKeys + kloc;   // key in the raw stage
-                const uint4 q = *reinterpret_cast<const uint4*>(rb + kRawKq + key * 128 + ((g ^ (key & 7)) << 4));
-                const __half dh = *reinterpret_cast<const __half*>(rb + kRawKd + key * 8 + (g >> 1) * 2);
+                const uint4 q = qk[it];
+                const __half dh = dk[it];
                 const __half2 d2 = __halves2half2(dh, dh);
                 const __half2 bias = __float2half2_rn(1152.0f);
                 const uint32_t w[4] = {q.x ^ 0x80808080u, q.y ^ 0x80808080u, q.z ^ 0x80808080u, q.w ^ 0x80808080u};
@@ -442,6 +458,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 *reinterpret_cast<uint4*>(sKh + off1) = make_uint4(o[4], o[5], o[6], o[7]);
                 *reinterpret_cast<uint4*>(sKl + off0) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
                 *reinterpret_cast<uint4*>(sKl + off1) = make_uint4(ol[4], ol[5], ol[6], ol[7]);
+            }
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -486,22 +503,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         *reinterpret_cast<const uint4*>(rb + kRawVq + key * (kHeadDim * 2) + 16 * c);
                 }
             } else
-            for (int un = ptid; un < kSubKeys * kBlocks; un += kProdThreads) {
+            {
+            // each thread's (up to two) units: loads first, then conversions and stores
+            constexpr int kVUnits = kSubKeys * kBlocks, kVIters = (kVUnits + kProdThreads - 1) / kProdThreads;
+            uint4 qv[kVIters];
+            __half dvv[kVIters], mvv[kVIters];
+            uint32_t hvv[kVIters];
+#pragma unroll
+            for (int it = 0; it < kVIters; ++it) {
+                const int un = ptid + it * kProdThreads;
+                if (un < kVUnits) {
+                    const int blk = un & 3, key = sub * kSubKeys + (un >> 2);
+                    qv[it] = *reinterpret_cast<const uint4*>(rb + kRawVq + key * 64 + blk * 16);
+                    dvv[it] = *reinterpret_cast<const __half*>(rb + kRawVd + key * 8 + blk * 2);
+                    hvv[it] = 0;
+                    if constexpr (v_has_fifth(VT)) hvv[it] = *reinterpret_cast<const uint32_t*>(rb + kRawVh + key * 16 + blk * 4);
+                    if constexpr (v_has_min(VT)) mvv[it] = *reinterpret_cast<const __half*>(rb + kRawVm + key * 8 + blk * 2);
+                }
+            }
+#pragma unroll
+            for (int it = 0; it < kVIters; ++it) {
+                const int un = ptid + it * kProdThreads;
+                if (un >= kVUnits) break;
                 // Q4_0 V: V^ = fp16(d * (q - 8)); Q5_0 V: the same nibbles with
                 // the fifth bits added, V^ = fp16(d * (q - 16)); Q4_1 / Q5_1 V:
                 // V^ = fp16(d * q + m) (one rounding)
                 const int blk = un & 3, kloc = un >> 2;
-                const int key = sub * kSubKeys + kloc;
-                const uint4 q = *reinterpret_cast<const uint4*>(rb + kRawVq + key * 64 + blk * 16);
-                const __half dh = *reinterpret_cast<const __half*>(rb + kRawVd + key * 8 + blk * 2);
-                uint32_t hw = 0;
-                if constexpr (v_has_fifth(VT)) hw = *reinterpret_cast<const uint32_t*>(rb + kRawVh + key * 16 + blk * 4);
+                const uint4 q = qv[it];
+                const __half dh = dvv[it];
+                const uint32_t hw = hvv[it];
                 const __half2 d2 = __halves2half2(dh, dh);
                 __half2 m2 = __float2half2_rn(0.0f);
-                if constexpr (v_has_min(VT)) {
-                    const __half mh = *reinterpret_cast<const __half*>(rb + kRawVm + key * 8 + blk * 2);
-                    m2 = __halves2half2(mh, mh);
-                }
+                if constexpr (v_has_min(VT)) m2 = __halves2half2(mvv[it], mvv[it]);
                 const __half2 bias = __float2half2_rn(v_has_min(VT) ? 1024.0f : (VT == kVQ5_0 ? 1040.0f : 1032.0f));
                 // code pair (exact in fp16) -> V^ pair
                 auto val = [&](uint32_t bits) {
@@ -524,6 +557,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 *reinterpret_cast<uint4*>(sVb + tile_off(kSubKeys, kloc, 32 * blk + 8)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
                 *reinterpret_cast<uint4*>(sVb + tile_off(kSubKeys, kloc, 32 * blk + 16)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
                 *reinterpret_cast<uint4*>(sVb + tile_off(kSubKeys, kloc, 32 * blk + 24)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+            }
             }
             // the stores above go to the tensor cores (async proxy); the raw
             // stage's reads are done before its buffer is handed back to TMA
@@ -552,43 +586,62 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
             const int sg = raw0 + (i >> 1);
             const int kbase = (a.page0 + (sg >> 1)) * kPageTokens + (sg & 1) * kRawKeys + (i & 1) * kSubKeys;
-            float v[64];
-            if (warp_active) tmem_ld64(t_s, v);
-            // row max over the 64 keys as eight independent chains
-            float mx = -CUDART_INF_F;
-            if (warp_active) {
-                if (kbase + 63 > kend) {
-#pragma unroll
-                    for (int e = 0; e < 64; ++e)
-                        if (kbase + e > kend) v[e] = -CUDART_INF_F;
-                }
-                float m8[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) m8[j] = v[j];
-#pragma unroll
-                for (int e = 8; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], v[e]);
-                mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                           fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-            }
-            // keep the reference max unless the row's max grew by more than 2^8
-            const float m_stage = mx * a.q_scale;
-            float m_use = m_ref;
-            if (m_stage > m_ref + 8.0f) m_use = m_stage;
-            const float mu = (m_use == -CUDART_INF_F) ? 0.0f : m_use;
-            const float alpha = (m_use == m_ref) ? 1.0f : ex2_approx(m_ref - mu);
-            m_ref = m_use;
-            l_run *= alpha;
+            const bool tail = kbase + 63 > kend;  // keys past the row's causal end in this sub-stage
             if (warp_active) {
                 uint32_t pk[32];
-                float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four independent partial sums
+                float lsum = 0.0f, alpha = 1.0f;
+                // p = 2^(s scale - m) with the reference max m, and the sub-stage's
+                // sum; masked keys give 2^-inf = 0
+                auto exp_row = [&](const float (&v)[64], float m) {
+                    float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four independent partial sums
 #pragma unroll
-                for (int e = 0; e < 64; e += 2) {
-                    const float p0 = ex2_approx(fmaf(v[e], a.q_scale, -mu));      // 2^-inf = 0
-                    const float p1 = ex2_approx(fmaf(v[e + 1], a.q_scale, -mu));
-                    l4[(e >> 1) & 3] += p0 + p1;
-                    pk[e >> 1] = h2u(__floats2half2_rn(p0, p1));
+                    for (int e = 0; e < 64; e += 2) {
+                        const float p0 = ex2_approx(fmaf(v[e], a.q_scale, -m));
+                        const float p1 = ex2_approx(fmaf(v[e + 1], a.q_scale, -m));
+                        l4[(e >> 1) & 3] += p0 + p1;
+                        pk[e >> 1] = h2u(__floats2half2_rn(p0, p1));
+                    }
+                    return (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                };
+                auto load_s = [&](float (&v)[64]) {
+                    tmem_ld64(t_s, v);
+                    if (tail) {
+#pragma unroll
+                        for (int e = 0; e < 64; ++e)
+                            if (kbase + e > kend) v[e] = -CUDART_INF_F;
+                    }
+                };
+                // Fast path: keep the reference max.  The sub-stage is accepted
+                // when its sum is at most 2^8, so every p <= 2^8 as the lazy max
+                // below guarantees; the row max is then never needed.
+                bool slow = __any_sync(0xffffffffu, m_ref == -CUDART_INF_F);
+                if (!slow) {
+                    float v[64];
+                    load_s(v);
+                    lsum = exp_row(v, m_ref);
+                    slow = __any_sync(0xffffffffu, !(lsum <= 256.0f));
                 }
-                l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                if (slow) {
+                    // the row max over the 64 keys (eight independent chains); the
+                    // reference max moves only if it grew by more than 2^8
+                    float v[64];
+                    load_s(v);
+                    float m8[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) m8[j] = v[j];
+#pragma unroll
+                    for (int e = 8; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], v[e]);
+                    const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                           fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                    const float m_stage = mx * a.q_scale;
+                    float m_use = m_ref;
+                    if (m_stage > m_ref + 8.0f) m_use = m_stage;
+                    const float mu = (m_use == -CUDART_INF_F) ? 0.0f : m_use;
+                    alpha = (m_use == m_ref) ? 1.0f : ex2_approx(m_ref - mu);
+                    m_ref = m_use;
+                    lsum = exp_row(v, mu);
+                }
+                l_run = fmaf(l_run, alpha, lsum);
                 tmem_st32u(t_s, pk);  // P_t over the first 32 S_t columns (waits for the store)
                 // rescale the row of O_t (stable: PV_t(i - 1) completed before S_t(i) was issued)
                 if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
