@@ -8,7 +8,7 @@
 // rows): both tiles share every dequantized K/V sub-stage, so the producers'
 // work and the shared-memory operand traffic they cause are paid once per two
 // tiles, and the tensor cores alternate between the tiles' products while
-// each tile's softmax runs.  512 threads in three warp-specialized roles on
+// each tile's softmax runs.  512 threads in four warp-specialized roles on
 // 64-key sub-stages, handing work to each other only through mbarriers:
 //
 //   softmax warps 0..3 (tile 0) and 4..7 (tile 1), thread = query row = TMEM
@@ -17,25 +17,28 @@
 //     the log2 domain, keep a per-row reference max that only moves when the
 //     row max exceeds it by more than 2^8 (then rescale the row of O in TMEM),
 //     and write P in fp16 over the S columns just read;
-//   producer warps 8..14
+//   producer warps 8..13
 //     dequantize each 64-key half of a raw Q8_0/Q4_0 stage (128 keys, landed
-//     by TMA, two raw stages in flight) into fp16 UMMA operand tiles with the
-//     128-byte swizzle:
+//     by TMA, three raw stages in flight where shared memory allows, else two)
+//     into fp16 UMMA operand tiles with the 128-byte swizzle:
 //       K^ = d*q8 as [keys][dims] (K-major), split into hi = fp16(d*q8) and
 //       lo = fp16(d*q8 - hi) so the scores carry no fp16 rounding of K
 //       (two buffers, free again once both tiles' S MMAs that read them
 //       complete);
 //       V^ = fp16(d*(q4-8)) as [keys][dims] (read as an MN-major B operand;
 //       three buffers, free again once both tiles' PV MMAs complete);
-//   MMA warp 15 (one elected lane)
+//   MMA warp 14 (one elected lane)
 //     polls the barriers without blocking and issues, whichever is ready
-//     first: the next raw TMA stage into a buffer the producers released;
-//     S_t = Q_t K^_hi^T + Q_t K^_lo^T (tcgen05.mma M=128 N=64 K=16, A = Q_t
-//     from tensor memory, fp32 accumulate) of tile t once the K^ buffer is
-//     full and the tile's previous PV product has completed (P_t lives in the
-//     S_t columns); and O_t += P_t V^ (M=128 N=128 K=16, A = P_t from tensor
-//     memory) once the softmax wrote P_t and V^ is written.  Only the B
-//     operands (K^, V^) are read from shared memory.
+//     first: S_t = Q_t K^_hi^T + Q_t K^_lo^T (tcgen05.mma M=128 N=64 K=16,
+//     A = Q_t from tensor memory, fp32 accumulate) of tile t once the K^
+//     buffer is full and the tile's previous PV product has completed (P_t
+//     lives in the S_t columns); and O_t += P_t V^ (M=128 N=128 K=16, A = P_t
+//     from tensor memory) once the softmax wrote P_t and V^ is written.  Only
+//     the B operands (K^, V^) are read from shared memory;
+//   load warp 15 (one lane)
+//     issues each raw stage (a TMA tile of the K quants, bulk copies of the
+//     other fields) as soon as the producers release its buffer, so the loads
+//     never wait behind the MMA issue.
 //
 // Tensor memory (512 columns, one CTA per SM), per tile t at 256 t: O_t (128
 // fp32 columns) at +0, S_t (64) at +128 with P_t (fp16 pairs, 32) over its
@@ -56,22 +59,25 @@ namespace {
 constexpr int kTiles = 2;                                   // M tiles per CTA
 constexpr int kTileWarps = 4;                               // softmax warps per tile
 constexpr int kSoftWarps = kTiles * kTileWarps;             // 8
-constexpr int kProdWarps = 7;
-constexpr int kMmaWarp = kSoftWarps + kProdWarps;           // 15
-constexpr int kTcThreads = (kMmaWarp + 1) * 32;             // 512
+constexpr int kProdWarps = 6;
+constexpr int kMmaWarp = kSoftWarps + kProdWarps;           // 14
+constexpr int kLoadWarp = kMmaWarp + 1;                     // 15
+constexpr int kTcThreads = (kLoadWarp + 1) * 32;            // 512
 constexpr int kProdThreads = kProdWarps * 32;
 constexpr int kMTile = 128;
 constexpr int kRawKeys = 128;  // keys per raw (TMA) stage
 constexpr int kSubKeys = 64;   // keys per dequant / MMA sub-stage
 constexpr int kRawKq = 0;
-constexpr int kRawKd = kRawKeys * kHeadDim;                 // 16384
-constexpr int kRawStages = 2;
+constexpr int kMaxRawStages = 3;  // raw stages in flight: three where they fit, else two
 constexpr int kKBufs = 2;
 constexpr int kVBufs = 3;
 constexpr int kKVBytes = kSubKeys * kHeadDim * 2;     // 16384: K^hi, K^lo or V^ [64][128] fp16
-// barriers: raw_full[2] raw_free[2] k_full[2] k_free[2] v_full[3] v_free[3]
+// barriers: raw_full[3] raw_free[3] k_full[2] k_free[2] v_full[3] v_free[3]
 //           s_full[tile] p_full[tile] o_free[tile]
-constexpr int kNumBars = 14 + 3 * kTiles;
+constexpr int kBarK = 2 * kMaxRawStages;           // 6
+constexpr int kBarV = kBarK + 2 * kKBufs;          // 10
+constexpr int kBarT = kBarV + 2 * 3;               // 16
+constexpr int kNumBars = kBarT + 3 * kTiles;       // 22
 constexpr uint32_t kTmemCols = 512;
 // columns within a tile's 256: O, S (P over its first 32 columns), Q
 constexpr uint32_t kTileCols = 256, kColO = 0, kColS = 128, kColQ = 192;
@@ -97,6 +103,9 @@ struct TcGeom {
     static constexpr int kRawVm = kRawVd + kRawKeys * PG::kVdRow;                // Q4_1 / Q5_1 minima
     static constexpr int kRawBytes = kRawVm + kRawKeys * PG::kVmRow;
     static constexpr int kKHalves = KT == kKF16 ? 1 : 2;                         // K^ tiles per buffer
+    // the dequantized tiles, barriers and slack; three raw stages where they fit
+    static constexpr size_t kRest = (size_t)(kKBufs * kKHalves + kVBufs) * kKVBytes + kNumBars * 8 + 1024 + 32;
+    static constexpr int kRawStages = (size_t)kMaxRawStages * kRawBytes + kRest <= 232448 ? kMaxRawStages : 2;
     static constexpr size_t kOffK = (size_t)kRawStages * kRawBytes;
     static constexpr size_t kOffV = kOffK + kKBufs * kKHalves * kKVBytes;
     static constexpr size_t kOffBar = kOffV + kVBufs * kKVBytes;
@@ -107,7 +116,8 @@ struct TcGeom {
                   "swizzled tiles need 1024-B alignment");
     static_assert(kSmem <= 232448, "shared memory budget");
 };
-static_assert(TcGeom<kVQ4_0>::kOffBar == 167936, "Q4_0 geometry");
+static_assert(TcGeom<kVQ4_0>::kRawStages == 3 && TcGeom<kVQ8_0>::kRawStages == 3 && TcGeom<kVF16>::kRawStages == 2,
+              "raw stages in flight");
 static_assert(TcGeom<kVQ5_0>::kRawBytes == 28672, "Q5_0 raw stage");
 static_assert(TcGeom<kVQ4_1>::kRawBytes == 27648 && TcGeom<kVQ5_1>::kRawBytes == 29696, "Q4_1 / Q5_1 raw stages");
 static_assert(TcGeom<kVF16>::kRawBytes == 50176, "F16 raw stage");
@@ -210,15 +220,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint8_t* sK = smem + kOffK;
     uint8_t* sV = smem + kOffV;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-    uint64_t* raw_full = bars + 0;   // [2] TMA bytes landed
-    uint64_t* raw_free = bars + 2;   // [2] producers done reading a raw stage (7 warp arrivals)
-    uint64_t* k_full = bars + 4;     // [2] producers wrote K^hi/K^lo (7 warp arrivals)
-    uint64_t* k_free = bars + 6;     // [2] both tiles' S MMAs reading a K^ buffer complete
-    uint64_t* v_full = bars + 8;     // [3] producers wrote V^ (7 warp arrivals)
-    uint64_t* v_free = bars + 11;    // [3] both tiles' PV MMAs reading a V^ buffer complete
-    uint64_t* s_full = bars + 14;    // [tile] S_t MMA complete
-    uint64_t* p_full = bars + 14 + kTiles;      // [tile] softmax wrote P_t (4 warp arrivals)
-    uint64_t* o_free = bars + 14 + 2 * kTiles;  // [tile] PV_t MMA complete (P_t / S_t columns free)
+    constexpr int kRS = TG::kRawStages;
+    uint64_t* raw_full = bars + 0;                 // [raw stage] TMA bytes landed
+    uint64_t* raw_free = bars + kMaxRawStages;     // [raw stage] producers done reading it (6 warp arrivals)
+    uint64_t* k_full = bars + kBarK;               // [2] producers wrote K^hi/K^lo (6 warp arrivals)
+    uint64_t* k_free = bars + kBarK + 2;           // [2] both tiles' S MMAs reading a K^ buffer complete
+    uint64_t* v_full = bars + kBarV;               // [3] producers wrote V^ (6 warp arrivals)
+    uint64_t* v_free = bars + kBarV + 3;           // [3] both tiles' PV MMAs reading a V^ buffer complete
+    uint64_t* s_full = bars + kBarT;               // [tile] S_t MMA complete
+    uint64_t* p_full = bars + kBarT + kTiles;      // [tile] softmax wrote P_t (4 warp arrivals)
+    uint64_t* o_free = bars + kBarT + 2 * kTiles;  // [tile] PV_t MMA complete (P_t / S_t columns free)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmem);
     // set by a thread whose bounded wait gave up; everyone then skips the
     // remaining waits and work (there are no named barriers to leave behind)
@@ -239,9 +250,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     if (tid == 32) {
         *sAbort = 0;
-        for (int k = 0; k < 2; ++k) {
+        for (int k = 0; k < kMaxRawStages; ++k) {
             mbar_init(&raw_full[k], 1);
             mbar_init(&raw_free[k], kProdWarps);
+        }
+        for (int k = 0; k < kKBufs; ++k) {
             mbar_init(&k_full[k], kProdWarps);
             mbar_init(&k_free[k], 1);
         }
@@ -295,16 +308,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         return false;
     };
 
-    if (warp == kMmaWarp) {
-        // ============================ MMA / TMA warp ============================
+    if (warp == kLoadWarp) {
+        // ============================ TMA load warp ============================
+        // raw stage r into buffer r % kRS once the producers released the
+        // stage that used it before (r - kRS)
         if (lane == 0) {
-            auto issue_raw = [&](int r) {  // raw stage r of this split into buffer r & 1
+            for (int r = 0; r < n_raw; ++r) {
+                const int buf = r % kRS;
+                if (r >= kRS && fail_wait(&raw_free[buf], ((r - kRS) / kRS) & 1)) break;
                 const int sg = raw0 + r;
                 const int u = sg >> 1, half = sg & 1;
                 const int slot = (a.slot0 + u) % a.region_slots;
                 const uint8_t* ph = a.region + ((size_t)slot * a.n_kv + h) * PG::kHeadBytes;
-                uint8_t* dst = raw + (r & 1) * kRawBytes;
-                uint64_t* b = &raw_full[r & 1];
+                uint8_t* dst = raw + buf * kRawBytes;
+                uint64_t* b = &raw_full[buf];
                 mbar_expect_tx(b, kRawBytes);
                 const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * PG::kRows + half * TG::kKRows;
 #pragma unroll
@@ -319,9 +336,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     bulk_load(dst + kRawVd, ph + PG::kOffVd + half * (kRawKeys * kBlocks * 2), kRawKeys * kBlocks * 2, b);
                 if constexpr (PG::kVmRow > 0)
                     bulk_load(dst + kRawVm, ph + PG::kOffVm + half * (kRawKeys * PG::kVmRow), kRawKeys * PG::kVmRow, b);
-            };
-            int ir = 0;        // next raw stage to load
-            for (; ir < kRawStages && ir < n_raw; ++ir) issue_raw(ir);
+            }
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ============================ MMA warp ============================
+        if (lane == 0) {
             // next S and PV sub-stage of tile 0 and tile 1 (an absent tile is always done)
             int is0 = 0, ip0 = 0, is1 = 0, ip1 = 0;
             if (n_tiles < kTiles) is1 = ip1 = n_sub;
@@ -370,11 +390,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             };
             const uint64_t t0 = globaltimer_ns();
             for (uint32_t spin = 0; ip0 < n_sub || ip1 < n_sub; ++spin) {
-                // raw stage ir reuses buffer ir & 1 once stage ir - 2 is dequantized
-                if (ir < n_raw && mbar_test(&raw_free[ir & 1], ((ir - 2) >> 1) & 1)) {
-                    issue_raw(ir);
-                    ++ir;
-                }
                 // S products first, the tile that is behind first; then PV products
                 if (is1 < is0) {
                     if (try_s(1, is1, ip1, is0) || try_s(0, is0, ip0, is1)) continue;
@@ -399,8 +414,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int ptid = tid - kSoftWarps * 32;
         for (int i = 0; i < n_sub; ++i) {
             const int r = i >> 1, sub = i & 1;
-            const uint8_t* rb = raw + (r & 1) * kRawBytes;
-            if (sub == 0 && fail_wait(&raw_full[r & 1], (r >> 1) & 1)) break;
+            const uint8_t* rb = raw + (r % kRS) * kRawBytes;
+            if (sub == 0 && fail_wait(&raw_full[r % kRS], (r / kRS) & 1)) break;
             // ---- K^ hi / lo for keys [64 sub, 64 sub + 64) of the raw stage,
             //      once the S MMAs of sub-stage i - 2 released the buffer ----
             if (i >= 2 && fail_wait(&k_free[i & 1], ((i - 2) >> 1) & 1)) break;
@@ -565,7 +580,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive_cta(&v_full[i % kVBufs]);
-                if (sub == 1) mbar_arrive_cta(&raw_free[r & 1]);
+                if (sub == 1) mbar_arrive_cta(&raw_free[r % kRS]);
             }
         }
     } else if (my_tile < n_tiles) {
