@@ -31,10 +31,11 @@
 //     polls the barriers without blocking and issues, whichever is ready
 //     first: S_t = Q_t K^_hi^T + Q_t K^_lo^T (tcgen05.mma M=128 N=64 K=16,
 //     A = Q_t from tensor memory, fp32 accumulate) of tile t once the K^
-//     buffer is full and the tile's previous PV product has completed (P_t
-//     lives in the S_t columns); and O_t += P_t V^ (M=128 N=128 K=16, A = P_t
-//     from tensor memory) once the softmax wrote P_t and V^ is written.  Only
-//     the B operands (K^, V^) are read from shared memory;
+//     buffer is full and the tile's previous PV product has been issued (P_t
+//     lives in the S_t columns; the tensor cores run the MMAs in issue order);
+//     and O_t += P_t V^ (M=128 N=128 K=16, A = P_t from tensor memory) once
+//     the softmax wrote P_t and V^ is written, with the tile's next S right
+//     behind it.  Only the B operands (K^, V^) are read from shared memory;
 //   load warp 15 (one lane)
 //     issues each raw stage (a TMA tile of the K quants, bulk copies of the
 //     other fields) as soon as the producers release its buffer, so the loads
@@ -346,11 +347,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int is0 = 0, ip0 = 0, is1 = 0, ip1 = 0;
             if (n_tiles < kTiles) is1 = ip1 = n_sub;
             // S_t(i) once K^(i) is written and PV_t(i - 1), which reads P_t
-            // from the S_t columns, has completed
+            // from the S_t columns, has been issued: the tensor cores run one
+            // thread's MMAs in issue order, so PV_t(i - 1) has read P_t before
+            // S_t(i) overwrites it, and the commit that reports S_t(i) also
+            // reports PV_t(i - 1) complete (the softmax may then rescale O_t)
             auto try_s = [&](const int t, int& is_t, const int ip_t, const int is_other) {
                 const int i = is_t;
-                if (!(i < n_sub && ip_t == i && mbar_test(&k_full[i & 1], (i >> 1) & 1) &&
-                      (i == 0 || mbar_test(&o_free[t], (i - 1) & 1))))
+                if (!(i < n_sub && ip_t == i && mbar_test(&k_full[i & 1], (i >> 1) & 1)))
                     return false;
                 tc_fence_after();
                 const uint32_t aKh = smem_u32(sK + (i & 1) * kKHalves * kKVBytes), aKl = aKh + kKVBytes;
@@ -390,13 +393,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             };
             const uint64_t t0 = globaltimer_ns();
             for (uint32_t spin = 0; ip0 < n_sub || ip1 < n_sub; ++spin) {
-                // S products first, the tile that is behind first; then PV products
+                // a tile's PV product first, with its next S product right behind
+                // it (it unblocks that tile's softmax soonest); then S products,
+                // the tile that is behind first
+                if (try_pv(0, ip0, is0, ip1)) { try_s(0, is0, ip0, is1); continue; }
+                if (try_pv(1, ip1, is1, ip0)) { try_s(1, is1, ip1, is0); continue; }
                 if (is1 < is0) {
                     if (try_s(1, is1, ip1, is0) || try_s(0, is0, ip0, is1)) continue;
                 } else {
                     if (try_s(0, is0, ip0, is1) || try_s(1, is1, ip1, is0)) continue;
                 }
-                if (try_pv(0, ip0, is0, ip1) || try_pv(1, ip1, is1, ip0)) continue;
                 if ((spin & 255) == 255) {
                     if (*sAbort) { ok = false; break; }
                     if (globaltimer_ns() - t0 > kWaitLimitNs * 4) {
@@ -594,8 +600,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t t_s = taddr + tcol + kColS + lane_off, t_o = taddr + tcol + kColO + lane_off;
         float m_ref = -CUDART_INF_F, l_run = 0.0f;
         for (int i = 0; i < n_sub; ++i) {
-            // S_t(i) is issued only after PV_t(i - 1) completed, so once it has
-            // landed O_t is stable and the S_t columns may take P_t(i)
+            // S_t(i) is issued after PV_t(i - 1) and its commit covers both, so
+            // once it has landed O_t is stable and the S_t columns may take P_t(i)
             const bool bad = fail_wait(&s_full[my_tile], i & 1);
             if (!__all_sync(0xffffffffu, !bad)) break;
             tc_fence_after();
@@ -658,7 +664,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 l_run = fmaf(l_run, alpha, lsum);
                 tmem_st32u(t_s, pk);  // P_t over the first 32 S_t columns (waits for the store)
-                // rescale the row of O_t (stable: PV_t(i - 1) completed before S_t(i) was issued)
+                // rescale the row of O_t (stable: S_t(i) landing means PV_t(i - 1) completed)
                 if (i > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
                     float o[32];
 #pragma unroll 1
