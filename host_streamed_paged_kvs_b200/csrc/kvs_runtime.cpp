@@ -91,7 +91,7 @@ constexpr int kSms = 148;
 
 // Splits of the resident launch and of one ring-chunk launch (each split is an
 // equal share of the launch's half-page stages).
-int res_splits(const kvs_config& c, long R_eff, int n_q) {
+int res_splits(const kvs_config& c, long R_eff, int n_q, bool ring) {
     const long stages = 2 * R_eff;
     if (use_tcgen05(c, n_q)) {
         // one CTA per SM: pick the split count that minimizes waves x stages
@@ -102,6 +102,10 @@ int res_splits(const kvs_config& c, long R_eff, int n_q) {
             const long cost = ((units * sp + kSms - 1) / kSms) * ((stages + sp - 1) / sp);
             if (best_cost < 0 || cost < best_cost) { best = sp; best_cost = cost; }
         }
+        // Beside ring-chunk launches, short resident CTAs (at most 4 raw
+        // stages each): a CTA holds its SM until it ends, and a ring chunk
+        // whose copy has landed must not wait behind a long resident CTA.
+        if (ring) best = std::max(best, std::min(std::min(stages, 32L), (stages + 3) / 4));
         return (int)best;
     }
     if (wide_regime(c, n_q)) return (int)std::min(stages, 8L);
@@ -135,8 +139,8 @@ int zc_splits(const kvs_config& c, long S_zc, int n_q) {
 }
 
 long count_splits(const kvs_config& c, int n_q, long R_eff, long S) {
-    long n = res_splits(c, R_eff, n_q);
     const long S_zc = zero_copy_pages(c, n_q, S), S_ring = S - S_zc;
+    long n = res_splits(c, R_eff, n_q, S_ring > 0 && c.chunk_pages > 0);
     if (S_zc > 0) n += zc_splits(c, S_zc, n_q);
     if (S_ring > 0 && c.chunk_pages > 0) {
         const long full = S_ring / c.chunk_pages, tail = S_ring % c.chunk_pages;
@@ -1148,7 +1152,7 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         d.slot0 = (int)(first_res % R);
         d.page0 = (int)first_res;
         d.n_units = (int)R_eff;
-        const int ns = res_splits(c, R_eff, n_q);
+        const int ns = res_splits(c, R_eff, n_q, S_ring > 0);
         d.n_splits = ns;
         d.split_base = split_base;
         KVS_CK(kv, cudaEventRecord(kv->ev_fork, s));
