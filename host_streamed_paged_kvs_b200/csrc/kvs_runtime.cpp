@@ -91,6 +91,9 @@ constexpr int kSms = 148;
 
 // Splits of the resident launch and of one ring-chunk launch (each split is an
 // equal share of the launch's half-page stages).
+constexpr long kResCtaStages = 4;  // raw stages per resident CTA beside ring launches
+constexpr long kResSplits = 8;     // splits per such resident launch
+
 int res_splits(const kvs_config& c, long R_eff, int n_q, bool ring) {
     const long stages = 2 * R_eff;
     if (use_tcgen05(c, n_q)) {
@@ -102,10 +105,12 @@ int res_splits(const kvs_config& c, long R_eff, int n_q, bool ring) {
             const long cost = ((units * sp + kSms - 1) / kSms) * ((stages + sp - 1) / sp);
             if (best_cost < 0 || cost < best_cost) { best = sp; best_cost = cost; }
         }
-        // Beside ring-chunk launches, short resident CTAs (at most 4 raw
-        // stages each): a CTA holds its SM until it ends, and a ring chunk
-        // whose copy has landed must not wait behind a long resident CTA.
-        if (ring) best = std::max(best, std::min(std::min(stages, 32L), (stages + 3) / 4));
+        // Beside ring-chunk launches the resident pages go in a sequence of
+        // launches of short CTAs (kResCtaStages raw stages each, kResSplits
+        // per launch) that fold into one set of records: a CTA holds its SM
+        // until it ends, and a ring chunk whose copy has landed must not wait
+        // behind a long resident CTA.
+        if (ring) return (int)std::min<long>(stages, kResSplits);
         return (int)best;
     }
     if (wide_regime(c, n_q)) return (int)std::min(stages, 8L);
@@ -1179,11 +1184,28 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
             for (int li = 0; li < c.n_layers; ++li)
                 if (kv->hist_cap[li]) kv->hist_cap[li] = 0;
         }
-        {
+        if (tc && S_ring > 0) {
+            // launches of kResSplits CTAs of kResCtaStages raw stages each, in
+            // page order on the resident stream; later ones fold their partials
+            // into the first one's records (the first is the widest)
+            const long per_launch = ns * kResCtaStages;  // raw stages = 2 per page; even
+            for (long st0 = 0; st0 < 2 * R_eff; st0 += per_launch) {
+                const long n_st = std::min(per_launch, 2 * R_eff - st0);
+                d.slot0 = (int)((first_res + st0 / 2) % R);
+                d.page0 = (int)(first_res + st0 / 2);
+                d.n_units = (int)(n_st / 2);
+                d.n_splits = (int)std::min<long>(ns, n_st);
+                d.accumulate = st0 > 0 ? 1 : 0;
+                TimedScope ts(kv, rstream, kTChunkMma, (uint64_t)(n_st / 2) * kv->page_bytes);
+                KVS_CK(kv, launch_chunk_mma(d, lres.map, d.n_splits, rstream));
+                kv->stats.kernel_launches++;
+            }
+            d.accumulate = 0;
+        } else {
             TimedScope ts(kv, rstream, tc ? kTChunkMma : kTDecodeRes, (uint64_t)R_eff * kv->page_bytes);
             KVS_CK(kv, tc ? launch_chunk_mma(d, lres.map, ns, rstream) : launch_decode(d, lres.map, ns, rstream));
+            kv->stats.kernel_launches++;
         }
-        kv->stats.kernel_launches++;
         split_base += ns;
         kv->stats.bytes_resident_read += (uint64_t)R_eff * kv->page_bytes;
     }
