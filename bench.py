@@ -371,16 +371,20 @@ def run_gpu(args, w: W.Workload):
     dev = torch.device("cuda", local)
 
     L = w.n_layers
-    # decode-width steps with streamed pages can read a share of them in place
+    # steps with streamed pages can read a share of them in place: the decode
+    # share for decode widths, the wide share for the tensor-core path
     r0 = kvs.kvs_resolve_config(kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx,
                                                 n_resident_pages=w.n_resident_pages,
                                                 n_ring_slots=w.n_ring_slots, type_v=w.type_v))[0]
-    zc_able = (w.n_q * (w.n_q_heads // w.n_kv_heads) <= 8 and r0.n_resident_pages < w.n_pages
-               and w.n_ring_slots > 0)
-    zc_pct = (W.ZERO_COPY_PCT if args.zero_copy_pct < 0 else args.zero_copy_pct) if zc_able else 0
+    wide = w.n_q * (w.n_q_heads // w.n_kv_heads) > 8
+    zc_able = r0.n_resident_pages < w.n_pages and w.n_ring_slots > 0
+    tuned = W.ZERO_COPY_PCT_WIDE if wide else W.ZERO_COPY_PCT
+    zc_pct = (tuned if args.zero_copy_pct < 0 else args.zero_copy_pct) if zc_able else 0
+    zc_pct_wide = zc_pct if wide else 0
     cfg = kvs.make_config(L, w.n_q_heads, w.n_kv_heads, w.ctx, n_resident_pages=w.n_resident_pages,
                           n_ring_slots=w.n_ring_slots, max_q_tokens=w.n_q,
-                          chunk_pages=args.chunk_pages, zero_copy_pct=zc_pct, type_v=w.type_v)
+                          chunk_pages=args.chunk_pages, zero_copy_pct=0 if wide else zc_pct,
+                          zero_copy_pct_wide=zc_pct_wide, type_v=w.type_v)
     h = kvs.kvs_create(cfg, local)
     rc = kvs.kvs_get_config(h)
     pb = kvs.kvs_page_bytes(rc)
@@ -503,7 +507,7 @@ def run_gpu(args, w: W.Workload):
         for name, pct in (("ring_only", 0), ("zero_copy_only", 100)):
             if pct == zc_pct:
                 continue
-            kvs.kvs_set_zero_copy_pct(h, pct)
+            kvs.kvs_set_zero_copy_pct(h, -1 if wide else pct, pct if wide else -1)
             for _ in range(args.warmup):
                 one_step(ks, vs, qs, out, lse)
             barrier()
@@ -518,7 +522,7 @@ def run_gpu(args, w: W.Workload):
                           "value": job_value(world, w.ctx, L, ms_a), "unit": UNIT,
                           "h2d_gbs_achieved": L * S_a * pb / (ms_a * 1e-3) / 1e9,
                           "launch": "plain library calls"}
-        kvs.kvs_set_zero_copy_pct(h, zc_pct)
+        kvs.kvs_set_zero_copy_pct(h, 0 if wide else zc_pct, zc_pct_wide)
 
     # ---- end to end through the C ABI with pinned host buffers ----
     kh = [x.cpu().pin_memory() for x in ks]
@@ -583,7 +587,7 @@ def run_gpu(args, w: W.Workload):
         timeline = {}
         shares = [("tuned", zc_pct)] + ([("ring_only", 0)] if zc_able and zc_pct != 0 else [])
         for tag, pct in shares:
-            kvs.kvs_set_zero_copy_pct(h, pct)
+            kvs.kvs_set_zero_copy_pct(h, -1 if wide else pct, pct if wide else -1)
             for _ in range(2):
                 one_step(ks, vs, qs, out, lse)
             path = os.path.join(args.timeline, f"timeline_{w.name}_{tag}.json")
@@ -592,7 +596,7 @@ def run_gpu(args, w: W.Workload):
             timeline[tag] = timeline_summary(path, n_tl, h2d_peak)
             if timeline[tag] is not None:
                 timeline[tag]["zero_copy_pct"] = pct
-        kvs.kvs_set_zero_copy_pct(h, zc_pct)
+        kvs.kvs_set_zero_copy_pct(h, 0 if wide else zc_pct, zc_pct_wide)
 
     hbm_peak, peak_src = peaks()
     P = w.n_pages
@@ -656,11 +660,26 @@ def run_gpu(args, w: W.Workload):
                 "kernel": "decode_kernel (in-place reads of streamed pages)", "launches": n_zc,
                 "avg_launch_us": ms_zc / n_zc * 1e3, "bytes_per_launch": st_prof["bytes_decode_zc"] / n_zc,
                 "peak_note": "best pinned host-to-device copy rate measured in this run"})
+        ms_tz, n_tz = st_prof["ms_chunk_zc"], st_prof["n_chunk_zc"]
+        if n_tz > 0:
+            achieved = st_prof["bytes_chunk_zc"] / (ms_tz * 1e-3) / 1e9
+            kinds["chunk_mma_kernel_in_place"] = (ms_tz, {
+                "bound": "h2d", "bound_note": "the host-to-device PCIe link: the launch reads host memory",
+                "achieved": achieved, "peak": h2d_peak, "unit": "GB/s", "frac": achieved / h2d_peak,
+                "traffic": None, "kernel": "chunk_mma_kernel (in-place reads of streamed pages)",
+                "launches": n_tz, "avg_launch_us": ms_tz / n_tz * 1e3,
+                "bytes_per_launch": st_prof["bytes_chunk_zc"] / n_tz,
+                "peak_note": "best pinned host-to-device copy rate measured in this run"})
         ms_tc, n_tc = st_prof["ms_chunk_mma"], st_prof["n_chunk_mma"]
         if n_tc > 0:
             # algorithmic flops: QK^T and PV over every visible key of every query row
             vis = sum(w.pos0 + j + 1 for j in range(w.n_q))
             flops = prof_steps * L * 4.0 * w.n_q_heads * 128 * vis
+            # the share of the keys these (TMA-fed) launches attend; the
+            # in-place launches attend the rest
+            S_ = w.n_pages - min(rc.n_resident_pages, w.n_pages)
+            S_zc_ = min(S_, (S_ * zc_pct_wide + 50) // 100)
+            flops *= (w.n_pages - S_zc_) / w.n_pages
             achieved = flops / (ms_tc * 1e-3) / 1e12
             tc_peak = peak_tflops()
             n_res_l = prof_steps * L
@@ -696,7 +715,7 @@ def run_gpu(args, w: W.Workload):
                    "kv_types": "K q8_0 / V " + {8: "q8_0", 6: "q5_0", 3: "q4_1", 7: "q5_1"}.get(w.type_v, "q4_0"),
                    "page_tokens": 256, "resident_pages": R,
                    "streamed_pages": S, "ring_slots": rc.n_ring_slots, "chunk_pages": rc.chunk_pages,
-                   "zero_copy_pct": zc_pct,
+                   "zero_copy_pct": zc_pct, "zero_copy_share_of": "tensor-core calls" if wide else "decode calls",
                    "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (resident "
                    f"{L * R * pb / 1e6:.0f} MB + streamed {L * S * pb / 1e6:.0f} MB per step)",
                    },

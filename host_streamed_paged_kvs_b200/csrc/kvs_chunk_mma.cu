@@ -204,7 +204,10 @@ __device__ __forceinline__ uint32_t fifth_bits(uint32_t hw, int j) {
 }
 
 
-template <int VT, int KT>
+// ZC = true: the raw stages are read in place from mapped pinned host memory
+// (the history's device alias) by the load warp's 16-byte asynchronous copies,
+// the K quants placed in the swizzle the tensor map would produce.
+template <int VT, int KT, bool ZC>
 __global__ void __launch_bounds__(kTcThreads, 1)
     chunk_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap) {
     using TG = TcGeom<VT, KT>;
@@ -252,7 +255,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (tid == 32) {
         *sAbort = 0;
         for (int k = 0; k < kMaxRawStages; ++k) {
-            mbar_init(&raw_full[k], 1);
+            mbar_init(&raw_full[k], ZC ? 32 : 1);  // in place: one arrival per load lane
             mbar_init(&raw_free[k], kProdWarps);
         }
         for (int k = 0; k < kKBufs; ++k) {
@@ -310,10 +313,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     };
 
     if (warp == kLoadWarp) {
-        // ============================ TMA load warp ============================
+        // ============================ load warp ============================
         // raw stage r into buffer r % kRS once the producers released the
         // stage that used it before (r - kRS)
-        if (lane == 0) {
+        if (ZC || lane == 0) {
             for (int r = 0; r < n_raw; ++r) {
                 const int buf = r % kRS;
                 if (r >= kRS && fail_wait(&raw_free[buf], ((r - kRS) / kRS) & 1)) break;
@@ -323,20 +326,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const uint8_t* ph = a.region + ((size_t)slot * a.n_kv + h) * PG::kHeadBytes;
                 uint8_t* dst = raw + buf * kRawBytes;
                 uint64_t* b = &raw_full[buf];
-                mbar_expect_tx(b, kRawBytes);
-                const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * PG::kRows + half * TG::kKRows;
+                if constexpr (ZC) {
+                    // K quants (or f16 K values): 128-byte row kr of the half
+                    // page, 16-byte chunk k -> swizzled; the other fields as they lie
+                    const uint8_t* kq = ph + PG::kOffKq + half * (kRawKeys * PG::kKqRow);
+#pragma unroll 4
+                    for (int c = lane; c < TG::kKRows * 8; c += 32) {
+                        const int kr = c >> 3, k = c & 7;
+                        cp_async16(dst + kRawKq + kr * 128 + ((k ^ (kr & 7)) << 4), kq + kr * 128 + k * 16);
+                    }
+                    auto copy_field = [&](int dst_off, int src_off, int row_bytes) {
+                        const uint8_t* src = ph + src_off + half * (kRawKeys * row_bytes);
+                        for (int c = lane; c < kRawKeys * row_bytes / 16; c += 32)
+                            cp_async16(dst + dst_off + c * 16, src + c * 16);
+                    };
+                    if constexpr (PG::kKdRow > 0) copy_field(kRawKd, PG::kOffKd, PG::kKdRow);
+                    copy_field(kRawVq, PG::kOffVq, PG::kVqRow);
+                    if constexpr (PG::kVhRow > 0) copy_field(kRawVh, PG::kOffVh, PG::kVhRow);
+                    if constexpr (PG::kVdRow > 0) copy_field(kRawVd, PG::kOffVd, PG::kVdRow);
+                    if constexpr (PG::kVmRow > 0) copy_field(kRawVm, PG::kOffVm, PG::kVmRow);
+                    cp_async_arrive(b);
+                } else {
+                    mbar_expect_tx(b, kRawBytes);
+                    const int krow = ((a.region_slot_base + slot) * a.n_kv + h) * PG::kRows + half * TG::kKRows;
 #pragma unroll
-                for (int kr = 0; kr < TG::kKRows; kr += 128)  // boxes of 128 rows of 128 B
-                    tma_load_2d(dst + kRawKq + kr * 128, &kmap, 0, krow + kr, b);
-                if constexpr (PG::kKdRow > 0)
-                    bulk_load(dst + kRawKd, ph + PG::kOffKd + half * (kRawKeys * PG::kKdRow), kRawKeys * PG::kKdRow, b);
-                bulk_load(dst + kRawVq, ph + PG::kOffVq + half * (kRawKeys * PG::kVqRow), kRawKeys * PG::kVqRow, b);
-                if constexpr (PG::kVhRow > 0)
-                    bulk_load(dst + kRawVh, ph + PG::kOffVh + half * (kRawKeys * PG::kVhRow), kRawKeys * PG::kVhRow, b);
-                if constexpr (PG::kVdRow > 0)
-                    bulk_load(dst + kRawVd, ph + PG::kOffVd + half * (kRawKeys * kBlocks * 2), kRawKeys * kBlocks * 2, b);
-                if constexpr (PG::kVmRow > 0)
-                    bulk_load(dst + kRawVm, ph + PG::kOffVm + half * (kRawKeys * PG::kVmRow), kRawKeys * PG::kVmRow, b);
+                    for (int kr = 0; kr < TG::kKRows; kr += 128)  // boxes of 128 rows of 128 B
+                        tma_load_2d(dst + kRawKq + kr * 128, &kmap, 0, krow + kr, b);
+                    if constexpr (PG::kKdRow > 0)
+                        bulk_load(dst + kRawKd, ph + PG::kOffKd + half * (kRawKeys * PG::kKdRow), kRawKeys * PG::kKdRow, b);
+                    bulk_load(dst + kRawVq, ph + PG::kOffVq + half * (kRawKeys * PG::kVqRow), kRawKeys * PG::kVqRow, b);
+                    if constexpr (PG::kVhRow > 0)
+                        bulk_load(dst + kRawVh, ph + PG::kOffVh + half * (kRawKeys * PG::kVhRow), kRawKeys * PG::kVhRow, b);
+                    if constexpr (PG::kVdRow > 0)
+                        bulk_load(dst + kRawVd, ph + PG::kOffVd + half * (kRawKeys * kBlocks * 2), kRawKeys * kBlocks * 2, b);
+                    if constexpr (PG::kVmRow > 0)
+                        bulk_load(dst + kRawVm, ph + PG::kOffVm + half * (kRawKeys * PG::kVmRow), kRawKeys * PG::kVmRow, b);
+                }
             }
         }
         __syncwarp();
@@ -738,7 +763,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 }
 
-template <int VT, int KT = kKQ8_0>
+template <int VT, int KT = kKQ8_0, bool ZC = false>
 static cudaError_t launch_chunk_t(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits, cudaStream_t s) {
     // devices whose shared-memory opt-in is done (calls from several host
     // threads may race to set a bit; the attribute call is idempotent)
@@ -746,29 +771,38 @@ static cudaError_t launch_chunk_t(const DecodeArgs& a, const CUtensorMap* kmap, 
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !(configured.load(std::memory_order_acquire) & (1ull << dev))) {
-        const cudaError_t e = cudaFuncSetAttribute(chunk_mma_kernel<VT, KT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        const cudaError_t e = cudaFuncSetAttribute(chunk_mma_kernel<VT, KT, ZC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                    (int)TcGeom<VT, KT>::kSmem);
         if (e != cudaSuccess) return e;
         if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_acq_rel);
     }
     const int m_tiles = (a.n_q * a.group + kMTile - 1) / kMTile;
     dim3 grid(n_splits, a.n_kv, (m_tiles + kTiles - 1) / kTiles);
-    chunk_mma_kernel<VT, KT><<<grid, kTcThreads, TcGeom<VT, KT>::kSmem, s>>>(a, *kmap);
+    chunk_mma_kernel<VT, KT, ZC><<<grid, kTcThreads, TcGeom<VT, KT>::kSmem, s>>>(a, *kmap);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits, cudaStream_t s) {
-    if (a.k_type == kKF16) return launch_chunk_t<kVF16, kKF16>(a, kmap, n_splits, s);
+template <bool ZC>
+static cudaError_t launch_chunk_types(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits, cudaStream_t s) {
+    if (a.k_type == kKF16) return launch_chunk_t<kVF16, kKF16, ZC>(a, kmap, n_splits, s);
     switch (a.v_type) {
-        case kVQ8_0: return launch_chunk_t<kVQ8_0>(a, kmap, n_splits, s);
-        case kVQ5_0: return launch_chunk_t<kVQ5_0>(a, kmap, n_splits, s);
-        case kVQ4_1: return launch_chunk_t<kVQ4_1>(a, kmap, n_splits, s);
-        case kVQ5_1: return launch_chunk_t<kVQ5_1>(a, kmap, n_splits, s);
-        case kVF16: return launch_chunk_t<kVF16>(a, kmap, n_splits, s);
-        default: return launch_chunk_t<kVQ4_0>(a, kmap, n_splits, s);
+        case kVQ8_0: return launch_chunk_t<kVQ8_0, kKQ8_0, ZC>(a, kmap, n_splits, s);
+        case kVQ5_0: return launch_chunk_t<kVQ5_0, kKQ8_0, ZC>(a, kmap, n_splits, s);
+        case kVQ4_1: return launch_chunk_t<kVQ4_1, kKQ8_0, ZC>(a, kmap, n_splits, s);
+        case kVQ5_1: return launch_chunk_t<kVQ5_1, kKQ8_0, ZC>(a, kmap, n_splits, s);
+        case kVF16: return launch_chunk_t<kVF16, kKQ8_0, ZC>(a, kmap, n_splits, s);
+        default: return launch_chunk_t<kVQ4_0, kKQ8_0, ZC>(a, kmap, n_splits, s);
     }
+}
+
+cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits, cudaStream_t s) {
+    return launch_chunk_types<false>(a, kmap, n_splits, s);
+}
+
+cudaError_t launch_chunk_mma_zero_copy(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits, cudaStream_t s) {
+    return launch_chunk_types<true>(a, kmap, n_splits, s);
 }
 
 }  // namespace kvs

@@ -200,6 +200,9 @@ cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s);
 // arguments and partial format as launch_decode
 cudaError_t launch_chunk_mma(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
                              cudaStream_t s);
+// the same kernel reading the pages in place from mapped pinned host memory
+cudaError_t launch_chunk_mma_zero_copy(const DecodeArgs& a, const CUtensorMap* kmap, int n_splits,
+                                       cudaStream_t s);
 size_t decode_smem_bytes();
 
 // bounded-wait self-test kernel (one thread, an mbarrier nothing completes)

@@ -134,11 +134,20 @@ int ring_splits(const kvs_config& c, int n_q, int chunk_pages) {
 // ones nearest the resident window) are read in place by one launch, about one
 // CTA per SM (the resident and ring launches share the SMs); the ring brings
 // the older ones.
+// Calls on the tensor-core path take the wide share; their in-place launch
+// keeps to about kZcTcCtas CTAs (one per SM), leaving SMs to the resident and
+// ring launches beside it.
+constexpr int kZcTcCtas = 120;
 long zero_copy_pages(const kvs_config& c, int n_q, long S) {
-    if (use_tcgen05(c, n_q) || c.zero_copy_pct <= 0) return 0;
-    return std::min(S, (S * c.zero_copy_pct + 50) / 100);
+    const int pct = use_tcgen05(c, n_q) ? c.zero_copy_pct_wide : c.zero_copy_pct;
+    if (pct <= 0) return 0;
+    return std::min(S, (S * pct + 50) / 100);
 }
 int zc_splits(const kvs_config& c, long S_zc, int n_q) {
+    if (use_tcgen05(c, n_q)) {
+        const long units = (long)c.n_kv_heads * tile_pairs(c, n_q);
+        return (int)std::min(2 * S_zc, std::max(1L, (long)kZcTcCtas / units));
+    }
     const long per_split = (long)c.n_kv_heads * ((n_q * (c.n_q_heads / c.n_kv_heads) + 7) / 8);
     return (int)std::min(2 * S_zc, std::max(1L, (long)kSms / per_split));
 }
@@ -172,10 +181,14 @@ size_t partial_records_r(const kvs_config& c, long R) {
     size_t best = 1;
     for (int n_q = 1; n_q <= c.max_q_tokens; ++n_q) {
         kvs_config cz = c;
-        // the share only matters for decode widths
-        const int shares = use_tcgen05(c, n_q) ? 1 : 101;
-        for (int pct = 0; pct < shares; ++pct) {
-            if (shares > 1) cz.zero_copy_pct = pct;
+        const bool tc = use_tcgen05(c, n_q);
+        // decode widths: every share; wider calls: ring only, in place only, and
+        // both together bound the counts (the in-place and ring launches have
+        // fixed split counts there)
+        const int shares = tc ? 3 : 101;
+        for (int k = 0; k < shares; ++k) {
+            if (tc) cz.zero_copy_pct_wide = k * 50;
+            else cz.zero_copy_pct = k;
             best = std::max(best, (size_t)count_splits(cz, n_q, R_eff, S) * (size_t)(n_q * c.n_q_heads));
         }
     }
@@ -260,8 +273,8 @@ int resolve(const kvs_config* in, kvs_config* out, size_t* host_bytes, std::stri
         why = "negative page counts";
         return KVS_E_INVAL;
     }
-    if (c.zero_copy_pct < 0 || c.zero_copy_pct > 100) {
-        why = fmt("zero_copy_pct %d outside 0..100", c.zero_copy_pct);
+    if (c.zero_copy_pct < 0 || c.zero_copy_pct > 100 || c.zero_copy_pct_wide < 0 || c.zero_copy_pct_wide > 100) {
+        why = fmt("zero_copy_pct %d / zero_copy_pct_wide %d outside 0..100", c.zero_copy_pct, c.zero_copy_pct_wide);
         return KVS_E_INVAL;
     }
     // a phase arena: a fixed budget with the resident set fitted to it (a
@@ -390,7 +403,7 @@ struct LayerState {
     bool hist_recorded = false;
 };
 
-enum TimedKind { kTDecodeRes, kTDecodeRing, kTMerge, kTAppend, kTChunkMma, kTDecodeZc };
+enum TimedKind { kTDecodeRes, kTDecodeRing, kTMerge, kTAppend, kTChunkMma, kTDecodeZc, kTChunkZc };
 
 struct Timed {
     cudaEvent_t a, b;
@@ -722,6 +735,8 @@ void fold_timed_upto(kvs_t* kv, size_t n) {
             case kTChunkMma: kv->stats.ms_chunk_mma += ms; kv->stats.n_chunk_mma++; break;
             case kTDecodeZc: kv->stats.ms_decode_zc += ms; kv->stats.n_decode_zc++;
                              kv->stats.bytes_decode_zc += t.bytes; break;
+            case kTChunkZc: kv->stats.ms_chunk_zc += ms; kv->stats.n_chunk_zc++;
+                            kv->stats.bytes_chunk_zc += t.bytes; break;
         }
         kv->ev_pool.push_back(t.a);
         kv->ev_pool.push_back(t.b);
@@ -1226,8 +1241,9 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         d.n_splits = ns;
         d.split_base = split_base;
         {
-            TimedScope ts(kv, zstream, kTDecodeZc, (uint64_t)S_zc * kv->page_bytes);
-            KVS_CK(kv, launch_decode_zero_copy(d, &kv->map_res, ns, zstream));
+            TimedScope ts(kv, zstream, tc ? kTChunkZc : kTDecodeZc, (uint64_t)S_zc * kv->page_bytes);
+            KVS_CK(kv, tc ? launch_chunk_mma_zero_copy(d, &kv->map_res, ns, zstream)
+                          : launch_decode_zero_copy(d, &kv->map_res, ns, zstream));
         }
         KVS_CK(kv, cudaEventRecord(kv->ev_zc, zstream));
         kv->stats.kernel_launches++;
@@ -1427,10 +1443,13 @@ int kvs_reset_stats(kvs_t* kv) {
     return KVS_OK;
 }
 
-int kvs_set_zero_copy_pct(kvs_t* kv, int pct) {
+int kvs_set_zero_copy_pct(kvs_t* kv, int pct, int pct_wide) {
     if (!kv) return fail(nullptr, KVS_E_INVAL, "null handle");
-    if (pct < 0 || pct > 100) return fail(kv, KVS_E_INVAL, fmt("zero_copy_pct %d outside 0..100", pct));
-    kv->cfg.zero_copy_pct = pct;  // the partial buffer is sized for every share
+    if (pct < -1 || pct > 100 || pct_wide < -1 || pct_wide > 100)
+        return fail(kv, KVS_E_INVAL, fmt("in-place shares %d / %d outside -1..100", pct, pct_wide));
+    // the partial buffer is sized for every share
+    if (pct >= 0) kv->cfg.zero_copy_pct = pct;
+    if (pct_wide >= 0) kv->cfg.zero_copy_pct_wide = pct_wide;
     return KVS_OK;
 }
 

@@ -59,7 +59,7 @@ class kvs_config(ctypes.Structure):
                 ("type_v", ctypes.c_int), ("chunk_pages", ctypes.c_int),
                 ("flags", ctypes.c_int), ("zero_copy_pct", ctypes.c_int),
                 ("arena_bytes", ctypes.c_size_t), ("n_aux_layers", ctypes.c_int),
-                ("aux_resident_pages", ctypes.c_int)]
+                ("aux_resident_pages", ctypes.c_int), ("zero_copy_pct_wide", ctypes.c_int)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -84,7 +84,9 @@ class kvs_stats(ctypes.Structure):
                   "ms_decode_zc")] +
                 [(n, ctypes.c_uint64) for n in
                  ("n_decode_resident", "n_decode_ring", "n_merge", "n_append", "n_chunk_mma",
-                  "n_decode_zc", "bytes_decode_resident", "bytes_decode_ring", "bytes_decode_zc")])
+                  "n_decode_zc", "bytes_decode_resident", "bytes_decode_ring", "bytes_decode_zc")] +
+                [("ms_chunk_zc", ctypes.c_double), ("n_chunk_zc", ctypes.c_uint64),
+                 ("bytes_chunk_zc", ctypes.c_uint64)])
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -122,7 +124,7 @@ def _load():
     L.kvs_get_stats.argtypes = [vp, cp(kvs_stats)]
     L.kvs_reset_stats.argtypes = [vp]
     L.kvs_set_profiling.argtypes = [vp, i]
-    L.kvs_set_zero_copy_pct.argtypes = [vp, i]
+    L.kvs_set_zero_copy_pct.argtypes = [vp, i, i]
     L.kvs_sync.argtypes = [vp, vp, ctypes.c_double]
     L.kvs_measure_h2d.argtypes = [vp, ctypes.c_size_t, ctypes.c_size_t, i, cp(ctypes.c_double)]
     L.kvs_attend_pages_static.argtypes = [vp, i, i, i, i, i, i, vp, vp, vp, vp]
@@ -179,10 +181,12 @@ def _check(rc: int, handle=None):
 def make_config(n_layers, n_q_heads, n_kv_heads, max_ctx, n_resident_pages=0, n_ring_slots=0,
                 max_q_tokens=1, chunk_pages=0, flags=0, arena_bytes=0, head_dim=128,
                 page_tokens=256, type_k=KVS_TYPE_Q8_0, type_v=KVS_TYPE_Q4_0,
-                zero_copy_pct=0, n_aux_layers=0, aux_resident_pages=0) -> kvs_config:
+                zero_copy_pct=0, n_aux_layers=0, aux_resident_pages=0,
+                zero_copy_pct_wide=0) -> kvs_config:
     return kvs_config(n_layers, n_q_heads, n_kv_heads, head_dim, page_tokens, max_ctx,
                       n_resident_pages, n_ring_slots, max_q_tokens, type_k, type_v, chunk_pages,
-                      flags, zero_copy_pct, arena_bytes, n_aux_layers, aux_resident_pages)
+                      flags, zero_copy_pct, arena_bytes, n_aux_layers, aux_resident_pages,
+                      zero_copy_pct_wide)
 
 
 # ---- functions with the C names ------------------------------------------
@@ -258,8 +262,9 @@ def kvs_set_profiling(h, enable: bool) -> None:
     _check(lib.kvs_set_profiling(h, int(bool(enable))), h)
 
 
-def kvs_set_zero_copy_pct(h, pct: int) -> None:
-    _check(lib.kvs_set_zero_copy_pct(h, int(pct)), h)
+def kvs_set_zero_copy_pct(h, pct: int = -1, pct_wide: int = -1) -> None:
+    """In-place shares for decode calls and wider calls; -1 leaves one unchanged."""
+    _check(lib.kvs_set_zero_copy_pct(h, int(pct), int(pct_wide)), h)
 
 
 def kvs_phase_layout(cfg: kvs_config, width: int, pinned_bytes: int = 0, draft_active: bool = True) -> dict:

@@ -103,6 +103,9 @@ DEFAULT_BENCH = "long_decode_256k"
 # copying ahead into the next layer.  Tuned on the 32K streamed decode
 # workload (70-90 % within noise of each other, ring-only 4 % slower).
 ZERO_COPY_PCT = 80
+# The same share for the wider calls of the tensor-core path (verify batches,
+# prefill chunks), whose in-place launch holds about 120 of the 148 SMs.
+ZERO_COPY_PCT_WIDE = 100
 
 
 def _page_kv(w: Workload, layer: int, page: int):

@@ -111,8 +111,8 @@ typedef struct kvs_config {
                              no per-copy cost; the ring can copy ahead into the next layer.
                              100 = no ring copies for decode (the design the "Feature/adaptive
                              kv stream integration" pull request's review found in its
-                             kernels).  Wider calls always use the ring, so a ring is still
-                             required when pages stream. */
+                             kernels).  Wider calls take zero_copy_pct_wide instead; a ring
+                             is still required when pages stream. */
     size_t arena_bytes;   /* device arena budget; 0 = exact fit; else must hold one page and all
                              resident pages + ring + partials + staging (KVS_E_ARENA if not).
                              With n_resident_pages = 0 the handle runs a phase arena: it
@@ -125,6 +125,10 @@ typedef struct kvs_config {
                              the pool; 0 = none */
     int aux_resident_pages; /* resident pages per auxiliary layer (in the pinned region); 0 = the
                              10 % rule of the target layers */
+    int zero_copy_pct_wide; /* 0..100: the in-place share, as zero_copy_pct, for calls wider than
+                             decode (verify batches, prefill chunks: the tensor-core kernel),
+                             whose in-place launch reads its pages over PCIe with 16-byte
+                             asynchronous copies; 0 = those calls stream through the ring only */
 } kvs_config;
 
 /* ---- phase arena ------------------------------------------------------------
@@ -171,6 +175,9 @@ typedef struct kvs_stats {
     double ms_decode_resident, ms_decode_ring, ms_merge, ms_append, ms_chunk_mma, ms_decode_zc;
     uint64_t n_decode_resident, n_decode_ring, n_merge, n_append, n_chunk_mma, n_decode_zc;
     uint64_t bytes_decode_resident, bytes_decode_ring, bytes_decode_zc; /* page bytes read */
+    /* the tensor-core kernel's launches that read streamed pages in place */
+    double ms_chunk_zc;
+    uint64_t n_chunk_zc, bytes_chunk_zc;
 } kvs_stats;
 
 typedef struct kvs_s kvs_t;
@@ -306,12 +313,13 @@ int kvs_get_config(kvs_t* kv, kvs_config* out);
 int kvs_get_stats(kvs_t* kv, kvs_stats* out);
 int kvs_reset_stats(kvs_t* kv);
 
-/* Change the in-place share of decode calls' streamed pages (kvs_config
- * zero_copy_pct, 0..100) for later calls, e.g. to compare the copy-engine ring
- * alone (0) with in-place reads alone (100) on one handle.  The split
- * partials are sized for every share at kvs_create.  KVS_E_INVAL outside
- * 0..100.  A CUDA graph captured earlier keeps the share it was captured with. */
-int kvs_set_zero_copy_pct(kvs_t* kv, int pct);
+/* Change the in-place shares of streamed pages (kvs_config zero_copy_pct for
+ * decode calls and zero_copy_pct_wide for wider calls, 0..100; -1 leaves a
+ * share as it is) for later calls, e.g. to compare the copy-engine ring alone
+ * (0) with in-place reads alone (100) on one handle.  The split partials are
+ * sized for every share at kvs_create.  KVS_E_INVAL outside -1..100.  A CUDA
+ * graph captured earlier keeps the shares it was captured with. */
+int kvs_set_zero_copy_pct(kvs_t* kv, int pct, int pct_wide);
 
 /* Pure host: the layout a phase arena (resolved config with a budget and
  * auto resident pages) takes for a phase of the given width (1..max_q_tokens)

@@ -59,10 +59,10 @@ def test_header_constants_match_binding_and_oracle(kvs):
 
 
 def test_struct_sizes_match_header(kvs):
-    # 14 ints + size_t + 2 ints (padded to 8) ; 8 u64, 6 double, 9 u64
-    assert ctypes.sizeof(kvs.kvs_config) == 14 * 4 + 8 + 2 * 4
+    # 14 ints + size_t + 3 ints (padded to 8) ; 8 u64, 6 double, 9 u64, double + 2 u64
+    assert ctypes.sizeof(kvs.kvs_config) == 14 * 4 + 8 + 3 * 4 + 4
     assert ctypes.sizeof(kvs.kvs_arena_status) == 6 * 4 + 7 * 8
-    assert ctypes.sizeof(kvs.kvs_stats) == (8 + 6 + 9) * 8
+    assert ctypes.sizeof(kvs.kvs_stats) == (8 + 6 + 9 + 3) * 8
 
 
 def test_auto_resident_matches_oracle_and_pages(kvs):
@@ -218,7 +218,10 @@ def test_static_entry_rejects_misaligned_pointers_on_the_host(kvs):
 
 
 def test_zero_copy_share_setter_range(kvs):
-    assert kvs.lib.kvs_set_zero_copy_pct(None, 10) == kvs.KVS_E_INVAL
+    assert kvs.lib.kvs_set_zero_copy_pct(None, 10, -1) == kvs.KVS_E_INVAL
+    for over in (dict(zero_copy_pct_wide=101), dict(zero_copy_pct_wide=-1)):
+        with pytest.raises(kvs.KvsError):
+            kvs.kvs_resolve_config(kvs.make_config(1, 8, 2, 1000, n_ring_slots=2, **over))
 
 
 def test_f16_f16_pair_geometry_and_gates(kvs):

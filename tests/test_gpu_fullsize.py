@@ -19,17 +19,21 @@ def kvs():
     return K
 
 
-def bench_pct(w):
-    """The in-place share bench.py gives this workload: the tuned share for
-    decode-width steps with streamed pages, else none."""
-    decode = w.n_q * (w.n_q_heads // w.n_kv_heads) <= 8
-    return W.ZERO_COPY_PCT if decode and w.n_ring_slots > 0 else 0
+def bench_shares(w):
+    """The in-place shares bench.py gives this workload: the tuned share of its
+    width (decode or the tensor-core path) when pages stream, else none."""
+    if w.n_ring_slots == 0:
+        return 0, 0
+    if w.n_q * (w.n_q_heads // w.n_kv_heads) <= 8:
+        return W.ZERO_COPY_PCT, 0
+    return 0, W.ZERO_COPY_PCT_WIDE
 
 
 def _full(kvs, name, layers, sample_q=None):
     t = torch()
     w = W.WORKLOADS[name]
-    h = kvs.kvs_create(make_cfg(w, zero_copy_pct=bench_pct(w), type_v=w.type_v), 0)
+    pct, pct_wide = bench_shares(w)
+    h = kvs.kvs_create(make_cfg(w, zero_copy_pct=pct, zero_copy_pct_wide=pct_wide, type_v=w.type_v), 0)
     try:
         for layer in layers:
             prefill(h, w, layer, w.pos0)

@@ -72,6 +72,41 @@ def test_wide_calls_keep_the_ring(kvs):
         kvs.kvs_destroy(h)
 
 
+@pytest.mark.parametrize("n_q,ctx,R,N,pct", [
+    (4, 5000, 3, 4, 100),     # verify width: one M tile per kv head, every streamed page in place
+    (4, 5000, 3, 4, 60),      # in place and through the ring in one call
+    (64, 3000, 2, 4, 100),    # three M tiles: two tile pairs per kv head
+    (256, 6000, 4, 8, 80),    # a prefill chunk: ten M tiles
+])
+def test_wide_zero_copy_matches_oracle_and_ring(kvs, n_q, ctx, R, N, pct):
+    """Calls on the tensor-core path read the wide share of the streamed pages
+    in place (16-byte asynchronous copies from the mapped history): parity with
+    the oracle (sampled query tokens in every tile for wide batches) and with the
+    ring-only path on the same inputs."""
+    w = W.Workload("zcwide", n_layers=1, n_q=n_q, n_q_heads=40, n_kv_heads=8, ctx=ctx,
+                   n_resident_pages=R, n_ring_slots=N, seed=44)
+    hz = kvs.kvs_create(make_cfg(w, zero_copy_pct_wide=pct), 0)
+    hr = kvs.kvs_create(make_cfg(w), 0)
+    try:
+        for h in (hz, hr):
+            prefill(h, w, 0, w.pos0)
+        oz, lz = step(hz, w, 0, w.pos0, n_q)
+        orr, lr = step(hr, w, 0, w.pos0, n_q)
+        ro, rl = oracle_step(w, 0, w.pos0, n_q)
+        rows = range(n_q) if n_q <= 4 else sorted({0, n_q // 3, n_q // 2, n_q - 1} | set(range(0, n_q, 26)))
+        for j in rows:
+            assert_close(oz[j:j + 1], lz[j:j + 1], ro[j:j + 1], rl[j:j + 1])
+        assert np.allclose(oz, orr, rtol=0, atol=2e-5) and np.allclose(lz, lr, rtol=0, atol=2e-5)
+        st = kvs.kvs_get_stats(hz)
+        S = w.n_pages - R
+        zc = min(S, (S * pct + 50) // 100)
+        assert st["pages_streamed"] == S
+        assert (st["h2d_copies"] == 0) == (zc == S)
+    finally:
+        kvs.kvs_destroy(hz)
+        kvs.kvs_destroy(hr)
+
+
 def test_zero_copy_full_size_32k_layer(kvs):
     """The 32K decode workload's layer 0 in the bench configuration, a share of
     the streamed pages in place."""
