@@ -96,7 +96,10 @@ def test_wide_zero_copy_matches_oracle_and_ring(kvs, n_q, ctx, R, N, pct):
         rows = range(n_q) if n_q <= 4 else sorted({0, n_q // 3, n_q // 2, n_q - 1} | set(range(0, n_q, 26)))
         for j in rows:
             assert_close(oz[j:j + 1], lz[j:j + 1], ro[j:j + 1], rl[j:j + 1])
-        assert np.allclose(oz, orr, rtol=0, atol=2e-5) and np.allclose(lz, lr, rtol=0, atol=2e-5)
+        # same arithmetic, other split layout: each split keeps its own
+        # reference max, so P rounds to fp16 at other scales (out within
+        # 2^-11 of the weights' share); l is summed in fp32 before rounding
+        assert np.allclose(oz, orr, rtol=0, atol=1e-4) and np.allclose(lz, lr, rtol=0, atol=2e-5)
         st = kvs.kvs_get_stats(hz)
         S = w.n_pages - R
         zc = min(S, (S * pct + 50) // 100)
