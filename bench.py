@@ -35,42 +35,59 @@ METRIC = "streamed decode-attn KV tokens/s/layer; % of max(HBM,H2D) roofline, 1x
 UNIT = "KV tokens/s/layer"
 
 
-# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# the ncu captures summarized under profiles/.  A figure is used only for the
-# workload it was captured on and only while the kernel source is unchanged
-# (sha256 prefix of the .cu file); otherwise traffic is reported as null.
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the launches
+# captured with ncu and summarized under profiles/, as (bytes, pages the launch
+# attended).  A launch of another size is scaled by its pages (the traffic of
+# these launches grows with the pages they read); the decode kernel's figures
+# serve every workload with the captured page format, the tensor-core kernel's
+# only the captured workload (its re-reads depend on the query tiles).  A
+# figure is used only while the kernel source is unchanged (sha256 prefix of
+# the .cu file); otherwise traffic is reported as null.
 NCU_TRAFFIC = {
-    "decode_kernel": {"src": "kvs_kernels.cu", "sha": "afede6bf62475eb3",
-                      "workload": "streamed_decode_32k", "resident": 27296256, "ring": 1737472,
-                      # in-place launches (51 pages): DRAM bytes, and host-memory bytes read over PCIe
-                      "in_place": 35328, "in_place_sysmem": 21725184},
-    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "d15b6e259e840f49",
-                         "workload": "prefill_chunk_64k", "resident": 35606272, "ring": 6079232},
+    "decode_kernel": {"src": "kvs_kernels.cu", "sha": "fa1a72c4e1cd72cf",
+                      "workload": "streamed_decode_32k", "type_v": 2,
+                      "resident": (27297280, 64), "ring": (1737472, 4),
+                      # in-place launch: DRAM bytes (Q and split records; they do not grow
+                      # with the pages), and host-memory bytes read over PCIe
+                      "in_place": (86272, 51), "in_place_pcie": (23763968, 51)},
+    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "2a0a2ccd8250adad",
+                         "workload": "prefill_chunk_64k", "type_v": 2,
+                         "resident": (52743168, 16), "ring": (6115072, 8)},
 }
 
 
-def ncu_traffic(kernel: str, workload: str, n_resident: int, n_ring: int):
+def _ncu_entry(kernel: str, w, same_workload: bool):
     import hashlib
     t = NCU_TRAFFIC.get(kernel)
-    if not t or t["workload"] != workload or n_resident + n_ring == 0:
+    if not t or t["type_v"] != w.type_v or (same_workload and t["workload"] != w.name):
         return None
     path = os.path.join(ROOT, "host_streamed_paged_kvs_b200", "csrc", t["src"])
     with open(path, "rb") as f:
         if hashlib.sha256(f.read()).hexdigest()[:16] != t["sha"]:
             return None
-    return (n_resident * t["resident"] + n_ring * t["ring"]) / (n_resident + n_ring)
+    return t
 
 
-def ncu_in_place(workload: str, field: str):
-    """Per-launch traffic of the in-place decode launches, same guards as ncu_traffic."""
-    import hashlib
-    t = NCU_TRAFFIC["decode_kernel"]
-    if t["workload"] != workload:
+def ncu_traffic(kernel: str, w, page_bytes: int, res_bytes: float, ring_bytes: float, n_launches: int):
+    """Average DRAM traffic of one launch: the captured bytes per page of the
+    resident and ring launches applied to the page bytes these launches read."""
+    t = _ncu_entry(kernel, w, same_workload=(kernel != "decode_kernel"))
+    if t is None or n_launches == 0:
         return None
-    with open(os.path.join(ROOT, "host_streamed_paged_kvs_b200", "csrc", t["src"]), "rb") as f:
-        if hashlib.sha256(f.read()).hexdigest()[:16] != t["sha"]:
-            return None
-    return t[field]
+    per_page = {k: t[k][0] / (t[k][1] * page_bytes) for k in ("resident", "ring")}
+    return (per_page["resident"] * res_bytes + per_page["ring"] * ring_bytes) / n_launches
+
+
+def ncu_in_place(w, page_bytes: int, field: str, pages_per_launch: float):
+    """Traffic of one in-place decode launch: its DRAM bytes as captured, or its
+    PCIe reads scaled by the pages it reads."""
+    t = _ncu_entry("decode_kernel", w, same_workload=False)
+    if t is None:
+        return None
+    if field == "dram":
+        return t["in_place"][0]
+    b, n = t["in_place_pcie"]
+    return b / n * pages_per_launch
 
 
 def reduce_max(x: float, dist=None, device=None) -> float:
@@ -632,8 +649,8 @@ def run_gpu(args, w: W.Workload):
             kinds["decode_kernel"] = (ms_dec, {
                 "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak,
-                "traffic": ncu_traffic("decode_kernel", w.name, st_prof["n_decode_resident"],
-                                       st_prof["n_decode_ring"]),
+                "traffic": ncu_traffic("decode_kernel", w, pb, st_prof["bytes_decode_resident"],
+                                       st_prof["bytes_decode_ring"], n_dec),
                 "kernel": "decode_kernel", "launches": n_dec, "avg_launch_us": ms_dec / n_dec * 1e3,
                 "bytes_per_launch": bytes_k / n_dec,
                 "resident_only": {
@@ -643,10 +660,7 @@ def run_gpu(args, w: W.Workload):
         ms_zc, n_zc = st_prof["ms_decode_zc"], st_prof["n_decode_zc"]
 
         def zc_traffic(kind):
-            # the capture's figures hold for this workload at the tuned share only
-            if zc_pct != W.ZERO_COPY_PCT:
-                return None
-            return ncu_in_place(w.name, "in_place" if kind == "dram" else "in_place_sysmem")
+            return ncu_in_place(w, pb, kind, st_prof["bytes_decode_zc"] / pb / n_zc)
 
         if n_zc > 0:
             achieved = st_prof["bytes_decode_zc"] / (ms_zc * 1e-3) / 1e9
@@ -654,9 +668,10 @@ def run_gpu(args, w: W.Workload):
                 "bound": "h2d", "bound_note": "the host-to-device PCIe link: the launch reads host memory",
                 "achieved": achieved, "peak": h2d_peak, "unit": "GB/s",
                 "frac": achieved / h2d_peak, "traffic": zc_traffic("dram"),
-                "sysmem_traffic": zc_traffic("sysmem"),
-                "traffic_note": "traffic: DRAM bytes of a launch (the split partials); sysmem_traffic: "
-                                "host-memory bytes it read over PCIe (ncu sysmem sectors x 32 B)",
+                "sysmem_traffic": zc_traffic("pcie"),
+                "traffic_note": "traffic: DRAM bytes of a launch (Q and the split partials); "
+                                "sysmem_traffic: host-memory bytes it reads over PCIe (ncu "
+                                "pcie__read_bytes.sum per page of the capture x its pages)",
                 "kernel": "decode_kernel (in-place reads of streamed pages)", "launches": n_zc,
                 "avg_launch_us": ms_zc / n_zc * 1e3, "bytes_per_launch": st_prof["bytes_decode_zc"] / n_zc,
                 "peak_note": "best pinned host-to-device copy rate measured in this run"})
@@ -682,11 +697,12 @@ def run_gpu(args, w: W.Workload):
             flops *= (w.n_pages - S_zc_) / w.n_pages
             achieved = flops / (ms_tc * 1e-3) / 1e12
             tc_peak = peak_tflops()
-            n_res_l = prof_steps * L
+            res_b = prof_steps * L * min(rc.n_resident_pages, w.n_pages) * pb
+            ring_b = prof_steps * L * (S_ - S_zc_) * pb
             kinds["chunk_mma_kernel"] = (ms_tc, {
                 "bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": achieved / tc_peak,
-                "traffic": ncu_traffic("chunk_mma_kernel", w.name, n_res_l, n_tc - n_res_l),
+                "traffic": ncu_traffic("chunk_mma_kernel", w, pb, res_b, ring_b, n_tc),
                 "kernel": "chunk_mma_kernel", "launches": n_tc, "avg_launch_us": ms_tc / n_tc * 1e3,
                 "flops_per_launch": flops / n_tc,
                 "peak_note": "measured dense bf16 burst; fp16 has the same nominal rate"})

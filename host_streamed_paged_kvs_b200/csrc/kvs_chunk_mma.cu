@@ -12,12 +12,14 @@
 // 64-key sub-stages, handing work to each other only through mbarriers:
 //
 //   softmax warps 0..3 (tile 0) and 4..7 (tile 1), thread = query row = TMEM
-//     lane, whole 64-key rows: put the tile's Q into tensor memory once, then
+//     lane, whole 64-key rows: put the tile's Q into tensor memory once (and
+//     report it on the tile's Q barrier: the loads and dequantization start
+//     without waiting for Q), then
 //     per sub-stage read S, apply the causal mask and the 1/sqrt(128) scale in
 //     the log2 domain, keep a per-row reference max that only moves when the
 //     row max exceeds it by more than 2^8 (then rescale the row of O in TMEM),
 //     and write P in fp16 over the S columns just read;
-//   producer warps 8..13
+//   producer warps 8, 9, 11, 12, 13 and 15
 //     dequantize each 64-key half of a raw Q8_0/Q4_0 stage (128 keys, landed
 //     by TMA, three raw stages in flight where shared memory allows, else two)
 //     into fp16 UMMA operand tiles with the 128-byte swizzle:
@@ -27,7 +29,7 @@
 //       complete);
 //       V^ = fp16(d*(q4-8)) as [keys][dims] (read as an MN-major B operand;
 //       three buffers, free again once both tiles' PV MMAs complete);
-//   MMA warp 14 (one elected lane)
+//   MMA warp 10 (one elected lane)
 //     polls the barriers without blocking and issues, whichever is ready
 //     first: S_t = Q_t K^_hi^T + Q_t K^_lo^T (tcgen05.mma M=128 N=64 K=16,
 //     A = Q_t from tensor memory, fp32 accumulate) of tile t once the K^
@@ -36,7 +38,7 @@
 //     and O_t += P_t V^ (M=128 N=128 K=16, A = P_t from tensor memory) once
 //     the softmax wrote P_t and V^ is written, with the tile's next S right
 //     behind it.  Only the B operands (K^, V^) are read from shared memory;
-//   load warp 15 (one lane)
+//   load warp 14 (one lane)
 //     issues each raw stage (a TMA tile of the K quants, bulk copies of the
 //     other fields) as soon as the producers release its buffer, so the loads
 //     never wait behind the MMA issue.
@@ -45,7 +47,16 @@
 // fp32 columns) at +0, S_t (64) at +128 with P_t (fp16 pairs, 32) over its
 // first half, Q_t (fp16 pairs, 64) at +192.
 // At the end O, m, l of every valid row are written as the split's partials
-// for the LSE merge.  No cluster, no multicast.
+// for the LSE merge, each warp's 32 rows staged in shared memory so that a
+// record row (and the previous record folded into it) moves as whole 128-byte
+// lines.  No cluster, no multicast.
+//
+// Warp w issues on sub-partition w mod 4 of the SM, and every softmax warp's
+// arithmetic there delays the tensor-core issue of an MMA warp on the same
+// sub-partition (each sub-partition holds two softmax warps: the lane
+// quarter a warp may read from tensor memory is w mod 4).  So the MMA and load
+// warps share sub-partition 2 and the producers' dequantization runs on the
+// other three.
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
@@ -61,9 +72,11 @@ constexpr int kTiles = 2;                                   // M tiles per CTA
 constexpr int kTileWarps = 4;                               // softmax warps per tile
 constexpr int kSoftWarps = kTiles * kTileWarps;             // 8
 constexpr int kProdWarps = 6;
-constexpr int kMmaWarp = kSoftWarps + kProdWarps;           // 14
-constexpr int kLoadWarp = kMmaWarp + 1;                     // 15
-constexpr int kTcThreads = (kLoadWarp + 1) * 32;            // 512
+constexpr int kMmaWarp = 10;                                // sub-partition 2, beside the load warp
+constexpr int kLoadWarp = 14;
+constexpr int kTcThreads = (kSoftWarps + kProdWarps + 2) * 32;  // 512
+static_assert(kMmaWarp % 4 == kLoadWarp % 4 && kMmaWarp >= kSoftWarps && kLoadWarp < kTcThreads / 32,
+              "MMA and load warps on one sub-partition");
 constexpr int kProdThreads = kProdWarps * 32;
 constexpr int kMTile = 128;
 constexpr int kRawKeys = 128;  // keys per raw (TMA) stage
@@ -74,11 +87,11 @@ constexpr int kKBufs = 2;
 constexpr int kVBufs = 3;
 constexpr int kKVBytes = kSubKeys * kHeadDim * 2;     // 16384: K^hi, K^lo or V^ [64][128] fp16
 // barriers: raw_full[3] raw_free[3] k_full[2] k_free[2] v_full[3] v_free[3]
-//           s_full[tile] p_full[tile] o_free[tile]
+//           s_full[tile] p_full[tile] o_free[tile] q_full[tile]
 constexpr int kBarK = 2 * kMaxRawStages;           // 6
 constexpr int kBarV = kBarK + 2 * kKBufs;          // 10
 constexpr int kBarT = kBarV + 2 * 3;               // 16
-constexpr int kNumBars = kBarT + 3 * kTiles;       // 22
+constexpr int kNumBars = kBarT + 4 * kTiles;       // 24
 constexpr uint32_t kTmemCols = 512;
 // columns within a tile's 256: O, S (P over its first 32 columns), Q
 constexpr uint32_t kTileCols = 256, kColO = 0, kColS = 128, kColQ = 192;
@@ -234,6 +247,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t* s_full = bars + kBarT;               // [tile] S_t MMA complete
     uint64_t* p_full = bars + kBarT + kTiles;      // [tile] softmax wrote P_t (4 warp arrivals)
     uint64_t* o_free = bars + kBarT + 2 * kTiles;  // [tile] PV_t MMA complete (P_t / S_t columns free)
+    uint64_t* q_full = bars + kBarT + 3 * kTiles;  // [tile] softmax wrote Q_t to tensor memory (4 warp arrivals)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmem);
     // set by a thread whose bounded wait gave up; everyone then skips the
     // remaining waits and work (there are no named barriers to leave behind)
@@ -270,6 +284,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(&s_full[t], 1);
             mbar_init(&p_full[t], kTileWarps);
             mbar_init(&o_free[t], 1);
+            mbar_init(&q_full[t], kTileWarps);
         }
         fence_mbar_init();
     }
@@ -280,31 +295,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int my_tile = warp / kTileWarps;
     const uint32_t tcol = (uint32_t)my_tile * kTileCols;
     const uint32_t lane_off = (uint32_t)((warp % kTileWarps) * 32) << 16;
-    if (warp < kSoftWarps && my_tile < n_tiles) {
-        // Q tile into tensor memory: lane r = local query row (2 z + t) 128 + r
-        // (rows past the head's rows are zero), dims 2c, 2c+1 in column Q + c
-        const int r = (warp % kTileWarps) * 32 + lane;
-        const int lr = (2 * blockIdx.z + my_tile) * kMTile + r;
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-            uint32_t qv[32];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (lr < rows_head) {
-                    const int j = lr / a.group, g = lr - j * a.group;
-                    v = *reinterpret_cast<const uint4*>(a.q + ((size_t)j * a.n_qh + h * a.group + g) * kHeadDim +
-                                                        half * 64 + c * 8);
-                }
-                qv[4 * c] = v.x; qv[4 * c + 1] = v.y; qv[4 * c + 2] = v.z; qv[4 * c + 3] = v.w;
-            }
-            tmem_st32u(taddr + lane_off + tcol + kColQ + half * 32, qv);
-        }
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
     bool ok = true;
     auto fail_wait = [&](uint64_t* bar, uint32_t parity) {  // true if the wait gave up
         if (!ok || *sAbort) { ok = false; return true; }
@@ -380,6 +370,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int i = is_t;
                 if (!(i < n_sub && ip_t == i && mbar_test(&k_full[i & 1], (i >> 1) & 1)))
                     return false;
+                if (i == 0 && !mbar_test(&q_full[t], 0)) return false;  // Q_t in tensor memory
                 tc_fence_after();
                 const uint32_t aKh = smem_u32(sK + (i & 1) * kKHalves * kKVBytes), aKl = aKh + kKVBytes;
                 const uint32_t t_s = taddr + t * kTileCols + kColS;
@@ -442,7 +433,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
     } else if (warp >= kSoftWarps) {
         // ============================ producer warps ============================
-        const int ptid = tid - kSoftWarps * 32;
+        const int pw = warp - kSoftWarps - (warp > kMmaWarp) - (warp > kLoadWarp);  // 0..5
+        const int ptid = pw * 32 + lane;
         for (int i = 0; i < n_sub; ++i) {
             const int r = i >> 1, sub = i & 1;
             const uint8_t* rb = raw + (r % kRS) * kRawBytes;
@@ -616,6 +608,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (my_tile < n_tiles) {
         // ============================ softmax warps ============================
+        {
+            // Q tile into tensor memory: lane r = local query row (2 z + t) 128 + r
+            // (rows past the head's rows are zero), dims 2c, 2c+1 in column Q + c;
+            // all sixteen 16-byte loads in flight together
+            const int r = (warp % kTileWarps) * 32 + lane;
+            const int lr = (2 * blockIdx.z + my_tile) * kMTile + r;
+            uint4 qa[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) qa[c] = make_uint4(0, 0, 0, 0);
+            if (lr < rows_head) {
+                const int j = lr / a.group, g = lr - j * a.group;
+                const uint4* qrow = reinterpret_cast<const uint4*>(a.q + ((size_t)j * a.n_qh + h * a.group + g) * kHeadDim);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) qa[c] = qrow[c];
+            }
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t qv[32];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 v = qa[half * 8 + c];
+                    qv[4 * c] = v.x; qv[4 * c + 1] = v.y; qv[4 * c + 2] = v.z; qv[4 * c + 3] = v.w;
+                }
+                tmem_st32u(taddr + lane_off + tcol + kColQ + half * 32, qv);
+            }
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cta(&q_full[my_tile]);
+        }
         const int srow = (warp % kTileWarps) * 32 + lane;  // TMEM lane = query row of the tile
         const int lrow = (2 * blockIdx.z + my_tile) * kMTile + srow;
         const bool row_valid = lrow < rows_head;
@@ -730,27 +752,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 l_out = w_old * prev.y + w_new * l_run;
             }
+            // 32 columns of the warp's 32 rows at a time: each thread puts its
+            // row's w_new-weighted O into shared memory (33-float row stride:
+            // no bank conflicts either way), then lane l takes column l of every
+            // row, so each row moves as one 128-byte line.  The staging area is
+            // the raw stages: the tile's last PV has completed, so every raw
+            // stage has landed and been dequantized.
+            float* stg = reinterpret_cast<float*>(raw) + warp * (32 * 33);
+            float* acc_split = a.part.acc + (size_t)split_g * a.n_rows * kHeadDim;
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 float o[32];
                 tmem_ld32(t_o + c * 32, o);
-                if (n_sub == 0) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = 0.0f;
-                }
-                if (row_valid) {
-                    float* dst = a.part.acc + ((size_t)split_g * a.n_rows + grow) * kHeadDim + c * 32;
+                for (int e = 0; e < 32; ++e) stg[lane * 33 + e] = (n_sub == 0) ? 0.0f : o[e] * w_new;
+                __syncwarp();
+                float pv[32];
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        float4 v = make_float4(o[e] * w_new, o[e + 1] * w_new, o[e + 2] * w_new, o[e + 3] * w_new);
-                        if (w_old != 0.0f) {
-                            const float4 pv = *reinterpret_cast<const float4*>(dst + e);
-                            v.x = fmaf(w_old, pv.x, v.x); v.y = fmaf(w_old, pv.y, v.y);
-                            v.z = fmaf(w_old, pv.z, v.z); v.w = fmaf(w_old, pv.w, v.w);
-                        }
-                        *reinterpret_cast<float4*>(dst + e) = v;
-                    }
+                for (int rr = 0; rr < 32; ++rr) {
+                    const float wo = __shfl_sync(0xffffffffu, w_old, rr);
+                    const int gr = __shfl_sync(0xffffffffu, grow, rr);
+                    pv[rr] = 0.0f;
+                    if (wo != 0.0f) pv[rr] = acc_split[(size_t)gr * kHeadDim + c * 32 + lane];
                 }
+#pragma unroll
+                for (int rr = 0; rr < 32; ++rr) {
+                    const float wo = __shfl_sync(0xffffffffu, w_old, rr);
+                    const int gr = __shfl_sync(0xffffffffu, grow, rr);
+                    const int rv = __shfl_sync(0xffffffffu, (int)row_valid, rr);
+                    if (rv) acc_split[(size_t)gr * kHeadDim + c * 32 + lane] = fmaf(wo, pv[rr], stg[rr * 33 + lane]);
+                }
+                __syncwarp();
             }
             if (row_valid) a.part.ml[(size_t)split_g * a.n_rows + grow] = make_float2(m_out, l_out);
         }
