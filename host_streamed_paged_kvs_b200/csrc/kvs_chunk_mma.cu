@@ -19,7 +19,7 @@
 //     the log2 domain, keep a per-row reference max that only moves when the
 //     row max exceeds it by more than 2^8 (then rescale the row of O in TMEM),
 //     and write P in fp16 over the S columns just read;
-//   producer warps 8, 9, 11, 12, 13 and 15
+//   producer warps 8, 9, 11, 12 and 13
 //     dequantize each 64-key half of a raw Q8_0/Q4_0 stage (128 keys, landed
 //     by TMA, three raw stages in flight where shared memory allows, else two)
 //     into fp16 UMMA operand tiles with the 128-byte swizzle:
@@ -29,11 +29,13 @@
 //       complete);
 //       V^ = fp16(d*(q4-8)) as [keys][dims] (read as an MN-major B operand;
 //       three buffers, free again once both tiles' PV MMAs complete);
-//   MMA warp 10 (one elected lane)
-//     polls the barriers without blocking and issues, whichever is ready
+//   MMA warps 10 (tile 0) and 15 (tile 1), one lane each
+//     poll the barriers without blocking and issue, whichever is ready
 //     first: S_t = Q_t K^_hi^T + Q_t K^_lo^T (tcgen05.mma M=128 N=64 K=16,
 //     A = Q_t from tensor memory, fp32 accumulate) of tile t once the K^
-//     buffer is full and the tile's previous PV product has been issued (P_t
+//     buffer is full, it is the tile's turn (the tiles' S products alternate,
+//     so one tile's softmax overlaps the other's products instead of both
+//     running at once) and the tile's previous PV product has been issued (P_t
 //     lives in the S_t columns; the tensor cores run the MMAs in issue order);
 //     and O_t += P_t V^ (M=128 N=128 K=16, A = P_t from tensor memory) once
 //     the softmax wrote P_t and V^ is written, with the tile's next S right
@@ -51,12 +53,12 @@
 // record row (and the previous record folded into it) moves as whole 128-byte
 // lines.  No cluster, no multicast.
 //
-// Warp w issues on sub-partition w mod 4 of the SM, and every softmax warp's
-// arithmetic there delays the tensor-core issue of an MMA warp on the same
+// Warp w issues on sub-partition w mod 4 of the SM, and the arithmetic of the
+// other warps there delays the tensor-core issue of an MMA warp on the same
 // sub-partition (each sub-partition holds two softmax warps: the lane
-// quarter a warp may read from tensor memory is w mod 4).  So the MMA and load
-// warps share sub-partition 2 and the producers' dequantization runs on the
-// other three.
+// quarter a warp may read from tensor memory is w mod 4).  So each tile has
+// its own MMA warp, on sub-partitions 2 and 3, and the producers run on the
+// others but one (warp 11).
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
@@ -71,12 +73,13 @@ namespace {
 constexpr int kTiles = 2;                                   // M tiles per CTA
 constexpr int kTileWarps = 4;                               // softmax warps per tile
 constexpr int kSoftWarps = kTiles * kTileWarps;             // 8
-constexpr int kProdWarps = 6;
-constexpr int kMmaWarp = 10;                                // sub-partition 2, beside the load warp
-constexpr int kLoadWarp = 14;
-constexpr int kTcThreads = (kSoftWarps + kProdWarps + 2) * 32;  // 512
-static_assert(kMmaWarp % 4 == kLoadWarp % 4 && kMmaWarp >= kSoftWarps && kLoadWarp < kTcThreads / 32,
-              "MMA and load warps on one sub-partition");
+constexpr int kProdWarps = 5;                               // warps 8, 9, 11, 12, 13
+constexpr int kMmaWarp0 = 10;                               // tile 0's products, sub-partition 2
+constexpr int kMmaWarp1 = 15;                               // tile 1's products, sub-partition 3
+constexpr int kLoadWarp = 14;                               // sub-partition 2, beside MMA warp 0
+constexpr int kTcThreads = (kSoftWarps + kProdWarps + 3) * 32;  // 512
+static_assert(kMmaWarp0 % 4 != kMmaWarp1 % 4 && kMmaWarp0 % 4 == kLoadWarp % 4 && kTcThreads == 512,
+              "one MMA warp per tile on two sub-partitions");
 constexpr int kProdThreads = kProdWarps * 32;
 constexpr int kMTile = 128;
 constexpr int kRawKeys = 128;  // keys per raw (TMA) stage
@@ -125,6 +128,7 @@ struct TcGeom {
     static constexpr size_t kOffBar = kOffV + kVBufs * kKVBytes;
     static constexpr size_t kOffTmem = kOffBar + kNumBars * 8;
     static constexpr size_t kOffAbort = kOffTmem + 4;
+    static constexpr size_t kOffTurn = kOffTmem + 8;  // S batches issued, per tile
     static constexpr size_t kSmem = 1024 + kOffTmem + 16;
     static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kRawBytes % 1024 == 0,
                   "swizzled tiles need 1024-B alignment");
@@ -173,6 +177,24 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// packed pairs of fp32 (one instruction for two lanes of arithmetic)
+__device__ __forceinline__ unsigned long long f2_bits(float2 v) {
+    return (unsigned long long)__float_as_uint(v.x) | ((unsigned long long)__float_as_uint(v.y) << 32);
+}
+__device__ __forceinline__ float2 bits_f2(unsigned long long b) {
+    return make_float2(__uint_as_float((uint32_t)b), __uint_as_float((uint32_t)(b >> 32)));
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {  // a * b + c, each lane rounded once
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+    return bits_f2(r);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    unsigned long long r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+    return bits_f2(r);
 }
 
 // D (+)= A B with A (M=128 rows, 16-bit pairs per column) read from tensor memory
@@ -252,6 +274,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // set by a thread whose bounded wait gave up; everyone then skips the
     // remaining waits and work (there are no named barriers to leave behind)
     volatile int* sAbort = reinterpret_cast<volatile int*>(smem + kOffAbort);
+    // S batches fully issued by each tile's MMA warp: the two tiles take turns
+    volatile int* sIssued = reinterpret_cast<volatile int*>(smem + TG::kOffTurn);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.y;
@@ -268,17 +292,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     if (tid == 32) {
         *sAbort = 0;
+        sIssued[0] = 0;
+        sIssued[1] = 0;
         for (int k = 0; k < kMaxRawStages; ++k) {
             mbar_init(&raw_full[k], ZC ? 32 : 1);  // in place: one arrival per load lane
             mbar_init(&raw_free[k], kProdWarps);
         }
         for (int k = 0; k < kKBufs; ++k) {
             mbar_init(&k_full[k], kProdWarps);
-            mbar_init(&k_free[k], 1);
+            mbar_init(&k_free[k], n_tiles);  // one commit per tile's MMA warp
         }
         for (int k = 0; k < kVBufs; ++k) {
             mbar_init(&v_full[k], kProdWarps);
-            mbar_init(&v_free[k], 1);
+            mbar_init(&v_free[k], n_tiles);
         }
         for (int t = 0; t < kTiles; ++t) {
             mbar_init(&s_full[t], 1);
@@ -355,69 +381,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == kMmaWarp) {
-        // ============================ MMA warp ============================
-        if (lane == 0) {
-            // next S and PV sub-stage of tile 0 and tile 1 (an absent tile is always done)
-            int is0 = 0, ip0 = 0, is1 = 0, ip1 = 0;
-            if (n_tiles < kTiles) is1 = ip1 = n_sub;
-            // S_t(i) once K^(i) is written and PV_t(i - 1), which reads P_t
-            // from the S_t columns, has been issued: the tensor cores run one
-            // thread's MMAs in issue order, so PV_t(i - 1) has read P_t before
-            // S_t(i) overwrites it, and the commit that reports S_t(i) also
-            // reports PV_t(i - 1) complete (the softmax may then rescale O_t)
-            auto try_s = [&](const int t, int& is_t, const int ip_t, const int is_other) {
-                const int i = is_t;
-                if (!(i < n_sub && ip_t == i && mbar_test(&k_full[i & 1], (i >> 1) & 1)))
-                    return false;
-                if (i == 0 && !mbar_test(&q_full[t], 0)) return false;  // Q_t in tensor memory
-                tc_fence_after();
-                const uint32_t aKh = smem_u32(sK + (i & 1) * kKHalves * kKVBytes), aKl = aKh + kKVBytes;
-                const uint32_t t_s = taddr + t * kTileCols + kColS;
-                const uint32_t t_q = taddr + t * kTileCols + kColQ;
+    } else if (warp == kMmaWarp0 || warp == kMmaWarp1) {
+        // ============================ MMA warps ============================
+        // one per tile, on different sub-partitions: while one waits for an
+        // issue slot the other's products keep the tensor cores busy
+        const int t = warp == kMmaWarp1 ? 1 : 0;
+        if (lane == 0 && t < n_tiles) {
+            int is = 0, ip = 0;  // next S and PV sub-stage of tile t
+            const uint32_t t_s = taddr + t * kTileCols + kColS;
+            const uint32_t t_q = taddr + t * kTileCols + kColQ;
+            const uint32_t t_o = taddr + t * kTileCols + kColO;
+            const uint64_t t0 = globaltimer_ns();
+            for (uint32_t spin = 0; ip < n_sub; ++spin) {
+                // O_t += P_t(i) V^(i) once the softmax wrote P_t(i) and V^(i) is
+                // written; the V^ buffer is free once every tile's PV(i) has
+                // completed (one commit per tile); the epilogue waits for the last
+                if (ip < is && mbar_test(&p_full[t], ip & 1) && mbar_test(&v_full[ip % kVBufs], (ip / kVBufs) & 1)) {
+                    tc_fence_after();
+                    const uint32_t aV = smem_u32(sV + (ip % kVBufs) * kKVBytes);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc_mma_f16_ts(t_s, t_q + 8 * kk, desc_k(aKh, kSubKeys, kk), kIdescS, kk > 0);
-                if constexpr (KT == kKQ8_0) {
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma_f16_ts(t_o, t_s + 8 * kk, desc_mn(aV, kk), kIdescPV, (ip > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&v_free[ip % kVBufs]);
+                    if (ip == n_sub - 1) tc_commit(&o_free[t]);
+                    ++ip;
+                    continue;
+                }
+                // S_t(i) once K^(i) (and, the first time, Q_t) is written and
+                // PV_t(i - 1), which reads P_t from the S_t columns, has been
+                // issued: the tensor cores run one thread's MMAs in issue order,
+                // so PV_t(i - 1) has read P_t before S_t(i) overwrites it, and the
+                // commit that reports S_t(i) also reports PV_t(i - 1) complete
+                // (the softmax may then rescale O_t); the K^ buffer is free once
+                // every tile's S(i) has completed (one commit per tile)
+                // turns: S_0(i) after S_1(i - 1) was issued, S_1(i) after S_0(i),
+                // so one tile's softmax runs while the other's products do
+                const bool turn = n_tiles < kTiles || (t == 0 ? sIssued[1] >= is : sIssued[0] > is);
+                if (is < n_sub && ip == is && turn && mbar_test(&k_full[is & 1], (is >> 1) & 1) &&
+                    (is > 0 || mbar_test(&q_full[t], 0))) {
+                    tc_fence_after();
+                    const uint32_t aKh = smem_u32(sK + (is & 1) * kKHalves * kKVBytes), aKl = aKh + kKVBytes;
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        tc_mma_f16_ts(t_s, t_q + 8 * kk, desc_k(aKl, kSubKeys, kk), kIdescS, 1u);
-                }
-                tc_commit(&s_full[t]);
-                is_t = i + 1;
-                // the K^ buffer is free once every tile's S(i) has completed
-                if (is_other > i) tc_commit(&k_free[i & 1]);
-                return true;
-            };
-            // O_t += P_t(i) V^(i) once the softmax wrote P_t(i) and V^(i) is written
-            auto try_pv = [&](const int t, int& ip_t, const int is_t, const int ip_other) {
-                const int i = ip_t;
-                if (!(i < is_t && mbar_test(&p_full[t], i & 1) && mbar_test(&v_full[i % kVBufs], (i / kVBufs) & 1)))
-                    return false;
-                tc_fence_after();
-                const uint32_t aV = smem_u32(sV + (i % kVBufs) * kKVBytes);
-                const uint32_t t_p = taddr + t * kTileCols + kColS;
-                const uint32_t t_o = taddr + t * kTileCols + kColO;
+                        tc_mma_f16_ts(t_s, t_q + 8 * kk, desc_k(aKh, kSubKeys, kk), kIdescS, kk > 0);
+                    if constexpr (KT == kKQ8_0) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc_mma_f16_ts(t_o, t_p + 8 * kk, desc_mn(aV, kk), kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(&o_free[t]);
-                ip_t = i + 1;
-                // the V^ buffer is free once every tile's PV(i) has completed
-                if (ip_other > i) tc_commit(&v_free[i % kVBufs]);
-                return true;
-            };
-            const uint64_t t0 = globaltimer_ns();
-            for (uint32_t spin = 0; ip0 < n_sub || ip1 < n_sub; ++spin) {
-                // a tile's PV product first, with its next S product right behind
-                // it (it unblocks that tile's softmax soonest); then S products,
-                // the tile that is behind first
-                if (try_pv(0, ip0, is0, ip1)) { try_s(0, is0, ip0, is1); continue; }
-                if (try_pv(1, ip1, is1, ip0)) { try_s(1, is1, ip1, is0); continue; }
-                if (is1 < is0) {
-                    if (try_s(1, is1, ip1, is0) || try_s(0, is0, ip0, is1)) continue;
-                } else {
-                    if (try_s(0, is0, ip0, is1) || try_s(1, is1, ip1, is0)) continue;
+                        for (int kk = 0; kk < 8; ++kk)
+                            tc_mma_f16_ts(t_s, t_q + 8 * kk, desc_k(aKl, kSubKeys, kk), kIdescS, 1u);
+                    }
+                    tc_commit(&s_full[t]);
+                    tc_commit(&k_free[is & 1]);
+                    ++is;
+                    sIssued[t] = is;
+                    continue;
                 }
                 if ((spin & 255) == 255) {
                     if (*sAbort) { ok = false; break; }
@@ -433,7 +449,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
     } else if (warp >= kSoftWarps) {
         // ============================ producer warps ============================
-        const int pw = warp - kSoftWarps - (warp > kMmaWarp) - (warp > kLoadWarp);  // 0..5
+        const int pw = warp - kSoftWarps - (warp > kMmaWarp0);  // 0..4 (warps 8, 9, 11, 12, 13)
         const int ptid = pw * 32 + lane;
         for (int i = 0; i < n_sub; ++i) {
             const int r = i >> 1, sub = i & 1;
@@ -659,17 +675,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 uint32_t pk[32];
                 float lsum = 0.0f, alpha = 1.0f;
                 // p = 2^(s scale - m) with the reference max m, and the sub-stage's
-                // sum; masked keys give 2^-inf = 0
+                // sum; masked keys give 2^-inf = 0.  The scaling and the sums run
+                // on packed pairs: the fewer instructions the softmax issues, the
+                // sooner an MMA warp on the same sub-partition gets its turn.
                 auto exp_row = [&](const float (&v)[64], float m) {
-                    float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four independent partial sums
+                    const float2 sc = make_float2(a.q_scale, a.q_scale), nm = make_float2(-m, -m);
+                    float2 la = make_float2(0.0f, 0.0f), lb = make_float2(0.0f, 0.0f);  // independent partial sums
 #pragma unroll
-                    for (int e = 0; e < 64; e += 2) {
-                        const float p0 = ex2_approx(fmaf(v[e], a.q_scale, -m));
-                        const float p1 = ex2_approx(fmaf(v[e + 1], a.q_scale, -m));
-                        l4[(e >> 1) & 3] += p0 + p1;
-                        pk[e >> 1] = h2u(__floats2half2_rn(p0, p1));
+                    for (int e = 0; e < 64; e += 4) {
+                        const float2 x0 = fma2(make_float2(v[e], v[e + 1]), sc, nm);
+                        const float2 x1 = fma2(make_float2(v[e + 2], v[e + 3]), sc, nm);
+                        const float2 p01 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+                        const float2 p23 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+                        la = add2(la, p01);
+                        lb = add2(lb, p23);
+                        pk[e >> 1] = h2u(__floats2half2_rn(p01.x, p01.y));
+                        pk[(e >> 1) + 1] = h2u(__floats2half2_rn(p23.x, p23.y));
                     }
-                    return (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                    const float2 l2 = add2(la, lb);
+                    return l2.x + l2.y;
                 };
                 auto load_s = [&](float (&v)[64]) {
                     tmem_ld64(t_s, v);
@@ -728,7 +752,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (lane == 0) mbar_arrive_cta(&p_full[my_tile]);
         }
         // ---- epilogue: wait for the tile's last PV, write the split's partials ----
-        const bool bad3 = (n_sub > 0) && fail_wait(&o_free[my_tile], (n_sub - 1) & 1);
+        const bool bad3 = (n_sub > 0) && fail_wait(&o_free[my_tile], 0);  // the tile's last PV
         tc_fence_after();
         if (__all_sync(0xffffffffu, !bad3 && ok) && warp_active) {
             const int split_g = a.split_base + blockIdx.x;

@@ -447,7 +447,7 @@ struct kvs_s {
     cudaStream_t rs = nullptr;       // side stream: resident-page attention (lowest priority)
     cudaStream_t xs = nullptr;       // ring attention stream (highest priority)
     cudaStream_t zs = nullptr;       // in-place (zero-copy) attention of streamed pages (lowest)
-    cudaEvent_t ev_fork = nullptr, ev_res = nullptr, ev_ring = nullptr, ev_zc = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_res = nullptr, ev_ring = nullptr, ev_zc = nullptr, ev_join = nullptr;
     size_t partial_capacity = 0;     // (split x row) records
     int n_groups = 0;
     std::vector<cudaEvent_t> ev_full, ev_free, ev_hist;
@@ -683,6 +683,7 @@ void release(kvs_t* kv) {
     if (kv->ev_res) cudaEventDestroy(kv->ev_res);
     if (kv->ev_ring) cudaEventDestroy(kv->ev_ring);
     if (kv->ev_zc) cudaEventDestroy(kv->ev_zc);
+    if (kv->ev_join) cudaEventDestroy(kv->ev_join);
     if (kv->zs) cudaStreamDestroy(kv->zs);
     if (kv->xs) cudaStreamDestroy(kv->xs);
     if (kv->cs) cudaStreamDestroy(kv->cs);
@@ -931,7 +932,8 @@ int kvs_create(const kvs_config* cfg, int device, kvs_t** out) {
     if (cudaEventCreateWithFlags(&kv->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&kv->ev_res, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&kv->ev_ring, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&kv->ev_zc, cudaEventDisableTiming) != cudaSuccess)
+        cudaEventCreateWithFlags(&kv->ev_zc, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&kv->ev_join, cudaEventDisableTiming) != cudaSuccess)
         return bail(KVS_E_CUDA, "cudaEventCreate failed");
     kv->n_groups = c.n_ring_slots > 0 ? c.n_ring_slots / c.chunk_pages : 0;
     kv->ev_full.assign(kv->n_groups, nullptr);
@@ -1006,6 +1008,25 @@ int kvs_append(kvs_t* kv, int layer, int pos0, int n_tok, const void* k_f16, con
         return fail(kv, KVS_E_INVAL, fmt("append beyond max_ctx (%d)", c.max_ctx));
     DeviceGuard g(kv->device);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // Stream capture: the copy stream joins the capture here, ahead of the
+    // append kernel, so a captured step's first ring copy starts with the
+    // graph instead of after the append.  The copies read only history pages
+    // that no append of this capture has written (kvs_attend waits for the
+    // append's history write when one of its pages is streamed).
+    {
+        const unsigned long long cap = capture_id(s);
+        if (cap && c.n_ring_slots > 0 && kv->cs_cap != cap) {
+            KVS_CK(kv, cudaEventRecord(kv->ev_fork, s));
+            KVS_CK(kv, cudaStreamWaitEvent(kv->cs, kv->ev_fork, 0));
+            // joined straight back, so a capture that ends before any attend
+            // call leaves no stream behind (the caller's stream gains no wait:
+            // the copy stream holds nothing yet)
+            KVS_CK(kv, cudaEventRecord(kv->ev_join, kv->cs));
+            KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_join, 0));
+            kv->cs_cap = cap;
+            kv->capture_seen = true;
+        }
+    }
     const size_t kv_elems = (size_t)n_tok * c.n_kv_heads * kHeadDim;
     const __half* k = static_cast<const __half*>(k_f16);
     const __half* v = static_cast<const __half*>(v_f16);
@@ -1264,8 +1285,15 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         // partials into the records of the first one
         const int ring_base = split_base;
         int ring_width = 0;
-        for (long i0 = 0; i0 < S_ring; i0 += chunk) {
-            const int cpages = (int)std::min<long>(chunk, S_ring - i0);
+        // Wide tensor-core calls send the last full chunk as two halves: the
+        // launch after the final copy, which nothing overlaps, then attends
+        // half as many pages (the first half's launch runs under the second
+        // half's copy).
+        const bool split_tail = tc && m_tiles(c, n_q) > 1 && chunk >= 2;
+        int cpages = 0;
+        for (long i0 = 0; i0 < S_ring; i0 += cpages) {
+            cpages = (int)std::min<long>(chunk, S_ring - i0);
+            if (split_tail && cpages == chunk && i0 + cpages == S_ring) cpages = chunk / 2;
             const int gidx = (int)(kv->ring_ctr % kv->n_groups);
             kv->ring_ctr++;
             if (kv->free_valid[gidx] && kv->free_cap[gidx] == cap)
