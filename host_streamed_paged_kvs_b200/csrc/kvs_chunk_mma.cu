@@ -777,34 +777,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 l_out = w_old * prev.y + w_new * l_run;
             }
             // 32 columns of the warp's 32 rows at a time: each thread puts its
-            // row's w_new-weighted O into shared memory (33-float row stride:
-            // no bank conflicts either way), then lane l takes column l of every
-            // row, so each row moves as one 128-byte line.  The staging area is
-            // the raw stages: the tile's last PV has completed, so every raw
-            // stage has landed and been dequantized.
-            float* stg = reinterpret_cast<float*>(raw) + warp * (32 * 33);
+            // row's w_new-weighted O into shared memory (36-float row stride),
+            // then 8 lanes take a row's 32 columns as 16-byte pieces, 4 rows per
+            // instruction, so each row (and the previous record folded into
+            // it) moves as one 128-byte line.  The staging area is the raw
+            // stages: the tile's last PV has completed, so every raw stage has
+            // landed and been dequantized.
+            float* stg = reinterpret_cast<float*>(raw) + warp * (32 * 36);
             float* acc_split = a.part.acc + (size_t)split_g * a.n_rows * kHeadDim;
+            const int sub_r = lane >> 3, q4 = lane & 7;  // row within a group of 4, 16-byte piece of the row
+            float wo_k[8];
+            int gr_k[8];  // record row of row 4 k + sub_r, -1 when the row is past the head's rows
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                wo_k[k] = __shfl_sync(0xffffffffu, w_old, 4 * k + sub_r);
+                gr_k[k] = __shfl_sync(0xffffffffu, row_valid ? grow : -1, 4 * k + sub_r);
+            }
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 float o[32];
                 tmem_ld32(t_o + c * 32, o);
+                const float wn = (n_sub == 0) ? 0.0f : w_new;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) stg[lane * 33 + e] = (n_sub == 0) ? 0.0f : o[e] * w_new;
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<float4*>(stg + lane * 36 + 4 * j) =
+                        make_float4(o[4 * j] * wn, o[4 * j + 1] * wn, o[4 * j + 2] * wn, o[4 * j + 3] * wn);
                 __syncwarp();
-                float pv[32];
+                float4 pv[8];
 #pragma unroll
-                for (int rr = 0; rr < 32; ++rr) {
-                    const float wo = __shfl_sync(0xffffffffu, w_old, rr);
-                    const int gr = __shfl_sync(0xffffffffu, grow, rr);
-                    pv[rr] = 0.0f;
-                    if (wo != 0.0f) pv[rr] = acc_split[(size_t)gr * kHeadDim + c * 32 + lane];
+                for (int k = 0; k < 8; ++k) {
+                    pv[k] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    if (wo_k[k] != 0.0f)
+                        pv[k] = *reinterpret_cast<const float4*>(acc_split + (size_t)gr_k[k] * kHeadDim + c * 32 + 4 * q4);
                 }
 #pragma unroll
-                for (int rr = 0; rr < 32; ++rr) {
-                    const float wo = __shfl_sync(0xffffffffu, w_old, rr);
-                    const int gr = __shfl_sync(0xffffffffu, grow, rr);
-                    const int rv = __shfl_sync(0xffffffffu, (int)row_valid, rr);
-                    if (rv) acc_split[(size_t)gr * kHeadDim + c * 32 + lane] = fmaf(wo, pv[rr], stg[rr * 33 + lane]);
+                for (int k = 0; k < 8; ++k) {
+                    if (gr_k[k] < 0) continue;
+                    const float4 sv = *reinterpret_cast<const float4*>(stg + (4 * k + sub_r) * 36 + 4 * q4);
+                    const float wo = wo_k[k];
+                    *reinterpret_cast<float4*>(acc_split + (size_t)gr_k[k] * kHeadDim + c * 32 + 4 * q4) =
+                        make_float4(fmaf(wo, pv[k].x, sv.x), fmaf(wo, pv[k].y, sv.y), fmaf(wo, pv[k].z, sv.z),
+                                    fmaf(wo, pv[k].w, sv.w));
                 }
                 __syncwarp();
             }

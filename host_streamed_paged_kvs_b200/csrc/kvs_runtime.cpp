@@ -1285,15 +1285,15 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         // partials into the records of the first one
         const int ring_base = split_base;
         int ring_width = 0;
-        // Wide tensor-core calls send the last full chunk as two halves: the
-        // launch after the final copy, which nothing overlaps, then attends
-        // half as many pages (the first half's launch runs under the second
-        // half's copy).
+        // Wide tensor-core calls send the last chunk in halving pieces (8 pages
+        // as 4, 2, 2): the launch after the final copy, which nothing
+        // overlaps, then attends two pages (each earlier piece's launch runs
+        // under the next piece's copy).
         const bool split_tail = tc && m_tiles(c, n_q) > 1 && chunk >= 2;
         int cpages = 0;
         for (long i0 = 0; i0 < S_ring; i0 += cpages) {
             cpages = (int)std::min<long>(chunk, S_ring - i0);
-            if (split_tail && cpages == chunk && i0 + cpages == S_ring) cpages = chunk / 2;
+            if (split_tail && i0 + cpages == S_ring && cpages > 2) cpages = (cpages + 1) / 2;
             const int gidx = (int)(kv->ring_ctr % kv->n_groups);
             kv->ring_ctr++;
             if (kv->free_valid[gidx] && kv->free_cap[gidx] == cap)
@@ -1303,6 +1303,10 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
             KVS_CK(kv, cudaMemcpyAsync(dst, src, (size_t)cpages * kv->page_bytes, cudaMemcpyHostToDevice, kv->cs));
             KVS_CK(kv, cudaEventRecord(kv->ev_full[gidx], kv->cs));
             KVS_CK(kv, cudaStreamWaitEvent(xstream, kv->ev_full[gidx], 0));
+            // the merge follows the last ring launch on its stream: order it
+            // after the resident splits now, while this launch waits for its
+            // copy anyway (the resident launches end long before)
+            if (i0 + cpages == S_ring) KVS_CK(kv, cudaStreamWaitEvent(xstream, kv->ev_res, 0));
             d.region = kv->ring;
             d.region_slot_base = 0;
             d.region_slots = c.n_ring_slots;
@@ -1330,13 +1334,14 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
             kv->stats.h2d_copies++;
         }
         split_base += ring_width;
-        KVS_CK(kv, cudaEventRecord(kv->ev_ring, xstream));
-        KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_ring, 0));
     }
 
-    // 3) log-sum-exp merge of all splits (after the side stream's resident splits)
-    KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_res, 0));
-    if (S_zc > 0) KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_zc, 0));
+    // 3) log-sum-exp merge of all splits, after the resident (and in-place)
+    //    splits; with a ring it runs right behind the last ring launch on its
+    //    stream, and the caller's stream waits for it
+    cudaStream_t mstream = S_ring > 0 ? xstream : s;
+    if (S_ring == 0) KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_res, 0));
+    if (S_zc > 0) KVS_CK(kv, cudaStreamWaitEvent(mstream, kv->ev_zc, 0));
     MergeArgs m;
     m.part = kv->part;
     m.n_splits = split_base;
@@ -1345,10 +1350,14 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
     m.lse = dlse;
     m.err = nullptr;  // a timed-out wait is reported by kvs_sync / kvs_get_stats
     {
-        TimedScope ts(kv, s, kTMerge, 0);
-        KVS_CK(kv, launch_merge(m, s));
+        TimedScope ts(kv, mstream, kTMerge, 0);
+        KVS_CK(kv, launch_merge(m, mstream));
     }
     kv->stats.kernel_launches++;
+    if (mstream != s) {
+        KVS_CK(kv, cudaEventRecord(kv->ev_ring, mstream));
+        KVS_CK(kv, cudaStreamWaitEvent(s, kv->ev_ring, 0));
+    }
     if (host_out)
         KVS_CK(kv, cudaMemcpyAsync(out, dout, (size_t)rows * kHeadDim * 4, cudaMemcpyDeviceToHost, s));
     if (host_lse) KVS_CK(kv, cudaMemcpyAsync(lse, dlse, (size_t)rows * 4, cudaMemcpyDeviceToHost, s));
