@@ -50,9 +50,9 @@ NCU_TRAFFIC = {
                       # in-place launch: DRAM bytes (Q and split records; they do not grow
                       # with the pages), and host-memory bytes read over PCIe
                       "in_place": (86272, 51), "in_place_pcie": (23763968, 51)},
-    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "2a0a2ccd8250adad",
+    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "fa2afd4f1478448d",
                          "workload": "prefill_chunk_64k", "type_v": 2,
-                         "resident": (52743168, 16), "ring": (6115072, 8)},
+                         "resident": (52468224, 16), "ring": (6090496, 8)},
 }
 
 
