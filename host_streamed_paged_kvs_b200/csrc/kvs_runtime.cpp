@@ -92,7 +92,7 @@ constexpr int kSms = 148;
 // Splits of the resident launch and of one ring-chunk launch (each split is an
 // equal share of the launch's half-page stages).
 constexpr long kResCtaStages = 4;  // raw stages per resident CTA beside ring launches
-constexpr long kResSplits = 8;     // splits per such resident launch
+constexpr long kResSplits = 4;     // splits per such resident launch
 
 int res_splits(const kvs_config& c, long R_eff, int n_q, bool ring) {
     const long stages = 2 * R_eff;
@@ -1217,8 +1217,14 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
             kv->cs_cap = 0;
             for (int gi = 0; gi < kv->n_groups; ++gi)
                 if (kv->free_cap[gi]) kv->free_valid[gi] = 0;
+            // a history write last recorded inside a capture ran on the
+            // caller's stream before this call, so the wait above covers it
+            // (its event may not be waited on outside the capture)
             for (int li = 0; li < c.n_layers; ++li)
-                if (kv->hist_cap[li]) kv->hist_cap[li] = 0;
+                if (kv->hist_cap[li]) {
+                    kv->hist_cap[li] = 0;
+                    kv->layers[li].pending_min_page = INT_MAX;
+                }
         }
         if (tc && S_ring > 0) {
             // launches of kResSplits CTAs of kResCtaStages raw stages each, in
