@@ -133,6 +133,8 @@ struct TcGeom {
     static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kRawBytes % 1024 == 0,
                   "swizzled tiles need 1024-B alignment");
     static_assert(kSmem <= 232448, "shared memory budget");
+    static_assert((size_t)kSoftWarps * 32 * 272 <= (size_t)(kKBufs * kKHalves + kVBufs) * kKVBytes,
+                  "the softmax warps' Q staging fits the operand buffers");
 };
 static_assert(TcGeom<kVQ4_0>::kRawStages == 3 && TcGeom<kVQ8_0>::kRawStages == 3 && TcGeom<kVF16>::kRawStages == 2,
               "raw stages in flight");
@@ -455,6 +457,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int r = i >> 1, sub = i & 1;
             const uint8_t* rb = raw + (r % kRS) * kRawBytes;
             if (sub == 0 && fail_wait(&raw_full[r % kRS], (r / kRS) & 1)) break;
+            // the operand buffers hold the softmax warps' Q staging until every
+            // tile's Q is in tensor memory
+            if (i == 0 && (fail_wait(&q_full[0], 0) || (n_tiles > 1 && fail_wait(&q_full[1], 0)))) break;
             // ---- K^ hi / lo for keys [64 sub, 64 sub + 64) of the raw stage,
             //      once the S MMAs of sub-stage i - 2 released the buffer ----
             if (i >= 2 && fail_wait(&k_free[i & 1], ((i - 2) >> 1) & 1)) break;
@@ -626,25 +631,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // ============================ softmax warps ============================
         {
             // Q tile into tensor memory: lane r = local query row (2 z + t) 128 + r
-            // (rows past the head's rows are zero), dims 2c, 2c+1 in column Q + c;
-            // all sixteen 16-byte loads in flight together
-            const int r = (warp % kTileWarps) * 32 + lane;
-            const int lr = (2 * blockIdx.z + my_tile) * kMTile + r;
+            // (rows past the head's rows are zero), dims 2c, 2c+1 in column Q + c.
+            // The warp reads its 32 rows two at a time as whole 256-byte rows
+            // (all sixteen loads in flight), transposes them through shared
+            // memory (272-byte row stride: no bank conflicts either way) and each
+            // thread stores its own row.  The staging area is the K^/V^ operand
+            // buffers, which the producers write only after every tile's Q barrier.
+            const int wrow0 = (2 * blockIdx.z + my_tile) * kMTile + (warp % kTileWarps) * 32;
+            uint8_t* qst = sK + warp * (32 * 272);
+            const int c16 = lane & 15;
             uint4 qa[16];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) qa[c] = make_uint4(0, 0, 0, 0);
-            if (lr < rows_head) {
-                const int j = lr / a.group, g = lr - j * a.group;
-                const uint4* qrow = reinterpret_cast<const uint4*>(a.q + ((size_t)j * a.n_qh + h * a.group + g) * kHeadDim);
-#pragma unroll
-                for (int c = 0; c < 16; ++c) qa[c] = qrow[c];
+            for (int k = 0; k < 16; ++k) {
+                const int lr = wrow0 + 2 * k + (lane >> 4);
+                qa[k] = make_uint4(0, 0, 0, 0);
+                if (lr < rows_head) {
+                    const int j = lr / a.group, g = lr - j * a.group;
+                    qa[k] = *reinterpret_cast<const uint4*>(a.q + ((size_t)j * a.n_qh + h * a.group + g) * kHeadDim +
+                                                            c16 * 8);
+                }
             }
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                *reinterpret_cast<uint4*>(qst + (2 * k + (lane >> 4)) * 272 + c16 * 16) = qa[k];
+            __syncwarp();
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t qv[32];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const uint4 v = qa[half * 8 + c];
+                    const uint4 v = *reinterpret_cast<const uint4*>(qst + lane * 272 + (half * 8 + c) * 16);
                     qv[4 * c] = v.x; qv[4 * c + 1] = v.y; qv[4 * c + 2] = v.z; qv[4 * c + 3] = v.w;
                 }
                 tmem_st32u(taddr + lane_off + tcol + kColQ + half * 32, qv);
