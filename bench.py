@@ -50,9 +50,9 @@ NCU_TRAFFIC = {
                       # in-place launch: DRAM bytes (Q and split records; they do not grow
                       # with the pages), and host-memory bytes read over PCIe
                       "in_place": (86272, 51), "in_place_pcie": (23763968, 51)},
-    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "fa2afd4f1478448d",
+    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "ddf6c72e984edc9a",
                          "workload": "prefill_chunk_64k", "type_v": 2,
-                         "resident": (52468224, 16), "ring": (6090496, 8)},
+                         "resident": (27399936, 8), "ring": (6100736, 8)},
 }
 
 
@@ -624,6 +624,25 @@ def run_gpu(args, w: W.Workload):
             if timeline[tag] is not None:
                 timeline[tag]["zero_copy_pct"] = pct
         kvs.kvs_set_zero_copy_pct(h, 0 if wide else zc_pct, zc_pct_wide)
+        if args.graph:
+            # replays of one captured step at the tuned share: consecutive
+            # replays cannot overlap, so each boundary shows its tail
+            g_tl = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_tl, stream=stream):
+                one_step(ks, vs, qs, out, lse)
+
+            def replay():
+                with torch.cuda.stream(stream):
+                    g_tl.replay()
+
+            for _ in range(2):
+                replay()
+            path = os.path.join(args.timeline, f"timeline_{w.name}_tuned_graph.json")
+            n_tl = 4
+            capture_timeline(replay, n_tl, path, barrier)
+            timeline["tuned_graph"] = timeline_summary(path, n_tl, h2d_peak)
+            del g_tl
+            barrier()
 
     hbm_peak, peak_src = peaks()
     P = w.n_pages
