@@ -104,9 +104,11 @@ static_assert(kKVBytes % 1024 == 0, "swizzled tiles need 1024-B alignment");
 // pages hold them): Kq [128][128] @ 0, Kd @ 16384, Vq @ 17408 (64 B per key
 // for Q4_0 and Q5_0 V, 128 B for Q8_0 V, 256 B of values for F16 V), the Q5_x
 // fifth bits (16 B per key), Vd (none for F16), then the Q4_1 / Q5_1 minima
-// (8 B per key).  Shared memory: two raw
-// stages, then [2] x (K^hi | K^lo), [3] x V^, the barriers, the TMEM slot and
-// the abort flag (Q4_0 V: K^ @ 53248, V^ @ 118784, barriers @ 167936).
+// (8 B per key).  Shared memory: three raw stages where they fit (else two),
+// then [2] x (K^hi | K^lo), [3] x V^, the barriers, the TMEM slot, the abort
+// flag and the tiles' S turn counters (Q4_0 V: K^ @ 79872, V^ @ 145408,
+// barriers @ 194560).  The K^/V^ buffers also stage Q before the first
+// operand is written, and the raw stages the epilogue's record rows.
 // f16 K (the f16-f16 pair): the raw stage holds each key's values as two
 // 128-byte rows (dims 0..63, 64..127) and K^ needs no lo tile.
 template <int VT, int KT = kKQ8_0>
