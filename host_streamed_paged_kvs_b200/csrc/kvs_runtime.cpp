@@ -1295,9 +1295,9 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         // 5 + 3) into the slots of one group: the launch after the final copy,
         // which nothing overlaps, then attends three pages, the first piece's
         // launch runs under the second piece's copy, and only the first piece
-        // waits for the group to be free.  (A launch costs about 14 us plus
-        // 2.7 us per page, an 8-page copy 65.5 us: 5 + 3 ends the step
-        // earliest of the splits tried.)
+        // waits for the group to be free.  (On B200 a launch costs about 14 us
+        // plus 2.7 us per page and an 8-page copy 65.5 us: a first piece of 5/8
+        // is the largest whose launch ends before the second piece's copy.)
         const bool split_tail = tc && m_tiles(c, n_q) > 1 && chunk >= 2;
         const long last0 = (S_ring - 1) / chunk * chunk;  // first page of the last chunk
         int cpages = 0, gidx = 0, slot_off = 0;
