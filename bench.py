@@ -50,7 +50,7 @@ NCU_TRAFFIC = {
                       # in-place launch: DRAM bytes (Q and split records; they do not grow
                       # with the pages), and host-memory bytes read over PCIe
                       "in_place": (86272, 51), "in_place_pcie": (23763968, 51)},
-    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "2dbdf84af5ee07a7",
+    "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "18d03cf82c7cfd65",
                          "workload": "prefill_chunk_64k", "type_v": 2,
                          "resident": (27399936, 8), "ring": (6100736, 8)},
 }

@@ -12,9 +12,10 @@
 // 64-key sub-stages, handing work to each other only through mbarriers:
 //
 //   softmax warps 0..3 (tile 0) and 4..7 (tile 1), thread = query row = TMEM
-//     lane, whole 64-key rows: put the tile's Q into tensor memory once (and
-//     report it on the tile's Q barrier: the loads and dequantization start
-//     without waiting for Q), then
+//     lane, whole 64-key rows: put the tile's Q into tensor memory once,
+//     staged through the K^/V^ operand buffers, and report it on the tile's Q
+//     barrier (the loads start without waiting for Q; the producers' first
+//     operand write and the tile's first S wait for it), then
 //     per sub-stage read S, apply the causal mask and the 1/sqrt(128) scale in
 //     the log2 domain, keep a per-row reference max that only moves when the
 //     row max exceeds it by more than 2^8 (then rescale the row of O in TMEM),
