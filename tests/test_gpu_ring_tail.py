@@ -31,3 +31,22 @@ def test_ring_tail_pieces_match_oracle(streamed, pct_wide):
         assert st["pages_streamed"] == 2 * streamed
     finally:
         kvs.kvs_destroy(h)
+
+
+# every K/V pair: their raw stages, K^ halves and raw-stage counts differ, and
+# with them the shared-memory regions that stage Q and the epilogue's records
+@pytest.mark.parametrize("type_k,type_v", [(8, 8), (8, 6), (8, 3), (8, 7), (8, 1), (1, 1)])
+@pytest.mark.parametrize("streamed", [8, 13])
+def test_ring_tail_every_pair(type_k, type_v, streamed):
+    from host_streamed_paged_kvs_b200 import kvs
+    R = 2
+    w = W.Workload("ring_tail_pair", n_layers=1, n_q=64, n_q_heads=40, n_kv_heads=8,
+                   ctx=(streamed + R) * W.PAGE_TOKENS, n_resident_pages=R, n_ring_slots=16,
+                   seed=60 + streamed, outlier_frac=0.01, outlier_scale=8.0, type_v=type_v)
+    h = kvs.kvs_create(make_cfg(w, type_k=type_k, type_v=type_v), 0)
+    try:
+        prefill(h, w, 0, w.pos0)
+        out, lse = step(h, w, 0, w.pos0, w.n_q)
+        assert_close(out, lse, *oracle_step(w, 0, w.pos0, w.n_q, v_type=type_v, k_type=type_k))
+    finally:
+        kvs.kvs_destroy(h)
