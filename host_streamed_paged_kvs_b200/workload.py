@@ -106,9 +106,10 @@ ZERO_COPY_PCT = 80
 # The same share for the wider calls of the tensor-core path (verify batches,
 # prefill chunks), whose in-place launch holds about 120 of the 148 SMs.
 # Measured on the verify workload, in place only (100) ran 3 % slower than the
-# ring alone (8-page ring copies are as fast as the link allows); on the
-# prefill chunk every tile pair of a kv head reads the host pages itself, five
-# times the PCIe bytes, so the ring alone (0) is the default.
+# ring alone and shares of 30-70 % were no faster (8-page ring copies are as
+# fast as the link allows); on the prefill chunk every tile pair of a kv head
+# reads the host pages itself, five times the PCIe bytes, so the ring alone (0)
+# is the default.
 ZERO_COPY_PCT_WIDE = 0
 
 
