@@ -119,6 +119,52 @@ int res_splits(const kvs_config& c, long R_eff, int n_q, bool ring) {
     return (int)std::min(stages, std::max(1L, (long)kTargetCtas / per_split));
 }
 
+// One copy of a call's ring schedule: streamed pages [page0, page0 + pages)
+// into ring slots [slot0, slot0 + pages).  new_group: the copy starts a ring
+// group (and waits for that group's previous launch); otherwise it continues
+// the group of the copy before it.
+struct RingCopy {
+    long page0;
+    int pages;
+    int slot0;
+    bool new_group;
+};
+
+// The ring schedule of one call whose streamed pages [0, S_ring) go through
+// the ring, in ascending page order: one copy per chunk_pages pages, each into
+// the next group (ring_ctr0, ring_ctr0 + 1, ... mod the group count).  Wide
+// tensor-core calls (more than one M tile) send the last chunk as two pieces
+// into the slots of one group: the first (5 p + 7) / 8 of its p pages, then
+// the rest.  The launch after the final copy, which nothing overlaps, then
+// attends fewer pages; only the first piece waits for the group to be free.
+// (On B200 a launch costs about 14 us plus 2.7 us per page and an 8-page copy
+// 65.5 us: a first piece of 5/8 is the largest whose launch ends before the
+// second piece's copy.)  Returns the groups used (the ring counter's advance).
+long plan_ring(const kvs_config& c, int n_q, long S_ring, long long ring_ctr0, std::vector<RingCopy>& out) {
+    out.clear();
+    const int chunk = c.chunk_pages;
+    const long n_groups = chunk > 0 ? c.n_ring_slots / chunk : 0;
+    if (S_ring <= 0 || n_groups <= 0) return 0;
+    const bool split_tail = use_tcgen05(c, n_q) && m_tiles(c, n_q) > 1 && chunk >= 2;
+    const long last0 = (S_ring - 1) / chunk * chunk;  // first page of the last chunk
+    long groups = 0;
+    int gidx = 0, slot_off = 0, cpages = 0;
+    for (long i0 = 0; i0 < S_ring; i0 += cpages) {
+        cpages = (int)std::min<long>(chunk, S_ring - i0);
+        const bool piece = split_tail && i0 >= last0;
+        if (piece && i0 == last0 && cpages >= 2) cpages = (5 * cpages + 7) / 8;
+        const bool fresh = !piece || i0 == last0;
+        if (fresh) {
+            gidx = (int)((ring_ctr0 + groups) % n_groups);
+            ++groups;
+            slot_off = 0;
+        }
+        out.push_back(RingCopy{i0, cpages, gidx * chunk + slot_off, fresh});
+        slot_off += cpages;
+    }
+    return groups;
+}
+
 int ring_splits(const kvs_config& c, int n_q, int chunk_pages) {
     const int stages = 2 * chunk_pages;
     if (use_tcgen05(c, n_q)) {
@@ -459,6 +505,7 @@ struct kvs_s {
     unsigned long long cs_cap = 0;
     bool capture_seen = false;
     uint64_t ring_ctr = 0;
+    std::vector<RingCopy> ring_plan;  // the current call's ring schedule
     std::vector<LayerState> layers;
     kvs_stats stats{};
     std::vector<Timed> timed;
@@ -808,6 +855,24 @@ int kvs_plan_page(const kvs_config* c, int n_tokens, int page, int* kind, int* i
         return KVS_E_INVAL;
     }
     return plan_page(*c, n_tokens, page, kind, index);
+}
+
+int kvs_plan_ring(const kvs_config* c, int n_q, int s_ring, long long ring_ctr0, int* page0, int* pages,
+                  int* slot0, int max_copies) {
+    if (!c || n_q < 1 || s_ring < 0 || ring_ctr0 < 0 || max_copies < 0 ||
+        (max_copies > 0 && (!page0 || !pages || !slot0)) || c->n_ring_slots < 0 || c->chunk_pages < 0 ||
+        (c->n_ring_slots > 0 && c->chunk_pages < 1)) {
+        g_last_error = "kvs_plan_ring: bad arguments (config must be resolved)";
+        return KVS_E_INVAL;
+    }
+    std::vector<RingCopy> plan;
+    plan_ring(*c, n_q, s_ring, ring_ctr0, plan);
+    for (int i = 0; i < (int)plan.size() && i < max_copies; ++i) {
+        page0[i] = (int)plan[i].page0;
+        pages[i] = plan[i].pages;
+        slot0[i] = plan[i].slot0;
+    }
+    return (int)plan.size();
 }
 
 int kvs_eject_init(kvs_eject_params* p, kvs_eject_state* s) {
@@ -1291,28 +1356,14 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
         // partials into the records of the first one
         const int ring_base = split_base;
         int ring_width = 0;
-        // Wide tensor-core calls send the last chunk as two pieces (8 pages as
-        // 5 + 3) into the slots of one group: the launch after the final copy,
-        // which nothing overlaps, then attends three pages, the first piece's
-        // launch runs under the second piece's copy, and only the first piece
-        // waits for the group to be free.  (On B200 a launch costs about 14 us
-        // plus 2.7 us per page and an 8-page copy 65.5 us: a first piece of 5/8
-        // is the largest whose launch ends before the second piece's copy.)
-        const bool split_tail = tc && m_tiles(c, n_q) > 1 && chunk >= 2;
-        const long last0 = (S_ring - 1) / chunk * chunk;  // first page of the last chunk
-        int cpages = 0, gidx = 0, slot_off = 0;
-        for (long i0 = 0; i0 < S_ring; i0 += cpages) {
-            cpages = (int)std::min<long>(chunk, S_ring - i0);
-            const bool piece = split_tail && i0 >= last0;
-            if (piece && i0 == last0 && cpages >= 2) cpages = (5 * cpages + 7) / 8;
-            if (!piece || i0 == last0) {
-                gidx = (int)(kv->ring_ctr % kv->n_groups);
-                kv->ring_ctr++;
-                slot_off = 0;
-                if (kv->free_valid[gidx] && kv->free_cap[gidx] == cap)
-                    KVS_CK(kv, cudaStreamWaitEvent(kv->cs, kv->ev_free[gidx], 0));
-            }
-            uint8_t* dst = kv->ring + ((size_t)gidx * chunk + slot_off) * kv->page_bytes;
+        kv->ring_ctr += (uint64_t)plan_ring(c, n_q, S_ring, (long long)kv->ring_ctr, kv->ring_plan);
+        for (const RingCopy& rc : kv->ring_plan) {
+            const long i0 = rc.page0;
+            const int cpages = rc.pages;
+            const int gidx = rc.slot0 / chunk;
+            if (rc.new_group && kv->free_valid[gidx] && kv->free_cap[gidx] == cap)
+                KVS_CK(kv, cudaStreamWaitEvent(kv->cs, kv->ev_free[gidx], 0));
+            uint8_t* dst = kv->ring + (size_t)rc.slot0 * kv->page_bytes;
             const uint8_t* src = kv->host + ((size_t)layer * kv->P_max + (size_t)i0) * kv->page_bytes;
             KVS_CK(kv, cudaMemcpyAsync(dst, src, (size_t)cpages * kv->page_bytes, cudaMemcpyHostToDevice, kv->cs));
             KVS_CK(kv, cudaEventRecord(kv->ev_full[gidx], kv->cs));
@@ -1324,10 +1375,9 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
             d.region = kv->ring;
             d.region_slot_base = 0;
             d.region_slots = c.n_ring_slots;
-            d.slot0 = gidx * chunk + slot_off;
+            d.slot0 = rc.slot0;
             d.page0 = (int)i0;
             d.n_units = cpages;
-            slot_off += cpages;
             const int ns = ring_splits(c, n_q, cpages);
             d.n_splits = ns;
             d.split_base = tc ? ring_base : split_base;

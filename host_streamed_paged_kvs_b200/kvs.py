@@ -40,7 +40,7 @@ ERROR_NAMES = {0: "KVS_OK", -1: "KVS_E_INVAL", -2: "KVS_E_ARENA", -3: "KVS_E_WID
                -4: "KVS_E_ORDER", -5: "KVS_E_CUDA", -6: "KVS_E_TIMEOUT", -7: "KVS_E_NOMEM"}
 
 # every symbol the header declares
-EXPORTS = ["kvs_resolve_config", "kvs_page_bytes", "kvs_plan_page", "kvs_create", "kvs_destroy",
+EXPORTS = ["kvs_resolve_config", "kvs_page_bytes", "kvs_plan_page", "kvs_plan_ring", "kvs_create", "kvs_destroy",
            "kvs_append", "kvs_attend", "kvs_export_page", "kvs_page_location", "kvs_layer_length",
            "kvs_get_config", "kvs_get_stats", "kvs_reset_stats", "kvs_set_profiling",
            "kvs_set_zero_copy_pct", "kvs_sync",
@@ -112,6 +112,7 @@ def _load():
     L.kvs_page_bytes.restype = ctypes.c_size_t
     L.kvs_page_bytes.argtypes = [cp(kvs_config)]
     L.kvs_plan_page.argtypes = [cp(kvs_config), i, i, cp(i), cp(i)]
+    L.kvs_plan_ring.argtypes = [cp(kvs_config), i, i, ctypes.c_longlong, cp(i), cp(i), cp(i), i]
     L.kvs_create.argtypes = [cp(kvs_config), i, cp(vp)]
     L.kvs_destroy.argtypes = [vp]
     L.kvs_destroy.restype = None
@@ -206,6 +207,15 @@ def kvs_plan_page(cfg: kvs_config, n_tokens: int, page: int):
     k, i = ctypes.c_int(), ctypes.c_int()
     _check(lib.kvs_plan_page(ctypes.byref(cfg), n_tokens, page, ctypes.byref(k), ctypes.byref(i)))
     return k.value, i.value
+
+
+def kvs_plan_ring(cfg: kvs_config, n_q: int, s_ring: int, ring_ctr0: int = 0):
+    """The ring schedule of one attend call: [(page0, pages, slot0), ...]."""
+    n = lib.kvs_plan_ring(ctypes.byref(cfg), n_q, s_ring, ring_ctr0, None, None, None, 0)
+    _check(n if n < 0 else 0)
+    p0, pg, sl = (ctypes.c_int * max(1, n))(), (ctypes.c_int * max(1, n))(), (ctypes.c_int * max(1, n))()
+    _check(min(0, lib.kvs_plan_ring(ctypes.byref(cfg), n_q, s_ring, ring_ctr0, p0, pg, sl, n)))
+    return [(p0[k], pg[k], sl[k]) for k in range(n)]
 
 
 def kvs_create(cfg: kvs_config, device: int = 0) -> int:

@@ -200,6 +200,22 @@ size_t kvs_page_bytes(const kvs_config* cfg);
  * or KVS_PAGE_ABSENT.  The R most recent pages are resident. */
 int kvs_plan_page(const kvs_config* resolved, int n_tokens, int page, int* kind, int* index);
 
+/* The ring schedule of one kvs_attend call of n_q query tokens whose streamed
+ * pages 0..s_ring-1 go through the transfer ring ("RaymondHuang210129/
+ * llama.cpp-adaptive-kv-streaming", Summary: one shared ring buffer), with the
+ * handle's ring counter at ring_ctr0: the host-to-device copies in order, copy
+ * i moving pages page0[i] .. page0[i]+pages[i]-1 into ring slots slot0[i] ..
+ * slot0[i]+pages[i]-1.  One copy per chunk_pages pages, each into the next
+ * group of chunk_pages slots; on the tensor-core path with more than one
+ * 128-row tile per kv head, the last chunk goes as two pieces into one group
+ * (the first (5p + 7) / 8 of its p pages, then the rest).  Writes at most
+ * max_copies entries (the arrays may be NULL when max_copies is 0) and returns
+ * the number of copies, or KVS_E_INVAL for a null config, n_q < 1, a negative
+ * s_ring, ring_ctr0 or max_copies, or an unresolved ring (slots without a
+ * chunk size).  Pure host logic: no device is touched. */
+int kvs_plan_ring(const kvs_config* resolved, int n_q, int s_ring, long long ring_ctr0, int* page0, int* pages,
+                  int* slot0, int max_copies);
+
 /* ---- draft eject controller (pure host) ------------------------------------
  * The dynamic draft eject of "llama.cpp adaptive KV streaming - spec fork
  * notes" (Dynamic draft eject; Results): a pinned draft (an MTP block and its
