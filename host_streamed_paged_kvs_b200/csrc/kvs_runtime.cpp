@@ -92,7 +92,7 @@ constexpr int kSms = 148;
 // Splits of the resident launch and of one ring-chunk launch (each split is an
 // equal share of the launch's half-page stages).
 constexpr long kResCtaStages = 4;  // raw stages per resident CTA beside ring launches
-constexpr long kResSplits = 4;     // splits per such resident launch
+constexpr long kResSplitsMax = 16; // splits per such resident launch, at most
 
 int res_splits(const kvs_config& c, long R_eff, int n_q, bool ring) {
     const long stages = 2 * R_eff;
@@ -106,11 +106,12 @@ int res_splits(const kvs_config& c, long R_eff, int n_q, bool ring) {
             if (best_cost < 0 || cost < best_cost) { best = sp; best_cost = cost; }
         }
         // Beside ring-chunk launches the resident pages go in a sequence of
-        // launches of short CTAs (kResCtaStages raw stages each, kResSplits
-        // per launch) that fold into one set of records: a CTA holds its SM
-        // until it ends, and a ring chunk whose copy has landed must not wait
-        // behind a long resident CTA.
-        if (ring) return (int)std::min<long>(stages, kResSplits);
+        // launches of short CTAs (kResCtaStages raw stages each) that fold
+        // into one set of records: a CTA holds its SM until it ends, and a
+        // ring chunk whose copy has landed must not wait behind a long
+        // resident CTA.  A launch is about one wave (3 splits for the 40 units
+        // of a 256-token prefill chunk, 16 for the 8 of a verify batch).
+        if (ring) return (int)std::min<long>(stages, std::max(1L, std::min(kResSplitsMax, (long)kSms / units)));
         return (int)best;
     }
     if (wide_regime(c, n_q)) return (int)std::min(stages, 8L);
@@ -1292,7 +1293,7 @@ int kvs_attend(kvs_t* kv, int layer, int pos0, int n_q, const void* q_f16, float
                 }
         }
         if (tc && S_ring > 0) {
-            // launches of kResSplits CTAs of kResCtaStages raw stages each, in
+            // launches of res_splits CTAs of kResCtaStages raw stages each, in
             // page order on the resident stream; later ones fold their partials
             // into the first one's records (the first is the widest)
             const long per_launch = ns * kResCtaStages;  // raw stages = 2 per page; even
