@@ -52,7 +52,7 @@ NCU_TRAFFIC = {
                       "in_place": (86272, 51), "in_place_pcie": (23763968, 51)},
     "chunk_mma_kernel": {"src": "kvs_chunk_mma.cu", "sha": "18d03cf82c7cfd65",
                          "workload": "prefill_chunk_64k", "type_v": 2,
-                         "resident": (27399936, 8), "ring": (6100736, 8)},
+                         "resident": (21223680, 6), "ring": (6100480, 8)},
 }
 
 
